@@ -1,0 +1,336 @@
+"""Pins for the CPU oracle (runs without a GPU).
+
+Each test ties one oracle function to something other than itself: a hand-worked case,
+brute force, an independent library routine, a closed form, or an invariant.  Together
+they are chosen so that a dropped term, a wrong sign, a swapped index or a transposed
+operand anywhere in the oracle fails at least one of them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+from oracle import moe_oracle as O
+from routing_dispatch_expert_warp_b200 import workload as W
+
+
+def _hand(golden_dir):
+    with open(os.path.join(golden_dir, "hand_e4_k2_t8.json")) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- hand-worked case
+def test_hand_case_routing(golden_dir):
+    g = _hand(golden_dir)
+    z = np.array(g["logits"], dtype=np.float32)
+    idx = O.select_topk(z, g["k"])
+    assert idx.tolist() == g["topk_idx"]
+    C = O.capacity(g["capacity_factor"], g["T"], g["k"], g["E"])
+    assert C == g["capacity"]
+    for layout, key in ((O.LAYOUT_COMPACT, "compact"), (O.LAYOUT_PADDED, "padded")):
+        a = O.assign(idx, g["E"], C, layout)
+        assert a["routed"].tolist() == g["routed"]
+        assert a["kept"].tolist() == g["kept"]
+        assert a["offsets"].tolist() == g[key]["offsets"]
+        assert a["assign_row"].tolist() == g[key]["assign_row"]
+        assert a["token_of_row"].tolist() == g[key]["token_of_row"]
+
+
+def test_hand_case_weights(golden_dir):
+    g = _hand(golden_dir)
+    z = np.array(g["logits"], dtype=np.float32)
+    idx = np.array(g["topk_idx"])
+    w = O.gate_weights(z, idx, O.SOFTMAX)
+    np.testing.assert_allclose(w, np.array(g["softmax_w"]), rtol=0, atol=1e-15)
+
+
+def test_hand_case_stats(golden_dir):
+    g = _hand(golden_dir)
+    a = O.assign(np.array(g["topk_idx"]), g["E"], g["capacity"])
+    s = O.load_stats(a["routed"], a["kept"], a["assign_row"], g["capacity"])
+    for key, v in g["stats"].items():
+        if isinstance(v, list):
+            assert s[key] == v, key
+        else:
+            assert s[key] == pytest.approx(v, abs=1e-12), key
+    assert s["tokens_per_expert"] == g["kept"]
+
+
+def test_sigmoid_weights_hand_values():
+    # sigma(3) = 0.9525741268224334, sigma(2) = 0.8807970779778823 (tabulated values)
+    z = np.array([[3.0, 2.0, -1.0]], dtype=np.float32)
+    w = O.gate_weights(z, np.array([[0, 1]]), O.SIGMOID)
+    s3, s2 = 0.9525741268224334, 0.8807970779778823
+    np.testing.assert_allclose(w[0], [s3 / (s3 + s2), s2 / (s3 + s2)], rtol=0, atol=1e-15)
+    # equal logits share the weight equally; the order of picks is respected
+    w = O.gate_weights(np.array([[0.5, -2.0, 0.5]], dtype=np.float32), np.array([[2, 1, 0]]),
+                       O.SIGMOID)
+    assert w[0, 0] == pytest.approx(w[0, 2], abs=1e-15)
+    assert w[0, 1] < w[0, 0]
+
+
+# ---------------------------------------------------------------- brute force top-k
+def _brute_topk(zrow, k):
+    """Among all k-subsets, the unique one in which every member beats every non-member
+    under (larger value, then lower index); ordered the same way."""
+    E = len(zrow)
+    beats = lambda i, j: zrow[i] > zrow[j] or (zrow[i] == zrow[j] and i < j)
+    found = []
+    for S in itertools.combinations(range(E), k):
+        rest = [j for j in range(E) if j not in S]
+        if all(beats(i, j) for i in S for j in rest):
+            found.append(S)
+    assert len(found) == 1
+    S = list(found[0])
+    # order within the subset: insertion by 'beats'
+    ordered = []
+    for i in S:
+        pos = 0
+        while pos < len(ordered) and beats(ordered[pos], i):
+            pos += 1
+        ordered.insert(pos, i)
+    return ordered
+
+
+@pytest.mark.parametrize("E,k", [(4, 1), (4, 2), (6, 3), (8, 2), (8, 8), (7, 5)])
+def test_topk_brute_force(E, k):
+    rng = np.random.default_rng(E * 100 + k)
+    for trial in range(40):
+        if trial % 2:
+            z = rng.integers(-2, 3, size=(1, E)).astype(np.float32)   # many ties
+        else:
+            z = rng.standard_normal((1, E)).astype(np.float32)
+        idx = O.select_topk(z, k)
+        assert idx[0].tolist() == _brute_topk(z[0].tolist(), k)
+
+
+def test_topk_signed_zero_is_a_tie():
+    z = np.array([[-0.0, 0.0, -1.0]], dtype=np.float32)
+    assert O.select_topk(z, 2)[0].tolist() == [0, 1]
+
+
+# ---------------------------------------------------------------- permutation
+@pytest.mark.parametrize("T,E,k,cf", [(37, 5, 2, 1.0), (64, 8, 2, 1.25), (50, 16, 4, 0.5),
+                                      (40, 8, 3, 0.0), (9, 3, 3, 2.0)])
+def test_assign_matches_stable_sort_and_bincount(T, E, k, cf):
+    rng = np.random.default_rng(T + E)
+    z = rng.standard_normal((T, E)).astype(np.float32)
+    z[:, 0] += 1.0   # make expert 0 hot so capacity bites
+    idx = O.select_topk(z, k)
+    C = O.capacity(cf, T, k, E)
+    a = O.assign(idx, E, C)
+    # counts: bincount
+    assert a["routed"].tolist() == np.bincount(idx.ravel(), minlength=E).tolist()
+    # permutation: stable sort of the assignment list on key e*T + t
+    flat_e = idx.ravel()
+    flat_t = np.repeat(np.arange(T), k)
+    order = np.argsort(flat_e.astype(np.int64) * T + flat_t, kind="stable")
+    slot = np.empty(T * k, dtype=np.int64)
+    start = np.concatenate([[0], np.cumsum(np.bincount(flat_e, minlength=E))])
+    slot[order] = np.arange(T * k) - start[flat_e[order]]
+    assert a["slot"].ravel().tolist() == slot.tolist()
+    kept_mask = slot < (C if C is not None else T * k + 1)
+    kept = np.bincount(flat_e[kept_mask], minlength=E)
+    assert a["kept"].tolist() == kept.tolist()
+    # rows of the kept assignments, in stable-sort order, are 0..Σkept-1 (COMPACT)
+    kept_order = [i for i in order if kept_mask[i]]
+    assert [int(a["assign_row"].ravel()[i]) for i in kept_order] == list(range(int(kept.sum())))
+    # invariants
+    assert int(a["kept"].sum()) == T * k - int((a["assign_row"] < 0).sum())
+    if C is not None:
+        assert (a["kept"] <= C).all()
+    used = a["token_of_row"]
+    assert (used >= 0).all()
+    # every kept assignment appears exactly once
+    rows = a["assign_row"][a["assign_row"] >= 0]
+    assert len(set(rows.tolist())) == len(rows)
+    for t in range(T):
+        for j in range(k):
+            r = a["assign_row"][t, j]
+            if r >= 0:
+                assert used[r] == t
+
+
+def test_padded_layout_rows():
+    rng = np.random.default_rng(3)
+    z = rng.standard_normal((30, 4)).astype(np.float32)
+    idx = O.select_topk(z, 2)
+    C = O.capacity(1.0, 30, 2, 4)
+    a = O.assign(idx, 4, C, O.LAYOUT_PADDED)
+    b = O.assign(idx, 4, C, O.LAYOUT_COMPACT)
+    assert a["rows"] == 4 * C
+    for t in range(30):
+        for j in range(2):
+            e = idx[t, j]
+            if b["assign_row"][t, j] < 0:
+                assert a["assign_row"][t, j] == -1
+            else:
+                assert a["assign_row"][t, j] - e * C == b["assign_row"][t, j] - b["offsets"][e]
+    with pytest.raises(ValueError):
+        O.assign(idx, 4, None, O.LAYOUT_PADDED)
+
+
+def test_capacity_values():
+    assert O.capacity(1.25, 64, 2, 8) == 20
+    assert O.capacity(1.0, 16384, 8, 256) == 512
+    assert O.capacity(1.25, 8192, 2, 8) == 2560
+    assert O.capacity(1.0, 10, 1, 3) == 4          # 10/3 rounded up
+    assert O.capacity(0.01, 10, 1, 3) == 1         # never below one slot
+    assert O.capacity(0.0, 10, 1, 3) is None
+    assert O.capacity(-1.0, 10, 1, 3) is None
+
+
+# ---------------------------------------------------------------- weights
+def test_softmax_k_equals_E_is_full_softmax():
+    rng = np.random.default_rng(5)
+    z = rng.standard_normal((20, 6)).astype(np.float32)
+    idx = O.select_topk(z, 6)
+    w = O.gate_weights(z, idx, O.SOFTMAX)
+    full = scipy.special.softmax(z.astype(np.float64), axis=1)
+    np.testing.assert_allclose(w, np.take_along_axis(full, idx.astype(np.int64), 1),
+                               rtol=1e-14, atol=0)
+
+
+def test_weights_sum_to_one_and_follow_rank():
+    rng = np.random.default_rng(6)
+    z = (rng.standard_normal((50, 16)) * 3).astype(np.float32)
+    for gating in (O.SOFTMAX, O.SIGMOID):
+        idx = O.select_topk(z, 4)
+        w = O.gate_weights(z, idx, gating)
+        np.testing.assert_allclose(w.sum(1), 1.0, rtol=0, atol=1e-14)
+        assert (np.diff(w, axis=1) <= 1e-15).all()   # best pick weighs most
+
+
+def test_sigmoid_matches_scipy_expit():
+    rng = np.random.default_rng(8)
+    z = (rng.standard_normal((10, 12)) * 4).astype(np.float32)
+    idx = O.select_topk(z, 3)
+    s = scipy.special.expit(np.take_along_axis(z.astype(np.float64), idx.astype(np.int64), 1))
+    np.testing.assert_allclose(O.gate_weights(z, idx, O.SIGMOID), s / s.sum(1, keepdims=True),
+                               rtol=1e-14)
+
+
+# ---------------------------------------------------------------- logits
+def test_router_logits_brute_force():
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((3, 5))
+    wr = rng.standard_normal((5, 4))
+    b = rng.standard_normal(4)
+    z = O.router_logits(x, wr, b)
+    for t in range(3):
+        for e in range(4):
+            ref = math.fsum(x[t, i] * wr[i, e] for i in range(5)) + b[e]
+            assert z[t, e] == pytest.approx(ref, abs=1e-13)
+    b2 = rng.standard_normal((3, 4))
+    z2 = O.router_logits(x, wr, b2)
+    np.testing.assert_allclose(z2 - b2, z - b, atol=1e-13)
+    assert O.router_logits(np.eye(5)[:3], wr).tolist() == wr[:3].tolist()
+
+
+def test_fp32_rounding_of_logits():
+    z = np.array([[1.0 + 2.0 ** -24, 1.0 + 3 * 2.0 ** -24, -(1.0 + 2.0 ** -24)]])
+    r = O.logits_to_fp32(z)
+    assert r.dtype == np.float32
+    assert r[0].tolist() == [1.0, 1.0 + 2.0 ** -22, -1.0]
+
+
+# ---------------------------------------------------------------- FFN, combine, layer
+def _dense_swiglu_torch(x, wg, wu, wd):
+    xt = torch.from_numpy(np.asarray(x, dtype=np.float64))
+    g = torch.nn.functional.linear(xt, torch.from_numpy(np.asarray(wg, dtype=np.float64)))
+    u = torch.nn.functional.linear(xt, torch.from_numpy(np.asarray(wu, dtype=np.float64)))
+    h = torch.nn.functional.silu(g) * u
+    return torch.nn.functional.linear(h, torch.from_numpy(np.asarray(wd, dtype=np.float64))).numpy()
+
+
+def test_single_expert_layer_is_dense_swiglu():
+    rng = np.random.default_rng(10)
+    T, d, f = 11, 16, 24
+    x = rng.standard_normal((T, d))
+    wr = rng.standard_normal((d, 1))
+    wg = rng.standard_normal((1, f, d)) / 4
+    wu = rng.standard_normal((1, f, d)) / 4
+    wd = rng.standard_normal((1, d, f)) / 5
+    for gating in (O.SOFTMAX, O.SIGMOID):
+        r = O.moe_layer(x, wr, None, wg, wu, wd, k=1, gating=gating, capacity_factor=0.0)
+        np.testing.assert_allclose(r["out"], _dense_swiglu_torch(x, wg[0], wu[0], wd[0]),
+                                   rtol=1e-12, atol=1e-12)
+
+
+def test_swiglu_operand_orientation():
+    # non-square weights: a transposed operand cannot even be multiplied
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((2, 3))
+    wg, wu, wd = rng.standard_normal((5, 3)), rng.standard_normal((5, 3)), rng.standard_normal((3, 5))
+    h, y = O.swiglu_expert(x, wg, wu, wd)
+    assert h.shape == (2, 5) and y.shape == (2, 3)
+    # hand value: one input, one hidden unit
+    h1, y1 = O.swiglu_expert([[2.0]], [[1.0]], [[3.0]], [[0.5]])
+    silu2 = 2.0 / (1.0 + math.exp(-2.0))
+    assert h1[0, 0] == pytest.approx(silu2 * 6.0, abs=1e-15)
+    assert y1[0, 0] == pytest.approx(silu2 * 3.0, abs=1e-15)
+
+
+def test_combine_one_hot_reproduces_rows():
+    rng = np.random.default_rng(12)
+    y = rng.standard_normal((6, 4))
+    assign_row = np.array([[3, 1], [0, -1], [-1, -1]])
+    w = np.array([[1.0, 0.0], [0.0, 1.0], [0.5, 0.5]])
+    out = O.combine(y, assign_row, w)
+    np.testing.assert_array_equal(out[0], y[3])
+    np.testing.assert_array_equal(out[1], np.zeros(4))   # kept pick has weight 0, dropped pick ignored
+    np.testing.assert_array_equal(out[2], np.zeros(4))   # fully dropped token
+    w2 = np.array([[0.25, 0.75], [1.0, 0.3], [1.0, 1.0]])
+    out2 = O.combine(y, assign_row, w2)
+    np.testing.assert_allclose(out2[0], 0.25 * y[3] + 0.75 * y[1], atol=1e-15)
+    np.testing.assert_allclose(out2[1], y[0], atol=1e-15)   # no renormalisation over survivors
+
+
+def test_layer_equals_per_token_sum_of_experts():
+    """Whole-layer output equals the per-token definition computed one token at a time."""
+    shape = W.reduced(W.TINY_FP32, 24, 32, 48, capacity_factor=1.0)
+    inp = W.make_inputs(shape)
+    npx = lambda t: t.float().numpy()
+    r = O.moe_layer(npx(inp.x), npx(inp.w_router), None, npx(inp.w_gate), npx(inp.w_up),
+                    npx(inp.w_down), shape.k, shape.gating, shape.capacity_factor)
+    toks = list(range(shape.T))
+    o = O.token_outputs(toks, npx(inp.x), r["idx"], r["w"], r["assign_row"] >= 0,
+                        lambda e: (npx(inp.w_gate[e]), npx(inp.w_up[e]), npx(inp.w_down[e])))
+    np.testing.assert_allclose(r["out"], o, rtol=1e-12, atol=1e-12)
+    assert r["stats"]["dropped"] > 0        # capacity 1.0 with a skewed router drops
+
+
+def test_page_stats_example(golden_dir):
+    with open(os.path.join(golden_dir, "page_stats_example.json")) as f:
+        g = json.load(f)
+    n = g["tokens_per_expert"]
+    # the printed list is an excerpt of the layer's experts; max and max/mean over it are
+    # what the page's record shows
+    s = O.load_stats(n, n, np.zeros((1, 1), dtype=np.int64), None)
+    assert s["max"] == g["expert_max"]
+    assert round(s["max_to_mean"], g["printed_decimals"]) == g["expert_max_to_mean_printed"]
+    assert s["mean"] == pytest.approx(sum(n) / len(n))
+
+
+def test_percentiles_match_numpy_linear():
+    rng = np.random.default_rng(13)
+    for n in (1, 2, 4, 7, 256):
+        v = rng.integers(0, 1000, size=n)
+        for p in (0.5, 0.95, 0.99):
+            assert O.percentile_linear(v, p) == pytest.approx(
+                float(np.percentile(v, 100 * p, method="linear")), abs=1e-9)
+
+
+def test_stats_top5_counts_experts():
+    kept = list(range(40))          # E = 40 -> ceil(2.0) = 2 experts
+    s = O.load_stats(kept, kept, np.zeros((10, 1), dtype=np.int64), None)
+    assert s["top5pct_share"] == pytest.approx((39 + 38) / sum(kept))
+    kept = [0] * 10
+    s = O.load_stats(kept, kept, -np.ones((3, 2), dtype=np.int64), 0)
+    assert s["top5pct_share"] == 0.0 and s["max_to_mean"] == 0.0
+    assert s["tokens_fully_dropped"] == 3 and s["dropped_by_rank"] == [3, 3]
