@@ -1,0 +1,363 @@
+"""Benchmark of one MoE layer forward on B200: tokens/s of the whole layer, with the grouped
+GEMM's tensor throughput and the permute/combine bandwidth beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl reference]
+
+One step = the whole hot path on one batch: route -> dispatch (count, scan, rank, permute)
+-> expert SwiGLU grouped GEMM (gate/up, down) -> combine -> load statistics, each stage one
+C-ABI call on the same stream with CUDA events between them.  Inputs are resident in HBM;
+L2 is flushed (a 256 MB write) between timed steps, outside the timed events.  With N > 1
+(torchrun, one process per GPU) every GPU runs its own replica of the layer on its own batch
+-- the path has no exchange at EP=1 -- and the slowest rank's time is taken.
+
+--impl reference times the CPU oracle (fp64 numpy) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import routing_dispatch_expert_warp_b200 as M  # noqa: E402
+from routing_dispatch_expert_warp_b200 import workload as W  # noqa: E402
+
+DEFAULT = W.MIXTRAL_8X7B
+METRIC = "MoE-layer tokens/s on 1 B200; grouped-GEMM % BF16 peak; permute/combine % HBM BW"
+L2_FLUSH_BYTES = 256 << 20
+KERNELS_PER_STEP_E_SMALL = 9   # router, count, scan, rank, permute, gemm x2, combine, stats
+KERNELS_PER_STEP_E_LARGE = 10  # + separate top-k kernel
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=d["hbm_gbs"], bf16_tflops=d["bf16_tflops"],
+                    bf16_tflops_sustained=d.get("bf16_tflops_sustained"), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    def __init__(self, index: int):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv")
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(index), f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def algorithmic_work(shape, kept_total: int) -> dict:
+    T, d, f, E, k, s = (shape.T, shape.d_model, shape.d_ff, shape.E, shape.k,
+                        2 if shape.dtype == W.BF16 else 4)
+    A = T * k
+    return {
+        "gemm_flops": 6.0 * d * f * kept_total,
+        "route_bytes": T * d * s + d * E * 4 + T * E * 4 + T * k * 8,
+        "permute_bytes": T * d * s + kept_total * d * s + A * 4,
+        "combine_bytes": kept_total * d * s + A * 8 + T * d * s,
+    }
+
+
+def run_gpu(args) -> None:
+    shape = W.WORKLOADS[args.config] if args.config else DEFAULT
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    # every rank holds a full replica; ranks draw different token batches
+    shape_r = shape.replace(seed=shape.seed + 1000 * rank) if rank else shape
+    inp = W.make_inputs(shape_r, device=dev)
+    cfg = M.config_from_shape(shape)
+    ws = M.alloc_workspace(cfg, dev)
+    b = M.LayerBuffers.allocate(cfg, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev):
+        ev[0].record(stream)
+        M.moe_route(cfg, inp.x, inp.w_router, inp.logit_bias, b.logits, b.topk_idx, b.topk_w, ws)
+        ev[1].record(stream)
+        M.moe_dispatch(cfg, inp.x, b.topk_idx, b.routed_counts, b.kept_counts, b.expert_offsets,
+                       b.assign_row, b.token_of_row, b.x_perm, ws)
+        ev[2].record(stream)
+        M.moe_expert_ffn(cfg, b.x_perm, b.expert_offsets, b.kept_counts, inp.w_gate, inp.w_up,
+                         inp.w_down, b.h, b.y_perm, ws)
+        ev[3].record(stream)
+        M.moe_combine(cfg, b.y_perm, b.assign_row, b.topk_w, b.out)
+        ev[4].record(stream)
+        M.moe_load_stats(cfg, b.routed_counts, b.kept_counts, b.assign_row, b.stats, host=False)
+        ev[5].record(stream)
+
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(mk())
+    M.moe_check_device_error(ws)
+
+    evs = [mk() for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        step(evs[i])
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    time.sleep(0.2)
+    clk = clocks.stop()
+    M.moe_check_device_error(ws)
+
+    names = ["route", "dispatch", "expert_ffn", "combine", "stats"]
+    per_stage = {n: [] for n in names}
+    step_ms = []
+    for ev in evs:
+        for j, n in enumerate(names):
+            per_stage[n].append(ev[j].elapsed_time(ev[j + 1]))
+        step_ms.append(ev[0].elapsed_time(ev[5]))
+    total_ms = sum(step_ms)
+    if dist:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    stats = b.stats_dict()
+    kept_total = stats["kept_total"]
+    work = algorithmic_work(shape, kept_total)
+    peaks = measured_peaks()
+    ffn_ms = sum(per_stage["expert_ffn"]) / args.steps
+    tflops = work["gemm_flops"] / (ffn_ms * 1e-3) / 1e12
+    gbs = lambda byts, n: byts / (sum(per_stage[n]) / args.steps * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host x -> device, layer, device -> host out
+    layer = M.MoELayer(cfg, inp.w_router, inp.w_gate, inp.w_up, inp.w_down, inp.logit_bias,
+                       device=dev)
+    x_host = inp.x.cpu().pin_memory()
+    out_host = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
+    x_dev = torch.empty_like(inp.x)
+    for _ in range(max(1, args.warmup)):
+        x_dev.copy_(x_host, non_blocking=True)
+        out_host.copy_(layer(x_dev), non_blocking=True)
+    torch.cuda.synchronize(dev)
+    e2e_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        out_host.copy_(layer(x_dev), non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        e2e_ms.append(e0.elapsed_time(e1))
+    e2e_total = sum(e2e_ms)
+    if dist:
+        t = torch.tensor([e2e_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    M.moe_check_device_error(layer.ws)
+
+    if rank == 0:
+        cpu = cpu_baseline(shape, args.cpu_sample_tokens) if (world == 1 and not args.no_cpu) else None
+        per_step_kernels = KERNELS_PER_STEP_E_SMALL if shape.E <= 32 else KERNELS_PER_STEP_E_LARGE
+        line = {
+            "metric": METRIC,
+            "value": shape.T * world / (ms_per_step * 1e-3),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_per_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if shape.dtype == W.BF16 else "f32",
+            "data": "synthetic (seeded; x~N(0,1), weights~N(0,1/fan_in))",
+            "config": {"workload": shape.name, "T": shape.T, "d_model": shape.d_model,
+                       "d_ff": shape.d_ff, "E": shape.E, "k": shape.k,
+                       "gating": "softmax" if shape.gating == W.SOFTMAX else "sigmoid",
+                       "capacity_factor": shape.capacity_factor,
+                       "l2": "flushed between timed steps (256 MB write)",
+                       "parallelism": f"replicas x{world} (EP=1, no exchange)"},
+            "roofline": {
+                "kernel": "grouped_gemm_tc_kernel (expert FFN: gate/up + down launches)",
+                "bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
+                "peak_source": f"{peaks['source']} bf16 burst",
+                "frac_of_sustained": (tflops / peaks["bf16_tflops_sustained"]
+                                      if peaks.get("bf16_tflops_sustained") else None),
+                "traffic": None,
+                "algorithmic_flops_per_step": work["gemm_flops"],
+            },
+            "stages_ms": {n: sum(v) / args.steps for n, v in per_stage.items()},
+            "stage_bandwidth": {
+                "route": {"GB/s": gbs(work["route_bytes"], "route"),
+                          "frac_hbm": gbs(work["route_bytes"], "route") / peaks["hbm_gbs"]},
+                "dispatch": {"GB/s": gbs(work["permute_bytes"], "dispatch"),
+                             "frac_hbm": gbs(work["permute_bytes"], "dispatch") / peaks["hbm_gbs"]},
+                "combine": {"GB/s": gbs(work["combine_bytes"], "combine"),
+                            "frac_hbm": gbs(work["combine_bytes"], "combine") / peaks["hbm_gbs"]},
+                "hbm_peak_gbs": peaks["hbm_gbs"],
+            },
+            "load_stats": {k2: stats[k2] for k2 in ("kept_total", "dropped", "p50", "p95", "max",
+                                                    "max_to_mean")},
+            "e2e": {"value": shape.T * world / (e2e_total / args.steps * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": inp.x.numel() * inp.x.element_size(),
+                    "d2h_bytes_per_step": b.out.numel() * b.out.element_size(),
+                    "api": "MoELayer.forward -> moe_layer_forward (pinned host buffers)"},
+            "gpu_launches": per_step_kernels * args.steps,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _cpu_cores() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+class CpuSample:
+    """The oracle as it stands, on the first `sample_tokens` tokens of the workload (full
+    weights, the same routing rule; capacity follows T as its definition says)."""
+
+    def __init__(self, shape, sample_tokens: int):
+        self.shape, self.n = shape, sample_tokens
+        self.sub = shape.replace(T=sample_tokens)
+        inp = W.make_inputs(self.sub, device="cpu")
+        f = lambda t: t.float().numpy()
+        bias = None if inp.logit_bias is None else f(inp.logit_bias)
+        self.args = (f(inp.x), f(inp.w_router), bias, f(inp.w_gate), f(inp.w_up),
+                     f(inp.w_down))
+
+    def run(self) -> dict:
+        from oracle import moe_oracle as O
+        s = self.sub
+        t0 = time.perf_counter()
+        O.moe_layer(*self.args, k=s.k, gating=s.gating, capacity_factor=s.capacity_factor,
+                    layout=s.layout)
+        dt = time.perf_counter() - t0
+        return {"value": self.n / dt, "unit": "tokens/s", "cores": _cpu_cores(),
+                "kind": "oracle", "seconds": dt,
+                "sample": f"oracle moe_layer on the first {self.n} tokens of {self.shape.name} "
+                          f"(full-size weights, fp64 numpy), {dt:.1f} s"}
+
+
+def cpu_baseline(shape, sample_tokens: int) -> dict:
+    return CpuSample(shape, sample_tokens).run()
+
+
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    shape = W.WORKLOADS[args.config] if args.config else DEFAULT
+    sample = CpuSample(shape, args.ref_sample_tokens)
+    for _ in range(args.warmup):
+        sample.run()
+    vals = [sample.run() for _ in range(args.steps)]
+    v = statistics.median(x["value"] for x in vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": args.ref_sample_tokens / v * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": shape.name, "T": shape.T, "d_model": shape.d_model,
+                   "d_ff": shape.d_ff, "E": shape.E, "k": shape.k},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[0]["cores"],
+                         "kind": "oracle", "sample": vals[0]["sample"]},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default=None, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-sample-tokens", type=int, default=64)
+    ap.add_argument("--ref-sample-tokens", type=int, default=32)
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)   # at least three untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,286 @@
+/*
+ * moe.h -- C ABI of a B200 (sm_100a) library for one Mixture-of-Experts layer forward on
+ * one GPU:  route -> dispatch -> expert SwiGLU grouped GEMM -> combine -> load statistics.
+ *
+ * Sources (page title, section):
+ *   [EP-serving] "Expert Parallelism for MoE Serving" (aiunderstanding.org): "Deep dive"
+ *                (a router picks the top-k experts per token, often 1 or 2; tokens are
+ *                shuffled to their experts, the FFN runs, results are shuffled back) and
+ *                "Technical insight" (two all-to-alls per layer, dispatch and combine;
+ *                capacity factors, expert buffers and dropping or padding tokens keep the
+ *                GEMMs uniform); FAQ (capacity = max tokens per expert, pad or drop past it).
+ *   [EP-checks]  "MoE expert parallelism needs measurements before launch" (airouter.kz):
+ *                "Mean expert load proves almost nothing" (mu = sum n_e / E; the per-layer
+ *                record of tokens_per_expert, p50, p95, max, max/mean, top-5% share,
+ *                dropped_tokens), "Capacity factor changes quality, memory and the latency
+ *                tail" (capacity = mean tokens per expert x factor for top-1; overflow
+ *                dropped; drop_tokens=false = unlimited; drop rate per route),
+ *                "Profile all-to-all separately from compute" (router, pack/permute,
+ *                dispatch, expert compute, combine, unpack; EP=1 keeps experts local with
+ *                no all-to-all).
+ *   [MegaScale]  "MegaScale-Infer: expert parallelism" slides (polomodov.tech), slide 11
+ *                (the exchange library makes no GPU->CPU copies and no GPU synchronisation).
+ *
+ * On one GPU the two all-to-alls of [EP-serving] become a local permutation (dispatch)
+ * and its inverse with a gate-weighted sum (combine), as in the EP=1 control run of
+ * [EP-checks].
+ *
+ * Conventions for every entry point
+ *   - All tensors are row-major and contiguous.  Weights are stored "out x in", i.e. the
+ *     reduction dimension is innermost.
+ *   - Device pointers are CUDA global memory of the current device.  The caller owns and
+ *     allocates every buffer, including the workspace; the library allocates nothing and
+ *     keeps no state besides a per-thread error string and a process-wide wait limit.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default stream) and
+ *     the call returns without synchronising, except where a host output is requested.
+ *     Following [MegaScale] slide 11, per-expert counts never travel to the host: every
+ *     kernel reads them from device memory.
+ *   - Pointers passed to the library must be 16-byte aligned; T, d_model and d_ff must be
+ *     such that every row is a multiple of 16 bytes.
+ *   - Errors: a host-side check fails with MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED /
+ *     MOE_ERR_WORKSPACE before anything is enqueued; a CUDA launch error gives
+ *     MOE_ERR_CUDA.  Errors found by kernels (an expert index out of range, a bounded
+ *     device wait that ran out) are recorded in the workspace's status word and reported
+ *     by moe_check_device_error().  moe_last_error() gives a message for the last failure
+ *     on the calling thread.
+ *   - Inputs are finite; NaN and Inf inputs give unspecified results.
+ */
+#ifndef MOE_B200_MOE_H
+#define MOE_B200_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+#define MOE_MAX_EXPERTS 256
+#define MOE_MAX_TOPK 8
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer, k > E ...   */
+  MOE_ERR_UNSUPPORTED = 2,   /* a valid request this build does not implement           */
+  MOE_ERR_WORKSPACE = 3,     /* ws_bytes smaller than moe_workspace_size() asks          */
+  MOE_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed                        */
+  MOE_ERR_TIMEOUT = 5,       /* a bounded device wait ran out (reported lazily)          */
+  MOE_ERR_DEVICE_DATA = 6    /* a kernel met invalid data, e.g. expert index >= E        */
+} moe_status_t;
+
+typedef enum { MOE_GATE_SOFTMAX = 0, MOE_GATE_SIGMOID = 1 } moe_gating_t;
+typedef enum { MOE_LAYOUT_COMPACT = 0, MOE_LAYOUT_PADDED = 1 } moe_layout_t;
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+
+/*
+ * One layer's shape and routing rule.
+ *   T               tokens in the batch ([EP-checks] "First fix the workload unit": the
+ *                   active tokens of this layer and batch), >= 1
+ *   d_model, d_ff   model and expert hidden widths
+ *   E, k            experts (1..256) and picks per token (1..min(E, 8)) [EP-serving]
+ *   gating          MOE_GATE_SOFTMAX: w_j = exp(z_j - z_max) / sum over the k picks;
+ *                   MOE_GATE_SIGMOID: w_j = s(z_j) / sum over the k picks of s(z)
+ *   layout          MOE_LAYOUT_COMPACT: expert buckets back to back, Sum(kept) rows;
+ *                   MOE_LAYOUT_PADDED: bucket e starts at row e*C, E*C rows (needs a
+ *                   finite capacity) [EP-serving "Technical insight": pad or drop]
+ *   dtype           element type of x, expert weights, x_perm, h, y_perm and out
+ *                   (MOE_F32: fp32 everywhere, fp32 FMA arithmetic;
+ *                    MOE_BF16: bf16 storage, fp32 accumulation on tensor cores).
+ *                   The router weight, logit bias, logits and gate weights are fp32.
+ *   capacity_factor cf > 0: capacity C = ceil(cf * T * k / E) slots per expert;
+ *                   cf <= 0: dropless ([EP-checks] "Capacity factor ...").
+ */
+typedef struct moe_config {
+  int64_t T;
+  int64_t d_model;
+  int64_t d_ff;
+  int32_t E;
+  int32_t k;
+  int32_t gating;   /* moe_gating_t */
+  int32_t layout;   /* moe_layout_t */
+  int32_t dtype;    /* moe_dtype_t  */
+  float capacity_factor;
+} moe_config_t;
+
+/*
+ * Per-layer load statistics ([EP-checks] "Mean expert load proves almost nothing" and
+ * "Capacity factor ...": per-layer and per-route drop rate).
+ *   tokens_per_expert is the kept count of each expert (the caller's kept_counts array);
+ *   p50/p95/p99/max/mean/max_to_mean/top5pct_share are over those E kept counts, empty
+ *   experts included; percentiles use linear interpolation between order statistics;
+ *   mean = Sum kept / E; top5pct_share = (sum of the ceil(0.05 E) largest) / Sum kept;
+ *   dropped counts dropped (token, expert) assignments = T*k - Sum kept;
+ *   dropped_by_rank[j] counts drops of the j-th pick (j < k; the rest are 0);
+ *   routed_* describe demand before the capacity limit.  Unused fields are 0.
+ */
+typedef struct moe_load_stats {
+  int32_t E;
+  int32_t k;
+  int64_t active_tokens;
+  int64_t capacity;            /* -1: dropless */
+  int64_t routed_total;
+  int64_t kept_total;
+  int64_t dropped;
+  int64_t tokens_with_drop;
+  int64_t tokens_fully_dropped;
+  double p50;
+  double p95;
+  double p99;
+  double max;
+  double mean;
+  double max_to_mean;
+  double routed_max;
+  double routed_max_to_mean;
+  double top5pct_share;
+  int64_t dropped_by_rank[MOE_MAX_TOPK];
+} moe_load_stats_t;
+
+/* Inputs of a whole layer (device pointers). */
+typedef struct moe_layer_inputs {
+  const void* x;             /* [T, d_model] dtype                                        */
+  const float* w_router;     /* [d_model, E] fp32                                         */
+  const float* logit_bias;   /* NULL, or fp32 rows of E values, see bias_row_stride       */
+  int64_t bias_row_stride;   /* 0: one [E] vector for all tokens; >= E: row t at t*stride */
+  const void* w_gate;        /* [E, d_ff, d_model] dtype                                  */
+  const void* w_up;          /* [E, d_ff, d_model] dtype                                  */
+  const void* w_down;        /* [E, d_model, d_ff] dtype                                  */
+} moe_layer_inputs_t;
+
+/* Outputs and intermediates of a whole layer (device pointers, caller-allocated). */
+typedef struct moe_layer_buffers {
+  float* logits;             /* [T, E] fp32, or NULL to keep them in the workspace        */
+  int32_t* topk_idx;         /* [T, k] experts, best first                               */
+  float* topk_w;             /* [T, k] gate weights                                      */
+  int32_t* routed_counts;    /* [E] assignments routed to each expert                    */
+  int32_t* kept_counts;      /* [E] assignments kept (= tokens_per_expert)               */
+  int32_t* expert_offsets;   /* [E+1] first row of each bucket; [E] = rows in use/alloc  */
+  int32_t* assign_row;       /* [T, k] row of x_perm holding pick j of token t; -1 dropped*/
+  int32_t* token_of_row;     /* [max_rows] token of each row; -1 for unused rows          */
+  void* x_perm;              /* [max_rows, d_model] dtype                                */
+  void* h;                   /* [max_rows, d_ff] dtype                                   */
+  void* y_perm;              /* [max_rows, d_model] dtype                                */
+  void* out;                 /* [T, d_model] dtype                                       */
+  moe_load_stats_t* stats;   /* device struct, or NULL to skip the statistics            */
+} moe_layer_buffers_t;
+
+/* ---------------------------------------------------------------- sizes */
+
+/* Bytes of workspace every entry point below needs for `cfg` (the maximum over them). */
+moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes);
+
+/* Enqueue the zeroing of the workspace's status word.  Call once after allocating. */
+moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Capacity C = ceil(cf * T * k / E) for cf > 0, -1 when dropless, -2 on a bad cfg. */
+int64_t moe_capacity(const moe_config_t* cfg);
+
+/* Rows to allocate for x_perm, h, y_perm and token_of_row: T*k when dropless,
+ * min(T*k, E*C) when COMPACT with a capacity, E*C when PADDED.  -2 on a bad cfg. */
+int64_t moe_max_rows(const moe_config_t* cfg);
+
+/* ---------------------------------------------------------------- stages */
+
+/*
+ * Router scoring, top-k selection and gate weights ([EP-serving] "Deep dive").
+ *   z[t, e] = sum_i x[t, i] * w_router[i, e] + b[t, e]   (fp32 accumulation)
+ *   topk_idx[t, :] = the k largest z[t, :], best first; equal z -> lower expert index
+ *   topk_w[t, :]   = gate weights renormalised over the k picks (cfg->gating)
+ * logits may be NULL (then z lives in the workspace).  Needs the workspace.
+ */
+moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_router,
+                       const float* logit_bias, int64_t bias_row_stride, float* logits,
+                       int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/*
+ * Dispatch ([EP-serving] "Technical insight"; [EP-checks] "Profile all-to-all ...": pack
+ * and permute; "Capacity factor ...": overflow dropped).  Assignments are ranked within
+ * each expert in token order; slot < C is kept, the rest dropped.
+ *   routed_counts[e], kept_counts[e] = min(routed, C), expert_offsets[e] = first row of
+ *   bucket e (COMPACT: exclusive scan of kept; PADDED: e*C), expert_offsets[E] = rows.
+ *   assign_row[t, j] = expert_offsets[e] + slot, or -1 if dropped.
+ *   token_of_row[r] = token copied into row r; -1 for rows no assignment uses.
+ *   x_perm[assign_row[t, j], :] = x[t, :] for every kept pick; unused rows untouched.
+ */
+moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                          int32_t* routed_counts, int32_t* kept_counts,
+                          int32_t* expert_offsets, int32_t* assign_row,
+                          int32_t* token_of_row, void* x_perm, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/*
+ * Expert SwiGLU FFN as a grouped GEMM over the variable-sized buckets ([EP-checks]
+ * "Profile all-to-all ...": grouped GEMMs over many experts).  For each expert e and each
+ * row r in [expert_offsets[e], expert_offsets[e] + kept_counts[e]):
+ *   h[r, :]      = silu(x_perm[r] . w_gate[e]^T) * (x_perm[r] . w_up[e]^T),
+ *                  silu(u) = u / (1 + exp(-u))
+ *   y_perm[r, :] = h[r] . w_down[e]^T
+ * Rows outside every bucket are not written.  bf16 needs d_model and d_ff to be multiples
+ * of 64 (MOE_ERR_UNSUPPORTED otherwise).  Needs the workspace (status word).
+ */
+moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
+                            const int32_t* expert_offsets, const int32_t* kept_counts,
+                            const void* w_gate, const void* w_up, const void* w_down, void* h,
+                            void* y_perm, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Combine ([EP-serving] "Deep dive": results shuffled back; [EP-checks]: combine, unpack):
+ *   out[t, :] = sum over j = 0..k-1 with assign_row[t, j] >= 0 of
+ *               topk_w[t, j] * y_perm[assign_row[t, j], :]
+ * summed in pick order in fp32, so the result is bitwise reproducible run to run.  A
+ * dropped pick contributes nothing (no renormalisation); a fully dropped token gets 0.
+ */
+moe_status_t moe_combine(const moe_config_t* cfg, const void* y_perm,
+                         const int32_t* assign_row, const float* topk_w, void* out,
+                         void* stream);
+
+/*
+ * Per-layer load statistics (moe_load_stats_t above) from the dispatch outputs, written to
+ * the device struct dev_out.  If host_out is not NULL the struct is also copied to host
+ * memory and the stream is synchronised -- the only call that synchronises.
+ */
+moe_status_t moe_load_stats(const moe_config_t* cfg, const int32_t* routed_counts,
+                            const int32_t* kept_counts, const int32_t* assign_row,
+                            moe_load_stats_t* dev_out, moe_load_stats_t* host_out,
+                            void* stream);
+
+/*
+ * The whole layer: moe_route, moe_dispatch, moe_expert_ffn, moe_combine and (when
+ * bufs->stats is not NULL) moe_load_stats, enqueued back to back on one stream without a
+ * host synchronisation.  Returns the first failing stage's status.
+ */
+moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_layer_inputs_t* in,
+                               const moe_layer_buffers_t* bufs, void* ws, size_t ws_bytes,
+                               void* stream);
+
+/* ---------------------------------------------------------------- errors */
+
+/* Synchronise `stream`, read and clear the workspace status word.  MOE_OK if no kernel
+ * recorded an error since the last check; MOE_ERR_TIMEOUT or MOE_ERR_DEVICE_DATA
+ * otherwise (details in moe_last_error()). */
+moe_status_t moe_check_device_error(void* ws, size_t ws_bytes, void* stream);
+
+/* Message for the last failing call on this thread ("" if none). */
+const char* moe_last_error(void);
+
+/* Static name of a status code. */
+const char* moe_status_string(moe_status_t status);
+
+/* Limit, in nanoseconds, on every wait a kernel makes on an on-chip barrier before it gives
+ * up, records MOE_ERR_TIMEOUT and returns (default 2e9).  0 restores the default. */
+void moe_set_wait_limit_ns(uint64_t ns);
+
+/* Self-test of the bounded wait: one block waits on an on-chip barrier that nothing
+ * completes, with the current limit, records MOE_ERR_TIMEOUT in the workspace status
+ * word and returns.  Used to check that a run-out wait leaves the context usable. */
+moe_status_t moe_selftest_bounded_wait(void* ws, size_t ws_bytes, void* stream);
+
+/* MOE_ABI_VERSION of the loaded library. */
+int32_t moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_MOE_H */

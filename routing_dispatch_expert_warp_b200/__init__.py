@@ -1,2 +1,223 @@
 """B200-native MoE layer forward (route -> dispatch -> SwiGLU grouped GEMM -> combine ->
-load statistics) behind a C-ABI library; this package is its thin Python binding."""
+load statistics) behind the C-ABI library libmoe.so.
+
+This package is the thin Python binding: it turns torch tensors into pointers and sizes
+and calls the entry points of include/moe.h under the same names.  Every step of the layer
+runs in the library's CUDA kernels; PyTorch only provides device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _abi
+from ._abi import MoEError, MoeConfig, MoeLayerBuffers, MoeLayerInputs, MoeLoadStats, check
+
+SOFTMAX, SIGMOID = 0, 1
+COMPACT, PADDED = 0, 1
+F32, BF16 = 0, 1
+
+__all__ = ["MoEError", "make_config", "workspace_size", "capacity", "max_rows",
+           "alloc_workspace", "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine",
+           "moe_load_stats", "moe_layer_forward", "moe_check_device_error",
+           "moe_selftest_bounded_wait", "set_wait_limit_ns", "LayerBuffers", "MoELayer"]
+
+
+def _lib():
+    return _abi.lib()
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the MoE library must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def make_config(T: int, d_model: int, d_ff: int, E: int, k: int, gating: int = SOFTMAX,
+                capacity_factor: float = 0.0, layout: int = COMPACT,
+                dtype: int = BF16) -> MoeConfig:
+    return MoeConfig(T=T, d_model=d_model, d_ff=d_ff, E=E, k=k, gating=gating, layout=layout,
+                     dtype=dtype, capacity_factor=capacity_factor)
+
+
+def config_from_shape(shape) -> MoeConfig:
+    """moe_config_t for a workload.MoEShape."""
+    return make_config(shape.T, shape.d_model, shape.d_ff, shape.E, shape.k, shape.gating,
+                       shape.capacity_factor, shape.layout, shape.dtype)
+
+
+def workspace_size(cfg: MoeConfig) -> int:
+    n = ctypes.c_size_t(0)
+    check(_lib().moe_workspace_size(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
+def capacity(cfg: MoeConfig) -> int:
+    return _lib().moe_capacity(ctypes.byref(cfg))
+
+
+def max_rows(cfg: MoeConfig) -> int:
+    r = _lib().moe_max_rows(ctypes.byref(cfg))
+    if r < 0:
+        raise MoEError(1, _lib().moe_last_error().decode())
+    return r
+
+
+def alloc_workspace(cfg: MoeConfig, device="cuda", stream=None) -> torch.Tensor:
+    ws = torch.empty(workspace_size(cfg), dtype=torch.uint8, device=device)
+    check(_lib().moe_workspace_init(_ptr(ws), ws.numel(), _stream(stream)))
+    return ws
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    _lib().moe_set_wait_limit_ns(ns)
+
+
+# ------------------------------------------------------------------ stages
+def moe_route(cfg, x, w_router, logit_bias, logits, topk_idx, topk_w, ws, stream=None):
+    stride = 0 if (logit_bias is None or logit_bias.dim() == 1) else logit_bias.shape[1]
+    check(_lib().moe_route(ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(logit_bias), stride,
+                           _ptr(logits), _ptr(topk_idx), _ptr(topk_w), _ptr(ws), ws.numel(),
+                           _stream(stream)))
+
+
+def moe_dispatch(cfg, x, topk_idx, routed_counts, kept_counts, expert_offsets, assign_row,
+                 token_of_row, x_perm, ws, stream=None):
+    check(_lib().moe_dispatch(ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(routed_counts),
+                              _ptr(kept_counts), _ptr(expert_offsets), _ptr(assign_row),
+                              _ptr(token_of_row), _ptr(x_perm), _ptr(ws), ws.numel(),
+                              _stream(stream)))
+
+
+def moe_expert_ffn(cfg, x_perm, expert_offsets, kept_counts, w_gate, w_up, w_down, h, y_perm,
+                   ws, stream=None):
+    check(_lib().moe_expert_ffn(ctypes.byref(cfg), _ptr(x_perm), _ptr(expert_offsets),
+                                _ptr(kept_counts), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                                _ptr(h), _ptr(y_perm), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_combine(cfg, y_perm, assign_row, topk_w, out, stream=None):
+    check(_lib().moe_combine(ctypes.byref(cfg), _ptr(y_perm), _ptr(assign_row), _ptr(topk_w),
+                             _ptr(out), _stream(stream)))
+
+
+def stats_buffer(device="cuda") -> torch.Tensor:
+    return torch.zeros(ctypes.sizeof(MoeLoadStats), dtype=torch.uint8, device=device)
+
+
+def moe_load_stats(cfg, routed_counts, kept_counts, assign_row, dev_out, host: bool = True,
+                   stream=None) -> Optional[dict]:
+    hs = MoeLoadStats()
+    check(_lib().moe_load_stats(ctypes.byref(cfg), _ptr(routed_counts), _ptr(kept_counts),
+                                _ptr(assign_row), _ptr(dev_out),
+                                ctypes.byref(hs) if host else None, _stream(stream)))
+    return hs.as_dict() if host else None
+
+
+def moe_layer_forward(cfg, inputs: MoeLayerInputs, bufs: MoeLayerBuffers, ws, stream=None):
+    check(_lib().moe_layer_forward(ctypes.byref(cfg), ctypes.byref(inputs), ctypes.byref(bufs),
+                                   _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_check_device_error(ws, stream=None):
+    check(_lib().moe_check_device_error(_ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_selftest_bounded_wait(ws, stream=None):
+    check(_lib().moe_selftest_bounded_wait(_ptr(ws), ws.numel(), _stream(stream)))
+
+
+# ------------------------------------------------------------------ whole layer
+@dataclass
+class LayerBuffers:
+    """Every output and intermediate of one layer forward, allocated with torch."""
+    logits: torch.Tensor
+    topk_idx: torch.Tensor
+    topk_w: torch.Tensor
+    routed_counts: torch.Tensor
+    kept_counts: torch.Tensor
+    expert_offsets: torch.Tensor
+    assign_row: torch.Tensor
+    token_of_row: torch.Tensor
+    x_perm: torch.Tensor
+    h: torch.Tensor
+    y_perm: torch.Tensor
+    out: torch.Tensor
+    stats: torch.Tensor
+
+    @staticmethod
+    def allocate(cfg: MoeConfig, device="cuda") -> "LayerBuffers":
+        T, d, f, E, k = cfg.T, cfg.d_model, cfg.d_ff, cfg.E, cfg.k
+        R = max_rows(cfg)
+        dt = torch.float32 if cfg.dtype == F32 else torch.bfloat16
+        i32 = dict(dtype=torch.int32, device=device)
+        return LayerBuffers(
+            logits=torch.empty((T, E), dtype=torch.float32, device=device),
+            topk_idx=torch.empty((T, k), **i32), topk_w=torch.empty((T, k), dtype=torch.float32,
+                                                                    device=device),
+            routed_counts=torch.empty(E, **i32), kept_counts=torch.empty(E, **i32),
+            expert_offsets=torch.empty(E + 1, **i32), assign_row=torch.empty((T, k), **i32),
+            token_of_row=torch.empty(max(R, 1), **i32),
+            x_perm=torch.empty((max(R, 1), d), dtype=dt, device=device),
+            h=torch.empty((max(R, 1), f), dtype=dt, device=device),
+            y_perm=torch.empty((max(R, 1), d), dtype=dt, device=device),
+            out=torch.empty((T, d), dtype=dt, device=device),
+            stats=stats_buffer(device))
+
+    def as_struct(self, with_stats: bool = True) -> MoeLayerBuffers:
+        return MoeLayerBuffers(
+            logits=_ptr(self.logits), topk_idx=_ptr(self.topk_idx), topk_w=_ptr(self.topk_w),
+            routed_counts=_ptr(self.routed_counts), kept_counts=_ptr(self.kept_counts),
+            expert_offsets=_ptr(self.expert_offsets), assign_row=_ptr(self.assign_row),
+            token_of_row=_ptr(self.token_of_row), x_perm=_ptr(self.x_perm), h=_ptr(self.h),
+            y_perm=_ptr(self.y_perm), out=_ptr(self.out),
+            stats=_ptr(self.stats) if with_stats else None)
+
+    def stats_dict(self) -> dict:
+        hs = MoeLoadStats()
+        ctypes.memmove(ctypes.byref(hs), self.stats.cpu().numpy().ctypes.data,
+                       ctypes.sizeof(MoeLoadStats))
+        return hs.as_dict()
+
+
+class MoELayer:
+    """One MoE layer with resident weights: the public entry point for a forward pass.
+
+    forward(x) enqueues the whole layer (moe_layer_forward) on the current stream and
+    returns the output tensor (a view of the layer's own buffer, overwritten by the next
+    call)."""
+
+    def __init__(self, cfg: MoeConfig, w_router, w_gate, w_up, w_down, logit_bias=None,
+                 device="cuda"):
+        self.cfg = cfg
+        self.w_router, self.w_gate, self.w_up, self.w_down = w_router, w_gate, w_up, w_down
+        self.logit_bias = logit_bias
+        self.ws = alloc_workspace(cfg, device)
+        self.bufs = LayerBuffers.allocate(cfg, device)
+        self._structs = self.bufs.as_struct(True)
+
+    def inputs(self, x) -> MoeLayerInputs:
+        b = self.logit_bias
+        return MoeLayerInputs(
+            x=_ptr(x), w_router=_ptr(self.w_router), logit_bias=_ptr(b),
+            bias_row_stride=0 if (b is None or b.dim() == 1) else b.shape[1],
+            w_gate=_ptr(self.w_gate), w_up=_ptr(self.w_up), w_down=_ptr(self.w_down))
+
+    def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+        moe_layer_forward(self.cfg, self.inputs(x), self._structs, self.ws, stream)
+        return self.bufs.out
+
+    __call__ = forward

@@ -1,0 +1,374 @@
+// The C ABI (include/moe.h): argument checks, workspace layout and the stage sequence.
+// Host code only; every step of the layer runs in the kernels of the other files.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <atomic>
+#include <mutex>
+#include <string>
+
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<uint64_t> g_wait_ns{2000000000ull};
+
+moe_status_t fail(moe_status_t st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+moe_status_t cuda_fail(cudaError_t err, const char* what) {
+  return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(err));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t v) { return (v + kWsAlign - 1) / kWsAlign * kWsAlign; }
+
+moe_status_t check_config(const moe_config_t* cfg, Shape* s) {
+  if (cfg == nullptr) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
+  if (cfg->T < 1) return fail(MOE_ERR_INVALID_ARG, "T must be >= 1 (got %lld)", (long long)cfg->T);
+  if (cfg->d_model < 8 || cfg->d_model % 8 != 0)
+    return fail(MOE_ERR_INVALID_ARG, "d_model must be a positive multiple of 8 (got %lld)",
+                (long long)cfg->d_model);
+  if (cfg->d_ff < 4 || cfg->d_ff % 4 != 0)
+    return fail(MOE_ERR_INVALID_ARG, "d_ff must be a positive multiple of 4 (got %lld)",
+                (long long)cfg->d_ff);
+  if (cfg->E < 1 || cfg->E > MOE_MAX_EXPERTS)
+    return fail(MOE_ERR_INVALID_ARG, "E must be in [1, %d] (got %d)", MOE_MAX_EXPERTS, cfg->E);
+  if (cfg->k < 1 || cfg->k > cfg->E || cfg->k > MOE_MAX_TOPK)
+    return fail(MOE_ERR_INVALID_ARG, "k must be in [1, min(E, %d)] (got k=%d, E=%d)",
+                MOE_MAX_TOPK, cfg->k, cfg->E);
+  if (cfg->gating != MOE_GATE_SOFTMAX && cfg->gating != MOE_GATE_SIGMOID)
+    return fail(MOE_ERR_INVALID_ARG, "unknown gating %d", cfg->gating);
+  if (cfg->layout != MOE_LAYOUT_COMPACT && cfg->layout != MOE_LAYOUT_PADDED)
+    return fail(MOE_ERR_INVALID_ARG, "unknown layout %d", cfg->layout);
+  if (cfg->dtype != MOE_F32 && cfg->dtype != MOE_BF16)
+    return fail(MOE_ERR_INVALID_ARG, "unknown dtype %d", cfg->dtype);
+  if (!(cfg->capacity_factor == cfg->capacity_factor))
+    return fail(MOE_ERR_INVALID_ARG, "capacity_factor is NaN");
+  s->T = cfg->T;
+  s->d = cfg->d_model;
+  s->f = cfg->d_ff;
+  s->E = cfg->E;
+  s->k = cfg->k;
+  s->gating = cfg->gating;
+  s->layout = cfg->layout;
+  s->dtype = cfg->dtype;
+  s->elem = cfg->dtype == MOE_F32 ? 4 : 2;
+  const int64_t A = cfg->T * cfg->k;
+  if (cfg->capacity_factor > 0.0f) {
+    const double c = ceil(static_cast<double>(cfg->capacity_factor) * static_cast<double>(cfg->T) *
+                          static_cast<double>(cfg->k) / static_cast<double>(cfg->E));
+    if (c > 2147483647.0) return fail(MOE_ERR_INVALID_ARG, "capacity too large");
+    s->C = static_cast<int64_t>(c);
+  } else {
+    s->C = -1;
+  }
+  if (s->layout == MOE_LAYOUT_PADDED) {
+    if (s->C < 0)
+      return fail(MOE_ERR_INVALID_ARG, "PADDED layout needs capacity_factor > 0");
+    s->max_rows = static_cast<int64_t>(s->E) * s->C;
+  } else {
+    s->max_rows = s->C < 0 ? A : (A < s->E * s->C ? A : s->E * s->C);
+  }
+  if (s->max_rows > 2147483647LL || A > 2147483647LL)
+    return fail(MOE_ERR_INVALID_ARG, "too many rows for 32-bit row indices");
+  if (cfg->dtype == MOE_F32 && cfg->d_ff % 4 != 0)
+    return fail(MOE_ERR_INVALID_ARG, "fp32 d_ff must be a multiple of 4");
+  return MOE_OK;
+}
+
+moe_status_t check_ws(const Shape& s, const void* ws, size_t ws_bytes, WsLayout* lay) {
+  *lay = workspace_layout(s);
+  if (ws == nullptr) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(ws) & (kWsAlign - 1)) != 0)
+    return fail(MOE_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (ws_bytes < lay->total)
+    return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, lay->total);
+  return MOE_OK;
+}
+
+#define MOE_REQUIRE(cond, ...)                                 \
+  do {                                                         \
+    if (!(cond)) return fail(MOE_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+
+DevStatus* ws_status(void* ws, const WsLayout& lay) {
+  return reinterpret_cast<DevStatus*>(static_cast<uint8_t*>(ws) + lay.status);
+}
+
+}  // namespace
+
+WsLayout workspace_layout(const Shape& s) {
+  WsLayout l;
+  size_t off = 0;
+  l.status = off;
+  off += round_up(sizeof(DevStatus));
+  l.hist = off;
+  l.hist_bytes = round_up(static_cast<size_t>(dispatch_blocks(s.T)) * s.E * sizeof(int32_t));
+  off += l.hist_bytes;
+  l.logits = off;
+  l.logits_bytes = round_up(static_cast<size_t>(s.T) * s.E * sizeof(float));
+  off += l.logits_bytes;
+  l.total = off;
+  return l;
+}
+
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// ------------------------------------------------------------------ bounded-wait self-test
+namespace {
+__global__ void wait_selftest_kernel(DevStatus* status, uint64_t wait_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    // nothing ever arrives on `bar`: the wait must run out and report, not hang
+    if (!mbar_wait(&bar, 0, wait_ns, nullptr)) record_error(status, DEV_TIMEOUT, 99, 0);
+  }
+}
+}  // namespace
+
+cudaError_t launch_wait_selftest(DevStatus* status, uint64_t wait_ns, cudaStream_t st) {
+  wait_selftest_kernel<<<1, 32, 0, st>>>(status, wait_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_last_error(void) { return g_last_error.c_str(); }
+
+const char* moe_status_string(moe_status_t st) {
+  switch (st) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_DEVICE_DATA: return "MOE_ERR_DEVICE_DATA";
+  }
+  return "unknown";
+}
+
+void moe_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns == 0 ? 2000000000ull : ns); }
+
+moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
+  Shape s;
+  moe_status_t st = check_config(cfg, &s);
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(bytes != nullptr, "bytes is NULL");
+  *bytes = workspace_layout(s).total;
+  return MOE_OK;
+}
+
+moe_status_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  MOE_REQUIRE(ws != nullptr, "workspace is NULL");
+  MOE_REQUIRE(ws_bytes >= sizeof(DevStatus), "workspace too small");
+  cudaError_t err = cudaMemsetAsync(ws, 0, sizeof(DevStatus), static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_workspace_init");
+  return MOE_OK;
+}
+
+int64_t moe_capacity(const moe_config_t* cfg) {
+  Shape s;
+  if (check_config(cfg, &s) != MOE_OK) return -2;
+  return s.C;
+}
+
+int64_t moe_max_rows(const moe_config_t* cfg) {
+  Shape s;
+  if (check_config(cfg, &s) != MOE_OK) return -2;
+  return s.max_rows;
+}
+
+moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_router,
+                       const float* logit_bias, int64_t bias_row_stride, float* logits,
+                       int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
+                       void* stream) {
+  Shape s;
+  moe_status_t st = check_config(cfg, &s);
+  if (st != MOE_OK) return st;
+  WsLayout lay;
+  if ((st = check_ws(s, ws, ws_bytes, &lay)) != MOE_OK) return st;
+  MOE_REQUIRE(x && w_router && topk_idx && topk_w, "moe_route: NULL input/output pointer");
+  MOE_REQUIRE(aligned16(x) && aligned16(w_router), "moe_route: x and w_router must be 16-byte aligned");
+  MOE_REQUIRE(bias_row_stride == 0 || bias_row_stride >= s.E,
+              "moe_route: bias_row_stride must be 0 or >= E");
+  float* z = logits;
+  if (z == nullptr && s.E > 32) z = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + lay.logits);
+  cudaError_t err = launch_router(s, x, w_router, logit_bias, bias_row_stride, z, topk_idx, topk_w,
+                                  static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_route launch");
+  return MOE_OK;
+}
+
+moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
+                          int32_t* routed_counts, int32_t* kept_counts,
+                          int32_t* expert_offsets, int32_t* assign_row,
+                          int32_t* token_of_row, void* x_perm, void* ws, size_t ws_bytes,
+                          void* stream) {
+  Shape s;
+  moe_status_t st = check_config(cfg, &s);
+  if (st != MOE_OK) return st;
+  WsLayout lay;
+  if ((st = check_ws(s, ws, ws_bytes, &lay)) != MOE_OK) return st;
+  MOE_REQUIRE(x && topk_idx && routed_counts && kept_counts && expert_offsets && assign_row &&
+                  token_of_row && x_perm,
+              "moe_dispatch: NULL pointer");
+  MOE_REQUIRE(aligned16(x) && aligned16(x_perm), "moe_dispatch: x and x_perm must be 16-byte aligned");
+  int32_t* hist = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + lay.hist);
+  cudaError_t err = launch_dispatch(s, x, topk_idx, routed_counts, kept_counts, expert_offsets,
+                                    assign_row, token_of_row, x_perm, hist, ws_status(ws, lay),
+                                    g_wait_ns.load(), static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_dispatch launch");
+  return MOE_OK;
+}
+
+moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
+                            const int32_t* expert_offsets, const int32_t* kept_counts,
+                            const void* w_gate, const void* w_up, const void* w_down, void* h,
+                            void* y_perm, void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  moe_status_t st = check_config(cfg, &s);
+  if (st != MOE_OK) return st;
+  WsLayout lay;
+  if ((st = check_ws(s, ws, ws_bytes, &lay)) != MOE_OK) return st;
+  MOE_REQUIRE(x_perm && expert_offsets && kept_counts && w_gate && w_up && w_down && h && y_perm,
+              "moe_expert_ffn: NULL pointer");
+  MOE_REQUIRE(aligned16(x_perm) && aligned16(w_gate) && aligned16(w_up) && aligned16(w_down) &&
+                  aligned16(h) && aligned16(y_perm),
+              "moe_expert_ffn: tensors must be 16-byte aligned");
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  cudaError_t err;
+  if (s.dtype == MOE_F32) {
+    err = launch_ffn_simt(s, static_cast<const float*>(x_perm), expert_offsets, kept_counts,
+                          static_cast<const float*>(w_gate), static_cast<const float*>(w_up),
+                          static_cast<const float*>(w_down), static_cast<float*>(h),
+                          static_cast<float*>(y_perm), strm);
+    if (err != cudaSuccess) return cuda_fail(err, "moe_expert_ffn (fp32) launch");
+    return MOE_OK;
+  }
+  if (s.d % 64 != 0 || s.f % 64 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "bf16 expert FFN needs d_model and d_ff multiples of 64");
+  const char* why = "";
+  err = launch_ffn_tc(s, x_perm, expert_offsets, kept_counts, w_gate, w_up, w_down, h, y_perm,
+                      ws_status(ws, lay), g_wait_ns.load(), strm, &why);
+  if (err != cudaSuccess) {
+    if (why[0]) return fail(MOE_ERR_CUDA, "moe_expert_ffn: %s", why);
+    return cuda_fail(err, "moe_expert_ffn (bf16) launch");
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_combine(const moe_config_t* cfg, const void* y_perm,
+                         const int32_t* assign_row, const float* topk_w, void* out,
+                         void* stream) {
+  Shape s;
+  moe_status_t st = check_config(cfg, &s);
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(y_perm && assign_row && topk_w && out, "moe_combine: NULL pointer");
+  MOE_REQUIRE(aligned16(y_perm) && aligned16(out), "moe_combine: y_perm and out must be 16-byte aligned");
+  cudaError_t err = launch_combine(s, y_perm, assign_row, topk_w, out,
+                                   static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_combine launch");
+  return MOE_OK;
+}
+
+moe_status_t moe_load_stats(const moe_config_t* cfg, const int32_t* routed_counts,
+                            const int32_t* kept_counts, const int32_t* assign_row,
+                            moe_load_stats_t* dev_out, moe_load_stats_t* host_out,
+                            void* stream) {
+  Shape s;
+  moe_status_t st = check_config(cfg, &s);
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(routed_counts && kept_counts && assign_row && dev_out, "moe_load_stats: NULL pointer");
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  cudaError_t err = launch_stats(s, routed_counts, kept_counts, assign_row, dev_out, strm);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_load_stats launch");
+  if (host_out != nullptr) {
+    err = cudaMemcpyAsync(host_out, dev_out, sizeof(moe_load_stats_t), cudaMemcpyDeviceToHost,
+                          strm);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(strm);
+    if (err != cudaSuccess) return cuda_fail(err, "moe_load_stats copy");
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_layer_inputs_t* in,
+                               const moe_layer_buffers_t* b, void* ws, size_t ws_bytes,
+                               void* stream) {
+  MOE_REQUIRE(in != nullptr && b != nullptr, "moe_layer_forward: NULL inputs or buffers");
+  moe_status_t st = moe_route(cfg, in->x, in->w_router, in->logit_bias, in->bias_row_stride,
+                              b->logits, b->topk_idx, b->topk_w, ws, ws_bytes, stream);
+  if (st != MOE_OK) return st;
+  st = moe_dispatch(cfg, in->x, b->topk_idx, b->routed_counts, b->kept_counts,
+                    b->expert_offsets, b->assign_row, b->token_of_row, b->x_perm, ws, ws_bytes,
+                    stream);
+  if (st != MOE_OK) return st;
+  st = moe_expert_ffn(cfg, b->x_perm, b->expert_offsets, b->kept_counts, in->w_gate, in->w_up,
+                      in->w_down, b->h, b->y_perm, ws, ws_bytes, stream);
+  if (st != MOE_OK) return st;
+  st = moe_combine(cfg, b->y_perm, b->assign_row, b->topk_w, b->out, stream);
+  if (st != MOE_OK) return st;
+  if (b->stats != nullptr)
+    st = moe_load_stats(cfg, b->routed_counts, b->kept_counts, b->assign_row, b->stats, nullptr,
+                        stream);
+  return st;
+}
+
+moe_status_t moe_check_device_error(void* ws, size_t ws_bytes, void* stream) {
+  MOE_REQUIRE(ws != nullptr && ws_bytes >= sizeof(DevStatus), "moe_check_device_error: bad workspace");
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  cudaError_t err = cudaStreamSynchronize(strm);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_check_device_error sync");
+  DevStatus h;
+  err = cudaMemcpy(&h, ws, sizeof(DevStatus), cudaMemcpyDeviceToHost);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_check_device_error read");
+  if (h.code == DEV_OK) return MOE_OK;
+  err = cudaMemset(ws, 0, sizeof(DevStatus));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_check_device_error clear");
+  if (h.code == DEV_TIMEOUT)
+    return fail(MOE_ERR_TIMEOUT, "a device wait ran out (site %u, item %llu)", h.where,
+                (unsigned long long)h.info);
+  return fail(MOE_ERR_DEVICE_DATA, "invalid expert index in topk_idx (flat index %llu)",
+              (unsigned long long)h.info);
+}
+
+moe_status_t moe_selftest_bounded_wait(void* ws, size_t ws_bytes, void* stream) {
+  MOE_REQUIRE(ws != nullptr && ws_bytes >= sizeof(DevStatus), "moe_selftest_bounded_wait: bad workspace");
+  cudaError_t err = launch_wait_selftest(static_cast<DevStatus*>(ws), g_wait_ns.load(),
+                                         static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_selftest_bounded_wait launch");
+  return MOE_OK;
+}
+
+}  // extern "C"

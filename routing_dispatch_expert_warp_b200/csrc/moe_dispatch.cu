@@ -1,0 +1,267 @@
+// Dispatch on one GPU: per-expert histogram, prefix scan with the capacity limit, stable
+// ranking of every (token, pick) assignment inside its expert, and the row permutation of
+// x into expert-major buckets.
+//
+// "Expert Parallelism for MoE Serving" (aiunderstanding.org), "Technical insight": the
+// dispatch all-to-all sends every token to its experts; capacity factors and expert
+// buffers bound the rows per expert, and tokens past the capacity are dropped or the
+// bucket is padded.  "MoE expert parallelism needs measurements before launch"
+// (airouter.kz), "Profile all-to-all separately from compute": pack/permute comes before
+// the exchange, and with EP=1 the exchange itself disappears -- what remains is this
+// local permutation.
+//
+// Assignment order: within expert e, assignments are ranked by token index (a token picks
+// an expert at most once, so its pick slot j does not matter).  slot < C is kept.
+//
+// Kernels (no host synchronisation anywhere):
+//   1. count:  block b of 256 tokens builds, per warp w and expert e, the 32-bit mask of
+//              lanes (tokens) that picked e; per-block counts = sum of popcounts.
+//   2. scan:   one block: per expert, exclusive scan of the block counts (the block's base
+//              slot), routed = total, kept = min(routed, C), bucket offsets.
+//   3. rank:   block b rebuilds its masks; slot = block base + earlier warps' counts +
+//              popcount(mask & lanes below me).  Writes assign_row and token_of_row.
+//   4. permute: token-major row copy with bulk (TMA) copies: each row of x is read from HBM
+//              once into shared memory and written to each of its kept rows of x_perm.
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kWarps = kDispatchBlockTokens / 32;
+
+// Fill masks[w][e] for the block's tokens.  Returns nothing; invalid experts are recorded.
+__device__ __forceinline__ void build_masks(const int32_t* __restrict__ topk_idx, int64_t T,
+                                            int k, int E, uint32_t (*masks)[MOE_MAX_EXPERTS],
+                                            DevStatus* status) {
+  for (int i = threadIdx.x; i < kWarps * MOE_MAX_EXPERTS; i += blockDim.x)
+    (&masks[0][0])[i] = 0u;
+  __syncthreads();
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kDispatchBlockTokens + threadIdx.x;
+  const int w = threadIdx.x >> 5;
+  const uint32_t bit = 1u << (threadIdx.x & 31);
+  if (t < T) {
+    for (int j = 0; j < k; ++j) {
+      const int e = topk_idx[t * k + j];
+      if (e < 0 || e >= E) {
+        record_error(status, DEV_BAD_EXPERT, 1, static_cast<unsigned long long>(t * k + j));
+        continue;
+      }
+      atomicOr(&masks[w][e], bit);
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_count_kernel(
+    const int32_t* __restrict__ topk_idx, int64_t T, int k, int E, int32_t* __restrict__ hist,
+    DevStatus* status) {
+  __shared__ uint32_t masks[kWarps][MOE_MAX_EXPERTS];
+  build_masks(topk_idx, T, k, E, masks, status);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) c += __popc(masks[w][e]);
+    hist[static_cast<int64_t>(blockIdx.x) * E + e] = c;
+  }
+}
+
+// One block of MOE_MAX_EXPERTS threads, thread e owns expert e.
+__global__ void __launch_bounds__(MOE_MAX_EXPERTS) dispatch_scan_kernel(
+    int32_t* __restrict__ hist, int64_t nblk, int E, int64_t C, int layout,
+    int32_t* __restrict__ routed, int32_t* __restrict__ kept, int32_t* __restrict__ offsets) {
+  __shared__ int64_t scan[MOE_MAX_EXPERTS];
+  const int e = threadIdx.x;
+  int64_t run = 0;
+  if (e < E) {
+    for (int64_t b = 0; b < nblk; ++b) {
+      const int32_t c = hist[b * E + e];
+      hist[b * E + e] = static_cast<int32_t>(run);  // becomes the block's base slot
+      run += c;
+    }
+  }
+  const int64_t kp = (e < E) ? ((C >= 0 && run > C) ? C : run) : 0;
+  if (e < E) {
+    routed[e] = static_cast<int32_t>(run);
+    kept[e] = static_cast<int32_t>(kp);
+  }
+  // inclusive scan of kept over experts (Hillis-Steele, 256 entries)
+  scan[e] = kp;
+  __syncthreads();
+  for (int off = 1; off < MOE_MAX_EXPERTS; off <<= 1) {
+    const int64_t add = e >= off ? scan[e - off] : 0;
+    __syncthreads();
+    scan[e] += add;
+    __syncthreads();
+  }
+  if (e < E) {
+    if (layout == MOE_LAYOUT_PADDED) {
+      offsets[e] = static_cast<int32_t>(static_cast<int64_t>(e) * C);
+      if (e == E - 1) offsets[E] = static_cast<int32_t>(static_cast<int64_t>(E) * C);
+    } else {
+      offsets[e] = static_cast<int32_t>(scan[e] - kp);
+      if (e == E - 1) offsets[E] = static_cast<int32_t>(scan[e]);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
+    const int32_t* __restrict__ topk_idx, int64_t T, int k, int E, int64_t C,
+    const int32_t* __restrict__ base, const int32_t* __restrict__ offsets,
+    int32_t* __restrict__ assign_row, int32_t* __restrict__ token_of_row, DevStatus* status) {
+  __shared__ uint32_t masks[kWarps][MOE_MAX_EXPERTS];
+  __shared__ int32_t wbase[kWarps][MOE_MAX_EXPERTS];
+  __shared__ int32_t off_s[MOE_MAX_EXPERTS];
+  build_masks(topk_idx, T, k, E, masks, nullptr);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int32_t run = base[static_cast<int64_t>(blockIdx.x) * E + e];
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      wbase[w][e] = run;
+      run += __popc(masks[w][e]);
+    }
+    off_s[e] = offsets[e];
+  }
+  __syncthreads();
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * kDispatchBlockTokens + threadIdx.x;
+  if (t >= T) return;
+  const int w = threadIdx.x >> 5;
+  const uint32_t below = (1u << (threadIdx.x & 31)) - 1u;
+  for (int j = 0; j < k; ++j) {
+    const int e = topk_idx[t * k + j];
+    int32_t row = -1;
+    if (e >= 0 && e < E) {
+      const int64_t slot = wbase[w][e] + __popc(masks[w][e] & below);
+      if (C < 0 || slot < C) {
+        row = off_s[e] + static_cast<int32_t>(slot);
+        token_of_row[row] = static_cast<int32_t>(t);
+      }
+    }
+    assign_row[t * k + j] = row;
+  }
+}
+
+// Token-major bulk copy.  One thread per block issues everything: a ring of NBUF shared
+// buffers, LOOKAHEAD loads in flight, stores of the rows already loaded in flight
+// behind them.  A work item is one segment (<= 16 KB) of one token's row.
+constexpr int kPermNBuf = 8;
+constexpr int kPermLookahead = 4;
+constexpr uint32_t kPermMaxSeg = 16384;
+
+__global__ void __launch_bounds__(32) permute_rows_kernel(
+    const uint8_t* __restrict__ x, const int32_t* __restrict__ assign_row, int64_t T, int k,
+    int64_t row_bytes, uint32_t seg_bytes, int64_t segs_per_row, uint8_t* __restrict__ x_perm,
+    DevStatus* status, uint64_t wait_ns) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ __align__(8) uint64_t full[kPermNBuf];
+  if (threadIdx.x != 0) return;
+  for (int b = 0; b < kPermNBuf; ++b) mbar_init(&full[b], 1);
+  fence_barrier_init();
+
+  const int64_t items = T * segs_per_row;
+  const int64_t first = blockIdx.x, step = gridDim.x;
+  const int64_t n = first < items ? (items - first + step - 1) / step : 0;
+  uint32_t phase_bits = 0;  // parity of the next completion per buffer
+  uint32_t armed = 0;       // buffers with a load in flight
+
+  auto item_rows_any = [&](int64_t it) {
+    const int64_t t = it / segs_per_row;
+    for (int j = 0; j < k; ++j)
+      if (assign_row[t * k + j] >= 0) return true;
+    return false;
+  };
+  auto issue_load = [&](int64_t i) {
+    const int64_t it = first + i * step;
+    const int64_t t = it / segs_per_row, sg = it % segs_per_row;
+    const int b = static_cast<int>(i % kPermNBuf);
+    const int64_t off = sg * seg_bytes;
+    const uint32_t bytes = static_cast<uint32_t>(
+        row_bytes - off < static_cast<int64_t>(seg_bytes) ? row_bytes - off : seg_bytes);
+    armed |= 1u << b;
+    mbar_arrive_expect_tx(&full[b], bytes);
+    bulk_load(smem + static_cast<size_t>(b) * seg_bytes, x + t * row_bytes + off, bytes,
+              &full[b]);
+  };
+
+  // Tokens whose picks were all dropped are skipped: their buffer is never filled and
+  // their barrier never armed, so skipping must be decided identically at issue and use.
+  for (int64_t i = 0; i < n && i < kPermLookahead; ++i)
+    if (item_rows_any(first + i * step)) issue_load(i);
+
+  for (int64_t i = 0; i < n; ++i) {
+    const int64_t it = first + i * step;
+    const int b = static_cast<int>(i % kPermNBuf);
+    if (item_rows_any(it)) {
+      const int64_t t = it / segs_per_row, sg = it % segs_per_row;
+      const int64_t off = sg * seg_bytes;
+      const uint32_t bytes = static_cast<uint32_t>(
+          row_bytes - off < static_cast<int64_t>(seg_bytes) ? row_bytes - off : seg_bytes);
+      if (!mbar_wait(&full[b], (phase_bits >> b) & 1u, wait_ns, nullptr)) {
+        record_error(status, DEV_TIMEOUT, 10, static_cast<unsigned long long>(it));
+        // drain: let every load still in flight land before the block exits
+        for (int q = 0; q < kPermNBuf; ++q)
+          if ((armed >> q) & 1u) mbar_wait(&full[q], (phase_bits >> q) & 1u, wait_ns, nullptr);
+        bulk_wait_all();
+        return;
+      }
+      phase_bits ^= (1u << b);
+      armed &= ~(1u << b);
+      for (int j = 0; j < k; ++j) {
+        const int32_t r = assign_row[t * k + j];
+        if (r >= 0)
+          bulk_store(x_perm + static_cast<int64_t>(r) * row_bytes + off,
+                     smem + static_cast<size_t>(b) * seg_bytes, bytes);
+      }
+    }
+    bulk_commit();  // one group per item (possibly empty) keeps the group count regular
+    const int64_t nxt = i + kPermLookahead;
+    if (nxt < n) {
+      // buffer nxt % NBUF was last read by the stores of item nxt - NBUF; at most
+      // NBUF - LOOKAHEAD groups committed after it may still be reading
+      bulk_wait_read<kPermNBuf - kPermLookahead>();
+      if (item_rows_any(first + nxt * step)) issue_load(nxt);
+    }
+  }
+  bulk_wait_all();
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_idx,
+                            int32_t* routed, int32_t* kept, int32_t* offsets,
+                            int32_t* assign_row, int32_t* token_of_row, void* x_perm,
+                            int32_t* hist, DevStatus* status, uint64_t wait_ns,
+                            cudaStream_t st) {
+  const int64_t nblk = dispatch_blocks(s.T);
+  cudaError_t err = cudaMemsetAsync(token_of_row, 0xFF, sizeof(int32_t) * s.max_rows, st);
+  if (err != cudaSuccess) return err;
+  dispatch_count_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
+      topk_idx, s.T, s.k, s.E, hist, status);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  dispatch_scan_kernel<<<1, MOE_MAX_EXPERTS, 0, st>>>(hist, nblk, s.E, s.C, s.layout, routed,
+                                                      kept, offsets);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  dispatch_rank_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
+      topk_idx, s.T, s.k, s.E, s.C, hist, offsets, assign_row, token_of_row, status);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+
+  const int64_t row_bytes = s.d * s.elem;
+  const int64_t segs = (row_bytes + kPermMaxSeg - 1) / kPermMaxSeg;
+  // equal segments, each a multiple of 16 bytes
+  int64_t seg = (row_bytes + segs - 1) / segs;
+  seg = (seg + 15) / 16 * 16;
+  const size_t smem = static_cast<size_t>(kPermNBuf) * seg;
+  err = cudaFuncSetAttribute(permute_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kPermNBuf * kPermMaxSeg));
+  if (err != cudaSuccess) return err;
+  const int64_t items = s.T * segs;
+  const int64_t per_sm = smem <= 64 * 1024 ? 3 : (smem <= 100 * 1024 ? 2 : 1);
+  int64_t grid = static_cast<int64_t>(sm_count()) * per_sm;
+  if (grid > items) grid = items;
+  if (grid < 1) grid = 1;
+  permute_rows_kernel<<<static_cast<unsigned>(grid), 32, smem, st>>>(
+      static_cast<const uint8_t*>(x), assign_row, s.T, s.k, row_bytes,
+      static_cast<uint32_t>(seg), segs, static_cast<uint8_t*>(x_perm), status, wait_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

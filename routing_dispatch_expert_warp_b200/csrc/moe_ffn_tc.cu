@@ -1,0 +1,420 @@
+// Expert SwiGLU FFN for bf16 layers: a grouped GEMM on the 5th-generation tensor cores
+// (tcgen05 MMA with accumulators in tensor memory), fed by TMA, over the variable-sized
+// expert buckets that dispatch produced.
+//
+// "MoE expert parallelism needs measurements before launch" (airouter.kz), "Profile
+// all-to-all separately from compute": expert compute runs as grouped GEMMs over many
+// experts; "Expert Parallelism for MoE Serving" (aiunderstanding.org), "Technical
+// insight": capacity and padding exist to keep those GEMMs regular -- here the kernel
+// takes the ragged buckets as they are and masks the tails.
+//
+// Two launches of one persistent kernel template:
+//   gate/up (GATED): for a 128-row x 128-column tile of h, the B operand is the 128 rows of
+//     W_g[e] stacked on the same 128 rows of W_u[e] (256 rows), so one 128x256x16 MMA per
+//     K step produces the gate tile in TMEM columns [0,128) and the up tile in [128,256);
+//     the epilogue writes h = silu(gate) * up as bf16.
+//   down: a 128 x 256 tile of y_perm = h . W_d[e]^T with a plain bf16 epilogue.
+//
+// Block = 6 warps, one block per SM, persistent over tiles:
+//   warp 0 (one lane)   TMA producer: A = 128 x 64 bf16 slice of x_perm/h rows, B = 256 x 64
+//                       slice of the expert's weights, 128-byte swizzle, 4-stage ring.
+//   warp 1 (one lane)   MMA issuer: 4 MMAs (K = 16 each) per stage into one of two TMEM
+//                       accumulators (256 fp32 columns each); commits free the smem stage
+//                       and, at the end of a tile, hand the accumulator to the epilogue.
+//   warps 2-5           epilogue: each thread owns one accumulator row (TMEM lane), reads
+//                       it 32 columns at a time, converts and stores; the accumulator is
+//                       returned while the MMA warp already fills the other one.
+// Tiles are numbered expert by expert, n-block by n-block, with the m-blocks of one
+// (expert, n-block) consecutive, so the blocks running at the same time share weight tiles
+// through L2.  The tile table is built on the device from the bucket counts: no host read.
+// Every barrier wait is bounded; a wait that runs out records MOE_ERR_TIMEOUT, makes the
+// other roles stop, drains the copies and MMAs in flight, frees TMEM and returns.
+#include <mutex>
+
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int MMA_N = 256;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = MMA_N * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int THREADS = 192;
+constexpr int ACC_COLS = 256;
+constexpr int TMEM_COLS = 512;
+constexpr int DYN_SMEM = STAGES * STAGE_BYTES + 1024;  // + alignment slack
+
+struct TcParams {
+  const int32_t* seg_start;  // [E] first row of each bucket
+  const int32_t* seg_count;  // [E] rows of each bucket
+  int E;
+  int K;         // reduction length (multiple of 64)
+  int n_blocks;  // output column blocks
+  int N_out;     // output columns (multiple of 64)
+  __nv_bfloat16* out;
+  DevStatus* status;
+  uint64_t wait_ns;
+};
+
+__device__ __forceinline__ void decode_tile(int tile, const int* tile_base, const int* mblocks,
+                                            int E, int& e, int& mb, int& nb) {
+  int lo = 0, hi = E - 1;  // largest e with tile_base[e] <= tile
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tile_base[mid] <= tile) lo = mid;
+    else hi = mid - 1;
+  }
+  e = lo;
+  const int local = tile - tile_base[e];
+  const int mbs = mblocks[e];
+  nb = local / mbs;
+  mb = local - nb * mbs;
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return g / (1.0f + __expf(-g)) * u;
+}
+
+template <bool GATED>
+__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
+    const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
+    const __grid_constant__ CUtensorMap tm_b1, const TcParams p) {
+  constexpr int BN_OUT = GATED ? 128 : 256;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int abort_s;
+  __shared__ int tile_base[MOE_MAX_EXPERTS + 1];
+  __shared__ int mblocks[MOE_MAX_EXPERTS];
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (warp == 0) {  // tile table: m-blocks per expert and their prefix (x n_blocks)
+    int carry = 0;
+    for (int e0 = 0; e0 < p.E; e0 += 32) {
+      const int e = e0 + lane;
+      const int mb = e < p.E ? (p.seg_count[e] + BM - 1) / BM : 0;
+      int v = mb;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += o;
+      }
+      if (e < p.E) {
+        mblocks[e] = mb;
+        tile_base[e] = (carry + v - mb) * p.n_blocks;
+      }
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) tile_base[p.E] = carry * p.n_blocks;
+    if (lane == 0) {
+      prefetch_tensormap(&tm_a);
+      prefetch_tensormap(&tm_b0);
+      if (GATED) prefetch_tensormap(&tm_b1);
+    }
+  } else if (warp == 1) {
+    tmem_alloc(&tmem_base_s, TMEM_COLS);
+    tmem_relinquish();
+  } else if (threadIdx.x == 64) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 128);
+    }
+    mbar_init(&drain_bar, 1);
+    abort_s = 0;
+    fence_barrier_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem_base = tmem_base_s;
+  const int total_tiles = tile_base[p.E];
+  const int KB = p.K / BK;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    int s = 0;
+    uint32_t ph = 0;
+    uint32_t armed = 0, armed_parity = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      int e, mb, nb;
+      decode_tile(tile, tile_base, mblocks, p.E, e, mb, nb);
+      const int row0 = p.seg_start[e] + mb * BM;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&empty_bar[s], ph ^ 1u, p.wait_ns, &abort_s)) {
+          if (!abort_s) record_error(p.status, DEV_TIMEOUT, 20, static_cast<unsigned long long>(tile));
+          abort_s = 1;
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + s * STAGE_BYTES;
+        uint8_t* sb = sa + A_BYTES;
+        mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
+        armed |= 1u << s;
+        armed_parity = (armed_parity & ~(1u << s)) | (ph << s);
+        tma_load_2d(sa, &tm_a, &full_bar[s], kb * BK, row0);
+        if (GATED) {
+          tma_load_3d(sb, &tm_b0, &full_bar[s], kb * BK, nb * 128, e);
+          tma_load_3d(sb + B_BYTES / 2, &tm_b1, &full_bar[s], kb * BK, nb * 128, e);
+        } else {
+          tma_load_3d(sb, &tm_b0, &full_bar[s], kb * BK, nb * 256, e);
+        }
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+    // every fill this thread armed must land before the block can exit
+    for (int q = 0; q < STAGES; ++q)
+      if ((armed >> q) & 1u) mbar_wait(&full_bar[q], (armed_parity >> q) & 1u, p.wait_ns, nullptr);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(BM, MMA_N);
+    int s = 0;
+    uint32_t ph = 0;
+    int acc = 0;
+    uint32_t aph = 0;
+    bool ok = true;
+    bool issued = false;
+    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      if (!mbar_wait(&tempty_bar[acc], aph ^ 1u, p.wait_ns, &abort_s)) {
+        if (!abort_s) record_error(p.status, DEV_TIMEOUT, 21, static_cast<unsigned long long>(tile));
+        abort_s = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_COLS);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&full_bar[s], ph, p.wait_ns, &abort_s)) {
+          if (!abort_s) record_error(p.status, DEV_TIMEOUT, 22, static_cast<unsigned long long>(tile));
+          abort_s = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = smem_addr(smem + s * STAGE_BYTES);
+        const uint32_t b_addr = a_addr + A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          tc_mma_f16(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
+                     sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+        issued = true;
+        tc_commit(&empty_bar[s]);
+        if (++s == STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (!ok) break;
+      tc_commit(&tfull_bar[acc]);
+      acc ^= 1;
+      if (acc == 0) aph ^= 1u;
+    }
+    if (!ok && issued) {  // MMAs still reading smem / writing TMEM must finish first
+      tc_commit(&drain_bar);
+      mbar_wait(&drain_bar, 0, p.wait_ns, nullptr);
+    }
+  } else if (warp >= 2) {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;             // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;        // accumulator row owned by this thread
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+      int e, mb, nb;
+      decode_tile(tile, tile_base, mblocks, p.E, e, mb, nb);
+      const int row0 = p.seg_start[e] + mb * BM;
+      const int valid = p.seg_count[e] - mb * BM;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&tfull_bar[acc], aph, p.wait_ns, &abort_s) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0 && !abort_s) record_error(p.status, DEV_TIMEOUT, 23, static_cast<unsigned long long>(tile));
+        abort_s = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * ACC_COLS);
+      const bool row_ok = r < valid;
+      __nv_bfloat16* orow =
+          p.out + static_cast<int64_t>(row0 + r) * p.N_out + static_cast<int64_t>(nb) * BN_OUT;
+      const int cols_left = p.N_out - nb * BN_OUT;
+      if (GATED) {
+#pragma unroll 1
+        for (int c = 0; c < BN_OUT / 32; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld32(taddr + c * 32, g);
+          tmem_ld32(taddr + 128 + c * 32, u);
+          tmem_ld_wait();
+          if (row_ok && c * 32 < cols_left) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                                  silu_mul(__uint_as_float(g[2 * i + 1]),
+                                           __uint_as_float(u[2 * i + 1])));
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN_OUT / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c * 32, v);
+          tmem_ld_wait();
+          if (row_ok && c * 32 < cols_left) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty_bar[acc]);
+      acc ^= 1;
+      if (acc == 0) aph ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
+                                         cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// [rows, K] bf16 row-major, box 128 rows x 64 columns, 128-byte swizzle
+bool make_map_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K * 2)};
+  const cuuint32_t box[2] = {BK, BM};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [E, N, K] bf16 weights, box 1 x box_n x 64, 128-byte swizzle
+bool make_map_weights(CUtensorMap* m, const void* base, int E, int64_t N, int64_t K,
+                      int box_n) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(E)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K * 2),
+                                 static_cast<cuuint64_t>(N * K * 2)};
+  const cuuint32_t box[3] = {BK, static_cast<cuuint32_t>(box_n), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_tc(const Shape& s, const void* x_perm, const int32_t* offsets,
+                          const int32_t* kept, const void* wg, const void* wu, const void* wd,
+                          void* h, void* y, DevStatus* status, uint64_t wait_ns,
+                          cudaStream_t st, const char** why) {
+  if (encode_fn() == nullptr) {
+    *why = "cuTensorMapEncodeTiled is not available from the driver";
+    return cudaErrorNotSupported;
+  }
+  CUtensorMap ta1, tg, tu, ta2, td;
+  if (!make_map_rows(&ta1, x_perm, s.max_rows, s.d) ||
+      !make_map_weights(&tg, wg, s.E, s.f, s.d, 128) ||
+      !make_map_weights(&tu, wu, s.E, s.f, s.d, 128) ||
+      !make_map_rows(&ta2, h, s.max_rows, s.f) ||
+      !make_map_weights(&td, wd, s.E, s.d, s.f, 256)) {
+    *why = "tensor map encoding failed (pointer alignment or sizes)";
+    return cudaErrorInvalidValue;
+  }
+  cudaError_t err;
+  err = cudaFuncSetAttribute(grouped_gemm_tc_kernel<true>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, DYN_SMEM);
+  if (err != cudaSuccess) return err;
+  err = cudaFuncSetAttribute(grouped_gemm_tc_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, DYN_SMEM);
+  if (err != cudaSuccess) return err;
+
+  const int64_t row_blocks_bound = (s.max_rows + BM - 1) / BM + s.E;
+  const int sms = sm_count();
+
+  TcParams p1;
+  p1.seg_start = offsets;
+  p1.seg_count = kept;
+  p1.E = s.E;
+  p1.K = static_cast<int>(s.d);
+  p1.n_blocks = static_cast<int>((s.f + 127) / 128);
+  p1.N_out = static_cast<int>(s.f);
+  p1.out = static_cast<__nv_bfloat16*>(h);
+  p1.status = status;
+  p1.wait_ns = wait_ns;
+  int64_t g1 = row_blocks_bound * p1.n_blocks;
+  if (g1 > sms) g1 = sms;
+  grouped_gemm_tc_kernel<true><<<static_cast<unsigned>(g1), THREADS, DYN_SMEM, st>>>(ta1, tg, tu,
+                                                                                    p1);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+
+  TcParams p2 = p1;
+  p2.K = static_cast<int>(s.f);
+  p2.n_blocks = static_cast<int>((s.d + 255) / 256);
+  p2.N_out = static_cast<int>(s.d);
+  p2.out = static_cast<__nv_bfloat16*>(y);
+  int64_t g2 = row_blocks_bound * p2.n_blocks;
+  if (g2 > sms) g2 = sms;
+  grouped_gemm_tc_kernel<false><<<static_cast<unsigned>(g2), THREADS, DYN_SMEM, st>>>(ta2, td, td,
+                                                                                     p2);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

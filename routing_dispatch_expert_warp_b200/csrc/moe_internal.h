@@ -1,0 +1,65 @@
+// Host-side declarations shared by the translation units of the MoE library: the checked
+// layer shape, the workspace layout and the kernel launchers.  Not part of the C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+#include "moe_device.cuh"
+
+namespace moe {
+
+constexpr int kDispatchBlockTokens = 256;   // tokens per block of the ranking kernels
+constexpr size_t kWsAlign = 256;
+
+// A validated moe_config_t with the derived sizes.
+struct Shape {
+  int64_t T, d, f;
+  int E, k, gating, layout, dtype;
+  int64_t C;         // capacity, -1 when dropless
+  int64_t max_rows;  // rows of x_perm / h / y_perm / token_of_row
+  int64_t elem;      // bytes per element of x, weights and activations
+};
+
+// Offsets (bytes) of the workspace sections.
+struct WsLayout {
+  size_t status;        // DevStatus, 256 B
+  size_t hist;          // [n_dispatch_blocks, E] int32 per-block counts, then bases
+  size_t hist_bytes;
+  size_t logits;        // [T, E] fp32 logits when the caller passes none
+  size_t logits_bytes;
+  size_t total;
+};
+
+inline int64_t dispatch_blocks(int64_t T) {
+  return (T + kDispatchBlockTokens - 1) / kDispatchBlockTokens;
+}
+WsLayout workspace_layout(const Shape& s);
+
+// Kernel launchers (return the CUDA error of the launch).
+cudaError_t launch_router(const Shape& s, const void* x, const float* w_router,
+                          const float* bias, int64_t bias_stride, float* logits,
+                          int32_t* topk_idx, float* topk_w, cudaStream_t st);
+cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_idx,
+                            int32_t* routed, int32_t* kept, int32_t* offsets,
+                            int32_t* assign_row, int32_t* token_of_row, void* x_perm,
+                            int32_t* hist, DevStatus* status, uint64_t wait_ns,
+                            cudaStream_t st);
+cudaError_t launch_ffn_simt(const Shape& s, const float* x_perm, const int32_t* offsets,
+                            const int32_t* kept, const float* wg, const float* wu,
+                            const float* wd, float* h, float* y, cudaStream_t st);
+cudaError_t launch_ffn_tc(const Shape& s, const void* x_perm, const int32_t* offsets,
+                          const int32_t* kept, const void* wg, const void* wu, const void* wd,
+                          void* h, void* y, DevStatus* status, uint64_t wait_ns,
+                          cudaStream_t st, const char** why);
+cudaError_t launch_combine(const Shape& s, const void* y_perm, const int32_t* assign_row,
+                           const float* topk_w, void* out, cudaStream_t st);
+cudaError_t launch_stats(const Shape& s, const int32_t* routed, const int32_t* kept,
+                         const int32_t* assign_row, moe_load_stats_t* out, cudaStream_t st);
+cudaError_t launch_wait_selftest(DevStatus* status, uint64_t wait_ns, cudaStream_t st);
+
+int sm_count();
+
+}  // namespace moe

@@ -1,0 +1,366 @@
+// Router scoring, top-k selection and renormalised gate weights.
+//
+// "Expert Parallelism for MoE Serving" (aiunderstanding.org), "Deep dive": a router
+// scores the experts for every token and picks the top-k of them.  Here:
+//   z[t, e]  = sum_i x[t, i] * W_r[i, e] + b[t, e]        (fp32 FMA, fixed order)
+//   picks    = the k largest z[t, :], best first; equal z -> lower expert index
+//   weights  = softmax or sigmoid of the picked logits, renormalised over the k picks.
+//
+// Two kernels:
+//   * E <= 32: one fused kernel.  A warp scores 32/ET tokens at once (ET = 8, 16 or 32
+//     expert slots), every lane walking a strided slice of d with 16-byte loads of x; a
+//     transposing butterfly reduction leaves lane l with the logit of (token l / ET,
+//     expert l % ET); each group of ET lanes then selects its token's top-k with
+//     shuffles.  The pass is bound by reading x once from HBM.
+//   * E > 32: a tiled fp32 GEMM writes z (64 tokens x 128 experts per block), then a warp
+//     per token selects the top-k from z.
+#include <math.h>
+
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+template <typename TX>
+struct XLoad;
+template <>
+struct XLoad<float> {
+  // 8 consecutive fp32 values (two 16-byte loads)
+  static __device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+};
+template <>
+struct XLoad<__nv_bfloat16> {
+  // 8 consecutive bf16 values (one 16-byte load), widened exactly to fp32
+  static __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+    v[0] = bf16_lo(a.x); v[1] = bf16_hi(a.x); v[2] = bf16_lo(a.y); v[3] = bf16_hi(a.y);
+    v[4] = bf16_lo(a.z); v[5] = bf16_hi(a.z); v[6] = bf16_lo(a.w); v[7] = bf16_hi(a.w);
+  }
+};
+
+// (valid, value, index) ordering of the top-k: larger value first, then lower index.
+__device__ __forceinline__ bool better(bool va, float a, int ia, bool vb, float b, int ib) {
+  if (va != vb) return va;
+  if (a != b) return a > b;
+  return ia < ib;
+}
+
+// Gate weights of one token from its k picked logits (best first), fp32.
+__device__ __forceinline__ void gate_weights(const float* zsel, int k, int gating, float* w) {
+  float s = 0.f;
+  if (gating == MOE_GATE_SOFTMAX) {
+    const float m = zsel[0];
+    for (int j = 0; j < k; ++j) {
+      w[j] = expf(zsel[j] - m);
+      s += w[j];
+    }
+  } else {
+    for (int j = 0; j < k; ++j) {
+      w[j] = 1.0f / (1.0f + expf(-zsel[j]));
+      s += w[j];
+    }
+  }
+  const float inv = 1.0f / s;
+  for (int j = 0; j < k; ++j) w[j] *= inv;
+}
+
+template <typename TX, int ET>
+__global__ void __launch_bounds__(256) router_small_e_kernel(
+    const TX* __restrict__ x, const float* __restrict__ w_router, const float* __restrict__ bias,
+    int64_t bias_stride, int64_t T, int d, int E, int k, int gating, float* __restrict__ logits,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  constexpr int TW = 32 / ET;  // tokens per warp
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const bool e_vec4 = (E % 4) == 0;
+
+  for (int64_t t0 = warp * TW; t0 < T; t0 += nwarps * TW) {
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = 0.f;
+
+    for (int i0 = lane * 8; i0 < d; i0 += 256) {
+      float xv[TW][8];
+#pragma unroll
+      for (int tw = 0; tw < TW; ++tw) {
+        if (t0 + tw < T) {
+          XLoad<TX>::load8(x + (t0 + tw) * d + i0, xv[tw]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) xv[tw][q] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int ii = 0; ii < 8; ++ii) {
+        float wv[ET];
+        const float* wrow = w_router + static_cast<int64_t>(i0 + ii) * E;
+        if (e_vec4) {
+#pragma unroll
+          for (int q = 0; q < ET / 4; ++q) {
+            if (4 * q < E) {
+              const float4 f = __ldg(reinterpret_cast<const float4*>(wrow) + q);
+              wv[4 * q] = f.x; wv[4 * q + 1] = f.y; wv[4 * q + 2] = f.z; wv[4 * q + 3] = f.w;
+            } else {
+              wv[4 * q] = wv[4 * q + 1] = wv[4 * q + 2] = wv[4 * q + 3] = 0.f;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < ET; ++e) wv[e] = e < E ? __ldg(wrow + e) : 0.f;
+        }
+#pragma unroll
+        for (int tw = 0; tw < TW; ++tw)
+#pragma unroll
+          for (int e = 0; e < ET; ++e) v[tw * ET + e] = fmaf(xv[tw][ii], wv[e], v[tw * ET + e]);
+      }
+    }
+
+    // Butterfly transpose-reduction: afterwards lane l holds the full sum of value l.
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      const bool upper = (lane & off) != 0;
+#pragma unroll
+      for (int i = 0; i < off; ++i) {
+        const float send = upper ? v[i] : v[i + off];
+        const float keep = upper ? v[i + off] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+      }
+    }
+
+    const int tw = lane / ET;
+    const int e = lane % ET;
+    const int64_t t = t0 + tw;
+    const bool valid = (e < E) && (t < T);
+    float z = v[0];
+    if (valid) {
+      if (bias != nullptr) z += bias[t * bias_stride + e];
+      if (logits != nullptr) logits[t * E + e] = z;
+    }
+
+    // top-k within each group of ET lanes (one token per group)
+    bool taken = false;
+    float zsel[MOE_MAX_TOPK];
+    int isel[MOE_MAX_TOPK];
+    for (int j = 0; j < k; ++j) {
+      bool bv = valid && !taken;
+      float bz = z;
+      int bi = e;
+#pragma unroll
+      for (int off = ET / 2; off >= 1; off >>= 1) {
+        const bool ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const float oz = __shfl_xor_sync(0xffffffffu, bz, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (better(ov, oz, oi, bv, bz, bi)) {
+          bv = ov; bz = oz; bi = oi;
+        }
+      }
+      if (bi == e) taken = true;
+      zsel[j] = bz;
+      isel[j] = bi;
+    }
+    if (e == 0 && t < T) {
+      float w[MOE_MAX_TOPK];
+      gate_weights(zsel, k, gating, w);
+      for (int j = 0; j < k; ++j) {
+        topk_idx[t * k + j] = isel[j];
+        topk_w[t * k + j] = w[j];
+      }
+    }
+  }
+}
+
+// z = x W_r + b as a tiled fp32 GEMM: 64 tokens x 128 experts per block, K steps of 32.
+constexpr int RT_M = 64, RT_N = 128, RT_K = 32;
+
+template <typename TX>
+__global__ void __launch_bounds__(256) router_gemm_kernel(
+    const TX* __restrict__ x, const float* __restrict__ w_router, const float* __restrict__ bias,
+    int64_t bias_stride, int64_t T, int d, int E, float* __restrict__ z) {
+  __shared__ __align__(16) float xs[RT_K][RT_M];
+  __shared__ __align__(16) float ws[RT_K][RT_N];
+  const int tid = threadIdx.x;
+  const int ty = tid / 16, tx = tid % 16;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * RT_M;
+  const int n0 = blockIdx.x * RT_N;
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+  for (int k0 = 0; k0 < d; k0 += RT_K) {
+    {  // x tile: 64 rows x 32 columns, 8 consecutive elements per thread, stored transposed
+      const int r = tid / 4, c = (tid % 4) * 8;
+      float v[8];
+      const int64_t t = m0 + r;
+      if (t < T && k0 + c + 8 <= d) {
+        XLoad<TX>::load8(x + t * d + k0 + c, v);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          v[q] = (t < T && k0 + c + q < d) ? static_cast<float>(x[t * d + k0 + c + q]) : 0.f;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) xs[c + q][r] = v[q];
+    }
+    {  // W tile: 32 rows x 128 experts
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int r = tid / 32 + 8 * q, c = (tid % 32) * 4;
+        const int kk = k0 + r;
+        float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (kk < d) {
+          const float* src = w_router + static_cast<int64_t>(kk) * E + n0 + c;
+          if (n0 + c + 4 <= E && (E % 4) == 0) {
+            f = __ldg(reinterpret_cast<const float4*>(src));
+          } else {
+            f.x = n0 + c + 0 < E ? src[0] : 0.f;
+            f.y = n0 + c + 1 < E ? src[1] : 0.f;
+            f.z = n0 + c + 2 < E ? src[2] : 0.f;
+            f.w = n0 + c + 3 < E ? src[3] : 0.f;
+          }
+        }
+        *reinterpret_cast<float4*>(&ws[r][c]) = f;
+      }
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < RT_K; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&xs[kk][4 * ty]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&ws[kk][4 * tx]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&ws[kk][64 + 4 * tx]);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t t = m0 + 4 * ty + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = n0 + (j < 4 ? 4 * tx + j : 64 + 4 * tx + (j - 4));
+      if (e >= E) continue;
+      float zz = acc[i][j];
+      if (bias != nullptr) zz += bias[t * bias_stride + e];
+      z[t * E + e] = zz;
+    }
+  }
+}
+
+// A warp per token: the top-k of z[t, 0..E) (E <= 256, up to 8 values per lane).
+__global__ void __launch_bounds__(256) topk_from_logits_kernel(
+    const float* __restrict__ z, int64_t T, int E, int k, int gating,
+    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  for (int64_t t = warp; t < T; t += nwarps) {
+    float zv[8];
+    bool live[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int e = lane + 32 * q;
+      live[q] = e < E;
+      zv[q] = live[q] ? z[t * E + e] : 0.f;
+    }
+    float zsel[MOE_MAX_TOPK];
+    int isel[MOE_MAX_TOPK];
+    for (int j = 0; j < k; ++j) {
+      // best of this lane
+      bool bv = false;
+      float bz = 0.f;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (better(live[q], zv[q], lane + 32 * q, bv, bz, bi)) {
+          bv = live[q]; bz = zv[q]; bi = lane + 32 * q;
+        }
+      }
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) {
+        const bool ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const float oz = __shfl_xor_sync(0xffffffffu, bz, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+        if (better(ov, oz, oi, bv, bz, bi)) {
+          bv = ov; bz = oz; bi = oi;
+        }
+      }
+      zsel[j] = bz;
+      isel[j] = bi;
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (lane + 32 * q == bi) live[q] = false;
+    }
+    if (lane == 0) {
+      float w[MOE_MAX_TOPK];
+      gate_weights(zsel, k, gating, w);
+      for (int j = 0; j < k; ++j) {
+        topk_idx[t * k + j] = isel[j];
+        topk_w[t * k + j] = w[j];
+      }
+    }
+  }
+}
+
+template <typename TX>
+cudaError_t launch_router_typed(const Shape& s, const TX* x, const float* w_router,
+                                const float* bias, int64_t bias_stride, float* logits,
+                                int32_t* topk_idx, float* topk_w, cudaStream_t st) {
+  const int d = static_cast<int>(s.d);
+  if (s.E <= 32) {
+    const int ET = s.E <= 8 ? 8 : (s.E <= 16 ? 16 : 32);
+    const int TW = 32 / ET;
+    const int64_t warps = (s.T + TW - 1) / TW;
+    const int64_t blocks_needed = (warps + 7) / 8;
+    const int blocks = static_cast<int>(blocks_needed < 148 * 16 ? blocks_needed : 148 * 16);
+    if (ET == 8)
+      router_small_e_kernel<TX, 8><<<blocks, 256, 0, st>>>(x, w_router, bias, bias_stride, s.T, d,
+                                                           s.E, s.k, s.gating, logits, topk_idx,
+                                                           topk_w);
+    else if (ET == 16)
+      router_small_e_kernel<TX, 16><<<blocks, 256, 0, st>>>(x, w_router, bias, bias_stride, s.T,
+                                                            d, s.E, s.k, s.gating, logits,
+                                                            topk_idx, topk_w);
+    else
+      router_small_e_kernel<TX, 32><<<blocks, 256, 0, st>>>(x, w_router, bias, bias_stride, s.T,
+                                                            d, s.E, s.k, s.gating, logits,
+                                                            topk_idx, topk_w);
+    return cudaGetLastError();
+  }
+  dim3 grid((s.E + RT_N - 1) / RT_N, static_cast<unsigned>((s.T + RT_M - 1) / RT_M));
+  router_gemm_kernel<TX><<<grid, 256, 0, st>>>(x, w_router, bias, bias_stride, s.T, d, s.E,
+                                               logits);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const int64_t blocks_needed = (s.T + 7) / 8;
+  const int blocks = static_cast<int>(blocks_needed < 148 * 16 ? blocks_needed : 148 * 16);
+  topk_from_logits_kernel<<<blocks, 256, 0, st>>>(logits, s.T, s.E, s.k, s.gating, topk_idx,
+                                                  topk_w);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_router(const Shape& s, const void* x, const float* w_router,
+                          const float* bias, int64_t bias_stride, float* logits,
+                          int32_t* topk_idx, float* topk_w, cudaStream_t st) {
+  if (s.dtype == MOE_F32)
+    return launch_router_typed(s, static_cast<const float*>(x), w_router, bias, bias_stride,
+                               logits, topk_idx, topk_w, st);
+  return launch_router_typed(s, static_cast<const __nv_bfloat16*>(x), w_router, bias,
+                             bias_stride, logits, topk_idx, topk_w, st);
+}
+
+}  // namespace moe

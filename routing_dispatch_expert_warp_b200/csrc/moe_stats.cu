@@ -1,0 +1,134 @@
+// Per-layer load statistics.
+//
+// "MoE expert parallelism needs measurements before launch" (airouter.kz), "Mean expert
+// load proves almost nothing": with n_e the tokens assigned to expert e, mu = sum n_e / E;
+// every layer reports tokens_per_expert, p50, p95, max, max/mean, the share of the top 5%
+// of experts and dropped tokens.  "Capacity factor changes quality, memory and the latency
+// tail": drop rate per layer and per route (first pick, second pick, ...).
+//
+// One block: the E kept counts are sorted in shared memory (bitonic network over 256
+// slots), the drops are counted per pick rank over assign_row, and one thread evaluates
+// the fp64 formulas.  Percentiles interpolate linearly between order statistics:
+// h = (E - 1) p, v = s[floor h] + (h - floor h) (s[floor h + 1] - s[floor h]).
+#include <limits.h>
+
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+__device__ double percentile_linear(const int32_t* s, int n, double p) {
+  const double h = __dmul_rn(static_cast<double>(n - 1), p);
+  const double fl = floor(h);
+  const int lo = static_cast<int>(fl);
+  const int hi = lo + 1 < n ? lo + 1 : n - 1;
+  const double diff = __dadd_rn(static_cast<double>(s[hi]), -static_cast<double>(s[lo]));
+  return __dadd_rn(static_cast<double>(s[lo]), __dmul_rn(__dadd_rn(h, -fl), diff));
+}
+
+__global__ void __launch_bounds__(MOE_MAX_EXPERTS) stats_kernel(
+    const int32_t* __restrict__ routed, const int32_t* __restrict__ kept,
+    const int32_t* __restrict__ assign_row, int64_t T, int k, int E, int64_t C,
+    moe_load_stats_t* __restrict__ out) {
+  __shared__ int32_t sorted[MOE_MAX_EXPERTS];
+  __shared__ unsigned long long sum_kept, sum_routed;
+  __shared__ int max_routed;
+  __shared__ unsigned long long drop_rank[MOE_MAX_TOPK];
+  __shared__ unsigned long long tok_drop, tok_full;
+  const int tid = threadIdx.x;
+  sorted[tid] = tid < E ? kept[tid] : INT_MAX;
+  if (tid == 0) {
+    sum_kept = 0;
+    sum_routed = 0;
+    max_routed = 0;
+    tok_drop = 0;
+    tok_full = 0;
+  }
+  if (tid < MOE_MAX_TOPK) drop_rank[tid] = 0;
+  __syncthreads();
+  if (tid < E) {
+    atomicAdd(&sum_kept, static_cast<unsigned long long>(kept[tid]));
+    atomicAdd(&sum_routed, static_cast<unsigned long long>(routed[tid]));
+    atomicMax(&max_routed, routed[tid]);
+  }
+  // bitonic sort, ascending
+  for (int size = 2; size <= MOE_MAX_EXPERTS; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const int partner = tid ^ stride;
+      if (partner > tid) {
+        const bool asc = (tid & size) == 0;
+        const int32_t a = sorted[tid], b = sorted[partner];
+        if ((a > b) == asc) {
+          sorted[tid] = b;
+          sorted[partner] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // drops per pick rank and per token
+  unsigned long long rank_local[MOE_MAX_TOPK];
+#pragma unroll
+  for (int j = 0; j < MOE_MAX_TOPK; ++j) rank_local[j] = 0;
+  unsigned long long td = 0, tf = 0;
+  for (int64_t t = tid; t < T; t += blockDim.x) {
+    int nd = 0;
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+      if (j < k && assign_row[t * k + j] < 0) {
+        ++rank_local[j];
+        ++nd;
+      }
+    }
+    td += nd > 0;
+    tf += nd == k;
+  }
+#pragma unroll
+  for (int j = 0; j < MOE_MAX_TOPK; ++j)
+    if (j < k && rank_local[j]) atomicAdd(&drop_rank[j], rank_local[j]);
+  if (td) atomicAdd(&tok_drop, td);
+  if (tf) atomicAdd(&tok_full, tf);
+  __syncthreads();
+
+  if (tid == 0) {
+    moe_load_stats_t st;
+    st.E = E;
+    st.k = k;
+    st.active_tokens = T;
+    st.capacity = C;
+    st.routed_total = static_cast<int64_t>(sum_routed);
+    st.kept_total = static_cast<int64_t>(sum_kept);
+    st.dropped = T * k - static_cast<int64_t>(sum_kept);
+    st.tokens_with_drop = static_cast<int64_t>(tok_drop);
+    st.tokens_fully_dropped = static_cast<int64_t>(tok_full);
+    st.p50 = percentile_linear(sorted, E, 0.50);
+    st.p95 = percentile_linear(sorted, E, 0.95);
+    st.p99 = percentile_linear(sorted, E, 0.99);
+    st.max = static_cast<double>(sorted[E - 1]);
+    const double mean = static_cast<double>(sum_kept) / static_cast<double>(E);
+    st.mean = mean;
+    st.max_to_mean = mean > 0.0 ? st.max / mean : 0.0;
+    st.routed_max = static_cast<double>(max_routed);
+    const double rmean = static_cast<double>(sum_routed) / static_cast<double>(E);
+    st.routed_max_to_mean = rmean > 0.0 ? st.routed_max / rmean : 0.0;
+    const int n_top = (E + 19) / 20;  // ceil(0.05 E)
+    long long top = 0;
+    for (int i = 0; i < n_top; ++i) top += sorted[E - 1 - i];
+    st.top5pct_share =
+        sum_kept > 0 ? static_cast<double>(top) / static_cast<double>(sum_kept) : 0.0;
+    for (int j = 0; j < MOE_MAX_TOPK; ++j)
+      st.dropped_by_rank[j] = j < k ? static_cast<int64_t>(drop_rank[j]) : 0;
+    *out = st;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_stats(const Shape& s, const int32_t* routed, const int32_t* kept,
+                         const int32_t* assign_row, moe_load_stats_t* out, cudaStream_t st) {
+  stats_kernel<<<1, MOE_MAX_EXPERTS, 0, st>>>(routed, kept, assign_row, s.T, s.k, s.E, s.C,
+                                              out);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

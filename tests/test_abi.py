@@ -1,0 +1,146 @@
+"""The C-ABI library without a GPU: it builds, loads, exports every declared entry point,
+its structs match the ctypes mirror, and its host-side checks and sizes are right.
+No kernel is launched here."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as O
+from routing_dispatch_expert_warp_b200 import _abi, build as B
+import routing_dispatch_expert_warp_b200 as M
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return _abi.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 15
+    assert set(names) == set(_abi.PROTOTYPES), "ctypes prototypes and header disagree"
+    nm = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True,
+                        text=True, check=True).stdout
+    exported = set(re.findall(r"\b(moe_[a-z0-9_]+)$", nm, flags=re.M))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert getattr(lib, n) is not None
+    assert lib.moe_abi_version() == 1
+
+
+def test_struct_layout_matches_header(tmp_path):
+    prog = tmp_path / "layout.c"
+    prog.write_text("""
+#include <stdio.h>
+#include <stddef.h>
+#include "moe.h"
+int main(void) {
+  printf("%zu %zu %zu %zu\\n", sizeof(moe_config_t), sizeof(moe_load_stats_t),
+         sizeof(moe_layer_inputs_t), sizeof(moe_layer_buffers_t));
+  printf("%zu %zu %zu\\n", offsetof(moe_config_t, capacity_factor),
+         offsetof(moe_load_stats_t, p50), offsetof(moe_load_stats_t, dropped_by_rank));
+  printf("%zu %zu\\n", offsetof(moe_layer_inputs_t, bias_row_stride),
+         offsetof(moe_layer_buffers_t, stats));
+  return 0;
+}
+""")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(prog), "-o",
+                    str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    got = [int(v) for v in out]
+    want = [ctypes.sizeof(_abi.MoeConfig), ctypes.sizeof(_abi.MoeLoadStats),
+            ctypes.sizeof(_abi.MoeLayerInputs), ctypes.sizeof(_abi.MoeLayerBuffers),
+            _abi.MoeConfig.capacity_factor.offset, _abi.MoeLoadStats.p50.offset,
+            _abi.MoeLoadStats.dropped_by_rank.offset, _abi.MoeLayerInputs.bias_row_stride.offset,
+            _abi.MoeLayerBuffers.stats.offset]
+    assert got == want
+
+
+@pytest.mark.parametrize("T,E,k,cf", [(64, 8, 2, 1.25), (16384, 256, 8, 1.0), (8192, 8, 2, 1.25),
+                                      (10, 3, 1, 1.0), (10, 3, 1, 0.01), (4096, 8, 2, 0.0),
+                                      (37, 5, 2, 0.7)])
+def test_capacity_matches_oracle(lib, T, E, k, cf):
+    cfg = M.make_config(T, 64, 64, E, k, capacity_factor=cf)
+    C = O.capacity(float(np.float32(cf)), T, k, E)
+    assert M.capacity(cfg) == (-1 if C is None else C)
+    A = T * k
+    assert M.max_rows(cfg) == (A if C is None else min(A, E * C))
+    if C is not None:
+        cfg.layout = M.PADDED
+        assert M.max_rows(cfg) == E * C
+
+
+def test_workspace_size_and_bad_configs(lib):
+    cfg = M.make_config(4096, 4096, 14336, 8, 2)
+    n = M.workspace_size(cfg)
+    assert n >= 256 + 16 * 8 * 4 + 4096 * 8 * 4
+    bad = [dict(E=0), dict(E=257), dict(k=0), dict(k=9), dict(T=0), dict(d_model=12),
+           dict(gating=3), dict(layout=2), dict(dtype=7)]
+    for b in bad:
+        kw = dict(T=64, d_model=128, d_ff=256, E=8, k=2)
+        kw.update({kk: v for kk, v in b.items() if kk in kw})
+        c = M.make_config(**kw)
+        for kk, v in b.items():
+            if kk not in kw:
+                setattr(c, kk, v)
+        with pytest.raises(M.MoEError) as ei:
+            M.workspace_size(c)
+        assert ei.value.status == 1, b
+    # k > E
+    with pytest.raises(M.MoEError):
+        M.workspace_size(M.make_config(64, 128, 256, 4, 5))
+    # PADDED without a capacity
+    with pytest.raises(M.MoEError):
+        M.workspace_size(M.make_config(64, 128, 256, 8, 2, layout=M.PADDED))
+
+
+def test_null_and_misaligned_pointers_rejected_on_host(lib):
+    cfg = M.make_config(64, 128, 256, 8, 2, dtype=M.F32)
+    ws_bytes = M.workspace_size(cfg)
+    L = lib
+    # NULL workspace
+    st = L.moe_route(ctypes.byref(cfg), 16, 16, None, 0, None, 16, 16, None, ws_bytes, None)
+    assert st == 1 and b"workspace" in L.moe_last_error()
+    # workspace too small (aligned fake address; nothing is dereferenced on the host)
+    st = L.moe_route(ctypes.byref(cfg), 16, 16, None, 0, None, 16, 16, 256, 16, None)
+    assert st == 3
+    # misaligned x
+    st = L.moe_route(ctypes.byref(cfg), 17, 16, None, 0, None, 16, 16, 256, ws_bytes, None)
+    assert st == 1 and b"aligned" in L.moe_last_error()
+    # NULL outputs
+    st = L.moe_dispatch(ctypes.byref(cfg), 16, 16, None, 16, 16, 16, 16, 16, 256, ws_bytes, None)
+    assert st == 1
+    st = L.moe_combine(ctypes.byref(cfg), 16, None, 16, 16, None)
+    assert st == 1
+    st = L.moe_load_stats(ctypes.byref(cfg), 16, 16, 16, None, None, None)
+    assert st == 1
+    # bf16 FFN needs multiples of 64
+    cfg2 = M.make_config(64, 96, 256, 8, 2, dtype=M.BF16)
+    st = L.moe_expert_ffn(ctypes.byref(cfg2), 16, 16, 16, 16, 16, 16, 16, 16, 256,
+                          M.workspace_size(cfg2), None)
+    assert st == 2
+    assert L.moe_status_string(5) == b"MOE_ERR_TIMEOUT"
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_abi, "_lib", None)
+    monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        _abi.lib()

@@ -1,0 +1,41 @@
+"""The five named workloads at their full sizes, in the launch configuration the benchmark
+times.  Routing, counts, permutation indices, drops and statistics are compared in full;
+logits, permuted rows, FFN rows and combined tokens on samples the oracle computes one by
+one (the largest, the smallest and random buckets, first and last rows included)."""
+import numpy as np
+import pytest
+import torch
+
+from routing_dispatch_expert_warp_b200 import workload as W
+
+from moe_parity import (GpuRun, check_combine, check_ffn_rows, check_permute, check_routing,
+                        check_stats)
+
+pytestmark = pytest.mark.gpu
+
+FULL = [W.TINY_FP32, W.MIXTRAL_8X7B, W.DSV3_DECODE, W.DSV3_PREFILL_ZIPF, W.MIXTRAL_8X22B_MIXED]
+
+
+@pytest.mark.parametrize("shape", FULL, ids=lambda s: s.name)
+def test_full_size_sampled(shape):
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    torch.cuda.empty_cache()
+    run = GpuRun(shape)
+    st = run.all_stages()
+    rng = np.random.default_rng(shape.seed)
+    sample_rows = np.unique(np.concatenate([[0, shape.T - 1], rng.choice(shape.T, 64)]))
+    r = check_routing(run, sample_rows=sample_rows)
+    check_permute(run, r, sample=512)
+    kept = r["kept"]
+    nz = np.nonzero(kept)[0]
+    experts = {int(nz[np.argmax(kept[nz])]), int(nz[np.argmin(kept[nz])])}
+    experts |= set(int(e) for e in rng.choice(nz, min(2, len(nz)), replace=False))
+    check_ffn_rows(run, r, experts=sorted(experts), rows_per_expert=24)
+    toks = np.unique(np.concatenate([[0, shape.T - 1], rng.choice(shape.T, 256)]))
+    check_combine(run, r, tokens=toks)
+    check_stats(st, r)
+    if shape.capacity_factor > 0:
+        assert st["max"] <= st["capacity"]
+    del run
+    torch.cuda.empty_cache()

@@ -1,0 +1,191 @@
+"""GPU vs oracle parity through the C ABI, stage by stage and end to end.
+
+Reduced workloads keep each routing regime of the five named layers (E, k, gating, capacity
+factor, dtype, bias kind) at sizes the oracle finishes in seconds, while still spanning
+several GEMM tiles and ragged tails.  The full-size workloads are checked on sampled rows
+and tokens plus properties that hold at any size.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe_oracle as O
+import routing_dispatch_expert_warp_b200 as M
+from routing_dispatch_expert_warp_b200 import workload as W
+
+from moe_parity import (GpuRun, check_combine, check_ffn_rows, check_layer_output,
+                        check_permute, check_routing, check_stats, f64, i64, rel_fro)
+
+pytestmark = pytest.mark.gpu
+
+REDUCED = [
+    W.TINY_FP32,
+    W.reduced(W.TINY_FP32, 300, 96, 160, capacity_factor=1.0),
+    W.reduced(W.MIXTRAL_8X7B, 1000, 512, 768),
+    W.reduced(W.DSV3_DECODE, 128, 512, 256),
+    W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256),
+    W.reduced(W.MIXTRAL_8X22B_MIXED, 1200, 384, 640, n_decode_tokens=16),
+    W.reduced(W.MIXTRAL_8X7B, 700, 256, 384, layout=W.LAYOUT_PADDED, capacity_factor=1.1),
+]
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    yield
+
+
+@pytest.mark.parametrize("shape", REDUCED, ids=lambda s: s.name)
+def test_stages_match_oracle(shape):
+    run = GpuRun(shape)
+    st = run.all_stages()
+    r = check_routing(run)
+    check_permute(run, r)
+    check_ffn_rows(run, r)
+    check_combine(run, r)
+    check_stats(st, r)
+    check_layer_output(run, run.b.out, r)
+
+
+@pytest.mark.parametrize("shape", REDUCED[:3] + REDUCED[4:6], ids=lambda s: s.name)
+def test_layer_forward_matches_stages_and_is_deterministic(shape):
+    run = GpuRun(shape)
+    run.all_stages()
+    layer, out1 = run.layer_forward()
+    out1 = out1.clone()
+    assert torch.equal(out1, run.b.out), "moe_layer_forward differs from the staged calls"
+    out2 = layer(run.inp.x)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2), "two runs differ bitwise"
+    st = layer.bufs.stats_dict()
+    r = check_routing(run)
+    check_stats(st, r)
+
+
+# ------------------------------------------------------------------ edge cases
+def _edge(T, d, f, E, k, gating=W.SOFTMAX, cf=0.0, dtype=W.BF16, layout=W.LAYOUT_COMPACT,
+          seed=7):
+    return W.MoEShape(f"edge_T{T}_d{d}_f{f}_E{E}_k{k}_cf{cf}_dt{dtype}_l{layout}", T, d, f, E, k,
+                      gating, cf, dtype, layout=layout, seed=seed)
+
+
+EDGES = [
+    _edge(1, 128, 128, 8, 2),                    # a single token
+    _edge(1, 64, 64, 4, 4, cf=1.0, dtype=W.F32),  # k = E, capacity 1
+    _edge(33, 64, 128, 8, 8, gating=W.SIGMOID),  # k = E, sigmoid
+    _edge(65, 128, 192, 1, 1),                   # one expert: a dense FFN
+    _edge(200, 64, 64, 16, 1, cf=0.05),          # capacity 1 with top-1
+    _edge(129, 128, 128, 32, 3, gating=W.SIGMOID, dtype=W.F32),
+    _edge(300, 256, 128, 200, 6, cf=1.0),         # E not a power of two, > 32
+]
+
+
+@pytest.mark.parametrize("shape", EDGES, ids=lambda s: s.name)
+def test_edge_shapes(shape):
+    run = GpuRun(shape)
+    st = run.all_stages()
+    r = check_routing(run)
+    check_permute(run, r)
+    check_ffn_rows(run, r)
+    check_combine(run, r)
+    check_stats(st, r)
+    check_layer_output(run, run.b.out, r)
+
+
+def test_all_tokens_to_one_expert_with_drops():
+    shape = _edge(500, 128, 128, 8, 2, cf=1.0)
+    inp = W.make_inputs(shape, device="cuda")
+    bias = torch.zeros(8, device="cuda")
+    bias[5] = 100.0          # every token picks expert 5 first
+    inp.logit_bias = bias
+    run = GpuRun(shape.replace(bias="none"), inp)
+    st = run.all_stages()
+    r = check_routing(run)
+    C = O.capacity(1.0, 500, 2, 8)
+    assert int(r["kept"][5]) == C and st["dropped"] >= 500 - C
+    assert st["dropped_by_rank"][0] == 500 - C
+    check_ffn_rows(run, r)
+    check_combine(run, r)
+    check_stats(st, r)
+
+
+def test_capacity_exactly_hit_keeps_everything():
+    # T*k/E with cf = 1 and a uniform assignment: every expert gets exactly C
+    T, E, k = 64, 8, 1
+    shape = _edge(T, 64, 64, E, k, cf=1.0)
+    inp = W.make_inputs(shape, device="cuda")
+    bias = torch.full((T, E), -50.0, device="cuda")
+    bias[torch.arange(T), torch.arange(T) % E] = 50.0
+    inp.logit_bias = bias.contiguous()
+    run = GpuRun(shape, inp)
+    st = run.all_stages()
+    r = check_routing(run)
+    assert (r["kept"] == T // E).all() and st["dropped"] == 0
+    check_ffn_rows(run, r)
+    check_combine(run, r)
+    check_stats(st, r)
+
+
+def test_tied_logits_pick_lower_index():
+    shape = _edge(40, 64, 64, 16, 4, gating=W.SIGMOID)
+    inp = W.make_inputs(shape, device="cuda")
+    inp.x.zero_()                                      # every logit equals its bias
+    bias = torch.zeros(16, device="cuda")
+    bias[[3, 7, 9, 12]] = 1.0                          # four tied winners
+    inp.logit_bias = bias
+    run = GpuRun(shape, inp)
+    run.all_stages()
+    r = check_routing(run)
+    assert (r["idx"] == np.array([3, 7, 9, 12])).all()
+    assert np.allclose(f64(run.b.topk_w), 0.25)
+
+
+def test_empty_experts_and_padded_layout():
+    shape = _edge(256, 128, 128, 64, 2, cf=2.0, layout=W.LAYOUT_PADDED)
+    inp = W.make_inputs(shape, device="cuda")
+    bias = torch.full((64,), -30.0, device="cuda")
+    bias[:5] = 0.0                                     # only 5 of 64 experts ever picked
+    inp.logit_bias = bias
+    run = GpuRun(shape, inp)
+    st = run.all_stages()
+    r = check_routing(run)
+    assert (r["kept"][5:] == 0).all()
+    check_permute(run, r)
+    check_ffn_rows(run, r)
+    check_combine(run, r)
+    check_stats(st, r)
+
+
+# ------------------------------------------------------------------ errors without faults
+def test_bad_expert_index_is_reported_not_faulted():
+    shape = _edge(50, 64, 64, 8, 2)
+    run = GpuRun(shape)
+    run.route()
+    run.b.topk_idx[3, 1] = 999
+    run.dispatch()
+    with pytest.raises(M.MoEError) as ei:
+        M.moe_check_device_error(run.ws)
+    assert ei.value.status == 6
+    M.moe_check_device_error(run.ws)   # cleared
+    run.route()
+    run.dispatch()
+    M.moe_check_device_error(run.ws)
+
+
+def test_bounded_wait_runs_out_and_context_survives():
+    cfg = M.make_config(8, 64, 64, 4, 2)
+    ws = M.alloc_workspace(cfg)
+    M.set_wait_limit_ns(20_000_000)    # 20 ms
+    try:
+        M.moe_selftest_bounded_wait(ws)
+        with pytest.raises(M.MoEError) as ei:
+            M.moe_check_device_error(ws)
+        assert ei.value.status == 5
+    finally:
+        M.set_wait_limit_ns(0)
+    # the context still works: a normal layer forward afterwards
+    run = GpuRun(_edge(64, 128, 128, 8, 2))
+    st = run.all_stages()
+    r = check_routing(run)
+    check_stats(st, r)
