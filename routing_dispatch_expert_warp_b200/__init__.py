@@ -187,10 +187,8 @@ class LayerBuffers:
             stats=_ptr(self.stats) if with_stats else None)
 
     def stats_dict(self) -> dict:
-        hs = MoeLoadStats()
-        ctypes.memmove(ctypes.byref(hs), self.stats.cpu().numpy().ctypes.data,
-                       ctypes.sizeof(MoeLoadStats))
-        return hs.as_dict()
+        raw = bytes(self.stats.cpu().numpy().tobytes())
+        return MoeLoadStats.from_buffer_copy(raw).as_dict()
 
 
 class MoELayer:
