@@ -109,6 +109,8 @@ def algorithmic_work(shape, kept_total: int) -> dict:
 
 def run_gpu(args) -> None:
     shape = W.WORKLOADS[args.config] if args.config else DEFAULT
+    if args.tokens:
+        shape = shape.replace(name=f"{shape.name}_with_T{args.tokens}", T=args.tokens)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -347,6 +349,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--config", default=None, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override T of the workload (small profiling cases)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-sample-tokens", type=int, default=64)
     ap.add_argument("--ref-sample-tokens", type=int, default=32)
