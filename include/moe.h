@@ -210,6 +210,34 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
                           void* stream);
 
 /*
+ * moe_dispatch without a workspace.  The pages have no counterpart to this entry point; it
+ * exists for callers that cannot allocate device memory when they dispatch, for example
+ * code inside a serving engine whose memory pool owns the whole GPU, or a plugin host that
+ * hands kernels only their input and output tensors.  cudaMalloc is not an option there:
+ * it synchronises the device and may fail once the pool has taken the memory.
+ *
+ * Same arguments, results and ordering as moe_dispatch minus (ws, ws_bytes).  The scratch
+ * it needs (a status record and ceil(T/256)*E int32 block counts) lives in one fixed
+ * 1 MiB + 256 B array in device memory, which every GPU that loads this library keeps
+ * until the process exits; the call allocates nothing (no cudaMalloc, no cudaFree, no
+ * allocating library routine).  Limits and behaviour:
+ *   - ceil(T/256) * E * 4 bytes must fit in 1 MiB (e.g. T <= 262144 at E = 256); larger
+ *     sizes return MOE_ERR_UNSUPPORTED with a message, before anything is enqueued.
+ *   - The first call on each device looks up the array's device address with that device
+ *     current; make that first call before any stream capture.
+ *   - Every call shares the one array: two calls that run on the GPU at the same time
+ *     (other streams, other host threads) race and give wrong results.  Order them.
+ *   - The status record is cleared at the start of each call and kernel-side errors are
+ *     not reported: an expert index outside [0, E) is skipped like a dropped pick.  Use
+ *     moe_dispatch with a workspace to have such errors reported.
+ */
+moe_status_t moe_dispatch_static_scratch(const moe_config_t* cfg, const void* x,
+                                         const int32_t* topk_idx, int32_t* routed_counts,
+                                         int32_t* kept_counts, int32_t* expert_offsets,
+                                         int32_t* assign_row, int32_t* token_of_row,
+                                         void* x_perm, void* stream);
+
+/*
  * Expert SwiGLU FFN as a grouped GEMM over the variable-sized buckets ([EP-checks]
  * "Profile all-to-all ...": grouped GEMMs over many experts).  For each expert e and each
  * row r in [expert_offsets[e], expert_offsets[e] + kept_counts[e]):

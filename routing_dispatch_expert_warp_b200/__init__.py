@@ -21,7 +21,8 @@ COMPACT, PADDED = 0, 1
 F32, BF16 = 0, 1
 
 __all__ = ["MoEError", "make_config", "workspace_size", "capacity", "max_rows",
-           "alloc_workspace", "moe_route", "moe_dispatch", "moe_expert_ffn", "moe_combine",
+           "alloc_workspace", "moe_route", "moe_dispatch", "moe_dispatch_static_scratch",
+           "moe_expert_ffn", "moe_combine",
            "moe_load_stats", "moe_layer_forward", "moe_check_device_error",
            "moe_selftest_bounded_wait", "set_wait_limit_ns", "LayerBuffers", "MoELayer"]
 
@@ -100,6 +101,17 @@ def moe_dispatch(cfg, x, topk_idx, routed_counts, kept_counts, expert_offsets, a
                               _ptr(kept_counts), _ptr(expert_offsets), _ptr(assign_row),
                               _ptr(token_of_row), _ptr(x_perm), _ptr(ws), ws.numel(),
                               _stream(stream)))
+
+
+def moe_dispatch_static_scratch(cfg, x, topk_idx, routed_counts, kept_counts, expert_offsets,
+                                assign_row, token_of_row, x_perm, stream=None):
+    """moe_dispatch for callers that cannot allocate device memory: no workspace argument;
+    the library's fixed device scratch is used instead (see include/moe.h for the limit and
+    for why concurrent calls must be ordered)."""
+    check(_lib().moe_dispatch_static_scratch(
+        ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(routed_counts), _ptr(kept_counts),
+        _ptr(expert_offsets), _ptr(assign_row), _ptr(token_of_row), _ptr(x_perm),
+        _stream(stream)))
 
 
 def moe_expert_ffn(cfg, x_perm, expert_offsets, kept_counts, w_gate, w_up, w_down, h, y_perm,

@@ -66,6 +66,8 @@ PROTOTYPES = {
                           c_vp]),
     "moe_dispatch": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                              c_vp, c_sz, c_vp]),
+    "moe_dispatch_static_scratch": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                            c_vp, c_vp, c_vp]),
     "moe_expert_ffn": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                c_vp, c_sz, c_vp]),
     "moe_combine": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_vp]),

@@ -253,6 +253,32 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
   return MOE_OK;
 }
 
+moe_status_t moe_dispatch_static_scratch(const moe_config_t* cfg, const void* x,
+                                         const int32_t* topk_idx, int32_t* routed_counts,
+                                         int32_t* kept_counts, int32_t* expert_offsets,
+                                         int32_t* assign_row, int32_t* token_of_row,
+                                         void* x_perm, void* stream) {
+  Shape s;
+  moe_status_t st = check_config(cfg, &s);
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(x && topk_idx && routed_counts && kept_counts && expert_offsets && assign_row &&
+                  token_of_row && x_perm,
+              "moe_dispatch_static_scratch: NULL pointer");
+  MOE_REQUIRE(aligned16(x) && aligned16(x_perm),
+              "moe_dispatch_static_scratch: x and x_perm must be 16-byte aligned");
+  const size_t need = static_cast<size_t>(dispatch_blocks(s.T)) * s.E * sizeof(int32_t);
+  if (need > kStaticDispatchHistBytes)
+    return fail(MOE_ERR_UNSUPPORTED,
+                "moe_dispatch_static_scratch: ceil(T/%d)*E*4 = %zu bytes of scratch needed, the "
+                "fixed scratch holds %zu (use moe_dispatch with a workspace)",
+                kDispatchBlockTokens, need, kStaticDispatchHistBytes);
+  cudaError_t err = dispatch_static_scratch(s, x, topk_idx, routed_counts, kept_counts,
+                                            expert_offsets, assign_row, token_of_row, x_perm,
+                                            g_wait_ns.load(), static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_dispatch_static_scratch");
+  return MOE_OK;
+}
+
 moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
                             const int32_t* expert_offsets, const int32_t* kept_counts,
                             const void* w_gate, const void* w_up, const void* w_down, void* h,

@@ -22,6 +22,8 @@
 //              popcount(mask & lanes below me).  Writes assign_row and token_of_row.
 //   4. permute: token-major row copy with bulk (TMA) copies: each row of x is read from HBM
 //              once into shared memory and written to each of its kept rows of x_perm.
+#include <mutex>
+
 #include "moe_internal.h"
 
 namespace moe {
@@ -262,6 +264,49 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
       static_cast<const uint8_t*>(x), assign_row, s.T, s.k, row_bytes,
       static_cast<uint32_t>(seg), segs, static_cast<uint8_t*>(x_perm), status, wait_ns);
   return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ allocation-free variant
+// Scratch for moe_dispatch_static_scratch(): a status record followed by the per-block
+// expert histogram, in a fixed array that every GPU loading this library keeps until the
+// process exits.  All calls share it, so calls that run on the GPU at the same time race.
+constexpr size_t kStaticStatusBytes = 256;
+static __device__ __align__(256) uint8_t g_dispatch_scratch[kStaticStatusBytes +
+                                                            kStaticDispatchHistBytes];
+
+namespace {
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {nullptr};
+}  // namespace
+
+cudaError_t dispatch_static_scratch(const Shape& s, const void* x, const int32_t* topk_idx,
+                                    int32_t* routed, int32_t* kept, int32_t* offsets,
+                                    int32_t* assign_row, int32_t* token_of_row, void* x_perm,
+                                    uint64_t wait_ns, cudaStream_t st) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  void* base = nullptr;
+  {
+    // Set-up, once per device with that device current: the host-side name of the array
+    // is not a device address, so ask the runtime for the device address and keep it.
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      err = cudaGetSymbolAddress(&p, g_dispatch_scratch);
+      if (err != cudaSuccess) return err;
+      g_scratch_ptr[dev] = p;
+    }
+    base = g_scratch_ptr[dev];
+  }
+  DevStatus* status = static_cast<DevStatus*>(base);
+  int32_t* hist = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(base) + kStaticStatusBytes);
+  // the status record must start at zero; the histogram is fully rewritten by every call
+  err = cudaMemsetAsync(status, 0, sizeof(DevStatus), st);
+  if (err != cudaSuccess) return err;
+  return launch_dispatch(s, x, topk_idx, routed, kept, offsets, assign_row, token_of_row,
+                         x_perm, hist, status, wait_ns, st);
 }
 
 }  // namespace moe
