@@ -107,6 +107,20 @@ def algorithmic_work(shape, kept_total: int) -> dict:
     }
 
 
+def rank_shape(shape, rank: int):
+    """Replicas draw different token batches (and weights) per rank: seed + 1000 * rank."""
+    return shape.replace(seed=shape.seed + 1000 * rank) if rank else shape
+
+
+def max_over_ranks(values, dist, device) -> list:
+    """Element-wise max of per-rank timings (the slowest rank sets the job's time)."""
+    if dist is None:
+        return list(values)
+    t = torch.tensor(list(values), device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def run_gpu(args) -> None:
     shape = W.WORKLOADS[args.config] if args.config else DEFAULT
     if args.tokens:
@@ -126,8 +140,7 @@ def run_gpu(args) -> None:
                                 device_id=dev)
 
     # every rank holds a full replica; ranks draw different token batches
-    shape_r = shape.replace(seed=shape.seed + 1000 * rank) if rank else shape
-    inp = W.make_inputs(shape_r, device=dev)
+    inp = W.make_inputs(rank_shape(shape, rank), device=dev)
     cfg = M.config_from_shape(shape)
     ws = M.alloc_workspace(cfg, dev)
     b = M.LayerBuffers.allocate(cfg, dev)
@@ -180,11 +193,7 @@ def run_gpu(args) -> None:
         for j, n in enumerate(names):
             per_stage[n].append(ev[j].elapsed_time(ev[j + 1]))
         step_ms.append(ev[0].elapsed_time(ev[5]))
-    total_ms = sum(step_ms)
-    if dist:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks([sum(step_ms)], dist, dev)[0]
     ms_per_step = total_ms / args.steps
     stats = b.stats_dict()
     kept_total = stats["kept_total"]
@@ -214,11 +223,7 @@ def run_gpu(args) -> None:
         e1.record(stream)
         e1.synchronize()
         e2e_ms.append(e0.elapsed_time(e1))
-    e2e_total = sum(e2e_ms)
-    if dist:
-        t = torch.tensor([e2e_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
+    e2e_total = max_over_ranks([sum(e2e_ms)], dist, dev)[0]
     M.moe_check_device_error(layer.ws)
 
     if rank == 0:

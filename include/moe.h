@@ -187,6 +187,10 @@ int64_t moe_max_rows(const moe_config_t* cfg);
  *   topk_idx[t, :] = the k largest z[t, :], best first; equal z -> lower expert index
  *   topk_w[t, :]   = gate weights renormalised over the k picks (cfg->gating)
  * logits may be NULL (then z lives in the workspace).  Needs the workspace.
+ * Precision of z: fp32 FMA on CUDA cores, except for bf16 layers with E > 32, T >= 512 and
+ * d_model a multiple of 64, where z = x . hi + x . lo runs on the tensor cores with W_r
+ * split into two bf16 terms (|z - exact| <= 1e-4 (1 + |z|)).  The top-k is always taken on
+ * the fp32 z that is returned, so picks, weights and everything downstream follow z.
  */
 moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_router,
                        const float* logit_bias, int64_t bias_row_stride, float* logits,

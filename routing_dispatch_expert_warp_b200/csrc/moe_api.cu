@@ -120,6 +120,14 @@ WsLayout workspace_layout(const Shape& s) {
   l.logits = off;
   l.logits_bytes = round_up(static_cast<size_t>(s.T) * s.E * sizeof(float));
   off += l.logits_bytes;
+  const int splits = router_splits(s);
+  l.partials = off;
+  l.partials_bytes =
+      splits > 1 ? round_up(static_cast<size_t>(splits) * s.T * s.E * sizeof(float)) : 0;
+  off += l.partials_bytes;
+  l.router_tc = off;
+  l.router_tc_bytes = round_up(router_tc_workspace_bytes(s));
+  off += l.router_tc_bytes;
   l.total = off;
   return l;
 }
@@ -225,8 +233,21 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
               "moe_route: bias_row_stride must be 0 or >= E");
   float* z = logits;
   if (z == nullptr && s.E > 32) z = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + lay.logits);
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  if (router_uses_tensor_cores(s)) {
+    const char* why = "";
+    cudaError_t err = launch_router_tc(s, x, w_router, logit_bias, bias_row_stride, z, topk_idx,
+                                       topk_w, static_cast<uint8_t*>(ws) + lay.router_tc,
+                                       ws_status(ws, lay), g_wait_ns.load(), strm, &why);
+    if (err != cudaSuccess) {
+      if (why[0]) return fail(MOE_ERR_CUDA, "moe_route: %s", why);
+      return cuda_fail(err, "moe_route (tensor cores) launch");
+    }
+    return MOE_OK;
+  }
+  float* partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + lay.partials);
   cudaError_t err = launch_router(s, x, w_router, logit_bias, bias_row_stride, z, topk_idx, topk_w,
-                                  static_cast<cudaStream_t>(stream));
+                                  partials, strm);
   if (err != cudaSuccess) return cuda_fail(err, "moe_route launch");
   return MOE_OK;
 }

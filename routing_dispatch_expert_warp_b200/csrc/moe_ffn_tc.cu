@@ -14,6 +14,9 @@
 //     K step produces the gate tile in TMEM columns [0,128) and the up tile in [128,256);
 //     the epilogue writes h = silu(gate) * up as bf16.
 //   down: a 128 x 256 tile of y_perm = h . W_d[e]^T with a plain bf16 epilogue.
+//   router (E > 32, bf16 x): z = x . W_r with W_r split into two bf16 terms hi + lo; the
+//     B tile stacks 128 experts of hi on the same 128 experts of lo, and the epilogue writes
+//     z = (x . hi) + (x . lo) + bias in fp32.
 //
 // Block = 6 warps, one block per SM, persistent over tiles:
 //   warp 0 (one lane)   TMA producer: A = 128 x 64 bf16 slice of x_perm/h rows, B = 256 x 64
@@ -48,20 +51,27 @@ constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 constexpr int DYN_SMEM = STAGES * STAGE_BYTES + 1024;  // + alignment slack
 
+enum TcMode { MODE_DOWN = 0, MODE_SWIGLU = 1, MODE_ROUTER = 2 };
+
 struct TcParams {
   const int32_t* seg_start;  // [E] first row of each bucket
   const int32_t* seg_count;  // [E] rows of each bucket
   int E;
   int K;         // reduction length (multiple of 64)
   int n_blocks;  // output column blocks
-  int N_out;     // output columns (multiple of 64)
+  int N_out;     // output columns
+  int mb_outer;  // 1: tiles of one m-block consecutive (all n-blocks share the A rows)
   __nv_bfloat16* out;
+  float* out_f32;            // MODE_ROUTER output
+  const float* bias;         // MODE_ROUTER logit bias (or nullptr)
+  int64_t bias_stride;
   DevStatus* status;
   uint64_t wait_ns;
 };
 
 __device__ __forceinline__ void decode_tile(int tile, const int* tile_base, const int* mblocks,
-                                            int E, int& e, int& mb, int& nb) {
+                                            int E, int n_blocks, int mb_outer, int& e, int& mb,
+                                            int& nb) {
   int lo = 0, hi = E - 1;  // largest e with tile_base[e] <= tile
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -70,19 +80,25 @@ __device__ __forceinline__ void decode_tile(int tile, const int* tile_base, cons
   }
   e = lo;
   const int local = tile - tile_base[e];
-  const int mbs = mblocks[e];
-  nb = local / mbs;
-  mb = local - nb * mbs;
+  if (mb_outer) {
+    mb = local / n_blocks;
+    nb = local - mb * n_blocks;
+  } else {
+    const int mbs = mblocks[e];
+    nb = local / mbs;
+    mb = local - nb * mbs;
+  }
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) {
   return g / (1.0f + __expf(-g)) * u;
 }
 
-template <bool GATED>
+template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
     const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
     const __grid_constant__ CUtensorMap tm_b1, const TcParams p) {
+  constexpr bool GATED = MODE != MODE_DOWN;  // B tile = two stacked 128-row halves
   constexpr int BN_OUT = GATED ? 128 : 256;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
@@ -155,7 +171,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
       int e, mb, nb;
-      decode_tile(tile, tile_base, mblocks, p.E, e, mb, nb);
+      decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, p.mb_outer, e, mb, nb);
       const int row0 = p.seg_start[e] + mb * BM;
       for (int kb = 0; kb < KB; ++kb) {
         if (!mbar_wait(&empty_bar[s], ph ^ 1u, p.wait_ns, &abort_s)) {
@@ -241,7 +257,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
     uint32_t aph = 0;
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       int e, mb, nb;
-      decode_tile(tile, tile_base, mblocks, p.E, e, mb, nb);
+      decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, p.mb_outer, e, mb, nb);
       const int row0 = p.seg_start[e] + mb * BM;
       const int valid = p.seg_count[e] - mb * BM;
       int ok = 1;
@@ -259,7 +275,31 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
       __nv_bfloat16* orow =
           p.out + static_cast<int64_t>(row0 + r) * p.N_out + static_cast<int64_t>(nb) * BN_OUT;
       const int cols_left = p.N_out - nb * BN_OUT;
-      if (GATED) {
+      if (MODE == MODE_ROUTER) {
+        const int64_t grow = static_cast<int64_t>(row0 + r);
+        float* zrow = p.out_f32 + grow * p.N_out + static_cast<int64_t>(nb) * BN_OUT;
+        const float* brow =
+            p.bias != nullptr ? p.bias + grow * p.bias_stride + static_cast<int64_t>(nb) * BN_OUT
+                              : nullptr;
+#pragma unroll 1
+        for (int c = 0; c < BN_OUT / 32; ++c) {
+          uint32_t hi[32], lo[32];
+          tmem_ld32(taddr + c * 32, hi);
+          tmem_ld32(taddr + 128 + c * 32, lo);
+          tmem_ld_wait();
+          if (row_ok) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const int col = c * 32 + i;
+              if (col < cols_left) {
+                float z = __uint_as_float(hi[i]) + __uint_as_float(lo[i]);
+                if (brow != nullptr) z += brow[col];
+                zrow[col] = z;
+              }
+            }
+          }
+        }
+      } else if (GATED) {
 #pragma unroll 1
         for (int c = 0; c < BN_OUT / 32; ++c) {
           uint32_t g[32], u[32];
@@ -309,6 +349,37 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// W_r [d, E] fp32 -> hi, lo [E, d] bf16 with hi = bf16(W), lo = bf16(W - hi), so that
+// x . W = x . hi + x . lo up to the rounding of lo (a relative 2^-17 of each weight).
+// 32 x 32 tiles transposed through shared memory.  Block (0, 0) also writes the one-bucket
+// table {start 0, count T} the grouped GEMM reads.
+__global__ void __launch_bounds__(256) split_router_weight_kernel(
+    const float* __restrict__ w, int d, int E, __nv_bfloat16* __restrict__ hi,
+    __nv_bfloat16* __restrict__ lo, int32_t* __restrict__ seg, int32_t T) {
+  __shared__ float tile[32][33];
+  const int e0 = blockIdx.x * 32, i0 = blockIdx.y * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int r = ty; r < 32; r += 8) {
+    const int i = i0 + r, e = e0 + tx;
+    tile[r][tx] = (i < d && e < E) ? w[static_cast<int64_t>(i) * E + e] : 0.f;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int e = e0 + r, i = i0 + tx;
+    if (e < E && i < d) {
+      const float v = tile[tx][r];
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      const __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
+      hi[static_cast<int64_t>(e) * d + i] = h;
+      lo[static_cast<int64_t>(e) * d + i] = l;
+    }
+  }
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    seg[0] = 0;
+    seg[1] = T;
   }
 }
 
@@ -379,17 +450,17 @@ cudaError_t launch_ffn_tc(const Shape& s, const void* x_perm, const int32_t* off
     return cudaErrorInvalidValue;
   }
   cudaError_t err;
-  err = cudaFuncSetAttribute(grouped_gemm_tc_kernel<true>,
+  err = cudaFuncSetAttribute(grouped_gemm_tc_kernel<MODE_SWIGLU>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, DYN_SMEM);
   if (err != cudaSuccess) return err;
-  err = cudaFuncSetAttribute(grouped_gemm_tc_kernel<false>,
+  err = cudaFuncSetAttribute(grouped_gemm_tc_kernel<MODE_DOWN>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, DYN_SMEM);
   if (err != cudaSuccess) return err;
 
   const int64_t row_blocks_bound = (s.max_rows + BM - 1) / BM + s.E;
   const int sms = sm_count();
 
-  TcParams p1;
+  TcParams p1 = {};
   p1.seg_start = offsets;
   p1.seg_count = kept;
   p1.E = s.E;
@@ -401,7 +472,7 @@ cudaError_t launch_ffn_tc(const Shape& s, const void* x_perm, const int32_t* off
   p1.wait_ns = wait_ns;
   int64_t g1 = row_blocks_bound * p1.n_blocks;
   if (g1 > sms) g1 = sms;
-  grouped_gemm_tc_kernel<true><<<static_cast<unsigned>(g1), THREADS, DYN_SMEM, st>>>(ta1, tg, tu,
+  grouped_gemm_tc_kernel<MODE_SWIGLU><<<static_cast<unsigned>(g1), THREADS, DYN_SMEM, st>>>(ta1, tg, tu,
                                                                                     p1);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
 
@@ -412,9 +483,65 @@ cudaError_t launch_ffn_tc(const Shape& s, const void* x_perm, const int32_t* off
   p2.out = static_cast<__nv_bfloat16*>(y);
   int64_t g2 = row_blocks_bound * p2.n_blocks;
   if (g2 > sms) g2 = sms;
-  grouped_gemm_tc_kernel<false><<<static_cast<unsigned>(g2), THREADS, DYN_SMEM, st>>>(ta2, td, td,
+  grouped_gemm_tc_kernel<MODE_DOWN><<<static_cast<unsigned>(g2), THREADS, DYN_SMEM, st>>>(ta2, td, td,
                                                                                      p2);
   return cudaGetLastError();
+}
+
+bool router_uses_tensor_cores(const Shape& s) {
+  return s.dtype == MOE_BF16 && s.E > 32 && s.d % 64 == 0 && s.T >= 512;
+}
+
+size_t router_tc_workspace_bytes(const Shape& s) {
+  if (!router_uses_tensor_cores(s)) return 0;
+  return 256 + 2 * static_cast<size_t>(s.E) * s.d * sizeof(__nv_bfloat16);
+}
+
+cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_router,
+                             const float* bias, int64_t bias_stride, float* logits,
+                             int32_t* topk_idx, float* topk_w, void* split_ws,
+                             DevStatus* status, uint64_t wait_ns, cudaStream_t st,
+                             const char** why) {
+  if (encode_fn() == nullptr) {
+    *why = "cuTensorMapEncodeTiled is not available from the driver";
+    return cudaErrorNotSupported;
+  }
+  int32_t* seg = static_cast<int32_t*>(split_ws);
+  __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(split_ws) + 256);
+  __nv_bfloat16* lo = hi + static_cast<size_t>(s.E) * s.d;
+  dim3 sgrid((s.E + 31) / 32, static_cast<unsigned>((s.d + 31) / 32));
+  split_router_weight_kernel<<<sgrid, 256, 0, st>>>(w_router, static_cast<int>(s.d), s.E, hi, lo,
+                                                    seg, static_cast<int32_t>(s.T));
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  CUtensorMap ta, th, tl;
+  if (!make_map_rows(&ta, x, s.T, s.d) || !make_map_weights(&th, hi, 1, s.E, s.d, 128) ||
+      !make_map_weights(&tl, lo, 1, s.E, s.d, 128)) {
+    *why = "tensor map encoding failed for the router";
+    return cudaErrorInvalidValue;
+  }
+  err = cudaFuncSetAttribute(grouped_gemm_tc_kernel<MODE_ROUTER>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, DYN_SMEM);
+  if (err != cudaSuccess) return err;
+  TcParams p = {};
+  p.seg_start = seg;
+  p.seg_count = seg + 1;
+  p.E = 1;
+  p.K = static_cast<int>(s.d);
+  p.n_blocks = (s.E + 127) / 128;
+  p.N_out = s.E;
+  p.mb_outer = 1;
+  p.out_f32 = logits;
+  p.bias = bias;
+  p.bias_stride = bias_stride;
+  p.status = status;
+  p.wait_ns = wait_ns;
+  int64_t g = ((s.T + BM - 1) / BM) * p.n_blocks;
+  if (g > sm_count()) g = sm_count();
+  grouped_gemm_tc_kernel<MODE_ROUTER><<<static_cast<unsigned>(g), THREADS, DYN_SMEM, st>>>(
+      ta, th, tl, p);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  return launch_topk_from_logits(s, logits, topk_idx, topk_w, st);
 }
 
 }  // namespace moe

@@ -30,6 +30,10 @@ struct WsLayout {
   size_t hist_bytes;
   size_t logits;        // [T, E] fp32 logits when the caller passes none
   size_t logits_bytes;
+  size_t partials;      // split-K router partial sums
+  size_t partials_bytes;
+  size_t router_tc;     // bf16 split of W_r for the tensor-core router
+  size_t router_tc_bytes;
   size_t total;
 };
 
@@ -39,9 +43,24 @@ inline int64_t dispatch_blocks(int64_t T) {
 WsLayout workspace_layout(const Shape& s);
 
 // Kernel launchers (return the CUDA error of the launch).
+// Router on CUDA cores: fused top-k for E <= 32; for E > 32 a tiled fp32 GEMM, split along
+// d into router_splits(s) pieces (partials: that many [T, E] fp32 buffers) when the token
+// count alone cannot fill the GPU.
+constexpr int kMaxRouterSplits = 64;
+int router_splits(const Shape& s);
 cudaError_t launch_router(const Shape& s, const void* x, const float* w_router,
                           const float* bias, int64_t bias_stride, float* logits,
-                          int32_t* topk_idx, float* topk_w, cudaStream_t st);
+                          int32_t* topk_idx, float* topk_w, float* partials, cudaStream_t st);
+// Router on tensor cores (bf16 layers, E > 32): W_r split into two bf16 terms.
+bool router_uses_tensor_cores(const Shape& s);
+cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_router,
+                             const float* bias, int64_t bias_stride, float* logits,
+                             int32_t* topk_idx, float* topk_w, void* split_ws,
+                             DevStatus* status, uint64_t wait_ns, cudaStream_t st,
+                             const char** why);
+size_t router_tc_workspace_bytes(const Shape& s);
+cudaError_t launch_topk_from_logits(const Shape& s, const float* logits, int32_t* topk_idx,
+                                    float* topk_w, cudaStream_t st);
 cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_idx,
                             int32_t* routed, int32_t* kept, int32_t* offsets,
                             int32_t* assign_row, int32_t* token_of_row, void* x_perm,

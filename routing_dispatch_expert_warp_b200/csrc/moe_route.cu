@@ -69,59 +69,92 @@ __device__ __forceinline__ void gate_weights(const float* zsel, int k, int gatin
   for (int j = 0; j < k; ++j) w[j] *= inv;
 }
 
+// One block scores TW = 32 / ET tokens.  The d axis is cut into 256-element chunks dealt
+// round-robin to the 8 warps.  Inside a chunk, lane l owns the element pairs
+// (64 q + 2 l, 64 q + 2 l + 1), q = 0..3: the warp's loads of x are 128 contiguous bytes per
+// token and q, and its loads of the matching W_r rows are contiguous too (lane l reads rows
+// 2l and 2l+1), so both streams are coalesced.  Each warp folds its 32 partial values (TW
+// tokens x ET experts) with a butterfly transpose-reduction, the 8 warp partials are added
+// in warp order through shared memory, and warp 0 finishes: bias, logits, top-k and gate
+// weights.
+template <typename TX>
+__device__ __forceinline__ void load_pair(const TX* p, float& a, float& b);
+template <>
+__device__ __forceinline__ void load_pair<float>(const float* p, float& a, float& b) {
+  const float2 v = __ldg(reinterpret_cast<const float2*>(p));
+  a = v.x;
+  b = v.y;
+}
+template <>
+__device__ __forceinline__ void load_pair<__nv_bfloat16>(const __nv_bfloat16* p, float& a,
+                                                         float& b) {
+  const uint32_t v = __ldg(reinterpret_cast<const unsigned int*>(p));
+  a = bf16_lo(v);
+  b = bf16_hi(v);
+}
+
 template <typename TX, int ET>
 __global__ void __launch_bounds__(256) router_small_e_kernel(
     const TX* __restrict__ x, const float* __restrict__ w_router, const float* __restrict__ bias,
     int64_t bias_stride, int64_t T, int d, int E, int k, int gating, float* __restrict__ logits,
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
-  constexpr int TW = 32 / ET;  // tokens per warp
+  constexpr int TW = 32 / ET;  // tokens per block
+  constexpr int NW = 8;        // warps per block
+  __shared__ float part[NW][32];
   const int lane = threadIdx.x & 31;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int warp = threadIdx.x >> 5;
   const bool e_vec4 = (E % 4) == 0;
+  const int nchunks = (d + 255) / 256;
 
-  for (int64_t t0 = warp * TW; t0 < T; t0 += nwarps * TW) {
+  for (int64_t t0 = static_cast<int64_t>(blockIdx.x) * TW; t0 < T;
+       t0 += static_cast<int64_t>(gridDim.x) * TW) {
     float v[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = 0.f;
 
-    for (int i0 = lane * 8; i0 < d; i0 += 256) {
-      float xv[TW][8];
+    for (int c = warp; c < nchunks; c += NW) {
 #pragma unroll
-      for (int tw = 0; tw < TW; ++tw) {
-        if (t0 + tw < T) {
-          XLoad<TX>::load8(x + (t0 + tw) * d + i0, xv[tw]);
-        } else {
+      for (int q = 0; q < 4; ++q) {
+        const int i0 = c * 256 + q * 64 + 2 * lane;
+        if (i0 >= d) continue;
+        float xa[TW], xb[TW];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) xv[tw][q] = 0.f;
-        }
-      }
-#pragma unroll
-      for (int ii = 0; ii < 8; ++ii) {
-        float wv[ET];
-        const float* wrow = w_router + static_cast<int64_t>(i0 + ii) * E;
-        if (e_vec4) {
-#pragma unroll
-          for (int q = 0; q < ET / 4; ++q) {
-            if (4 * q < E) {
-              const float4 f = __ldg(reinterpret_cast<const float4*>(wrow) + q);
-              wv[4 * q] = f.x; wv[4 * q + 1] = f.y; wv[4 * q + 2] = f.z; wv[4 * q + 3] = f.w;
-            } else {
-              wv[4 * q] = wv[4 * q + 1] = wv[4 * q + 2] = wv[4 * q + 3] = 0.f;
-            }
+        for (int tw = 0; tw < TW; ++tw) {
+          if (t0 + tw < T) {
+            load_pair<TX>(x + (t0 + tw) * d + i0, xa[tw], xb[tw]);
+          } else {
+            xa[tw] = xb[tw] = 0.f;
           }
-        } else {
-#pragma unroll
-          for (int e = 0; e < ET; ++e) wv[e] = e < E ? __ldg(wrow + e) : 0.f;
         }
 #pragma unroll
-        for (int tw = 0; tw < TW; ++tw)
+        for (int r = 0; r < 2; ++r) {
+          float wv[ET];
+          const float* wrow = w_router + static_cast<int64_t>(i0 + r) * E;
+          if (e_vec4) {
 #pragma unroll
-          for (int e = 0; e < ET; ++e) v[tw * ET + e] = fmaf(xv[tw][ii], wv[e], v[tw * ET + e]);
+            for (int qq = 0; qq < ET / 4; ++qq) {
+              if (4 * qq < E) {
+                const float4 f = __ldg(reinterpret_cast<const float4*>(wrow) + qq);
+                wv[4 * qq] = f.x; wv[4 * qq + 1] = f.y; wv[4 * qq + 2] = f.z; wv[4 * qq + 3] = f.w;
+              } else {
+                wv[4 * qq] = wv[4 * qq + 1] = wv[4 * qq + 2] = wv[4 * qq + 3] = 0.f;
+              }
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < ET; ++e) wv[e] = e < E ? __ldg(wrow + e) : 0.f;
+          }
+#pragma unroll
+          for (int tw = 0; tw < TW; ++tw) {
+            const float xv = r == 0 ? xa[tw] : xb[tw];
+#pragma unroll
+            for (int e = 0; e < ET; ++e) v[tw * ET + e] = fmaf(xv, wv[e], v[tw * ET + e]);
+          }
+        }
       }
     }
 
-    // Butterfly transpose-reduction: afterwards lane l holds the full sum of value l.
+    // Butterfly transpose-reduction: afterwards lane l holds the warp's sum of value l.
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) {
       const bool upper = (lane & off) != 0;
@@ -132,56 +165,65 @@ __global__ void __launch_bounds__(256) router_small_e_kernel(
         v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
       }
     }
+    part[warp][lane] = v[0];
+    __syncthreads();
 
-    const int tw = lane / ET;
-    const int e = lane % ET;
-    const int64_t t = t0 + tw;
-    const bool valid = (e < E) && (t < T);
-    float z = v[0];
-    if (valid) {
-      if (bias != nullptr) z += bias[t * bias_stride + e];
-      if (logits != nullptr) logits[t * E + e] = z;
-    }
-
-    // top-k within each group of ET lanes (one token per group)
-    bool taken = false;
-    float zsel[MOE_MAX_TOPK];
-    int isel[MOE_MAX_TOPK];
-    for (int j = 0; j < k; ++j) {
-      bool bv = valid && !taken;
-      float bz = z;
-      int bi = e;
+    if (warp == 0) {
+      float z = part[0][lane];
 #pragma unroll
-      for (int off = ET / 2; off >= 1; off >>= 1) {
-        const bool ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const float oz = __shfl_xor_sync(0xffffffffu, bz, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (better(ov, oz, oi, bv, bz, bi)) {
-          bv = ov; bz = oz; bi = oi;
+      for (int w = 1; w < NW; ++w) z += part[w][lane];
+      const int tw = lane / ET;
+      const int e = lane % ET;
+      const int64_t t = t0 + tw;
+      const bool valid = (e < E) && (t < T);
+      if (valid) {
+        if (bias != nullptr) z += bias[t * bias_stride + e];
+        if (logits != nullptr) logits[t * E + e] = z;
+      }
+      // top-k within each group of ET lanes (one token per group)
+      bool taken = false;
+      float zsel[MOE_MAX_TOPK];
+      int isel[MOE_MAX_TOPK];
+      for (int j = 0; j < k; ++j) {
+        bool bv = valid && !taken;
+        float bz = z;
+        int bi = e;
+#pragma unroll
+        for (int off = ET / 2; off >= 1; off >>= 1) {
+          const bool ov = __shfl_xor_sync(0xffffffffu, bv, off);
+          const float oz = __shfl_xor_sync(0xffffffffu, bz, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+          if (better(ov, oz, oi, bv, bz, bi)) {
+            bv = ov; bz = oz; bi = oi;
+          }
+        }
+        if (bi == e) taken = true;
+        zsel[j] = bz;
+        isel[j] = bi;
+      }
+      if (e == 0 && t < T) {
+        float w[MOE_MAX_TOPK];
+        gate_weights(zsel, k, gating, w);
+        for (int j = 0; j < k; ++j) {
+          topk_idx[t * k + j] = isel[j];
+          topk_w[t * k + j] = w[j];
         }
       }
-      if (bi == e) taken = true;
-      zsel[j] = bz;
-      isel[j] = bi;
     }
-    if (e == 0 && t < T) {
-      float w[MOE_MAX_TOPK];
-      gate_weights(zsel, k, gating, w);
-      for (int j = 0; j < k; ++j) {
-        topk_idx[t * k + j] = isel[j];
-        topk_w[t * k + j] = w[j];
-      }
-    }
+    __syncthreads();
   }
 }
 
 // z = x W_r + b as a tiled fp32 GEMM: 64 tokens x 128 experts per block, K steps of 32.
 constexpr int RT_M = 64, RT_N = 128, RT_K = 32;
 
+// With gridDim.z = S > 1 the K range is split in S contiguous pieces and block z writes its
+// partial sums to z + blockIdx.z * T * E (bias left out); the top-k kernel adds the S
+// partials in order, so the result does not depend on scheduling.
 template <typename TX>
 __global__ void __launch_bounds__(256) router_gemm_kernel(
     const TX* __restrict__ x, const float* __restrict__ w_router, const float* __restrict__ bias,
-    int64_t bias_stride, int64_t T, int d, int E, float* __restrict__ z) {
+    int64_t bias_stride, int64_t T, int d, int E, int k_per_split, float* __restrict__ z) {
   __shared__ __align__(16) float xs[RT_K][RT_M];
   __shared__ __align__(16) float ws[RT_K][RT_N];
   const int tid = threadIdx.x;
@@ -194,17 +236,23 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 
-  for (int k0 = 0; k0 < d; k0 += RT_K) {
+  const int kbeg = blockIdx.z * k_per_split;
+  const int kend = kbeg + k_per_split < d ? kbeg + k_per_split : d;
+  if (gridDim.z > 1) {
+    z += static_cast<int64_t>(blockIdx.z) * T * E;
+    bias = nullptr;
+  }
+  for (int k0 = kbeg; k0 < kend; k0 += RT_K) {
     {  // x tile: 64 rows x 32 columns, 8 consecutive elements per thread, stored transposed
       const int r = tid / 4, c = (tid % 4) * 8;
       float v[8];
       const int64_t t = m0 + r;
-      if (t < T && k0 + c + 8 <= d) {
+      if (t < T && k0 + c + 8 <= kend) {
         XLoad<TX>::load8(x + t * d + k0 + c, v);
       } else {
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          v[q] = (t < T && k0 + c + q < d) ? static_cast<float>(x[t * d + k0 + c + q]) : 0.f;
+          v[q] = (t < T && k0 + c + q < kend) ? static_cast<float>(x[t * d + k0 + c + q]) : 0.f;
       }
 #pragma unroll
       for (int q = 0; q < 8; ++q) xs[c + q][r] = v[q];
@@ -215,7 +263,7 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(
         const int r = tid / 32 + 8 * q, c = (tid % 32) * 4;
         const int kk = k0 + r;
         float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (kk < d) {
+        if (kk < kend) {
           const float* src = w_router + static_cast<int64_t>(kk) * E + n0 + c;
           if (n0 + c + 4 <= E && (E % 4) == 0) {
             f = __ldg(reinterpret_cast<const float4*>(src));
@@ -260,8 +308,11 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(
 }
 
 // A warp per token: the top-k of z[t, 0..E) (E <= 256, up to 8 values per lane).
+// With nsplit > 1, z holds nsplit partial sums per logit (split-K); they are added in split
+// order with the bias and the result is written to `logits`.
 __global__ void __launch_bounds__(256) topk_from_logits_kernel(
-    const float* __restrict__ z, int64_t T, int E, int k, int gating,
+    const float* __restrict__ z, int nsplit, const float* __restrict__ bias, int64_t bias_stride,
+    float* __restrict__ logits, int64_t T, int E, int k, int gating,
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -273,7 +324,17 @@ __global__ void __launch_bounds__(256) topk_from_logits_kernel(
     for (int q = 0; q < 8; ++q) {
       const int e = lane + 32 * q;
       live[q] = e < E;
-      zv[q] = live[q] ? z[t * E + e] : 0.f;
+      if (!live[q]) {
+        zv[q] = 0.f;
+      } else if (nsplit == 1) {
+        zv[q] = z[t * E + e];
+      } else {
+        float acc = z[t * E + e];
+        for (int sp = 1; sp < nsplit; ++sp) acc += z[static_cast<int64_t>(sp) * T * E + t * E + e];
+        if (bias != nullptr) acc += bias[t * bias_stride + e];
+        if (logits != nullptr) logits[t * E + e] = acc;
+        zv[q] = acc;
+      }
     }
     float zsel[MOE_MAX_TOPK];
     int isel[MOE_MAX_TOPK];
@@ -317,14 +378,15 @@ __global__ void __launch_bounds__(256) topk_from_logits_kernel(
 template <typename TX>
 cudaError_t launch_router_typed(const Shape& s, const TX* x, const float* w_router,
                                 const float* bias, int64_t bias_stride, float* logits,
-                                int32_t* topk_idx, float* topk_w, cudaStream_t st) {
+                                int32_t* topk_idx, float* topk_w, float* partials,
+                                cudaStream_t st) {
   const int d = static_cast<int>(s.d);
   if (s.E <= 32) {
     const int ET = s.E <= 8 ? 8 : (s.E <= 16 ? 16 : 32);
     const int TW = 32 / ET;
-    const int64_t warps = (s.T + TW - 1) / TW;
-    const int64_t blocks_needed = (warps + 7) / 8;
-    const int blocks = static_cast<int>(blocks_needed < 148 * 16 ? blocks_needed : 148 * 16);
+    const int64_t blocks_needed = (s.T + TW - 1) / TW;
+    const int64_t cap = static_cast<int64_t>(sm_count()) * 64;
+    const int blocks = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
     if (ET == 8)
       router_small_e_kernel<TX, 8><<<blocks, 256, 0, st>>>(x, w_router, bias, bias_stride, s.T, d,
                                                            s.E, s.k, s.gating, logits, topk_idx,
@@ -339,28 +401,55 @@ cudaError_t launch_router_typed(const Shape& s, const TX* x, const float* w_rout
                                                             topk_idx, topk_w);
     return cudaGetLastError();
   }
-  dim3 grid((s.E + RT_N - 1) / RT_N, static_cast<unsigned>((s.T + RT_M - 1) / RT_M));
+  const int tiles_n = (s.E + RT_N - 1) / RT_N;
+  const int64_t tiles_m = (s.T + RT_M - 1) / RT_M;
+  const int nsplit = router_splits(s);
+  int k_per_split = (d + nsplit - 1) / nsplit;
+  k_per_split = (k_per_split + RT_K - 1) / RT_K * RT_K;
+  dim3 grid(tiles_n, static_cast<unsigned>(tiles_m), nsplit);
   router_gemm_kernel<TX><<<grid, 256, 0, st>>>(x, w_router, bias, bias_stride, s.T, d, s.E,
-                                               logits);
+                                               k_per_split, nsplit > 1 ? partials : logits);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const int64_t blocks_needed = (s.T + 7) / 8;
   const int blocks = static_cast<int>(blocks_needed < 148 * 16 ? blocks_needed : 148 * 16);
-  topk_from_logits_kernel<<<blocks, 256, 0, st>>>(logits, s.T, s.E, s.k, s.gating, topk_idx,
-                                                  topk_w);
+  topk_from_logits_kernel<<<blocks, 256, 0, st>>>(nsplit > 1 ? partials : logits, nsplit, bias,
+                                                  bias_stride, logits, s.T, s.E, s.k, s.gating,
+                                                  topk_idx, topk_w);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+cudaError_t launch_topk_from_logits(const Shape& s, const float* logits, int32_t* topk_idx,
+                                    float* topk_w, cudaStream_t st) {
+  const int64_t blocks_needed = (s.T + 7) / 8;
+  const int blocks = static_cast<int>(blocks_needed < 148 * 16 ? blocks_needed : 148 * 16);
+  topk_from_logits_kernel<<<blocks, 256, 0, st>>>(logits, 1, nullptr, 0, nullptr, s.T, s.E, s.k,
+                                                  s.gating, topk_idx, topk_w);
+  return cudaGetLastError();
+}
+
+int router_splits(const Shape& s) {
+  if (s.E <= 32) return 1;
+  const int64_t tiles = ((s.E + RT_N - 1) / RT_N) * ((s.T + RT_M - 1) / RT_M);
+  const int64_t target = 296;  // two waves of blocks on a 148-SM part; device-independent
+  if (tiles >= target) return 1;
+  int64_t sp = (target + tiles - 1) / tiles;
+  const int64_t max_sp = (s.d + 4 * RT_K - 1) / (4 * RT_K);  // at least 4 K steps per split
+  if (sp > max_sp) sp = max_sp;
+  if (sp > kMaxRouterSplits) sp = kMaxRouterSplits;
+  return sp < 1 ? 1 : static_cast<int>(sp);
+}
+
 cudaError_t launch_router(const Shape& s, const void* x, const float* w_router,
                           const float* bias, int64_t bias_stride, float* logits,
-                          int32_t* topk_idx, float* topk_w, cudaStream_t st) {
+                          int32_t* topk_idx, float* topk_w, float* partials, cudaStream_t st) {
   if (s.dtype == MOE_F32)
     return launch_router_typed(s, static_cast<const float*>(x), w_router, bias, bias_stride,
-                               logits, topk_idx, topk_w, st);
+                               logits, topk_idx, topk_w, partials, st);
   return launch_router_typed(s, static_cast<const __nv_bfloat16*>(x), w_router, bias,
-                             bias_stride, logits, topk_idx, topk_w, st);
+                             bias_stride, logits, topk_idx, topk_w, partials, st);
 }
 
 }  // namespace moe

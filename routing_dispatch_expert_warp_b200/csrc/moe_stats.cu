@@ -26,7 +26,9 @@ __device__ double percentile_linear(const int32_t* s, int n, double p) {
   return __dadd_rn(static_cast<double>(s[lo]), __dmul_rn(__dadd_rn(h, -fl), diff));
 }
 
-__global__ void __launch_bounds__(MOE_MAX_EXPERTS) stats_kernel(
+constexpr int kStatsThreads = 1024;
+
+__global__ void __launch_bounds__(kStatsThreads) stats_kernel(
     const int32_t* __restrict__ routed, const int32_t* __restrict__ kept,
     const int32_t* __restrict__ assign_row, int64_t T, int k, int E, int64_t C,
     moe_load_stats_t* __restrict__ out) {
@@ -36,7 +38,7 @@ __global__ void __launch_bounds__(MOE_MAX_EXPERTS) stats_kernel(
   __shared__ unsigned long long drop_rank[MOE_MAX_TOPK];
   __shared__ unsigned long long tok_drop, tok_full;
   const int tid = threadIdx.x;
-  sorted[tid] = tid < E ? kept[tid] : INT_MAX;
+  if (tid < MOE_MAX_EXPERTS) sorted[tid] = tid < E ? kept[tid] : INT_MAX;
   if (tid == 0) {
     sum_kept = 0;
     sum_routed = 0;
@@ -55,7 +57,7 @@ __global__ void __launch_bounds__(MOE_MAX_EXPERTS) stats_kernel(
   for (int size = 2; size <= MOE_MAX_EXPERTS; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       const int partner = tid ^ stride;
-      if (partner > tid) {
+      if (tid < MOE_MAX_EXPERTS && partner > tid) {
         const bool asc = (tid & size) == 0;
         const int32_t a = sorted[tid], b = sorted[partner];
         if ((a > b) == asc) {
@@ -126,8 +128,7 @@ __global__ void __launch_bounds__(MOE_MAX_EXPERTS) stats_kernel(
 
 cudaError_t launch_stats(const Shape& s, const int32_t* routed, const int32_t* kept,
                          const int32_t* assign_row, moe_load_stats_t* out, cudaStream_t st) {
-  stats_kernel<<<1, MOE_MAX_EXPERTS, 0, st>>>(routed, kept, assign_row, s.T, s.k, s.E, s.C,
-                                              out);
+  stats_kernel<<<1, kStatsThreads, 0, st>>>(routed, kept, assign_row, s.T, s.k, s.E, s.C, out);
   return cudaGetLastError();
 }
 

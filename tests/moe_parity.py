@@ -16,7 +16,14 @@ from routing_dispatch_expert_warp_b200 import workload as W
 # 1e-5 (fp32 layers) and 2e-2 (bf16 layers).  Logits: fp32 accumulation over d terms.
 TOL_OUT = {W.F32: 1e-5, W.BF16: 2e-2}
 TOL_W = 1e-6
-TOL_LOGIT = 1e-5
+TOL_LOGIT = 1e-5          # fp32 FMA router
+TOL_LOGIT_SPLIT = 1e-4    # tensor-core router with W_r split into two bf16 terms
+
+
+def router_on_tensor_cores(shape) -> bool:
+    """The library's documented rule (include/moe.h, moe_route)."""
+    return (shape.dtype == W.BF16 and shape.E > 32 and shape.d_model % 64 == 0
+            and shape.T >= 512)
 
 
 def rel_fro(a, b) -> float:
@@ -103,7 +110,8 @@ def check_routing(run: GpuRun, sample_rows=None) -> dict:
         bias = f64(i.logit_bias) if i.logit_bias.dim() == 1 else f64(i.logit_bias[trows])
     z64 = O.router_logits(f64(i.x[trows]), f64(i.w_router), bias)
     err = np.abs(z32[rows].astype(np.float64) - z64) / (1.0 + np.abs(z64))
-    assert err.max() <= TOL_LOGIT, f"logits max scaled error {err.max():.3g}"
+    tol = TOL_LOGIT_SPLIT if router_on_tensor_cores(s) else TOL_LOGIT
+    assert err.max() <= tol, f"logits max scaled error {err.max():.3g} (tol {tol})"
     r = O.route(z32, s.k, s.gating, cf32(s), s.layout)
     np.testing.assert_array_equal(i64(b.topk_idx), r["idx"])
     w_err = np.abs(f64(b.topk_w) - r["w"]).max()

@@ -78,6 +78,8 @@ EDGES = [
     _edge(200, 64, 64, 16, 1, cf=0.05),          # capacity 1 with top-1
     _edge(129, 128, 128, 32, 3, gating=W.SIGMOID, dtype=W.F32),
     _edge(300, 256, 128, 200, 6, cf=1.0),         # E not a power of two, > 32
+    _edge(600, 256, 128, 200, 4, gating=W.SIGMOID, cf=1.5),   # tensor-core router, ragged E
+    _edge(520, 128, 128, 64, 8, gating=W.SIGMOID),            # tensor-core router, E = 64
 ]
 
 
