@@ -75,9 +75,21 @@ __global__ void __launch_bounds__(MOE_MAX_EXPERTS) dispatch_scan_kernel(
   const int e = threadIdx.x;
   int64_t run = 0;
   if (e < E) {
-    for (int64_t b = 0; b < nblk; ++b) {
+    // exclusive scan over the blocks; loads issued 8 at a time, sums in block order
+    int64_t b = 0;
+    for (; b + 8 <= nblk; b += 8) {
+      int32_t c[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) c[u] = hist[(b + u) * E + e];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        hist[(b + u) * E + e] = static_cast<int32_t>(run);  // becomes the block's base slot
+        run += c[u];
+      }
+    }
+    for (; b < nblk; ++b) {
       const int32_t c = hist[b * E + e];
-      hist[b * E + e] = static_cast<int32_t>(run);  // becomes the block's base slot
+      hist[b * E + e] = static_cast<int32_t>(run);
       run += c;
     }
   }

@@ -329,8 +329,19 @@ __global__ void __launch_bounds__(256) topk_from_logits_kernel(
       } else if (nsplit == 1) {
         zv[q] = z[t * E + e];
       } else {
-        float acc = z[t * E + e];
-        for (int sp = 1; sp < nsplit; ++sp) acc += z[static_cast<int64_t>(sp) * T * E + t * E + e];
+        // loads in batches of 8 (independent), additions strictly in split order
+        const float* zp = z + t * E + e;
+        const int64_t stride = T * E;
+        float acc = zp[0];
+        int sp = 1;
+        for (; sp + 8 <= nsplit; sp += 8) {
+          float b[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) b[u] = zp[(sp + u) * stride];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) acc += b[u];
+        }
+        for (; sp < nsplit; ++sp) acc += zp[sp * stride];
         if (bias != nullptr) acc += bias[t * bias_stride + e];
         if (logits != nullptr) logits[t * E + e] = acc;
         zv[q] = acc;

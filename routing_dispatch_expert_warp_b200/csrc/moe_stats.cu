@@ -28,16 +28,24 @@ __device__ double percentile_linear(const int32_t* s, int n, double p) {
 
 constexpr int kStatsThreads = 1024;
 
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+// Counters are reduced within each warp first and then added with 32-bit shared atomics
+// (one per warp), so the block never serialises on a contended 64-bit atomic.
 __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
     const int32_t* __restrict__ routed, const int32_t* __restrict__ kept,
     const int32_t* __restrict__ assign_row, int64_t T, int k, int E, int64_t C,
     moe_load_stats_t* __restrict__ out) {
   __shared__ int32_t sorted[MOE_MAX_EXPERTS];
-  __shared__ unsigned long long sum_kept, sum_routed;
-  __shared__ int max_routed;
-  __shared__ unsigned long long drop_rank[MOE_MAX_TOPK];
-  __shared__ unsigned long long tok_drop, tok_full;
+  __shared__ int sum_kept, sum_routed, max_routed;
+  __shared__ int drop_rank[MOE_MAX_TOPK];
+  __shared__ int tok_drop, tok_full;
   const int tid = threadIdx.x;
+  const int lane = tid & 31;
   if (tid < MOE_MAX_EXPERTS) sorted[tid] = tid < E ? kept[tid] : INT_MAX;
   if (tid == 0) {
     sum_kept = 0;
@@ -48,12 +56,20 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
   }
   if (tid < MOE_MAX_TOPK) drop_rank[tid] = 0;
   __syncthreads();
-  if (tid < E) {
-    atomicAdd(&sum_kept, static_cast<unsigned long long>(kept[tid]));
-    atomicAdd(&sum_routed, static_cast<unsigned long long>(routed[tid]));
-    atomicMax(&max_routed, routed[tid]);
+  if (tid < MOE_MAX_EXPERTS) {  // warps 0..7 cover the experts
+    const int kv = tid < E ? kept[tid] : 0;
+    const int rv = tid < E ? routed[tid] : 0;
+    int mx = rv;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    const int sk = warp_sum(kv), sr = warp_sum(rv);
+    if (lane == 0) {
+      atomicAdd(&sum_kept, sk);
+      atomicAdd(&sum_routed, sr);
+      atomicMax(&max_routed, mx);
+    }
   }
-  // bitonic sort, ascending
+  // bitonic sort of the 256 slots, ascending
   for (int size = 2; size <= MOE_MAX_EXPERTS; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       const int partner = tid ^ stride;
@@ -68,16 +84,16 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
       __syncthreads();
     }
   }
-  // drops per pick rank and per token
-  unsigned long long rank_local[MOE_MAX_TOPK];
+  // drops per pick rank and per token (thread per token, counters in registers)
+  int rank_local[MOE_MAX_TOPK];
 #pragma unroll
   for (int j = 0; j < MOE_MAX_TOPK; ++j) rank_local[j] = 0;
-  unsigned long long td = 0, tf = 0;
+  int td = 0, tf = 0;
   for (int64_t t = tid; t < T; t += blockDim.x) {
     int nd = 0;
 #pragma unroll
     for (int j = 0; j < MOE_MAX_TOPK; ++j) {
-      if (j < k && assign_row[t * k + j] < 0) {
+      if (j < k && __ldg(assign_row + t * k + j) < 0) {
         ++rank_local[j];
         ++nd;
       }
@@ -86,10 +102,16 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
     tf += nd == k;
   }
 #pragma unroll
-  for (int j = 0; j < MOE_MAX_TOPK; ++j)
-    if (j < k && rank_local[j]) atomicAdd(&drop_rank[j], rank_local[j]);
-  if (td) atomicAdd(&tok_drop, td);
-  if (tf) atomicAdd(&tok_full, tf);
+  for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+    const int v = warp_sum(rank_local[j]);
+    if (lane == 0 && v) atomicAdd(&drop_rank[j], v);
+  }
+  td = warp_sum(td);
+  tf = warp_sum(tf);
+  if (lane == 0) {
+    if (td) atomicAdd(&tok_drop, td);
+    if (tf) atomicAdd(&tok_full, tf);
+  }
   __syncthreads();
 
   if (tid == 0) {
@@ -98,11 +120,11 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
     st.k = k;
     st.active_tokens = T;
     st.capacity = C;
-    st.routed_total = static_cast<int64_t>(sum_routed);
-    st.kept_total = static_cast<int64_t>(sum_kept);
+    st.routed_total = sum_routed;
+    st.kept_total = sum_kept;
     st.dropped = T * k - static_cast<int64_t>(sum_kept);
-    st.tokens_with_drop = static_cast<int64_t>(tok_drop);
-    st.tokens_fully_dropped = static_cast<int64_t>(tok_full);
+    st.tokens_with_drop = tok_drop;
+    st.tokens_fully_dropped = tok_full;
     st.p50 = percentile_linear(sorted, E, 0.50);
     st.p95 = percentile_linear(sorted, E, 0.95);
     st.p99 = percentile_linear(sorted, E, 0.99);
@@ -118,8 +140,7 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
     for (int i = 0; i < n_top; ++i) top += sorted[E - 1 - i];
     st.top5pct_share =
         sum_kept > 0 ? static_cast<double>(top) / static_cast<double>(sum_kept) : 0.0;
-    for (int j = 0; j < MOE_MAX_TOPK; ++j)
-      st.dropped_by_rank[j] = j < k ? static_cast<int64_t>(drop_rank[j]) : 0;
+    for (int j = 0; j < MOE_MAX_TOPK; ++j) st.dropped_by_rank[j] = j < k ? drop_rank[j] : 0;
     *out = st;
   }
 }
