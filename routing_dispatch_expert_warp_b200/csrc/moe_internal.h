@@ -12,6 +12,7 @@
 namespace moe {
 
 constexpr int kDispatchBlockTokens = 256;   // tokens per block of the ranking kernels
+constexpr int kMaxDevices = 64;
 constexpr size_t kWsAlign = 256;
 
 // A validated moe_config_t with the derived sizes.
@@ -83,7 +84,6 @@ int sm_count();
 
 // Allocation-free dispatch: scratch lives in a fixed device array (moe_dispatch.cu).
 constexpr size_t kStaticDispatchHistBytes = size_t(1) << 20;  // 1 MiB of block histograms
-constexpr int kMaxDevices = 64;
 cudaError_t dispatch_static_scratch(const Shape& s, const void* x, const int32_t* topk_idx,
                                     int32_t* routed, int32_t* kept, int32_t* offsets,
                                     int32_t* assign_row, int32_t* token_of_row, void* x_perm,

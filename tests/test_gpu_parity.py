@@ -129,6 +129,35 @@ def test_capacity_exactly_hit_keeps_everything():
     check_stats(st, r)
 
 
+@pytest.mark.parametrize("counts,d,f", [
+    ((129, 176, 177, 256), 256, 384),     # tails 1, 48 (folded into the last tile), 49, 0
+    ((16, 17, 300, 140), 384, 256),       # buckets below one tile; tails 44 and 12; d not /256
+    ((170, 208, 131, 175), 128, 640),     # tails 42, 80, 3, 47
+])
+def test_bucket_tails_of_every_size(counts, d, f):
+    """Exact per-expert bucket sizes (top-1 picks forced by a [T, E] bias) so that the grouped
+    GEMM meets tails that ride along with the last full tile, tails that get a tile of their
+    own, buckets smaller than a tile and buckets of whole tiles."""
+    E, k = len(counts), 1
+    T = sum(counts)
+    shape = _edge(T, d, f, E, k)
+    inp = W.make_inputs(shape, device="cuda")
+    owner = torch.cat([torch.full((c,), e, dtype=torch.long) for e, c in enumerate(counts)])
+    owner = owner[torch.randperm(T, generator=torch.Generator().manual_seed(5))].cuda()
+    bias = torch.full((T, E), -40.0, device="cuda")
+    bias[torch.arange(T, device="cuda"), owner] = 40.0
+    inp.logit_bias = bias.contiguous()
+    run = GpuRun(shape, inp)
+    st = run.all_stages()
+    r = check_routing(run)
+    assert tuple(int(c) for c in r["kept"]) == counts
+    check_permute(run, r)
+    check_ffn_rows(run, r)
+    check_combine(run, r)
+    check_stats(st, r)
+    check_layer_output(run, run.b.out, r)
+
+
 def test_tied_logits_pick_lower_index():
     shape = _edge(40, 64, 64, 16, 4, gating=W.SIGMOID)
     inp = W.make_inputs(shape, device="cuda")
