@@ -122,8 +122,13 @@ WsLayout workspace_layout(const Shape& s) {
   off += l.logits_bytes;
   const int splits = router_splits(s);
   l.partials = off;
-  l.partials_bytes =
-      splits > 1 ? round_up(static_cast<size_t>(splits) * s.T * s.E * sizeof(float)) : 0;
+  if (s.E <= 32) {  // lane-ordered copy of W_r for the small-E router
+    const size_t et = s.E <= 8 ? 8 : (s.E <= 16 ? 16 : 32);
+    l.partials_bytes = round_up(static_cast<size_t>((s.d + 255) / 256) * 256 * et * sizeof(float));
+  } else {
+    l.partials_bytes =
+        splits > 1 ? round_up(static_cast<size_t>(splits) * s.T * s.E * sizeof(float)) : 0;
+  }
   off += l.partials_bytes;
   l.router_tc = off;
   l.router_tc_bytes = round_up(router_tc_workspace_bytes(s));

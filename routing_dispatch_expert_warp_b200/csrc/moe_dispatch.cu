@@ -16,11 +16,11 @@
 // Kernels (no host synchronisation anywhere):
 //   1. count:  block b of 256 tokens builds, per warp w and expert e, the 32-bit mask of
 //              lanes (tokens) that picked e; per-block counts = sum of popcounts.
-//   2. scan:   one block: per expert, exclusive scan of the block counts (the block's base
-//              slot), routed = total, kept = min(routed, C), bucket offsets.
-//   3. rank:   block b rebuilds its masks; slot = block base + earlier warps' counts +
-//              popcount(mask & lanes below me).  Writes assign_row and token_of_row.
-//   4. permute: token-major row copy with bulk (TMA) copies: each row of x is read from HBM
+//   2. rank:   block b rebuilds its masks and, from all blocks' counts, its base slot per
+//              expert, routed = total, kept = min(routed, C) and the bucket offsets; then
+//              slot = block base + earlier warps' counts + popcount(mask & lanes below me).
+//              Writes assign_row and token_of_row (-1 for rows no assignment uses).
+//   3. permute: token-major row copy with bulk (TMA) copies: each row of x is read from HBM
 //              once into shared memory and written to each of its kept rows of x_perm.
 #include <mutex>
 
@@ -67,106 +67,123 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_count_kernel(
   }
 }
 
-// One block of MOE_MAX_EXPERTS threads, thread e owns expert e.
-__global__ void __launch_bounds__(MOE_MAX_EXPERTS) dispatch_scan_kernel(
-    int32_t* __restrict__ hist, int64_t nblk, int E, int64_t C, int layout,
-    int32_t* __restrict__ routed, int32_t* __restrict__ kept, int32_t* __restrict__ offsets) {
+// Ranking.  Every block first derives what it needs from the per-block counts of all
+// blocks: thread e adds up expert e's counts over the blocks (routed total, and the part
+// that comes from blocks before this one), caps the total at C (kept), and the block scans
+// kept over the experts (bucket offsets).  Block 0 publishes routed / kept / offsets; the
+// others only use them.  Then slot = base from earlier blocks + earlier warps of this block
+// + popcount(mask & lanes below me), kept iff slot < C, row = offset + slot.  Finally the
+// rows no assignment uses are marked -1 in token_of_row.
+__global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
+    const int32_t* __restrict__ topk_idx, int64_t T, int k, int E, int64_t C, int layout,
+    int64_t nblk, const int32_t* __restrict__ hist, int32_t* __restrict__ routed,
+    int32_t* __restrict__ kept, int32_t* __restrict__ offsets, int32_t* __restrict__ assign_row,
+    int32_t* __restrict__ token_of_row, int64_t max_rows) {
+  static_assert(kDispatchBlockTokens == MOE_MAX_EXPERTS, "one thread per expert");
+  __shared__ uint32_t masks[kWarps][MOE_MAX_EXPERTS];
+  __shared__ int32_t wbase[kWarps][MOE_MAX_EXPERTS];
+  __shared__ int32_t off_s[MOE_MAX_EXPERTS];
+  __shared__ int32_t kept_s[MOE_MAX_EXPERTS];
   __shared__ int64_t scan[MOE_MAX_EXPERTS];
+  build_masks(topk_idx, T, k, E, masks, nullptr);
+
   const int e = threadIdx.x;
-  int64_t run = 0;
+  int64_t run = 0, before = 0;
   if (e < E) {
-    // exclusive scan over the blocks; loads issued 8 at a time, sums in block order
     int64_t b = 0;
-    for (; b + 8 <= nblk; b += 8) {
+    for (; b + 8 <= nblk; b += 8) {  // loads issued 8 at a time, sums in block order
       int32_t c[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) c[u] = hist[(b + u) * E + e];
+      for (int u = 0; u < 8; ++u) c[u] = __ldg(hist + (b + u) * E + e);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        hist[(b + u) * E + e] = static_cast<int32_t>(run);  // becomes the block's base slot
+        if (b + u == blockIdx.x) before = run;
         run += c[u];
       }
     }
     for (; b < nblk; ++b) {
-      const int32_t c = hist[b * E + e];
-      hist[b * E + e] = static_cast<int32_t>(run);
-      run += c;
+      if (b == blockIdx.x) before = run;
+      run += __ldg(hist + b * E + e);
     }
   }
   const int64_t kp = (e < E) ? ((C >= 0 && run > C) ? C : run) : 0;
-  if (e < E) {
-    routed[e] = static_cast<int32_t>(run);
-    kept[e] = static_cast<int32_t>(kp);
-  }
-  // inclusive scan of kept over experts (Hillis-Steele, 256 entries)
   scan[e] = kp;
   __syncthreads();
-  for (int off = 1; off < MOE_MAX_EXPERTS; off <<= 1) {
+  for (int off = 1; off < MOE_MAX_EXPERTS; off <<= 1) {  // inclusive scan over experts
     const int64_t add = e >= off ? scan[e - off] : 0;
     __syncthreads();
     scan[e] += add;
     __syncthreads();
   }
+  const int64_t total_kept = scan[MOE_MAX_EXPERTS - 1];
   if (e < E) {
-    if (layout == MOE_LAYOUT_PADDED) {
-      offsets[e] = static_cast<int32_t>(static_cast<int64_t>(e) * C);
-      if (e == E - 1) offsets[E] = static_cast<int32_t>(static_cast<int64_t>(E) * C);
-    } else {
-      offsets[e] = static_cast<int32_t>(scan[e] - kp);
-      if (e == E - 1) offsets[E] = static_cast<int32_t>(scan[e]);
-    }
-  }
-}
-
-__global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
-    const int32_t* __restrict__ topk_idx, int64_t T, int k, int E, int64_t C,
-    const int32_t* __restrict__ base, const int32_t* __restrict__ offsets,
-    int32_t* __restrict__ assign_row, int32_t* __restrict__ token_of_row, DevStatus* status) {
-  __shared__ uint32_t masks[kWarps][MOE_MAX_EXPERTS];
-  __shared__ int32_t wbase[kWarps][MOE_MAX_EXPERTS];
-  __shared__ int32_t off_s[MOE_MAX_EXPERTS];
-  build_masks(topk_idx, T, k, E, masks, nullptr);
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int32_t run = base[static_cast<int64_t>(blockIdx.x) * E + e];
+    const int64_t off =
+        layout == MOE_LAYOUT_PADDED ? static_cast<int64_t>(e) * C : scan[e] - kp;
+    off_s[e] = static_cast<int32_t>(off);
+    kept_s[e] = static_cast<int32_t>(kp);
+    int32_t wb = static_cast<int32_t>(before);
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
-      wbase[w][e] = run;
-      run += __popc(masks[w][e]);
+      wbase[w][e] = wb;
+      wb += __popc(masks[w][e]);
     }
-    off_s[e] = offsets[e];
+    if (blockIdx.x == 0) {
+      routed[e] = static_cast<int32_t>(run);
+      kept[e] = static_cast<int32_t>(kp);
+      offsets[e] = static_cast<int32_t>(off);
+      if (e == E - 1)
+        offsets[E] = static_cast<int32_t>(layout == MOE_LAYOUT_PADDED
+                                              ? static_cast<int64_t>(E) * C
+                                              : total_kept);
+    }
   }
   __syncthreads();
+
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kDispatchBlockTokens + threadIdx.x;
-  if (t >= T) return;
-  const int w = threadIdx.x >> 5;
-  const uint32_t below = (1u << (threadIdx.x & 31)) - 1u;
-  for (int j = 0; j < k; ++j) {
-    const int e = topk_idx[t * k + j];
-    int32_t row = -1;
-    if (e >= 0 && e < E) {
-      const int64_t slot = wbase[w][e] + __popc(masks[w][e] & below);
-      if (C < 0 || slot < C) {
-        row = off_s[e] + static_cast<int32_t>(slot);
-        token_of_row[row] = static_cast<int32_t>(t);
+  if (t < T) {
+    const int w = threadIdx.x >> 5;
+    const uint32_t below = (1u << (threadIdx.x & 31)) - 1u;
+    for (int j = 0; j < k; ++j) {
+      const int ee = topk_idx[t * k + j];
+      int32_t row = -1;
+      if (ee >= 0 && ee < E) {
+        const int64_t slot = wbase[w][ee] + __popc(masks[w][ee] & below);
+        if (C < 0 || slot < C) {
+          row = off_s[ee] + static_cast<int32_t>(slot);
+          token_of_row[row] = static_cast<int32_t>(t);
+        }
       }
+      assign_row[t * k + j] = row;
     }
-    assign_row[t * k + j] = row;
+  }
+
+  // unused rows: COMPACT [total_kept, max_rows); PADDED the slots past kept in each bucket
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (layout == MOE_LAYOUT_PADDED) {
+    for (int64_t r = first; r < max_rows; r += stride) {
+      const int64_t ee = r / C;
+      if (ee < E && r - ee * C >= kept_s[ee]) token_of_row[r] = -1;
+    }
+  } else {
+    for (int64_t r = total_kept + first; r < max_rows; r += stride) token_of_row[r] = -1;
   }
 }
 
 // Token-major bulk copy.  One thread per block issues everything: a ring of NBUF shared
 // buffers, LOOKAHEAD loads in flight, stores of the rows already loaded in flight
 // behind them.  A work item is one segment (<= 16 KB) of one token's row.
-constexpr int kPermNBuf = 8;
-constexpr int kPermLookahead = 4;
 constexpr uint32_t kPermMaxSeg = 16384;
+constexpr int kPermMaxNBuf = 16;
 
+template <int kPermNBuf, int kPermLookahead>
 __global__ void __launch_bounds__(32) permute_rows_kernel(
     const uint8_t* __restrict__ x, const int32_t* __restrict__ assign_row, int64_t T, int k,
     int64_t row_bytes, uint32_t seg_bytes, int64_t segs_per_row, uint8_t* __restrict__ x_perm,
     DevStatus* status, uint64_t wait_ns) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full[kPermNBuf];
+  static_assert(kPermNBuf <= kPermMaxNBuf && kPermLookahead < kPermNBuf, "ring shape");
   if (threadIdx.x != 0) return;
   for (int b = 0; b < kPermNBuf; ++b) mbar_init(&full[b], 1);
   fence_barrier_init();
@@ -246,16 +263,13 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
                             int32_t* hist, DevStatus* status, uint64_t wait_ns,
                             cudaStream_t st) {
   const int64_t nblk = dispatch_blocks(s.T);
-  cudaError_t err = cudaMemsetAsync(token_of_row, 0xFF, sizeof(int32_t) * s.max_rows, st);
-  if (err != cudaSuccess) return err;
+  cudaError_t err;
   dispatch_count_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
       topk_idx, s.T, s.k, s.E, hist, status);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  dispatch_scan_kernel<<<1, MOE_MAX_EXPERTS, 0, st>>>(hist, nblk, s.E, s.C, s.layout, routed,
-                                                      kept, offsets);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
   dispatch_rank_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
-      topk_idx, s.T, s.k, s.E, s.C, hist, offsets, assign_row, token_of_row, status);
+      topk_idx, s.T, s.k, s.E, s.C, s.layout, nblk, hist, routed, kept, offsets, assign_row,
+      token_of_row, s.max_rows);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
 
   const int64_t row_bytes = s.d * s.elem;
@@ -263,18 +277,36 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
   // equal segments, each a multiple of 16 bytes
   int64_t seg = (row_bytes + segs - 1) / segs;
   seg = (seg + 15) / 16 * 16;
-  const size_t smem = static_cast<size_t>(kPermNBuf) * seg;
-  err = cudaFuncSetAttribute(permute_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kPermNBuf * kPermMaxSeg));
-  if (err != cudaSuccess) return err;
+  // about 96 KB of ring per block, two blocks per SM; half the ring is loads in flight
   const int64_t items = s.T * segs;
-  const int64_t per_sm = smem <= 64 * 1024 ? 3 : (smem <= 100 * 1024 ? 2 : 1);
-  int64_t grid = static_cast<int64_t>(sm_count()) * per_sm;
+  int64_t grid = static_cast<int64_t>(sm_count()) * 2;
   if (grid > items) grid = items;
   if (grid < 1) grid = 1;
-  permute_rows_kernel<<<static_cast<unsigned>(grid), 32, smem, st>>>(
-      static_cast<const uint8_t*>(x), assign_row, s.T, s.k, row_bytes,
-      static_cast<uint32_t>(seg), segs, static_cast<uint8_t*>(x_perm), status, wait_ns);
+  const uint8_t* xb = static_cast<const uint8_t*>(x);
+  uint8_t* xp = static_cast<uint8_t*>(x_perm);
+  const uint32_t sg = static_cast<uint32_t>(seg);
+  if (seg <= 6 * 1024) {
+    const size_t smem = 16 * static_cast<size_t>(seg);
+    err = cudaFuncSetAttribute(permute_rows_kernel<16, 8>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    permute_rows_kernel<16, 8><<<static_cast<unsigned>(grid), 32, smem, st>>>(
+        xb, assign_row, s.T, s.k, row_bytes, sg, segs, xp, status, wait_ns);
+  } else if (seg <= 8 * 1024) {
+    const size_t smem = 12 * static_cast<size_t>(seg);
+    err = cudaFuncSetAttribute(permute_rows_kernel<12, 6>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    permute_rows_kernel<12, 6><<<static_cast<unsigned>(grid), 32, smem, st>>>(
+        xb, assign_row, s.T, s.k, row_bytes, sg, segs, xp, status, wait_ns);
+  } else {
+    const size_t smem = 6 * static_cast<size_t>(seg);
+    err = cudaFuncSetAttribute(permute_rows_kernel<6, 3>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    permute_rows_kernel<6, 3><<<static_cast<unsigned>(grid), 32, smem, st>>>(
+        xb, assign_row, s.T, s.k, row_bytes, sg, segs, xp, status, wait_ns);
+  }
   return cudaGetLastError();
 }
 

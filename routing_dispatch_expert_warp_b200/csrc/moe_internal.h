@@ -31,7 +31,7 @@ struct WsLayout {
   size_t hist_bytes;
   size_t logits;        // [T, E] fp32 logits when the caller passes none
   size_t logits_bytes;
-  size_t partials;      // split-K router partial sums
+  size_t partials;      // split-K router partial sums (E > 32) / lane-ordered W_r (E <= 32)
   size_t partials_bytes;
   size_t router_tc;     // bf16 split of W_r for the tensor-core router
   size_t router_tc_bytes;

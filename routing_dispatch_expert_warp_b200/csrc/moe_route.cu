@@ -16,6 +16,8 @@
 //     per token selects the top-k from z.
 #include <math.h>
 
+#include <type_traits>
+
 #include "moe_internal.h"
 
 namespace moe {
@@ -77,6 +79,49 @@ __device__ __forceinline__ void gate_weights(const float* zsel, int k, int gatin
 // tokens x ET experts) with a butterfly transpose-reduction, the 8 warp partials are added
 // in warp order through shared memory, and warp 0 finishes: bias, logits, top-k and gate
 // weights.
+// 8 consecutive elements of x kept in their storage form until used (4 registers for bf16).
+template <typename TX>
+struct XRaw;
+template <>
+struct XRaw<__nv_bfloat16> {
+  uint4 v;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) {
+    v = __ldg(reinterpret_cast<const uint4*>(p));
+  }
+  __device__ __forceinline__ void zero() { v = make_uint4(0u, 0u, 0u, 0u); }
+  template <int I>
+  __device__ __forceinline__ float get() const {
+    const uint32_t w = I < 2 ? v.x : (I < 4 ? v.y : (I < 6 ? v.z : v.w));
+    return (I & 1) ? bf16_hi(w) : bf16_lo(w);
+  }
+};
+template <>
+struct XRaw<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = __ldg(reinterpret_cast<const float4*>(p));
+    b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  }
+  __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+  template <int I>
+  __device__ __forceinline__ float get() const {
+    const float4& q = I < 4 ? a : b;
+    constexpr int J = I & 3;
+    return J == 0 ? q.x : (J == 1 ? q.y : (J == 2 ? q.z : q.w));
+  }
+};
+
+template <int RR, typename TX, int ET, int TW, int CPW>
+__device__ __forceinline__ void router_row_fma(const XRaw<TX> (&xr)[CPW][TW], int j,
+                                               const float (&wv)[ET], float (&v)[32]) {
+#pragma unroll
+  for (int tw = 0; tw < TW; ++tw) {
+    const float xval = xr[j][tw].template get<RR>();
+#pragma unroll
+    for (int e = 0; e < ET; ++e) v[tw * ET + e] = fmaf(xval, wv[e], v[tw * ET + e]);
+  }
+}
+
 template <typename TX>
 __device__ __forceinline__ void load_pair(const TX* p, float& a, float& b);
 template <>
@@ -93,17 +138,56 @@ __device__ __forceinline__ void load_pair<__nv_bfloat16>(const __nv_bfloat16* p,
   b = bf16_hi(v);
 }
 
+// W_r [d, E] re-laid out for the warp access pattern of the small-E router: in chunk c
+// (256 rows of d) lane l owns rows c*256 + 8l .. 8l+7; vector u = rr * (ET/4) + qq holds
+// row 8l + rr, experts 4qq .. 4qq+3, and the 32 lanes' vectors u are consecutive (512 B),
+// so every W load of the router is one fully used 512-byte span.  Experts past E and rows
+// past d are zero.
+template <int ET>
+__global__ void __launch_bounds__(256) router_weight_lanes_kernel(const float* __restrict__ w,
+                                                                  int d, int E,
+                                                                  float4* __restrict__ wl) {
+  constexpr int U = 8 * ET / 4;
+  const int nchunks = (d + 255) / 256;
+  const int64_t total = static_cast<int64_t>(nchunks) * U * 32;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int lane = static_cast<int>(i % 32);
+    const int u = static_cast<int>((i / 32) % U);
+    const int64_t c = i / (32 * U);
+    const int rr = u / (ET / 4), qq = u % (ET / 4);
+    const int64_t row = c * 256 + 8 * lane + rr;
+    const int e0 = qq * 4;
+    float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (row < d) {
+      const float* src = w + row * E;
+      f.x = e0 + 0 < E ? src[e0 + 0] : 0.f;
+      f.y = e0 + 1 < E ? src[e0 + 1] : 0.f;
+      f.z = e0 + 2 < E ? src[e0 + 2] : 0.f;
+      f.w = e0 + 3 < E ? src[e0 + 3] : 0.f;
+    }
+    wl[i] = f;
+  }
+}
+
+// One block scores TW = 32 / ET tokens.  The d axis is cut into 256-element chunks dealt
+// round-robin to the 8 warps; in a chunk lane l owns 8 consecutive elements (one 16-byte
+// load of x per token).  A warp first issues the x loads of up to CPW chunks at once, then
+// walks the lane-ordered W rows.  Each warp folds its 32 partial values (TW tokens x ET
+// experts) with a butterfly transpose-reduction, the 8 warp partials are added in warp
+// order through shared memory, and warp 0 finishes: bias, logits, top-k and gate weights.
 template <typename TX, int ET>
-__global__ void __launch_bounds__(256) router_small_e_kernel(
-    const TX* __restrict__ x, const float* __restrict__ w_router, const float* __restrict__ bias,
+__global__ void __launch_bounds__(256, ET == 8 ? 2 : 3) router_small_e_kernel(
+    const TX* __restrict__ x, const float4* __restrict__ wl, const float* __restrict__ bias,
     int64_t bias_stride, int64_t T, int d, int E, int k, int gating, float* __restrict__ logits,
     int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
   constexpr int TW = 32 / ET;  // tokens per block
   constexpr int NW = 8;        // warps per block
+  constexpr int CPW = sizeof(TX) == 2 ? 2 : 1;  // chunks whose x loads are in flight together
+  constexpr int U = 8 * ET / 4;
   __shared__ float part[NW][32];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const bool e_vec4 = (E % 4) == 0;
   const int nchunks = (d + 255) / 256;
 
   for (int64_t t0 = static_cast<int64_t>(blockIdx.x) * TW; t0 < T;
@@ -112,45 +196,40 @@ __global__ void __launch_bounds__(256) router_small_e_kernel(
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = 0.f;
 
-    for (int c = warp; c < nchunks; c += NW) {
+    for (int cb = warp; cb < nchunks; cb += NW * CPW) {
+      XRaw<TX> xr[CPW][TW];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int i0 = c * 256 + q * 64 + 2 * lane;
-        if (i0 >= d) continue;
-        float xa[TW], xb[TW];
+      for (int j = 0; j < CPW; ++j) {
+        const int i0 = (cb + NW * j) * 256 + lane * 8;
 #pragma unroll
         for (int tw = 0; tw < TW; ++tw) {
-          if (t0 + tw < T) {
-            load_pair<TX>(x + (t0 + tw) * d + i0, xa[tw], xb[tw]);
-          } else {
-            xa[tw] = xb[tw] = 0.f;
-          }
+          if (i0 < d && t0 + tw < T) xr[j][tw].load(x + (t0 + tw) * d + i0);
+          else xr[j][tw].zero();
         }
+      }
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
+      for (int j = 0; j < CPW; ++j) {
+        const int c = cb + NW * j;
+        if (c >= nchunks) continue;
+        const float4* wq = wl + static_cast<int64_t>(c) * U * 32 + lane;
+        auto row = [&](auto rr_const) {
+          constexpr int RR = decltype(rr_const)::value;
           float wv[ET];
-          const float* wrow = w_router + static_cast<int64_t>(i0 + r) * E;
-          if (e_vec4) {
 #pragma unroll
-            for (int qq = 0; qq < ET / 4; ++qq) {
-              if (4 * qq < E) {
-                const float4 f = __ldg(reinterpret_cast<const float4*>(wrow) + qq);
-                wv[4 * qq] = f.x; wv[4 * qq + 1] = f.y; wv[4 * qq + 2] = f.z; wv[4 * qq + 3] = f.w;
-              } else {
-                wv[4 * qq] = wv[4 * qq + 1] = wv[4 * qq + 2] = wv[4 * qq + 3] = 0.f;
-              }
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < ET; ++e) wv[e] = e < E ? __ldg(wrow + e) : 0.f;
+          for (int qq = 0; qq < ET / 4; ++qq) {
+            const float4 f = __ldg(wq + (RR * (ET / 4) + qq) * 32);
+            wv[4 * qq] = f.x; wv[4 * qq + 1] = f.y; wv[4 * qq + 2] = f.z; wv[4 * qq + 3] = f.w;
           }
-#pragma unroll
-          for (int tw = 0; tw < TW; ++tw) {
-            const float xv = r == 0 ? xa[tw] : xb[tw];
-#pragma unroll
-            for (int e = 0; e < ET; ++e) v[tw * ET + e] = fmaf(xv, wv[e], v[tw * ET + e]);
-          }
-        }
+          router_row_fma<RR, TX, ET, TW, CPW>(xr, j, wv, v);
+        };
+        row(std::integral_constant<int, 0>{});
+        row(std::integral_constant<int, 1>{});
+        row(std::integral_constant<int, 2>{});
+        row(std::integral_constant<int, 3>{});
+        row(std::integral_constant<int, 4>{});
+        row(std::integral_constant<int, 5>{});
+        row(std::integral_constant<int, 6>{});
+        row(std::integral_constant<int, 7>{});
       }
     }
 
@@ -386,6 +465,25 @@ __global__ void __launch_bounds__(256) topk_from_logits_kernel(
   }
 }
 
+template <typename TX, int ET>
+cudaError_t launch_small_e(const Shape& s, const TX* x, const float* w_router, const float* bias,
+                           int64_t bias_stride, float* logits, int32_t* topk_idx, float* topk_w,
+                           float4* wl, cudaStream_t st) {
+  const int d = static_cast<int>(s.d);
+  const int64_t lanes_total = static_cast<int64_t>((d + 255) / 256) * (8 * ET / 4) * 32;
+  const int pblocks = static_cast<int>((lanes_total + 255) / 256 < 1024 ? (lanes_total + 255) / 256 : 1024);
+  router_weight_lanes_kernel<ET><<<pblocks, 256, 0, st>>>(w_router, d, s.E, wl);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  constexpr int TW = 32 / ET;
+  const int64_t blocks_needed = (s.T + TW - 1) / TW;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 64;
+  const int blocks = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
+  router_small_e_kernel<TX, ET><<<blocks, 256, 0, st>>>(x, wl, bias, bias_stride, s.T, d, s.E,
+                                                        s.k, s.gating, logits, topk_idx, topk_w);
+  return cudaGetLastError();
+}
+
 template <typename TX>
 cudaError_t launch_router_typed(const Shape& s, const TX* x, const float* w_router,
                                 const float* bias, int64_t bias_stride, float* logits,
@@ -393,24 +491,15 @@ cudaError_t launch_router_typed(const Shape& s, const TX* x, const float* w_rout
                                 cudaStream_t st) {
   const int d = static_cast<int>(s.d);
   if (s.E <= 32) {
-    const int ET = s.E <= 8 ? 8 : (s.E <= 16 ? 16 : 32);
-    const int TW = 32 / ET;
-    const int64_t blocks_needed = (s.T + TW - 1) / TW;
-    const int64_t cap = static_cast<int64_t>(sm_count()) * 64;
-    const int blocks = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
-    if (ET == 8)
-      router_small_e_kernel<TX, 8><<<blocks, 256, 0, st>>>(x, w_router, bias, bias_stride, s.T, d,
-                                                           s.E, s.k, s.gating, logits, topk_idx,
-                                                           topk_w);
-    else if (ET == 16)
-      router_small_e_kernel<TX, 16><<<blocks, 256, 0, st>>>(x, w_router, bias, bias_stride, s.T,
-                                                            d, s.E, s.k, s.gating, logits,
-                                                            topk_idx, topk_w);
-    else
-      router_small_e_kernel<TX, 32><<<blocks, 256, 0, st>>>(x, w_router, bias, bias_stride, s.T,
-                                                            d, s.E, s.k, s.gating, logits,
-                                                            topk_idx, topk_w);
-    return cudaGetLastError();
+    float4* wl = reinterpret_cast<float4*>(partials);  // the workspace's router area
+    if (s.E <= 8)
+      return launch_small_e<TX, 8>(s, x, w_router, bias, bias_stride, logits, topk_idx, topk_w,
+                                   wl, st);
+    if (s.E <= 16)
+      return launch_small_e<TX, 16>(s, x, w_router, bias, bias_stride, logits, topk_idx, topk_w,
+                                    wl, st);
+    return launch_small_e<TX, 32>(s, x, w_router, bias, bias_stride, logits, topk_idx, topk_w,
+                                  wl, st);
   }
   const int tiles_n = (s.E + RT_N - 1) / RT_N;
   const int64_t tiles_m = (s.T + RT_M - 1) / RT_M;
