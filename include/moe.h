@@ -55,7 +55,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 #define MOE_MAX_EXPERTS 256
 #define MOE_MAX_TOPK 8
 
@@ -72,6 +72,8 @@ typedef enum {
 typedef enum { MOE_GATE_SOFTMAX = 0, MOE_GATE_SIGMOID = 1 } moe_gating_t;
 typedef enum { MOE_LAYOUT_COMPACT = 0, MOE_LAYOUT_PADDED = 1 } moe_layout_t;
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
+typedef enum { MOE_BIAS_SCORE_AND_WEIGHT = 0, MOE_BIAS_SELECTION_ONLY = 1 } moe_bias_mode_t;
+typedef enum { MOE_DROP_TOKEN_ORDER = 0, MOE_DROP_PICK_RANK = 1 } moe_drop_policy_t;
 
 /*
  * One layer's shape and routing rule.
@@ -90,6 +92,23 @@ typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
  *                   The router weight, logit bias, logits and gate weights are fp32.
  *   capacity_factor cf > 0: capacity C = ceil(cf * T * k / E) slots per expert;
  *                   cf <= 0: dropless ([EP-checks] "Capacity factor ...").
+ * Routing variants (all zero = the plain rule above):
+ *   n_groups, topk_groups   group-limited routing ([EP-serving] "Real-world implementation":
+ *                   DeepSeek-V3 limits the nodes a token's experts span).  With n_groups > 1
+ *                   the experts form n_groups equal contiguous groups; a group's score is
+ *                   the largest selection score of its experts; a token keeps the
+ *                   topk_groups best groups (equal scores -> lower group index) and takes
+ *                   its k experts from them only.  Needs E % n_groups == 0 and
+ *                   topk_groups * E / n_groups >= k.
+ *   bias_mode       MOE_BIAS_SCORE_AND_WEIGHT: the logit bias enters selection and weights;
+ *                   MOE_BIAS_SELECTION_ONLY: selection uses fp32(z + b) while the gate
+ *                   weights and the returned logits use the unbiased z (the bias-only
+ *                   balancing [EP-serving] "Future" names as loss-free load balancing).
+ *   drop_policy     MOE_DROP_TOKEN_ORDER: within an expert, slots go by token index;
+ *                   MOE_DROP_PICK_RANK: all first picks (in token order) before all second
+ *                   picks, and so on, so capacity drops later picks first ([EP-checks]
+ *                   "Top-2 does not insure against hot experts": second choices measured
+ *                   and dropped separately).
  */
 typedef struct moe_config {
   int64_t T;
@@ -101,6 +120,10 @@ typedef struct moe_config {
   int32_t layout;   /* moe_layout_t */
   int32_t dtype;    /* moe_dtype_t  */
   float capacity_factor;
+  int32_t n_groups;     /* 0 or 1: no group limit */
+  int32_t topk_groups;
+  int32_t bias_mode;    /* moe_bias_mode_t   */
+  int32_t drop_policy;  /* moe_drop_policy_t */
 } moe_config_t;
 
 /*

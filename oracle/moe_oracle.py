@@ -44,6 +44,14 @@ Readings taken where the pages are silent (each one is listed in the design note
   * tokens_per_expert = kept counts; percentiles = linear interpolation (type 7) over all
     E experts including empty ones; top-5% share = sum of the ceil(0.05 E) largest kept
     counts over the total; dropped_tokens counts dropped (token, expert) assignments.
+  Routing variants ([EP-serving] "Real-world implementation": node-limited routing;
+  "Future": loss-free balancing; [EP-checks] "Top-2 does not insure against hot experts"):
+  * group-limited: experts form n_groups equal contiguous groups, a group's score is its
+    best selection score, a token keeps the topk_groups best groups (equal scores -> lower
+    group index) and picks its k experts among them;
+  * selection-only bias: selection on fp32(z + b), gate weights from the unbiased z;
+  * pick-rank drop order: within an expert, all first picks (token order), then all second
+    picks, and so on.
 
 Every function below is pinned by tests in tests/test_oracle.py against hand-worked
 cases, brute force, closed forms or independent textbook routines.
@@ -59,6 +67,10 @@ SOFTMAX = 0
 SIGMOID = 1
 LAYOUT_COMPACT = 0
 LAYOUT_PADDED = 1
+BIAS_SCORE_AND_WEIGHT = 0
+BIAS_SELECTION_ONLY = 1
+DROP_TOKEN_ORDER = 0
+DROP_PICK_RANK = 1
 
 
 # --------------------------------------------------------------------------------------
@@ -87,18 +99,33 @@ def logits_to_fp32(z64) -> np.ndarray:
 # --------------------------------------------------------------------------------------
 # Top-k selection  [EP-serving, "Deep dive": router picks the top-k experts per token]
 # --------------------------------------------------------------------------------------
-def select_topk(z32, k: int) -> np.ndarray:
-    """idx[t, 0..k-1]: the k experts with the largest fp32 logit, best first; equal
-    logits rank the lower expert index first."""
+def select_topk(z32, k: int, n_groups: int = 0, topk_groups: int = 0) -> np.ndarray:
+    """idx[t, 0..k-1]: the k experts with the largest fp32 score, best first; equal
+    scores rank the lower expert index first.  With n_groups > 1, only the experts of the
+    token's topk_groups best groups (group score = best score in the group, equal group
+    scores -> lower group index) are eligible."""
     z = np.asarray(z32, dtype=np.float32)
     T, E = z.shape
     if not (1 <= k <= E):
         raise ValueError("need 1 <= k <= E")
+    grouped = n_groups > 1
+    if grouped:
+        if E % n_groups or not (1 <= topk_groups <= n_groups) or topk_groups * (E // n_groups) < k:
+            raise ValueError("bad group configuration")
+        gsize = E // n_groups
     idx = np.empty((T, k), dtype=np.int32)
     experts = np.arange(E)
     for t in range(T):
-        # lexsort: last key is primary -> by -z, then by expert index
-        order = np.lexsort((experts, -z[t].astype(np.float64)))
+        zt = z[t].astype(np.float64)
+        eligible = np.ones(E, dtype=bool)
+        if grouped:
+            gscore = zt.reshape(n_groups, gsize).max(axis=1)
+            gorder = np.lexsort((np.arange(n_groups), -gscore))
+            eligible[:] = False
+            for g in gorder[:topk_groups]:
+                eligible[g * gsize:(g + 1) * gsize] = True
+        # lexsort: last key is primary -> eligible first, then by -z, then by expert index
+        order = np.lexsort((experts, -zt, ~eligible))
         idx[t] = order[:k]
     return idx
 
@@ -134,10 +161,13 @@ def capacity(capacity_factor: float, T: int, k: int, E: int) -> Optional[int]:
 # Dispatch bookkeeping  [EP-serving, "Technical insight": expert buffers, drop or pad;
 #                        EP-checks, "Profile all-to-all ...": pack/permute before dispatch]
 # --------------------------------------------------------------------------------------
-def assign(idx, E: int, C: Optional[int], layout: int = LAYOUT_COMPACT) -> Dict[str, np.ndarray]:
+def assign(idx, E: int, C: Optional[int], layout: int = LAYOUT_COMPACT,
+           drop_policy: int = DROP_TOKEN_ORDER) -> Dict[str, np.ndarray]:
     """Walk the assignments in (expert ascending, token ascending) order, which for a
     top-k (distinct experts per token) is the same as walking tokens in order and giving
-    each pick the next free slot of its expert.  Slot pos < C is kept, the rest dropped.
+    each pick the next free slot of its expert.  With drop_policy = DROP_PICK_RANK the walk
+    goes pick rank by pick rank (all first picks in token order, then all second picks...).
+    Slot pos < C is kept, the rest dropped.
 
     Returns routed[E], kept[E], offsets[E+1] (bucket starts), assign_row[T, k]
     (-1 = dropped), token_of_row[rows] (-1 = unused padding row) and rows.
@@ -148,11 +178,14 @@ def assign(idx, E: int, C: Optional[int], layout: int = LAYOUT_COMPACT) -> Dict[
         raise ValueError("PADDED layout needs a finite capacity")
     pos = np.full((T, k), -1, dtype=np.int64)
     next_slot = [0] * E
-    for t in range(T):
-        for j in range(k):
-            e = int(idx[t, j])
-            pos[t, j] = next_slot[e]
-            next_slot[e] += 1
+    if drop_policy == DROP_PICK_RANK:
+        walk = [(t, j) for j in range(k) for t in range(T)]
+    else:
+        walk = [(t, j) for t in range(T) for j in range(k)]
+    for t, j in walk:
+        e = int(idx[t, j])
+        pos[t, j] = next_slot[e]
+        next_slot[e] += 1
     routed = np.array(next_slot, dtype=np.int64)
     kept = routed.copy() if C is None else np.minimum(routed, C)
     offsets = np.zeros(E + 1, dtype=np.int64)
@@ -292,25 +325,43 @@ def load_stats(routed, kept, assign_row, C: Optional[int]) -> dict:
 # --------------------------------------------------------------------------------------
 # Whole layer
 # --------------------------------------------------------------------------------------
-def route(z32, k: int, gating: int, capacity_factor: float, layout: int = LAYOUT_COMPACT):
-    """Everything that follows from the fp32 logits: picks, weights and bookkeeping."""
+def selection_scores(z32, bias=None, bias_mode: int = BIAS_SCORE_AND_WEIGHT) -> np.ndarray:
+    """The fp32 scores the top-k is taken on.  In the default mode the bias is already part
+    of the logits z32; in selection-only mode the score is fp32(z32 + b), one fp32 addition."""
+    z32 = np.asarray(z32, dtype=np.float32)
+    if bias_mode != BIAS_SELECTION_ONLY or bias is None:
+        return z32
+    b = np.asarray(bias, dtype=np.float32)
+    return (z32 + (b[None, :] if b.ndim == 1 else b)).astype(np.float32)
+
+
+def route(z32, k: int, gating: int, capacity_factor: float, layout: int = LAYOUT_COMPACT,
+          n_groups: int = 0, topk_groups: int = 0, bias=None,
+          bias_mode: int = BIAS_SCORE_AND_WEIGHT, drop_policy: int = DROP_TOKEN_ORDER):
+    """Everything that follows from the fp32 logits z32: picks (on the selection scores),
+    weights (on z32) and bookkeeping."""
     z32 = np.asarray(z32, dtype=np.float32)
     T, E = z32.shape
-    idx = select_topk(z32, k)
+    idx = select_topk(selection_scores(z32, bias, bias_mode), k, n_groups, topk_groups)
     w = gate_weights(z32, idx, gating)
     C = capacity(capacity_factor, T, k, E)
-    a = assign(idx, E, C, layout)
+    a = assign(idx, E, C, layout, drop_policy)
     return dict(idx=idx, w=w, C=C, **a)
 
 
 def moe_layer(x, w_router, logit_bias, w_gate, w_up, w_down, k: int, gating: int,
-              capacity_factor: float, layout: int = LAYOUT_COMPACT, z32=None) -> dict:
+              capacity_factor: float, layout: int = LAYOUT_COMPACT, z32=None,
+              n_groups: int = 0, topk_groups: int = 0, bias_mode: int = BIAS_SCORE_AND_WEIGHT,
+              drop_policy: int = DROP_TOKEN_ORDER) -> dict:
     """The whole forward on small inputs.  If z32 is given, routing starts from those fp32
-    logits (the parity protocol); otherwise from fp32(z64)."""
-    z64 = router_logits(x, w_router, logit_bias)
+    logits (the parity protocol); otherwise from fp32(z64).  In selection-only bias mode
+    the logits carry no bias and the bias only shifts the selection scores."""
+    sel_only = bias_mode == BIAS_SELECTION_ONLY
+    z64 = router_logits(x, w_router, None if sel_only else logit_bias)
     if z32 is None:
         z32 = logits_to_fp32(z64)
-    r = route(z32, k, gating, capacity_factor, layout)
+    r = route(z32, k, gating, capacity_factor, layout, n_groups, topk_groups,
+              logit_bias if sel_only else None, bias_mode, drop_policy)
     x_perm = permute(x, r["token_of_row"])
 
     def weights_of(e):

@@ -19,6 +19,8 @@ from ._abi import MoEError, MoeConfig, MoeLayerBuffers, MoeLayerInputs, MoeLoadS
 SOFTMAX, SIGMOID = 0, 1
 COMPACT, PADDED = 0, 1
 F32, BF16 = 0, 1
+BIAS_SCORE_AND_WEIGHT, BIAS_SELECTION_ONLY = 0, 1
+DROP_TOKEN_ORDER, DROP_PICK_RANK = 0, 1
 
 __all__ = ["MoEError", "make_config", "workspace_size", "capacity", "max_rows",
            "alloc_workspace", "moe_route", "moe_dispatch", "moe_dispatch_static_scratch",
@@ -48,16 +50,19 @@ def _stream(stream) -> Optional[int]:
 
 
 def make_config(T: int, d_model: int, d_ff: int, E: int, k: int, gating: int = SOFTMAX,
-                capacity_factor: float = 0.0, layout: int = COMPACT,
-                dtype: int = BF16) -> MoeConfig:
+                capacity_factor: float = 0.0, layout: int = COMPACT, dtype: int = BF16,
+                n_groups: int = 0, topk_groups: int = 0, bias_mode: int = BIAS_SCORE_AND_WEIGHT,
+                drop_policy: int = DROP_TOKEN_ORDER) -> MoeConfig:
     return MoeConfig(T=T, d_model=d_model, d_ff=d_ff, E=E, k=k, gating=gating, layout=layout,
-                     dtype=dtype, capacity_factor=capacity_factor)
+                     dtype=dtype, capacity_factor=capacity_factor, n_groups=n_groups,
+                     topk_groups=topk_groups, bias_mode=bias_mode, drop_policy=drop_policy)
 
 
 def config_from_shape(shape) -> MoeConfig:
     """moe_config_t for a workload.MoEShape."""
     return make_config(shape.T, shape.d_model, shape.d_ff, shape.E, shape.k, shape.gating,
-                       shape.capacity_factor, shape.layout, shape.dtype)
+                       shape.capacity_factor, shape.layout, shape.dtype, shape.n_groups,
+                       shape.topk_groups, shape.bias_mode, shape.drop_policy)
 
 
 def workspace_size(cfg: MoeConfig) -> int:

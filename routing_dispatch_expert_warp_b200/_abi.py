@@ -25,7 +25,8 @@ c_vp, c_sz = ctypes.c_void_p, ctypes.c_size_t
 class MoeConfig(ctypes.Structure):
     _fields_ = [("T", c_i64), ("d_model", c_i64), ("d_ff", c_i64), ("E", c_i32), ("k", c_i32),
                 ("gating", c_i32), ("layout", c_i32), ("dtype", c_i32),
-                ("capacity_factor", c_f32)]
+                ("capacity_factor", c_f32), ("n_groups", c_i32), ("topk_groups", c_i32),
+                ("bias_mode", c_i32), ("drop_policy", c_i32)]
 
 
 class MoeLoadStats(ctypes.Structure):

@@ -53,6 +53,10 @@ class MoEShape:
     zipf_beta: float = 0.11  # fitted: routed max/mean 2.96 on the 16384-token DeepSeek-shaped prefill
     chunk_bias_std: float = 0.5
     n_decode_tokens: int = 64
+    n_groups: int = 0          # group-limited routing (0: off)
+    topk_groups: int = 0
+    bias_mode: int = 0         # 0: bias in score and weights; 1: selection only
+    drop_policy: int = 0       # 0: token order; 1: pick rank first
 
     def replace(self, **kw) -> "MoEShape":
         return dataclasses.replace(self, **kw)

@@ -334,3 +334,93 @@ def test_stats_top5_counts_experts():
     s = O.load_stats(kept, kept, -np.ones((3, 2), dtype=np.int64), 0)
     assert s["top5pct_share"] == 0.0 and s["max_to_mean"] == 0.0
     assert s["tokens_fully_dropped"] == 3 and s["dropped_by_rank"] == [3, 3]
+
+
+# ---------------------------------------------------------------- routing variants
+def test_group_limited_hand_case():
+    # 8 experts in 4 groups of 2: {0,1} {2,3} {4,5} {6,7}
+    z = np.array([[5.0, 4.9, 0.0, 0.0, 4.95, 0.0, 4.8, 4.7]], dtype=np.float32)
+    assert O.select_topk(z, 2).tolist() == [[0, 4]]                     # no group limit
+    assert O.select_topk(z, 2, n_groups=4, topk_groups=1).tolist() == [[0, 1]]
+    # groups 0 (5.0) and 2 (4.95) survive; group 3 (4.8) is out
+    assert O.select_topk(z, 3, n_groups=4, topk_groups=2).tolist() == [[0, 4, 1]]
+    # equal group scores -> lower group index
+    z2 = np.array([[1.0, 0.0, 1.0, 0.5, 0.0, 0.0]], dtype=np.float32)
+    assert O.select_topk(z2, 2, n_groups=3, topk_groups=1).tolist() == [[0, 1]]
+    with pytest.raises(ValueError):
+        O.select_topk(z, 3, n_groups=4, topk_groups=1)   # 1 group of 2 cannot hold 3 picks
+
+
+@pytest.mark.parametrize("E,G,M,k", [(8, 4, 2, 2), (12, 3, 2, 4), (16, 8, 3, 3), (6, 2, 1, 3)])
+def test_group_limited_brute_force(E, G, M, k):
+    rng = np.random.default_rng(E + G + M + k)
+    gs = E // G
+    beats = lambda a, b, i, j: a > b or (a == b and i < j)
+    for trial in range(30):
+        z = (rng.integers(-2, 3, size=E) if trial % 2 else rng.standard_normal(E)).astype(np.float32)
+        idx = O.select_topk(z[None], k, G, M)[0].tolist()
+        gscore = [max(z[g * gs:(g + 1) * gs]) for g in range(G)]
+        # the chosen groups: every chosen group beats every other group
+        chosen = [g for g in range(G)
+                  if sum(beats(gscore[h], gscore[g], h, g) for h in range(G) if h != g) < M]
+        assert len(chosen) == M
+        allowed = [e for e in range(E) if e // gs in chosen]
+        sub = [float(z[e]) for e in allowed]
+        want = [allowed[i] for i in _brute_topk(sub, k)]
+        assert idx == want
+
+
+def test_selection_only_bias_hand_case():
+    z = np.array([[1.0, 2.0, 3.0]], dtype=np.float32)
+    b = np.array([3.0, 0.0, 0.0], dtype=np.float32)
+    r = O.route(z, 2, O.SOFTMAX, 0.0, bias=b, bias_mode=O.BIAS_SELECTION_ONLY)
+    assert r["idx"].tolist() == [[0, 2]]          # scores 4, 2, 3
+    e1, e3 = math.exp(1.0), math.exp(3.0)        # weights from the unbiased logits 1 and 3
+    np.testing.assert_allclose(r["w"][0], [e1 / (e1 + e3), e3 / (e1 + e3)], rtol=0, atol=1e-15)
+    # in the default mode the bias is already inside the logits: nothing added again
+    r0 = O.route(z, 2, O.SOFTMAX, 0.0, bias=b, bias_mode=O.BIAS_SCORE_AND_WEIGHT)
+    assert r0["idx"].tolist() == [[2, 1]]
+
+
+def test_selection_only_bias_is_one_fp32_addition():
+    z = np.array([[1.0, 1.0 + 2.0 ** -23]], dtype=np.float32)
+    b = np.array([2.0 ** -24, 0.0], dtype=np.float32)    # 1 + 2^-24 rounds back to 1 in fp32
+    s = O.selection_scores(z, b, O.BIAS_SELECTION_ONLY)
+    assert s.dtype == np.float32 and s[0].tolist() == [1.0, 1.0 + 2.0 ** -23]
+    assert O.select_topk(s, 1).tolist() == [[1]]
+
+
+def test_pick_rank_drop_order_hand_case():
+    idx = np.array([[0, 1], [1, 0], [0, 1]])
+    tok = O.assign(idx, 2, 2, drop_policy=O.DROP_TOKEN_ORDER)
+    rank = O.assign(idx, 2, 2, drop_policy=O.DROP_PICK_RANK)
+    # expert 0 slots, token order: t0.j0, t1.j1, t2.j0 -> t2's first pick dropped
+    assert tok["assign_row"].tolist() == [[0, 2], [3, 1], [-1, -1]]
+    # pick rank: first picks t0->e0 s0, t1->e1 s0, t2->e0 s1; then second picks
+    # t0->e1 s1, t1->e0 s2 (dropped), t2->e1 s2 (dropped); rows = offset (0 or 2) + slot
+    assert rank["assign_row"].tolist() == [[0, 3], [2, -1], [1, -1]]
+    assert rank["kept"].tolist() == [2, 2] and rank["routed"].tolist() == [3, 3]
+
+
+@pytest.mark.parametrize("T,E,k,cf", [(60, 6, 2, 0.8), (45, 8, 3, 1.0), (30, 4, 4, 0.5)])
+def test_pick_rank_slots_match_stable_sort(T, E, k, cf):
+    rng = np.random.default_rng(T * k)
+    z = rng.standard_normal((T, E)).astype(np.float32)
+    z[:, 1] += 1.5
+    idx = O.select_topk(z, k)
+    C = O.capacity(cf, T, k, E)
+    a = O.assign(idx, E, C, drop_policy=O.DROP_PICK_RANK)
+    flat_e = idx.ravel().astype(np.int64)
+    flat_t = np.repeat(np.arange(T), k)
+    flat_j = np.tile(np.arange(k), T)
+    order = np.argsort(flat_e * (k * T) + flat_j * T + flat_t, kind="stable")
+    start = np.concatenate([[0], np.cumsum(np.bincount(flat_e, minlength=E))])
+    slot = np.empty(T * k, dtype=np.int64)
+    slot[order] = np.arange(T * k) - start[flat_e[order]]
+    assert a["slot"].ravel().tolist() == slot.tolist()
+    # no later pick is kept while an earlier-ranked pick to the same expert was dropped
+    for e in range(E):
+        for j in range(1, k):
+            later_kept = ((idx[:, j] == e) & (a["assign_row"][:, j] >= 0)).any()
+            earlier_dropped = ((idx[:, :j] == e) & (a["assign_row"][:, :j] < 0)).any()
+            assert not (later_kept and earlier_dropped)
