@@ -248,8 +248,9 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
  * 1 MiB + 256 B array in device memory, which every GPU that loads this library keeps
  * until the process exits; the call allocates nothing (no cudaMalloc, no cudaFree, no
  * allocating library routine).  Limits and behaviour:
- *   - ceil(T/256) * E * 4 bytes must fit in 1 MiB (e.g. T <= 262144 at E = 256); larger
- *     sizes return MOE_ERR_UNSUPPORTED with a message, before anything is enqueued.
+ *   - ceil(T/256) * E * 4 bytes (times k with MOE_DROP_PICK_RANK) must fit in 1 MiB (e.g.
+ *     T <= 262144 at E = 256); larger sizes return MOE_ERR_UNSUPPORTED with a message,
+ *     before anything is enqueued.
  *   - The first call on each device looks up the array's device address with that device
  *     current; make that first call before any stream capture.
  *   - Every call shares the one array: two calls that run on the GPU at the same time

@@ -56,6 +56,21 @@ moe_status_t check_config(const moe_config_t* cfg, Shape* s) {
     return fail(MOE_ERR_INVALID_ARG, "unknown dtype %d", cfg->dtype);
   if (!(cfg->capacity_factor == cfg->capacity_factor))
     return fail(MOE_ERR_INVALID_ARG, "capacity_factor is NaN");
+  if (cfg->n_groups > 1) {
+    if (cfg->E % cfg->n_groups != 0)
+      return fail(MOE_ERR_INVALID_ARG, "E (%d) must be a multiple of n_groups (%d)", cfg->E,
+                  cfg->n_groups);
+    if (cfg->topk_groups < 1 || cfg->topk_groups > cfg->n_groups ||
+        static_cast<int64_t>(cfg->topk_groups) * (cfg->E / cfg->n_groups) < cfg->k)
+      return fail(MOE_ERR_INVALID_ARG,
+                  "topk_groups must be in [1, n_groups] and hold at least k experts");
+  } else if (cfg->n_groups < 0) {
+    return fail(MOE_ERR_INVALID_ARG, "n_groups must be >= 0");
+  }
+  if (cfg->bias_mode != MOE_BIAS_SCORE_AND_WEIGHT && cfg->bias_mode != MOE_BIAS_SELECTION_ONLY)
+    return fail(MOE_ERR_INVALID_ARG, "unknown bias_mode %d", cfg->bias_mode);
+  if (cfg->drop_policy != MOE_DROP_TOKEN_ORDER && cfg->drop_policy != MOE_DROP_PICK_RANK)
+    return fail(MOE_ERR_INVALID_ARG, "unknown drop_policy %d", cfg->drop_policy);
   s->T = cfg->T;
   s->d = cfg->d_model;
   s->f = cfg->d_ff;
@@ -64,6 +79,10 @@ moe_status_t check_config(const moe_config_t* cfg, Shape* s) {
   s->gating = cfg->gating;
   s->layout = cfg->layout;
   s->dtype = cfg->dtype;
+  s->n_groups = cfg->n_groups > 1 ? cfg->n_groups : 0;
+  s->topk_groups = cfg->n_groups > 1 ? cfg->topk_groups : 0;
+  s->bias_mode = cfg->bias_mode;
+  s->drop_policy = cfg->drop_policy;
   s->elem = cfg->dtype == MOE_F32 ? 4 : 2;
   const int64_t A = cfg->T * cfg->k;
   if (cfg->capacity_factor > 0.0f) {
@@ -115,7 +134,7 @@ WsLayout workspace_layout(const Shape& s) {
   l.status = off;
   off += round_up(sizeof(DevStatus));
   l.hist = off;
-  l.hist_bytes = round_up(static_cast<size_t>(dispatch_blocks(s.T)) * s.E * sizeof(int32_t));
+  l.hist_bytes = round_up(dispatch_hist_bytes(s));
   off += l.hist_bytes;
   l.logits = off;
   l.logits_bytes = round_up(static_cast<size_t>(s.T) * s.E * sizeof(float));
@@ -237,7 +256,7 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
   MOE_REQUIRE(bias_row_stride == 0 || bias_row_stride >= s.E,
               "moe_route: bias_row_stride must be 0 or >= E");
   float* z = logits;
-  if (z == nullptr && s.E > 32) z = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + lay.logits);
+  if (z == nullptr) z = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + lay.logits);
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   if (router_uses_tensor_cores(s)) {
     const char* why = "";
@@ -292,11 +311,12 @@ moe_status_t moe_dispatch_static_scratch(const moe_config_t* cfg, const void* x,
               "moe_dispatch_static_scratch: NULL pointer");
   MOE_REQUIRE(aligned16(x) && aligned16(x_perm),
               "moe_dispatch_static_scratch: x and x_perm must be 16-byte aligned");
-  const size_t need = static_cast<size_t>(dispatch_blocks(s.T)) * s.E * sizeof(int32_t);
+  const size_t need = dispatch_hist_bytes(s);
   if (need > kStaticDispatchHistBytes)
     return fail(MOE_ERR_UNSUPPORTED,
-                "moe_dispatch_static_scratch: ceil(T/%d)*E*4 = %zu bytes of scratch needed, the "
-                "fixed scratch holds %zu (use moe_dispatch with a workspace)",
+                "moe_dispatch_static_scratch: ceil(T/%d)*E*4 bytes (times k for pick-rank drops) "
+                "= %zu bytes of scratch needed, the fixed scratch holds %zu (use moe_dispatch "
+                "with a workspace)",
                 kDispatchBlockTokens, need, kStaticDispatchHistBytes);
   cudaError_t err = dispatch_static_scratch(s, x, topk_idx, routed_counts, kept_counts,
                                             expert_offsets, assign_row, token_of_row, x_perm,

@@ -31,10 +31,12 @@ namespace {
 
 constexpr int kWarps = kDispatchBlockTokens / 32;
 
-// Fill masks[w][e] for the block's tokens.  Returns nothing; invalid experts are recorded.
+// Fill masks[w][e] for the block's tokens, counting the picks of `plane` only when the
+// assignments are ranked pick rank by pick rank (planes == k), all picks otherwise
+// (planes == 1).  Invalid experts are recorded and skipped.
 __device__ __forceinline__ void build_masks(const int32_t* __restrict__ topk_idx, int64_t T,
                                             int k, int E, uint32_t (*masks)[MOE_MAX_EXPERTS],
-                                            DevStatus* status) {
+                                            DevStatus* status, int plane, int planes) {
   for (int i = threadIdx.x; i < kWarps * MOE_MAX_EXPERTS; i += blockDim.x)
     (&masks[0][0])[i] = 0u;
   __syncthreads();
@@ -43,6 +45,7 @@ __device__ __forceinline__ void build_masks(const int32_t* __restrict__ topk_idx
   const uint32_t bit = 1u << (threadIdx.x & 31);
   if (t < T) {
     for (int j = 0; j < k; ++j) {
+      if (planes > 1 && j != plane) continue;
       const int e = topk_idx[t * k + j];
       if (e < 0 || e >= E) {
         record_error(status, DEV_BAD_EXPERT, 1, static_cast<unsigned long long>(t * k + j));
@@ -54,56 +57,67 @@ __device__ __forceinline__ void build_masks(const int32_t* __restrict__ topk_idx
   __syncthreads();
 }
 
+// hist[b][p][e]: assignments of plane p (a pick rank, or all picks) from block b to expert e.
 __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_count_kernel(
-    const int32_t* __restrict__ topk_idx, int64_t T, int k, int E, int32_t* __restrict__ hist,
-    DevStatus* status) {
+    const int32_t* __restrict__ topk_idx, int64_t T, int k, int E, int planes,
+    int32_t* __restrict__ hist, DevStatus* status) {
   __shared__ uint32_t masks[kWarps][MOE_MAX_EXPERTS];
-  build_masks(topk_idx, T, k, E, masks, status);
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int c = 0;
+  for (int p = 0; p < planes; ++p) {
+    build_masks(topk_idx, T, k, E, masks, p == 0 ? status : nullptr, p, planes);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      int c = 0;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) c += __popc(masks[w][e]);
-    hist[static_cast<int64_t>(blockIdx.x) * E + e] = c;
+      for (int w = 0; w < kWarps; ++w) c += __popc(masks[w][e]);
+      hist[(static_cast<int64_t>(blockIdx.x) * planes + p) * E + e] = c;
+    }
+    __syncthreads();  // masks are rebuilt for the next plane
   }
 }
 
 // Ranking.  Every block first derives what it needs from the per-block counts of all
-// blocks: thread e adds up expert e's counts over the blocks (routed total, and the part
-// that comes from blocks before this one), caps the total at C (kept), and the block scans
-// kept over the experts (bucket offsets).  Block 0 publishes routed / kept / offsets; the
-// others only use them.  Then slot = base from earlier blocks + earlier warps of this block
-// + popcount(mask & lanes below me), kept iff slot < C, row = offset + slot.  Finally the
+// blocks: thread e adds up expert e's counts per plane over the blocks (plane totals, and
+// the part that comes from blocks before this one), caps the routed total at C (kept), and
+// the block scans kept over the experts (bucket offsets).  Block 0 publishes routed / kept /
+// offsets; the others only use them.  A plane is all picks (token-order drops) or one pick
+// rank (pick-rank drops: plane p starts after the totals of planes < p).  Then, plane by
+// plane, slot = plane start + base from earlier blocks + earlier warps of this block +
+// popcount(mask & lanes below me), kept iff slot < C, row = offset + slot.  Finally the
 // rows no assignment uses are marked -1 in token_of_row.
 __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
     const int32_t* __restrict__ topk_idx, int64_t T, int k, int E, int64_t C, int layout,
-    int64_t nblk, const int32_t* __restrict__ hist, int32_t* __restrict__ routed,
+    int planes, int64_t nblk, const int32_t* __restrict__ hist, int32_t* __restrict__ routed,
     int32_t* __restrict__ kept, int32_t* __restrict__ offsets, int32_t* __restrict__ assign_row,
     int32_t* __restrict__ token_of_row, int64_t max_rows) {
   static_assert(kDispatchBlockTokens == MOE_MAX_EXPERTS, "one thread per expert");
   __shared__ uint32_t masks[kWarps][MOE_MAX_EXPERTS];
   __shared__ int32_t wbase[kWarps][MOE_MAX_EXPERTS];
+  __shared__ int32_t pbase[MOE_MAX_TOPK][MOE_MAX_EXPERTS];  // plane start + earlier blocks
   __shared__ int32_t off_s[MOE_MAX_EXPERTS];
   __shared__ int32_t kept_s[MOE_MAX_EXPERTS];
   __shared__ int64_t scan[MOE_MAX_EXPERTS];
-  build_masks(topk_idx, T, k, E, masks, nullptr);
 
   const int e = threadIdx.x;
-  int64_t run = 0, before = 0;
+  int64_t run = 0;  // routed total over all planes
   if (e < E) {
-    int64_t b = 0;
-    for (; b + 8 <= nblk; b += 8) {  // loads issued 8 at a time, sums in block order
-      int32_t c[8];
+    for (int p = 0; p < planes; ++p) {
+      int64_t tot = 0, before = 0;
+      int64_t b = 0;
+      for (; b + 8 <= nblk; b += 8) {  // loads issued 8 at a time, sums in block order
+        int32_t c[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) c[u] = __ldg(hist + (b + u) * E + e);
+        for (int u = 0; u < 8; ++u) c[u] = __ldg(hist + ((b + u) * planes + p) * E + e);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (b + u == blockIdx.x) before = run;
-        run += c[u];
+        for (int u = 0; u < 8; ++u) {
+          if (b + u == blockIdx.x) before = tot;
+          tot += c[u];
+        }
       }
-    }
-    for (; b < nblk; ++b) {
-      if (b == blockIdx.x) before = run;
-      run += __ldg(hist + b * E + e);
+      for (; b < nblk; ++b) {
+        if (b == blockIdx.x) before = tot;
+        tot += __ldg(hist + (b * planes + p) * E + e);
+      }
+      pbase[p][e] = static_cast<int32_t>(run + before);
+      run += tot;
     }
   }
   const int64_t kp = (e < E) ? ((C >= 0 && run > C) ? C : run) : 0;
@@ -121,12 +135,6 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
         layout == MOE_LAYOUT_PADDED ? static_cast<int64_t>(e) * C : scan[e] - kp;
     off_s[e] = static_cast<int32_t>(off);
     kept_s[e] = static_cast<int32_t>(kp);
-    int32_t wb = static_cast<int32_t>(before);
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      wbase[w][e] = wb;
-      wb += __popc(masks[w][e]);
-    }
     if (blockIdx.x == 0) {
       routed[e] = static_cast<int32_t>(run);
       kept[e] = static_cast<int32_t>(kp);
@@ -137,23 +145,36 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
                                               : total_kept);
     }
   }
-  __syncthreads();
 
   const int64_t t = static_cast<int64_t>(blockIdx.x) * kDispatchBlockTokens + threadIdx.x;
-  if (t < T) {
-    const int w = threadIdx.x >> 5;
-    const uint32_t below = (1u << (threadIdx.x & 31)) - 1u;
-    for (int j = 0; j < k; ++j) {
-      const int ee = topk_idx[t * k + j];
-      int32_t row = -1;
-      if (ee >= 0 && ee < E) {
-        const int64_t slot = wbase[w][ee] + __popc(masks[w][ee] & below);
-        if (C < 0 || slot < C) {
-          row = off_s[ee] + static_cast<int32_t>(slot);
-          token_of_row[row] = static_cast<int32_t>(t);
-        }
+  const int w = threadIdx.x >> 5;
+  const uint32_t below = (1u << (threadIdx.x & 31)) - 1u;
+  for (int p = 0; p < planes; ++p) {
+    __syncthreads();  // pbase / off_s ready; masks of the previous plane no longer read
+    build_masks(topk_idx, T, k, E, masks, nullptr, p, planes);
+    if (e < E) {
+      int32_t wb = pbase[p][e];
+#pragma unroll
+      for (int ww = 0; ww < kWarps; ++ww) {
+        wbase[ww][e] = wb;
+        wb += __popc(masks[ww][e]);
       }
-      assign_row[t * k + j] = row;
+    }
+    __syncthreads();
+    if (t < T) {
+      for (int j = 0; j < k; ++j) {
+        if (planes > 1 && j != p) continue;
+        const int ee = topk_idx[t * k + j];
+        int32_t row = -1;
+        if (ee >= 0 && ee < E) {
+          const int64_t slot = wbase[w][ee] + __popc(masks[w][ee] & below);
+          if (C < 0 || slot < C) {
+            row = off_s[ee] + static_cast<int32_t>(slot);
+            token_of_row[row] = static_cast<int32_t>(t);
+          }
+        }
+        assign_row[t * k + j] = row;
+      }
     }
   }
 
@@ -162,8 +183,8 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
   const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (layout == MOE_LAYOUT_PADDED) {
     for (int64_t r = first; r < max_rows; r += stride) {
-      const int64_t ee = r / C;
-      if (ee < E && r - ee * C >= kept_s[ee]) token_of_row[r] = -1;
+      const int64_t eb = r / C;
+      if (eb < E && r - eb * C >= kept_s[eb]) token_of_row[r] = -1;
     }
   } else {
     for (int64_t r = total_kept + first; r < max_rows; r += stride) token_of_row[r] = -1;
@@ -264,12 +285,13 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
                             cudaStream_t st) {
   const int64_t nblk = dispatch_blocks(s.T);
   cudaError_t err;
+  const int planes = dispatch_planes(s);
   dispatch_count_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
-      topk_idx, s.T, s.k, s.E, hist, status);
+      topk_idx, s.T, s.k, s.E, planes, hist, status);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   dispatch_rank_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
-      topk_idx, s.T, s.k, s.E, s.C, s.layout, nblk, hist, routed, kept, offsets, assign_row,
-      token_of_row, s.max_rows);
+      topk_idx, s.T, s.k, s.E, s.C, s.layout, planes, nblk, hist, routed, kept, offsets,
+      assign_row, token_of_row, s.max_rows);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
 
   const int64_t row_bytes = s.d * s.elem;

@@ -532,7 +532,8 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_route
   p.N_out = s.E;
   p.mb_outer = 1;
   p.out_f32 = logits;
-  p.bias = bias;
+  // logits carry the bias unless it is for selection only (then the top-k adds it)
+  p.bias = s.bias_mode == MOE_BIAS_SELECTION_ONLY ? nullptr : bias;
   p.bias_stride = bias_stride;
   p.status = status;
   p.wait_ns = wait_ns;
@@ -541,7 +542,7 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_route
   grouped_gemm_tc_kernel<MODE_ROUTER><<<static_cast<unsigned>(g), THREADS, DYN_SMEM, st>>>(
       ta, th, tl, p);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  return launch_topk_from_logits(s, logits, topk_idx, topk_w, st);
+  return launch_topk_from_logits(s, logits, bias, bias_stride, topk_idx, topk_w, st);
 }
 
 }  // namespace moe

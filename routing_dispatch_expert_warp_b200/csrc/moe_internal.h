@@ -19,6 +19,7 @@ constexpr size_t kWsAlign = 256;
 struct Shape {
   int64_t T, d, f;
   int E, k, gating, layout, dtype;
+  int n_groups, topk_groups, bias_mode, drop_policy;
   int64_t C;         // capacity, -1 when dropless
   int64_t max_rows;  // rows of x_perm / h / y_perm / token_of_row
   int64_t elem;      // bytes per element of x, weights and activations
@@ -27,7 +28,7 @@ struct Shape {
 // Offsets (bytes) of the workspace sections.
 struct WsLayout {
   size_t status;        // DevStatus, 256 B
-  size_t hist;          // [n_dispatch_blocks, E] int32 per-block counts, then bases
+  size_t hist;          // [n_dispatch_blocks, planes, E] int32 per-block counts
   size_t hist_bytes;
   size_t logits;        // [T, E] fp32 logits when the caller passes none
   size_t logits_bytes;
@@ -40,6 +41,14 @@ struct WsLayout {
 
 inline int64_t dispatch_blocks(int64_t T) {
   return (T + kDispatchBlockTokens - 1) / kDispatchBlockTokens;
+}
+// Count planes of dispatch: one per pick rank when drops go by pick rank, else one.
+inline int dispatch_planes(const Shape& s) {
+  return s.drop_policy == MOE_DROP_PICK_RANK ? s.k : 1;
+}
+// Bytes of per-block expert counts dispatch needs.
+inline size_t dispatch_hist_bytes(const Shape& s) {
+  return static_cast<size_t>(dispatch_blocks(s.T)) * dispatch_planes(s) * s.E * sizeof(int32_t);
 }
 WsLayout workspace_layout(const Shape& s);
 
@@ -60,8 +69,9 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_route
                              DevStatus* status, uint64_t wait_ns, cudaStream_t st,
                              const char** why);
 size_t router_tc_workspace_bytes(const Shape& s);
-cudaError_t launch_topk_from_logits(const Shape& s, const float* logits, int32_t* topk_idx,
-                                    float* topk_w, cudaStream_t st);
+cudaError_t launch_topk_from_logits(const Shape& s, const float* logits, const float* bias,
+                                    int64_t bias_stride, int32_t* topk_idx, float* topk_w,
+                                    cudaStream_t st);
 cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_idx,
                             int32_t* routed, int32_t* kept, int32_t* offsets,
                             int32_t* assign_row, int32_t* token_of_row, void* x_perm,

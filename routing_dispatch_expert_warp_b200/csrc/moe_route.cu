@@ -56,7 +56,8 @@ __device__ __forceinline__ bool better(bool va, float a, int ia, bool vb, float 
 __device__ __forceinline__ void gate_weights(const float* zsel, int k, int gating, float* w) {
   float s = 0.f;
   if (gating == MOE_GATE_SOFTMAX) {
-    const float m = zsel[0];
+    float m = zsel[0];  // the picks are ordered by selection score, not necessarily by z
+    for (int j = 1; j < k; ++j) m = fmaxf(m, zsel[j]);
     for (int j = 0; j < k; ++j) {
       w[j] = expf(zsel[j] - m);
       s += w[j];
@@ -179,8 +180,8 @@ __global__ void __launch_bounds__(256) router_weight_lanes_kernel(const float* _
 template <typename TX, int ET>
 __global__ void __launch_bounds__(256, ET == 8 ? 2 : 3) router_small_e_kernel(
     const TX* __restrict__ x, const float4* __restrict__ wl, const float* __restrict__ bias,
-    int64_t bias_stride, int64_t T, int d, int E, int k, int gating, float* __restrict__ logits,
-    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+    int64_t bias_stride, int64_t T, int d, int E, int k, int gating, int bias_mode,
+    float* __restrict__ logits, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
   constexpr int TW = 32 / ET;  // tokens per block
   constexpr int NW = 8;        // warps per block
   constexpr int CPW = sizeof(TX) == 2 ? 2 : 1;  // chunks whose x loads are in flight together
@@ -255,8 +256,17 @@ __global__ void __launch_bounds__(256, ET == 8 ? 2 : 3) router_small_e_kernel(
       const int e = lane % ET;
       const int64_t t = t0 + tw;
       const bool valid = (e < E) && (t < T);
+      float key = z;  // selection score
       if (valid) {
-        if (bias != nullptr) z += bias[t * bias_stride + e];
+        if (bias != nullptr) {
+          const float b = bias[t * bias_stride + e];
+          if (bias_mode == MOE_BIAS_SELECTION_ONLY) {
+            key = z + b;
+          } else {
+            z += b;
+            key = z;
+          }
+        }
         if (logits != nullptr) logits[t * E + e] = z;
       }
       // top-k within each group of ET lanes (one token per group)
@@ -265,15 +275,16 @@ __global__ void __launch_bounds__(256, ET == 8 ? 2 : 3) router_small_e_kernel(
       int isel[MOE_MAX_TOPK];
       for (int j = 0; j < k; ++j) {
         bool bv = valid && !taken;
-        float bz = z;
+        float bk = key, bz = z;
         int bi = e;
 #pragma unroll
         for (int off = ET / 2; off >= 1; off >>= 1) {
           const bool ov = __shfl_xor_sync(0xffffffffu, bv, off);
+          const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
           const float oz = __shfl_xor_sync(0xffffffffu, bz, off);
           const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-          if (better(ov, oz, oi, bv, bz, bi)) {
-            bv = ov; bz = oz; bi = oi;
+          if (better(ov, ok, oi, bv, bk, bi)) {
+            bv = ov; bk = ok; bz = oz; bi = oi;
           }
         }
         if (bi == e) taken = true;
@@ -387,65 +398,129 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(
 }
 
 // A warp per token: the top-k of z[t, 0..E) (E <= 256, up to 8 values per lane).
-// With nsplit > 1, z holds nsplit partial sums per logit (split-K); they are added in split
-// order with the bias and the result is written to `logits`.
+// A warp per token (E <= 256, lane holds experts lane + 32 q).  z holds nsplit partial sums
+// per logit (split-K) that are added in split order; `bias_into_z` adds the bias to them
+// (logits with bias), `bias_into_key` adds it to the selection score only.  The summed
+// logits are written to `logits` when nsplit > 1.  With n_groups > 1, the token first keeps
+// its topk_groups best expert groups (group score = best score in the group).
 __global__ void __launch_bounds__(256) topk_from_logits_kernel(
     const float* __restrict__ z, int nsplit, const float* __restrict__ bias, int64_t bias_stride,
-    float* __restrict__ logits, int64_t T, int E, int k, int gating,
-    int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+    int bias_into_z, int bias_into_key, float* __restrict__ logits, int64_t T, int E, int k,
+    int gating, int n_groups, int topk_groups, int32_t* __restrict__ topk_idx,
+    float* __restrict__ topk_w) {
+  __shared__ float gscore_s[8][MOE_MAX_EXPERTS];
   const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int gsize = n_groups > 1 ? E / n_groups : E;
   for (int64_t t = warp; t < T; t += nwarps) {
-    float zv[8];
+    float zv[8], key[8];
     bool live[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const int e = lane + 32 * q;
       live[q] = e < E;
-      if (!live[q]) {
-        zv[q] = 0.f;
-      } else if (nsplit == 1) {
-        zv[q] = z[t * E + e];
-      } else {
-        // loads in batches of 8 (independent), additions strictly in split order
-        const float* zp = z + t * E + e;
-        const int64_t stride = T * E;
-        float acc = zp[0];
-        int sp = 1;
-        for (; sp + 8 <= nsplit; sp += 8) {
-          float b[8];
+      float acc = 0.f;
+      if (live[q]) {
+        if (nsplit == 1) {
+          acc = z[t * E + e];
+        } else {
+          // loads issued 8 at a time, additions strictly in split order
+          const float* zp = z + t * E + e;
+          const int64_t stride = T * E;
+          acc = zp[0];
+          int sp = 1;
+          for (; sp + 8 <= nsplit; sp += 8) {
+            float b8[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) b[u] = zp[(sp + u) * stride];
+            for (int u = 0; u < 8; ++u) b8[u] = zp[(sp + u) * stride];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) acc += b[u];
+            for (int u = 0; u < 8; ++u) acc += b8[u];
+          }
+          for (; sp < nsplit; ++sp) acc += zp[sp * stride];
         }
-        for (; sp < nsplit; ++sp) acc += zp[sp * stride];
-        if (bias != nullptr) acc += bias[t * bias_stride + e];
-        if (logits != nullptr) logits[t * E + e] = acc;
-        zv[q] = acc;
+        if (bias != nullptr && bias_into_z) acc += bias[t * bias_stride + e];
+        if (nsplit > 1 && logits != nullptr) logits[t * E + e] = acc;
       }
+      zv[q] = acc;
+      key[q] = (live[q] && bias != nullptr && bias_into_key) ? acc + bias[t * bias_stride + e]
+                                                             : acc;
+    }
+    if (n_groups > 1) {
+      // group scores through shared memory, then topk_groups rounds of a warp argmax
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (live[q]) gscore_s[wib][lane + 32 * q] = key[q];
+      __syncwarp();
+      float gs[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const int g = lane + 32 * q;
+        float m = -INFINITY;
+        if (g < n_groups)
+          for (int i = 0; i < gsize; ++i) m = fmaxf(m, gscore_s[wib][g * gsize + i]);
+        gs[q] = m;
+      }
+      __syncwarp();
+      uint32_t chosen = 0;  // bit q: group lane + 32 q kept
+      for (int r = 0; r < topk_groups; ++r) {
+        bool bv = false;
+        float bz = 0.f;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int g = lane + 32 * q;
+          const bool ok = g < n_groups && !((chosen >> q) & 1u);
+          if (better(ok, gs[q], g, bv, bz, bi)) {
+            bv = ok; bz = gs[q]; bi = g;
+          }
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) {
+          const bool ov = __shfl_xor_sync(0xffffffffu, bv, off);
+          const float oz = __shfl_xor_sync(0xffffffffu, bz, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+          if (better(ov, oz, oi, bv, bz, bi)) {
+            bv = ov; bz = oz; bi = oi;
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (lane + 32 * q == bi) chosen |= 1u << q;
+      }
+      // publish the chosen groups, then keep only their experts
+      uint32_t* flags = reinterpret_cast<uint32_t*>(gscore_s[wib]);
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (lane + 32 * q < n_groups) flags[lane + 32 * q] = (chosen >> q) & 1u;
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (live[q]) live[q] = flags[(lane + 32 * q) / gsize] != 0u;
+      __syncwarp();
     }
     float zsel[MOE_MAX_TOPK];
     int isel[MOE_MAX_TOPK];
     for (int j = 0; j < k; ++j) {
       // best of this lane
       bool bv = false;
-      float bz = 0.f;
+      float bk = 0.f, bz = 0.f;
       int bi = 0x7fffffff;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        if (better(live[q], zv[q], lane + 32 * q, bv, bz, bi)) {
-          bv = live[q]; bz = zv[q]; bi = lane + 32 * q;
+        if (better(live[q], key[q], lane + 32 * q, bv, bk, bi)) {
+          bv = live[q]; bk = key[q]; bz = zv[q]; bi = lane + 32 * q;
         }
       }
 #pragma unroll
       for (int off = 16; off >= 1; off >>= 1) {
         const bool ov = __shfl_xor_sync(0xffffffffu, bv, off);
+        const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
         const float oz = __shfl_xor_sync(0xffffffffu, bz, off);
         const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (better(ov, oz, oi, bv, bz, bi)) {
-          bv = ov; bz = oz; bi = oi;
+        if (better(ov, ok, oi, bv, bk, bi)) {
+          bv = ov; bk = ok; bz = oz; bi = oi;
         }
       }
       zsel[j] = bz;
@@ -480,7 +555,8 @@ cudaError_t launch_small_e(const Shape& s, const TX* x, const float* w_router, c
   const int64_t cap = static_cast<int64_t>(sm_count()) * 64;
   const int blocks = static_cast<int>(blocks_needed < cap ? blocks_needed : cap);
   router_small_e_kernel<TX, ET><<<blocks, 256, 0, st>>>(x, wl, bias, bias_stride, s.T, d, s.E,
-                                                        s.k, s.gating, logits, topk_idx, topk_w);
+                                                        s.k, s.gating, s.bias_mode, logits,
+                                                        topk_idx, topk_w);
   return cudaGetLastError();
 }
 
@@ -490,7 +566,7 @@ cudaError_t launch_router_typed(const Shape& s, const TX* x, const float* w_rout
                                 int32_t* topk_idx, float* topk_w, float* partials,
                                 cudaStream_t st) {
   const int d = static_cast<int>(s.d);
-  if (s.E <= 32) {
+  if (s.E <= 32 && s.n_groups <= 1) {
     float4* wl = reinterpret_cast<float4*>(partials);  // the workspace's router area
     if (s.E <= 8)
       return launch_small_e<TX, 8>(s, x, w_router, bias, bias_stride, logits, topk_idx, topk_w,
@@ -507,26 +583,34 @@ cudaError_t launch_router_typed(const Shape& s, const TX* x, const float* w_rout
   int k_per_split = (d + nsplit - 1) / nsplit;
   k_per_split = (k_per_split + RT_K - 1) / RT_K * RT_K;
   dim3 grid(tiles_n, static_cast<unsigned>(tiles_m), nsplit);
-  router_gemm_kernel<TX><<<grid, 256, 0, st>>>(x, w_router, bias, bias_stride, s.T, d, s.E,
+  const bool sel_only = s.bias_mode == MOE_BIAS_SELECTION_ONLY;
+  // the GEMM adds the bias itself only when it writes finished logits that carry it
+  const float* gemm_bias = (nsplit == 1 && !sel_only) ? bias : nullptr;
+  router_gemm_kernel<TX><<<grid, 256, 0, st>>>(x, w_router, gemm_bias, bias_stride, s.T, d, s.E,
                                                k_per_split, nsplit > 1 ? partials : logits);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const int64_t blocks_needed = (s.T + 7) / 8;
   const int blocks = static_cast<int>(blocks_needed < 148 * 16 ? blocks_needed : 148 * 16);
-  topk_from_logits_kernel<<<blocks, 256, 0, st>>>(nsplit > 1 ? partials : logits, nsplit, bias,
-                                                  bias_stride, logits, s.T, s.E, s.k, s.gating,
-                                                  topk_idx, topk_w);
+  topk_from_logits_kernel<<<blocks, 256, 0, st>>>(
+      nsplit > 1 ? partials : logits, nsplit, bias, bias_stride,
+      (nsplit > 1 && !sel_only) ? 1 : 0, sel_only ? 1 : 0, logits, s.T, s.E, s.k, s.gating,
+      s.n_groups, s.topk_groups, topk_idx, topk_w);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_topk_from_logits(const Shape& s, const float* logits, int32_t* topk_idx,
-                                    float* topk_w, cudaStream_t st) {
+cudaError_t launch_topk_from_logits(const Shape& s, const float* logits, const float* bias,
+                                    int64_t bias_stride, int32_t* topk_idx, float* topk_w,
+                                    cudaStream_t st) {
   const int64_t blocks_needed = (s.T + 7) / 8;
   const int blocks = static_cast<int>(blocks_needed < 148 * 16 ? blocks_needed : 148 * 16);
-  topk_from_logits_kernel<<<blocks, 256, 0, st>>>(logits, 1, nullptr, 0, nullptr, s.T, s.E, s.k,
-                                                  s.gating, topk_idx, topk_w);
+  const bool sel_only = s.bias_mode == MOE_BIAS_SELECTION_ONLY;
+  topk_from_logits_kernel<<<blocks, 256, 0, st>>>(logits, 1, sel_only ? bias : nullptr,
+                                                  bias_stride, 0, sel_only ? 1 : 0, nullptr, s.T,
+                                                  s.E, s.k, s.gating, s.n_groups, s.topk_groups,
+                                                  topk_idx, topk_w);
   return cudaGetLastError();
 }
 

@@ -106,13 +106,18 @@ def check_routing(run: GpuRun, sample_rows=None) -> dict:
     rows = np.arange(s.T) if sample_rows is None else np.asarray(sample_rows)
     bias = None
     trows = torch.from_numpy(rows).to(i.x.device)
-    if i.logit_bias is not None:
+    sel_only = s.bias_mode == O.BIAS_SELECTION_ONLY
+    if i.logit_bias is not None and not sel_only:
         bias = f64(i.logit_bias) if i.logit_bias.dim() == 1 else f64(i.logit_bias[trows])
     z64 = O.router_logits(f64(i.x[trows]), f64(i.w_router), bias)
     err = np.abs(z32[rows].astype(np.float64) - z64) / (1.0 + np.abs(z64))
     tol = TOL_LOGIT_SPLIT if router_on_tensor_cores(s) else TOL_LOGIT
     assert err.max() <= tol, f"logits max scaled error {err.max():.3g} (tol {tol})"
-    r = O.route(z32, s.k, s.gating, cf32(s), s.layout)
+    sel_bias = None
+    if sel_only and i.logit_bias is not None:
+        sel_bias = i.logit_bias.detach().cpu().numpy().astype(np.float32)
+    r = O.route(z32, s.k, s.gating, cf32(s), s.layout, s.n_groups, s.topk_groups, sel_bias,
+                s.bias_mode, s.drop_policy)
     np.testing.assert_array_equal(i64(b.topk_idx), r["idx"])
     w_err = np.abs(f64(b.topk_w) - r["w"]).max()
     assert w_err <= TOL_W, f"gate weights max abs error {w_err:.3g}"

@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(lib):
     assert not missing, missing
     for n in names:
         assert getattr(lib, n) is not None
-    assert lib.moe_abi_version() == 1
+    assert lib.moe_abi_version() == 2
 
 
 def test_struct_layout_matches_header(tmp_path):
@@ -109,6 +109,18 @@ def test_workspace_size_and_bad_configs(lib):
     # PADDED without a capacity
     with pytest.raises(M.MoEError):
         M.workspace_size(M.make_config(64, 128, 256, 8, 2, layout=M.PADDED))
+    # group limits that cannot hold k experts, or groups that do not divide E
+    with pytest.raises(M.MoEError):
+        M.workspace_size(M.make_config(64, 128, 256, 8, 4, n_groups=4, topk_groups=1))
+    with pytest.raises(M.MoEError):
+        M.workspace_size(M.make_config(64, 128, 256, 8, 2, n_groups=3, topk_groups=1))
+    for bad in (dict(bias_mode=2), dict(drop_policy=5)):
+        with pytest.raises(M.MoEError):
+            M.workspace_size(M.make_config(64, 128, 256, 8, 2, **bad))
+    # pick-rank drops keep k count planes per block
+    a = M.workspace_size(M.make_config(4096, 4096, 4096, 8, 2))
+    b = M.workspace_size(M.make_config(4096, 4096, 4096, 8, 2, drop_policy=M.DROP_PICK_RANK))
+    assert b - a == 16 * 8 * 4
 
 
 def test_null_and_misaligned_pointers_rejected_on_host(lib):

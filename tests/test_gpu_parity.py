@@ -188,6 +188,39 @@ def test_empty_experts_and_padded_layout():
     check_stats(st, r)
 
 
+# ------------------------------------------------------------------ routing variants
+VARIANTS = [
+    # group-limited top-8 of 256 (8 groups, 4 kept), bias for selection only, pick-rank drops;
+    # 1024 tokens: tensor-core router
+    W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256, n_groups=8, topk_groups=4, bias_mode=1,
+              drop_policy=1),
+    # the same regime through the fp32 router (T < 512) and token-order drops
+    W.reduced(W.DSV3_PREFILL_ZIPF, 300, 256, 128, n_groups=16, topk_groups=2, bias_mode=1),
+    # E = 8 with groups (general top-k path), pick-rank drops, chunk bias in score and weight
+    W.reduced(W.MIXTRAL_8X22B_MIXED, 900, 256, 384, n_decode_tokens=8, n_groups=4,
+              topk_groups=2, drop_policy=1),
+    # E = 8 fused router with selection-only bias; fp32 layer
+    W.reduced(W.TINY_FP32, 200, 64, 96, bias="chunks", bias_mode=1, drop_policy=1,
+              capacity_factor=0.9),
+]
+
+
+@pytest.mark.parametrize("shape", VARIANTS, ids=lambda s: s.name + f"_g{s.n_groups}_b{s.bias_mode}_d{s.drop_policy}")
+def test_routing_variants_match_oracle(shape):
+    run = GpuRun(shape)
+    st = run.all_stages()
+    r = check_routing(run)
+    check_permute(run, r)
+    check_ffn_rows(run, r)
+    check_combine(run, r)
+    check_stats(st, r)
+    check_layer_output(run, run.b.out, r)
+    if shape.n_groups > 1:   # every token's experts lie in at most topk_groups groups
+        gsize = shape.E // shape.n_groups
+        spans = [len(set(int(e) // gsize for e in row)) for row in r["idx"]]
+        assert max(spans) <= shape.topk_groups
+
+
 # ------------------------------------------------------------------ errors without faults
 def test_bad_expert_index_is_reported_not_faulted():
     shape = _edge(50, 64, 64, 8, 2)
