@@ -33,8 +33,6 @@ from routing_dispatch_expert_warp_b200 import workload as W  # noqa: E402
 DEFAULT = W.MIXTRAL_8X7B
 METRIC = "MoE-layer tokens/s on 1 B200; grouped-GEMM % BF16 peak; permute/combine % HBM BW"
 L2_FLUSH_BYTES = 256 << 20
-KERNELS_PER_STEP_E_SMALL = 9   # router, count, scan, rank, permute, gemm x2, combine, stats
-KERNELS_PER_STEP_E_LARGE = 10  # + separate top-k kernel
 
 
 def measured_peaks() -> dict:
@@ -125,6 +123,8 @@ def run_gpu(args) -> None:
     shape = W.WORKLOADS[args.config] if args.config else DEFAULT
     if args.tokens:
         shape = shape.replace(name=f"{shape.name}_with_T{args.tokens}", T=args.tokens)
+    if args.d_ff:
+        shape = shape.replace(name=f"{shape.name}_with_f{args.d_ff}", d_ff=args.d_ff)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -175,9 +175,11 @@ def run_gpu(args) -> None:
     torch.cuda.synchronize(dev)
     clocks = ClockSampler(local)
     time.sleep(0.3)
+    launches0 = M.kernel_launch_count()
     for i in range(args.steps):
         flush.zero_()
         step(evs[i])
+    timed_launches = M.kernel_launch_count() - launches0
     torch.cuda.synchronize(dev)
     if dist:
         dist.barrier()
@@ -228,7 +230,6 @@ def run_gpu(args) -> None:
 
     if rank == 0:
         cpu = cpu_baseline(shape, args.cpu_sample_tokens) if (world == 1 and not args.no_cpu) else None
-        per_step_kernels = KERNELS_PER_STEP_E_SMALL if shape.E <= 32 else KERNELS_PER_STEP_E_LARGE
         line = {
             "metric": METRIC,
             "value": shape.T * world / (ms_per_step * 1e-3),
@@ -274,7 +275,7 @@ def run_gpu(args) -> None:
                     "h2d_bytes_per_step": inp.x.numel() * inp.x.element_size(),
                     "d2h_bytes_per_step": b.out.numel() * b.out.element_size(),
                     "api": "MoELayer.forward -> moe_layer_forward (pinned host buffers)"},
-            "gpu_launches": per_step_kernels * args.steps,
+            "gpu_launches": timed_launches,
             "clocks": clk,
             "cpu_baseline": cpu,
         }
@@ -356,6 +357,9 @@ def main():
     ap.add_argument("--config", default=None, choices=sorted(W.WORKLOADS))
     ap.add_argument("--tokens", type=int, default=0,
                     help="override T of the workload (small profiling cases)")
+    ap.add_argument("--d-ff", type=int, default=0,
+                    help="override d_ff of the workload (small profiling cases of the router "
+                         "and dispatch kernels)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-sample-tokens", type=int, default=64)
     ap.add_argument("--ref-sample-tokens", type=int, default=32)

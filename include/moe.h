@@ -335,6 +335,11 @@ moe_status_t moe_selftest_bounded_wait(void* ws, size_t ws_bytes, void* stream);
 /* MOE_ABI_VERSION of the loaded library. */
 int32_t moe_abi_version(void);
 
+/* Number of kernels this library has launched in this process so far, over every device
+ * and stream (a launch is counted when it is issued, not when it runs).  The difference of
+ * two readings around a region counts the library's kernels in it.  Never fails. */
+uint64_t moe_kernel_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

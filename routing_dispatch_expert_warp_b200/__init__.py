@@ -26,7 +26,8 @@ __all__ = ["MoEError", "make_config", "workspace_size", "capacity", "max_rows",
            "alloc_workspace", "moe_route", "moe_dispatch", "moe_dispatch_static_scratch",
            "moe_expert_ffn", "moe_combine",
            "moe_load_stats", "moe_layer_forward", "moe_check_device_error",
-           "moe_selftest_bounded_wait", "set_wait_limit_ns", "LayerBuffers", "MoELayer"]
+           "moe_selftest_bounded_wait", "set_wait_limit_ns", "kernel_launch_count",
+           "LayerBuffers", "MoELayer"]
 
 
 def _lib():
@@ -155,6 +156,11 @@ def moe_check_device_error(ws, stream=None):
 
 def moe_selftest_bounded_wait(ws, stream=None):
     check(_lib().moe_selftest_bounded_wait(_ptr(ws), ws.numel(), _stream(stream)))
+
+
+def kernel_launch_count() -> int:
+    """Kernels the library has launched in this process so far (all devices and streams)."""
+    return int(_lib().moe_kernel_launch_count())
 
 
 # ------------------------------------------------------------------ whole layer

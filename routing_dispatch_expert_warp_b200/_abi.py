@@ -81,6 +81,7 @@ PROTOTYPES = {
     "moe_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "moe_selftest_bounded_wait": (c_i32, [c_vp, c_sz, c_vp]),
     "moe_abi_version": (c_i32, []),
+    "moe_kernel_launch_count": (ctypes.c_uint64, []),
 }
 
 _lib = None

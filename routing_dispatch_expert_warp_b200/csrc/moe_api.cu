@@ -183,8 +183,15 @@ __global__ void wait_selftest_kernel(DevStatus* status, uint64_t wait_ns) {
 }
 }  // namespace
 
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}  // namespace
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 cudaError_t launch_wait_selftest(DevStatus* status, uint64_t wait_ns, cudaStream_t st) {
   wait_selftest_kernel<<<1, 32, 0, st>>>(status, wait_ns);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -195,6 +202,8 @@ using namespace moe;
 extern "C" {
 
 int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+uint64_t moe_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char* moe_last_error(void) { return g_last_error.c_str(); }
 

@@ -89,6 +89,7 @@ cudaError_t launch_combine_typed(const Shape& s, const void* y_perm, const int32
   else
     combine_kernel<BF16, 1><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
         y, assign_row, topk_w, s.T, s.k, vec_per_row, o);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -288,10 +288,12 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
   const int planes = dispatch_planes(s);
   dispatch_count_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
       topk_idx, s.T, s.k, s.E, planes, hist, status);
+  note_launch();
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   dispatch_rank_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
       topk_idx, s.T, s.k, s.E, s.C, s.layout, planes, nblk, hist, routed, kept, offsets,
       assign_row, token_of_row, s.max_rows);
+  note_launch();
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
 
   const int64_t row_bytes = s.d * s.elem;
@@ -314,6 +316,7 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
     if (err != cudaSuccess) return err;
     permute_rows_kernel<16, 8><<<static_cast<unsigned>(grid), 32, smem, st>>>(
         xb, assign_row, s.T, s.k, row_bytes, sg, segs, xp, status, wait_ns);
+    note_launch();
   } else if (seg <= 8 * 1024) {
     const size_t smem = 12 * static_cast<size_t>(seg);
     err = cudaFuncSetAttribute(permute_rows_kernel<12, 6>,
@@ -321,6 +324,7 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
     if (err != cudaSuccess) return err;
     permute_rows_kernel<12, 6><<<static_cast<unsigned>(grid), 32, smem, st>>>(
         xb, assign_row, s.T, s.k, row_bytes, sg, segs, xp, status, wait_ns);
+    note_launch();
   } else {
     const size_t smem = 6 * static_cast<size_t>(seg);
     err = cudaFuncSetAttribute(permute_rows_kernel<6, 3>,
@@ -328,6 +332,7 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
     if (err != cudaSuccess) return err;
     permute_rows_kernel<6, 3><<<static_cast<unsigned>(grid), 32, smem, st>>>(
         xb, assign_row, s.T, s.k, row_bytes, sg, segs, xp, status, wait_ns);
+    note_launch();
   }
   return cudaGetLastError();
 }

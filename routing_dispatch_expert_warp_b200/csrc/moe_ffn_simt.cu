@@ -92,10 +92,12 @@ cudaError_t launch_ffn_simt(const Shape& s, const float* x_perm, const int32_t* 
   const int d = static_cast<int>(s.d), f = static_cast<int>(s.f);
   dim3 g1((f + ST - 1) / ST, gy, s.E);
   ffn_simt_kernel<true><<<g1, 256, 0, st>>>(x_perm, wg, wu, f, d, offsets, kept, h);
+  note_launch();
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   dim3 g2((d + ST - 1) / ST, gy, s.E);
   ffn_simt_kernel<false><<<g2, 256, 0, st>>>(h, wd, nullptr, d, f, offsets, kept, y);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -474,6 +474,7 @@ cudaError_t launch_ffn_tc(const Shape& s, const void* x_perm, const int32_t* off
   if (g1 > sms) g1 = sms;
   grouped_gemm_tc_kernel<MODE_SWIGLU><<<static_cast<unsigned>(g1), THREADS, DYN_SMEM, st>>>(ta1, tg, tu,
                                                                                     p1);
+  note_launch();
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
 
   TcParams p2 = p1;
@@ -485,6 +486,7 @@ cudaError_t launch_ffn_tc(const Shape& s, const void* x_perm, const int32_t* off
   if (g2 > sms) g2 = sms;
   grouped_gemm_tc_kernel<MODE_DOWN><<<static_cast<unsigned>(g2), THREADS, DYN_SMEM, st>>>(ta2, td, td,
                                                                                      p2);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -512,6 +514,7 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_route
   dim3 sgrid((s.E + 31) / 32, static_cast<unsigned>((s.d + 31) / 32));
   split_router_weight_kernel<<<sgrid, 256, 0, st>>>(w_router, static_cast<int>(s.d), s.E, hi, lo,
                                                     seg, static_cast<int32_t>(s.T));
+  note_launch();
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   CUtensorMap ta, th, tl;
@@ -541,6 +544,7 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_route
   if (g > sm_count()) g = sm_count();
   grouped_gemm_tc_kernel<MODE_ROUTER><<<static_cast<unsigned>(g), THREADS, DYN_SMEM, st>>>(
       ta, th, tl, p);
+  note_launch();
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   return launch_topk_from_logits(s, logits, bias, bias_stride, topk_idx, topk_w, st);
 }

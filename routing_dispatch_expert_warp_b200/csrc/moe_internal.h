@@ -92,6 +92,9 @@ cudaError_t launch_wait_selftest(DevStatus* status, uint64_t wait_ns, cudaStream
 
 int sm_count();
 
+// Process-wide count of this library's kernel launches (every launch site calls it once).
+void note_launch();
+
 // Allocation-free dispatch: scratch lives in a fixed device array (moe_dispatch.cu).
 constexpr size_t kStaticDispatchHistBytes = size_t(1) << 20;  // 1 MiB of block histograms
 cudaError_t dispatch_static_scratch(const Shape& s, const void* x, const int32_t* topk_idx,

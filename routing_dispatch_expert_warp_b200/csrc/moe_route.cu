@@ -397,32 +397,57 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(
   }
 }
 
-// A warp per token: the top-k of z[t, 0..E) (E <= 256, up to 8 values per lane).
+// Selection scores as unsigned keys whose integer order is the float order: a larger key
+// is a larger score.  -0 and +0 map to one key (they compare equal as floats), a NaN maps to
+// 1, below every number, and 0 is left for "not eligible".
+__device__ __forceinline__ uint32_t order_key(float f) {
+  if (f != f) return 1u;
+  const uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Warp-wide argmax over keys held as lane + 32 q: the largest key, equal keys -> the lower
+// index.  Two warp reductions (max of the keys, then min of the indices holding it).
+template <int Q>
+__device__ __forceinline__ int warp_argmax(const uint32_t (&key)[Q], int lane) {
+  uint32_t m = key[0];
+#pragma unroll
+  for (int q = 1; q < Q; ++q) m = max(m, key[q]);
+  m = __reduce_max_sync(0xffffffffu, m);
+  int bi = 0x7fffffff;
+#pragma unroll
+  for (int q = Q - 1; q >= 0; --q)
+    if (key[q] == m) bi = lane + 32 * q;
+  return __reduce_min_sync(0xffffffffu, bi);
+}
+
 // A warp per token (E <= 256, lane holds experts lane + 32 q).  z holds nsplit partial sums
 // per logit (split-K) that are added in split order; `bias_into_z` adds the bias to them
 // (logits with bias), `bias_into_key` adds it to the selection score only.  The summed
 // logits are written to `logits` when nsplit > 1.  With n_groups > 1, the token first keeps
-// its topk_groups best expert groups (group score = best score in the group).
+// its topk_groups best expert groups (group score = best score in the group, equal scores
+// -> lower group index).  Every selection round is one warp_argmax over order keys; lane j
+// keeps the j-th pick, and lanes 0..k-1 write the token's picks and gate weights.
 __global__ void __launch_bounds__(256) topk_from_logits_kernel(
     const float* __restrict__ z, int nsplit, const float* __restrict__ bias, int64_t bias_stride,
     int bias_into_z, int bias_into_key, float* __restrict__ logits, int64_t T, int E, int k,
     int gating, int n_groups, int topk_groups, int32_t* __restrict__ topk_idx,
     float* __restrict__ topk_w) {
-  __shared__ float gscore_s[8][MOE_MAX_EXPERTS];
+  __shared__ uint32_t gkey_s[8][MOE_MAX_EXPERTS];
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const int gsize = n_groups > 1 ? E / n_groups : E;
   for (int64_t t = warp; t < T; t += nwarps) {
-    float zv[8], key[8];
-    bool live[8];
+    float zv[8];
+    uint32_t key[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const int e = lane + 32 * q;
-      live[q] = e < E;
       float acc = 0.f;
-      if (live[q]) {
+      key[q] = 0u;
+      if (e < E) {
         if (nsplit == 1) {
           acc = z[t * E + e];
         } else {
@@ -442,100 +467,92 @@ __global__ void __launch_bounds__(256) topk_from_logits_kernel(
         }
         if (bias != nullptr && bias_into_z) acc += bias[t * bias_stride + e];
         if (nsplit > 1 && logits != nullptr) logits[t * E + e] = acc;
+        key[q] = order_key((bias != nullptr && bias_into_key) ? acc + bias[t * bias_stride + e]
+                                                              : acc);
       }
       zv[q] = acc;
-      key[q] = (live[q] && bias != nullptr && bias_into_key) ? acc + bias[t * bias_stride + e]
-                                                             : acc;
     }
     if (n_groups > 1) {
-      // group scores through shared memory, then topk_groups rounds of a warp argmax
+      uint32_t* ks = gkey_s[wib];
 #pragma unroll
       for (int q = 0; q < 8; ++q)
-        if (live[q]) gscore_s[wib][lane + 32 * q] = key[q];
+        if (lane + 32 * q < E) ks[lane + 32 * q] = key[q];
       __syncwarp();
-      float gs[8];
+      // group scores (the largest key of each group), lane g + 32 q holds group g + 32 q
+      uint32_t gk[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const int g = lane + 32 * q;
-        float m = -INFINITY;
-        if (g < n_groups)
-          for (int i = 0; i < gsize; ++i) m = fmaxf(m, gscore_s[wib][g * gsize + i]);
-        gs[q] = m;
-      }
-      __syncwarp();
-      uint32_t chosen = 0;  // bit q: group lane + 32 q kept
-      for (int r = 0; r < topk_groups; ++r) {
-        bool bv = false;
-        float bz = 0.f;
-        int bi = 0x7fffffff;
+      for (int q = 0; q < 8; ++q) gk[q] = 0u;
+      if (gsize >= 32) {
+        for (int g = 0; g < n_groups; ++g) {
+          uint32_t m = 0u;
+          for (int i = lane; i < gsize; i += 32) m = max(m, ks[g * gsize + i]);
+          m = __reduce_max_sync(0xffffffffu, m);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (lane + 32 * q == g) gk[q] = m;
+        }
+      } else {
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const int g = lane + 32 * q;
-          const bool ok = g < n_groups && !((chosen >> q) & 1u);
-          if (better(ok, gs[q], g, bv, bz, bi)) {
-            bv = ok; bz = gs[q]; bi = g;
+          if (g < n_groups) {
+            uint32_t m = 0u;
+            for (int i = 0; i < gsize; ++i) m = max(m, ks[g * gsize + i]);
+            gk[q] = m;
           }
         }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) {
-          const bool ov = __shfl_xor_sync(0xffffffffu, bv, off);
-          const float oz = __shfl_xor_sync(0xffffffffu, bz, off);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-          if (better(ov, oz, oi, bv, bz, bi)) {
-            bv = ov; bz = oz; bi = oi;
-          }
-        }
+      }
+      __syncwarp();
+      // keep the topk_groups best groups; flags[g] != 0 marks a kept group
+      uint32_t chosen = 0;  // bit q: group lane + 32 q kept
+      for (int r = 0; r < topk_groups; ++r) {
+        const int bg = warp_argmax(gk, lane);
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-          if (lane + 32 * q == bi) chosen |= 1u << q;
+          if (lane + 32 * q == bg) {
+            chosen |= 1u << q;
+            gk[q] = 0u;
+          }
       }
-      // publish the chosen groups, then keep only their experts
-      uint32_t* flags = reinterpret_cast<uint32_t*>(gscore_s[wib]);
 #pragma unroll
       for (int q = 0; q < 8; ++q)
-        if (lane + 32 * q < n_groups) flags[lane + 32 * q] = (chosen >> q) & 1u;
+        if (lane + 32 * q < n_groups) ks[lane + 32 * q] = (chosen >> q) & 1u;
       __syncwarp();
 #pragma unroll
       for (int q = 0; q < 8; ++q)
-        if (live[q]) live[q] = flags[(lane + 32 * q) / gsize] != 0u;
+        if (lane + 32 * q < E && ks[(lane + 32 * q) / gsize] == 0u) key[q] = 0u;
       __syncwarp();
     }
-    float zsel[MOE_MAX_TOPK];
-    int isel[MOE_MAX_TOPK];
+    int mysel = 0;  // lane j < k: the j-th pick
     for (int j = 0; j < k; ++j) {
-      // best of this lane
-      bool bv = false;
-      float bk = 0.f, bz = 0.f;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (better(live[q], key[q], lane + 32 * q, bv, bk, bi)) {
-          bv = live[q]; bk = key[q]; bz = zv[q]; bi = lane + 32 * q;
-        }
-      }
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) {
-        const bool ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-        const float oz = __shfl_xor_sync(0xffffffffu, bz, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (better(ov, ok, oi, bv, bk, bi)) {
-          bv = ov; bk = ok; bz = oz; bi = oi;
-        }
-      }
-      zsel[j] = bz;
-      isel[j] = bi;
+      const int bi = warp_argmax(key, lane);
+      if (lane == j) mysel = bi;
 #pragma unroll
       for (int q = 0; q < 8; ++q)
-        if (lane + 32 * q == bi) live[q] = false;
+        if (lane + 32 * q == bi) key[q] = 0u;
     }
-    if (lane == 0) {
-      float w[MOE_MAX_TOPK];
-      gate_weights(zsel, k, gating, w);
-      for (int j = 0; j < k; ++j) {
-        topk_idx[t * k + j] = isel[j];
-        topk_w[t * k + j] = w[j];
-      }
+    // the picked logits, from the lanes that hold them
+    float myz = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float v = __shfl_sync(0xffffffffu, zv[q], mysel & 31);
+      if ((mysel >> 5) == q) myz = v;
+    }
+    // gate weights over the k picks; the normaliser is summed in pick order
+    float w;
+    if (gating == MOE_GATE_SOFTMAX) {
+      float m = myz;
+      for (int j = 1; j < k; ++j) m = fmaxf(m, __shfl_sync(0xffffffffu, myz, j));
+      m = __shfl_sync(0xffffffffu, m, 0);
+      w = expf(myz - m);
+    } else {
+      w = 1.0f / (1.0f + expf(-myz));
+    }
+    float ssum = 0.f;
+    for (int j = 0; j < k; ++j) ssum += __shfl_sync(0xffffffffu, w, j);
+    if (lane < k) {
+      topk_idx[t * k + lane] = mysel;
+      topk_w[t * k + lane] = w * (1.0f / ssum);
     }
   }
 }
@@ -548,6 +565,7 @@ cudaError_t launch_small_e(const Shape& s, const TX* x, const float* w_router, c
   const int64_t lanes_total = static_cast<int64_t>((d + 255) / 256) * (8 * ET / 4) * 32;
   const int pblocks = static_cast<int>((lanes_total + 255) / 256 < 1024 ? (lanes_total + 255) / 256 : 1024);
   router_weight_lanes_kernel<ET><<<pblocks, 256, 0, st>>>(w_router, d, s.E, wl);
+  note_launch();
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   constexpr int TW = 32 / ET;
@@ -557,6 +575,7 @@ cudaError_t launch_small_e(const Shape& s, const TX* x, const float* w_router, c
   router_small_e_kernel<TX, ET><<<blocks, 256, 0, st>>>(x, wl, bias, bias_stride, s.T, d, s.E,
                                                         s.k, s.gating, s.bias_mode, logits,
                                                         topk_idx, topk_w);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -588,6 +607,7 @@ cudaError_t launch_router_typed(const Shape& s, const TX* x, const float* w_rout
   const float* gemm_bias = (nsplit == 1 && !sel_only) ? bias : nullptr;
   router_gemm_kernel<TX><<<grid, 256, 0, st>>>(x, w_router, gemm_bias, bias_stride, s.T, d, s.E,
                                                k_per_split, nsplit > 1 ? partials : logits);
+  note_launch();
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   const int64_t blocks_needed = (s.T + 7) / 8;
@@ -596,6 +616,7 @@ cudaError_t launch_router_typed(const Shape& s, const TX* x, const float* w_rout
       nsplit > 1 ? partials : logits, nsplit, bias, bias_stride,
       (nsplit > 1 && !sel_only) ? 1 : 0, sel_only ? 1 : 0, logits, s.T, s.E, s.k, s.gating,
       s.n_groups, s.topk_groups, topk_idx, topk_w);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -611,6 +632,7 @@ cudaError_t launch_topk_from_logits(const Shape& s, const float* logits, const f
                                                   bias_stride, 0, sel_only ? 1 : 0, nullptr, s.T,
                                                   s.E, s.k, s.gating, s.n_groups, s.topk_groups,
                                                   topk_idx, topk_w);
+  note_launch();
   return cudaGetLastError();
 }
 

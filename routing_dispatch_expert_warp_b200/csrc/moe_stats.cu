@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
 cudaError_t launch_stats(const Shape& s, const int32_t* routed, const int32_t* kept,
                          const int32_t* assign_row, moe_load_stats_t* out, cudaStream_t st) {
   stats_kernel<<<1, kStatsThreads, 0, st>>>(routed, kept, assign_row, s.T, s.k, s.E, s.C, out);
+  note_launch();
   return cudaGetLastError();
 }
 

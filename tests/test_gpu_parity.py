@@ -253,3 +253,19 @@ def test_bounded_wait_runs_out_and_context_survives():
     st = run.all_stages()
     r = check_routing(run)
     check_stats(st, r)
+
+
+# ------------------------------------------------------------------ launch accounting
+@pytest.mark.parametrize("shape,router_kernels", [
+    (W.reduced(W.MIXTRAL_8X7B, 1000, 512, 768), 2),          # lane-ordered W_r + fused router
+    (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256), 3),     # W_r split + tensor-core GEMM + top-k
+    (W.reduced(W.DSV3_DECODE, 128, 512, 256), 2),            # split-K fp32 GEMM + top-k
+])
+def test_kernel_launch_count_per_layer(shape, router_kernels):
+    """One staged layer forward launches the router's kernels, count + rank + permute, the two
+    grouped GEMMs, combine and stats -- and the library's own counter says so."""
+    run = GpuRun(shape)
+    run.all_stages()
+    c0 = M.kernel_launch_count()
+    run.all_stages()
+    assert M.kernel_launch_count() - c0 == router_kernels + 3 + 2 + 1 + 1
