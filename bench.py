@@ -34,6 +34,30 @@ DEFAULT = W.MIXTRAL_8X7B
 METRIC = "MoE-layer tokens/s on 1 B200; grouped-GEMM % BF16 peak; permute/combine % HBM BW"
 L2_FLUSH_BYTES = 256 << 20
 
+# DRAM traffic of the grouped GEMM (gate/up + down launch, bytes per layer step) from one
+# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload and dispatch
+# mode, with the hash of the GEMM's sources at capture time: a changed kernel reports null.
+GEMM_SOURCES = ("routing_dispatch_expert_warp_b200/csrc/moe_ffn_tc.cu",
+                "routing_dispatch_expert_warp_b200/csrc/moe_device.cuh",
+                "routing_dispatch_expert_warp_b200/csrc/moe_internal.h")
+RECORDED_GEMM_TRAFFIC = {}
+
+
+def gemm_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, gather: bool):
+    rec = RECORDED_GEMM_TRAFFIC.get((workload, gather))
+    if rec is None or rec["sources"] != gemm_source_hash():
+        return None
+    return rec
+
 
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -143,7 +167,7 @@ def run_gpu(args) -> None:
     inp = W.make_inputs(rank_shape(shape, rank), device=dev)
     cfg = M.config_from_shape(shape)
     ws = M.alloc_workspace(cfg, dev)
-    b = M.LayerBuffers.allocate(cfg, dev)
+    b = M.LayerBuffers.allocate(cfg, dev, gather=args.gather)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -154,8 +178,12 @@ def run_gpu(args) -> None:
         M.moe_dispatch(cfg, inp.x, b.topk_idx, b.routed_counts, b.kept_counts, b.expert_offsets,
                        b.assign_row, b.token_of_row, b.x_perm, ws)
         ev[2].record(stream)
-        M.moe_expert_ffn(cfg, b.x_perm, b.expert_offsets, b.kept_counts, inp.w_gate, inp.w_up,
-                         inp.w_down, b.h, b.y_perm, ws)
+        if args.gather:
+            M.moe_expert_ffn_gather(cfg, inp.x, b.token_of_row, b.expert_offsets, b.kept_counts,
+                                    inp.w_gate, inp.w_up, inp.w_down, b.h, b.y_perm, ws)
+        else:
+            M.moe_expert_ffn(cfg, b.x_perm, b.expert_offsets, b.kept_counts, inp.w_gate,
+                             inp.w_up, inp.w_down, b.h, b.y_perm, ws)
         ev[3].record(stream)
         M.moe_combine(cfg, b.y_perm, b.assign_row, b.topk_w, b.out)
         ev[4].record(stream)
@@ -207,7 +235,7 @@ def run_gpu(args) -> None:
 
     # end to end through the public API: pinned host x -> device, layer, device -> host out
     layer = M.MoELayer(cfg, inp.w_router, inp.w_gate, inp.w_up, inp.w_down, inp.logit_bias,
-                       device=dev)
+                       device=dev, gather=args.gather)
     x_host = inp.x.cpu().pin_memory()
     out_host = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
     x_dev = torch.empty_like(inp.x)
@@ -248,6 +276,8 @@ def run_gpu(args) -> None:
                        "gating": "softmax" if shape.gating == W.SOFTMAX else "sigmoid",
                        "capacity_factor": shape.capacity_factor,
                        "l2": "flushed between timed steps (256 MB write)",
+                       "dispatch": ("no x_perm: gate/up GEMM gathers rows of x" if args.gather
+                                    else "permuted copy x_perm"),
                        "parallelism": f"replicas x{world} (EP=1, no exchange)"},
             "roofline": {
                 "kernel": "grouped_gemm_tc_kernel (expert FFN: gate/up + down launches)",
@@ -256,15 +286,18 @@ def run_gpu(args) -> None:
                 "peak_source": f"{peaks['source']} bf16 burst",
                 "frac_of_sustained": (tflops / peaks["bf16_tflops_sustained"]
                                       if peaks.get("bf16_tflops_sustained") else None),
-                "traffic": None,
+                "traffic": (recorded_traffic(shape.name, args.gather) or {}).get("bytes"),
+                "traffic_source": (recorded_traffic(shape.name, args.gather) or {}).get("profile"),
                 "algorithmic_flops_per_step": work["gemm_flops"],
             },
             "stages_ms": {n: sum(v) / args.steps for n, v in per_stage.items()},
             "stage_bandwidth": {
                 "route": {"GB/s": gbs(work["route_bytes"], "route"),
                           "frac_hbm": gbs(work["route_bytes"], "route") / peaks["hbm_gbs"]},
-                "dispatch": {"GB/s": gbs(work["permute_bytes"], "dispatch"),
-                             "frac_hbm": gbs(work["permute_bytes"], "dispatch") / peaks["hbm_gbs"]},
+                "dispatch": ({"us": sum(per_stage["dispatch"]) / args.steps * 1e3,
+                              "note": "bookkeeping only (no copy)"} if args.gather else
+                             {"GB/s": gbs(work["permute_bytes"], "dispatch"),
+                              "frac_hbm": gbs(work["permute_bytes"], "dispatch") / peaks["hbm_gbs"]}),
                 "combine": {"GB/s": gbs(work["combine_bytes"], "combine"),
                             "frac_hbm": gbs(work["combine_bytes"], "combine") / peaks["hbm_gbs"]},
                 "hbm_peak_gbs": peaks["hbm_gbs"],
@@ -364,6 +397,8 @@ def main():
     ap.add_argument("--cpu-sample-tokens", type=int, default=64)
     ap.add_argument("--ref-sample-tokens", type=int, default=32)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--gather", action="store_true",
+                    help="dispatch without the permuted copy: the gate/up GEMM gathers rows of x")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)   # at least three untimed warm-up steps
     if args.impl == "reference":

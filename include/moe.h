@@ -180,7 +180,8 @@ typedef struct moe_layer_buffers {
   int32_t* expert_offsets;   /* [E+1] first row of each bucket; [E] = rows in use/alloc  */
   int32_t* assign_row;       /* [T, k] row of x_perm holding pick j of token t; -1 dropped*/
   int32_t* token_of_row;     /* [max_rows] token of each row; -1 for unused rows          */
-  void* x_perm;              /* [max_rows, d_model] dtype                                */
+  void* x_perm;              /* [max_rows, d_model] dtype, or NULL: no permuted copy, the */
+                             /* gate/up GEMM gathers rows of x (moe_expert_ffn_gather)   */
   void* h;                   /* [max_rows, d_ff] dtype                                   */
   void* y_perm;              /* [max_rows, d_model] dtype                                */
   void* out;                 /* [T, d_model] dtype                                       */
@@ -229,6 +230,8 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
  *   assign_row[t, j] = expert_offsets[e] + slot, or -1 if dropped.
  *   token_of_row[r] = token copied into row r; -1 for rows no assignment uses.
  *   x_perm[assign_row[t, j], :] = x[t, :] for every kept pick; unused rows untouched.
+ * x_perm may be NULL (x may then be NULL too): only the counts, offsets, assign_row and
+ * token_of_row are produced, for moe_expert_ffn_gather.
  */
 moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
                           int32_t* routed_counts, int32_t* kept_counts,
@@ -279,6 +282,23 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
                             const int32_t* expert_offsets, const int32_t* kept_counts,
                             const void* w_gate, const void* w_up, const void* w_down, void* h,
                             void* y_perm, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_expert_ffn without the permuted copy of x: the gate/up GEMM reads bucket row r as
+ * x[token_of_row[r], :] (TMA row gathers straight from x), so dispatch need not write
+ * x_perm.  This is the dispatch half of the fused dispatch-compute-combine kernels that
+ * [EP-serving] names as the direction of expert parallelism (its closing section on the
+ * future of EP serving, in the Wolof edition of the page).  Results are identical to
+ * moe_dispatch + moe_expert_ffn.  token_of_row is
+ * moe_dispatch's output ([max_rows] int32); an entry outside [0, T) inside a bucket reads
+ * row 0 instead (never out of range).  Other arguments, layouts and errors as
+ * moe_expert_ffn.
+ */
+moe_status_t moe_expert_ffn_gather(const moe_config_t* cfg, const void* x,
+                                   const int32_t* token_of_row, const int32_t* expert_offsets,
+                                   const int32_t* kept_counts, const void* w_gate,
+                                   const void* w_up, const void* w_down, void* h, void* y_perm,
+                                   void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Combine ([EP-serving] "Deep dive": results shuffled back; [EP-checks]: combine, unpack):

@@ -24,7 +24,7 @@ DROP_TOKEN_ORDER, DROP_PICK_RANK = 0, 1
 
 __all__ = ["MoEError", "make_config", "workspace_size", "capacity", "max_rows",
            "alloc_workspace", "moe_route", "moe_dispatch", "moe_dispatch_static_scratch",
-           "moe_expert_ffn", "moe_combine",
+           "moe_expert_ffn", "moe_expert_ffn_gather", "moe_combine",
            "moe_load_stats", "moe_layer_forward", "moe_check_device_error",
            "moe_selftest_bounded_wait", "set_wait_limit_ns", "kernel_launch_count",
            "LayerBuffers", "MoELayer"]
@@ -127,6 +127,15 @@ def moe_expert_ffn(cfg, x_perm, expert_offsets, kept_counts, w_gate, w_up, w_dow
                                 _ptr(h), _ptr(y_perm), _ptr(ws), ws.numel(), _stream(stream)))
 
 
+def moe_expert_ffn_gather(cfg, x, token_of_row, expert_offsets, kept_counts, w_gate, w_up,
+                          w_down, h, y_perm, ws, stream=None):
+    """moe_expert_ffn reading bucket row r as x[token_of_row[r]] (no permuted copy of x)."""
+    check(_lib().moe_expert_ffn_gather(ctypes.byref(cfg), _ptr(x), _ptr(token_of_row),
+                                       _ptr(expert_offsets), _ptr(kept_counts), _ptr(w_gate),
+                                       _ptr(w_up), _ptr(w_down), _ptr(h), _ptr(y_perm),
+                                       _ptr(ws), ws.numel(), _stream(stream)))
+
+
 def moe_combine(cfg, y_perm, assign_row, topk_w, out, stream=None):
     check(_lib().moe_combine(ctypes.byref(cfg), _ptr(y_perm), _ptr(assign_row), _ptr(topk_w),
                              _ptr(out), _stream(stream)))
@@ -175,14 +184,14 @@ class LayerBuffers:
     expert_offsets: torch.Tensor
     assign_row: torch.Tensor
     token_of_row: torch.Tensor
-    x_perm: torch.Tensor
+    x_perm: Optional[torch.Tensor]   # None: the gate/up GEMM gathers rows of x
     h: torch.Tensor
     y_perm: torch.Tensor
     out: torch.Tensor
     stats: torch.Tensor
 
     @staticmethod
-    def allocate(cfg: MoeConfig, device="cuda") -> "LayerBuffers":
+    def allocate(cfg: MoeConfig, device="cuda", gather: bool = False) -> "LayerBuffers":
         T, d, f, E, k = cfg.T, cfg.d_model, cfg.d_ff, cfg.E, cfg.k
         R = max_rows(cfg)
         dt = torch.float32 if cfg.dtype == F32 else torch.bfloat16
@@ -194,7 +203,7 @@ class LayerBuffers:
             routed_counts=torch.empty(E, **i32), kept_counts=torch.empty(E, **i32),
             expert_offsets=torch.empty(E + 1, **i32), assign_row=torch.empty((T, k), **i32),
             token_of_row=torch.empty(max(R, 1), **i32),
-            x_perm=torch.empty((max(R, 1), d), dtype=dt, device=device),
+            x_perm=None if gather else torch.empty((max(R, 1), d), dtype=dt, device=device),
             h=torch.empty((max(R, 1), f), dtype=dt, device=device),
             y_perm=torch.empty((max(R, 1), d), dtype=dt, device=device),
             out=torch.empty((T, d), dtype=dt, device=device),
@@ -219,15 +228,16 @@ class MoELayer:
 
     forward(x) enqueues the whole layer (moe_layer_forward) on the current stream and
     returns the output tensor (a view of the layer's own buffer, overwritten by the next
-    call)."""
+    call).  gather=True drops the permuted copy of x: dispatch only ranks the assignments
+    and the gate/up GEMM gathers its rows from x (same results, less memory traffic)."""
 
     def __init__(self, cfg: MoeConfig, w_router, w_gate, w_up, w_down, logit_bias=None,
-                 device="cuda"):
+                 device="cuda", gather: bool = False):
         self.cfg = cfg
         self.w_router, self.w_gate, self.w_up, self.w_down = w_router, w_gate, w_up, w_down
         self.logit_bias = logit_bias
         self.ws = alloc_workspace(cfg, device)
-        self.bufs = LayerBuffers.allocate(cfg, device)
+        self.bufs = LayerBuffers.allocate(cfg, device, gather=gather)
         self._structs = self.bufs.as_struct(True)
 
     def inputs(self, x) -> MoeLayerInputs:

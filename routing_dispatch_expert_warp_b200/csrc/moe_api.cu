@@ -295,10 +295,11 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
   if (st != MOE_OK) return st;
   WsLayout lay;
   if ((st = check_ws(s, ws, ws_bytes, &lay)) != MOE_OK) return st;
-  MOE_REQUIRE(x && topk_idx && routed_counts && kept_counts && expert_offsets && assign_row &&
-                  token_of_row && x_perm,
+  MOE_REQUIRE(topk_idx && routed_counts && kept_counts && expert_offsets && assign_row &&
+                  token_of_row && (x || !x_perm),
               "moe_dispatch: NULL pointer");
-  MOE_REQUIRE(aligned16(x) && aligned16(x_perm), "moe_dispatch: x and x_perm must be 16-byte aligned");
+  MOE_REQUIRE(x_perm == nullptr || (aligned16(x) && aligned16(x_perm)),
+              "moe_dispatch: x and x_perm must be 16-byte aligned");
   int32_t* hist = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + lay.hist);
   cudaError_t err = launch_dispatch(s, x, topk_idx, routed_counts, kept_counts, expert_offsets,
                                     assign_row, token_of_row, x_perm, hist, ws_status(ws, lay),
@@ -334,40 +335,68 @@ moe_status_t moe_dispatch_static_scratch(const moe_config_t* cfg, const void* x,
   return MOE_OK;
 }
 
-moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
-                            const int32_t* expert_offsets, const int32_t* kept_counts,
-                            const void* w_gate, const void* w_up, const void* w_down, void* h,
-                            void* y_perm, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Both FFN entry points: A rows from x_perm (a_rows == nullptr) or gathered from x.
+moe_status_t expert_ffn(const char* name, const moe_config_t* cfg, const void* a,
+                        const int32_t* a_rows, const int32_t* expert_offsets,
+                        const int32_t* kept_counts, const void* w_gate, const void* w_up,
+                        const void* w_down, void* h, void* y_perm, void* ws, size_t ws_bytes,
+                        void* stream) {
   Shape s;
   moe_status_t st = check_config(cfg, &s);
   if (st != MOE_OK) return st;
   WsLayout lay;
   if ((st = check_ws(s, ws, ws_bytes, &lay)) != MOE_OK) return st;
-  MOE_REQUIRE(x_perm && expert_offsets && kept_counts && w_gate && w_up && w_down && h && y_perm,
-              "moe_expert_ffn: NULL pointer");
-  MOE_REQUIRE(aligned16(x_perm) && aligned16(w_gate) && aligned16(w_up) && aligned16(w_down) &&
+  MOE_REQUIRE(a && expert_offsets && kept_counts && w_gate && w_up && w_down && h && y_perm,
+              "%s: NULL pointer", name);
+  MOE_REQUIRE(aligned16(a) && aligned16(w_gate) && aligned16(w_up) && aligned16(w_down) &&
                   aligned16(h) && aligned16(y_perm),
-              "moe_expert_ffn: tensors must be 16-byte aligned");
+              "%s: tensors must be 16-byte aligned", name);
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   cudaError_t err;
   if (s.dtype == MOE_F32) {
-    err = launch_ffn_simt(s, static_cast<const float*>(x_perm), expert_offsets, kept_counts,
+    err = launch_ffn_simt(s, static_cast<const float*>(a), a_rows, expert_offsets, kept_counts,
                           static_cast<const float*>(w_gate), static_cast<const float*>(w_up),
                           static_cast<const float*>(w_down), static_cast<float*>(h),
                           static_cast<float*>(y_perm), strm);
-    if (err != cudaSuccess) return cuda_fail(err, "moe_expert_ffn (fp32) launch");
+    if (err != cudaSuccess) return cuda_fail(err, "expert FFN (fp32) launch");
     return MOE_OK;
   }
   if (s.d % 64 != 0 || s.f % 64 != 0)
     return fail(MOE_ERR_UNSUPPORTED, "bf16 expert FFN needs d_model and d_ff multiples of 64");
   const char* why = "";
-  err = launch_ffn_tc(s, x_perm, expert_offsets, kept_counts, w_gate, w_up, w_down, h, y_perm,
+  err = launch_ffn_tc(s, a, a_rows, expert_offsets, kept_counts, w_gate, w_up, w_down, h, y_perm,
                       ws_status(ws, lay), g_wait_ns.load(), strm, &why);
   if (err != cudaSuccess) {
-    if (why[0]) return fail(MOE_ERR_CUDA, "moe_expert_ffn: %s", why);
-    return cuda_fail(err, "moe_expert_ffn (bf16) launch");
+    if (why[0]) return fail(MOE_ERR_CUDA, "%s: %s", name, why);
+    return cuda_fail(err, "expert FFN (bf16) launch");
   }
   return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
+                            const int32_t* expert_offsets, const int32_t* kept_counts,
+                            const void* w_gate, const void* w_up, const void* w_down, void* h,
+                            void* y_perm, void* ws, size_t ws_bytes, void* stream) {
+  return expert_ffn("moe_expert_ffn", cfg, x_perm, nullptr, expert_offsets, kept_counts, w_gate,
+                    w_up, w_down, h, y_perm, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_expert_ffn_gather(const moe_config_t* cfg, const void* x,
+                                   const int32_t* token_of_row, const int32_t* expert_offsets,
+                                   const int32_t* kept_counts, const void* w_gate,
+                                   const void* w_up, const void* w_down, void* h, void* y_perm,
+                                   void* ws, size_t ws_bytes, void* stream) {
+  MOE_REQUIRE(token_of_row != nullptr, "moe_expert_ffn_gather: NULL token_of_row");
+  return expert_ffn("moe_expert_ffn_gather", cfg, x, token_of_row, expert_offsets, kept_counts,
+                    w_gate, w_up, w_down, h, y_perm, ws, ws_bytes, stream);
 }
 
 moe_status_t moe_combine(const moe_config_t* cfg, const void* y_perm,
@@ -415,8 +444,13 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_layer_inputs_t
                     b->expert_offsets, b->assign_row, b->token_of_row, b->x_perm, ws, ws_bytes,
                     stream);
   if (st != MOE_OK) return st;
-  st = moe_expert_ffn(cfg, b->x_perm, b->expert_offsets, b->kept_counts, in->w_gate, in->w_up,
-                      in->w_down, b->h, b->y_perm, ws, ws_bytes, stream);
+  if (b->x_perm != nullptr)
+    st = moe_expert_ffn(cfg, b->x_perm, b->expert_offsets, b->kept_counts, in->w_gate,
+                        in->w_up, in->w_down, b->h, b->y_perm, ws, ws_bytes, stream);
+  else
+    st = moe_expert_ffn_gather(cfg, in->x, b->token_of_row, b->expert_offsets, b->kept_counts,
+                               in->w_gate, in->w_up, in->w_down, b->h, b->y_perm, ws, ws_bytes,
+                               stream);
   if (st != MOE_OK) return st;
   st = moe_combine(cfg, b->y_perm, b->assign_row, b->topk_w, b->out, stream);
   if (st != MOE_OK) return st;

@@ -295,6 +295,7 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
       assign_row, token_of_row, s.max_rows);
   note_launch();
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if (x_perm == nullptr) return cudaSuccess;  // bookkeeping only: the FFN gathers rows of x
 
   const int64_t row_bytes = s.d * s.elem;
   const int64_t segs = (row_bytes + kPermMaxSeg - 1) / kPermMaxSeg;

@@ -67,6 +67,10 @@ struct TcParams {
   int64_t bias_stride;
   DevStatus* status;
   uint64_t wait_ns;
+  // Gathered A (gate/up only): A row i of a bucket is row a_rows[seg_start[e] + i] of the
+  // tensor behind tm_a (x itself, [a_rows_limit, K]); nullptr: A rows are the bucket rows.
+  const int32_t* a_rows;
+  int32_t a_rows_limit;
 };
 
 __device__ __forceinline__ void decode_tile(int tile, const int* tile_base, const int* mblocks,
@@ -163,8 +167,54 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
   const int total_tiles = tile_base[p.E];
   const int KB = p.K / BK;
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0 && p.a_rows == nullptr) {
     // ---------------------------------------------------------------- TMA producer
+    // One lane: waits for a free stage, arms it, loads the A tile (128 bucket rows) and B.
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      uint32_t armed = 0, armed_parity = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+        int e, mb, nb;
+        decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, p.mb_outer, e, mb, nb);
+        const int row0 = p.seg_start[e] + mb * BM;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty_bar[s], ph ^ 1u, p.wait_ns, &abort_s)) {
+            if (!abort_s)
+              record_error(p.status, DEV_TIMEOUT, 20, static_cast<unsigned long long>(tile));
+            abort_s = 1;
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + s * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
+          armed |= 1u << s;
+          armed_parity = (armed_parity & ~(1u << s)) | (ph << s);
+          tma_load_2d(sa, &tm_a, &full_bar[s], kb * BK, row0);
+          if (GATED) {
+            tma_load_3d(sb, &tm_b0, &full_bar[s], kb * BK, nb * 128, e);
+            tma_load_3d(sb + B_BYTES / 2, &tm_b1, &full_bar[s], kb * BK, nb * 128, e);
+          } else {
+            tma_load_3d(sb, &tm_b0, &full_bar[s], kb * BK, nb * 256, e);
+          }
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      // every fill this thread armed must land before the block can exit
+      for (int q = 0; q < STAGES; ++q)
+        if ((armed >> q) & 1u)
+          mbar_wait(&full_bar[q], (armed_parity >> q) & 1u, p.wait_ns, nullptr);
+    }
+  } else if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer, gathered A
+    // Lane 0 waits for free stages, arms them and loads B; every lane then loads four of
+    // the tile's 128 rows of x (one gather4 each) into their own places in the swizzled
+    // stage, so the MMA sees the same layout as with a tile load of x_perm.
     int s = 0;
     uint32_t ph = 0;
     uint32_t armed = 0, armed_parity = 0;
@@ -173,34 +223,55 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
       int e, mb, nb;
       decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, p.mb_outer, e, mb, nb);
       const int row0 = p.seg_start[e] + mb * BM;
+      // rows past the bucket read token 0; the epilogue never stores them
+      int rr[4] = {0, 0, 0, 0};
+      const int valid = p.seg_count[e] - mb * BM;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 4 * lane + i;
+        if (r < valid) {
+          const int t = __ldg(p.a_rows + row0 + r);
+          rr[i] = (t >= 0 && t < p.a_rows_limit) ? t : 0;
+        }
+      }
       for (int kb = 0; kb < KB; ++kb) {
-        if (!mbar_wait(&empty_bar[s], ph ^ 1u, p.wait_ns, &abort_s)) {
-          if (!abort_s) record_error(p.status, DEV_TIMEOUT, 20, static_cast<unsigned long long>(tile));
+        int got = 1;
+        if (lane == 0) got = mbar_wait(&empty_bar[s], ph ^ 1u, p.wait_ns, &abort_s) ? 1 : 0;
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) {
+          if (lane == 0 && !abort_s)
+            record_error(p.status, DEV_TIMEOUT, 20, static_cast<unsigned long long>(tile));
           abort_s = 1;
           ok = false;
           break;
         }
         uint8_t* sa = smem + s * STAGE_BYTES;
         uint8_t* sb = sa + A_BYTES;
-        mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
+          if (GATED) {
+            tma_load_3d(sb, &tm_b0, &full_bar[s], kb * BK, nb * 128, e);
+            tma_load_3d(sb + B_BYTES / 2, &tm_b1, &full_bar[s], kb * BK, nb * 128, e);
+          } else {
+            tma_load_3d(sb, &tm_b0, &full_bar[s], kb * BK, nb * 256, e);
+          }
+        }
         armed |= 1u << s;
         armed_parity = (armed_parity & ~(1u << s)) | (ph << s);
-        tma_load_2d(sa, &tm_a, &full_bar[s], kb * BK, row0);
-        if (GATED) {
-          tma_load_3d(sb, &tm_b0, &full_bar[s], kb * BK, nb * 128, e);
-          tma_load_3d(sb + B_BYTES / 2, &tm_b1, &full_bar[s], kb * BK, nb * 128, e);
-        } else {
-          tma_load_3d(sb, &tm_b0, &full_bar[s], kb * BK, nb * 256, e);
-        }
+        __syncwarp();
+        tma_gather4(sa + lane * 4 * BK * 2, &tm_a, &full_bar[s], kb * BK, rr[0], rr[1], rr[2],
+                    rr[3]);
         if (++s == STAGES) {
           s = 0;
           ph ^= 1u;
         }
       }
     }
-    // every fill this thread armed must land before the block can exit
-    for (int q = 0; q < STAGES; ++q)
-      if ((armed >> q) & 1u) mbar_wait(&full_bar[q], (armed_parity >> q) & 1u, p.wait_ns, nullptr);
+    // every fill this warp armed must land before the block can exit
+    if (lane == 0)
+      for (int q = 0; q < STAGES; ++q)
+        if ((armed >> q) & 1u)
+          mbar_wait(&full_bar[q], (armed_parity >> q) & 1u, p.wait_ns, nullptr);
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------------- MMA issuer
     constexpr uint32_t idesc = idesc_bf16_f32(BM, MMA_N);
@@ -415,6 +486,18 @@ bool make_map_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows, K] bf16 row-major, box 1 row x 64 columns (for gather4), 128-byte swizzle
+bool make_map_gather(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K * 2)};
+  const cuuint32_t box[2] = {BK, 1};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // [E, N, K] bf16 weights, box 1 x box_n x 64, 128-byte swizzle
 bool make_map_weights(CUtensorMap* m, const void* base, int E, int64_t N, int64_t K,
                       int box_n) {
@@ -432,16 +515,18 @@ bool make_map_weights(CUtensorMap* m, const void* base, int E, int64_t N, int64_
 
 }  // namespace
 
-cudaError_t launch_ffn_tc(const Shape& s, const void* x_perm, const int32_t* offsets,
-                          const int32_t* kept, const void* wg, const void* wu, const void* wd,
-                          void* h, void* y, DevStatus* status, uint64_t wait_ns,
-                          cudaStream_t st, const char** why) {
+cudaError_t launch_ffn_tc(const Shape& s, const void* a, const int32_t* a_rows,
+                          const int32_t* offsets, const int32_t* kept, const void* wg,
+                          const void* wu, const void* wd, void* h, void* y, DevStatus* status,
+                          uint64_t wait_ns, cudaStream_t st, const char** why) {
   if (encode_fn() == nullptr) {
     *why = "cuTensorMapEncodeTiled is not available from the driver";
     return cudaErrorNotSupported;
   }
   CUtensorMap ta1, tg, tu, ta2, td;
-  if (!make_map_rows(&ta1, x_perm, s.max_rows, s.d) ||
+  const bool a_ok = a_rows != nullptr ? make_map_gather(&ta1, a, s.T, s.d)
+                                      : make_map_rows(&ta1, a, s.max_rows, s.d);
+  if (!a_ok ||
       !make_map_weights(&tg, wg, s.E, s.f, s.d, 128) ||
       !make_map_weights(&tu, wu, s.E, s.f, s.d, 128) ||
       !make_map_rows(&ta2, h, s.max_rows, s.f) ||
@@ -470,6 +555,8 @@ cudaError_t launch_ffn_tc(const Shape& s, const void* x_perm, const int32_t* off
   p1.out = static_cast<__nv_bfloat16*>(h);
   p1.status = status;
   p1.wait_ns = wait_ns;
+  p1.a_rows = a_rows;
+  p1.a_rows_limit = static_cast<int32_t>(s.T);
   int64_t g1 = row_blocks_bound * p1.n_blocks;
   if (g1 > sms) g1 = sms;
   grouped_gemm_tc_kernel<MODE_SWIGLU><<<static_cast<unsigned>(g1), THREADS, DYN_SMEM, st>>>(ta1, tg, tu,
@@ -478,6 +565,7 @@ cudaError_t launch_ffn_tc(const Shape& s, const void* x_perm, const int32_t* off
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
 
   TcParams p2 = p1;
+  p2.a_rows = nullptr;
   p2.K = static_cast<int>(s.f);
   p2.n_blocks = static_cast<int>((s.d + 255) / 256);
   p2.N_out = static_cast<int>(s.d);

@@ -77,13 +77,16 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
                             int32_t* assign_row, int32_t* token_of_row, void* x_perm,
                             int32_t* hist, DevStatus* status, uint64_t wait_ns,
                             cudaStream_t st);
-cudaError_t launch_ffn_simt(const Shape& s, const float* x_perm, const int32_t* offsets,
-                            const int32_t* kept, const float* wg, const float* wu,
-                            const float* wd, float* h, float* y, cudaStream_t st);
-cudaError_t launch_ffn_tc(const Shape& s, const void* x_perm, const int32_t* offsets,
-                          const int32_t* kept, const void* wg, const void* wu, const void* wd,
-                          void* h, void* y, DevStatus* status, uint64_t wait_ns,
-                          cudaStream_t st, const char** why);
+// Expert FFN.  `a` holds the gate/up GEMM's A rows: x_perm (a_rows == nullptr) or x itself,
+// bucket row r reading row a_rows[r] of x (token_of_row: dispatch without the permute copy).
+cudaError_t launch_ffn_simt(const Shape& s, const float* a, const int32_t* a_rows,
+                            const int32_t* offsets, const int32_t* kept, const float* wg,
+                            const float* wu, const float* wd, float* h, float* y,
+                            cudaStream_t st);
+cudaError_t launch_ffn_tc(const Shape& s, const void* a, const int32_t* a_rows,
+                          const int32_t* offsets, const int32_t* kept, const void* wg,
+                          const void* wu, const void* wd, void* h, void* y, DevStatus* status,
+                          uint64_t wait_ns, cudaStream_t st, const char** why);
 cudaError_t launch_combine(const Shape& s, const void* y_perm, const int32_t* assign_row,
                            const float* topk_w, void* out, cudaStream_t st);
 cudaError_t launch_stats(const Shape& s, const int32_t* routed, const int32_t* kept,

@@ -269,3 +269,61 @@ def test_kernel_launch_count_per_layer(shape, router_kernels):
     c0 = M.kernel_launch_count()
     run.all_stages()
     assert M.kernel_launch_count() - c0 == router_kernels + 3 + 2 + 1 + 1
+
+
+# ------------------------------------------------------------------ dispatch without x_perm
+GATHER = [
+    W.TINY_FP32,
+    W.reduced(W.MIXTRAL_8X7B, 1000, 512, 768),
+    W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256),
+    W.reduced(W.MIXTRAL_8X22B_MIXED, 1200, 384, 640, n_decode_tokens=16),
+    W.reduced(W.MIXTRAL_8X7B, 700, 256, 384, layout=W.LAYOUT_PADDED, capacity_factor=1.1),
+    _edge(1, 128, 128, 8, 2),
+    _edge(65, 128, 192, 1, 1),
+    _edge(300, 256, 128, 200, 6, cf=1.0),
+]
+
+
+@pytest.mark.parametrize("shape", GATHER, ids=lambda s: s.name)
+def test_gathered_ffn_equals_permuted_ffn_and_oracle(shape):
+    """moe_dispatch without x_perm + moe_expert_ffn_gather gives h, y_perm and out bitwise equal
+    to the permute path (the GEMM sees the same A tiles), and so matches the oracle too."""
+    run = GpuRun(shape)
+    st = run.all_stages()
+    ref_h, ref_y, ref_out = run.b.h.clone(), run.b.y_perm.clone(), run.b.out.clone()
+    b = run.b
+    b.h.zero_(), b.y_perm.zero_(), b.out.zero_()
+    M.moe_dispatch(run.cfg, None, b.topk_idx, b.routed_counts, b.kept_counts, b.expert_offsets,
+                   b.assign_row, b.token_of_row, None, run.ws)
+    M.moe_expert_ffn_gather(run.cfg, run.inp.x, b.token_of_row, b.expert_offsets, b.kept_counts,
+                            run.inp.w_gate, run.inp.w_up, run.inp.w_down, b.h, b.y_perm, run.ws)
+    run.combine()
+    M.moe_check_device_error(run.ws)
+    torch.cuda.synchronize()
+    used = int(b.expert_offsets[-1])
+    rows = torch.nonzero(b.token_of_row[:used] >= 0).flatten()
+    assert torch.equal(b.h[rows], ref_h[rows])
+    assert torch.equal(b.y_perm[rows], ref_y[rows])
+    assert torch.equal(b.out, ref_out)
+    r = check_routing(run)
+    check_ffn_rows(run, r)
+    check_combine(run, r)
+    check_layer_output(run, run.b.out, r)
+
+
+@pytest.mark.parametrize("shape", [W.reduced(W.MIXTRAL_8X7B, 1000, 512, 768), W.TINY_FP32],
+                         ids=lambda s: s.name)
+def test_layer_forward_without_x_perm(shape):
+    run = GpuRun(shape)
+    run.all_stages()
+    i = run.inp
+    layer = M.MoELayer(run.cfg, i.w_router, i.w_gate, i.w_up, i.w_down, i.logit_bias,
+                       gather=True)
+    assert layer.bufs.x_perm is None
+    c0 = M.kernel_launch_count()
+    out = layer(i.x)
+    launched = M.kernel_launch_count() - c0
+    M.moe_check_device_error(layer.ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out, run.b.out)
+    assert launched == 8    # the permute kernel is gone
