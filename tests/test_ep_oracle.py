@@ -1,0 +1,101 @@
+"""Pins of the expert-parallel oracle (no GPU): a hand-worked case, layout invariants, and
+the identity that drop-before-exchange EP equals the single-GPU layer on each rank's tokens."""
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import ep_oracle as EP
+from oracle import moe_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "ep_hand_g2_e4.json")
+
+
+def test_hand_case_layout_and_stats():
+    g = json.load(open(GOLDEN))
+    for case in g["cases"]:
+        lay = EP.recv_layout(g["kept_by_src"], case["expert_rank"])
+        assert lay["base"].tolist() == case["base"]
+        assert lay["offsets"] == case["offsets"]
+        assert lay["rows"] == case["rows"]
+        st = EP.ep_stats(g["kept_by_src"], case["expert_rank"], case["ranks_per_node"],
+                         g["row_bytes"])
+        for key, want in case["stats"].items():
+            got = st[key]
+            if isinstance(want, float):
+                assert got == pytest.approx(want, rel=1e-12, abs=1e-12), key
+            else:
+                assert got == want, key
+
+
+@pytest.mark.parametrize("G,E,seed", [(2, 8, 0), (4, 16, 1), (8, 256, 2), (3, 9, 3)])
+def test_layout_invariants(G, E, seed):
+    rng = np.random.default_rng(seed)
+    kept = rng.integers(0, 7, size=(G, E))
+    er = rng.permutation(EP.contiguous_placement(E, G))
+    lay = EP.recv_layout(kept, er)
+    for g in range(G):
+        mine = EP.local_experts(er, g)
+        offs = lay["offsets"][g]
+        assert offs[0] == 0 and len(offs) == len(mine) + 1
+        assert lay["rows"][g] == kept[:, mine].sum()
+        for i, e in enumerate(mine):
+            assert offs[i + 1] - offs[i] == kept[:, e].sum()
+            # inside the bucket, sources in ascending order, back to back
+            starts = [lay["base"][s, e] for s in range(G)]
+            assert starts[0] == offs[i]
+            for s in range(1, G):
+                assert starts[s] == starts[s - 1] + kept[s - 1, e]
+    st = EP.ep_stats(kept, er, 2, 100)
+    assert sum(st["rank_load"]) == st["total_assignments"] == kept.sum()
+    assert sum(st["bytes_sent"]) == sum(st["bytes_recv"]) == st["remote_bytes"]
+    assert st["remote_bytes"] == (kept.sum() - st["local_assignments"]) * 100
+    assert EP.ep_stats(kept, er, G, 100)["cross_node_bytes"] == 0
+    assert EP.ep_stats(kept, er, 1, 100)["cross_node_bytes"] == st["remote_bytes"]
+
+
+def _ranks(G, T, d, f, E, k, seed):
+    rng = np.random.default_rng(seed)
+    xs = [rng.standard_normal((T, d)) for _ in range(G)]
+    w_router = rng.standard_normal((d, E)) / np.sqrt(d)
+    wg = rng.standard_normal((E, f, d)) / np.sqrt(d)
+    wu = rng.standard_normal((E, f, d)) / np.sqrt(d)
+    wd = rng.standard_normal((E, d, f)) / np.sqrt(f)
+    return xs, w_router, wg, wu, wd
+
+
+@pytest.mark.parametrize("G,E,k,cf,permuted", [(2, 4, 2, 1.0, False), (4, 8, 2, 1.25, True),
+                                                (2, 8, 3, 0.0, True), (1, 4, 2, 1.0, False)])
+def test_ep_layer_equals_local_layer_per_rank(G, E, k, cf, permuted):
+    T, d, f = 24, 16, 12
+    xs, w_router, wg, wu, wd = _ranks(G, T, d, f, E, k, seed=G * 100 + E)
+    er = EP.contiguous_placement(E, G)
+    if permuted:
+        er = np.random.default_rng(7).permutation(er)
+    ep = EP.ep_layer(xs, w_router, None, wg, wu, wd, k, O.SOFTMAX, cf, er)
+    for s in range(G):
+        ref = O.moe_layer(xs[s], w_router, None, wg, wu, wd, k, O.SOFTMAX, cf)
+        np.testing.assert_allclose(ep["out"][s], ref["out"], rtol=1e-12, atol=1e-12)
+        # every kept pick's row in the owner's buffer is the token's x row
+        r = ep["routes"][s]
+        sr = ep["send_rows"][s]
+        for t in range(T):
+            for j in range(k):
+                if sr[t, j] >= 0:
+                    owner = er[r["idx"][t, j]]
+                    np.testing.assert_array_equal(ep["recv"][owner][sr[t, j]], xs[s][t])
+                else:
+                    assert r["assign_row"][t, j] < 0
+    if G == 1:
+        assert ep["stats"]["local_fraction"] == 1.0 and ep["stats"]["remote_bytes"] == 0
+    # each destination receives every kept row for its experts exactly once
+    for g in range(G):
+        used = np.zeros(ep["layout"]["rows"][g], dtype=int)
+        for s in range(G):
+            r, sr = ep["routes"][s], ep["send_rows"][s]
+            for t in range(T):
+                for j in range(k):
+                    if sr[t, j] >= 0 and er[r["idx"][t, j]] == g:
+                        used[sr[t, j]] += 1
+        assert (used == 1).all()
