@@ -40,7 +40,11 @@ L2_FLUSH_BYTES = 256 << 20
 GEMM_SOURCES = ("routing_dispatch_expert_warp_b200/csrc/moe_ffn_tc.cu",
                 "routing_dispatch_expert_warp_b200/csrc/moe_device.cuh",
                 "routing_dispatch_expert_warp_b200/csrc/moe_internal.h")
-RECORDED_GEMM_TRAFFIC = {}
+RECORDED_GEMM_TRAFFIC = {
+    ("mixtral8x7b_prefill_T4096", False): {
+        "bytes": 3669197056, "sources": "2260dce9c4829cdf",
+        "profile": "profiles/grouped_gemm_tc_mixtral8x7b_T4096_traffic.md"},
+}
 
 
 def gemm_source_hash() -> str:

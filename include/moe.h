@@ -55,7 +55,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 2
+#define MOE_ABI_VERSION 3
 #define MOE_MAX_EXPERTS 256
 #define MOE_MAX_TOPK 8
 
@@ -187,6 +187,68 @@ typedef struct moe_layer_buffers {
   void* out;                 /* [T, d_model] dtype                                       */
   moe_load_stats_t* stats;   /* device struct, or NULL to skip the statistics            */
 } moe_layer_buffers_t;
+
+/* ---------------------------------------------------------------- expert parallelism
+ *
+ * [EP-serving] "Deep dive" / "Technical insight": with expert parallelism each rank (one
+ * GPU) owns a subset of the experts, and every MoE layer runs two all-to-alls: dispatch
+ * sends each token's row to the owners of its experts, combine returns the results.
+ * [EP-checks] "Capacity factor changes quality, memory and the latency tail": tokens past
+ * the capacity are dropped before the exchange, so each rank routes, ranks and drops its
+ * own tokens with moe_route + moe_dispatch (x_perm may be NULL) exactly as on one GPU, and
+ * the EP result on a rank equals the single-GPU layer on that rank's tokens.
+ *
+ * No collective library moves the rows: every rank can address every rank's count
+ * matrix, receive buffer and result buffer (peer pointers through NVLink, opened with
+ * moe_ipc_open; or plain pointers when ranks share one device), and the exchange is fused
+ * into the kernels:
+ *   1. moe_ep_put_counts   my kept_counts -> row `rank` of every rank's count matrix
+ *   --- all ranks' step 1 complete (barrier) ---
+ *   2. moe_ep_plan         send_row of my picks; my local bucket table
+ *   3. moe_ep_dispatch     my token rows -> the owners' receive buffers
+ *   --- all ranks' step 3 complete (barrier) ---
+ *   4. moe_ep_expert_ffn   grouped GEMM of my experts over my receive buffer
+ *   --- all ranks' step 4 complete (barrier) ---
+ *   5. moe_ep_combine      out[t] from the owners' result buffers, in pick order
+ *   6. moe_ep_stats        the per-layer rank / node / pair-traffic record
+ *   --- all ranks' step 5 complete before anyone's next step 1 or 3 (barrier) ---
+ * The barriers are the caller's (for instance a stream-ordered all-reduce of one element
+ * across the ranks); when all ranks run on one device in one stream, stream order is the
+ * barrier.  Every kernel here is stream-ordered and never waits on another rank.
+ *
+ * Receive layout of rank g (rows of d_model elements): g's experts in ascending index; in
+ * each expert the rows of source rank 0, then 1, ...; in each source its slot order.
+ */
+typedef struct moe_ep_config {
+  int32_t world;           /* ranks, 1 .. 64                                               */
+  int32_t rank;            /* this rank, 0 .. world-1                                      */
+  int32_t ranks_per_node;  /* rank r sits on node r / ranks_per_node (>= 1)                */
+  int32_t n_local;         /* experts this rank owns (= count of expert_rank[e] == rank)   */
+  const int32_t* expert_rank; /* device [E]: owner of each expert (same on every rank)     */
+  int64_t recv_rows;       /* rows of every rank's receive / result buffer (same on all)   */
+} moe_ep_config_t;
+
+/* Per-layer record of [EP-checks] "Expert and GPU can be balanced differently", from the
+ * count matrix (identical on every rank after step 1).  Loads count kept assignments;
+ * bytes count rows x d_model x element size sent between different ranks in one dispatch
+ * (the combine returns the same bytes).  Pair figures run over every ordered pair of
+ * different ranks, empty pairs included; percentiles interpolate linearly (type 7). */
+typedef struct moe_ep_stats {
+  int32_t world, ranks_per_node, nodes, reserved;
+  int64_t total_assignments;   /* kept assignments of all ranks                            */
+  int64_t local_assignments;   /* token and expert on the same rank                        */
+  int64_t remote_bytes;        /* bytes crossing between ranks                              */
+  int64_t cross_node_bytes;    /* of those, between ranks of different nodes               */
+  double local_fraction;       /* local / total                                            */
+  double cross_node_fraction;  /* cross_node_bytes / remote_bytes                          */
+  double pair_bytes_p50, pair_bytes_p99, pair_bytes_max;
+  double rank_load_max, rank_load_mean, rank_load_max_minus_mean, rank_load_max_to_mean;
+  double node_load_max_to_mean;
+  int64_t rank_load[64];       /* assignments of the experts each rank owns                */
+  int64_t node_load[64];
+  int64_t bytes_sent[64];      /* remote bytes each rank sends in a dispatch               */
+  int64_t bytes_recv[64];
+} moe_ep_stats_t;
 
 /* ---------------------------------------------------------------- sizes */
 
@@ -351,6 +413,78 @@ void moe_set_wait_limit_ns(uint64_t ns);
  * completes, with the current limit, records MOE_ERR_TIMEOUT in the workspace status
  * word and returns.  Used to check that a run-out wait leaves the context usable. */
 moe_status_t moe_selftest_bounded_wait(void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------- expert parallelism calls
+ * All take the layer's moe_config_t (global E, this rank's T) and the moe_ep_config_t.
+ * Pointer tables (`mats`, `recv`, `ybuf`) are DEVICE arrays of `world` device pointers,
+ * indexed by rank, that this rank may dereference.  Errors as for the single-GPU calls;
+ * a row that would land at or past recv_rows is skipped and reported by
+ * moe_check_device_error as MOE_ERR_DEVICE_DATA. */
+
+/* Rows a receive buffer needs so that no distribution of picks can overflow it: world x
+ * min(T*min(k, n_local), n_local*C) (C = capacity; T*min(k, n_local) when dropless),
+ * with T the largest per-rank token count. */
+int64_t moe_ep_recv_rows_bound(const moe_config_t* cfg, const moe_ep_config_t* ep);
+
+/* Step 1.  mats[g] -> rank g's count matrix [world, E] int32; row `rank` receives
+ * kept_counts [E] (moe_dispatch's output). */
+moe_status_t moe_ep_put_counts(const moe_config_t* cfg, const moe_ep_config_t* ep,
+                               const int32_t* kept_counts, int32_t* const* mats, void* stream);
+
+/* Step 2.  From this rank's full count matrix [world, E]:
+ *   send_row [T, k]         row of pick (t, j) in its owner's receive buffer, -1 dropped
+ *                           (= the owner's bucket start for the expert + the rows of lower
+ *                           source ranks + the pick's slot on this rank);
+ *   recv_offsets [n_local+1] start of each local expert's bucket in this rank's buffer
+ *                           ([n_local] = rows received); recv_counts [n_local] its rows.
+ * Buckets are cut at recv_rows (reported by moe_check_device_error as MOE_ERR_DEVICE_DATA),
+ * so the local GEMM never reaches past the buffer.
+ * topk_idx, assign_row, expert_offsets: this rank's moe_route / moe_dispatch outputs. */
+moe_status_t moe_ep_plan(const moe_config_t* cfg, const moe_ep_config_t* ep,
+                         const int32_t* count_mat, const int32_t* topk_idx,
+                         const int32_t* assign_row, const int32_t* expert_offsets,
+                         int32_t* send_row, int32_t* recv_offsets, int32_t* recv_counts,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* Step 3.  recv[g][send_row[t, j], :] = x[t, :] for every kept pick, g = the owner of
+ * topk_idx[t, j]; each row of x is read once.  recv buffers: [recv_rows, d_model] dtype. */
+moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const moe_ep_config_t* ep,
+                             const void* x, const int32_t* topk_idx, const int32_t* send_row,
+                             void* const* recv, void* ws, size_t ws_bytes, void* stream);
+
+/* Step 4.  moe_expert_ffn over this rank's receive buffer with its n_local experts'
+ * weights (w_gate_local, w_up_local [n_local, d_ff, d_model]; w_down_local [n_local,
+ * d_model, d_ff], local expert i = the i-th expert this rank owns in ascending index):
+ * h [recv_rows, d_ff], y_recv [recv_rows, d_model]. */
+moe_status_t moe_ep_expert_ffn(const moe_config_t* cfg, const moe_ep_config_t* ep,
+                               const void* recv_x, const int32_t* recv_offsets,
+                               const int32_t* recv_counts, const void* w_gate_local,
+                               const void* w_up_local, const void* w_down_local, void* h,
+                               void* y_recv, void* ws, size_t ws_bytes, void* stream);
+
+/* Step 5.  out[t, :] = sum over kept picks j, in pick order, of topk_w[t, j] *
+ * ybuf[g][send_row[t, j], :] (g = owner), fp32 accumulation: bitwise what moe_combine
+ * gives on one GPU. */
+moe_status_t moe_ep_combine(const moe_config_t* cfg, const moe_ep_config_t* ep,
+                            const void* const* ybuf, const int32_t* topk_idx,
+                            const int32_t* send_row, const float* topk_w, void* out,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Step 6.  The EP record from the count matrix; host_out non-NULL copies it to the host
+ * and synchronises the stream. */
+moe_status_t moe_ep_stats(const moe_config_t* cfg, const moe_ep_config_t* ep,
+                          const int32_t* count_mat, moe_ep_stats_t* dev_out,
+                          moe_ep_stats_t* host_out, void* stream);
+
+/* Peer memory for multi-process EP.  moe_ipc_handle gives the IPC handle (64 bytes) of the
+ * device allocation that contains dev_ptr and dev_ptr's byte offset in it (allocators hand
+ * out pieces of larger allocations); another process maps the allocation with
+ * moe_ipc_open and adds the offset, and unmaps it with moe_ipc_close.  Thin wrappers of
+ * the CUDA IPC calls; MOE_ERR_CUDA on failure. */
+moe_status_t moe_ipc_handle(const void* dev_ptr, unsigned char handle_out[64],
+                            int64_t* offset_out);
+moe_status_t moe_ipc_open(const unsigned char handle[64], void** dev_ptr_out);
+moe_status_t moe_ipc_close(void* dev_ptr);
 
 /* MOE_ABI_VERSION of the loaded library. */
 int32_t moe_abi_version(void);

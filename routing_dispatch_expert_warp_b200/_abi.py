@@ -56,6 +56,36 @@ class MoeLayerBuffers(ctypes.Structure):
                 ("y_perm", c_vp), ("out", c_vp), ("stats", c_vp)]
 
 
+class MoeEpConfig(ctypes.Structure):
+    _fields_ = [("world", c_i32), ("rank", c_i32), ("ranks_per_node", c_i32),
+                ("n_local", c_i32), ("expert_rank", c_vp), ("recv_rows", c_i64)]
+
+
+MOE_MAX_RANKS = 64
+
+
+class MoeEpStats(ctypes.Structure):
+    _fields_ = [("world", c_i32), ("ranks_per_node", c_i32), ("nodes", c_i32),
+                ("reserved", c_i32), ("total_assignments", c_i64),
+                ("local_assignments", c_i64), ("remote_bytes", c_i64),
+                ("cross_node_bytes", c_i64), ("local_fraction", c_f64),
+                ("cross_node_fraction", c_f64), ("pair_bytes_p50", c_f64),
+                ("pair_bytes_p99", c_f64), ("pair_bytes_max", c_f64),
+                ("rank_load_max", c_f64), ("rank_load_mean", c_f64),
+                ("rank_load_max_minus_mean", c_f64), ("rank_load_max_to_mean", c_f64),
+                ("node_load_max_to_mean", c_f64),
+                ("rank_load", c_i64 * MOE_MAX_RANKS), ("node_load", c_i64 * MOE_MAX_RANKS),
+                ("bytes_sent", c_i64 * MOE_MAX_RANKS), ("bytes_recv", c_i64 * MOE_MAX_RANKS)]
+
+    def as_dict(self) -> dict:
+        d = {name: getattr(self, name) for name, _ in self._fields_}
+        for key in ("rank_load", "bytes_sent", "bytes_recv"):
+            d[key] = list(getattr(self, key))[: self.world]
+        d["node_load"] = list(self.node_load)[: self.nodes]
+        d.pop("reserved")
+        return d
+
+
 P = ctypes.POINTER
 # name -> (restype, argtypes); every function declared in include/moe.h
 PROTOTYPES = {
@@ -82,6 +112,20 @@ PROTOTYPES = {
     "moe_status_string": (ctypes.c_char_p, [c_i32]),
     "moe_set_wait_limit_ns": (None, [ctypes.c_uint64]),
     "moe_selftest_bounded_wait": (c_i32, [c_vp, c_sz, c_vp]),
+    "moe_ep_recv_rows_bound": (c_i64, [P(MoeConfig), P(MoeEpConfig)]),
+    "moe_ep_put_counts": (c_i32, [P(MoeConfig), P(MoeEpConfig), c_vp, c_vp, c_vp]),
+    "moe_ep_plan": (c_i32, [P(MoeConfig), P(MoeEpConfig), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                            c_vp, c_vp, c_sz, c_vp]),
+    "moe_ep_dispatch": (c_i32, [P(MoeConfig), P(MoeEpConfig), c_vp, c_vp, c_vp, c_vp, c_vp,
+                                c_sz, c_vp]),
+    "moe_ep_expert_ffn": (c_i32, [P(MoeConfig), P(MoeEpConfig), c_vp, c_vp, c_vp, c_vp, c_vp,
+                                  c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "moe_ep_combine": (c_i32, [P(MoeConfig), P(MoeEpConfig), c_vp, c_vp, c_vp, c_vp, c_vp,
+                               c_vp, c_sz, c_vp]),
+    "moe_ep_stats": (c_i32, [P(MoeConfig), P(MoeEpConfig), c_vp, c_vp, P(MoeEpStats), c_vp]),
+    "moe_ipc_handle": (c_i32, [c_vp, ctypes.c_char_p, P(c_i64)]),
+    "moe_ipc_open": (c_i32, [ctypes.c_char_p, P(c_vp)]),
+    "moe_ipc_close": (c_i32, [c_vp]),
     "moe_abi_version": (c_i32, []),
     "moe_kernel_launch_count": (ctypes.c_uint64, []),
 }

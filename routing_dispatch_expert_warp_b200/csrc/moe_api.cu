@@ -3,6 +3,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <string.h>
 
 #include <atomic>
 #include <mutex>
@@ -152,6 +153,8 @@ WsLayout workspace_layout(const Shape& s) {
   l.router_tc = off;
   l.router_tc_bytes = round_up(router_tc_workspace_bytes(s));
   off += l.router_tc_bytes;
+  l.ep_base = off;
+  off += round_up(static_cast<size_t>(s.E) * sizeof(int32_t));
   l.total = off;
   return l;
 }
@@ -460,6 +463,229 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_layer_inputs_t
   return st;
 }
 
+}  // extern "C"
+
+namespace {
+
+moe_status_t check_ep(const moe_config_t* cfg, const moe_ep_config_t* ep, Shape* s,
+                      const char* name) {
+  moe_status_t st = check_config(cfg, s);
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(ep != nullptr, "%s: ep is NULL", name);
+  MOE_REQUIRE(ep->world >= 1 && ep->world <= kMaxDevices, "%s: world must be 1..%d", name,
+              kMaxDevices);
+  MOE_REQUIRE(ep->rank >= 0 && ep->rank < ep->world, "%s: rank outside [0, world)", name);
+  MOE_REQUIRE(ep->ranks_per_node >= 1, "%s: ranks_per_node must be >= 1", name);
+  MOE_REQUIRE(ep->n_local >= 1 && ep->n_local <= s->E, "%s: n_local must be 1..E", name);
+  MOE_REQUIRE(ep->expert_rank != nullptr, "%s: expert_rank is NULL", name);
+  MOE_REQUIRE(ep->recv_rows >= 0 && ep->recv_rows <= INT32_MAX,
+              "%s: recv_rows must be in [0, 2^31)", name);
+  return MOE_OK;
+}
+
+int64_t ep_bound(const Shape& s, const moe_ep_config_t* ep) {
+  const int64_t per_token = s.k < ep->n_local ? s.k : ep->n_local;
+  int64_t per_src = s.T * per_token;
+  if (s.C >= 0 && static_cast<int64_t>(ep->n_local) * s.C < per_src)
+    per_src = static_cast<int64_t>(ep->n_local) * s.C;
+  return per_src * ep->world;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t moe_ep_recv_rows_bound(const moe_config_t* cfg, const moe_ep_config_t* ep) {
+  Shape s;
+  moe_ep_config_t tmp;
+  if (ep == nullptr) return -2;
+  tmp = *ep;
+  if (tmp.expert_rank == nullptr) tmp.expert_rank = reinterpret_cast<const int32_t*>(16);
+  if (check_ep(cfg, &tmp, &s, "moe_ep_recv_rows_bound") != MOE_OK) return -2;
+  return ep_bound(s, ep);
+}
+
+moe_status_t moe_ep_put_counts(const moe_config_t* cfg, const moe_ep_config_t* ep,
+                               const int32_t* kept_counts, int32_t* const* mats, void* stream) {
+  Shape s;
+  moe_status_t st = check_ep(cfg, ep, &s, "moe_ep_put_counts");
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(kept_counts && mats, "moe_ep_put_counts: NULL pointer");
+  cudaError_t err = launch_ep_put_counts(s, kept_counts, ep->rank, ep->world, mats,
+                                         static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ep_put_counts launch");
+  return MOE_OK;
+}
+
+moe_status_t moe_ep_plan(const moe_config_t* cfg, const moe_ep_config_t* ep,
+                         const int32_t* count_mat, const int32_t* topk_idx,
+                         const int32_t* assign_row, const int32_t* expert_offsets,
+                         int32_t* send_row, int32_t* recv_offsets, int32_t* recv_counts,
+                         void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  moe_status_t st = check_ep(cfg, ep, &s, "moe_ep_plan");
+  if (st != MOE_OK) return st;
+  WsLayout lay;
+  if ((st = check_ws(s, ws, ws_bytes, &lay)) != MOE_OK) return st;
+  MOE_REQUIRE(count_mat && topk_idx && assign_row && expert_offsets && send_row && recv_offsets &&
+                  recv_counts,
+              "moe_ep_plan: NULL pointer");
+  int32_t* base = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + lay.ep_base);
+  cudaError_t err = launch_ep_plan(s, count_mat, ep->expert_rank, ep->world, ep->rank,
+                                   ep->n_local, ep->recv_rows, topk_idx, assign_row, expert_offsets, base,
+                                   send_row, recv_offsets, recv_counts, ws_status(ws, lay),
+                                   static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ep_plan launch");
+  return MOE_OK;
+}
+
+moe_status_t moe_ep_dispatch(const moe_config_t* cfg, const moe_ep_config_t* ep,
+                             const void* x, const int32_t* topk_idx, const int32_t* send_row,
+                             void* const* recv, void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  moe_status_t st = check_ep(cfg, ep, &s, "moe_ep_dispatch");
+  if (st != MOE_OK) return st;
+  WsLayout lay;
+  if ((st = check_ws(s, ws, ws_bytes, &lay)) != MOE_OK) return st;
+  MOE_REQUIRE(x && topk_idx && send_row && recv, "moe_ep_dispatch: NULL pointer");
+  MOE_REQUIRE(aligned16(x), "moe_ep_dispatch: x must be 16-byte aligned");
+  cudaError_t err = launch_ep_dispatch(s, x, topk_idx, send_row, ep->expert_rank, ep->world,
+                                       recv, ep->recv_rows, ws_status(ws, lay),
+                                       static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ep_dispatch launch");
+  return MOE_OK;
+}
+
+moe_status_t moe_ep_expert_ffn(const moe_config_t* cfg, const moe_ep_config_t* ep,
+                               const void* recv_x, const int32_t* recv_offsets,
+                               const int32_t* recv_counts, const void* w_gate_local,
+                               const void* w_up_local, const void* w_down_local, void* h,
+                               void* y_recv, void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  moe_status_t st = check_ep(cfg, ep, &s, "moe_ep_expert_ffn");
+  if (st != MOE_OK) return st;
+  WsLayout lay;
+  if ((st = check_ws(s, ws, ws_bytes, &lay)) != MOE_OK) return st;
+  MOE_REQUIRE(recv_x && recv_offsets && recv_counts && w_gate_local && w_up_local &&
+                  w_down_local && h && y_recv,
+              "moe_ep_expert_ffn: NULL pointer");
+  MOE_REQUIRE(aligned16(recv_x) && aligned16(w_gate_local) && aligned16(w_up_local) &&
+                  aligned16(w_down_local) && aligned16(h) && aligned16(y_recv),
+              "moe_ep_expert_ffn: tensors must be 16-byte aligned");
+  if (ep->recv_rows == 0) return MOE_OK;
+  // the local grouped GEMM: n_local buckets in a buffer of recv_rows rows; a bucket holds
+  // at most world x min(T, C) rows
+  Shape sl = s;
+  sl.E = ep->n_local;
+  sl.max_rows = ep->recv_rows;
+  sl.T = s.T * ep->world;
+  sl.C = s.C >= 0 ? s.C * ep->world : -1;
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  cudaError_t err;
+  if (s.dtype == MOE_F32) {
+    err = launch_ffn_simt(sl, static_cast<const float*>(recv_x), nullptr, recv_offsets,
+                          recv_counts, static_cast<const float*>(w_gate_local),
+                          static_cast<const float*>(w_up_local),
+                          static_cast<const float*>(w_down_local), static_cast<float*>(h),
+                          static_cast<float*>(y_recv), strm);
+    if (err != cudaSuccess) return cuda_fail(err, "moe_ep_expert_ffn (fp32) launch");
+    return MOE_OK;
+  }
+  if (s.d % 64 != 0 || s.f % 64 != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "bf16 expert FFN needs d_model and d_ff multiples of 64");
+  const char* why = "";
+  err = launch_ffn_tc(sl, recv_x, nullptr, recv_offsets, recv_counts, w_gate_local, w_up_local,
+                      w_down_local, h, y_recv, ws_status(ws, lay), g_wait_ns.load(), strm, &why);
+  if (err != cudaSuccess) {
+    if (why[0]) return fail(MOE_ERR_CUDA, "moe_ep_expert_ffn: %s", why);
+    return cuda_fail(err, "moe_ep_expert_ffn (bf16) launch");
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_ep_combine(const moe_config_t* cfg, const moe_ep_config_t* ep,
+                            const void* const* ybuf, const int32_t* topk_idx,
+                            const int32_t* send_row, const float* topk_w, void* out,
+                            void* ws, size_t ws_bytes, void* stream) {
+  Shape s;
+  moe_status_t st = check_ep(cfg, ep, &s, "moe_ep_combine");
+  if (st != MOE_OK) return st;
+  WsLayout lay;
+  if ((st = check_ws(s, ws, ws_bytes, &lay)) != MOE_OK) return st;
+  MOE_REQUIRE(ybuf && topk_idx && send_row && topk_w && out, "moe_ep_combine: NULL pointer");
+  MOE_REQUIRE(aligned16(out), "moe_ep_combine: out must be 16-byte aligned");
+  cudaError_t err = launch_ep_combine(s, ybuf, topk_idx, send_row, ep->expert_rank, ep->world,
+                                      ep->recv_rows, topk_w, out,
+                                      static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ep_combine launch");
+  return MOE_OK;
+}
+
+moe_status_t moe_ep_stats(const moe_config_t* cfg, const moe_ep_config_t* ep,
+                          const int32_t* count_mat, moe_ep_stats_t* dev_out,
+                          moe_ep_stats_t* host_out, void* stream) {
+  Shape s;
+  moe_status_t st = check_ep(cfg, ep, &s, "moe_ep_stats");
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(count_mat && dev_out, "moe_ep_stats: NULL pointer");
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  cudaError_t err = launch_ep_stats(s, count_mat, ep->expert_rank, ep->world,
+                                    ep->ranks_per_node, dev_out, strm);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ep_stats launch");
+  if (host_out != nullptr) {
+    err = cudaMemcpyAsync(host_out, dev_out, sizeof(moe_ep_stats_t), cudaMemcpyDeviceToHost,
+                          strm);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(strm);
+    if (err != cudaSuccess) return cuda_fail(err, "moe_ep_stats host copy");
+  }
+  return MOE_OK;
+}
+
+moe_status_t moe_ipc_handle(const void* dev_ptr, unsigned char handle_out[64],
+                            int64_t* offset_out) {
+  MOE_REQUIRE(dev_ptr && handle_out && offset_out, "moe_ipc_handle: NULL pointer");
+  typedef CUresult (*RangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+  static RangeFn range = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuMemGetAddressRange", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      range = reinterpret_cast<RangeFn>(fn);
+  });
+  if (range == nullptr)
+    return fail(MOE_ERR_CUDA, "moe_ipc_handle: cuMemGetAddressRange is not available");
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (range(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS)
+    return fail(MOE_ERR_CUDA, "moe_ipc_handle: pointer is not device memory of this process");
+  cudaIpcMemHandle_t hnd;
+  cudaError_t err = cudaIpcGetMemHandle(&hnd, reinterpret_cast<void*>(base));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ipc_handle");
+  static_assert(sizeof(hnd) == 64, "CUDA IPC handles are 64 bytes");
+  memcpy(handle_out, &hnd, sizeof(hnd));
+  *offset_out = static_cast<int64_t>(reinterpret_cast<CUdeviceptr>(dev_ptr) - base);
+  return MOE_OK;
+}
+
+moe_status_t moe_ipc_open(const unsigned char handle[64], void** dev_ptr_out) {
+  MOE_REQUIRE(handle && dev_ptr_out, "moe_ipc_open: NULL pointer");
+  cudaIpcMemHandle_t hnd;
+  memcpy(&hnd, handle, sizeof(hnd));
+  cudaError_t err = cudaIpcOpenMemHandle(dev_ptr_out, hnd, cudaIpcMemLazyEnablePeerAccess);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ipc_open");
+  return MOE_OK;
+}
+
+moe_status_t moe_ipc_close(void* dev_ptr) {
+  MOE_REQUIRE(dev_ptr, "moe_ipc_close: NULL pointer");
+  cudaError_t err = cudaIpcCloseMemHandle(dev_ptr);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_ipc_close");
+  return MOE_OK;
+}
+
 moe_status_t moe_check_device_error(void* ws, size_t ws_bytes, void* stream) {
   MOE_REQUIRE(ws != nullptr && ws_bytes >= sizeof(DevStatus), "moe_check_device_error: bad workspace");
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
@@ -473,6 +699,10 @@ moe_status_t moe_check_device_error(void* ws, size_t ws_bytes, void* stream) {
   if (err != cudaSuccess) return cuda_fail(err, "moe_check_device_error clear");
   if (h.code == DEV_TIMEOUT)
     return fail(MOE_ERR_TIMEOUT, "a device wait ran out (site %u, item %llu)", h.where,
+                (unsigned long long)h.info);
+  if (h.code == DEV_RECV_OVERFLOW)
+    return fail(MOE_ERR_DEVICE_DATA,
+                "expert-parallel row past the receive buffer's recv_rows (pick %llu)",
                 (unsigned long long)h.info);
   return fail(MOE_ERR_DEVICE_DATA, "invalid expert index in topk_idx (flat index %llu)",
               (unsigned long long)h.info);

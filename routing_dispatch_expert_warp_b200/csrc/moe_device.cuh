@@ -18,7 +18,12 @@ struct DevStatus {
   unsigned int where;       // which wait / check fired (kernel-specific tag)
   unsigned long long info;  // e.g. the offending index
 };
-enum DevError : unsigned int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_EXPERT = 2 };
+enum DevError : unsigned int {
+  DEV_OK = 0,
+  DEV_TIMEOUT = 1,
+  DEV_BAD_EXPERT = 2,
+  DEV_RECV_OVERFLOW = 3  // an expert-parallel row would land past the receive buffer
+};
 
 __device__ __forceinline__ void record_error(DevStatus* st, unsigned int code,
                                              unsigned int where, unsigned long long info) {

@@ -36,6 +36,7 @@ struct WsLayout {
   size_t partials_bytes;
   size_t router_tc;     // bf16 split of W_r for the tensor-core router
   size_t router_tc_bytes;
+  size_t ep_base;       // [E] int32: first row of this rank's rows per expert at the owner
   size_t total;
 };
 
@@ -94,6 +95,27 @@ cudaError_t launch_stats(const Shape& s, const int32_t* routed, const int32_t* k
 cudaError_t launch_wait_selftest(DevStatus* status, uint64_t wait_ns, cudaStream_t st);
 
 int sm_count();
+
+// Expert parallelism over peer (or shared-device) memory.
+cudaError_t launch_ep_put_counts(const Shape& s, const int32_t* kept, int rank, int world,
+                                 int32_t* const* mats, cudaStream_t st);
+cudaError_t launch_ep_plan(const Shape& s, const int32_t* mat, const int32_t* expert_rank,
+                           int world, int rank, int n_local, int64_t recv_rows,
+                           const int32_t* topk_idx,
+                           const int32_t* assign_row, const int32_t* expert_offsets,
+                           int32_t* base, int32_t* send_row, int32_t* recv_offsets,
+                           int32_t* recv_counts, DevStatus* status, cudaStream_t st);
+cudaError_t launch_ep_dispatch(const Shape& s, const void* x, const int32_t* topk_idx,
+                               const int32_t* send_row, const int32_t* expert_rank, int world,
+                               void* const* recv, int64_t recv_rows, DevStatus* status,
+                               cudaStream_t st);
+cudaError_t launch_ep_combine(const Shape& s, const void* const* ybuf, const int32_t* topk_idx,
+                              const int32_t* send_row, const int32_t* expert_rank, int world,
+                              int64_t recv_rows, const float* topk_w, void* out,
+                              cudaStream_t st);
+cudaError_t launch_ep_stats(const Shape& s, const int32_t* mat, const int32_t* expert_rank,
+                            int world, int ranks_per_node, moe_ep_stats_t* out,
+                            cudaStream_t st);
 
 // Process-wide count of this library's kernel launches (every launch site calls it once).
 void note_launch();

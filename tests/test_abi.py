@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(lib):
     assert not missing, missing
     for n in names:
         assert getattr(lib, n) is not None
-    assert lib.moe_abi_version() == 2
+    assert lib.moe_abi_version() == 3
 
 
 def test_struct_layout_matches_header(tmp_path):
@@ -57,6 +57,8 @@ int main(void) {
          offsetof(moe_load_stats_t, p50), offsetof(moe_load_stats_t, dropped_by_rank));
   printf("%zu %zu\\n", offsetof(moe_layer_inputs_t, bias_row_stride),
          offsetof(moe_layer_buffers_t, stats));
+  printf("%zu %zu %zu %zu\\n", sizeof(moe_ep_config_t), sizeof(moe_ep_stats_t),
+         offsetof(moe_ep_config_t, recv_rows), offsetof(moe_ep_stats_t, bytes_recv));
   return 0;
 }
 """)
@@ -69,7 +71,9 @@ int main(void) {
             ctypes.sizeof(_abi.MoeLayerInputs), ctypes.sizeof(_abi.MoeLayerBuffers),
             _abi.MoeConfig.capacity_factor.offset, _abi.MoeLoadStats.p50.offset,
             _abi.MoeLoadStats.dropped_by_rank.offset, _abi.MoeLayerInputs.bias_row_stride.offset,
-            _abi.MoeLayerBuffers.stats.offset]
+            _abi.MoeLayerBuffers.stats.offset,
+            ctypes.sizeof(_abi.MoeEpConfig), ctypes.sizeof(_abi.MoeEpStats),
+            _abi.MoeEpConfig.recv_rows.offset, _abi.MoeEpStats.bytes_recv.offset]
     assert got == want
 
 
