@@ -133,6 +133,35 @@ def algorithmic_work(shape, kept_total: int) -> dict:
     }
 
 
+def gemm_roofline(shape, kept_total: int, touched: int, ffn_ms: float, peaks: dict) -> dict:
+    """The grouped GEMM (both launches) against the roof that binds it.  FLOPs: 6 d f per kept
+    row.  Bytes: the weights of every expert that got rows (3 d f each), plus the kept rows of
+    x_perm read, h written and read back, y_perm written.  The binding roof is the one whose
+    time at the measured peak is longer (tensor for prefill, HBM for decode)."""
+    d, f = shape.d_model, shape.d_ff
+    s = 2 if shape.dtype == W.BF16 else 4
+    flops = 6.0 * d * f * kept_total
+    nbytes = touched * 3.0 * d * f * s + kept_total * (2.0 * d * s + 2.0 * f * s)
+    sec = ffn_ms * 1e-3
+    t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    base = {"kernel": "grouped_gemm_tc_kernel (expert FFN: gate/up + down launches)",
+            "algorithmic_flops_per_step": flops, "algorithmic_bytes_per_step": nbytes,
+            "experts_touched": touched}
+    if t_hbm > t_tensor:
+        achieved = nbytes / sec / 1e9
+        base.update(bound="hbm", achieved=achieved, peak=peaks["hbm_gbs"], unit="GB/s",
+                    frac=achieved / peaks["hbm_gbs"], peak_source=f"{peaks['source']} HBM copy")
+        return base
+    achieved = flops / sec / 1e12
+    base.update(bound="tensor", achieved=achieved, peak=peaks["bf16_tflops"], unit="TFLOP/s",
+                frac=achieved / peaks["bf16_tflops"],
+                peak_source=f"{peaks['source']} bf16 burst",
+                frac_of_sustained=(achieved / peaks["bf16_tflops_sustained"]
+                                   if peaks.get("bf16_tflops_sustained") else None))
+    return base
+
+
 def rank_shape(shape, rank: int):
     """Replicas draw different token batches (and weights) per rank: seed + 1000 * rank."""
     return shape.replace(seed=shape.seed + 1000 * rank) if rank else shape
@@ -234,7 +263,8 @@ def run_gpu(args) -> None:
     work = algorithmic_work(shape, kept_total)
     peaks = measured_peaks()
     ffn_ms = sum(per_stage["expert_ffn"]) / args.steps
-    tflops = work["gemm_flops"] / (ffn_ms * 1e-3) / 1e12
+    touched = int((b.kept_counts > 0).sum())
+    roof = gemm_roofline(shape, kept_total, touched, ffn_ms, peaks)
     gbs = lambda byts, n: byts / (sum(per_stage[n]) / args.steps * 1e-3) / 1e9
 
     # end to end through the public API: pinned host x -> device, layer, device -> host out
@@ -283,17 +313,10 @@ def run_gpu(args) -> None:
                        "dispatch": ("no x_perm: gate/up GEMM gathers rows of x" if args.gather
                                     else "permuted copy x_perm"),
                        "parallelism": f"replicas x{world} (EP=1, no exchange)"},
-            "roofline": {
-                "kernel": "grouped_gemm_tc_kernel (expert FFN: gate/up + down launches)",
-                "bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
-                "peak_source": f"{peaks['source']} bf16 burst",
-                "frac_of_sustained": (tflops / peaks["bf16_tflops_sustained"]
-                                      if peaks.get("bf16_tflops_sustained") else None),
-                "traffic": (recorded_traffic(shape.name, args.gather) or {}).get("bytes"),
-                "traffic_source": (recorded_traffic(shape.name, args.gather) or {}).get("profile"),
-                "algorithmic_flops_per_step": work["gemm_flops"],
-            },
+            "roofline": dict(
+                roof,
+                traffic=(recorded_traffic(shape.name, args.gather) or {}).get("bytes"),
+                traffic_source=(recorded_traffic(shape.name, args.gather) or {}).get("profile")),
             "stages_ms": {n: sum(v) / args.steps for n, v in per_stage.items()},
             "stage_bandwidth": {
                 "route": {"GB/s": gbs(work["route_bytes"], "route"),
