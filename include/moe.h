@@ -347,7 +347,8 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
 
 /*
  * moe_expert_ffn without the permuted copy of x: the gate/up GEMM reads bucket row r as
- * x[token_of_row[r], :] (TMA row gathers straight from x), so dispatch need not write
+ * x[token_of_row[r], :] (16-byte asynchronous copies straight from x into the GEMM's
+ * swizzled operand tiles), so dispatch need not write
  * x_perm.  This is the dispatch half of the fused dispatch-compute-combine kernels that
  * [EP-serving] names as the direction of expert parallelism (its closing section on the
  * future of EP serving, in the Wolof edition of the page).  Results are identical to
@@ -361,6 +362,27 @@ moe_status_t moe_expert_ffn_gather(const moe_config_t* cfg, const void* x,
                                    const int32_t* kept_counts, const void* w_gate,
                                    const void* w_up, const void* w_down, void* h, void* y_perm,
                                    void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_expert_ffn followed by moe_combine, with the combine fused into the down GEMM: as
+ * each bucket row's 256-column block of y_perm is stored, its token's counter for that
+ * block is bumped, and the thread completing the count sums the token's kept rows of the
+ * block in pick order (fp32) into out.  This is the combine half of the fused
+ * dispatch-compute-combine kernels that [EP-serving] names as the direction of expert
+ * parallelism (its closing section on the future of EP serving, Wolof edition); the
+ * combine's memory traffic overlaps the tensor-core work.  out is bitwise what
+ * moe_combine gives; y_perm and h are written as by moe_expert_ffn.  A rows come from
+ * x_perm, or, when x_perm is NULL, straight from x through token_of_row (as
+ * moe_expert_ffn_gather).  fp32 layers run moe_combine's kernel after the FFN instead.
+ * Uses the workspace's counters; calls on one workspace must not overlap.
+ */
+moe_status_t moe_expert_ffn_combine(const moe_config_t* cfg, const void* x, const void* x_perm,
+                                    const int32_t* token_of_row, const int32_t* expert_offsets,
+                                    const int32_t* kept_counts, const void* w_gate,
+                                    const void* w_up, const void* w_down, void* h,
+                                    void* y_perm, const int32_t* assign_row,
+                                    const float* topk_w, void* out, void* ws, size_t ws_bytes,
+                                    void* stream);
 
 /*
  * Combine ([EP-serving] "Deep dive": results shuffled back; [EP-checks]: combine, unpack):
@@ -386,7 +408,9 @@ moe_status_t moe_load_stats(const moe_config_t* cfg, const int32_t* routed_count
 /*
  * The whole layer: moe_route, moe_dispatch, moe_expert_ffn, moe_combine and (when
  * bufs->stats is not NULL) moe_load_stats, enqueued back to back on one stream without a
- * host synchronisation.  Returns the first failing stage's status.
+ * host synchronisation.  bufs->x_perm NULL: dispatch writes no permuted copy and the
+ * gate/up GEMM gathers rows of x (moe_expert_ffn_gather).  Returns the first failing
+ * stage's status.
  */
 moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_layer_inputs_t* in,
                                const moe_layer_buffers_t* bufs, void* ws, size_t ws_bytes,

@@ -24,7 +24,7 @@ DROP_TOKEN_ORDER, DROP_PICK_RANK = 0, 1
 
 __all__ = ["MoEError", "make_config", "workspace_size", "capacity", "max_rows",
            "alloc_workspace", "moe_route", "moe_dispatch", "moe_dispatch_static_scratch",
-           "moe_expert_ffn", "moe_expert_ffn_gather", "moe_combine",
+           "moe_expert_ffn", "moe_expert_ffn_gather", "moe_expert_ffn_combine", "moe_combine",
            "moe_load_stats", "moe_layer_forward", "moe_check_device_error",
            "moe_selftest_bounded_wait", "set_wait_limit_ns", "kernel_launch_count",
            "LayerBuffers", "MoELayer"]
@@ -134,6 +134,17 @@ def moe_expert_ffn_gather(cfg, x, token_of_row, expert_offsets, kept_counts, w_g
                                        _ptr(expert_offsets), _ptr(kept_counts), _ptr(w_gate),
                                        _ptr(w_up), _ptr(w_down), _ptr(h), _ptr(y_perm),
                                        _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_expert_ffn_combine(cfg, x, x_perm, token_of_row, expert_offsets, kept_counts, w_gate,
+                           w_up, w_down, h, y_perm, assign_row, topk_w, out, ws, stream=None):
+    """Expert FFN with the combine fused into the down GEMM (x_perm None: gather rows of x)."""
+    check(_lib().moe_expert_ffn_combine(ctypes.byref(cfg), _ptr(x), _ptr(x_perm),
+                                        _ptr(token_of_row), _ptr(expert_offsets),
+                                        _ptr(kept_counts), _ptr(w_gate), _ptr(w_up),
+                                        _ptr(w_down), _ptr(h), _ptr(y_perm), _ptr(assign_row),
+                                        _ptr(topk_w), _ptr(out), _ptr(ws), ws.numel(),
+                                        _stream(stream)))
 
 
 def moe_combine(cfg, y_perm, assign_row, topk_w, out, stream=None):

@@ -103,6 +103,8 @@ PROTOTYPES = {
                                c_vp, c_sz, c_vp]),
     "moe_expert_ffn_gather": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                       c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "moe_expert_ffn_combine": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                       c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "moe_combine": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_vp]),
     "moe_load_stats": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, P(MoeLoadStats), c_vp]),
     "moe_layer_forward": (c_i32, [P(MoeConfig), P(MoeLayerInputs), P(MoeLayerBuffers), c_vp,

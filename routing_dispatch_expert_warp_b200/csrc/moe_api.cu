@@ -155,6 +155,8 @@ WsLayout workspace_layout(const Shape& s) {
   off += l.router_tc_bytes;
   l.ep_base = off;
   off += round_up(static_cast<size_t>(s.E) * sizeof(int32_t));
+  l.arrive = off;
+  off += round_up(static_cast<size_t>(s.T) * ((s.d + 255) / 256) * sizeof(int32_t));
   l.total = off;
   return l;
 }
@@ -347,7 +349,9 @@ moe_status_t expert_ffn(const char* name, const moe_config_t* cfg, const void* a
                         const int32_t* a_rows, const int32_t* expert_offsets,
                         const int32_t* kept_counts, const void* w_gate, const void* w_up,
                         const void* w_down, void* h, void* y_perm, void* ws, size_t ws_bytes,
-                        void* stream) {
+                        void* stream, const int32_t* comb_token_of_row = nullptr,
+                        const int32_t* comb_assign_row = nullptr,
+                        const float* comb_topk_w = nullptr, void* comb_out = nullptr) {
   Shape s;
   moe_status_t st = check_config(cfg, &s);
   if (st != MOE_OK) return st;
@@ -360,19 +364,32 @@ moe_status_t expert_ffn(const char* name, const moe_config_t* cfg, const void* a
               "%s: tensors must be 16-byte aligned", name);
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   cudaError_t err;
+  const bool fuse = comb_out != nullptr;
   if (s.dtype == MOE_F32) {
     err = launch_ffn_simt(s, static_cast<const float*>(a), a_rows, expert_offsets, kept_counts,
                           static_cast<const float*>(w_gate), static_cast<const float*>(w_up),
                           static_cast<const float*>(w_down), static_cast<float*>(h),
                           static_cast<float*>(y_perm), strm);
     if (err != cudaSuccess) return cuda_fail(err, "expert FFN (fp32) launch");
+    if (fuse) {  // fp32 layers run the combine kernel after the FFN (same result)
+      err = launch_combine(s, y_perm, comb_assign_row, comb_topk_w, comb_out, strm);
+      if (err != cudaSuccess) return cuda_fail(err, "combine launch");
+    }
     return MOE_OK;
   }
   if (s.d % 64 != 0 || s.f % 64 != 0)
     return fail(MOE_ERR_UNSUPPORTED, "bf16 expert FFN needs d_model and d_ff multiples of 64");
   const char* why = "";
+  FusedCombine fc;
+  if (fuse) {
+    fc.token_of_row = comb_token_of_row;
+    fc.assign_row = comb_assign_row;
+    fc.topk_w = comb_topk_w;
+    fc.arrive = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + lay.arrive);
+    fc.out = comb_out;
+  }
   err = launch_ffn_tc(s, a, a_rows, expert_offsets, kept_counts, w_gate, w_up, w_down, h, y_perm,
-                      ws_status(ws, lay), g_wait_ns.load(), strm, &why);
+                      ws_status(ws, lay), g_wait_ns.load(), strm, &why, fuse ? &fc : nullptr);
   if (err != cudaSuccess) {
     if (why[0]) return fail(MOE_ERR_CUDA, "%s: %s", name, why);
     return cuda_fail(err, "expert FFN (bf16) launch");
@@ -390,6 +407,23 @@ moe_status_t moe_expert_ffn(const moe_config_t* cfg, const void* x_perm,
                             void* y_perm, void* ws, size_t ws_bytes, void* stream) {
   return expert_ffn("moe_expert_ffn", cfg, x_perm, nullptr, expert_offsets, kept_counts, w_gate,
                     w_up, w_down, h, y_perm, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_expert_ffn_combine(const moe_config_t* cfg, const void* x, const void* x_perm,
+                                    const int32_t* token_of_row, const int32_t* expert_offsets,
+                                    const int32_t* kept_counts, const void* w_gate,
+                                    const void* w_up, const void* w_down, void* h,
+                                    void* y_perm, const int32_t* assign_row,
+                                    const float* topk_w, void* out, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  MOE_REQUIRE(token_of_row && assign_row && topk_w && out && (x || x_perm),
+              "moe_expert_ffn_combine: NULL pointer");
+  MOE_REQUIRE(aligned16(out), "moe_expert_ffn_combine: out must be 16-byte aligned");
+  const void* a = x_perm != nullptr ? x_perm : x;
+  const int32_t* a_rows = x_perm != nullptr ? nullptr : token_of_row;
+  return expert_ffn("moe_expert_ffn_combine", cfg, a, a_rows, expert_offsets, kept_counts,
+                    w_gate, w_up, w_down, h, y_perm, ws, ws_bytes, stream, token_of_row,
+                    assign_row, topk_w, out);
 }
 
 moe_status_t moe_expert_ffn_gather(const moe_config_t* cfg, const void* x,

@@ -134,17 +134,18 @@ __device__ __forceinline__ void tma_load_3d(void* dst_smem, const CUtensorMap* m
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
-// Four rows of a 2D tensor (box: one row high, 64 bf16 wide) into consecutive 128-byte rows
-// of shared memory, with the map's swizzle; row coordinates may differ freely.
-__device__ __forceinline__ void tma_gather4(void* dst_smem, const CUtensorMap* map,
-                                            uint64_t* bar, int32_t c0, int32_t r0, int32_t r1,
-                                            int32_t r2, int32_t r3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_addr(dst_smem)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(c0), "r"(r0), "r"(r1),
-      "r"(r2), "r"(r3)
-      : "memory");
+// 16-byte asynchronous copy global -> shared that bypasses L1.
+__device__ __forceinline__ void cp_async16(uint32_t dst_smem, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+// One arrival on `bar`, made by the hardware once every cp.async this thread issued before
+// has landed (the arrival counts towards the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
 }
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -21,6 +21,8 @@
 // Block = 6 warps, one block per SM, persistent over tiles:
 //   warp 0 (one lane)   TMA producer: A = 128 x 64 bf16 slice of x_perm/h rows, B = 256 x 64
 //                       slice of the expert's weights, 128-byte swizzle, 4-stage ring.
+//                       With gathered A (dispatch without x_perm) the whole warp copies the
+//                       128 rows of x with cp.async into the same swizzled layout.
 //   warp 1 (one lane)   MMA issuer: 4 MMAs (K = 16 each) per stage into one of two TMEM
 //                       accumulators (256 fp32 columns each); commits free the smem stage
 //                       and, at the end of a tile, hand the accumulator to the epilogue.
@@ -71,7 +73,57 @@ struct TcParams {
   // tensor behind tm_a (x itself, [a_rows_limit, K]); nullptr: A rows are the bucket rows.
   const int32_t* a_rows;
   int32_t a_rows_limit;
+  const void* a_src;  // x itself, [a_rows_limit, K] bf16, when a_rows is set
+  // Combine fused into the down launch (comb_out != nullptr): after a row's 256-column
+  // block of y_perm is stored, the row's token counter for that block is bumped; the
+  // thread that completes it sums the token's kept rows in pick order into comb_out.
+  const int32_t* row_token;   // token_of_row
+  const int32_t* assign_row;  // [T, k]
+  const float* topk_w;        // [T, k]
+  int32_t* arrive;            // [T, n_blocks] counters, zero before the launch
+  __nv_bfloat16* comb_out;    // [T, N_out]
+  int k;
+  int32_t T;
 };
+
+// The last of a token's kept picks to finish column block nb has its warp sum the token's
+// rows of that block in pick order (fp32 FMA, then bf16: the arithmetic of the combine
+// kernel).  Lane l owns columns [8 l, 8 l + 8) of the 256-column block and loads its 16
+// bytes of every pick's row at once.  The other picks' rows were stored by other threads,
+// possibly of other blocks: their stores precede their counter increments (fence), the
+// increment seen here precedes these loads (fence), and the loads bypass L1.
+__device__ __forceinline__ void combine_token_block(const TcParams& p, int t, int nb, int lane) {
+  const int64_t col = static_cast<int64_t>(nb) * 256 + lane * 8;
+  if (col >= p.N_out) return;
+  const int32_t* ar = p.assign_row + static_cast<int64_t>(t) * p.k;
+  const float* tw = p.topk_w + static_cast<int64_t>(t) * p.k;
+  uint4 v[MOE_MAX_TOPK];
+  int32_t rr[MOE_MAX_TOPK];
+#pragma unroll
+  for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+    rr[j] = j < p.k ? ar[j] : -1;
+    if (rr[j] >= 0)
+      v[j] = __ldcg(reinterpret_cast<const uint4*>(p.out + static_cast<int64_t>(rr[j]) * p.N_out +
+                                                   col));
+  }
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+  for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+    if (rr[j] < 0) continue;
+    const float w = tw[j];
+    const uint32_t uu[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc[2 * q] = fmaf(w, bf16_lo(uu[q]), acc[2 * q]);
+      acc[2 * q + 1] = fmaf(w, bf16_hi(uu[q]), acc[2 * q + 1]);
+    }
+  }
+  *reinterpret_cast<uint4*>(p.comb_out + static_cast<int64_t>(t) * p.N_out + col) =
+      make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                 pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+}
 
 __device__ __forceinline__ void decode_tile(int tile, const int* tile_base, const int* mblocks,
                                             int E, int n_blocks, int mb_outer, int& e, int& mb,
@@ -147,8 +199,11 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
     tmem_alloc(&tmem_base_s, TMEM_COLS);
     tmem_relinquish();
   } else if (threadIdx.x == 64) {
+    // full: the producer's arm (+ TMA bytes), plus one arrival per lane of the producer warp
+    // when those lanes copy the A rows themselves (gathered A)
+    const unsigned full_count = p.a_rows != nullptr ? 33u : 1u;
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full_bar[s], 1);
+      mbar_init(&full_bar[s], full_count);
       mbar_init(&empty_bar[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -211,28 +266,37 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
           mbar_wait(&full_bar[q], (armed_parity >> q) & 1u, p.wait_ns, nullptr);
     }
   } else if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer, gathered A
-    // Lane 0 waits for free stages, arms them and loads B; every lane then loads four of
-    // the tile's 128 rows of x (one gather4 each) into their own places in the swizzled
-    // stage, so the MMA sees the same layout as with a tile load of x_perm.
+    // ---------------------------------------------------------------- producer, gathered A
+    // Lane 0 waits for free stages, arms them for the B bytes and loads B with TMA.  The A
+    // tile is 128 rows of x picked through a_rows: lane l copies rows l, l+32, l+64, l+96,
+    // eight 16-byte chunks each, with cp.async into the 128-byte-swizzled K-major layout a
+    // TMA tile load would produce (chunk c of row r at r * 128 + ((c ^ (r % 8)) * 16)), then
+    // has the hardware arrive on the stage's full barrier once its copies have landed; the
+    // full barrier expects 1 + 32 arrivals.  (Copying whole 128-byte row pieces per
+    // instruction, 8 lanes a row, measured slower: one warp then spends more instructions
+    // per copy than the copies save.)
     int s = 0;
     uint32_t ph = 0;
     uint32_t armed = 0, armed_parity = 0;
     bool ok = true;
+    const int64_t row_bytes = static_cast<int64_t>(p.K) * 2;
+    const uint8_t* xa = reinterpret_cast<const uint8_t*>(p.a_src);
     for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
       int e, mb, nb;
       decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, p.mb_outer, e, mb, nb);
       const int row0 = p.seg_start[e] + mb * BM;
       // rows past the bucket read token 0; the epilogue never stores them
-      int rr[4] = {0, 0, 0, 0};
+      const uint8_t* src[4];
       const int valid = p.seg_count[e] - mb * BM;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int r = 4 * lane + i;
+        const int r = lane + 32 * i;
+        int t = 0;
         if (r < valid) {
-          const int t = __ldg(p.a_rows + row0 + r);
-          rr[i] = (t >= 0 && t < p.a_rows_limit) ? t : 0;
+          t = __ldg(p.a_rows + row0 + r);
+          if (t < 0 || t >= p.a_rows_limit) t = 0;
         }
+        src[i] = xa + static_cast<int64_t>(t) * row_bytes;
       }
       for (int kb = 0; kb < KB; ++kb) {
         int got = 1;
@@ -245,10 +309,11 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
           ok = false;
           break;
         }
+        __syncwarp();  // the stage lane 0 saw released is released for every lane's copies
         uint8_t* sa = smem + s * STAGE_BYTES;
         uint8_t* sb = sa + A_BYTES;
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
+          mbar_arrive_expect_tx(&full_bar[s], B_BYTES);
           if (GATED) {
             tma_load_3d(sb, &tm_b0, &full_bar[s], kb * BK, nb * 128, e);
             tma_load_3d(sb + B_BYTES / 2, &tm_b1, &full_bar[s], kb * BK, nb * 128, e);
@@ -258,16 +323,24 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
         }
         armed |= 1u << s;
         armed_parity = (armed_parity & ~(1u << s)) | (ph << s);
-        __syncwarp();
-        tma_gather4(sa + lane * 4 * BK * 2, &tm_a, &full_bar[s], kb * BK, rr[0], rr[1], rr[2],
-                    rr[3]);
+        const uint32_t sa_addr = smem_addr(sa);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = lane + 32 * i;
+          const uint8_t* g = src[i] + static_cast<int64_t>(kb) * (BK * 2);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            cp_async16(sa_addr + r * 128 + ((c ^ (r & 7)) << 4), g + c * 16);
+        }
+        cp_async_arrive_noinc(&full_bar[s]);
         if (++s == STAGES) {
           s = 0;
           ph ^= 1u;
         }
       }
     }
-    // every fill this warp armed must land before the block can exit
+    cp_async_wait_all();  // every copy this lane issued lands before it exits
+    // every stage armed (its B bytes in flight) must complete before the block can exit
     if (lane == 0)
       for (int q = 0; q < STAGES; ++q)
         if ((armed >> q) & 1u)
@@ -412,6 +485,33 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
       mbar_arrive(&tempty_bar[acc]);
       acc ^= 1;
       if (acc == 0) aph ^= 1u;
+      if (MODE == MODE_DOWN && p.comb_out != nullptr) {
+        // the accumulator is already handed back: this overlaps the next tile's MMAs
+        int t = -1;
+        bool last = false;
+        if (row_ok) {
+          t = p.row_token[row0 + r];
+          if (t >= 0 && t < p.T) {
+            int picks = 0;
+            for (int j = 0; j < p.k; ++j)
+              picks += p.assign_row[static_cast<int64_t>(t) * p.k + j] >= 0 ? 1 : 0;
+            __threadfence();
+            const int before =
+                atomicAdd(&p.arrive[static_cast<int64_t>(t) * p.n_blocks + nb], 1);
+            last = before == picks - 1;
+          }
+        }
+        unsigned todo = __ballot_sync(0xffffffffu, last);
+        if (todo != 0u) {  // acquire by the last arrivers, then shared with the whole warp
+          __threadfence();
+          __syncwarp();
+        }
+        while (todo != 0u) {
+          const int src = __ffs(todo) - 1;
+          todo &= todo - 1u;
+          combine_token_block(p, __shfl_sync(0xffffffffu, t, src), nb, lane);
+        }
+      }
     }
   }
 
@@ -486,18 +586,6 @@ bool make_map_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [rows, K] bf16 row-major, box 1 row x 64 columns (for gather4), 128-byte swizzle
-bool make_map_gather(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K * 2)};
-  const cuuint32_t box[2] = {BK, 1};
-  const cuuint32_t estr[2] = {1, 1};
-  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // [E, N, K] bf16 weights, box 1 x box_n x 64, 128-byte swizzle
 bool make_map_weights(CUtensorMap* m, const void* base, int E, int64_t N, int64_t K,
                       int box_n) {
@@ -515,17 +603,36 @@ bool make_map_weights(CUtensorMap* m, const void* base, int E, int64_t N, int64_
 
 }  // namespace
 
+// Before a down launch with the combine fused in: zero the arrival counters and the output
+// rows of tokens none of whose picks was kept (no thread of the launch ever writes those).
+__global__ void combine_prep_kernel(int32_t* __restrict__ arrive, int64_t n_counters,
+                                    const int32_t* __restrict__ assign_row, int64_t T, int k,
+                                    uint4* __restrict__ out, int64_t vec_per_row) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (int64_t i = i0; i < n_counters; i += stride) arrive[i] = 0;
+  // a warp per token: lanes < k look at the picks; a token with none gets a zero row
+  const int lane = threadIdx.x & 31;
+  const int64_t nwarps = stride >> 5;
+  for (int64_t t = i0 >> 5; t < T; t += nwarps) {
+    const bool kept = lane < k && assign_row[t * k + lane] >= 0;
+    if (__ballot_sync(0xffffffffu, kept) != 0u) continue;
+    for (int64_t v = lane; v < vec_per_row; v += 32) out[t * vec_per_row + v] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 cudaError_t launch_ffn_tc(const Shape& s, const void* a, const int32_t* a_rows,
                           const int32_t* offsets, const int32_t* kept, const void* wg,
                           const void* wu, const void* wd, void* h, void* y, DevStatus* status,
-                          uint64_t wait_ns, cudaStream_t st, const char** why) {
+                          uint64_t wait_ns, cudaStream_t st, const char** why,
+                          const FusedCombine* comb) {
   if (encode_fn() == nullptr) {
     *why = "cuTensorMapEncodeTiled is not available from the driver";
     return cudaErrorNotSupported;
   }
   CUtensorMap ta1, tg, tu, ta2, td;
-  const bool a_ok = a_rows != nullptr ? make_map_gather(&ta1, a, s.T, s.d)
-                                      : make_map_rows(&ta1, a, s.max_rows, s.d);
+  // gathered A is copied by the producer warp itself; the A map then only stays valid
+  const bool a_ok = make_map_rows(&ta1, a, a_rows != nullptr ? s.T : s.max_rows, s.d);
   if (!a_ok ||
       !make_map_weights(&tg, wg, s.E, s.f, s.d, 128) ||
       !make_map_weights(&tu, wu, s.E, s.f, s.d, 128) ||
@@ -557,6 +664,7 @@ cudaError_t launch_ffn_tc(const Shape& s, const void* a, const int32_t* a_rows,
   p1.wait_ns = wait_ns;
   p1.a_rows = a_rows;
   p1.a_rows_limit = static_cast<int32_t>(s.T);
+  p1.a_src = a;
   int64_t g1 = row_blocks_bound * p1.n_blocks;
   if (g1 > sms) g1 = sms;
   grouped_gemm_tc_kernel<MODE_SWIGLU><<<static_cast<unsigned>(g1), THREADS, DYN_SMEM, st>>>(ta1, tg, tu,
@@ -570,6 +678,25 @@ cudaError_t launch_ffn_tc(const Shape& s, const void* a, const int32_t* a_rows,
   p2.n_blocks = static_cast<int>((s.d + 255) / 256);
   p2.N_out = static_cast<int>(s.d);
   p2.out = static_cast<__nv_bfloat16*>(y);
+  if (comb != nullptr) {
+    const int64_t vec_per_row = s.d * 2 / 16;
+    const int64_t n_counters = s.T * p2.n_blocks;
+    int64_t pb = (s.T * 32 + 255) / 256;  // a warp per token
+    if (pb > static_cast<int64_t>(sms) * 4) pb = static_cast<int64_t>(sms) * 4;
+    if (pb < 1) pb = 1;
+    combine_prep_kernel<<<static_cast<unsigned>(pb), 256, 0, st>>>(
+        comb->arrive, n_counters, comb->assign_row, s.T, s.k, static_cast<uint4*>(comb->out),
+        vec_per_row);
+    note_launch();
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    p2.row_token = comb->token_of_row;
+    p2.assign_row = comb->assign_row;
+    p2.topk_w = comb->topk_w;
+    p2.arrive = comb->arrive;
+    p2.comb_out = static_cast<__nv_bfloat16*>(comb->out);
+    p2.k = s.k;
+    p2.T = static_cast<int32_t>(s.T);
+  }
   int64_t g2 = row_blocks_bound * p2.n_blocks;
   if (g2 > sms) g2 = sms;
   grouped_gemm_tc_kernel<MODE_DOWN><<<static_cast<unsigned>(g2), THREADS, DYN_SMEM, st>>>(ta2, td, td,

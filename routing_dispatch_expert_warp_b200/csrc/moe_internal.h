@@ -37,6 +37,7 @@ struct WsLayout {
   size_t router_tc;     // bf16 split of W_r for the tensor-core router
   size_t router_tc_bytes;
   size_t ep_base;       // [E] int32: first row of this rank's rows per expert at the owner
+  size_t arrive;        // [T, ceil(d/256)] int32 counters of the combine fused into the FFN
   size_t total;
 };
 
@@ -84,10 +85,19 @@ cudaError_t launch_ffn_simt(const Shape& s, const float* a, const int32_t* a_row
                             const int32_t* offsets, const int32_t* kept, const float* wg,
                             const float* wu, const float* wd, float* h, float* y,
                             cudaStream_t st);
+// Combine fused into the bf16 down launch (bitwise the combine kernel's result).
+struct FusedCombine {
+  const int32_t* token_of_row;
+  const int32_t* assign_row;
+  const float* topk_w;
+  int32_t* arrive;  // workspace counters [T, ceil(d / 256)]
+  void* out;        // [T, d]
+};
 cudaError_t launch_ffn_tc(const Shape& s, const void* a, const int32_t* a_rows,
                           const int32_t* offsets, const int32_t* kept, const void* wg,
                           const void* wu, const void* wd, void* h, void* y, DevStatus* status,
-                          uint64_t wait_ns, cudaStream_t st, const char** why);
+                          uint64_t wait_ns, cudaStream_t st, const char** why,
+                          const FusedCombine* comb = nullptr);
 cudaError_t launch_combine(const Shape& s, const void* y_perm, const int32_t* assign_row,
                            const float* topk_w, void* out, cudaStream_t st);
 cudaError_t launch_stats(const Shape& s, const int32_t* routed, const int32_t* kept,

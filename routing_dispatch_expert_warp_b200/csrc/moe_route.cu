@@ -52,26 +52,6 @@ __device__ __forceinline__ bool better(bool va, float a, int ia, bool vb, float 
   return ia < ib;
 }
 
-// Gate weights of one token from its k picked logits (best first), fp32.
-__device__ __forceinline__ void gate_weights(const float* zsel, int k, int gating, float* w) {
-  float s = 0.f;
-  if (gating == MOE_GATE_SOFTMAX) {
-    float m = zsel[0];  // the picks are ordered by selection score, not necessarily by z
-    for (int j = 1; j < k; ++j) m = fmaxf(m, zsel[j]);
-    for (int j = 0; j < k; ++j) {
-      w[j] = expf(zsel[j] - m);
-      s += w[j];
-    }
-  } else {
-    for (int j = 0; j < k; ++j) {
-      w[j] = 1.0f / (1.0f + expf(-zsel[j]));
-      s += w[j];
-    }
-  }
-  const float inv = 1.0f / s;
-  for (int j = 0; j < k; ++j) w[j] *= inv;
-}
-
 // One block scores TW = 32 / ET tokens.  The d axis is cut into 256-element chunks dealt
 // round-robin to the 8 warps.  Inside a chunk, lane l owns the element pairs
 // (64 q + 2 l, 64 q + 2 l + 1), q = 0..3: the warp's loads of x are 128 contiguous bytes per
@@ -171,6 +151,76 @@ __global__ void __launch_bounds__(256) router_weight_lanes_kernel(const float* _
   }
 }
 
+// Lane l of a warp holds the logit z of (token t0 + l / ET, expert l % ET): add the bias,
+// write the logits, pick the top-k of each token (one ET-lane group per token) and write
+// the picks and gate weights.
+template <int ET>
+__device__ __forceinline__ void finish_small_e(float z, int lane, int64_t t0, int64_t T, int E,
+                                               int k, int gating, int bias_mode,
+                                               const float* __restrict__ bias,
+                                               int64_t bias_stride, float* __restrict__ logits,
+                                               int32_t* __restrict__ topk_idx,
+                                               float* __restrict__ topk_w) {
+  const int tw = lane / ET;
+  const int e = lane % ET;
+  const int64_t t = t0 + tw;
+  const bool valid = (e < E) && (t < T);
+  float key = z;  // selection score
+  if (valid) {
+    if (bias != nullptr) {
+      const float b = bias[t * bias_stride + e];
+      if (bias_mode == MOE_BIAS_SELECTION_ONLY) {
+        key = z + b;
+      } else {
+        z += b;
+        key = z;
+      }
+    }
+    if (logits != nullptr) logits[t * E + e] = z;
+  }
+  // top-k within each group of ET lanes (one token per group); lane j of the group keeps
+  // the j-th pick (k <= E <= ET)
+  bool taken = false;
+  float my_z = 0.f;
+  int my_i = 0;
+  for (int j = 0; j < k; ++j) {
+    bool bv = valid && !taken;
+    float bk = key, bz = z;
+    int bi = e;
+#pragma unroll
+    for (int off = ET / 2; off >= 1; off >>= 1) {
+      const bool ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+      const float oz = __shfl_xor_sync(0xffffffffu, bz, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (better(ov, ok, oi, bv, bk, bi)) {
+        bv = ov; bk = ok; bz = oz; bi = oi;
+      }
+    }
+    if (bi == e) taken = true;
+    if (e == j) {
+      my_z = bz;
+      my_i = bi;
+    }
+  }
+  // gate weights over the group's k picks; the normaliser is summed in pick order
+  const int base = lane - e;
+  float wgt;
+  if (gating == MOE_GATE_SOFTMAX) {
+    float m = __shfl_sync(0xffffffffu, my_z, base);
+    for (int j = 1; j < k; ++j) m = fmaxf(m, __shfl_sync(0xffffffffu, my_z, base + j));
+    wgt = expf(my_z - m);
+  } else {
+    wgt = 1.0f / (1.0f + expf(-my_z));
+  }
+  float ssum = 0.f;
+  for (int j = 0; j < k; ++j) ssum += __shfl_sync(0xffffffffu, wgt, base + j);
+  if (e < k && t < T) {
+    topk_idx[t * k + e] = my_i;
+    topk_w[t * k + e] = wgt * (1.0f / ssum);
+  }
+}
+
 // One block scores TW = 32 / ET tokens.  The d axis is cut into 256-element chunks dealt
 // round-robin to the 8 warps; in a chunk lane l owns 8 consecutive elements (one 16-byte
 // load of x per token).  A warp first issues the x loads of up to CPW chunks at once, then
@@ -252,53 +302,8 @@ __global__ void __launch_bounds__(256, ET == 8 ? 2 : 3) router_small_e_kernel(
       float z = part[0][lane];
 #pragma unroll
       for (int w = 1; w < NW; ++w) z += part[w][lane];
-      const int tw = lane / ET;
-      const int e = lane % ET;
-      const int64_t t = t0 + tw;
-      const bool valid = (e < E) && (t < T);
-      float key = z;  // selection score
-      if (valid) {
-        if (bias != nullptr) {
-          const float b = bias[t * bias_stride + e];
-          if (bias_mode == MOE_BIAS_SELECTION_ONLY) {
-            key = z + b;
-          } else {
-            z += b;
-            key = z;
-          }
-        }
-        if (logits != nullptr) logits[t * E + e] = z;
-      }
-      // top-k within each group of ET lanes (one token per group)
-      bool taken = false;
-      float zsel[MOE_MAX_TOPK];
-      int isel[MOE_MAX_TOPK];
-      for (int j = 0; j < k; ++j) {
-        bool bv = valid && !taken;
-        float bk = key, bz = z;
-        int bi = e;
-#pragma unroll
-        for (int off = ET / 2; off >= 1; off >>= 1) {
-          const bool ov = __shfl_xor_sync(0xffffffffu, bv, off);
-          const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-          const float oz = __shfl_xor_sync(0xffffffffu, bz, off);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-          if (better(ov, ok, oi, bv, bk, bi)) {
-            bv = ov; bk = ok; bz = oz; bi = oi;
-          }
-        }
-        if (bi == e) taken = true;
-        zsel[j] = bz;
-        isel[j] = bi;
-      }
-      if (e == 0 && t < T) {
-        float w[MOE_MAX_TOPK];
-        gate_weights(zsel, k, gating, w);
-        for (int j = 0; j < k; ++j) {
-          topk_idx[t * k + j] = isel[j];
-          topk_w[t * k + j] = w[j];
-        }
-      }
+      finish_small_e<ET>(z, lane, t0, T, E, k, gating, bias_mode, bias, bias_stride, logits,
+                         topk_idx, topk_w);
     }
     __syncthreads();
   }

@@ -6,8 +6,8 @@
 // of experts and dropped tokens.  "Capacity factor changes quality, memory and the latency
 // tail": drop rate per layer and per route (first pick, second pick, ...).
 //
-// One block: the E kept counts are sorted in shared memory (bitonic network over 256
-// slots), the drops are counted per pick rank over assign_row, and one thread evaluates
+// One block: the E kept counts are sorted in shared memory (bitonic network over the next
+// power of two of E), the drops are counted per pick rank over assign_row, and one thread evaluates
 // the fp64 formulas.  Percentiles interpolate linearly between order statistics:
 // h = (E - 1) p, v = s[floor h] + (h - floor h) (s[floor h + 1] - s[floor h]).
 #include <limits.h>
@@ -69,11 +69,14 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
       atomicMax(&max_routed, mx);
     }
   }
-  // bitonic sort of the 256 slots, ascending
-  for (int size = 2; size <= MOE_MAX_EXPERTS; size <<= 1) {
+  // bitonic sort, ascending, of the smallest power-of-two number of slots holding E (the
+  // slots past E hold INT_MAX and stay at the end)
+  int n2 = 2;
+  while (n2 < E) n2 <<= 1;
+  for (int size = 2; size <= n2; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
       const int partner = tid ^ stride;
-      if (tid < MOE_MAX_EXPERTS && partner > tid) {
+      if (tid < n2 && partner > tid) {
         const bool asc = (tid & size) == 0;
         const int32_t a = sorted[tid], b = sorted[partner];
         if ((a > b) == asc) {

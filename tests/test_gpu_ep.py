@@ -45,6 +45,9 @@ CASES = [
     (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 256, 128), 8, "contiguous"),     # capacity drops
     (W.reduced(W.DSV3_DECODE, 64, 256, 128), 4, "permuted"),
     (W.TINY_FP32, 2, "contiguous"),
+    # routing variants: group-limited top-k, selection-only bias, pick-rank drops
+    (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 256, 128, n_groups=8, topk_groups=4, bias_mode=1,
+               drop_policy=1), 4, "permuted"),
     (W.reduced(W.MIXTRAL_8X7B, 300, 128, 128), 1, "contiguous"),
 ]
 

@@ -80,6 +80,9 @@ EDGES = [
     _edge(300, 256, 128, 200, 6, cf=1.0),         # E not a power of two, > 32
     _edge(600, 256, 128, 200, 4, gating=W.SIGMOID, cf=1.5),   # tensor-core router, ragged E
     _edge(520, 128, 128, 64, 8, gating=W.SIGMOID),            # tensor-core router, E = 64
+    _edge(300, 2048, 128, 32, 4),       # E = 32 with a long d
+    _edge(150, 7168, 64, 8, 2, gating=W.SIGMOID),             # E = 8 at the DeepSeek d
+    _edge(77, 6144, 64, 8, 2),          # E = 8 at the Mixtral-8x22B d
 ]
 
 
@@ -326,4 +329,40 @@ def test_layer_forward_without_x_perm(shape):
     M.moe_check_device_error(layer.ws)
     torch.cuda.synchronize()
     assert torch.equal(out, run.b.out)
-    assert launched == 8    # the permute kernel is gone
+    assert launched == 8    # router (2), count + rank, two FFN launches, combine, stats: no permute
+
+
+# ------------------------------------------------------------------ combine fused into the FFN
+FUSED = GATHER + [
+    W.reduced(W.DSV3_DECODE, 128, 512, 256),
+    _edge(200, 64, 64, 16, 1, cf=0.05),                 # most tokens fully dropped
+    _edge(500, 128, 128, 8, 2, cf=0.3),
+    W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256, n_groups=8, topk_groups=4, bias_mode=1,
+              drop_policy=1),
+]
+
+
+@pytest.mark.parametrize("shape", FUSED, ids=lambda s: s.name)
+@pytest.mark.parametrize("gather", [False, True], ids=["x_perm", "gather"])
+def test_fused_combine_equals_separate_combine(shape, gather):
+    """moe_expert_ffn_combine writes h, y_perm and out bitwise equal to moe_expert_ffn +
+    moe_combine, with the A rows from x_perm or gathered from x, fully dropped tokens
+    included; a second call on the same workspace gives the same bits (counters reset)."""
+    run = GpuRun(shape)
+    run.all_stages()
+    ref_out, ref_y = run.b.out.clone(), run.b.y_perm.clone()
+    b = run.b
+    for _ in range(2):
+        b.out.fill_(7.0), b.y_perm.zero_()
+        M.moe_expert_ffn_combine(run.cfg, run.inp.x, None if gather else b.x_perm,
+                                 b.token_of_row, b.expert_offsets, b.kept_counts,
+                                 run.inp.w_gate, run.inp.w_up, run.inp.w_down, b.h, b.y_perm,
+                                 b.assign_row, b.topk_w, b.out, run.ws)
+        M.moe_check_device_error(run.ws)
+        torch.cuda.synchronize()
+        assert torch.equal(b.out, ref_out)
+        used = int(b.expert_offsets[-1])
+        rows = torch.nonzero(b.token_of_row[:used] >= 0).flatten()
+        assert torch.equal(b.y_perm[rows], ref_y[rows])
+    r = check_routing(run)
+    check_layer_output(run, run.b.out, r)
