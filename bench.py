@@ -356,6 +356,79 @@ def run_gpu(args) -> None:
         dist.destroy_process_group()
 
 
+def run_ep_emulated(args) -> None:
+    """The expert-parallel layer with args.ep_emulate ranks emulated on this one GPU: the
+    workload's T tokens split evenly over the ranks (capacity per source rank), experts in
+    contiguous blocks, every step of the EP schedule timed with CUDA events.  A measurement
+    of the EP kernels' cost next to the single-GPU layer on the same tokens; the NVLink
+    transfers of a real multi-GPU run are local copies here."""
+    from routing_dispatch_expert_warp_b200 import ep as EP
+    G = args.ep_emulate
+    base = W.WORKLOADS[args.config] if args.config else DEFAULT
+    if base.T % G or base.E % G:
+        raise SystemExit("T and E must be multiples of the emulated rank count")
+    shape = base.replace(name=f"{base.name}_ep{G}_emulated", T=base.T // G)
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = W.make_inputs(base, device=dev)
+    xs = [inp.x[r * shape.T:(r + 1) * shape.T].contiguous() for r in range(G)]
+    if inp.logit_bias is not None and inp.logit_bias.dim() == 2:
+        biases = [inp.logit_bias[r * shape.T:(r + 1) * shape.T].contiguous() for r in range(G)]
+    else:
+        biases = [inp.logit_bias] * G
+    cfg = M.config_from_shape(shape)
+    emu = EP.EpEmulator(cfg, G, inp.w_router, inp.w_gate, inp.w_up, inp.w_down, biases,
+                        device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    names = [s for s in EP.SCHEDULE if s != "barrier"] + ["end"]
+
+    def run(evs):
+        emu.forward(xs, on_step=lambda n: evs[n].record(stream))
+
+    mk = lambda: {n: torch.cuda.Event(enable_timing=True) for n in names}
+    for _ in range(args.warmup):
+        flush.zero_()
+        run(mk())
+    for r in emu.ranks:
+        M.moe_check_device_error(r.ws)
+    evs = [mk() for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(0)
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()
+        run(evs[i])
+    torch.cuda.synchronize(dev)
+    time.sleep(0.2)
+    clk = clocks.stop()
+    for r in emu.ranks:
+        M.moe_check_device_error(r.ws)
+    per = {n: sum(e[n].elapsed_time(e[names[i + 1]]) for e in evs) / args.steps
+           for i, n in enumerate(names[:-1])}
+    ms = sum(e[names[0]].elapsed_time(e["end"]) for e in evs) / args.steps
+    st = emu.ranks[0].stats_dict()
+    row_bytes = base.d_model * (2 if base.dtype == W.BF16 else 4)
+    moved = st["total_assignments"] * row_bytes          # rows written by dispatch
+    x_bytes = base.T * row_bytes
+    line = {
+        "metric": f"MoE-layer tokens/s, expert parallel over {G} ranks emulated on 1 B200",
+        "value": base.T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "dtype": "bf16" if base.dtype == W.BF16 else "f32", "data": "synthetic",
+        "config": {"workload": base.name, "ranks": G, "tokens_per_rank": shape.T,
+                   "placement": "contiguous", "l2": "flushed between timed steps (256 MB write)"},
+        "steps_ms": per,
+        "dispatch_GBps": (x_bytes + moved) / (per["dispatch"] * 1e-3) / 1e9,
+        "combine_GBps": (moved + x_bytes) / (per["combine"] * 1e-3) / 1e9,
+        "ep_stats": {k: st[k] for k in ("local_fraction", "remote_bytes", "pair_bytes_p50",
+                                         "pair_bytes_p99", "rank_load_max_to_mean",
+                                         "cross_node_fraction")},
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def _cpu_cores() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -435,6 +508,9 @@ def main():
     ap.add_argument("--cpu-sample-tokens", type=int, default=64)
     ap.add_argument("--ref-sample-tokens", type=int, default=32)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--ep-emulate", type=int, default=0,
+                    help="time the expert-parallel layer with this many ranks emulated on one "
+                         "GPU (a separate measurement, not the headline line)")
     ap.add_argument("--fused-combine", action="store_true",
                     help="time the expert FFN with the combine fused into its down GEMM")
     ap.add_argument("--gather", action="store_true",
@@ -443,6 +519,8 @@ def main():
     args.warmup = max(args.warmup, 3)   # at least three untimed warm-up steps
     if args.impl == "reference":
         run_reference(args)
+    elif args.ep_emulate:
+        run_ep_emulated(args)
     else:
         run_gpu(args)
 

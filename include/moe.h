@@ -447,7 +447,8 @@ moe_status_t moe_selftest_bounded_wait(void* ws, size_t ws_bytes, void* stream);
 
 /* Rows a receive buffer needs so that no distribution of picks can overflow it: world x
  * min(T*min(k, n_local), n_local*C) (C = capacity; T*min(k, n_local) when dropless),
- * with T the largest per-rank token count. */
+ * with T the largest per-rank token count.  Reads only the sizes of cfg and ep; -2 (and
+ * the reason in moe_last_error) when they are invalid. */
 int64_t moe_ep_recv_rows_bound(const moe_config_t* cfg, const moe_ep_config_t* ep);
 
 /* Step 1.  mats[g] -> rank g's count matrix [world, E] int32; row `rank` receives

@@ -501,8 +501,9 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_layer_inputs_t
 
 namespace {
 
-moe_status_t check_ep(const moe_config_t* cfg, const moe_ep_config_t* ep, Shape* s,
-                      const char* name) {
+// The EP fields that sizes depend on (everything but the placement pointer).
+moe_status_t check_ep_shape(const moe_config_t* cfg, const moe_ep_config_t* ep, Shape* s,
+                            const char* name) {
   moe_status_t st = check_config(cfg, s);
   if (st != MOE_OK) return st;
   MOE_REQUIRE(ep != nullptr, "%s: ep is NULL", name);
@@ -511,9 +512,16 @@ moe_status_t check_ep(const moe_config_t* cfg, const moe_ep_config_t* ep, Shape*
   MOE_REQUIRE(ep->rank >= 0 && ep->rank < ep->world, "%s: rank outside [0, world)", name);
   MOE_REQUIRE(ep->ranks_per_node >= 1, "%s: ranks_per_node must be >= 1", name);
   MOE_REQUIRE(ep->n_local >= 1 && ep->n_local <= s->E, "%s: n_local must be 1..E", name);
-  MOE_REQUIRE(ep->expert_rank != nullptr, "%s: expert_rank is NULL", name);
   MOE_REQUIRE(ep->recv_rows >= 0 && ep->recv_rows <= INT32_MAX,
               "%s: recv_rows must be in [0, 2^31)", name);
+  return MOE_OK;
+}
+
+moe_status_t check_ep(const moe_config_t* cfg, const moe_ep_config_t* ep, Shape* s,
+                      const char* name) {
+  moe_status_t st = check_ep_shape(cfg, ep, s, name);
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(ep->expert_rank != nullptr, "%s: expert_rank is NULL", name);
   return MOE_OK;
 }
 
@@ -531,11 +539,7 @@ extern "C" {
 
 int64_t moe_ep_recv_rows_bound(const moe_config_t* cfg, const moe_ep_config_t* ep) {
   Shape s;
-  moe_ep_config_t tmp;
-  if (ep == nullptr) return -2;
-  tmp = *ep;
-  if (tmp.expert_rank == nullptr) tmp.expert_rank = reinterpret_cast<const int32_t*>(16);
-  if (check_ep(cfg, &tmp, &s, "moe_ep_recv_rows_bound") != MOE_OK) return -2;
+  if (check_ep_shape(cfg, ep, &s, "moe_ep_recv_rows_bound") != MOE_OK) return -2;
   return ep_bound(s, ep);
 }
 

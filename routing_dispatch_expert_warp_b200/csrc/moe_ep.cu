@@ -266,9 +266,11 @@ __global__ void __launch_bounds__(kStatThreads) ep_stats_kernel(
     sorted_s[i] = v;
   }
   __syncthreads();
-  for (int size = 2; size <= kPairSort; size <<= 1) {
+  int n2 = 2;  // sort the smallest power of two that holds the pairs (padding sorts last)
+  while (n2 < n_pairs) n2 <<= 1;
+  for (int size = 2; size <= n2; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < kPairSort; i += blockDim.x) {
+      for (int i = tid; i < n2; i += blockDim.x) {
         const int j = i ^ stride;
         if (j > i) {
           const bool up = (i & size) == 0;

@@ -166,13 +166,17 @@ def _table(ptrs: Sequence[int], device) -> torch.Tensor:
 
 
 def run_schedule(ranks: Sequence[EpRank], xs: Sequence[torch.Tensor], tables: dict,
-                 barrier: Callable[[], None], stream=None) -> None:
+                 barrier: Callable[[], None], stream=None,
+                 on_step: Optional[Callable[[str], None]] = None) -> None:
     """The steps of SCHEDULE for the ranks held by this process (all ranks when emulated on
-    one GPU, one rank per process otherwise)."""
+    one GPU, one rank per process otherwise).  on_step(name) is called before each step (and
+    with "end" after the last), e.g. to record timing events."""
     for step in SCHEDULE:
         if step == "barrier":
             barrier()
             continue
+        if on_step is not None:
+            on_step(step)
         for r, x in zip(ranks, xs):
             if step == "route":
                 r.route(x, stream)
@@ -190,6 +194,8 @@ def run_schedule(ranks: Sequence[EpRank], xs: Sequence[torch.Tensor], tables: di
                 r.combine(tables["ybuf"], stream)
             elif step == "stats":
                 r.stats(False, stream)
+    if on_step is not None:
+        on_step("end")
 
 
 class EpEmulator:
@@ -218,8 +224,9 @@ class EpEmulator:
             "ybuf": _table([r.y_recv.data_ptr() for r in self.ranks], device),
         }
 
-    def forward(self, xs: Sequence[torch.Tensor], stream=None) -> List[torch.Tensor]:
-        run_schedule(self.ranks, xs, self.tables, lambda: None, stream)
+    def forward(self, xs: Sequence[torch.Tensor], stream=None,
+                on_step: Optional[Callable[[str], None]] = None) -> List[torch.Tensor]:
+        run_schedule(self.ranks, xs, self.tables, lambda: None, stream, on_step)
         return [r.out for r in self.ranks]
 
 

@@ -160,3 +160,40 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_abi, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         _abi.lib()
+
+
+def test_ep_sizes_and_argument_checks(lib):
+    """Expert-parallel host checks (no kernel runs): the receive-buffer bound and rejections."""
+    cfg = M.make_config(4096, 256, 128, 256, 8, capacity_factor=1.0)
+    C = O.capacity(1.0, 4096, 8, 256)
+    ep = _abi.MoeEpConfig(world=8, rank=3, ranks_per_node=4, n_local=32, expert_rank=None,
+                          recv_rows=0)
+    assert lib.moe_ep_recv_rows_bound(ctypes.byref(cfg), ctypes.byref(ep)) == 8 * min(4096 * 8, 32 * C)
+    dropless = M.make_config(100, 256, 128, 8, 2)
+    ep1 = _abi.MoeEpConfig(world=4, rank=0, ranks_per_node=1, n_local=2, expert_rank=None,
+                           recv_rows=0)
+    assert lib.moe_ep_recv_rows_bound(ctypes.byref(dropless), ctypes.byref(ep1)) == 4 * 100 * 2
+    ep1.n_local = 1     # a token picks an expert at most once
+    assert lib.moe_ep_recv_rows_bound(ctypes.byref(dropless), ctypes.byref(ep1)) == 4 * 100 * 1
+    for bad in (dict(world=0), dict(world=65), dict(rank=8), dict(rank=-1), dict(n_local=0),
+                dict(n_local=257), dict(ranks_per_node=0)):
+        e = _abi.MoeEpConfig(world=8, rank=3, ranks_per_node=1, n_local=32, expert_rank=None,
+                             recv_rows=0)
+        for key, val in bad.items():
+            setattr(e, key, val)
+        assert lib.moe_ep_recv_rows_bound(ctypes.byref(cfg), ctypes.byref(e)) == -2, bad
+    # calls that would launch: a missing placement or buffer is refused on the host
+    ep.recv_rows = 1024
+    ws = ctypes.c_size_t(0)
+    assert lib.moe_workspace_size(ctypes.byref(cfg), ctypes.byref(ws)) == 0
+    st = lib.moe_ep_put_counts(ctypes.byref(cfg), ctypes.byref(ep), 16, 16, None)
+    assert st == 1 and b"expert_rank" in lib.moe_last_error()
+    ep.expert_rank = 16
+    assert lib.moe_ep_put_counts(ctypes.byref(cfg), ctypes.byref(ep), None, 16, None) == 1
+    assert lib.moe_ep_dispatch(ctypes.byref(cfg), ctypes.byref(ep), 17, 16, 16, 16, 256,
+                               ws.value, None) == 1          # misaligned x
+    assert lib.moe_ep_combine(ctypes.byref(cfg), ctypes.byref(ep), None, 16, 16, 16, 16, 256,
+                              ws.value, None) == 1
+    assert lib.moe_ep_stats(ctypes.byref(cfg), ctypes.byref(ep), None, 16, None, None) == 1
+    assert lib.moe_ipc_handle(None, ctypes.create_string_buffer(64),
+                              ctypes.byref(ctypes.c_int64())) == 1
