@@ -27,7 +27,7 @@ __all__ = ["MoEError", "make_config", "workspace_size", "capacity", "max_rows",
            "moe_expert_ffn", "moe_expert_ffn_gather", "moe_expert_ffn_combine", "moe_combine",
            "moe_load_stats", "moe_layer_forward", "moe_check_device_error",
            "moe_selftest_bounded_wait", "set_wait_limit_ns", "kernel_launch_count",
-           "LayerBuffers", "MoELayer"]
+           "LayerBuffers", "MoELayer", "HostPipeline"]
 
 
 def _lib():
@@ -240,7 +240,8 @@ class MoELayer:
     forward(x) enqueues the whole layer (moe_layer_forward) on the current stream and
     returns the output tensor (a view of the layer's own buffer, overwritten by the next
     call).  gather=True drops the permuted copy of x: dispatch only ranks the assignments
-    and the gate/up GEMM gathers its rows from x (same results, less memory traffic)."""
+    and the gate/up GEMM gathers its rows from x (same results and less memory, but slower
+    than the permuted copy on B200)."""
 
     def __init__(self, cfg: MoeConfig, w_router, w_gate, w_up, w_down, logit_bias=None,
                  device="cuda", gather: bool = False):
@@ -263,3 +264,62 @@ class MoELayer:
         return self.bufs.out
 
     __call__ = forward
+
+
+class HostPipeline:
+    """Runs one MoE layer over a sequence of token batches held in pinned host memory,
+    overlapping every batch's host-to-device copy and the previous result's device-to-host
+    copy with the layer's kernels: two copy streams (in and out) around the compute stream,
+    and `depth` sets of device buffers used in turn.  The results are those of
+    MoELayer.forward on each batch."""
+
+    def __init__(self, cfg: MoeConfig, w_router, w_gate, w_up, w_down, logit_bias=None,
+                 device="cuda", depth: int = 2):
+        if depth < 2:
+            raise ValueError("depth must be >= 2 to overlap copies with compute")
+        self.device = torch.device(device)
+        self.layers = [MoELayer(cfg, w_router, w_gate, w_up, w_down, logit_bias, device)
+                       for _ in range(depth)]
+        dt = torch.float32 if cfg.dtype == F32 else torch.bfloat16
+        self.x_dev = [torch.empty((cfg.T, cfg.d_model), dtype=dt, device=self.device)
+                      for _ in range(depth)]
+        self.s_in = torch.cuda.Stream(self.device)
+        self.s_out = torch.cuda.Stream(self.device)
+
+    def run(self, xs_host, outs_host, stream=None) -> None:
+        """Enqueue every batch: xs_host[i] -> layer -> outs_host[i] (pinned host tensors of
+        shape [T, d_model]).  Returns once everything is enqueued; synchronise on `stream`
+        (default: the current stream) to wait for the last result."""
+        comp = stream or torch.cuda.current_stream(self.device)
+        depth = len(self.layers)
+        n = len(xs_host)
+        copied, computed, fetched = [], [], []
+        start = torch.cuda.Event()
+        start.record(comp)
+        self.s_in.wait_event(start)
+        self.s_out.wait_event(start)
+        for i in range(n):
+            slot = i % depth
+            with torch.cuda.stream(self.s_in):
+                if i >= depth:  # the slot's input buffer is free once its last layer ran
+                    self.s_in.wait_event(computed[i - depth])
+                self.x_dev[slot].copy_(xs_host[i], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(self.s_in)
+                copied.append(ev)
+            comp.wait_event(copied[i])
+            if i >= depth:      # the slot's output buffer is free once it was fetched
+                comp.wait_event(fetched[i - depth])
+            self.layers[slot].forward(self.x_dev[slot], comp)
+            ev = torch.cuda.Event()
+            ev.record(comp)
+            computed.append(ev)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(computed[i])
+                outs_host[i].copy_(self.layers[slot].bufs.out, non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(self.s_out)
+                fetched.append(ev)
+        if n:
+            comp.wait_event(fetched[-1])
+

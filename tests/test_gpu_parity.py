@@ -366,3 +366,25 @@ def test_fused_combine_equals_separate_combine(shape, gather):
         assert torch.equal(b.y_perm[rows], ref_y[rows])
     r = check_routing(run)
     check_layer_output(run, run.b.out, r)
+
+
+def test_host_pipeline_equals_layer_forward():
+    """HostPipeline over five distinct pinned host batches gives, for each, the bits of
+    MoELayer.forward on that batch, with copies overlapping the kernels of neighbours."""
+    shape = W.reduced(W.MIXTRAL_8X7B, 600, 256, 384)
+    inp = W.make_inputs(shape, device="cuda")
+    cfg = M.config_from_shape(shape)
+    xs = [W.make_inputs(shape.replace(seed=shape.seed + i), device="cuda", weights=False).x
+          for i in range(5)]
+    xs_host = [x.cpu().pin_memory() for x in xs]
+    outs_host = [torch.empty((shape.T, shape.d_model), dtype=xs[0].dtype).pin_memory()
+                 for _ in xs]
+    pipe = M.HostPipeline(cfg, inp.w_router, inp.w_gate, inp.w_up, inp.w_down, inp.logit_bias)
+    pipe.run(xs_host, outs_host)
+    torch.cuda.current_stream().synchronize()
+    for lyr in pipe.layers:
+        M.moe_check_device_error(lyr.ws)
+    layer = M.MoELayer(cfg, inp.w_router, inp.w_gate, inp.w_up, inp.w_down, inp.logit_bias)
+    for x, o in zip(xs, outs_host):
+        ref = layer(x).cpu()
+        assert torch.equal(o, ref)
