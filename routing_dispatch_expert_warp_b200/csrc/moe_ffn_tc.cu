@@ -347,7 +347,9 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
           mbar_wait(&full_bar[q], (armed_parity >> q) & 1u, p.wait_ns, nullptr);
   } else if (warp == 1 && lane == 0) {
     // ---------------------------------------------------------------- MMA issuer
-    constexpr uint32_t idesc = idesc_bf16_f32(BM, MMA_N);
+    // a bucket's last tile with at most 64 rows runs as M = 64 MMAs (half the tensor work)
+    constexpr uint32_t idesc_full = idesc_bf16_f32(BM, MMA_N);
+    constexpr uint32_t idesc_half = idesc_bf16_f32(BM / 2, MMA_N);
     int s = 0;
     uint32_t ph = 0;
     int acc = 0;
@@ -355,6 +357,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
     bool ok = true;
     bool issued = false;
     for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      int e, mb, nb;
+      decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, p.mb_outer, e, mb, nb);
+      const uint32_t idesc =
+          p.seg_count[e] - mb * BM <= BM / 2 ? idesc_half : idesc_full;
       if (!mbar_wait(&tempty_bar[acc], aph ^ 1u, p.wait_ns, &abort_s)) {
         if (!abort_s) record_error(p.status, DEV_TIMEOUT, 21, static_cast<unsigned long long>(tile));
         abort_s = 1;
@@ -415,12 +421,14 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                              static_cast<uint32_t>(acc * ACC_COLS);
-      const bool row_ok = r < valid;
+      // M = 64 tiles (valid <= 64) hold row 16 q + i in lane i < 16 of TMEM quarter q
+      const int rt = valid <= BM / 2 ? (lane < 16 ? q * 16 + lane : BM) : r;
+      const bool row_ok = rt < valid;
       __nv_bfloat16* orow =
-          p.out + static_cast<int64_t>(row0 + r) * p.N_out + static_cast<int64_t>(nb) * BN_OUT;
+          p.out + static_cast<int64_t>(row0 + rt) * p.N_out + static_cast<int64_t>(nb) * BN_OUT;
       const int cols_left = p.N_out - nb * BN_OUT;
       if (MODE == MODE_ROUTER) {
-        const int64_t grow = static_cast<int64_t>(row0 + r);
+        const int64_t grow = static_cast<int64_t>(row0 + rt);
         float* zrow = p.out_f32 + grow * p.N_out + static_cast<int64_t>(nb) * BN_OUT;
         const float* brow =
             p.bias != nullptr ? p.bias + grow * p.bias_stride + static_cast<int64_t>(nb) * BN_OUT
@@ -490,7 +498,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
         int t = -1;
         bool last = false;
         if (row_ok) {
-          t = p.row_token[row0 + r];
+          t = p.row_token[row0 + rt];
           if (t >= 0 && t < p.T) {
             int picks = 0;
             for (int j = 0; j < p.k; ++j)
