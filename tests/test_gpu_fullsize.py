@@ -39,3 +39,40 @@ def test_full_size_sampled(shape):
         assert st["max"] <= st["capacity"]
     del run
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("shape,world", [(W.MIXTRAL_8X7B, 8), (W.DSV3_PREFILL_ZIPF, 8)],
+                         ids=lambda v: getattr(v, "name", str(v)))
+def test_full_size_expert_parallel_equals_single_gpu(shape, world):
+    """The bench workloads' tokens split over `world` emulated EP ranks: every rank's output
+    is bitwise the single-GPU layer's on its own tokens, and the EP record's totals add up."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    import routing_dispatch_expert_warp_b200 as M
+    from routing_dispatch_expert_warp_b200 import ep as EP
+    torch.cuda.empty_cache()
+    per = shape.replace(T=shape.T // world)
+    inp = W.make_inputs(shape, device="cuda")
+    xs = [inp.x[r * per.T:(r + 1) * per.T].contiguous() for r in range(world)]
+    biases = ([inp.logit_bias[r * per.T:(r + 1) * per.T].contiguous() for r in range(world)]
+              if inp.logit_bias is not None and inp.logit_bias.dim() == 2
+              else [inp.logit_bias] * world)
+    cfg = M.config_from_shape(per)
+    emu = EP.EpEmulator(cfg, world, inp.w_router, inp.w_gate, inp.w_up, inp.w_down, biases)
+    outs = [o.clone() for o in emu.forward(xs)]
+    for r in emu.ranks:
+        M.moe_check_device_error(r.ws)
+    st = emu.ranks[0].stats_dict()
+    kept_total = sum(int(r.bufs.kept_counts.sum()) for r in emu.ranks)
+    assert st["total_assignments"] == kept_total
+    assert sum(st["rank_load"]) == kept_total
+    del emu
+    torch.cuda.empty_cache()
+    layer = M.MoELayer(cfg, inp.w_router, inp.w_gate, inp.w_up, inp.w_down, biases[0])
+    for g in range(world):
+        layer.logit_bias = biases[g]
+        ref = layer(xs[g])
+        torch.cuda.synchronize()
+        assert torch.equal(outs[g], ref), f"rank {g}"
+    del layer
+    torch.cuda.empty_cache()
