@@ -297,6 +297,28 @@ def run_gpu(args) -> None:
     e2e_total = max_over_ranks([sum(e2e_ms)], dist, dev)[0]
     M.moe_check_device_error(layer.ws)
 
+    # the whole layer replayed as one CUDA graph (no launch gaps between the kernels)
+    glayer = M.MoELayer(cfg, inp.w_router, inp.w_gate, inp.w_up, inp.w_down, inp.logit_bias,
+                        device=dev, gather=args.gather)
+    gx = inp.x.clone()
+    graph = glayer.capture(gx)
+    for _ in range(args.warmup):
+        flush.zero_()
+        graph.replay()
+    torch.cuda.synchronize(dev)
+    g_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        graph.replay()
+        g1.record(stream)
+        g1.synchronize()
+        g_ms.append(g0.elapsed_time(g1))
+    graph_total = max_over_ranks([sum(g_ms)], dist, dev)[0]
+    M.moe_check_device_error(glayer.ws)
+    del graph, glayer, gx
+
     # the same through HostPipeline: batch i's upload and batch i-1's download overlap the
     # layer's kernels (two copy streams, two sets of device buffers); every step still copies
     # its input in and its output out, all inside one timed region
@@ -372,6 +394,10 @@ def run_gpu(args) -> None:
                     "unpipelined": {"value": shape.T * world / (e2e_total / args.steps * 1e-3),
                                     "api": "MoELayer.forward with its copies in series, "
                                            "L2 flushed between steps"}},
+            "graph": {"ms_per_step": graph_total / args.steps,
+                      "tokens_per_s": shape.T * world / (graph_total / args.steps * 1e-3),
+                      "api": "MoELayer.capture -> CUDA graph replay of moe_layer_forward",
+                      "l2": "flushed between replays"},
             "gpu_launches": timed_launches,
             "clocks": clk,
             "cpu_baseline": cpu,

@@ -265,6 +265,22 @@ class MoELayer:
 
     __call__ = forward
 
+    def capture(self, x: torch.Tensor) -> "torch.cuda.CUDAGraph":
+        """Record one forward on the fixed input buffer x into a CUDA graph: replay() then
+        runs the whole layer (every kernel, no host work) on whatever x holds, into
+        self.bufs.out.  The layer enqueues no host synchronisation and allocates nothing, so
+        it captures as is; one eager forward first sets up the per-device state."""
+        self.forward(x)
+        torch.cuda.synchronize(x.device)
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(x.device)
+        side.wait_stream(torch.cuda.current_stream(x.device))
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(graph, stream=side):
+                self.forward(x, side)
+        torch.cuda.current_stream(x.device).wait_stream(side)
+        return graph
+
 
 class HostPipeline:
     """Runs one MoE layer over a sequence of token batches held in pinned host memory,

@@ -388,3 +388,25 @@ def test_host_pipeline_equals_layer_forward():
     for x, o in zip(xs, outs_host):
         ref = layer(x).cpu()
         assert torch.equal(o, ref)
+
+
+@pytest.mark.parametrize("shape", [W.reduced(W.MIXTRAL_8X7B, 600, 256, 384),
+                                   W.reduced(W.DSV3_DECODE, 128, 512, 256),
+                                   W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256)],
+                         ids=lambda s: s.name)
+def test_captured_layer_replays_bitwise(shape):
+    """MoELayer.capture: a CUDA graph of the whole layer replays to the eager bits, and picks
+    up new contents of the input buffer."""
+    inp = W.make_inputs(shape, device="cuda")
+    cfg = M.config_from_shape(shape)
+    layer = M.MoELayer(cfg, inp.w_router, inp.w_gate, inp.w_up, inp.w_down, inp.logit_bias)
+    x = inp.x.clone()
+    graph = layer.capture(x)
+    other = W.make_inputs(shape.replace(seed=shape.seed + 9), device="cuda", weights=False).x
+    eager = M.MoELayer(cfg, inp.w_router, inp.w_gate, inp.w_up, inp.w_down, inp.logit_bias)
+    for src in (inp.x, other, inp.x):
+        x.copy_(src)
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(layer.bufs.out, eager(src))
+    M.moe_check_device_error(layer.ws)
