@@ -37,7 +37,10 @@ size_t round_up(size_t v) { return (v + kWsAlign - 1) / kWsAlign * kWsAlign; }
 
 moe_status_t check_config(const moe_config_t* cfg, Shape* s) {
   if (cfg == nullptr) return fail(MOE_ERR_INVALID_ARG, "cfg is NULL");
-  if (cfg->T < 1) return fail(MOE_ERR_INVALID_ARG, "T must be >= 1 (got %lld)", (long long)cfg->T);
+  if (cfg->T < 1 || cfg->T > 2147483647LL)
+    return fail(MOE_ERR_INVALID_ARG, "T must be in [1, 2^31) (got %lld)", (long long)cfg->T);
+  if (cfg->d_model > (1LL << 24) || cfg->d_ff > (1LL << 24))
+    return fail(MOE_ERR_INVALID_ARG, "d_model and d_ff must be at most 2^24");
   if (cfg->d_model < 8 || cfg->d_model % 8 != 0)
     return fail(MOE_ERR_INVALID_ARG, "d_model must be a positive multiple of 8 (got %lld)",
                 (long long)cfg->d_model);

@@ -95,8 +95,9 @@ def test_workspace_size_and_bad_configs(lib):
     cfg = M.make_config(4096, 4096, 14336, 8, 2)
     n = M.workspace_size(cfg)
     assert n >= 256 + 16 * 8 * 4 + 4096 * 8 * 4
-    bad = [dict(E=0), dict(E=257), dict(k=0), dict(k=9), dict(T=0), dict(d_model=12),
-           dict(gating=3), dict(layout=2), dict(dtype=7)]
+    bad = [dict(E=0), dict(E=257), dict(k=0), dict(k=9), dict(T=0), dict(T=1 << 40),
+           dict(d_model=12), dict(d_model=1 << 26), dict(d_ff=1 << 26), dict(gating=3),
+           dict(layout=2), dict(dtype=7)]
     for b in bad:
         kw = dict(T=64, d_model=128, d_ff=256, E=8, k=2)
         kw.update({kk: v for kk, v in b.items() if kk in kw})
