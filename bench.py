@@ -185,6 +185,8 @@ def run_gpu(args) -> None:
         shape = shape.replace(name=f"{shape.name}_with_T{args.tokens}", T=args.tokens)
     if args.d_ff:
         shape = shape.replace(name=f"{shape.name}_with_f{args.d_ff}", d_ff=args.d_ff)
+    if args.experts:
+        shape = shape.replace(name=f"{shape.name}_with_E{args.experts}", E=args.experts)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -559,6 +561,9 @@ def main():
     ap.add_argument("--d-ff", type=int, default=0,
                     help="override d_ff of the workload (small profiling cases of the router "
                          "and dispatch kernels)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override E of the workload (small profiling cases with the full "
+                         "per-expert GEMM shapes)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--cpu-sample-tokens", type=int, default=64)
     ap.add_argument("--ref-sample-tokens", type=int, default=32)

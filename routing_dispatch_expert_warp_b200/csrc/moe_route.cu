@@ -447,29 +447,44 @@ __global__ void __launch_bounds__(256) topk_from_logits_kernel(
   for (int64_t t = warp; t < T; t += nwarps) {
     float zv[8];
     uint32_t key[8];
+    // the nsplit partial sums of each of the lane's 8 logits, added strictly in split order;
+    // the loads of 4 splits x 8 logits are issued together
+    float part[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const int e = lane + 32 * q;
-      float acc = 0.f;
+      part[q] = e < E ? z[t * E + e] : 0.f;
+    }
+    if (nsplit > 1) {
+      const int64_t stride = T * E;
+      int sp = 1;
+      for (; sp + 4 <= nsplit; sp += 4) {
+        float b[4][8];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int e = lane + 32 * q;
+            b[u][q] = e < E ? z[(sp + u) * stride + t * E + e] : 0.f;
+          }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) part[q] += b[u][q];
+      }
+      for (; sp < nsplit; ++sp)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int e = lane + 32 * q;
+          if (e < E) part[q] += z[sp * stride + t * E + e];
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int e = lane + 32 * q;
+      float acc = part[q];
       key[q] = 0u;
       if (e < E) {
-        if (nsplit == 1) {
-          acc = z[t * E + e];
-        } else {
-          // loads issued 8 at a time, additions strictly in split order
-          const float* zp = z + t * E + e;
-          const int64_t stride = T * E;
-          acc = zp[0];
-          int sp = 1;
-          for (; sp + 8 <= nsplit; sp += 8) {
-            float b8[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) b8[u] = zp[(sp + u) * stride];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) acc += b8[u];
-          }
-          for (; sp < nsplit; ++sp) acc += zp[sp * stride];
-        }
         if (bias != nullptr && bias_into_z) acc += bias[t * bias_stride + e];
         if (nsplit > 1 && logits != nullptr) logits[t * E + e] = acc;
         key[q] = order_key((bias != nullptr && bias_into_key) ? acc + bias[t * bias_stride + e]
