@@ -19,6 +19,7 @@ SHAPES = [
     W.reduced(W.DSV3_PREFILL_ZIPF, 1500, 256, 128),                     # capacity drops, E=256
     W.reduced(W.MIXTRAL_8X22B_MIXED, 2000, 128, 128, n_decode_tokens=8,
               layout=W.LAYOUT_PADDED),
+    W.reduced(W.DSV3_PREFILL_ZIPF, 1500, 256, 128, drop_policy=1),     # k histogram planes
 ]
 
 
