@@ -40,8 +40,8 @@
  *   - Errors: a host-side check fails with MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED /
  *     MOE_ERR_WORKSPACE before anything is enqueued; a CUDA launch error gives
  *     MOE_ERR_CUDA.  Errors found by kernels (an expert index out of range, a bounded
- *     device wait that ran out) are recorded in the workspace's status word and reported
- *     by moe_check_device_error().  moe_last_error() gives a message for the last failure
+ *     device wait that ran out, an expert-parallel row past its receive buffer) are
+ *     recorded in the workspace's status word and reported by moe_check_device_error().  moe_last_error() gives a message for the last failure
  *     on the calling thread.
  *   - Inputs are finite; NaN and Inf inputs give unspecified results.
  */
@@ -78,8 +78,10 @@ typedef enum { MOE_DROP_TOKEN_ORDER = 0, MOE_DROP_PICK_RANK = 1 } moe_drop_polic
 /*
  * One layer's shape and routing rule.
  *   T               tokens in the batch ([EP-checks] "First fix the workload unit": the
- *                   active tokens of this layer and batch), >= 1
- *   d_model, d_ff   model and expert hidden widths
+ *                   active tokens of this layer and batch), 1 .. 2^31 - 1, with T*k and
+ *                   the row count also below 2^31
+ *   d_model, d_ff   model and expert hidden widths (d_model a multiple of 8, d_ff of 4,
+ *                   both at most 2^24; bf16 expert FFNs need multiples of 64)
  *   E, k            experts (1..256) and picks per token (1..min(E, 8)) [EP-serving]
  *   gating          MOE_GATE_SOFTMAX: w_j = exp(z_j - z_max) / sum over the k picks;
  *                   MOE_GATE_SIGMOID: w_j = s(z_j) / sum over the k picks of s(z)
