@@ -37,23 +37,32 @@ L2_FLUSH_BYTES = 256 << 20
 
 # DRAM traffic of the grouped GEMM (gate/up + down launch, bytes per layer step) from one
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload and dispatch
-# mode, with the hash of the GEMM's sources at capture time: a changed kernel reports null.
+# mode, with the hash of the GEMM's source code (comments stripped) at capture time: a
+# changed kernel reports null.
 GEMM_SOURCES = ("routing_dispatch_expert_warp_b200/csrc/moe_ffn_tc.cu",
                 "routing_dispatch_expert_warp_b200/csrc/moe_device.cuh",
                 "routing_dispatch_expert_warp_b200/csrc/moe_internal.h")
 RECORDED_GEMM_TRAFFIC = {
     ("mixtral8x7b_prefill_T4096", False): {
-        "bytes": 3667147264, "sources": "096e841a32b1e8d6",
+        "bytes": 3667147264, "sources": "a4c968e4ba6a13bd",
         "profile": "profiles/grouped_gemm_tc_mixtral8x7b_T4096_traffic.md"},
 }
+
+
+def _code_only(text: str) -> str:
+    """C/C++ source without its comments and blank lines (a comment edit keeps the hash)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
 
 
 def gemm_source_hash() -> str:
     import hashlib
     h = hashlib.sha256()
     for rel in GEMM_SOURCES:
-        with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), rel)) as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

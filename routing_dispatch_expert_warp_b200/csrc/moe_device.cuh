@@ -116,7 +116,7 @@ __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
-// Tiled tensor loads (no multicast).  `map` is a __grid_constant__ kernel parameter.
+// Tiled tensor loads into this CTA's shared memory.  `map` is a __grid_constant__ kernel parameter.
 __device__ __forceinline__ void tma_load_2d(void* dst_smem, const CUtensorMap* map,
                                             uint64_t* bar, int32_t c0, int32_t c1) {
   asm volatile(

@@ -24,8 +24,8 @@
 //               its owner's buffer (the combine all-to-all fused with the weighted sum).
 // Ordering between ranks (counts written before plan, rows before the FFN, results before
 // combine) is the caller's: a stream-ordered barrier on multi-GPU runs, stream order when
-// the ranks share one GPU.  Stores and loads are plain 16-byte global accesses (no TMA,
-// no multicast), so the same kernels run on peer and local memory.
+// the ranks share one GPU.  Stores and loads are plain 16-byte global accesses (no TMA, no
+// copies shared across a cluster), so the same kernels run on peer and local memory.
 #include "moe_internal.h"
 
 namespace moe {
