@@ -449,7 +449,9 @@ moe_status_t moe_selftest_bounded_wait(void* ws, size_t ws_bytes, void* stream);
 
 /* Rows a receive buffer needs so that no distribution of picks can overflow it: world x
  * min(T*min(k, n_local), n_local*C) (C = capacity; T*min(k, n_local) when dropless),
- * with T the largest per-rank token count.  Reads only the sizes of cfg and ep; -2 (and
+ * with T the largest per-rank token count.  recv_rows must be the same on every rank (the
+ * kernels check a row against the sender's value), so pass the n_local of the rank that
+ * owns the most experts.  Reads only the sizes of cfg and ep; -2 (and
  * the reason in moe_last_error) when they are invalid. */
 int64_t moe_ep_recv_rows_bound(const moe_config_t* cfg, const moe_ep_config_t* ep);
 

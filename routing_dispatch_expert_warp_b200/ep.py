@@ -63,6 +63,20 @@ def local_experts(expert_rank: torch.Tensor, rank: int) -> torch.Tensor:
     return torch.nonzero(expert_rank.cpu() == rank).flatten()
 
 
+def common_recv_rows(cfg, expert_rank: torch.Tensor, world: int) -> int:
+    """Receive-buffer rows every rank allocates: the library's bound for the rank that owns
+    the most experts.  The kernels check a destination row against the sender's recv_rows,
+    so the value must be the same on every rank."""
+    owners = expert_rank.cpu().to(torch.int64)
+    most = int(torch.bincount(owners, minlength=world).max())
+    probe = MoeEpConfig(world=world, rank=0, ranks_per_node=1, n_local=most, expert_rank=None,
+                        recv_rows=0)
+    rows = int(_lib().moe_ep_recv_rows_bound(ctypes.byref(cfg), ctypes.byref(probe)))
+    if rows < 0:
+        check(1)
+    return rows
+
+
 class EpRank:
     """One rank's state for the EP layer: its config, workspace, routing buffers, count
     matrix, receive / hidden / result buffers and its local experts' weights."""
@@ -79,10 +93,7 @@ class EpRank:
         self.ep = MoeEpConfig(world=world, rank=rank, ranks_per_node=ranks_per_node,
                               n_local=n_local, expert_rank=_p(self.expert_rank), recv_rows=0)
         if recv_rows is None:
-            recv_rows = int(_lib().moe_ep_recv_rows_bound(ctypes.byref(cfg),
-                                                          ctypes.byref(self.ep)))
-            if recv_rows < 0:
-                check(1)
+            recv_rows = common_recv_rows(cfg, self.expert_rank, world)
         self.ep.recv_rows = recv_rows
         self.w_router, self.logit_bias = w_router, logit_bias
         self.w_gate, self.w_up, self.w_down = w_gate_local, w_up_local, w_down_local
@@ -295,6 +306,10 @@ class EpGroup:
         self.me = EpRank(cfg, world, rank, expert_rank, w_router, w_gate_local, w_up_local,
                          w_down_local, logit_bias, ranks_per_node, recv_rows, self.device)
         torch.cuda.synchronize(self.device)   # buffers exist before peers map them
+        sizes: list = [None] * world
+        dist.all_gather_object(sizes, int(self.me.ep.recv_rows), group=group)
+        if len(set(sizes)) != 1:   # rows are checked against the sender's value: one size
+            raise ValueError(f"recv_rows differs across ranks: {sizes}")
         ex = exchange_peer_pointers({"mats": self.me.count_mat.data_ptr(),
                                      "recv": self.me.recv_x.data_ptr(),
                                      "ybuf": self.me.y_recv.data_ptr()},
