@@ -51,7 +51,15 @@ Readings taken where the pages are silent (each one is listed in the design note
     group index) and picks its k experts among them;
   * selection-only bias: selection on fp32(z + b), gate weights from the unbiased z;
   * pick-rank drop order: within an expert, all first picks (token order), then all second
-    picks, and so on.
+    picks, and so on;
+  * score drop order: an expert keeps the C picks with the highest fp32 selection score
+    (equal scores -> lower token; NaN below every number); its kept picks take slots in
+    token order;
+  * second-choice counters ([EP-checks] "Top-2 does not insure against hot experts"): per
+    pick rank and expert the assignments and the kept assignments, and per pick rank the
+    tokens whose pick lies in another group than their first pick, a group being any
+    caller-given map of experts (the experts themselves, routing groups, owner ranks or
+    nodes).
 
 Every function below is pinned by tests in tests/test_oracle.py against hand-worked
 cases, brute force, closed forms or independent textbook routines.
@@ -71,6 +79,7 @@ BIAS_SCORE_AND_WEIGHT = 0
 BIAS_SELECTION_ONLY = 1
 DROP_TOKEN_ORDER = 0
 DROP_PICK_RANK = 1
+DROP_SCORE = 2
 
 
 # --------------------------------------------------------------------------------------
@@ -162,12 +171,17 @@ def capacity(capacity_factor: float, T: int, k: int, E: int) -> Optional[int]:
 #                        EP-checks, "Profile all-to-all ...": pack/permute before dispatch]
 # --------------------------------------------------------------------------------------
 def assign(idx, E: int, C: Optional[int], layout: int = LAYOUT_COMPACT,
-           drop_policy: int = DROP_TOKEN_ORDER) -> Dict[str, np.ndarray]:
+           drop_policy: int = DROP_TOKEN_ORDER, scores=None) -> Dict[str, np.ndarray]:
     """Walk the assignments in (expert ascending, token ascending) order, which for a
     top-k (distinct experts per token) is the same as walking tokens in order and giving
     each pick the next free slot of its expert.  With drop_policy = DROP_PICK_RANK the walk
     goes pick rank by pick rank (all first picks in token order, then all second picks...).
     Slot pos < C is kept, the rest dropped.
+    With drop_policy = DROP_SCORE the walk only decides which picks are kept: each
+    expert keeps the C picks with the highest fp32 selection score scores[t, e] (equal
+    scores: lower token first; a NaN score below every number), and its kept picks then
+    take slots 0, 1, ... in token order, so that without overflow the rows are those of
+    the token-order policy.
 
     Returns routed[E], kept[E], offsets[E+1] (bucket starts), assign_row[T, k]
     (-1 = dropped), token_of_row[rows] (-1 = unused padding row) and rows.
@@ -180,6 +194,16 @@ def assign(idx, E: int, C: Optional[int], layout: int = LAYOUT_COMPACT,
     next_slot = [0] * E
     if drop_policy == DROP_PICK_RANK:
         walk = [(t, j) for j in range(k) for t in range(T)]
+    elif drop_policy == DROP_SCORE:
+        if scores is None:
+            raise ValueError("DROP_SCORE needs the selection scores")
+        sc = np.asarray(scores, dtype=np.float32)
+
+        def order(tj):
+            v = float(sc[tj[0], idx[tj[0], tj[1]]])
+            return (1 if v != v else 0, -v if v == v else 0.0, tj[0])
+
+        walk = sorted(((t, j) for t in range(T) for j in range(k)), key=order)
     else:
         walk = [(t, j) for t in range(T) for j in range(k)]
     for t, j in walk:
@@ -188,6 +212,17 @@ def assign(idx, E: int, C: Optional[int], layout: int = LAYOUT_COMPACT,
         next_slot[e] += 1
     routed = np.array(next_slot, dtype=np.int64)
     kept = routed.copy() if C is None else np.minimum(routed, C)
+    if drop_policy == DROP_SCORE:
+        # priority rank -> kept or not; kept picks re-slotted in token order (a dropped
+        # pick keeps its priority rank, >= C)
+        is_kept = (pos < C) if C is not None else np.ones_like(pos, dtype=bool)
+        next_slot = [0] * E
+        for t in range(T):
+            for j in range(k):
+                if is_kept[t, j]:
+                    e = int(idx[t, j])
+                    pos[t, j] = next_slot[e]
+                    next_slot[e] += 1
     offsets = np.zeros(E + 1, dtype=np.int64)
     if layout == LAYOUT_COMPACT:
         for e in range(E):
@@ -342,11 +377,41 @@ def route(z32, k: int, gating: int, capacity_factor: float, layout: int = LAYOUT
     weights (on z32) and bookkeeping."""
     z32 = np.asarray(z32, dtype=np.float32)
     T, E = z32.shape
-    idx = select_topk(selection_scores(z32, bias, bias_mode), k, n_groups, topk_groups)
+    sel = selection_scores(z32, bias, bias_mode)
+    idx = select_topk(sel, k, n_groups, topk_groups)
     w = gate_weights(z32, idx, gating)
     C = capacity(capacity_factor, T, k, E)
-    a = assign(idx, E, C, layout, drop_policy)
+    a = assign(idx, E, C, layout, drop_policy, scores=sel)
     return dict(idx=idx, w=w, C=C, **a)
+
+
+def pick_rank_counts(idx, assign_row, E: int, group_of_expert=None) -> dict:
+    """The three second-choice counters of [EP-checks] "Top-2 does not insure against hot
+    experts", kept for every pick rank j:
+      routed[j][e]  picks of rank j that chose expert e (where the second choices go),
+      kept[j][e]    those of them that reached the expert FFN (the rest were dropped),
+      differs[j]    tokens whose pick j lies in another group than their pick 0, with
+                    group = group_of_expert[e] (default: the expert itself).
+    Shares (each over the T tokens): differs / T and 1 - sum_e kept[j][e] / T."""
+    idx = np.asarray(idx)
+    ar = np.asarray(assign_row)
+    T, k = idx.shape
+    grp = np.arange(E) if group_of_expert is None else np.asarray(group_of_expert)
+    routed = np.zeros((k, E), dtype=np.int64)
+    kept = np.zeros((k, E), dtype=np.int64)
+    differs = np.zeros(k, dtype=np.int64)
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            routed[j, e] += 1
+            if ar[t, j] >= 0:
+                kept[j, e] += 1
+            if grp[e] != grp[int(idx[t, 0])]:
+                differs[j] += 1
+    share = (lambda n: n / T) if T else (lambda n: 0.0)
+    return dict(routed=routed, kept=kept, differs=differs,
+                differs_share=[share(int(n)) for n in differs],
+                dropped_share=[share(T - int(kept[j].sum())) for j in range(k)])
 
 
 def moe_layer(x, w_router, logit_bias, w_gate, w_up, w_down, k: int, gating: int,

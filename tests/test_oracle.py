@@ -424,3 +424,54 @@ def test_pick_rank_slots_match_stable_sort(T, E, k, cf):
             later_kept = ((idx[:, j] == e) & (a["assign_row"][:, j] >= 0)).any()
             earlier_dropped = ((idx[:, :j] == e) & (a["assign_row"][:, :j] < 0)).any()
             assert not (later_kept and earlier_dropped)
+
+
+def test_score_drop_order_hand_case():
+    # scores consistent with the picks: each row's picks are its top-2
+    idx = np.array([[0, 1], [1, 0], [0, 1]])
+    sc = np.array([[0.5, 0.2], [0.7, 0.9], [0.9, 0.1]], dtype=np.float32)
+    a = O.assign(idx, 2, 2, drop_policy=O.DROP_SCORE, scores=sc)
+    # expert 0 holds t0 (0.5), t1 (0.7), t2 (0.9): keeps t2 and t1, drops t0's first pick;
+    # expert 1 holds t0 (0.2), t1 (0.9), t2 (0.1): keeps t1 and t0, drops t2's second pick.
+    # Kept picks take rows in token order: e0 rows 0, 1 = t1, t2; e1 rows 2, 3 = t0, t1.
+    assert a["assign_row"].tolist() == [[-1, 2], [3, 0], [1, -1]]
+    assert a["token_of_row"].tolist() == [1, 2, 0, 1]
+    assert a["kept"].tolist() == [2, 2] and a["routed"].tolist() == [3, 3]
+    # dropless: every policy gives the token-order rows
+    free = O.assign(idx, 2, None, drop_policy=O.DROP_SCORE, scores=sc)
+    assert free["assign_row"].tolist() == O.assign(idx, 2, None)["assign_row"].tolist()
+    # the second-choice counters of the same case
+    c = O.pick_rank_counts(idx, a["assign_row"], 2)
+    assert c["routed"].tolist() == [[2, 1], [1, 2]]
+    assert c["kept"].tolist() == [[1, 1], [1, 1]]
+    assert c["differs"].tolist() == [0, 3]
+    assert c["dropped_share"] == [1 / 3, 1 / 3]
+    same = O.pick_rank_counts(idx, a["assign_row"], 2, group_of_expert=[0, 0])
+    assert same["differs"].tolist() == [0, 0]
+
+
+def test_score_drop_ties_signed_zero_and_nan():
+    one = np.zeros((3, 1), dtype=np.int64)          # three tokens, one expert, k = 1
+    def kept(scores, C):
+        a = O.assign(one, 1, C, drop_policy=O.DROP_SCORE,
+                     scores=np.array(scores, dtype=np.float32).reshape(3, 1))
+        return [int(r >= 0) for r in a["assign_row"][:, 0]]
+    assert kept([0.0, -0.0, 0.0], 1) == [1, 0, 0]          # -0 ties +0: lower token wins
+    assert kept([-0.0, 0.0, 0.0], 2) == [1, 1, 0]
+    assert kept([np.nan, 1.0, 1.0], 2) == [0, 1, 1]        # NaN ranks below every number
+    assert kept([np.nan, -np.inf, np.nan], 2) == [1, 1, 0]
+    assert kept([1.0, 2.0, 3.0], 0) == [0, 0, 0]
+
+
+def test_score_drop_uses_selection_scores():
+    # three tokens all pick expert 0 (C = ceil(0.5 * 3 * 1 / 2) = 1); with the
+    # selection-only bias the priority is z + b: t0 (1 + 5) beats t2 (3 - 1) and t1 (2)
+    z = np.array([[1.0, 0.0], [2.0, 0.0], [3.0, 0.0]], dtype=np.float32)
+    b = np.array([[5.0, 0.0], [0.0, 0.0], [-1.0, 0.0]], dtype=np.float32)
+    r = O.route(z, 1, O.SOFTMAX, 0.5, bias=b, bias_mode=O.BIAS_SELECTION_ONLY,
+                drop_policy=O.DROP_SCORE)
+    assert r["C"] == 1 and r["idx"][:, 0].tolist() == [0, 0, 0]
+    assert r["assign_row"][:, 0].tolist() == [0, -1, -1]
+    # the same logits without the bias keep the highest logit, t2
+    r = O.route(z, 1, O.SOFTMAX, 0.5, drop_policy=O.DROP_SCORE)
+    assert r["assign_row"][:, 0].tolist() == [-1, -1, 0]

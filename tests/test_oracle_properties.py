@@ -70,3 +70,59 @@ def test_topk_is_best_subset_in_order(T, E, kk, seed, ties):
         best = max(itertools.combinations(range(E), k), key=lambda c: sorted(
             (float(z[t, e]) for e in c), reverse=True))
         assert sorted(float(z[t, e]) for e in idx[t]) == sorted(float(z[t, e]) for e in best)
+
+
+def _prio(v):
+    """Larger = kept first: NaN below every number; -0 equals +0."""
+    return (0, 0.0) if v != v else (1, float(v))
+
+
+@settings(max_examples=300, deadline=None)
+@given(T=st.integers(1, 40), E=st.integers(1, 12), kk=st.integers(1, 8),
+       cf=st.sampled_from([0.0, 0.2, 0.5, 1.0, 1.25, 3.0]), padded=st.booleans(),
+       seed=st.integers(0, 2**31 - 1), ties=st.booleans())
+def test_score_drop_invariants(T, E, kk, cf, padded, seed, ties):
+    """Score priority, checked by exchange: no dropped pick of an expert outranks one of its
+    kept picks (higher score, or equal score and lower token); kept picks fill their bucket
+    in token order; the counts, and the pick-rank counters, agree with the assignment."""
+    k = min(kk, E)
+    rng = np.random.default_rng(seed)
+    idx = _topk_rows(rng, T, E, k)
+    sc = (rng.integers(-2, 3, size=(T, E)) if ties else rng.standard_normal((T, E)))
+    sc = sc.astype(np.float32)
+    if ties:
+        sc[rng.random((T, E)) < 0.1] = np.nan
+    C = O.capacity(cf, T, k, E)
+    if padded and C is None:
+        return
+    layout = O.LAYOUT_PADDED if padded else O.LAYOUT_COMPACT
+    a = O.assign(idx, E, C, layout, O.DROP_SCORE, scores=sc)
+    ar = a["assign_row"]
+    routed = np.bincount(idx.ravel(), minlength=E)
+    kept = routed if C is None else np.minimum(routed, C)
+    assert (a["routed"] == routed).all() and (a["kept"] == kept).all()
+    for e in range(E):
+        picks = [(t, j) for t in range(T) for j in range(k) if idx[t, j] == e]
+        kp = [(t, j) for t, j in picks if ar[t, j] >= 0]
+        dr = [(t, j) for t, j in picks if ar[t, j] < 0]
+        assert len(kp) == kept[e]
+        for tk, jk in kp:
+            for td, jd in dr:
+                pk, pd = _prio(sc[tk, e]), _prio(sc[td, e])
+                assert pk > pd or (pk == pd and tk < td)
+        start = e * C if padded else int(kept[:e].sum())
+        assert [ar[t, j] for t, j in kp] == list(range(start, start + len(kp)))
+        assert [a["token_of_row"][ar[t, j]] for t, j in kp] == [t for t, _ in kp]
+    if C is None or (routed <= C).all():
+        tok = O.assign(idx, E, C, layout, O.DROP_TOKEN_ORDER)
+        assert (tok["assign_row"] == ar).all()
+    c = O.pick_rank_counts(idx, ar, E)
+    assert (c["routed"].sum(axis=0) == routed).all() and (c["routed"].sum(axis=1) == T).all()
+    assert (c["kept"].sum(axis=0) == kept).all()
+    st_ = O.load_stats(a["routed"], a["kept"], ar, C)
+    assert [T - int(c["kept"][j].sum()) for j in range(k)] == st_["dropped_by_rank"][:k]
+    assert c["differs"][0] == 0 and all(c["differs"][1:] == T)    # distinct picks
+    g = rng.integers(0, 3, size=E)
+    cg = O.pick_rank_counts(idx, ar, E, group_of_expert=g)
+    for j in range(k):
+        assert cg["differs"][j] == sum(1 for t in range(T) if g[idx[t, j]] != g[idx[t, 0]])
