@@ -55,7 +55,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 3
+#define MOE_ABI_VERSION 4
 #define MOE_MAX_EXPERTS 256
 #define MOE_MAX_TOPK 8
 
@@ -73,7 +73,11 @@ typedef enum { MOE_GATE_SOFTMAX = 0, MOE_GATE_SIGMOID = 1 } moe_gating_t;
 typedef enum { MOE_LAYOUT_COMPACT = 0, MOE_LAYOUT_PADDED = 1 } moe_layout_t;
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype_t;
 typedef enum { MOE_BIAS_SCORE_AND_WEIGHT = 0, MOE_BIAS_SELECTION_ONLY = 1 } moe_bias_mode_t;
-typedef enum { MOE_DROP_TOKEN_ORDER = 0, MOE_DROP_PICK_RANK = 1 } moe_drop_policy_t;
+typedef enum {
+  MOE_DROP_TOKEN_ORDER = 0,
+  MOE_DROP_PICK_RANK = 1,
+  MOE_DROP_SCORE = 2
+} moe_drop_policy_t;
 
 /*
  * One layer's shape and routing rule.
@@ -110,7 +114,13 @@ typedef enum { MOE_DROP_TOKEN_ORDER = 0, MOE_DROP_PICK_RANK = 1 } moe_drop_polic
  *                   MOE_DROP_PICK_RANK: all first picks (in token order) before all second
  *                   picks, and so on, so capacity drops later picks first ([EP-checks]
  *                   "Top-2 does not insure against hot experts": second choices measured
- *                   and dropped separately).
+ *                   and dropped separately);
+ *                   MOE_DROP_SCORE: an overflowing expert keeps its C picks of highest
+ *                   selection score (the fp32 score the top-k used; equal scores -> lower
+ *                   token; NaN below every number, -0 equal to +0); the kept picks take
+ *                   slots in token order, so without overflow the rows are those of
+ *                   MOE_DROP_TOKEN_ORDER.  Dispatch then needs the scores:
+ *                   moe_dispatch_scored (moe_layer_forward passes them itself).
  */
 typedef struct moe_config {
   int64_t T;
@@ -296,12 +306,38 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
  *   x_perm[assign_row[t, j], :] = x[t, :] for every kept pick; unused rows untouched.
  * x_perm may be NULL (x may then be NULL too): only the counts, offsets, assign_row and
  * token_of_row are produced, for moe_expert_ffn_gather.
+ * With MOE_DROP_SCORE this call returns MOE_ERR_INVALID_ARG: use moe_dispatch_scored.
  */
 moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t* topk_idx,
                           int32_t* routed_counts, int32_t* kept_counts,
                           int32_t* expert_offsets, int32_t* assign_row,
                           int32_t* token_of_row, void* x_perm, void* ws, size_t ws_bytes,
                           void* stream);
+
+/*
+ * moe_dispatch with the selection scores, for MOE_DROP_SCORE ([EP-checks] "Top-2 does not
+ * insure against hot experts": which assignments an overflowing expert keeps).  The score
+ * of pick (t, e) is logits[t, e], plus logit_bias[t * bias_row_stride + e] (fp32, one
+ * addition) when cfg->bias_mode is MOE_BIAS_SELECTION_ONLY; with MOE_BIAS_SCORE_AND_WEIGHT
+ * the bias is already inside the logits and logit_bias is not read.  Pass the logits and
+ * bias moe_route used, so that the drop decision follows the same score as the pick.
+ *   logits           [T, E] fp32 device array (required with MOE_DROP_SCORE)
+ *   logit_bias       NULL, or fp32 rows as in moe_route; bias_row_stride 0 or >= E
+ * Outputs, ownership and x_perm as in moe_dispatch.  Each expert with routed > C keeps the
+ * C picks of highest priority (score, then lower token); its kept picks take slots 0, 1,
+ * ... in token order; the rest get assign_row -1.  Scratch for the ranking comes from the
+ * workspace (moe_workspace_size counts it for MOE_DROP_SCORE).  Six kernels (five without
+ * x_perm), no host synchronisation.  With the other drop policies the scores are not read
+ * and the call equals moe_dispatch.  An expert index outside [0, E) is skipped and reported
+ * through the workspace status.
+ */
+moe_status_t moe_dispatch_scored(const moe_config_t* cfg, const void* x,
+                                 const int32_t* topk_idx, const float* logits,
+                                 const float* logit_bias, int64_t bias_row_stride,
+                                 int32_t* routed_counts, int32_t* kept_counts,
+                                 int32_t* expert_offsets, int32_t* assign_row,
+                                 int32_t* token_of_row, void* x_perm, void* ws,
+                                 size_t ws_bytes, void* stream);
 
 /*
  * moe_dispatch without a workspace.  The pages have no counterpart to this entry point; it
@@ -317,7 +353,8 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
  * allocating library routine).  Limits and behaviour:
  *   - ceil(T/256) * E * 4 bytes (times k with MOE_DROP_PICK_RANK) must fit in 1 MiB (e.g.
  *     T <= 262144 at E = 256); larger sizes return MOE_ERR_UNSUPPORTED with a message,
- *     before anything is enqueued.
+ *     before anything is enqueued.  MOE_DROP_SCORE (which needs the scores and more
+ *     scratch) returns MOE_ERR_UNSUPPORTED.
  *   - The first call on each device looks up the array's device address with that device
  *     current; make that first call before any stream capture.
  *   - Every call shares the one array: two calls that run on the GPU at the same time
@@ -406,6 +443,29 @@ moe_status_t moe_load_stats(const moe_config_t* cfg, const int32_t* routed_count
                             const int32_t* kept_counts, const int32_t* assign_row,
                             moe_load_stats_t* dev_out, moe_load_stats_t* host_out,
                             void* stream);
+
+/*
+ * Second-choice counters ([EP-checks] "Top-2 does not insure against hot experts": the
+ * share of tokens whose second choice differs from the first, where second choices go, and
+ * the share of second assignments that never reached the experts), for every pick rank j
+ * (j = 0 the first choice, j = 1 the second, ...):
+ *   routed_by_rank[j * E + e]  picks of rank j that chose expert e         ([k, E] int32)
+ *   kept_by_rank[j * E + e]    those of them kept (assign_row >= 0)        ([k, E] int32)
+ *   differs_by_rank[j]         tokens whose pick j lies in another group   ([k] int32)
+ *                              than their pick 0; differs_by_rank[0] = 0
+ * group_of_expert: NULL (a group is one expert, so for distinct picks differs = T for
+ * j >= 1), or an [E] int32 device array mapping experts to any grouping the caller wants to
+ * watch: routing groups, owner ranks, nodes.  Shares over the T tokens: differs / T, and
+ * 1 - Sum_e kept_by_rank[j, e] / T dropped.  topk_idx and assign_row as moe_route and
+ * moe_dispatch produce them.  One kernel, integer counts (deterministic), no host
+ * synchronisation; every output element is written.  An expert index outside [0, E) is
+ * skipped and reported through the workspace status.
+ */
+moe_status_t moe_pick_rank_counts(const moe_config_t* cfg, const int32_t* topk_idx,
+                                  const int32_t* assign_row, const int32_t* group_of_expert,
+                                  int32_t* routed_by_rank, int32_t* kept_by_rank,
+                                  int32_t* differs_by_rank, void* ws, size_t ws_bytes,
+                                  void* stream);
 
 /*
  * The whole layer: moe_route, moe_dispatch, moe_expert_ffn, moe_combine and (when

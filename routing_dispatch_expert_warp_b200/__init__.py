@@ -20,10 +20,11 @@ SOFTMAX, SIGMOID = 0, 1
 COMPACT, PADDED = 0, 1
 F32, BF16 = 0, 1
 BIAS_SCORE_AND_WEIGHT, BIAS_SELECTION_ONLY = 0, 1
-DROP_TOKEN_ORDER, DROP_PICK_RANK = 0, 1
+DROP_TOKEN_ORDER, DROP_PICK_RANK, DROP_SCORE = 0, 1, 2
 
 __all__ = ["MoEError", "make_config", "workspace_size", "capacity", "max_rows",
-           "alloc_workspace", "moe_route", "moe_dispatch", "moe_dispatch_static_scratch",
+           "alloc_workspace", "moe_route", "moe_dispatch", "moe_dispatch_scored",
+           "moe_dispatch_static_scratch", "moe_pick_rank_counts",
            "moe_expert_ffn", "moe_expert_ffn_gather", "moe_expert_ffn_combine", "moe_combine",
            "moe_load_stats", "moe_layer_forward", "moe_check_device_error",
            "moe_selftest_bounded_wait", "set_wait_limit_ns", "kernel_launch_count",
@@ -107,6 +108,30 @@ def moe_dispatch(cfg, x, topk_idx, routed_counts, kept_counts, expert_offsets, a
                               _ptr(kept_counts), _ptr(expert_offsets), _ptr(assign_row),
                               _ptr(token_of_row), _ptr(x_perm), _ptr(ws), ws.numel(),
                               _stream(stream)))
+
+
+def moe_dispatch_scored(cfg, x, topk_idx, logits, logit_bias, routed_counts, kept_counts,
+                        expert_offsets, assign_row, token_of_row, x_perm, ws, stream=None):
+    """moe_dispatch with the selection scores (needed for DROP_SCORE): logits [T, E] fp32
+    as moe_route wrote them, logit_bias None, [E] or [T, >=E] fp32 as given to moe_route."""
+    stride = 0 if (logit_bias is None or logit_bias.dim() == 1) else logit_bias.shape[1]
+    check(_lib().moe_dispatch_scored(
+        ctypes.byref(cfg), _ptr(x), _ptr(topk_idx), _ptr(logits), _ptr(logit_bias), stride,
+        _ptr(routed_counts), _ptr(kept_counts), _ptr(expert_offsets), _ptr(assign_row),
+        _ptr(token_of_row), _ptr(x_perm), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_pick_rank_counts(cfg, topk_idx, assign_row, ws, group_of_expert=None, stream=None):
+    """Second-choice counters: returns (routed [k, E], kept [k, E], differs [k]) int32 device
+    tensors, enqueued on the stream (see include/moe.h)."""
+    dev = topk_idx.device
+    routed = torch.empty((cfg.k, cfg.E), dtype=torch.int32, device=dev)
+    kept = torch.empty((cfg.k, cfg.E), dtype=torch.int32, device=dev)
+    differs = torch.empty(cfg.k, dtype=torch.int32, device=dev)
+    check(_lib().moe_pick_rank_counts(
+        ctypes.byref(cfg), _ptr(topk_idx), _ptr(assign_row), _ptr(group_of_expert),
+        _ptr(routed), _ptr(kept), _ptr(differs), _ptr(ws), ws.numel(), _stream(stream)))
+    return routed, kept, differs
 
 
 def moe_dispatch_static_scratch(cfg, x, topk_idx, routed_counts, kept_counts, expert_offsets,
@@ -264,6 +289,12 @@ class MoELayer:
         return self.bufs.out
 
     __call__ = forward
+
+    def pick_rank_counts(self, group_of_expert=None, stream=None):
+        """The second-choice counters of the last forward: (routed [k, E], kept [k, E],
+        differs [k]) int32 device tensors; group_of_expert: None or an [E] int32 map."""
+        return moe_pick_rank_counts(self.cfg, self.bufs.topk_idx, self.bufs.assign_row,
+                                    self.ws, group_of_expert, stream)
 
     def capture(self, x: torch.Tensor) -> "torch.cuda.CUDAGraph":
         """Record one forward on the fixed input buffer x into a CUDA graph: replay() then

@@ -97,6 +97,8 @@ PROTOTYPES = {
                           c_vp]),
     "moe_dispatch": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                              c_vp, c_sz, c_vp]),
+    "moe_dispatch_scored": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp,
+                                    c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "moe_dispatch_static_scratch": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                             c_vp, c_vp, c_vp]),
     "moe_expert_ffn": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
@@ -107,6 +109,8 @@ PROTOTYPES = {
                                        c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_sz, c_vp]),
     "moe_combine": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_vp]),
     "moe_load_stats": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, P(MoeLoadStats), c_vp]),
+    "moe_pick_rank_counts": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                     c_sz, c_vp]),
     "moe_layer_forward": (c_i32, [P(MoeConfig), P(MoeLayerInputs), P(MoeLayerBuffers), c_vp,
                                   c_sz, c_vp]),
     "moe_check_device_error": (c_i32, [c_vp, c_sz, c_vp]),

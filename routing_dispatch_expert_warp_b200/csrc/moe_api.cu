@@ -73,7 +73,8 @@ moe_status_t check_config(const moe_config_t* cfg, Shape* s) {
   }
   if (cfg->bias_mode != MOE_BIAS_SCORE_AND_WEIGHT && cfg->bias_mode != MOE_BIAS_SELECTION_ONLY)
     return fail(MOE_ERR_INVALID_ARG, "unknown bias_mode %d", cfg->bias_mode);
-  if (cfg->drop_policy != MOE_DROP_TOKEN_ORDER && cfg->drop_policy != MOE_DROP_PICK_RANK)
+  if (cfg->drop_policy != MOE_DROP_TOKEN_ORDER && cfg->drop_policy != MOE_DROP_PICK_RANK &&
+      cfg->drop_policy != MOE_DROP_SCORE)
     return fail(MOE_ERR_INVALID_ARG, "unknown drop_policy %d", cfg->drop_policy);
   s->T = cfg->T;
   s->d = cfg->d_model;
@@ -160,6 +161,8 @@ WsLayout workspace_layout(const Shape& s) {
   off += round_up(static_cast<size_t>(s.E) * sizeof(int32_t));
   l.arrive = off;
   off += round_up(static_cast<size_t>(s.T) * ((s.d + 255) / 256) * sizeof(int32_t));
+  l.score = off;
+  off += round_up(dispatch_score_scratch_bytes(s));
   l.total = off;
   return l;
 }
@@ -298,6 +301,20 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
                           int32_t* expert_offsets, int32_t* assign_row,
                           int32_t* token_of_row, void* x_perm, void* ws, size_t ws_bytes,
                           void* stream) {
+  MOE_REQUIRE(cfg == nullptr || cfg->drop_policy != MOE_DROP_SCORE,
+              "moe_dispatch: MOE_DROP_SCORE needs the selection scores (moe_dispatch_scored)");
+  return moe_dispatch_scored(cfg, x, topk_idx, nullptr, nullptr, 0, routed_counts,
+                             kept_counts, expert_offsets, assign_row, token_of_row, x_perm, ws,
+                             ws_bytes, stream);
+}
+
+moe_status_t moe_dispatch_scored(const moe_config_t* cfg, const void* x,
+                                 const int32_t* topk_idx, const float* logits,
+                                 const float* logit_bias, int64_t bias_row_stride,
+                                 int32_t* routed_counts, int32_t* kept_counts,
+                                 int32_t* expert_offsets, int32_t* assign_row,
+                                 int32_t* token_of_row, void* x_perm, void* ws,
+                                 size_t ws_bytes, void* stream) {
   Shape s;
   moe_status_t st = check_config(cfg, &s);
   if (st != MOE_OK) return st;
@@ -308,10 +325,21 @@ moe_status_t moe_dispatch(const moe_config_t* cfg, const void* x, const int32_t*
               "moe_dispatch: NULL pointer");
   MOE_REQUIRE(x_perm == nullptr || (aligned16(x) && aligned16(x_perm)),
               "moe_dispatch: x and x_perm must be 16-byte aligned");
+  DispatchScores scores{};
+  if (s.drop_policy == MOE_DROP_SCORE) {
+    MOE_REQUIRE(logits != nullptr, "moe_dispatch_scored: logits is NULL");
+    MOE_REQUIRE(bias_row_stride == 0 || bias_row_stride >= s.E,
+                "moe_dispatch_scored: bias_row_stride must be 0 or >= E");
+    scores.logits = logits;
+    scores.bias = s.bias_mode == MOE_BIAS_SELECTION_ONLY ? logit_bias : nullptr;
+    scores.bias_stride = bias_row_stride;
+    scores.scratch = static_cast<uint8_t*>(ws) + lay.score;
+  }
   int32_t* hist = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + lay.hist);
   cudaError_t err = launch_dispatch(s, x, topk_idx, routed_counts, kept_counts, expert_offsets,
                                     assign_row, token_of_row, x_perm, hist, ws_status(ws, lay),
-                                    g_wait_ns.load(), static_cast<cudaStream_t>(stream));
+                                    g_wait_ns.load(), static_cast<cudaStream_t>(stream),
+                                    s.drop_policy == MOE_DROP_SCORE ? &scores : nullptr);
   if (err != cudaSuccess) return cuda_fail(err, "moe_dispatch launch");
   return MOE_OK;
 }
@@ -329,6 +357,10 @@ moe_status_t moe_dispatch_static_scratch(const moe_config_t* cfg, const void* x,
               "moe_dispatch_static_scratch: NULL pointer");
   MOE_REQUIRE(aligned16(x) && aligned16(x_perm),
               "moe_dispatch_static_scratch: x and x_perm must be 16-byte aligned");
+  if (s.drop_policy == MOE_DROP_SCORE)
+    return fail(MOE_ERR_UNSUPPORTED,
+                "moe_dispatch_static_scratch: MOE_DROP_SCORE needs the selection scores and "
+                "workspace scratch (use moe_dispatch_scored)");
   const size_t need = dispatch_hist_bytes(s);
   if (need > kStaticDispatchHistBytes)
     return fail(MOE_ERR_UNSUPPORTED,
@@ -473,6 +505,25 @@ moe_status_t moe_load_stats(const moe_config_t* cfg, const int32_t* routed_count
   return MOE_OK;
 }
 
+moe_status_t moe_pick_rank_counts(const moe_config_t* cfg, const int32_t* topk_idx,
+                                  const int32_t* assign_row, const int32_t* group_of_expert,
+                                  int32_t* routed_by_rank, int32_t* kept_by_rank,
+                                  int32_t* differs_by_rank, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  Shape s;
+  moe_status_t st = check_config(cfg, &s);
+  if (st != MOE_OK) return st;
+  WsLayout lay;
+  if ((st = check_ws(s, ws, ws_bytes, &lay)) != MOE_OK) return st;
+  MOE_REQUIRE(topk_idx && assign_row && routed_by_rank && kept_by_rank && differs_by_rank,
+              "moe_pick_rank_counts: NULL pointer");
+  cudaError_t err = launch_pick_rank_counts(s, topk_idx, assign_row, group_of_expert,
+                                            routed_by_rank, kept_by_rank, differs_by_rank,
+                                            ws_status(ws, lay), static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_pick_rank_counts launch");
+  return MOE_OK;
+}
+
 moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_layer_inputs_t* in,
                                const moe_layer_buffers_t* b, void* ws, size_t ws_bytes,
                                void* stream) {
@@ -480,9 +531,17 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_layer_inputs_t
   moe_status_t st = moe_route(cfg, in->x, in->w_router, in->logit_bias, in->bias_row_stride,
                               b->logits, b->topk_idx, b->topk_w, ws, ws_bytes, stream);
   if (st != MOE_OK) return st;
-  st = moe_dispatch(cfg, in->x, b->topk_idx, b->routed_counts, b->kept_counts,
-                    b->expert_offsets, b->assign_row, b->token_of_row, b->x_perm, ws, ws_bytes,
-                    stream);
+  // the logits moe_route wrote: the caller's array, else the workspace's
+  const float* z = b->logits;
+  if (z == nullptr) {
+    Shape s;
+    if ((st = check_config(cfg, &s)) != MOE_OK) return st;
+    z = reinterpret_cast<const float*>(static_cast<const uint8_t*>(ws) +
+                                       workspace_layout(s).logits);
+  }
+  st = moe_dispatch_scored(cfg, in->x, b->topk_idx, z, in->logit_bias, in->bias_row_stride,
+                           b->routed_counts, b->kept_counts, b->expert_offsets, b->assign_row,
+                           b->token_of_row, b->x_perm, ws, ws_bytes, stream);
   if (st != MOE_OK) return st;
   if (b->x_perm != nullptr)
     st = moe_expert_ffn(cfg, b->x_perm, b->expert_offsets, b->kept_counts, in->w_gate,

@@ -11,7 +11,12 @@
 // local permutation.
 //
 // Assignment order: within expert e, assignments are ranked by token index (a token picks
-// an expert at most once, so its pick slot j does not matter).  slot < C is kept.
+// an expert at most once, so its pick slot j does not matter).  slot < C is kept.  With
+// pick-rank drops the ranking goes pick rank by pick rank.  With score drops ("MoE expert
+// parallelism needs measurements before launch", "Top-2 does not insure against hot
+// experts": the second route has its own capacity and drops) an overflowing expert keeps
+// its C picks of highest selection score (equal scores: lower token), found by a radix
+// selection over each expert's picks; the kept picks are then ranked by token index.
 //
 // Kernels (no host synchronisation anywhere):
 //   1. count:  block b of 256 tokens builds, per warp w and expert e, the 32-bit mask of
@@ -25,18 +30,42 @@
 #include <mutex>
 
 #include "moe_internal.h"
+#include "moe_keys.cuh"
 
 namespace moe {
 namespace {
 
 constexpr int kWarps = kDispatchBlockTokens / 32;
 
+// Which picks the ranking kernels count.  thr == nullptr: all of them.  Otherwise pick
+// (t, e) counts (is kept) iff pick_priority(score of (t, e), t) >= thr[e], the score being
+// the fp32 logit plus, when the bias only steers selection, the fp32 bias: the same single
+// addition the top-k takes its decision on.
+struct ScoreFilter {
+  const uint64_t* thr;
+  const float* logits;
+  const float* bias;
+  int64_t bias_stride;
+};
+
+__device__ __forceinline__ float selection_score(const ScoreFilter& f, int64_t t, int E, int e) {
+  float v = f.logits[t * E + e];
+  if (f.bias != nullptr) v = v + f.bias[t * f.bias_stride + e];
+  return v;
+}
+
+__device__ __forceinline__ bool filter_keeps(const ScoreFilter& f, int64_t t, int E, int e) {
+  return f.thr == nullptr || pick_priority(selection_score(f, t, E, e), t) >= f.thr[e];
+}
+
 // Fill masks[w][e] for the block's tokens, counting the picks of `plane` only when the
 // assignments are ranked pick rank by pick rank (planes == k), all picks otherwise
-// (planes == 1).  Invalid experts are recorded and skipped.
+// (planes == 1), and only the picks the filter keeps.  Invalid experts are recorded and
+// skipped.
 __device__ __forceinline__ void build_masks(const int32_t* __restrict__ topk_idx, int64_t T,
                                             int k, int E, uint32_t (*masks)[MOE_MAX_EXPERTS],
-                                            DevStatus* status, int plane, int planes) {
+                                            DevStatus* status, int plane, int planes,
+                                            const ScoreFilter& flt) {
   for (int i = threadIdx.x; i < kWarps * MOE_MAX_EXPERTS; i += blockDim.x)
     (&masks[0][0])[i] = 0u;
   __syncthreads();
@@ -51,6 +80,7 @@ __device__ __forceinline__ void build_masks(const int32_t* __restrict__ topk_idx
         record_error(status, DEV_BAD_EXPERT, 1, static_cast<unsigned long long>(t * k + j));
         continue;
       }
+      if (!filter_keeps(flt, t, E, e)) continue;
       atomicOr(&masks[w][e], bit);
     }
   }
@@ -60,10 +90,10 @@ __device__ __forceinline__ void build_masks(const int32_t* __restrict__ topk_idx
 // hist[b][p][e]: assignments of plane p (a pick rank, or all picks) from block b to expert e.
 __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_count_kernel(
     const int32_t* __restrict__ topk_idx, int64_t T, int k, int E, int planes,
-    int32_t* __restrict__ hist, DevStatus* status) {
+    int32_t* __restrict__ hist, DevStatus* status, ScoreFilter flt) {
   __shared__ uint32_t masks[kWarps][MOE_MAX_EXPERTS];
   for (int p = 0; p < planes; ++p) {
-    build_masks(topk_idx, T, k, E, masks, p == 0 ? status : nullptr, p, planes);
+    build_masks(topk_idx, T, k, E, masks, p == 0 ? status : nullptr, p, planes, flt);
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
       int c = 0;
 #pragma unroll
@@ -82,12 +112,14 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_count_kernel(
 // rank (pick-rank drops: plane p starts after the totals of planes < p).  Then, plane by
 // plane, slot = plane start + base from earlier blocks + earlier warps of this block +
 // popcount(mask & lanes below me), kept iff slot < C, row = offset + slot.  Finally the
-// rows no assignment uses are marked -1 in token_of_row.
+// rows no assignment uses are marked -1 in token_of_row.  With a filter, hist counts the
+// kept picks only, the others get row -1, and routed (the demand, counted by an earlier
+// unfiltered pass) is left as it is.
 __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
     const int32_t* __restrict__ topk_idx, int64_t T, int k, int E, int64_t C, int layout,
     int planes, int64_t nblk, const int32_t* __restrict__ hist, int32_t* __restrict__ routed,
     int32_t* __restrict__ kept, int32_t* __restrict__ offsets, int32_t* __restrict__ assign_row,
-    int32_t* __restrict__ token_of_row, int64_t max_rows) {
+    int32_t* __restrict__ token_of_row, int64_t max_rows, ScoreFilter flt) {
   static_assert(kDispatchBlockTokens == MOE_MAX_EXPERTS, "one thread per expert");
   __shared__ uint32_t masks[kWarps][MOE_MAX_EXPERTS];
   __shared__ int32_t wbase[kWarps][MOE_MAX_EXPERTS];
@@ -136,7 +168,7 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
     off_s[e] = static_cast<int32_t>(off);
     kept_s[e] = static_cast<int32_t>(kp);
     if (blockIdx.x == 0) {
-      routed[e] = static_cast<int32_t>(run);
+      if (flt.thr == nullptr) routed[e] = static_cast<int32_t>(run);
       kept[e] = static_cast<int32_t>(kp);
       offsets[e] = static_cast<int32_t>(off);
       if (e == E - 1)
@@ -151,7 +183,7 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
   const uint32_t below = (1u << (threadIdx.x & 31)) - 1u;
   for (int p = 0; p < planes; ++p) {
     __syncthreads();  // pbase / off_s ready; masks of the previous plane no longer read
-    build_masks(topk_idx, T, k, E, masks, nullptr, p, planes);
+    build_masks(topk_idx, T, k, E, masks, nullptr, p, planes, flt);
     if (e < E) {
       int32_t wb = pbase[p][e];
 #pragma unroll
@@ -166,7 +198,7 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
         if (planes > 1 && j != p) continue;
         const int ee = topk_idx[t * k + j];
         int32_t row = -1;
-        if (ee >= 0 && ee < E) {
+        if (ee >= 0 && ee < E && filter_keeps(flt, t, E, ee)) {
           const int64_t slot = wbase[w][ee] + __popc(masks[w][ee] & below);
           if (C < 0 || slot < C) {
             row = off_s[ee] + static_cast<int32_t>(slot);
@@ -189,6 +221,132 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
   } else {
     for (int64_t r = total_kept + first; r < max_rows; r += stride) token_of_row[r] = -1;
   }
+}
+
+// Score-priority threshold of expert e (block e).  Its picks sit in rows
+// [offsets[e], offsets[e] + routed[e]) of the dropless token-order layout, token_of_row
+// giving each row's token.  When routed[e] > C the block writes every pick's priority to
+// its own rows of prio, then finds the C-th largest by most-significant-digit radix
+// selection, 8 bits a pass: a pass counts the candidates (priorities whose higher digits
+// equal the prefix found so far) per digit value, and the digit at which the running count
+// from the top reaches the rank still needed joins the prefix.  Priorities are unique per
+// expert, so after 8 passes the prefix is the C-th largest and the kept picks are exactly
+// those at or above it.  thr[e] = 0 keeps every pick (no overflow); C == 0 keeps none.
+constexpr int kSelectThreads = 512;
+
+__global__ void __launch_bounds__(kSelectThreads) score_select_kernel(
+    const int32_t* __restrict__ routed, const int32_t* __restrict__ offsets,
+    const int32_t* __restrict__ token_of_row, ScoreFilter flt, int E, int64_t C,
+    uint64_t* __restrict__ prio, uint64_t* __restrict__ thr) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint64_t s_prefix;
+  __shared__ uint32_t s_need;
+  const int e = blockIdx.x;
+  const int64_t n = routed[e];
+  if (C < 0 || n <= C) {
+    if (threadIdx.x == 0) thr[e] = 0;
+    return;
+  }
+  if (C == 0) {
+    if (threadIdx.x == 0) thr[e] = ~0ull;
+    return;
+  }
+  const int64_t start = offsets[e];
+  uint64_t* seg = prio + start;
+  for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+    const int64_t t = token_of_row[start + i];
+    seg[i] = pick_priority(selection_score(flt, t, E, e), t);
+  }
+  const int lane = threadIdx.x & 31;
+  uint64_t prefix = 0, mask = 0;
+  uint32_t need = static_cast<uint32_t>(C);  // 1-based rank among the candidates
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0u;
+    __syncthreads();  // seg written (first pass); s_prefix read by all (later passes)
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+      const uint64_t v = seg[i];
+      if ((v & mask) == prefix) atomicAdd(&hist[(v >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      // lane l holds digit values 255 - 8l down to 248 - 8l; counts run from the top
+      uint32_t c[8], sum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        c[i] = hist[255 - 8 * lane - i];
+        sum += c[i];
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      uint32_t acc = incl - sum;
+      if (acc < need && incl >= need) {  // exactly one lane
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (acc < need && acc + c[i] >= need) {
+            s_prefix = prefix | (static_cast<uint64_t>(255 - 8 * lane - i) << shift);
+            s_need = need - acc;
+          }
+          acc += c[i];
+        }
+      }
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    need = s_need;
+    mask |= 0xFFull << shift;
+  }
+  if (threadIdx.x == 0) thr[e] = prefix;
+}
+
+// Second-choice counters ("MoE expert parallelism needs measurements before launch", "Top-2
+// does not insure against hot experts").  Block j takes pick rank j over all tokens:
+// shared counts per expert of the picks and of the kept picks, and of the tokens whose
+// pick j lies in another group than their pick 0; then it writes its row of each output.
+// Integer sums: the result does not depend on the order of the additions.
+constexpr int kCountThreads = 1024;
+
+__global__ void __launch_bounds__(kCountThreads) pick_rank_counts_kernel(
+    const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ assign_row,
+    const int32_t* __restrict__ group_of_expert, int64_t T, int k, int E,
+    int32_t* __restrict__ routed, int32_t* __restrict__ kept, int32_t* __restrict__ differs,
+    DevStatus* status) {
+  __shared__ uint32_t r_s[MOE_MAX_EXPERTS];
+  __shared__ uint32_t k_s[MOE_MAX_EXPERTS];
+  __shared__ uint32_t d_s;
+  const int j = blockIdx.x;
+  for (int e = threadIdx.x; e < MOE_MAX_EXPERTS; e += blockDim.x) {
+    r_s[e] = 0u;
+    k_s[e] = 0u;
+  }
+  if (threadIdx.x == 0) d_s = 0u;
+  __syncthreads();
+  uint32_t dif = 0;
+  for (int64_t t = threadIdx.x; t < T; t += blockDim.x) {
+    const int e = topk_idx[t * k + j];
+    const int e0 = topk_idx[t * k];
+    if (e < 0 || e >= E || e0 < 0 || e0 >= E) {
+      record_error(status, DEV_BAD_EXPERT, 4, static_cast<unsigned long long>(t * k + j));
+      continue;
+    }
+    atomicAdd(&r_s[e], 1u);
+    if (assign_row[t * k + j] >= 0) atomicAdd(&k_s[e], 1u);
+    const bool other = group_of_expert != nullptr ? group_of_expert[e] != group_of_expert[e0]
+                                                  : e != e0;
+    dif += other ? 1u : 0u;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dif += __shfl_xor_sync(0xffffffffu, dif, o);
+  if ((threadIdx.x & 31) == 0 && dif != 0u) atomicAdd(&d_s, dif);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    routed[static_cast<int64_t>(j) * E + e] = static_cast<int32_t>(r_s[e]);
+    kept[static_cast<int64_t>(j) * E + e] = static_cast<int32_t>(k_s[e]);
+  }
+  if (threadIdx.x == 0) differs[j] = static_cast<int32_t>(d_s);
 }
 
 // Token-major bulk copy.  One thread per block issues everything: a ring of NBUF shared
@@ -278,23 +436,99 @@ __global__ void __launch_bounds__(32) permute_rows_kernel(
 
 }  // namespace
 
+namespace {
+inline size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+// Scratch of the score-priority dispatch: the dropless token-order layout of all picks
+// (row of each pick, token of each row, kept and offsets of that layout), the threshold
+// of each expert, and each pick's priority in its dropless row.
+struct ScoreScratch {
+  int32_t* assign_row;    // [T * k]
+  int32_t* token_of_row;  // [T * k]
+  int32_t* kept;          // [E]
+  int32_t* offsets;       // [E + 1]
+  uint64_t* thr;          // [E]
+  uint64_t* prio;         // [T * k]
+};
+
+ScoreScratch score_scratch(const Shape& s, void* base) {
+  const size_t a = static_cast<size_t>(s.T) * s.k;
+  uint8_t* p = static_cast<uint8_t*>(base);
+  ScoreScratch sc;
+  sc.assign_row = reinterpret_cast<int32_t*>(p);
+  p += round256(a * sizeof(int32_t));
+  sc.token_of_row = reinterpret_cast<int32_t*>(p);
+  p += round256(a * sizeof(int32_t));
+  sc.kept = reinterpret_cast<int32_t*>(p);
+  p += round256(static_cast<size_t>(s.E) * sizeof(int32_t));
+  sc.offsets = reinterpret_cast<int32_t*>(p);
+  p += round256(static_cast<size_t>(s.E + 1) * sizeof(int32_t));
+  sc.thr = reinterpret_cast<uint64_t*>(p);
+  p += round256(static_cast<size_t>(s.E) * sizeof(uint64_t));
+  sc.prio = reinterpret_cast<uint64_t*>(p);
+  return sc;
+}
+}  // namespace
+
+size_t dispatch_score_scratch_bytes(const Shape& s) {
+  if (s.drop_policy != MOE_DROP_SCORE) return 0;
+  const size_t a = static_cast<size_t>(s.T) * s.k;
+  return 2 * round256(a * sizeof(int32_t)) + round256(static_cast<size_t>(s.E) * 4) +
+         round256(static_cast<size_t>(s.E + 1) * 4) + round256(static_cast<size_t>(s.E) * 8) +
+         round256(a * sizeof(uint64_t));
+}
+
 cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_idx,
                             int32_t* routed, int32_t* kept, int32_t* offsets,
                             int32_t* assign_row, int32_t* token_of_row, void* x_perm,
                             int32_t* hist, DevStatus* status, uint64_t wait_ns,
-                            cudaStream_t st) {
+                            cudaStream_t st, const DispatchScores* scores) {
   const int64_t nblk = dispatch_blocks(s.T);
   cudaError_t err;
   const int planes = dispatch_planes(s);
-  dispatch_count_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
-      topk_idx, s.T, s.k, s.E, planes, hist, status);
-  note_launch();
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  dispatch_rank_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
-      topk_idx, s.T, s.k, s.E, s.C, s.layout, planes, nblk, hist, routed, kept, offsets,
-      assign_row, token_of_row, s.max_rows);
-  note_launch();
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const ScoreFilter all{nullptr, nullptr, nullptr, 0};
+  if (s.drop_policy == MOE_DROP_SCORE) {
+    if (scores == nullptr || scores->logits == nullptr || scores->scratch == nullptr)
+      return cudaErrorInvalidValue;
+    const ScoreScratch sc = score_scratch(s, scores->scratch);
+    ScoreFilter flt{nullptr, scores->logits, scores->bias, scores->bias_stride};
+    // 1. every pick, dropless, in token order: routed, and each expert's picks grouped
+    dispatch_count_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
+        topk_idx, s.T, s.k, s.E, 1, hist, status, all);
+    note_launch();
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    dispatch_rank_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
+        topk_idx, s.T, s.k, s.E, -1, MOE_LAYOUT_COMPACT, 1, nblk, hist, routed, sc.kept,
+        sc.offsets, sc.assign_row, sc.token_of_row, s.T * s.k, all);
+    note_launch();
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    // 2. per expert, the priority of its C-th best pick
+    score_select_kernel<<<static_cast<unsigned>(s.E), kSelectThreads, 0, st>>>(
+        routed, sc.offsets, sc.token_of_row, flt, s.E, s.C, sc.prio, sc.thr);
+    note_launch();
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    // 3. the kept picks, ranked in token order inside their buckets
+    flt.thr = sc.thr;
+    dispatch_count_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
+        topk_idx, s.T, s.k, s.E, 1, hist, nullptr, flt);
+    note_launch();
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    dispatch_rank_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
+        topk_idx, s.T, s.k, s.E, s.C, s.layout, 1, nblk, hist, routed, kept, offsets,
+        assign_row, token_of_row, s.max_rows, flt);
+    note_launch();
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  } else {
+    dispatch_count_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
+        topk_idx, s.T, s.k, s.E, planes, hist, status, all);
+    note_launch();
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    dispatch_rank_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
+        topk_idx, s.T, s.k, s.E, s.C, s.layout, planes, nblk, hist, routed, kept, offsets,
+        assign_row, token_of_row, s.max_rows, all);
+    note_launch();
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
   if (x_perm == nullptr) return cudaSuccess;  // bookkeeping only: the FFN gathers rows of x
 
   const int64_t row_bytes = s.d * s.elem;
@@ -335,6 +569,16 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
         xb, assign_row, s.T, s.k, row_bytes, sg, segs, xp, status, wait_ns);
     note_launch();
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pick_rank_counts(const Shape& s, const int32_t* topk_idx,
+                                    const int32_t* assign_row, const int32_t* group_of_expert,
+                                    int32_t* routed, int32_t* kept, int32_t* differs,
+                                    DevStatus* status, cudaStream_t st) {
+  pick_rank_counts_kernel<<<static_cast<unsigned>(s.k), kCountThreads, 0, st>>>(
+      topk_idx, assign_row, group_of_expert, s.T, s.k, s.E, routed, kept, differs, status);
+  note_launch();
   return cudaGetLastError();
 }
 

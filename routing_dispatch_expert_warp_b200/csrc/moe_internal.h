@@ -38,6 +38,7 @@ struct WsLayout {
   size_t router_tc_bytes;
   size_t ep_base;       // [E] int32: first row of this rank's rows per expert at the owner
   size_t arrive;        // [T, ceil(d/256)] int32 counters of the combine fused into the FFN
+  size_t score;         // score-priority dispatch scratch (dispatch_score_scratch_bytes)
   size_t total;
 };
 
@@ -74,11 +75,27 @@ size_t router_tc_workspace_bytes(const Shape& s);
 cudaError_t launch_topk_from_logits(const Shape& s, const float* logits, const float* bias,
                                     int64_t bias_stride, int32_t* topk_idx, float* topk_w,
                                     cudaStream_t st);
+// Selection scores for dispatch with drop_policy == MOE_DROP_SCORE: score of (t, e) =
+// logits[t, e] (+ bias[t * bias_stride + e] when the bias is selection-only), and the
+// scratch (dispatch_score_scratch_bytes, 256-byte aligned) the ranking by score needs.
+struct DispatchScores {
+  const float* logits;
+  const float* bias;
+  int64_t bias_stride;
+  void* scratch;
+};
+size_t dispatch_score_scratch_bytes(const Shape& s);
 cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_idx,
                             int32_t* routed, int32_t* kept, int32_t* offsets,
                             int32_t* assign_row, int32_t* token_of_row, void* x_perm,
                             int32_t* hist, DevStatus* status, uint64_t wait_ns,
-                            cudaStream_t st);
+                            cudaStream_t st, const DispatchScores* scores = nullptr);
+// Second-choice counters: per pick rank j and expert e the assignments (routed) and the
+// kept ones, and per j the tokens whose pick j lies in another group than pick 0.
+cudaError_t launch_pick_rank_counts(const Shape& s, const int32_t* topk_idx,
+                                    const int32_t* assign_row, const int32_t* group_of_expert,
+                                    int32_t* routed, int32_t* kept, int32_t* differs,
+                                    DevStatus* status, cudaStream_t st);
 // Expert FFN.  `a` holds the gate/up GEMM's A rows: x_perm (a_rows == nullptr) or x itself,
 // bucket row r reading row a_rows[r] of x (token_of_row: dispatch without the permute copy).
 cudaError_t launch_ffn_simt(const Shape& s, const float* a, const int32_t* a_rows,

@@ -19,6 +19,7 @@
 #include <type_traits>
 
 #include "moe_internal.h"
+#include "moe_keys.cuh"
 
 namespace moe {
 namespace {
@@ -402,14 +403,6 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(
   }
 }
 
-// Selection scores as unsigned keys whose integer order is the float order: a larger key
-// is a larger score.  -0 and +0 map to one key (they compare equal as floats), a NaN maps to
-// 1, below every number, and 0 is left for "not eligible".
-__device__ __forceinline__ uint32_t order_key(float f) {
-  if (f != f) return 1u;
-  const uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 // Warp-wide argmax over keys held as lane + 32 q: the largest key, equal keys -> the lower
 // index.  Two warp reductions (max of the keys, then min of the indices holding it).

@@ -25,7 +25,7 @@ import torch
 
 from . import _abi
 from ._abi import MoeEpConfig, MoeEpStats, check
-from . import (LayerBuffers, alloc_workspace, moe_dispatch, moe_route, F32)
+from . import (LayerBuffers, alloc_workspace, moe_dispatch_scored, moe_route, F32)
 
 # The per-layer step order (see include/moe.h, "expert parallelism"): a "barrier" entry
 # means every rank's previous steps must be complete before any rank's next one.
@@ -125,8 +125,9 @@ class EpRank:
 
     def rank_assignments(self, stream=None):
         b = self.bufs
-        moe_dispatch(self.cfg, None, b.topk_idx, b.routed_counts, b.kept_counts,
-                     b.expert_offsets, b.assign_row, b.token_of_row, None, self.ws, stream)
+        moe_dispatch_scored(self.cfg, None, b.topk_idx, b.logits, self.logit_bias,
+                            b.routed_counts, b.kept_counts, b.expert_offsets, b.assign_row,
+                            b.token_of_row, None, self.ws, stream)
 
     def put_counts(self, mats_table: torch.Tensor, stream=None):
         check(_lib().moe_ep_put_counts(ctypes.byref(self.cfg), ctypes.byref(self.ep),

@@ -56,7 +56,7 @@ class MoEShape:
     n_groups: int = 0          # group-limited routing (0: off)
     topk_groups: int = 0
     bias_mode: int = 0         # 0: bias in score and weights; 1: selection only
-    drop_policy: int = 0       # 0: token order; 1: pick rank first
+    drop_policy: int = 0       # 0: token order; 1: pick rank first; 2: score priority
 
     def replace(self, **kw) -> "MoEShape":
         return dataclasses.replace(self, **kw)

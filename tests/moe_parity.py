@@ -63,8 +63,14 @@ class GpuRun:
 
     def dispatch(self):
         b = self.b
-        M.moe_dispatch(self.cfg, self.inp.x, b.topk_idx, b.routed_counts, b.kept_counts,
-                       b.expert_offsets, b.assign_row, b.token_of_row, b.x_perm, self.ws)
+        if self.shape.drop_policy == O.DROP_SCORE:   # the drop decision reads the scores
+            M.moe_dispatch_scored(self.cfg, self.inp.x, b.topk_idx, b.logits,
+                                  self.inp.logit_bias, b.routed_counts, b.kept_counts,
+                                  b.expert_offsets, b.assign_row, b.token_of_row, b.x_perm,
+                                  self.ws)
+        else:
+            M.moe_dispatch(self.cfg, self.inp.x, b.topk_idx, b.routed_counts, b.kept_counts,
+                           b.expert_offsets, b.assign_row, b.token_of_row, b.x_perm, self.ws)
 
     def ffn(self):
         i, b = self.inp, self.b

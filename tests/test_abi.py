@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(lib):
     assert not missing, missing
     for n in names:
         assert getattr(lib, n) is not None
-    assert lib.moe_abi_version() == 3
+    assert lib.moe_abi_version() == 4
 
 
 def test_struct_layout_matches_header(tmp_path):
@@ -119,7 +119,7 @@ def test_workspace_size_and_bad_configs(lib):
         M.workspace_size(M.make_config(64, 128, 256, 8, 4, n_groups=4, topk_groups=1))
     with pytest.raises(M.MoEError):
         M.workspace_size(M.make_config(64, 128, 256, 8, 2, n_groups=3, topk_groups=1))
-    for bad in (dict(bias_mode=2), dict(drop_policy=5)):
+    for bad in (dict(bias_mode=2), dict(drop_policy=3)):
         with pytest.raises(M.MoEError):
             M.workspace_size(M.make_config(64, 128, 256, 8, 2, **bad))
     # pick-rank drops keep k count planes per block
@@ -154,6 +154,36 @@ def test_null_and_misaligned_pointers_rejected_on_host(lib):
                           M.workspace_size(cfg2), None)
     assert st == 2
     assert L.moe_status_string(5) == b"MOE_ERR_TIMEOUT"
+
+
+def test_score_drop_policy_host_checks(lib):
+    """MOE_DROP_SCORE: dispatch needs the scores, the workspace holds the ranking scratch,
+    the fixed-scratch dispatch refuses it; the counters check their pointers."""
+    L = lib
+    cfg = M.make_config(4096, 256, 256, 256, 8, capacity_factor=1.25, drop_policy=M.DROP_SCORE)
+    base = M.make_config(4096, 256, 256, 256, 8, capacity_factor=1.25)
+    A = 4096 * 8
+    r256 = lambda b: -(-b // 256) * 256
+    extra = 2 * r256(4 * A) + r256(4 * 256) + r256(4 * 257) + r256(8 * 256) + r256(8 * A)
+    assert M.workspace_size(cfg) - M.workspace_size(base) == extra
+    ws = M.workspace_size(cfg)
+    c = ctypes.byref(cfg)
+    st = L.moe_dispatch(c, 16, 16, 16, 16, 16, 16, 16, 16, 256, ws, None)
+    assert st == 1 and b"moe_dispatch_scored" in L.moe_last_error()
+    st = L.moe_dispatch_scored(c, 16, 16, None, None, 0, 16, 16, 16, 16, 16, 16, 256, ws, None)
+    assert st == 1 and b"logits" in L.moe_last_error()
+    st = L.moe_dispatch_scored(c, 16, 16, 16, 16, 3, 16, 16, 16, 16, 16, 16, 256, ws, None)
+    assert st == 1 and b"bias_row_stride" in L.moe_last_error()
+    st = L.moe_dispatch_scored(c, 16, 16, 16, None, 0, 16, 16, 16, 16, 16, 16, 256,
+                               M.workspace_size(base), None)
+    assert st == 3                       # the base workspace lacks the ranking scratch
+    st = L.moe_dispatch_static_scratch(c, 16, 16, 16, 16, 16, 16, 16, 16, None)
+    assert st == 2 and b"MOE_DROP_SCORE" in L.moe_last_error()
+    for ptrs in ((None, 16, 16, 16, 16), (16, None, 16, 16, 16), (16, 16, None, 16, 16),
+                 (16, 16, 16, None, 16), (16, 16, 16, 16, None)):
+        idx, ar, r, k, d = ptrs
+        st = L.moe_pick_rank_counts(c, idx, ar, None, r, k, d, 256, ws, None)
+        assert st == 1 and b"NULL" in L.moe_last_error()
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

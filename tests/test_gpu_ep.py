@@ -49,6 +49,9 @@ CASES = [
     (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 256, 128, n_groups=8, topk_groups=4, bias_mode=1,
                drop_policy=1), 4, "permuted"),
     (W.reduced(W.MIXTRAL_8X7B, 300, 128, 128), 1, "contiguous"),
+    # score-priority drops, decided on each rank before the exchange
+    (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 256, 128, capacity_factor=0.8, drop_policy=2), 4,
+     "permuted"),
 ]
 
 

@@ -13,10 +13,11 @@ from moe_parity import (GpuRun, check_combine, check_ffn_rows, check_permute, ch
 
 pytestmark = pytest.mark.gpu
 
-FULL = [W.TINY_FP32, W.MIXTRAL_8X7B, W.DSV3_DECODE, W.DSV3_PREFILL_ZIPF, W.MIXTRAL_8X22B_MIXED]
+FULL = [W.TINY_FP32, W.MIXTRAL_8X7B, W.DSV3_DECODE, W.DSV3_PREFILL_ZIPF, W.MIXTRAL_8X22B_MIXED,
+        W.DSV3_PREFILL_ZIPF.replace(drop_policy=2)]     # score-priority drops at full size
 
 
-@pytest.mark.parametrize("shape", FULL, ids=lambda s: s.name)
+@pytest.mark.parametrize("shape", FULL, ids=lambda s: s.name + ("_score_drops" if s.drop_policy == 2 else ""))
 def test_full_size_sampled(shape):
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA GPU")

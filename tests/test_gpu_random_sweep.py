@@ -38,7 +38,10 @@ def _draw(i: int) -> W.MoEShape:
             topk_groups = int(rng.integers(lo, n_groups + 1))
     bias_mode = 1 if (bias != "none" and rng.random() < 0.3) else 0
     drop_policy = 1 if (cf > 0 and rng.random() < 0.4) else 0
-    return W.MoEShape(f"rand{i}_T{T}_d{d}_f{f}_E{E}_k{k}_cf{cf}_{'bf16' if dtype else 'f32'}",
+    if drop_policy == 0 and rng.random() < (0.4 if cf > 0 else 0.1):
+        drop_policy = 2     # score priority (dropless: must equal token order)
+    return W.MoEShape(f"rand{i}_T{T}_d{d}_f{f}_E{E}_k{k}_cf{cf}_{'bf16' if dtype else 'f32'}"
+                      f"_d{drop_policy}",
                       T, d, f, E, k, gating, cf, dtype, bias=bias, layout=layout,
                       seed=7000 + i, n_decode_tokens=min(8, T), n_groups=n_groups,
                       topk_groups=topk_groups, bias_mode=bias_mode, drop_policy=drop_policy)
