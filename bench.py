@@ -44,7 +44,7 @@ GEMM_SOURCES = ("routing_dispatch_expert_warp_b200/csrc/moe_ffn_tc.cu",
                 "routing_dispatch_expert_warp_b200/csrc/moe_internal.h")
 RECORDED_GEMM_TRAFFIC = {
     ("mixtral8x7b_prefill_T4096", False): {
-        "bytes": 3667147264, "sources": "a4c968e4ba6a13bd",
+        "bytes": 3668033024, "sources": "56b4d857e1ce761e",
         "profile": "profiles/grouped_gemm_tc_mixtral8x7b_T4096_traffic.md"},
 }
 
@@ -188,6 +188,9 @@ def max_over_ranks(values, dist, device) -> list:
     return [float(v) for v in t.tolist()]
 
 
+DROP_POLICIES = {"token": 0, "pick_rank": 1, "score": 2}
+
+
 def run_gpu(args) -> None:
     shape = W.WORKLOADS[args.config] if args.config else DEFAULT
     if args.tokens:
@@ -196,6 +199,9 @@ def run_gpu(args) -> None:
         shape = shape.replace(name=f"{shape.name}_with_f{args.d_ff}", d_ff=args.d_ff)
     if args.experts:
         shape = shape.replace(name=f"{shape.name}_with_E{args.experts}", E=args.experts)
+    if args.drop_policy != "token":
+        shape = shape.replace(name=f"{shape.name}_drops_by_{args.drop_policy}",
+                              drop_policy=DROP_POLICIES[args.drop_policy])
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -222,8 +228,9 @@ def run_gpu(args) -> None:
         ev[0].record(stream)
         M.moe_route(cfg, inp.x, inp.w_router, inp.logit_bias, b.logits, b.topk_idx, b.topk_w, ws)
         ev[1].record(stream)
-        M.moe_dispatch(cfg, inp.x, b.topk_idx, b.routed_counts, b.kept_counts, b.expert_offsets,
-                       b.assign_row, b.token_of_row, b.x_perm, ws)
+        M.moe_dispatch_scored(cfg, inp.x, b.topk_idx, b.logits, inp.logit_bias, b.routed_counts,
+                              b.kept_counts, b.expert_offsets, b.assign_row, b.token_of_row,
+                              b.x_perm, ws)
         ev[2].record(stream)
         if args.fused_combine:
             M.moe_expert_ffn_combine(cfg, inp.x, b.x_perm, b.token_of_row, b.expert_offsets,
@@ -373,6 +380,7 @@ def run_gpu(args) -> None:
                        "d_ff": shape.d_ff, "E": shape.E, "k": shape.k,
                        "gating": "softmax" if shape.gating == W.SOFTMAX else "sigmoid",
                        "capacity_factor": shape.capacity_factor,
+                       "drop_order": args.drop_policy,
                        "l2": "flushed between timed steps (256 MB write)",
                        "dispatch": ("no x_perm: gate/up GEMM gathers rows of x" if args.gather
                                     else "permuted copy x_perm"),
@@ -522,7 +530,8 @@ class CpuSample:
         s = self.sub
         t0 = time.perf_counter()
         O.moe_layer(*self.args, k=s.k, gating=s.gating, capacity_factor=s.capacity_factor,
-                    layout=s.layout)
+                    layout=s.layout, n_groups=s.n_groups, topk_groups=s.topk_groups,
+                    bias_mode=s.bias_mode, drop_policy=s.drop_policy)
         dt = time.perf_counter() - t0
         return {"value": self.n / dt, "unit": "tokens/s", "cores": _cpu_cores(),
                 "kind": "oracle", "seconds": dt,
@@ -584,6 +593,9 @@ def main():
                     help="time the expert FFN with the combine fused into its down GEMM")
     ap.add_argument("--gather", action="store_true",
                     help="dispatch without the permuted copy: the gate/up GEMM gathers rows of x")
+    ap.add_argument("--drop-policy", default="token", choices=sorted(DROP_POLICIES),
+                    help="which picks an overflowing expert keeps: token order, pick rank "
+                         "first, or highest selection score")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)   # at least three untimed warm-up steps
     if args.impl == "reference":
