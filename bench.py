@@ -503,6 +503,109 @@ def run_ep_emulated(args) -> None:
     print(json.dumps(line), flush=True)
 
 
+def run_microbatch(args) -> None:
+    """The layer cut into args.microbatches microbatches that ping-pong over two streams
+    (with --ep-emulate G: the expert-parallel layer over G ranks emulated on this GPU, each
+    rank's tokens cut the same way), timed with CUDA events against the same layer on one
+    stream in the same process, plus the segments and critical path of one recorded step.
+    A separate measurement, not the headline line."""
+    from routing_dispatch_expert_warp_b200 import ep as EP
+    from routing_dispatch_expert_warp_b200 import microbatch as MB
+    m, G = args.microbatches, args.ep_emulate
+    base = W.WORKLOADS[args.config] if args.config else DEFAULT
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = W.make_inputs(base, device=dev)
+    if G:
+        if base.T % G or base.E % G:
+            raise SystemExit("T and E must be multiples of the emulated rank count")
+        shape = base.replace(T=base.T // G)
+        xs = [inp.x[r * shape.T:(r + 1) * shape.T].contiguous() for r in range(G)]
+        if inp.logit_bias is not None and inp.logit_bias.dim() == 2:
+            biases = [inp.logit_bias[r * shape.T:(r + 1) * shape.T].contiguous()
+                      for r in range(G)]
+        else:
+            biases = [inp.logit_bias] * G
+        cfg = M.config_from_shape(shape)
+        pp = MB.EpMicrobatchEmulator(cfg, G, inp.w_router, inp.w_gate, inp.w_up, inp.w_down,
+                                     biases, m=m, device=dev)
+        one = EP.EpEmulator(cfg, G, inp.w_router, inp.w_gate, inp.w_up, inp.w_down, biases,
+                            device=dev, local_weights=[(r.w_gate, r.w_up, r.w_down)
+                                                       for r in pp.emus[0].ranks])
+        run_pp = lambda rec=False: pp(xs, record=rec)
+        run_one = lambda: one.forward(xs)
+        errs = [r.ws for e in pp.emus + [one] for r in e.ranks]
+    else:
+        cfg = M.config_from_shape(base)
+        pp = MB.MicrobatchLayer(cfg, inp.w_router, inp.w_gate, inp.w_up, inp.w_down,
+                                inp.logit_bias, m=m, device=dev)
+        one = M.MoELayer(cfg, inp.w_router, inp.w_gate, inp.w_up, inp.w_down, inp.logit_bias,
+                         device=dev)
+        run_pp = lambda rec=False: pp(inp.x, record=rec)
+        run_one = lambda: one(inp.x)
+        errs = [p_["ws"] for p_ in pp.mbs] + [one.ws]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        evs = []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize(dev)
+        return sum(a.elapsed_time(b) for a, b in evs) / args.steps
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        run_pp()
+        flush.zero_()
+        run_one()
+    torch.cuda.synchronize(dev)
+    for ws in errs:
+        M.moe_check_device_error(ws)
+    clocks = ClockSampler(0)
+    time.sleep(0.3)
+    ms_pp = timed(run_pp)
+    ms_one = timed(run_one)
+    time.sleep(0.2)
+    clk = clocks.stop()
+    flush.zero_()
+    run_pp(True)
+    torch.cuda.synchronize(dev)
+    for ws in errs:
+        M.moe_check_device_error(ws)
+    tl = pp.timeline()
+    seg = tl["segments"]
+    name = lambda n: f"mb{n[0]}:{n[1]}"
+    line = {
+        "metric": (f"MoE-layer tokens/s, {m} microbatches ping-ponging on two streams"
+                   + (f", expert parallel over {G} ranks emulated on 1 B200" if G else "")),
+        "value": base.T / (ms_pp * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_pp,
+        "higher_is_better": True, "dtype": "bf16" if base.dtype == W.BF16 else "f32",
+        "data": "synthetic",
+        "config": {"workload": base.name, "microbatches": m, "ranks": G or 1,
+                   "tokens_per_microbatch": [n for _, n in pp.parts],
+                   "l2": "flushed between timed steps (256 MB write)"},
+        "single_stream_ms_per_step": ms_one,
+        "speedup_vs_single_stream": ms_one / ms_pp,
+        "timeline": {
+            "segments_ms": {name(n): [round(s_, 4), round(e_, 4)] for n, (s_, e_) in seg.items()},
+            "critical_path": [name(n) for n in tl["path"]],
+            "wall_ms": tl["wall"], "serial_ms": tl["serial"],
+            "path_busy_ms": tl["busy"], "path_gaps_ms": tl["gaps"],
+            "off_path_ms": tl["serial"] - tl["busy"],
+            "note": "one recorded step (events around every stage); off_path_ms is stage "
+                    "time that ran beside the critical path"},
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def _cpu_cores() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -593,6 +696,9 @@ def main():
                     help="time the expert FFN with the combine fused into its down GEMM")
     ap.add_argument("--gather", action="store_true",
                     help="dispatch without the permuted copy: the gate/up GEMM gathers rows of x")
+    ap.add_argument("--microbatches", type=int, default=1,
+                    help="time the layer as this many microbatches ping-ponging over two "
+                         "streams against the one-stream layer (a separate measurement)")
     ap.add_argument("--drop-policy", default="token", choices=sorted(DROP_POLICIES),
                     help="which picks an overflowing expert keeps: token order, pick rank "
                          "first, or highest selection score")
@@ -600,6 +706,8 @@ def main():
     args.warmup = max(args.warmup, 3)   # at least three untimed warm-up steps
     if args.impl == "reference":
         run_reference(args)
+    elif args.microbatches > 1:
+        run_microbatch(args)
     elif args.ep_emulate:
         run_ep_emulated(args)
     else:

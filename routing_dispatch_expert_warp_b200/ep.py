@@ -217,19 +217,26 @@ class EpEmulator:
 
     def __init__(self, cfg, world: int, w_router, w_gate, w_up, w_down,
                  logit_biases: Optional[Sequence] = None, expert_rank=None,
-                 ranks_per_node: int = 1, recv_rows: Optional[int] = None, device="cuda"):
+                 ranks_per_node: int = 1, recv_rows: Optional[int] = None, device="cuda",
+                 local_weights: Optional[Sequence] = None):
+        """local_weights: None, or per rank the (w_gate, w_up, w_down) of its local experts,
+        already sliced (another emulator's, to share them) -- then w_gate/w_up/w_down are
+        not read."""
         E = cfg.E
         self.world = world
         self.expert_rank = (contiguous_placement(E, world, device) if expert_rank is None
                             else expert_rank.to(device=device, dtype=torch.int32))
         self.ranks: List[EpRank] = []
         for r in range(world):
-            mine = local_experts(self.expert_rank, r).to(w_gate.device)
+            if local_weights is not None:
+                wg, wu, wd = local_weights[r]
+            else:
+                mine = local_experts(self.expert_rank, r).to(w_gate.device)
+                wg, wu, wd = (w_gate[mine].contiguous(), w_up[mine].contiguous(),
+                              w_down[mine].contiguous())
             bias = None if logit_biases is None else logit_biases[r]
-            self.ranks.append(EpRank(cfg, world, r, self.expert_rank, w_router,
-                                     w_gate[mine].contiguous(), w_up[mine].contiguous(),
-                                     w_down[mine].contiguous(), bias, ranks_per_node,
-                                     recv_rows, device))
+            self.ranks.append(EpRank(cfg, world, r, self.expert_rank, w_router, wg, wu, wd,
+                                     bias, ranks_per_node, recv_rows, device))
         self.tables = {
             "mats": _table([r.count_mat.data_ptr() for r in self.ranks], device),
             "recv": _table([r.recv_x.data_ptr() for r in self.ranks], device),
