@@ -146,7 +146,7 @@ WsLayout workspace_layout(const Shape& s) {
   off += l.logits_bytes;
   const int splits = router_splits(s);
   l.partials = off;
-  if (s.E <= 32 && splits == 1) {  // lane-ordered copy of W_r for the small-E router
+  if (s.E <= 32) {  // lane-ordered copy of W_r for the small-E router
     const size_t et = s.E <= 8 ? 8 : (s.E <= 16 ? 16 : 32);
     l.partials_bytes = round_up(static_cast<size_t>((s.d + 255) / 256) * 256 * et * sizeof(float));
   } else {

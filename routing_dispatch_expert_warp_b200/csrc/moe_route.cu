@@ -310,87 +310,6 @@ __global__ void __launch_bounds__(256, ET == 8 ? 2 : 3) router_small_e_kernel(
   }
 }
 
-// Router scores for E <= 8, split along d into 256-element chunks (chunk c = blockIdx.y).
-// Lane l owns elements c*256 + 8l .. 8l+7 and keeps their 8 rows of W_r (8 x 8 values, zero
-// past E) in registers for all the tokens of its warp, so W_r is read once per warp, not
-// once per token.  A warp takes RS_GROUPS groups of 4 consecutive tokens; the loads of all
-// of them (one 16-byte load of x per token and lane for bf16) are issued before the first
-// FMA.  Per group: 8 x 8 FMAs per token and lane (rows in order), then a butterfly
-// transpose-reduction leaves lane l with the chunk's partial sum of (token l / 8, expert
-// l % 8), stored to partial[c][t][e].  The top-k kernel adds the chunks' partials in chunk
-// order (and the bias), so the logits do not depend on scheduling.
-constexpr int RS_WARPS = 4;   // warps per block
-constexpr int RS_GROUPS = 4;  // groups of 4 tokens per warp
-
-template <typename TX>
-__global__ void __launch_bounds__(RS_WARPS * 32) router_split_e8_kernel(
-    const TX* __restrict__ x, const float* __restrict__ w_router, int64_t T, int d, int E,
-    float* __restrict__ partial) {
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const int c = blockIdx.y;
-  const int i0 = c * 256 + lane * 8;  // d is a multiple of 8: the lane's 8 elements all
-                                      // lie inside d or all past it
-  float wv[8][8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int64_t row = static_cast<int64_t>(i0) + i;
-    if (row < d && E == 8) {
-      const float4* src = reinterpret_cast<const float4*>(w_router + row * 8);
-      const float4 a = __ldg(src), b = __ldg(src + 1);
-      wv[i][0] = a.x; wv[i][1] = a.y; wv[i][2] = a.z; wv[i][3] = a.w;
-      wv[i][4] = b.x; wv[i][5] = b.y; wv[i][6] = b.z; wv[i][7] = b.w;
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) wv[i][e] = (row < d && e < E) ? __ldg(w_router + row * E + e) : 0.f;
-    }
-  }
-  const int64_t tbase =
-      (static_cast<int64_t>(blockIdx.x) * RS_WARPS + warp) * (4 * RS_GROUPS);
-  XRaw<TX> xr[RS_GROUPS][4];
-#pragma unroll
-  for (int g = 0; g < RS_GROUPS; ++g)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t t = tbase + 4 * g + j;
-      if (t < T && i0 < d) xr[g][j].load(x + t * d + i0);
-      else xr[g][j].zero();
-    }
-  const int64_t stride = T * E;
-#pragma unroll
-  for (int g = 0; g < RS_GROUPS; ++g) {
-    if (tbase + 4 * g >= T) break;
-    float v[32];
-#pragma unroll
-    for (int q = 0; q < 32; ++q) v[q] = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float xs[8] = {xr[g][j].template get<0>(), xr[g][j].template get<1>(),
-                           xr[g][j].template get<2>(), xr[g][j].template get<3>(),
-                           xr[g][j].template get<4>(), xr[g][j].template get<5>(),
-                           xr[g][j].template get<6>(), xr[g][j].template get<7>()};
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[8 * j + e] = fmaf(xs[i], wv[i][e], v[8 * j + e]);
-    }
-    // butterfly transpose-reduction: afterwards lane l holds the warp's sum of value l
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const bool upper = (lane & off) != 0;
-#pragma unroll
-      for (int i = 0; i < off; ++i) {
-        const float send = upper ? v[i] : v[i + off];
-        const float keep = upper ? v[i + off] : v[i];
-        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-      }
-    }
-    const int64_t t = tbase + 4 * g + (lane >> 3);
-    const int e = lane & 7;
-    if (t < T && e < E) partial[c * stride + t * E + e] = v[0];
-  }
-}
-
 // z = x W_r + b as a tiled fp32 GEMM: 64 tokens x 128 experts per block, K steps of 32.
 constexpr int RT_M = 64, RT_N = 128, RT_K = 32;
 
@@ -679,25 +598,6 @@ cudaError_t launch_router_typed(const Shape& s, const TX* x, const float* w_rout
                                 int32_t* topk_idx, float* topk_w, float* partials,
                                 cudaStream_t st) {
   const int d = static_cast<int>(s.d);
-  const bool sel_only = s.bias_mode == MOE_BIAS_SELECTION_ONLY;
-  if (s.E <= 8 && s.n_groups <= 1 && router_splits(s) > 1) {
-    const int nch = router_splits(s);  // one split per 256-element chunk of d
-    const int64_t tok_blocks = (s.T + 4 * RS_GROUPS * RS_WARPS - 1) / (4 * RS_GROUPS * RS_WARPS);
-    dim3 grid(static_cast<unsigned>(tok_blocks), static_cast<unsigned>(nch));
-    router_split_e8_kernel<TX><<<grid, RS_WARPS * 32, 0, st>>>(x, w_router, s.T, d, s.E,
-                                                               partials);
-    note_launch();
-    cudaError_t err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
-    const int64_t blocks_needed = (s.T + 7) / 8;
-    const int blocks = static_cast<int>(blocks_needed < 148 * 16 ? blocks_needed : 148 * 16);
-    topk_from_logits_kernel<<<blocks, 256, 0, st>>>(partials, nch, bias, bias_stride,
-                                                    sel_only ? 0 : 1, sel_only ? 1 : 0, logits,
-                                                    s.T, s.E, s.k, s.gating, s.n_groups,
-                                                    s.topk_groups, topk_idx, topk_w);
-    note_launch();
-    return cudaGetLastError();
-  }
   if (s.E <= 32 && s.n_groups <= 1) {
     float4* wl = reinterpret_cast<float4*>(partials);  // the workspace's router area
     if (s.E <= 8)
@@ -715,6 +615,7 @@ cudaError_t launch_router_typed(const Shape& s, const TX* x, const float* w_rout
   int k_per_split = (d + nsplit - 1) / nsplit;
   k_per_split = (k_per_split + RT_K - 1) / RT_K * RT_K;
   dim3 grid(tiles_n, static_cast<unsigned>(tiles_m), nsplit);
+  const bool sel_only = s.bias_mode == MOE_BIAS_SELECTION_ONLY;
   // the GEMM adds the bias itself only when it writes finished logits that carry it
   const float* gemm_bias = (nsplit == 1 && !sel_only) ? bias : nullptr;
   router_gemm_kernel<TX><<<grid, 256, 0, st>>>(x, w_router, gemm_bias, bias_stride, s.T, d, s.E,
@@ -749,10 +650,6 @@ cudaError_t launch_topk_from_logits(const Shape& s, const float* logits, const f
 }
 
 int router_splits(const Shape& s) {
-  if (s.E <= 8 && s.n_groups <= 1) {  // one split per 256-element chunk of d
-    const int64_t nch = (s.d + 255) / 256;
-    return (nch >= 2 && nch <= kMaxRouterSplits) ? static_cast<int>(nch) : 1;
-  }
   if (s.E <= 32) return 1;
   const int64_t tiles = ((s.E + RT_N - 1) / RT_N) * ((s.T + RT_M - 1) / RT_M);
   const int64_t target = 296;  // two waves of blocks on a 148-SM part; device-independent

@@ -258,8 +258,8 @@ def test_bounded_wait_runs_out_and_context_survives():
     check_stats(st, r)
 
 
-# ------------------------------------------------------------------ E <= 8 split-K router
-SPLIT_ROUTER = [
+# ------------------------------------------------------------------ E <= 8 router, wide d
+SMALL_E_WIDE = [
     W.reduced(W.MIXTRAL_8X7B, 1000, 2304, 128),                                  # 9 chunks
     W.reduced(W.MIXTRAL_8X7B, 500, 1024, 128).replace(E=4, k=2),                 # E < 8
     W.reduced(W.MIXTRAL_8X7B, 300, 768, 64).replace(E=6, k=3, gating=W.SIGMOID),
@@ -267,16 +267,16 @@ SPLIT_ROUTER = [
     W.reduced(W.MIXTRAL_8X22B_MIXED, 777, 768, 128, n_decode_tokens=8, bias_mode=1),
     W.reduced(W.MIXTRAL_8X7B, 1, 512, 64),                                       # one token
     W.reduced(W.MIXTRAL_8X7B, 70, 16384, 64),                                    # 64 chunks
-    W.reduced(W.MIXTRAL_8X7B, 70, 16640, 64),                 # 65 chunks: the fused router
+    W.reduced(W.MIXTRAL_8X7B, 70, 16640, 64),                                    # 65 chunks
 ]
 
 
-@pytest.mark.parametrize("shape", SPLIT_ROUTER,
+@pytest.mark.parametrize("shape", SMALL_E_WIDE,
                          ids=lambda s: f"{s.name}_E{s.E}_k{s.k}_b{s.bias_mode}")
-def test_split_router_small_e(shape):
-    """E <= 8 with d > 256: the logits come from per-chunk partial sums (W_r rows held in
-    registers), added in chunk order by the top-k kernel; logits within the fp32 tolerance,
-    everything downstream bit-exact from them."""
+def test_small_e_router_wide_d(shape):
+    """E <= 8 with d over many 256-element chunks, E below the lane group, fp32 x, a chunk
+    bias for selection only, one token: logits within the fp32 tolerance, everything
+    downstream bit-exact from them."""
     run = GpuRun(shape)
     run.all_stages()
     r = check_routing(run)
@@ -285,7 +285,7 @@ def test_split_router_small_e(shape):
 
 # ------------------------------------------------------------------ launch accounting
 @pytest.mark.parametrize("shape,router_kernels", [
-    (W.reduced(W.MIXTRAL_8X7B, 1000, 512, 768), 2),          # split-K router + top-k
+    (W.reduced(W.MIXTRAL_8X7B, 1000, 512, 768), 2),          # lane-ordered W_r + fused router
     (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256), 3),     # W_r split + tensor-core GEMM + top-k
     (W.reduced(W.DSV3_DECODE, 128, 512, 256), 2),            # split-K fp32 GEMM + top-k
 ])
