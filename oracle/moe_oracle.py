@@ -357,6 +357,20 @@ def load_stats(routed, kept, assign_row, C: Optional[int]) -> dict:
     )
 
 
+def replica_load_stats(parts) -> dict:
+    """The job's record over data-parallel replicas ([EP-checks] "Mean expert load proves
+    almost nothing": one record per layer for the job).  parts: per replica (routed, kept,
+    assign_row, C).  The job record is load_stats of the union of the replicas' picks: counts
+    added per expert, the replicas' assign_row stacked (only kept / dropped matters), and an
+    expert's capacity the sum of the replicas' capacities (dropless if any replica is)."""
+    routed = np.sum([np.asarray(p[0], dtype=np.int64) for p in parts], axis=0)
+    kept = np.sum([np.asarray(p[1], dtype=np.int64) for p in parts], axis=0)
+    rows = np.vstack([np.asarray(p[2]) for p in parts])
+    caps = [p[3] for p in parts]
+    C = None if any(c is None for c in caps) else int(sum(caps))
+    return load_stats(routed, kept, rows, C)
+
+
 # --------------------------------------------------------------------------------------
 # Whole layer
 # --------------------------------------------------------------------------------------

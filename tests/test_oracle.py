@@ -475,3 +475,35 @@ def test_score_drop_uses_selection_scores():
     # the same logits without the bias keep the highest logit, t2
     r = O.route(z, 1, O.SOFTMAX, 0.5, drop_policy=O.DROP_SCORE)
     assert r["assign_row"][:, 0].tolist() == [-1, -1, 0]
+
+
+def test_replica_stats_hand_case():
+    # replica A: 3 tokens, both picks of token 2 over capacity 2; replica B: 1 token, C = 1
+    a = (np.array([3, 3]), np.array([2, 2]), np.array([[0, 2], [1, 3], [-1, -1]]), 2)
+    b = (np.array([1, 1]), np.array([1, 1]), np.array([[1, 0]]), 1)
+    s = O.replica_load_stats([a, b])
+    assert (s["active_tokens"], s["capacity"], s["routed_total"], s["kept_total"]) == (4, 3, 8, 6)
+    assert (s["dropped"], s["tokens_with_drop"], s["tokens_fully_dropped"]) == (2, 1, 1)
+    assert s["dropped_by_rank"] == [1, 1]
+    assert (s["p50"], s["max"], s["mean"], s["max_to_mean"]) == (3.0, 3.0, 3.0, 1.0)
+    assert (s["routed_max"], s["routed_max_to_mean"], s["top5pct_share"]) == (4.0, 1.0, 0.5)
+    assert O.replica_load_stats([a, (b[0], b[1], b[2], None)])["capacity"] == -1
+
+
+@pytest.mark.parametrize("parts", [1, 2, 5])
+def test_replica_stats_of_a_dropless_split_equal_the_whole_batch(parts):
+    rng = np.random.default_rng(parts)
+    T, E, k = 103, 16, 4
+    z = rng.standard_normal((T, E)).astype(np.float32)
+    z[:, 3] += 1.0
+    idx = O.select_topk(z, k)
+    whole = O.assign(idx, E, None)
+    cuts = np.linspace(0, T, parts + 1).astype(int)
+    recs = []
+    for lo, hi in zip(cuts, cuts[1:]):
+        a = O.assign(idx[lo:hi], E, None)
+        recs.append((a["routed"], a["kept"], a["assign_row"], None))
+    got = O.replica_load_stats(recs)
+    want = O.load_stats(whole["routed"], whole["kept"], whole["assign_row"], None)
+    for key, val in want.items():
+        assert got[key] == val, key
