@@ -285,6 +285,10 @@ def run_gpu(args) -> None:
     total_ms = max_over_ranks([sum(step_ms)], dist, dev)[0]
     ms_per_step = total_ms / args.steps
     stats = b.stats_dict()
+    job_stats = None
+    if dist:  # the job's record of the layer over the replicas (every rank takes part)
+        from routing_dispatch_expert_warp_b200 import replicas as RP
+        job_stats = RP.job_load_stats(cfg, b)
     kept_total = stats["kept_total"]
     work = algorithmic_work(shape, kept_total)
     peaks = measured_peaks()
@@ -407,6 +411,10 @@ def run_gpu(args) -> None:
             },
             "load_stats": {k2: stats[k2] for k2 in ("kept_total", "dropped", "p50", "p95", "max",
                                                     "max_to_mean")},
+            "load_stats_job": (None if job_stats is None else
+                               {k2: job_stats[k2] for k2 in ("active_tokens", "kept_total",
+                                                             "dropped", "p50", "p95", "max",
+                                                             "max_to_mean", "top5pct_share")}),
             "e2e": {"value": shape.T * world / (pipe_total / args.steps * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": inp.x.numel() * inp.x.element_size(),
                     "d2h_bytes_per_step": b.out.numel() * b.out.element_size(),

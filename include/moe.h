@@ -445,6 +445,25 @@ moe_status_t moe_load_stats(const moe_config_t* cfg, const int32_t* routed_count
                             void* stream);
 
 /*
+ * The job's record over data-parallel replicas: every GPU runs the whole layer on its own
+ * tokens (no exchange) and the job reports one record per layer ([EP-checks] "Mean expert
+ * load proves almost nothing").  It is the record of the union of the replicas' picks: the
+ * per-expert counts added up, the drop counters and token counts added up, and an expert's
+ * capacity the sum of the replicas' capacities (-1 if any replica is dropless).
+ *   routed_sum, kept_sum  [E] int32 device arrays: element-wise sums over the replicas of
+ *                         their routed_counts and kept_counts (e.g. an all-reduce SUM of
+ *                         E ints each); every sum must be below 2^31
+ *   parts                 [n_parts] device array of the replicas' moe_load_stats_t records
+ *                         (e.g. an all-gather of the records moe_load_stats wrote), n_parts >= 1
+ * cfg gives E and k; T and the capacity come from the records.  dev_out and host_out as in
+ * moe_load_stats (a host copy synchronises the stream).  One kernel.
+ */
+moe_status_t moe_load_stats_merge(const moe_config_t* cfg, const int32_t* routed_sum,
+                                  const int32_t* kept_sum, const moe_load_stats_t* parts,
+                                  int32_t n_parts, moe_load_stats_t* dev_out,
+                                  moe_load_stats_t* host_out, void* stream);
+
+/*
  * Second-choice counters ([EP-checks] "Top-2 does not insure against hot experts": the
  * share of tokens whose second choice differs from the first, where second choices go, and
  * the share of second assignments that never reached the experts), for every pick rank j

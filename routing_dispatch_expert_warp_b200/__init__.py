@@ -26,7 +26,8 @@ __all__ = ["MoEError", "make_config", "workspace_size", "capacity", "max_rows",
            "alloc_workspace", "moe_route", "moe_dispatch", "moe_dispatch_scored",
            "moe_dispatch_static_scratch", "moe_pick_rank_counts",
            "moe_expert_ffn", "moe_expert_ffn_gather", "moe_expert_ffn_combine", "moe_combine",
-           "moe_load_stats", "moe_layer_forward", "moe_check_device_error",
+           "moe_load_stats", "moe_load_stats_merge", "moe_layer_forward",
+           "moe_check_device_error",
            "moe_selftest_bounded_wait", "set_wait_limit_ns", "kernel_launch_count",
            "LayerBuffers", "MoELayer", "HostPipeline"]
 
@@ -187,6 +188,17 @@ def moe_load_stats(cfg, routed_counts, kept_counts, assign_row, dev_out, host: b
     check(_lib().moe_load_stats(ctypes.byref(cfg), _ptr(routed_counts), _ptr(kept_counts),
                                 _ptr(assign_row), _ptr(dev_out),
                                 ctypes.byref(hs) if host else None, _stream(stream)))
+    return hs.as_dict() if host else None
+
+
+def moe_load_stats_merge(cfg, routed_sum, kept_sum, parts, dev_out, host: bool = True,
+                         stream=None) -> Optional[dict]:
+    """The job record of data-parallel replicas: routed_sum / kept_sum [E] int32 (summed over
+    the replicas), parts [n, sizeof(moe_load_stats_t)] uint8 (their records)."""
+    hs = MoeLoadStats()
+    check(_lib().moe_load_stats_merge(ctypes.byref(cfg), _ptr(routed_sum), _ptr(kept_sum),
+                                      _ptr(parts), int(parts.shape[0]), _ptr(dev_out),
+                                      ctypes.byref(hs) if host else None, _stream(stream)))
     return hs.as_dict() if host else None
 
 

@@ -111,6 +111,8 @@ PROTOTYPES = {
     "moe_load_stats": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, P(MoeLoadStats), c_vp]),
     "moe_pick_rank_counts": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                      c_sz, c_vp]),
+    "moe_load_stats_merge": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_i32, c_vp,
+                                     P(MoeLoadStats), c_vp]),
     "moe_layer_forward": (c_i32, [P(MoeConfig), P(MoeLayerInputs), P(MoeLayerBuffers), c_vp,
                                   c_sz, c_vp]),
     "moe_check_device_error": (c_i32, [c_vp, c_sz, c_vp]),

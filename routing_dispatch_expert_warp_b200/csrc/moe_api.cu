@@ -505,6 +505,27 @@ moe_status_t moe_load_stats(const moe_config_t* cfg, const int32_t* routed_count
   return MOE_OK;
 }
 
+moe_status_t moe_load_stats_merge(const moe_config_t* cfg, const int32_t* routed_sum,
+                                  const int32_t* kept_sum, const moe_load_stats_t* parts,
+                                  int32_t n_parts, moe_load_stats_t* dev_out,
+                                  moe_load_stats_t* host_out, void* stream) {
+  Shape s;
+  moe_status_t st = check_config(cfg, &s);
+  if (st != MOE_OK) return st;
+  MOE_REQUIRE(routed_sum && kept_sum && parts && dev_out, "moe_load_stats_merge: NULL pointer");
+  MOE_REQUIRE(n_parts >= 1, "moe_load_stats_merge: n_parts must be >= 1");
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  cudaError_t err = launch_stats_merge(s, routed_sum, kept_sum, parts, n_parts, dev_out, strm);
+  if (err != cudaSuccess) return cuda_fail(err, "moe_load_stats_merge launch");
+  if (host_out != nullptr) {
+    err = cudaMemcpyAsync(host_out, dev_out, sizeof(moe_load_stats_t), cudaMemcpyDeviceToHost,
+                          strm);
+    if (err == cudaSuccess) err = cudaStreamSynchronize(strm);
+    if (err != cudaSuccess) return cuda_fail(err, "moe_load_stats_merge copy");
+  }
+  return MOE_OK;
+}
+
 moe_status_t moe_pick_rank_counts(const moe_config_t* cfg, const int32_t* topk_idx,
                                   const int32_t* assign_row, const int32_t* group_of_expert,
                                   int32_t* routed_by_rank, int32_t* kept_by_rank,

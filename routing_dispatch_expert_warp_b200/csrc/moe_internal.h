@@ -119,6 +119,10 @@ cudaError_t launch_combine(const Shape& s, const void* y_perm, const int32_t* as
                            const float* topk_w, void* out, cudaStream_t st);
 cudaError_t launch_stats(const Shape& s, const int32_t* routed, const int32_t* kept,
                          const int32_t* assign_row, moe_load_stats_t* out, cudaStream_t st);
+// The job record of data-parallel replicas from their summed counts and their records.
+cudaError_t launch_stats_merge(const Shape& s, const int32_t* routed_sum,
+                               const int32_t* kept_sum, const moe_load_stats_t* parts,
+                               int n_parts, moe_load_stats_t* out, cudaStream_t st);
 cudaError_t launch_wait_selftest(DevStatus* status, uint64_t wait_ns, cudaStream_t st);
 
 int sm_count();

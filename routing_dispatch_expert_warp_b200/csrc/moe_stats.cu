@@ -8,7 +8,9 @@
 //
 // One block: the E kept counts are sorted in shared memory (bitonic network over the next
 // power of two of E), the drops are counted per pick rank over assign_row, and one thread evaluates
-// the fp64 formulas.  Percentiles interpolate linearly between order statistics:
+// the fp64 formulas.  The job record of data-parallel replicas runs the same kernel on the
+// replicas' summed counts, taking the token count, capacity and drop counters from the
+// replicas' own records instead of an assign_row.  Percentiles interpolate linearly between order statistics:
 // h = (E - 1) p, v = s[floor h] + (h - floor h) (s[floor h + 1] - s[floor h]).
 #include <limits.h>
 
@@ -39,17 +41,19 @@ __device__ __forceinline__ int warp_sum(int v) {
 __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
     const int32_t* __restrict__ routed, const int32_t* __restrict__ kept,
     const int32_t* __restrict__ assign_row, int64_t T, int k, int E, int64_t C,
+    const moe_load_stats_t* __restrict__ parts, int n_parts,
     moe_load_stats_t* __restrict__ out) {
   __shared__ int32_t sorted[MOE_MAX_EXPERTS];
-  __shared__ int sum_kept, sum_routed, max_routed;
+  __shared__ unsigned long long sum_kept, sum_routed;
+  __shared__ int max_routed;
   __shared__ int drop_rank[MOE_MAX_TOPK];
   __shared__ int tok_drop, tok_full;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   if (tid < MOE_MAX_EXPERTS) sorted[tid] = tid < E ? kept[tid] : INT_MAX;
   if (tid == 0) {
-    sum_kept = 0;
-    sum_routed = 0;
+    sum_kept = 0ull;
+    sum_routed = 0ull;
     max_routed = 0;
     tok_drop = 0;
     tok_full = 0;
@@ -62,7 +66,12 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
     int mx = rv;
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    const int sk = warp_sum(kv), sr = warp_sum(rv);
+    unsigned long long sk = static_cast<unsigned int>(kv), sr = static_cast<unsigned int>(rv);
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      sk += __shfl_xor_sync(0xffffffffu, sk, off);
+      sr += __shfl_xor_sync(0xffffffffu, sr, off);
+    }
     if (lane == 0) {
       atomicAdd(&sum_kept, sk);
       atomicAdd(&sum_routed, sr);
@@ -92,7 +101,7 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
 #pragma unroll
   for (int j = 0; j < MOE_MAX_TOPK; ++j) rank_local[j] = 0;
   int td = 0, tf = 0;
-  for (int64_t t = tid; t < T; t += blockDim.x) {
+  for (int64_t t = tid; assign_row != nullptr && t < T; t += blockDim.x) {
     int nd = 0;
 #pragma unroll
     for (int j = 0; j < MOE_MAX_TOPK; ++j) {
@@ -119,15 +128,31 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
 
   if (tid == 0) {
     moe_load_stats_t st;
+    int64_t drops[MOE_MAX_TOPK];
+    int64_t with_drop = tok_drop, fully = tok_full;
+    for (int j = 0; j < MOE_MAX_TOPK; ++j) drops[j] = j < k ? drop_rank[j] : 0;
+    if (parts != nullptr) {  // job record: tokens, capacity and drop counters of the replicas
+      T = 0;
+      C = 0;
+      with_drop = fully = 0;
+      for (int j = 0; j < MOE_MAX_TOPK; ++j) drops[j] = 0;
+      for (int p = 0; p < n_parts; ++p) {
+        T += parts[p].active_tokens;
+        C = (C < 0 || parts[p].capacity < 0) ? -1 : C + parts[p].capacity;
+        with_drop += parts[p].tokens_with_drop;
+        fully += parts[p].tokens_fully_dropped;
+        for (int j = 0; j < k; ++j) drops[j] += parts[p].dropped_by_rank[j];
+      }
+    }
     st.E = E;
     st.k = k;
     st.active_tokens = T;
     st.capacity = C;
-    st.routed_total = sum_routed;
-    st.kept_total = sum_kept;
+    st.routed_total = static_cast<int64_t>(sum_routed);
+    st.kept_total = static_cast<int64_t>(sum_kept);
     st.dropped = T * k - static_cast<int64_t>(sum_kept);
-    st.tokens_with_drop = tok_drop;
-    st.tokens_fully_dropped = tok_full;
+    st.tokens_with_drop = with_drop;
+    st.tokens_fully_dropped = fully;
     st.p50 = percentile_linear(sorted, E, 0.50);
     st.p95 = percentile_linear(sorted, E, 0.95);
     st.p99 = percentile_linear(sorted, E, 0.99);
@@ -143,7 +168,7 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
     for (int i = 0; i < n_top; ++i) top += sorted[E - 1 - i];
     st.top5pct_share =
         sum_kept > 0 ? static_cast<double>(top) / static_cast<double>(sum_kept) : 0.0;
-    for (int j = 0; j < MOE_MAX_TOPK; ++j) st.dropped_by_rank[j] = j < k ? drop_rank[j] : 0;
+    for (int j = 0; j < MOE_MAX_TOPK; ++j) st.dropped_by_rank[j] = drops[j];
     *out = st;
   }
 }
@@ -152,7 +177,17 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
 
 cudaError_t launch_stats(const Shape& s, const int32_t* routed, const int32_t* kept,
                          const int32_t* assign_row, moe_load_stats_t* out, cudaStream_t st) {
-  stats_kernel<<<1, kStatsThreads, 0, st>>>(routed, kept, assign_row, s.T, s.k, s.E, s.C, out);
+  stats_kernel<<<1, kStatsThreads, 0, st>>>(routed, kept, assign_row, s.T, s.k, s.E, s.C,
+                                            nullptr, 0, out);
+  note_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stats_merge(const Shape& s, const int32_t* routed_sum,
+                               const int32_t* kept_sum, const moe_load_stats_t* parts,
+                               int n_parts, moe_load_stats_t* out, cudaStream_t st) {
+  stats_kernel<<<1, kStatsThreads, 0, st>>>(routed_sum, kept_sum, nullptr, 0, s.k, s.E, 0,
+                                            parts, n_parts, out);
   note_launch();
   return cudaGetLastError();
 }
