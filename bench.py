@@ -44,7 +44,7 @@ GEMM_SOURCES = ("routing_dispatch_expert_warp_b200/csrc/moe_ffn_tc.cu",
                 "routing_dispatch_expert_warp_b200/csrc/moe_internal.h")
 RECORDED_GEMM_TRAFFIC = {
     ("mixtral8x7b_prefill_T4096", False): {
-        "bytes": 3668033024, "sources": "56b4d857e1ce761e",
+        "bytes": 3671601664, "sources": "d94c516aa4c2f235",
         "profile": "profiles/grouped_gemm_tc_mixtral8x7b_T4096_traffic.md"},
 }
 
