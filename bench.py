@@ -284,6 +284,14 @@ def run_gpu(args) -> None:
         step_ms.append(ev[0].elapsed_time(ev[5]))
     total_ms = max_over_ranks([sum(step_ms)], dist, dev)[0]
     ms_per_step = total_ms / args.steps
+    tensors_bytes = lambda ts: int(sum(t.numel() * t.element_size() for t in ts if t is not None))
+    memory = {"weights_bytes": tensors_bytes([inp.w_router, inp.w_gate, inp.w_up, inp.w_down]),
+              "layer_buffers_bytes": tensors_bytes(vars(b).values()),
+              "workspace_bytes": int(ws.numel()),
+              "peak_allocated_bytes": int(torch.cuda.max_memory_allocated(dev)),
+              "peak_reserved_bytes": int(torch.cuda.max_memory_reserved(dev)),
+              "note": "torch allocator peaks at the end of the timed region: inputs, weights, "
+                      "layer buffers, workspace and the L2-flush buffer"}
     stats = b.stats_dict()
     job_stats = None
     if dist:  # the job's record of the layer over the replicas (every rank takes part)
@@ -429,6 +437,7 @@ def run_gpu(args) -> None:
                       "api": "MoELayer.capture -> CUDA graph replay of moe_layer_forward",
                       "l2": "flushed between replays"},
             "gpu_launches": timed_launches,
+            "memory": memory,
             "clocks": clk,
             "cpu_baseline": cpu,
         }
@@ -607,6 +616,7 @@ def run_microbatch(args) -> None:
             "wall_ms": tl["wall"], "serial_ms": tl["serial"],
             "path_busy_ms": tl["busy"], "path_gaps_ms": tl["gaps"],
             "off_path_ms": tl["serial"] - tl["busy"],
+            "stage_record": MB.stage_record(tl),
             "note": "one recorded step (events around every stage); off_path_ms is stage "
                     "time that ran beside the critical path"},
         "clocks": clk,

@@ -94,6 +94,28 @@ def critical_path(intervals: Dict[tuple, Tuple[float, float]],
             "busy": busy, "gaps": wall - busy}
 
 
+# The per-stage record of "MoE expert parallelism needs measurements before launch",
+# "Profile all-to-all separately from compute": router, pack, dispatch, expert compute,
+# combine and unpack times.  Stage names of this library -> the record's fields.  With the
+# experts local, pack and dispatch are one stage (bookkeeping + permute), and so are combine
+# and unpack; under expert parallelism the count exchange and the plan are the pack.
+RECORD_FIELDS = {"route": "router_ms", "rank": "pack_ms", "put_counts": "pack_ms",
+                 "plan": "pack_ms", "dispatch": "dispatch_ms", "expert_ffn": "expert_compute_ms",
+                 "combine": "combine_ms", "stats": "stats_ms"}
+
+
+def stage_record(timeline: dict) -> dict:
+    """The per-stage record of one recorded forward: each field is the summed duration of
+    its stages over the microbatches (ms), plus the wall time and the critical path's
+    busy time and gaps."""
+    rec = {f: 0.0 for f in dict.fromkeys(RECORD_FIELDS.values())}
+    for (_, name), (s, e) in timeline["segments"].items():
+        rec[RECORD_FIELDS[name]] += e - s
+    rec.update(wall_ms=timeline["wall"], critical_path_busy_ms=timeline["busy"],
+               critical_path_gaps_ms=timeline["gaps"])
+    return rec
+
+
 class MicrobatchLayer:
     """One MoE layer on one GPU, run as m microbatches ping-ponging over two streams.
 

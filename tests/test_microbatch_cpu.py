@@ -53,3 +53,25 @@ def test_critical_path_follows_the_later_dependency():
     assert cp["path"] == [(0, "a"), (0, "b"), (0, "c"), (2, "a"), (2, "b"), (2, "c")]
     assert cp["wall"] == 12 and cp["gaps"] == 0
     assert MB.critical_path({}, {})["path"] == []
+
+
+def test_stage_record_sums_stages_into_the_record_fields():
+    iv = {(0, "route"): (0.0, 0.1), (0, "dispatch"): (0.1, 0.3), (0, "expert_ffn"): (0.3, 2.3),
+          (0, "combine"): (2.3, 2.4), (0, "stats"): (2.4, 2.45),
+          (1, "route"): (0.3, 0.35), (1, "dispatch"): (0.35, 0.5), (1, "expert_ffn"): (2.3, 4.0),
+          (1, "combine"): (4.0, 4.1), (1, "stats"): (4.1, 4.2)}
+    deps = MB.pingpong_deps(2, MB.STAGES, "dispatch")
+    rec = MB.stage_record({"segments": iv, **MB.critical_path(iv, deps)})
+    assert rec["router_ms"] == pytest.approx(0.15)
+    assert rec["dispatch_ms"] == pytest.approx(0.35)
+    assert rec["expert_compute_ms"] == pytest.approx(3.7)
+    assert rec["combine_ms"] == pytest.approx(0.2) and rec["stats_ms"] == pytest.approx(0.15)
+    assert rec["pack_ms"] == 0.0 and rec["wall_ms"] == pytest.approx(4.2)
+    # expert parallel steps: the count exchange and the plan are the pack
+    ep = {(0, "route"): (0, 1), (0, "rank"): (1, 2), (0, "put_counts"): (2, 3),
+          (0, "plan"): (3, 5), (0, "dispatch"): (5, 6), (0, "expert_ffn"): (6, 9),
+          (0, "combine"): (9, 10), (0, "stats"): (10, 11)}
+    steps = ["route", "rank", "put_counts", "plan", "dispatch", "expert_ffn", "combine", "stats"]
+    rec = MB.stage_record({"segments": ep, **MB.critical_path(ep, MB.pingpong_deps(1, steps,
+                                                                                 "dispatch"))})
+    assert rec["pack_ms"] == 4 and rec["dispatch_ms"] == 1 and rec["wall_ms"] == 11
