@@ -84,11 +84,62 @@ def measured_peaks() -> dict:
                 source="fallback")
 
 
-class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+# NVML clock-event reason bits (public NVML API constants) that the record names.
+CLOCK_REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                 "hw_thermal_slowdown": 0x40}
 
-    def __init__(self, index: int):
-        self.proc = None
+
+class ClockSampler:
+    """SM clock and clock-event reasons during the timed region, read (never set) through
+    NVML every `interval` seconds on a host thread; mark_start() / mark_end() bracket the
+    timed region, and the record is the median SM clock and the union of the reasons over
+    the samples inside it (all samples if none fell inside).  Without NVML it polls
+    nvidia-smi every 100 ms instead."""
+
+    def __init__(self, index: int, interval: float = 0.005, nvml=None):
+        import threading
+        self.samples, self.t0, self.t1 = [], None, None
+        self.proc, self.thread, self.source = None, None, None
+        try:
+            if nvml is None:
+                import pynvml as nvml
+            nvml.nvmlInit()
+            self.nvml, self.handle = nvml, self._handle(nvml, index)
+            self.source = "nvml"
+        except Exception:
+            self.nvml = None
+            self._start_smi(index)
+            return
+        self._stop = threading.Event()
+        self.interval = interval
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    @staticmethod
+    def _handle(nvml, index: int):
+        try:  # the CUDA device's own PCI address: CUDA and NVML may number GPUs differently
+            p = torch.cuda.get_device_properties(index)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return nvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nvml.nvmlDeviceGetHandleByIndex(index)
+
+    def _run(self) -> None:
+        n = self.nvml
+        get_reasons = getattr(n, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(n, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self._stop.is_set():
+            try:
+                self.samples.append((time.perf_counter(),
+                                     float(n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)),
+                                     float(n.nvmlDeviceGetMaxClockInfo(self.handle,
+                                                                       n.NVML_CLOCK_SM)),
+                                     int(get_reasons(self.handle))))
+            except Exception:
+                pass
+            self._stop.wait(self.interval)
+
+    def _start_smi(self, index: int) -> None:
         # BENCH_CLOCKS_DIR keeps the raw samples somewhere chosen; default: a temp dir
         out_dir = os.environ.get("BENCH_CLOCKS_DIR") or tempfile.gettempdir()
         self.path = os.path.join(out_dir, f"moe_bench_clocks_gpu{index}.csv")
@@ -101,10 +152,21 @@ class ClockSampler:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(index), f"--query-gpu={q}", "--format=csv,noheader,nounits",
                  "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi"
         except (OSError, FileNotFoundError):
             self.proc = None
 
+    def mark_start(self) -> None:
+        self.t0 = time.perf_counter()
+
+    def mark_end(self) -> None:
+        self.t1 = time.perf_counter()
+
     def stop(self) -> dict | None:
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=5)
+            return self.summary()
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -113,24 +175,30 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.f.close()
-        sm, mx, reasons = [], 0.0, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx = max(mx, float(parts[2]))
+                sm, mx = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
+            bits = sum(CLOCK_REASONS[n] for n, v in zip(names, parts[5:9]) if v.lower() == "active")
+            self.samples.append((None, sm, mx, bits))
+        return self.summary()
+
+    def summary(self) -> dict | None:
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        inside = [x for x in self.samples if x[0] is not None and self.t0 is not None and
+                  self.t1 is not None and self.t0 <= x[0] <= self.t1]
+        use = inside or self.samples
+        reasons = sorted(n for n, bit in CLOCK_REASONS.items() if any(x[3] & bit for x in use))
+        return {"sm_mhz": statistics.median(x[1] for x in use),
+                "sm_max_mhz": max(x[2] for x in use), "reasons": reasons,
+                "samples": len(use), "source": self.source,
+                "window": "timed region" if inside else "whole sampling period"}
 
 
 def algorithmic_work(shape, kept_total: int) -> dict:
@@ -263,11 +331,13 @@ def run_gpu(args) -> None:
     clocks = ClockSampler(local)
     time.sleep(0.3)
     launches0 = M.kernel_launch_count()
+    clocks.mark_start()
     for i in range(args.steps):
         flush.zero_()
         step(evs[i])
     timed_launches = M.kernel_launch_count() - launches0
     torch.cuda.synchronize(dev)
+    clocks.mark_end()
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -487,10 +557,12 @@ def run_ep_emulated(args) -> None:
     torch.cuda.synchronize(dev)
     clocks = ClockSampler(0)
     time.sleep(0.3)
+    clocks.mark_start()
     for i in range(args.steps):
         flush.zero_()
         run(evs[i])
     torch.cuda.synchronize(dev)
+    clocks.mark_end()
     time.sleep(0.2)
     clk = clocks.stop()
     for r in emu.ranks:
@@ -586,8 +658,10 @@ def run_microbatch(args) -> None:
         M.moe_check_device_error(ws)
     clocks = ClockSampler(0)
     time.sleep(0.3)
+    clocks.mark_start()
     ms_pp = timed(run_pp)
     ms_one = timed(run_one)
+    clocks.mark_end()
     time.sleep(0.2)
     clk = clocks.stop()
     flush.zero_()
