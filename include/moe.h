@@ -487,11 +487,12 @@ moe_status_t moe_pick_rank_counts(const moe_config_t* cfg, const int32_t* topk_i
                                   void* stream);
 
 /*
- * The whole layer: moe_route, moe_dispatch, moe_expert_ffn, moe_combine and (when
- * bufs->stats is not NULL) moe_load_stats, enqueued back to back on one stream without a
- * host synchronisation.  bufs->x_perm NULL: dispatch writes no permuted copy and the
- * gate/up GEMM gathers rows of x (moe_expert_ffn_gather).  Returns the first failing
- * stage's status.
+ * The whole layer: moe_route, moe_dispatch_scored (given the logits moe_route wrote:
+ * bufs->logits, or the workspace's copy when that is NULL; with the drop policies other than
+ * MOE_DROP_SCORE this is moe_dispatch), moe_expert_ffn, moe_combine and (when bufs->stats is
+ * not NULL) moe_load_stats, enqueued back to back on one stream without a host
+ * synchronisation.  bufs->x_perm NULL: dispatch writes no permuted copy and the gate/up GEMM
+ * gathers rows of x (moe_expert_ffn_gather).  Returns the first failing stage's status.
  */
 moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_layer_inputs_t* in,
                                const moe_layer_buffers_t* bufs, void* ws, size_t ws_bytes,
