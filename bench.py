@@ -366,7 +366,10 @@ def run_gpu(args) -> None:
     job_stats = None
     if dist:  # the job's record of the layer over the replicas (every rank takes part)
         from routing_dispatch_expert_warp_b200 import replicas as RP
-        job_stats = RP.job_load_stats(cfg, b)
+        try:
+            job_stats = RP.job_load_stats(cfg, b)
+        except Exception as exc:  # the timing stands without the record
+            job_stats = {"error": f"{type(exc).__name__}: {exc}"}
     kept_total = stats["kept_total"]
     work = algorithmic_work(shape, kept_total)
     peaks = measured_peaks()
@@ -489,7 +492,7 @@ def run_gpu(args) -> None:
             },
             "load_stats": {k2: stats[k2] for k2 in ("kept_total", "dropped", "p50", "p95", "max",
                                                     "max_to_mean")},
-            "load_stats_job": (None if job_stats is None else
+            "load_stats_job": (job_stats if (job_stats is None or "error" in job_stats) else
                                {k2: job_stats[k2] for k2 in ("active_tokens", "kept_total",
                                                              "dropped", "p50", "p95", "max",
                                                              "max_to_mean", "top5pct_share")}),
