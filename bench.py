@@ -757,7 +757,9 @@ def run_reference(args) -> None:
         "ms_per_step": args.ref_sample_tokens / v * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": shape.name, "T": shape.T, "d_model": shape.d_model,
-                   "d_ff": shape.d_ff, "E": shape.E, "k": shape.k},
+                   "d_ff": shape.d_ff, "E": shape.E, "k": shape.k,
+                   "gating": "softmax" if shape.gating == W.SOFTMAX else "sigmoid",
+                   "capacity_factor": shape.capacity_factor, "drop_order": "token"},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[0]["cores"],
                          "kind": "oracle", "sample": vals[0]["sample"]},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
