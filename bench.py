@@ -259,7 +259,8 @@ def max_over_ranks(values, dist, device) -> list:
 DROP_POLICIES = {"token": 0, "pick_rank": 1, "score": 2}
 
 
-def run_gpu(args) -> None:
+def workload_shape(args) -> "W.MoEShape":
+    """The workload the command line names, with its overrides applied."""
     shape = W.WORKLOADS[args.config] if args.config else DEFAULT
     if args.tokens:
         shape = shape.replace(name=f"{shape.name}_with_T{args.tokens}", T=args.tokens)
@@ -270,6 +271,11 @@ def run_gpu(args) -> None:
     if args.drop_policy != "token":
         shape = shape.replace(name=f"{shape.name}_drops_by_{args.drop_policy}",
                               drop_policy=DROP_POLICIES[args.drop_policy])
+    return shape
+
+
+def run_gpu(args) -> None:
+    shape = workload_shape(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -745,7 +751,7 @@ def run_reference(args) -> None:
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    shape = W.WORKLOADS[args.config] if args.config else DEFAULT
+    shape = workload_shape(args)
     sample = CpuSample(shape, args.ref_sample_tokens)
     for _ in range(args.warmup):
         sample.run()
@@ -759,7 +765,7 @@ def run_reference(args) -> None:
         "config": {"workload": shape.name, "T": shape.T, "d_model": shape.d_model,
                    "d_ff": shape.d_ff, "E": shape.E, "k": shape.k,
                    "gating": "softmax" if shape.gating == W.SOFTMAX else "sigmoid",
-                   "capacity_factor": shape.capacity_factor, "drop_order": "token"},
+                   "capacity_factor": shape.capacity_factor, "drop_order": args.drop_policy},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[0]["cores"],
                          "kind": "oracle", "sample": vals[0]["sample"]},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
