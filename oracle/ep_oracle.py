@@ -153,20 +153,25 @@ def ep_stats(kept_by_src, expert_rank, ranks_per_node: int, row_bytes: int) -> d
 
 def ep_layer(xs: Sequence, w_router, biases: Optional[Sequence], w_gate, w_up, w_down, k: int,
              gating: int, capacity_factor: float, expert_rank, z32s: Optional[Sequence] = None,
-             ranks_per_node: int = 1, row_bytes: int = 0) -> dict:
+             ranks_per_node: int = 1, row_bytes: int = 0, n_groups: int = 0,
+             topk_groups: int = 0, bias_mode: int = O.BIAS_SCORE_AND_WEIGHT,
+             drop_policy: int = O.DROP_TOKEN_ORDER) -> dict:
     """The EP layer over len(xs) ranks, steps in the pages' order.  xs[s]: rank s's tokens;
     biases[s]: its logit bias (or None); z32s[s]: its fp32 logits when routing is to start
-    from given logits (the parity protocol)."""
+    from given logits (the parity protocol).  The routing variants apply on every rank, before
+    the exchange, exactly as on one GPU."""
     G = len(xs)
     E = np.asarray(w_router).shape[1]
     er = np.asarray(expert_rank)
     # 1. route and drop locally
     routes = []
+    sel_only = bias_mode == O.BIAS_SELECTION_ONLY
     for s in range(G):
         b = None if biases is None else biases[s]
-        z32 = (O.logits_to_fp32(O.router_logits(xs[s], w_router, b)) if z32s is None
-               else np.asarray(z32s[s], dtype=np.float32))
-        routes.append(O.route(z32, k, gating, capacity_factor))
+        z32 = (O.logits_to_fp32(O.router_logits(xs[s], w_router, None if sel_only else b))
+               if z32s is None else np.asarray(z32s[s], dtype=np.float32))
+        routes.append(O.route(z32, k, gating, capacity_factor, O.LAYOUT_COMPACT, n_groups,
+                              topk_groups, b if sel_only else None, bias_mode, drop_policy))
     kept = np.stack([r["kept"] for r in routes])
     lay = recv_layout(kept, er)
     # 2. dispatch all-to-all: every kept row goes to its owner's buffer

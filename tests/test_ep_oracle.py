@@ -99,3 +99,25 @@ def test_ep_layer_equals_local_layer_per_rank(G, E, k, cf, permuted):
                     if sr[t, j] >= 0 and er[r["idx"][t, j]] == g:
                         used[sr[t, j]] += 1
         assert (used == 1).all()
+
+
+@pytest.mark.parametrize("variant", [
+    dict(n_groups=4, topk_groups=2),
+    dict(bias_mode=O.BIAS_SELECTION_ONLY),
+    dict(drop_policy=O.DROP_PICK_RANK),
+    dict(drop_policy=O.DROP_SCORE, bias_mode=O.BIAS_SELECTION_ONLY),
+], ids=["groups", "sel_bias", "pick_rank", "score_drops"])
+def test_ep_layer_with_routing_variants_equals_local_layer(variant):
+    G, E, k, cf, T, d, f = 4, 8, 2, 0.75, 30, 16, 12
+    xs, w_router, wg, wu, wd = _ranks(G, T, d, f, E, k, seed=99)
+    rng = np.random.default_rng(5)
+    biases = [rng.standard_normal((T, E)) * 2.0 for _ in range(G)]
+    er = np.random.default_rng(8).permutation(EP.contiguous_placement(E, G))
+    ep = EP.ep_layer(xs, w_router, biases, wg, wu, wd, k, O.SIGMOID, cf, er, **variant)
+    drops = 0
+    for s in range(G):
+        ref = O.moe_layer(xs[s], w_router, biases[s], wg, wu, wd, k, O.SIGMOID, cf, **variant)
+        np.testing.assert_allclose(ep["out"][s], ref["out"], rtol=1e-12, atol=1e-12)
+        np.testing.assert_array_equal(ep["routes"][s]["assign_row"], ref["assign_row"])
+        drops += int((ref["assign_row"] < 0).sum())
+    assert drops > 0      # the capacity binds, so the drop order matters
