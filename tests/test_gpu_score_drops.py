@@ -234,3 +234,29 @@ def test_pick_rank_counts_bad_expert_reported():
     with pytest.raises(M.MoEError) as ei:
         M.moe_check_device_error(run.ws)
     assert ei.value.status == 6
+
+
+def test_hand_case_from_golden_fixture(golden_dir):
+    """The hand-worked score-drop case and its counters, on the GPU, against the fixture's
+    values (derived by hand, not by the oracle)."""
+    import json
+    import os
+    with open(os.path.join(golden_dir, "hand_e4_k2_t8.json")) as f:
+        g = json.load(f)
+    with open(os.path.join(golden_dir, "hand_e4_k2_t8_score_drops.json")) as f:
+        want = json.load(f)
+    cfg = M.make_config(g["T"], 64, 64, g["E"], g["k"], capacity_factor=g["capacity_factor"],
+                        drop_policy=M.DROP_SCORE)
+    idx = torch.tensor(want["idx"], dtype=torch.int32, device="cuda")
+    z = torch.tensor(g["logits"], dtype=torch.float32, device="cuda")
+    got = _dispatch_scored(cfg, idx, z)
+    assert got["assign_row"].tolist() == want["assign_row"]
+    assert got["token_of_row"][:len(want["token_of_row"])].tolist() == want["token_of_row"]
+    assert got["kept"].tolist() == want["kept"]
+    ws = M.alloc_workspace(cfg)
+    ar = torch.tensor(want["assign_row"], dtype=torch.int32, device="cuda")
+    routed, kept, differs = M.moe_pick_rank_counts(cfg, idx, ar, ws)
+    M.moe_check_device_error(ws)
+    assert routed.cpu().tolist() == want["routed_by_rank"]
+    assert kept.cpu().tolist() == want["kept_by_rank"]
+    assert differs.cpu().tolist() == want["differs_by_rank"]

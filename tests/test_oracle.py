@@ -507,3 +507,20 @@ def test_replica_stats_of_a_dropless_split_equal_the_whole_batch(parts):
     want = O.load_stats(whole["routed"], whole["kept"], whole["assign_row"], None)
     for key, val in want.items():
         assert got[key] == val, key
+
+
+def test_hand_case_score_drops_and_counters(golden_dir):
+    g = _hand(golden_dir)
+    with open(os.path.join(golden_dir, "hand_e4_k2_t8_score_drops.json")) as f:
+        want = json.load(f)
+    z = np.array(g["logits"], dtype=np.float32)
+    r = O.route(z, g["k"], O.SOFTMAX, g["capacity_factor"], drop_policy=O.DROP_SCORE)
+    assert r["idx"].tolist() == want["idx"]
+    assert r["assign_row"].tolist() == want["assign_row"]
+    assert r["token_of_row"].tolist() == want["token_of_row"]
+    assert r["kept"].tolist() == want["kept"]
+    c = O.pick_rank_counts(r["idx"], r["assign_row"], g["E"])
+    assert c["routed"].tolist() == want["routed_by_rank"]
+    assert c["kept"].tolist() == want["kept_by_rank"]
+    assert c["differs"].tolist() == want["differs_by_rank"]
+    assert c["dropped_share"] == want["dropped_share_by_rank"]
