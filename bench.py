@@ -291,10 +291,19 @@ def run_gpu(args) -> None:
                                 device_id=dev)
 
     # every rank holds a full replica; ranks draw different token batches
+    mem_points = {}
+
+    def mem_point(name):  # allocator state at the points the memory record asks for
+        mem_points[name] = {"allocated_bytes": int(torch.cuda.memory_allocated(dev)),
+                            "reserved_bytes": int(torch.cuda.memory_reserved(dev)),
+                            "peak_allocated_bytes": int(torch.cuda.max_memory_allocated(dev))}
+
     inp = W.make_inputs(rank_shape(shape, rank), device=dev)
+    mem_point("inputs_and_weights")
     cfg = M.config_from_shape(shape)
     ws = M.alloc_workspace(cfg, dev)
     b = M.LayerBuffers.allocate(cfg, dev, gather=args.gather)
+    mem_point("layer_buffers_and_workspace")
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -328,6 +337,7 @@ def run_gpu(args) -> None:
         flush.zero_()
         step(mk())
     M.moe_check_device_error(ws)
+    mem_point("after_warmup")
 
     evs = [mk() for _ in range(args.steps)]
     torch.cuda.synchronize(dev)
@@ -368,6 +378,8 @@ def run_gpu(args) -> None:
               "peak_reserved_bytes": int(torch.cuda.max_memory_reserved(dev)),
               "note": "torch allocator peaks at the end of the timed region: inputs, weights, "
                       "layer buffers, workspace and the L2-flush buffer"}
+    mem_point("after_timed_region")
+    memory["points"] = mem_points
     stats = b.stats_dict()
     job_stats = None
     if dist:  # the job's record of the layer over the replicas (every rank takes part)
