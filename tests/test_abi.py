@@ -228,3 +228,14 @@ def test_ep_sizes_and_argument_checks(lib):
     assert lib.moe_ep_stats(ctypes.byref(cfg), ctypes.byref(ep), None, 16, None, None) == 1
     assert lib.moe_ipc_handle(None, ctypes.create_string_buffer(64),
                               ctypes.byref(ctypes.c_int64())) == 1
+
+
+def test_prototype_arity_matches_the_header():
+    """Every ctypes prototype takes as many arguments as the header's declaration."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    decls = re.findall(r"\b(moe_[a-z0-9_]+)\s*\(([^;{)]*)\)\s*;", src)
+    assert len(decls) == len(_abi.PROTOTYPES)
+    for name, params in decls:
+        params = " ".join(params.split())
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        assert n == len(_abi.PROTOTYPES[name][1]), (name, n, len(_abi.PROTOTYPES[name][1]))
