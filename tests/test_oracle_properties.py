@@ -4,6 +4,7 @@ definitions restated independently here (counting, sorting, and brute force)."""
 import itertools
 
 import numpy as np
+import pytest
 from hypothesis import given, settings
 from hypothesis import strategies as st
 
@@ -126,3 +127,34 @@ def test_score_drop_invariants(T, E, kk, cf, padded, seed, ties):
     cg = O.pick_rank_counts(idx, ar, E, group_of_expert=g)
     for j in range(k):
         assert cg["differs"][j] == sum(1 for t in range(T) if g[idx[t, j]] != g[idx[t, 0]])
+
+
+@settings(max_examples=150, deadline=None)
+@given(parts=st.integers(1, 5), E=st.integers(1, 12), kk=st.integers(1, 4),
+       cf=st.sampled_from([0.0, 0.5, 1.0, 2.0]), seed=st.integers(0, 2**31 - 1))
+def test_replica_record_invariants(parts, E, kk, cf, seed):
+    """The job record adds up the replicas': counts, drops and tokens are sums, the capacity
+    is the sum of the capacities, and the percentiles are those of the summed kept counts."""
+    k = min(kk, E)
+    rng = np.random.default_rng(seed)
+    recs, singles = [], []
+    for _ in range(parts):
+        T = int(rng.integers(1, 30))
+        idx = _topk_rows(rng, T, E, k)
+        C = O.capacity(cf, T, k, E)
+        a = O.assign(idx, E, C)
+        recs.append((a["routed"], a["kept"], a["assign_row"], C))
+        singles.append(O.load_stats(a["routed"], a["kept"], a["assign_row"], C))
+    job = O.replica_load_stats(recs)
+    for key in ("active_tokens", "routed_total", "kept_total", "dropped", "tokens_with_drop",
+                "tokens_fully_dropped"):
+        assert job[key] == sum(s[key] for s in singles), key
+    assert job["dropped_by_rank"] == [sum(s["dropped_by_rank"][j] for s in singles)
+                                      for j in range(k)]
+    caps = [r[3] for r in recs]
+    assert job["capacity"] == (-1 if any(c is None for c in caps) else sum(caps))
+    kept = np.sum([r[1] for r in recs], axis=0)
+    assert job["max"] == float(kept.max())
+    assert job["p50"] == pytest.approx(float(np.percentile(kept, 50)))
+    if job["capacity"] >= 0:
+        assert job["max"] <= job["capacity"]
