@@ -207,8 +207,9 @@ typedef struct moe_layer_buffers {
  * sends each token's row to the owners of its experts, combine returns the results.
  * [EP-checks] "Capacity factor changes quality, memory and the latency tail": tokens past
  * the capacity are dropped before the exchange, so each rank routes, ranks and drops its
- * own tokens with moe_route + moe_dispatch (x_perm may be NULL) exactly as on one GPU, and
- * the EP result on a rank equals the single-GPU layer on that rank's tokens.
+ * own tokens with moe_route + moe_dispatch (moe_dispatch_scored under MOE_DROP_SCORE; x_perm
+ * may be NULL) exactly as on one GPU, and the EP result on a rank equals the single-GPU layer
+ * on that rank's tokens.
  *
  * No collective library moves the rows: every rank can address every rank's count
  * matrix, receive buffer and result buffer (peer pointers through NVLink, opened with
