@@ -31,7 +31,7 @@ sys.path.insert(0, ROOT)
 import routing_dispatch_expert_warp_b200 as M  # noqa: E402
 from routing_dispatch_expert_warp_b200 import workload as W  # noqa: E402
 
-DEFAULT = W.MIXTRAL_8X7B
+DEFAULT = W.DSV3_PREFILL_ZIPF
 METRIC = "MoE-layer tokens/s on 1 B200; grouped-GEMM % BF16 peak; permute/combine % HBM BW"
 L2_FLUSH_BYTES = 256 << 20
 
@@ -465,7 +465,7 @@ def run_gpu(args) -> None:
         M.moe_check_device_error(lyr.ws)
 
     if rank == 0:
-        cpu = cpu_baseline(shape, args.cpu_sample_tokens) if (world == 1 and not args.no_cpu) else None
+        cpu = cpu_baseline(shape, args.cpu_sample_rows) if (world == 1 and not args.no_cpu) else None
         line = {
             "metric": METRIC,
             "value": shape.T * world / (ms_per_step * 1e-3),
@@ -719,44 +719,123 @@ def run_microbatch(args) -> None:
     print(json.dumps(line), flush=True)
 
 
-def _cpu_cores() -> int:
+def _cpu_cores() -> dict:
+    """Host cores this process may run on (its affinity mask) and the threads numpy's BLAS
+    pool uses, which is what the oracle's matrix products run on."""
+    cores = len(os.sched_getaffinity(0))
+    blas = None
     try:
         from threadpoolctl import threadpool_info
-        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
-        return int(n)
+        blas = max((int(i.get("num_threads", 1)) for i in threadpool_info()), default=None)
     except Exception:
-        return len(os.sched_getaffinity(0))
+        pass
+    return {"cores": cores, "blas_threads": blas}
 
 
 class CpuSample:
-    """The oracle as it stands, on the first `sample_tokens` tokens of the workload (full
-    weights, the same routing rule; capacity follows T as its definition says)."""
+    """The oracle as it stands, timed on the host cores on a bounded, seeded sample of the
+    workload, and extrapolated to the whole layer.
 
-    def __init__(self, shape, sample_tokens: int):
-        self.shape, self.n = shape, sample_tokens
-        self.sub = shape.replace(T=sample_tokens)
-        inp = W.make_inputs(self.sub, device="cpu")
-        f = lambda t: t.float().numpy()
-        bias = None if inp.logit_bias is None else f(inp.logit_bias)
-        self.args = (f(inp.x), f(inp.w_router), bias, f(inp.w_gate), f(inp.w_up),
-                     f(inp.w_down))
+    Routing (fp64 logits, fp32 top-k, capacity, slots) and the load statistics run on all T
+    tokens: capacity needs them all.  The expert FFN, with the permute of its rows and its
+    share of the combine, runs on a seeded sample of whole experts (every kept row of each),
+    drawn until the sample holds `sample_rows` kept rows; its time is scaled by kept_total /
+    kept rows in the sample.  Whole experts keep the oracle's per-row cost (each expert's
+    weights are converted to fp64 once, then used for all its rows) as it is at full size,
+    so the estimate does not change with the sample size.  Inputs are the workload's own
+    (generated on the GPU when there is one, as the GPU path's are) copied to the host."""
+
+    def __init__(self, shape, sample_rows: int):
+        import numpy as np
+        from oracle import moe_oracle as O
+        self.O, self.np = O, np
+        self.shape, self.sample_rows = shape, sample_rows
+        src = "cuda" if torch.cuda.is_available() else "cpu"
+        inp = W.make_inputs(shape, device=src, weights=False)
+        host = lambda t: None if t is None else t.detach().float().cpu().numpy()
+        self.x, self.w_router, self.bias = host(inp.x), host(inp.w_router), host(inp.logit_bias)
+        del inp
+        self.x64 = self.x.astype(np.float64)
+        r = self._route()
+        kept = r["kept"]
+        nz = np.nonzero(kept)[0]
+        order = np.random.default_rng(shape.seed).permutation(nz)
+        chosen, rows = [], 0
+        for e in order:
+            chosen.append(int(e))
+            rows += int(kept[e])
+            if rows >= sample_rows:
+                break
+        self.experts = sorted(chosen)
+        self.kept_sample, self.kept_total = rows, int(kept.sum())
+        self.weights = {}
+        for e in self.experts:
+            wg, wu, wd = W.expert_weights(shape, e, device=src)
+            self.weights[e] = (host(wg), host(wu), host(wd))
+        # the sample's part of the combine: the tokens with a kept pick in the sample, their
+        # other picks masked, rows renumbered into the sample's stacked FFN output
+        ar = r["assign_row"]
+        local = np.full(ar.shape, -1, dtype=np.int64)
+        base = 0
+        for e in self.experts:
+            s0, n = int(r["offsets"][e]), int(kept[e])
+            m = (ar >= s0) & (ar < s0 + n)
+            local[m] = ar[m] - s0 + base
+            base += n
+        self.tokens = np.nonzero((local >= 0).any(axis=1))[0]
+        self.local = local[self.tokens]
+
+    def _route(self):
+        O, s = self.O, self.shape
+        sel_only = s.bias_mode == O.BIAS_SELECTION_ONLY
+        z64 = O.router_logits(self.x, self.w_router, None if sel_only else self.bias)
+        z32 = O.logits_to_fp32(z64)
+        return O.route(z32, s.k, s.gating, float(self.np.float32(s.capacity_factor)), s.layout,
+                       s.n_groups, s.topk_groups, self.bias if sel_only else None, s.bias_mode,
+                       s.drop_policy)
+
+    def sample_outputs(self, r):
+        """The sample's FFN and combine: for the tokens with a kept pick among the sampled
+        experts, the gate-weighted sum of those picks' expert outputs (other picks left out)."""
+        O, np = self.O, self.np
+        ys = []
+        for e in self.experts:
+            s0, n = int(r["offsets"][e]), int(r["kept"][e])
+            x_rows = O.permute(self.x64, r["token_of_row"][s0:s0 + n])
+            _, y = O.swiglu_expert(x_rows, *self.weights[e])
+            ys.append(y)
+        return O.combine(np.concatenate(ys), self.local, r["w"][self.tokens])
 
     def run(self) -> dict:
-        from oracle import moe_oracle as O
-        s = self.sub
+        O = self.O
         t0 = time.perf_counter()
-        O.moe_layer(*self.args, k=s.k, gating=s.gating, capacity_factor=s.capacity_factor,
-                    layout=s.layout, n_groups=s.n_groups, topk_groups=s.topk_groups,
-                    bias_mode=s.bias_mode, drop_policy=s.drop_policy)
-        dt = time.perf_counter() - t0
-        return {"value": self.n / dt, "unit": "tokens/s", "cores": _cpu_cores(),
-                "kind": "oracle", "seconds": dt,
-                "sample": f"oracle moe_layer on the first {self.n} tokens of {self.shape.name} "
-                          f"(full-size weights, fp64 numpy), {dt:.1f} s"}
+        r = self._route()
+        t1 = time.perf_counter()
+        self.sample_outputs(r)
+        t2 = time.perf_counter()
+        O.load_stats(r["routed"], r["kept"], r["assign_row"], r["C"])
+        t3 = time.perf_counter()
+        scale = self.kept_total / max(self.kept_sample, 1)
+        est = (t1 - t0) + (t2 - t1) * scale + (t3 - t2)
+        cores = _cpu_cores()
+        return {"value": self.shape.T / est, "unit": "tokens/s", "cores": cores["cores"],
+                "blas_threads": cores["blas_threads"], "kind": "oracle",
+                "seconds_measured": t3 - t0, "seconds_extrapolated": est,
+                "sample": (f"{self.shape.name}: oracle routing and load statistics on all "
+                           f"{self.shape.T} tokens; permute + expert FFN + combine on "
+                           f"{len(self.experts)} seeded experts holding {self.kept_sample} of "
+                           f"{self.kept_total} kept rows, time scaled by {scale:.2f} "
+                           f"(extrapolated); fp64 numpy")}
 
 
-def cpu_baseline(shape, sample_tokens: int) -> dict:
-    return CpuSample(shape, sample_tokens).run()
+def cpu_baseline(shape, sample_rows: int, repeats: int = 3) -> dict:
+    """One untimed run, then the median of `repeats` timed runs."""
+    cs = CpuSample(shape, sample_rows)
+    cs.run()
+    vals = [cs.run() for _ in range(repeats)]
+    out = dict(vals[0])
+    out["value"] = statistics.median(v["value"] for v in vals)
+    return out
 
 
 def run_reference(args) -> None:
@@ -764,7 +843,7 @@ def run_reference(args) -> None:
     if rank != 0:
         return
     shape = workload_shape(args)
-    sample = CpuSample(shape, args.ref_sample_tokens)
+    sample = CpuSample(shape, args.cpu_sample_rows)
     for _ in range(args.warmup):
         sample.run()
     vals = [sample.run() for _ in range(args.steps)]
@@ -772,14 +851,15 @@ def run_reference(args) -> None:
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": args.ref_sample_tokens / v * 1e3, "higher_is_better": True,
+        "ms_per_step": shape.T / v * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": shape.name, "T": shape.T, "d_model": shape.d_model,
                    "d_ff": shape.d_ff, "E": shape.E, "k": shape.k,
                    "gating": "softmax" if shape.gating == W.SOFTMAX else "sigmoid",
                    "capacity_factor": shape.capacity_factor, "drop_order": args.drop_policy},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[0]["cores"],
-                         "kind": "oracle", "sample": vals[0]["sample"]},
+                         "blas_threads": vals[0]["blas_threads"], "kind": "oracle",
+                         "sample": vals[0]["sample"]},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -801,8 +881,9 @@ def main():
                     help="override E of the workload (small profiling cases with the full "
                          "per-expert GEMM shapes)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--cpu-sample-tokens", type=int, default=64)
-    ap.add_argument("--ref-sample-tokens", type=int, default=32)
+    ap.add_argument("--cpu-sample-rows", type=int, default=2048,
+                    help="kept rows of the seeded expert sample the CPU oracle's FFN runs on "
+                         "(both the cpu_baseline leg and --impl reference)")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--ep-emulate", type=int, default=0,
                     help="time the expert-parallel layer with this many ranks emulated on one "

@@ -360,15 +360,30 @@ moe_status_t moe_dispatch_scored(const moe_config_t* cfg, const void* x,
  *     current; make that first call before any stream capture.
  *   - Every call shares the one array: two calls that run on the GPU at the same time
  *     (other streams, other host threads) race and give wrong results.  Order them.
- *   - The status record is cleared at the start of each call and kernel-side errors are
- *     not reported: an expert index outside [0, E) is skipped like a dropped pick.  Use
- *     moe_dispatch with a workspace to have such errors reported.
+ *   - Kernel-side errors go to a status record in the same fixed array, which starts at
+ *     zero and keeps the first error since it was last read: an expert index outside
+ *     [0, E) (the pick is skipped, like a dropped one) or a bounded wait in the permute
+ *     that ran out (x_perm is then incomplete).  A call does not clear it;
+ *     moe_static_scratch_check() reports and clears it, without allocating.
  */
 moe_status_t moe_dispatch_static_scratch(const moe_config_t* cfg, const void* x,
                                          const int32_t* topk_idx, int32_t* routed_counts,
                                          int32_t* kept_counts, int32_t* expert_offsets,
                                          int32_t* assign_row, int32_t* token_of_row,
                                          void* x_perm, void* stream);
+
+/*
+ * The kernel-side errors of moe_dispatch_static_scratch on the current device, for the same
+ * callers (no counterpart on the pages; nothing is allocated).  Synchronises `stream`
+ * (enqueue order: after the dispatch calls to be checked), reads the fixed scratch's status
+ * record and, if it holds an error, clears it.  Returns MOE_OK if no call recorded an error
+ * since the last check, else MOE_ERR_DEVICE_DATA (invalid expert index; the flat index of
+ * the first one is in moe_last_error()) or MOE_ERR_TIMEOUT (a bounded wait in the permute
+ * ran out).  Like the dispatch calls it shares the one array: checks and dispatches that
+ * overlap on the GPU race.  Its first use on a device may do the device's set-up (see
+ * moe_dispatch_static_scratch).
+ */
+moe_status_t moe_static_scratch_check(void* stream);
 
 /*
  * Expert SwiGLU FFN as a grouped GEMM over the variable-sized buckets ([EP-checks]

@@ -24,7 +24,7 @@ DROP_TOKEN_ORDER, DROP_PICK_RANK, DROP_SCORE = 0, 1, 2
 
 __all__ = ["MoEError", "make_config", "workspace_size", "capacity", "max_rows",
            "alloc_workspace", "moe_route", "moe_dispatch", "moe_dispatch_scored",
-           "moe_dispatch_static_scratch", "moe_pick_rank_counts",
+           "moe_dispatch_static_scratch", "moe_static_scratch_check", "moe_pick_rank_counts",
            "moe_expert_ffn", "moe_expert_ffn_gather", "moe_expert_ffn_combine", "moe_combine",
            "moe_load_stats", "moe_load_stats_merge", "moe_layer_forward",
            "moe_check_device_error",
@@ -205,6 +205,12 @@ def moe_load_stats_merge(cfg, routed_sum, kept_sum, parts, dev_out, host: bool =
 def moe_layer_forward(cfg, inputs: MoeLayerInputs, bufs: MoeLayerBuffers, ws, stream=None):
     check(_lib().moe_layer_forward(ctypes.byref(cfg), ctypes.byref(inputs), ctypes.byref(bufs),
                                    _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def moe_static_scratch_check(stream=None):
+    """Report (MoEError) and clear the kernel-side errors recorded by
+    moe_dispatch_static_scratch since the last check; allocates nothing."""
+    check(_lib().moe_static_scratch_check(_stream(stream)))
 
 
 def moe_check_device_error(ws, stream=None):

@@ -115,6 +115,7 @@ PROTOTYPES = {
                                      P(MoeLoadStats), c_vp]),
     "moe_layer_forward": (c_i32, [P(MoeConfig), P(MoeLayerInputs), P(MoeLayerBuffers), c_vp,
                                   c_sz, c_vp]),
+    "moe_static_scratch_check": (c_i32, [c_vp]),
     "moe_check_device_error": (c_i32, [c_vp, c_sz, c_vp]),
     "moe_last_error": (ctypes.c_char_p, []),
     "moe_status_string": (ctypes.c_char_p, [c_i32]),

@@ -618,6 +618,21 @@ int64_t ep_bound(const Shape& s, const moe_ep_config_t* ep) {
 
 }  // namespace
 
+namespace {
+// A kernel-recorded status as the call's status and message.
+moe_status_t device_error_status(const DevStatus& h) {
+  if (h.code == DEV_TIMEOUT)
+    return fail(MOE_ERR_TIMEOUT, "a device wait ran out (site %u, item %llu)", h.where,
+                (unsigned long long)h.info);
+  if (h.code == DEV_RECV_OVERFLOW)
+    return fail(MOE_ERR_DEVICE_DATA,
+                "expert-parallel row past the receive buffer's recv_rows (pick %llu)",
+                (unsigned long long)h.info);
+  return fail(MOE_ERR_DEVICE_DATA, "invalid expert index in topk_idx (flat index %llu)",
+              (unsigned long long)h.info);
+}
+}  // namespace
+
 extern "C" {
 
 int64_t moe_ep_recv_rows_bound(const moe_config_t* cfg, const moe_ep_config_t* ep) {
@@ -818,15 +833,15 @@ moe_status_t moe_check_device_error(void* ws, size_t ws_bytes, void* stream) {
   if (h.code == DEV_OK) return MOE_OK;
   err = cudaMemset(ws, 0, sizeof(DevStatus));
   if (err != cudaSuccess) return cuda_fail(err, "moe_check_device_error clear");
-  if (h.code == DEV_TIMEOUT)
-    return fail(MOE_ERR_TIMEOUT, "a device wait ran out (site %u, item %llu)", h.where,
-                (unsigned long long)h.info);
-  if (h.code == DEV_RECV_OVERFLOW)
-    return fail(MOE_ERR_DEVICE_DATA,
-                "expert-parallel row past the receive buffer's recv_rows (pick %llu)",
-                (unsigned long long)h.info);
-  return fail(MOE_ERR_DEVICE_DATA, "invalid expert index in topk_idx (flat index %llu)",
-              (unsigned long long)h.info);
+  return device_error_status(h);
+}
+
+moe_status_t moe_static_scratch_check(void* stream) {
+  DevStatus h;
+  cudaError_t err = static_scratch_status(&h, static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_static_scratch_check");
+  if (h.code == DEV_OK) return MOE_OK;
+  return device_error_status(h);
 }
 
 moe_status_t moe_selftest_bounded_wait(void* ws, size_t ws_bytes, void* stream) {

@@ -593,36 +593,52 @@ static __device__ __align__(256) uint8_t g_dispatch_scratch[kStaticStatusBytes +
 namespace {
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+// The fixed array's device address on the current device.  Set-up, once per device with
+// that device current: the host-side name of the array is not a device address, so the
+// runtime is asked for the device address, which is kept.
+cudaError_t static_scratch_base(void** base) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    err = cudaGetSymbolAddress(&p, g_dispatch_scratch);
+    if (err != cudaSuccess) return err;
+    g_scratch_ptr[dev] = p;
+  }
+  *base = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
 }  // namespace
 
 cudaError_t dispatch_static_scratch(const Shape& s, const void* x, const int32_t* topk_idx,
                                     int32_t* routed, int32_t* kept, int32_t* offsets,
                                     int32_t* assign_row, int32_t* token_of_row, void* x_perm,
                                     uint64_t wait_ns, cudaStream_t st) {
-  int dev = 0;
-  cudaError_t err = cudaGetDevice(&dev);
-  if (err != cudaSuccess) return err;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   void* base = nullptr;
-  {
-    // Set-up, once per device with that device current: the host-side name of the array
-    // is not a device address, so ask the runtime for the device address and keep it.
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
-      void* p = nullptr;
-      err = cudaGetSymbolAddress(&p, g_dispatch_scratch);
-      if (err != cudaSuccess) return err;
-      g_scratch_ptr[dev] = p;
-    }
-    base = g_scratch_ptr[dev];
-  }
+  cudaError_t err = static_scratch_base(&base);
+  if (err != cudaSuccess) return err;
+  // The status record starts at zero (static storage) and holds the first error since the
+  // last static_scratch_status() read, which clears it; the histogram is fully rewritten
+  // by every call.
   DevStatus* status = static_cast<DevStatus*>(base);
   int32_t* hist = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(base) + kStaticStatusBytes);
-  // the status record must start at zero; the histogram is fully rewritten by every call
-  err = cudaMemsetAsync(status, 0, sizeof(DevStatus), st);
-  if (err != cudaSuccess) return err;
   return launch_dispatch(s, x, topk_idx, routed, kept, offsets, assign_row, token_of_row,
                          x_perm, hist, status, wait_ns, st);
+}
+
+cudaError_t static_scratch_status(DevStatus* out, cudaStream_t st) {
+  void* base = nullptr;
+  cudaError_t err = static_scratch_base(&base);
+  if (err != cudaSuccess) return err;
+  err = cudaStreamSynchronize(st);
+  if (err != cudaSuccess) return err;
+  err = cudaMemcpy(out, base, sizeof(DevStatus), cudaMemcpyDeviceToHost);
+  if (err != cudaSuccess || out->code == DEV_OK) return err;
+  return cudaMemset(base, 0, sizeof(DevStatus));
 }
 
 }  // namespace moe

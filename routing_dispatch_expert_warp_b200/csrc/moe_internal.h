@@ -157,5 +157,8 @@ cudaError_t dispatch_static_scratch(const Shape& s, const void* x, const int32_t
                                     int32_t* routed, int32_t* kept, int32_t* offsets,
                                     int32_t* assign_row, int32_t* token_of_row, void* x_perm,
                                     uint64_t wait_ns, cudaStream_t st);
+// Synchronise `st`, copy the fixed scratch's status record to *out and clear it if it holds
+// an error.  Allocates nothing.
+cudaError_t static_scratch_status(DevStatus* out, cudaStream_t st);
 
 }  // namespace moe

@@ -151,9 +151,22 @@ class MoEInputs:
         return self.logit_bias.shape[1]
 
 
+def expert_weights(shape: MoEShape, e: int, device="cpu"):
+    """(W_g[e] [f, d], W_u[e] [f, d], W_d[e] [d, f]) of expert e.  Every expert draws from
+    its own seeded stream, so one expert's weights can be made without the others'."""
+    dev = torch.device(device)
+    g = _gen(shape.seed * 65537 + 3 + e, dev)
+    d, f, dt = shape.d_model, shape.d_ff, shape.torch_dtype
+    wg = _randn((f, d), 1.0 / math.sqrt(d), g, dev).to(dt)
+    wu = _randn((f, d), 1.0 / math.sqrt(d), g, dev).to(dt)
+    wd = _randn((d, f), 1.0 / math.sqrt(f), g, dev).to(dt)
+    return wg, wu, wd
+
+
 def make_inputs(shape: MoEShape, device="cpu", weights: bool = True) -> MoEInputs:
     """Seeded inputs for `shape` on `device`.  Expert weights are drawn one expert at a time
-    so that the fp32 staging buffer stays small for the 22 GB DeepSeek-shaped layers."""
+    (expert_weights) so that the fp32 staging buffer stays small for the 22 GB
+    DeepSeek-shaped layers."""
     dev = torch.device(device)
     g = _gen(shape.seed, dev)
     T, d, f, E = shape.T, shape.d_model, shape.d_ff, shape.E
@@ -173,11 +186,8 @@ def make_inputs(shape: MoEShape, device="cpu", weights: bool = True) -> MoEInput
         w_gate = torch.empty((E, f, d), dtype=dt, device=dev)
         w_up = torch.empty((E, f, d), dtype=dt, device=dev)
         w_down = torch.empty((E, d, f), dtype=dt, device=dev)
-        gw = _gen(shape.seed + 3, dev)
         for e in range(E):
-            w_gate[e] = _randn((f, d), 1.0 / math.sqrt(d), gw, dev).to(dt)
-            w_up[e] = _randn((f, d), 1.0 / math.sqrt(d), gw, dev).to(dt)
-            w_down[e] = _randn((d, f), 1.0 / math.sqrt(f), gw, dev).to(dt)
+            w_gate[e], w_up[e], w_down[e] = expert_weights(shape, e, dev)
     else:
         w_gate = w_up = w_down = None
     return MoEInputs(shape, x, w_router, bias, w_gate, w_up, w_down)

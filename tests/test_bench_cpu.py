@@ -37,11 +37,23 @@ def test_binding_roof_per_workload():
 
 
 def test_recorded_traffic_only_for_the_captured_code(monkeypatch):
-    rec = bench.recorded_traffic("mixtral8x7b_prefill_T4096", False)
-    assert rec is not None and rec["sources"] == bench.gemm_source_hash()
-    monkeypatch.setattr(bench, "gemm_source_hash", lambda: "0" * 16)
-    assert bench.recorded_traffic("mixtral8x7b_prefill_T4096", False) is None
+    recs = {("some_workload", False): {"bytes": 123, "sources": bench.gemm_source_hash(),
+                                       "profile": "profiles/x.md"}}
+    monkeypatch.setattr(bench, "RECORDED_GEMM_TRAFFIC", recs)
+    rec = bench.recorded_traffic("some_workload", False)
+    assert rec is not None and rec["bytes"] == 123
+    assert bench.recorded_traffic("some_workload", True) is None
     assert bench.recorded_traffic("some_other_workload", False) is None
+    monkeypatch.setattr(bench, "gemm_source_hash", lambda: "0" * 16)
+    assert bench.recorded_traffic("some_workload", False) is None
+
+
+def test_every_recorded_traffic_names_its_profile():
+    import os
+    for (workload, _), rec in bench.RECORDED_GEMM_TRAFFIC.items():
+        assert workload in bench.W.WORKLOADS or "_with_" in workload
+        assert rec["bytes"] > 0 and len(rec["sources"]) == 16
+        assert os.path.exists(os.path.join(bench.ROOT, rec["profile"]))
 
 
 def test_code_hash_ignores_comments():
@@ -49,3 +61,54 @@ def test_code_hash_ignores_comments():
     edited = "int a;  // another comment\n/* a different\n block */\n\nint b;\n"
     assert bench._code_only(code) == bench._code_only(edited) == "int a;\nint b;"
     assert bench._code_only(code) != bench._code_only("int a;\nint c;")
+
+
+def _oracle_layer(shape):
+    import numpy as np
+    from oracle import moe_oracle as O
+    inp = W.make_inputs(shape)
+    f = lambda t: None if t is None else t.float().numpy()
+    return O.moe_layer(f(inp.x), f(inp.w_router), f(inp.logit_bias), f(inp.w_gate), f(inp.w_up),
+                       f(inp.w_down), shape.k, shape.gating,
+                       float(np.float32(shape.capacity_factor)), shape.layout), inp
+
+
+def test_cpu_sample_of_all_experts_is_the_whole_layer():
+    """A sample holding every kept row is the oracle's whole layer: scale 1, and the
+    sample's combine gives the layer's output for every token with a kept pick."""
+    import numpy as np
+    shape = W.reduced(W.DSV3_PREFILL_ZIPF, 96, 64, 32)
+    ref, _ = _oracle_layer(shape)
+    cs = bench.CpuSample(shape, sample_rows=10 ** 9)
+    assert cs.kept_sample == cs.kept_total == int(ref["kept"].sum())
+    out = cs.sample_outputs(cs._route())
+    np.testing.assert_allclose(out, ref["out"][cs.tokens], rtol=1e-12, atol=1e-12)
+    r = cs.run()
+    assert r["seconds_extrapolated"] == pytest.approx(r["seconds_measured"], rel=1e-9)
+    assert r["cores"] == len(__import__("os").sched_getaffinity(0))
+
+
+def test_cpu_sample_of_some_experts_is_their_share_of_the_layer():
+    """A partial sample: whole experts drawn until the row budget is met, the time scale is
+    kept_total / sampled rows, and the sample's combine is the layer's combine restricted to
+    the sampled experts' picks."""
+    import numpy as np
+    from oracle import moe_oracle as O
+    shape = W.reduced(W.MIXTRAL_8X22B_MIXED, 200, 64, 48)
+    ref, _ = _oracle_layer(shape)
+    cs = bench.CpuSample(shape, sample_rows=60)
+    kept = ref["kept"]
+    assert cs.kept_sample == int(kept[cs.experts].sum()) >= 60
+    ar = ref["assign_row"]
+    in_s = np.zeros(ar.shape, dtype=bool)
+    for e in cs.experts:
+        s0, n = int(ref["offsets"][e]), int(kept[e])
+        in_s |= (ar >= s0) & (ar < s0 + n)
+    masked = np.where(in_s, ar, -1)
+    want = O.combine(ref["y_perm"], masked, ref["w"])
+    toks = np.nonzero(in_s.any(axis=1))[0]
+    np.testing.assert_array_equal(cs.tokens, toks)
+    np.testing.assert_allclose(cs.sample_outputs(cs._route()), want[toks], rtol=1e-12, atol=1e-12)
+    r = cs.run()
+    scale = cs.kept_total / cs.kept_sample
+    assert scale > 1 and f"scaled by {scale:.2f}" in r["sample"]

@@ -5,7 +5,8 @@ dispatch (an engine whose pool owns the GPU, a plugin host that hands over only 
 output tensors): it takes no workspace and uses the library's fixed device scratch.  Its
 results must equal moe_dispatch's exactly -- this is integer and copy work -- on two calls
 in a row, the second with different routing so that stale scratch from the first call would
-show.  This file is collected last on purpose.
+show.  Its kernel-side errors are kept in the same fixed scratch and reported, without
+allocating, by moe_static_scratch_check.  This file is collected last on purpose.
 """
 import pytest
 import torch
@@ -51,6 +52,7 @@ def test_static_scratch_dispatch_matches_workspace_dispatch(shape):
                                       got.token_of_row, got.x_perm)
         torch.cuda.synchronize()
         M.moe_check_device_error(ws)
+        M.moe_static_scratch_check()      # no kernel-side error recorded
         for name in ("routed_counts", "kept_counts", "expert_offsets", "assign_row",
                      "token_of_row"):
             assert torch.equal(getattr(got, name), getattr(ref, name)), (call, name)
@@ -64,3 +66,32 @@ def test_static_scratch_rejects_sizes_beyond_its_limit():
     with pytest.raises(M.MoEError) as ei:
         M.moe_dispatch_static_scratch(cfg, *([torch.empty(16, dtype=torch.uint8)] * 8), stream=0)
     assert ei.value.status == 2 and "scratch" in str(ei.value)
+
+
+def test_static_scratch_reports_a_bad_expert_index():
+    """A host-made expert index outside [0, E) is skipped by the kernels and recorded in the
+    fixed scratch's status record; moe_static_scratch_check reports it once (and clears it),
+    and it stays recorded across a later clean call until it is read."""
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    dev = torch.device("cuda")
+    shape = SHAPES[0]
+    cfg = M.config_from_shape(shape)
+    inp = W.make_inputs(shape, device=dev, weights=False)
+    ws = M.alloc_workspace(cfg, dev)
+    b = _outputs(cfg, dev)
+    M.moe_route(cfg, inp.x, inp.w_router, inp.logit_bias, b.logits, b.topk_idx, b.topk_w, ws)
+    M.moe_check_device_error(ws)
+    M.moe_static_scratch_check()          # start from a clean record
+    good = b.topk_idx.clone()
+    b.topk_idx[5, 3] = shape.E + 7
+    args = (b.routed_counts, b.kept_counts, b.expert_offsets, b.assign_row, b.token_of_row,
+            b.x_perm)
+    M.moe_dispatch_static_scratch(cfg, inp.x, b.topk_idx, *args)
+    M.moe_dispatch_static_scratch(cfg, inp.x, good, *args)    # a clean call keeps the record
+    with pytest.raises(M.MoEError) as ei:
+        M.moe_static_scratch_check()
+    assert ei.value.status == 6 and str(5 * shape.k + 3) in str(ei.value)
+    M.moe_static_scratch_check()          # cleared by the read
+    M.moe_dispatch_static_scratch(cfg, inp.x, good, *args)
+    M.moe_static_scratch_check()
