@@ -489,6 +489,8 @@ def run_gpu(args) -> None:
                                     else "permuted copy x_perm"),
                        "combine": ("fused into the down GEMM epilogue" if args.fused_combine
                                    else "separate kernel"),
+                       "ffn_kernel": ("CTA pairs, 256 x 256 tiles" if args.ffn_kernel == "pairs"
+                                      else "single CTAs, 128 x 256 tiles"),
                        "parallelism": f"replicas x{world} (EP=1, no exchange)"},
             "roofline": dict(
                 roof,
@@ -895,11 +897,16 @@ def main():
     ap.add_argument("--microbatches", type=int, default=1,
                     help="time the layer as this many microbatches ping-ponging over two "
                          "streams against the one-stream layer (a separate measurement)")
+    ap.add_argument("--ffn-kernel", default="single", choices=["pairs", "single"],
+                    help="the plain expert FFN on CTA pairs (256 x 256 tiles over the two SMs "
+                         "of a TPC) or on single CTAs (128 x 256 tiles)")
     ap.add_argument("--drop-policy", default="token", choices=sorted(DROP_POLICIES),
                     help="which picks an overflowing expert keeps: token order, pick rank "
                          "first, or highest selection score")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)   # at least three untimed warm-up steps
+    if args.impl != "reference":
+        M.set_ffn_cta_pairs(args.ffn_kernel == "pairs")
     if args.impl == "reference":
         run_reference(args)
     elif args.microbatches > 1:

@@ -531,6 +531,17 @@ const char* moe_status_string(moe_status_t status);
  * up, records MOE_ERR_TIMEOUT and returns (default 2e9).  0 restores the default. */
 void moe_set_wait_limit_ns(uint64_t ns);
 
+/* Which kernel runs the bf16 expert FFN of moe_expert_ffn / moe_layer_forward (permuted
+ * rows, combine separate), for the whole process; a choice of schedule, not of results
+ * (both compute the same sums in the same K order and give bitwise the same h and y_perm).
+ * on == 0 (the default): one CTA per 128 x 256 output tile.  on != 0: each 256 x 256 tile
+ * is computed by a pair of CTAs on the two SMs of a TPC sharing one tensor-core MMA (a
+ * cluster of two), each CTA loading half of each operand -- a third fewer bytes from L2
+ * per FLOP, measured slower on the layer's shapes; if no cluster of two fits on the
+ * device, the single-CTA kernel runs.  The gathered-A and fused-combine forms and the
+ * expert-parallel FFN always use the single-CTA kernel. */
+void moe_set_ffn_cta_pairs(int on);
+
 /* Self-test of the bounded wait: one block waits on an on-chip barrier that nothing
  * completes, with the current limit, records MOE_ERR_TIMEOUT in the workspace status
  * word and returns.  Used to check that a run-out wait leaves the context usable. */

@@ -28,7 +28,7 @@ __all__ = ["MoEError", "make_config", "workspace_size", "capacity", "max_rows",
            "moe_expert_ffn", "moe_expert_ffn_gather", "moe_expert_ffn_combine", "moe_combine",
            "moe_load_stats", "moe_load_stats_merge", "moe_layer_forward",
            "moe_check_device_error",
-           "moe_selftest_bounded_wait", "set_wait_limit_ns", "kernel_launch_count",
+           "moe_selftest_bounded_wait", "set_wait_limit_ns", "set_ffn_cta_pairs", "kernel_launch_count",
            "LayerBuffers", "MoELayer", "HostPipeline"]
 
 
@@ -93,6 +93,11 @@ def alloc_workspace(cfg: MoeConfig, device="cuda", stream=None) -> torch.Tensor:
 
 def set_wait_limit_ns(ns: int) -> None:
     _lib().moe_set_wait_limit_ns(ns)
+
+
+def set_ffn_cta_pairs(on: bool) -> None:
+    """The plain expert FFN on CTA pairs (True) or on single CTAs (False, the default)."""
+    _lib().moe_set_ffn_cta_pairs(1 if on else 0)
 
 
 # ------------------------------------------------------------------ stages

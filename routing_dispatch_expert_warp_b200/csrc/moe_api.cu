@@ -233,6 +233,9 @@ const char* moe_status_string(moe_status_t st) {
 
 void moe_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns == 0 ? 2000000000ull : ns); }
 
+void moe_set_ffn_cta_pairs(int on) { set_ffn_cta_pairs(on); }
+
+
 moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
   Shape s;
   moe_status_t st = check_config(cfg, &s);

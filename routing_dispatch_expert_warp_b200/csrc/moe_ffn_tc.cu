@@ -34,6 +34,7 @@
 // through L2.  The tile table is built on the device from the bucket counts: no host read.
 // Every barrier wait is bounded; a wait that runs out records MOE_ERR_TIMEOUT, makes the
 // other roles stop, drains the copies and MMAs in flight, frees TMEM and returns.
+#include <atomic>
 #include <mutex>
 
 #include "moe_internal.h"
@@ -531,6 +532,277 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
   }
 }
 
+// ------------------------------------------------------------------ CTA-pair variant
+// The same grouped GEMM with each 256 x 256 tile shared by the two CTAs of a cluster, which
+// sit on the two SMs of a TPC and issue one tcgen05 MMA together (cta_group::2, 256x256x16):
+// CTA r loads rows [128 r, 128 r + 128) of the tile's A and rows [128 r, 128 r + 128) of its
+// 256 B rows (gate/up: rank 0 the W_g rows, rank 1 the same W_u rows), so each SM moves
+// 32 KB per 64-deep K step instead of 48 KB for the same MMA work, and a 6-stage ring fits
+// where the single-CTA kernel holds 4.  Rank 0's producer arms its stage barrier for both
+// CTAs' bytes, both CTAs' copies complete on it, rank 0's MMA warp waits on it alone and its
+// commits arrive on the stage-free and accumulator-full barriers of both CTAs.  Each CTA's
+// epilogue drains its own 128 accumulator rows (TMEM lane r = tile row 128 rank + r) and
+// arrives on rank 0's accumulator-free barrier.  Tiles: (expert, n-block, 256-row m-block),
+// m-blocks innermost, one cluster per tile.
+constexpr int PBM = 256;                               // rows of a pair tile
+constexpr int P_STAGES = 6;
+constexpr int P_A_BYTES = 128 * BK * 2;                // this CTA's 128 rows of A
+constexpr int P_B_BYTES = 128 * BK * 2;                // this CTA's 128 of the 256 B rows
+constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;   // 32 KB
+constexpr int P_DYN_SMEM = P_STAGES * P_STAGE_BYTES + 1024;
+constexpr uint32_t P_EPI_ARRIVALS = 8;                 // 4 epilogue warps x 2 CTAs
+
+template <int MODE>
+__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_pair_kernel(
+    const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
+    const __grid_constant__ CUtensorMap tm_b1, const TcParams p) {
+  static_assert(MODE == MODE_DOWN || MODE == MODE_SWIGLU, "expert FFN launches only");
+  constexpr bool GATED = MODE == MODE_SWIGLU;
+  constexpr int BN_OUT = GATED ? 128 : 256;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[P_STAGES];   // used in rank 0 only
+  __shared__ __align__(8) uint64_t empty_bar[P_STAGES];
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];        // used in rank 0 only
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int abort_s;
+  __shared__ int tile_base[MOE_MAX_EXPERTS + 1];
+  __shared__ int mblocks[MOE_MAX_EXPERTS];
+
+  // the same offsets in both CTAs: the MMA reads the peer's operands at this CTA's offsets
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int cluster = static_cast<int>(blockIdx.x >> 1);
+  const int clusters = static_cast<int>(gridDim.x >> 1);
+
+  if (warp == 0) {  // tile table: 256-row m-blocks per expert and their prefix (x n_blocks)
+    int carry = 0;
+    for (int e0 = 0; e0 < p.E; e0 += 32) {
+      const int e = e0 + lane;
+      const int mb = e < p.E ? (p.seg_count[e] + PBM - 1) / PBM : 0;
+      int v = mb;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += o;
+      }
+      if (e < p.E) {
+        mblocks[e] = mb;
+        tile_base[e] = (carry + v - mb) * p.n_blocks;
+      }
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) {
+      tile_base[p.E] = carry * p.n_blocks;
+      prefetch_tensormap(&tm_a);
+      prefetch_tensormap(&tm_b0);
+      if (GATED) prefetch_tensormap(&tm_b1);
+    }
+  } else if (warp == 1) {
+    tmem_alloc_pair(&tmem_base_s, TMEM_COLS);
+    tmem_relinquish_pair();
+  } else if (threadIdx.x == 64) {
+    for (int s = 0; s < P_STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], P_EPI_ARRIVALS);
+    }
+    mbar_init(&drain_bar, 1);
+    abort_s = 0;
+    fence_barrier_init();
+  }
+  // barriers of both CTAs initialised (the peer signals rank 0's) and the TMEM address known
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();
+  tc_fence_after();
+
+  const uint32_t tmem_base = tmem_base_s;
+  const int total_tiles = tile_base[p.E];
+  const int KB = p.K / BK;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- TMA producer (both)
+    int s = 0;
+    uint32_t ph = 0;
+    uint32_t armed = 0, armed_parity = 0;
+    bool ok = true;
+    for (int tile = cluster; ok && tile < total_tiles; tile += clusters) {
+      int e, mb, nb;
+      decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, 0, e, mb, nb);
+      const int row0 = p.seg_start[e] + mb * PBM + static_cast<int>(rank) * 128;
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&empty_bar[s], ph ^ 1u, p.wait_ns, &abort_s)) {
+          if (!abort_s)
+            record_error(p.status, DEV_TIMEOUT, 30, static_cast<unsigned long long>(tile));
+          abort_s = 1;
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + s * P_STAGE_BYTES;
+        uint8_t* sb = sa + P_A_BYTES;
+        const uint32_t full = cluster_addr(smem_addr(&full_bar[s]), 0);
+        if (rank == 0) {  // both CTAs' bytes complete on rank 0's barrier
+          mbar_arrive_expect_tx(&full_bar[s], 2 * P_STAGE_BYTES);
+          armed |= 1u << s;
+          armed_parity = (armed_parity & ~(1u << s)) | (ph << s);
+        }
+        tma_load_2d_pair(sa, &tm_a, full, kb * BK, row0);
+        if (GATED)
+          tma_load_3d_pair(sb, rank == 0 ? &tm_b0 : &tm_b1, full, kb * BK, nb * 128, e);
+        else
+          tma_load_3d_pair(sb, &tm_b0, full, kb * BK, nb * 256 + static_cast<int>(rank) * 128, e);
+        if (++s == P_STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+    // every fill rank 0 armed must land before the block can exit (the peer's own fills are
+    // counted there too; a peer that gave up waited at least the wait limit first)
+    for (int q = 0; q < P_STAGES; ++q)
+      if ((armed >> q) & 1u)
+        mbar_wait(&full_bar[q], (armed_parity >> q) & 1u, p.wait_ns, nullptr);
+  } else if (warp == 1 && lane == 0 && rank == 0) {
+    // ---------------------------------------------------------------- MMA issuer (rank 0)
+    constexpr uint32_t idesc = idesc_bf16_f32(PBM, MMA_N);
+    int s = 0;
+    uint32_t ph = 0;
+    int acc = 0;
+    uint32_t aph = 0;
+    bool ok = true;
+    bool issued = false;
+    for (int tile = cluster; ok && tile < total_tiles; tile += clusters) {
+      if (!mbar_wait(&tempty_bar[acc], aph ^ 1u, p.wait_ns, &abort_s)) {
+        if (!abort_s) record_error(p.status, DEV_TIMEOUT, 31, static_cast<unsigned long long>(tile));
+        abort_s = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_COLS);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&full_bar[s], ph, p.wait_ns, &abort_s)) {
+          if (!abort_s) record_error(p.status, DEV_TIMEOUT, 32, static_cast<unsigned long long>(tile));
+          abort_s = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = smem_addr(smem + s * P_STAGE_BYTES);
+        const uint32_t b_addr = a_addr + P_A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          tc_mma_f16_pair(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
+                          sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+        issued = true;
+        tc_commit_pair(&empty_bar[s], 0x3);
+        if (++s == P_STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (!ok) break;
+      tc_commit_pair(&tfull_bar[acc], 0x3);
+      acc ^= 1;
+      if (acc == 0) aph ^= 1u;
+    }
+    if (!ok && issued) {  // MMAs still reading shared memory / writing TMEM must finish first
+      tc_commit_pair(&drain_bar, 0x1);
+      mbar_wait(&drain_bar, 0, p.wait_ns, nullptr);
+    }
+  } else if (warp >= 2) {
+    // ---------------------------------------------------------------- epilogue (both)
+    const int q = warp & 3;             // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;        // accumulator row owned by this thread
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int tile = cluster; tile < total_tiles; tile += clusters) {
+      int e, mb, nb;
+      decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, 0, e, mb, nb);
+      const int half0 = mb * PBM + static_cast<int>(rank) * 128;
+      const int row0 = p.seg_start[e] + half0;
+      const int valid = p.seg_count[e] - half0;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&tfull_bar[acc], aph, p.wait_ns, &abort_s) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0 && !abort_s) record_error(p.status, DEV_TIMEOUT, 33, static_cast<unsigned long long>(tile));
+        abort_s = 1;
+        break;
+      }
+      tc_fence_after();
+      if (valid > q * 32) {  // this warp's 32 rows hold at least one of the bucket's rows
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                               static_cast<uint32_t>(acc * ACC_COLS);
+        const bool row_ok = r < valid;
+        __nv_bfloat16* orow = p.out + static_cast<int64_t>(row0 + r) * p.N_out +
+                              static_cast<int64_t>(nb) * BN_OUT;
+        const int cols_left = p.N_out - nb * BN_OUT;
+        if (GATED) {
+#pragma unroll 1
+          for (int c = 0; c < BN_OUT / 32; ++c) {
+            uint32_t g[32], u[32];
+            tmem_ld32(taddr + c * 32, g);
+            tmem_ld32(taddr + 128 + c * 32, u);
+            tmem_ld_wait();
+            if (row_ok && c * 32 < cols_left) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                                    silu_mul(__uint_as_float(g[2 * i + 1]),
+                                             __uint_as_float(u[2 * i + 1])));
+              uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int c = 0; c < BN_OUT / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(taddr + c * 32, v);
+            tmem_ld_wait();
+            if (row_ok && c * 32 < cols_left) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+              uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(cluster_addr(smem_addr(&tempty_bar[acc]), 0));
+      acc ^= 1;
+      if (acc == 0) aph ^= 1u;
+    }
+  }
+
+  // nothing of either CTA may still be signalled, read or written when one of them exits
+  tc_fence_before();
+  __syncwarp();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 // W_r [d, E] fp32 -> hi, lo [E, d] bf16 with hi = bf16(W), lo = bf16(W - hi), so that
 // x . W = x . hi + x . lo up to the rounding of lo (a relative 2^-17 of each weight).
 // 32 x 32 tiles transposed through shared memory.  Block (0, 0) also writes the one-bucket
@@ -609,7 +881,63 @@ bool make_map_weights(CUtensorMap* m, const void* base, int E, int64_t N, int64_
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Clusters of two of grouped_gemm_pair_kernel<MODE> that fit on the GPU at once (0: none).
+template <int MODE>
+int pair_clusters_resident(cudaLaunchConfig_t cfg) {
+  static int cached[2] = {-1, -1};
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  int& c = cached[MODE == MODE_SWIGLU ? 1 : 0];
+  if (c < 0) {
+    int n = 0;
+    cfg.gridDim = dim3(2 * static_cast<unsigned>(sm_count() / 2));
+    if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_pair_kernel<MODE>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    c = n;
+  }
+  return c;
+}
+
+// One launch of the pair kernel over at most `tiles` tiles; *launched = false (nothing
+// enqueued) when no cluster of two fits.
+template <int MODE>
+cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1,
+                        const TcParams& p, int64_t tiles, cudaStream_t st, bool* launched) {
+  *launched = false;
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_pair_kernel<MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, P_DYN_SMEM);
+  if (err != cudaSuccess) return err;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = P_DYN_SMEM;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int64_t clusters = pair_clusters_resident<MODE>(cfg);
+  if (clusters <= 0) return cudaSuccess;
+  if (clusters > tiles) clusters = tiles;
+  if (clusters < 1) clusters = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters));
+  err = cudaLaunchKernelEx(&cfg, grouped_gemm_pair_kernel<MODE>, ta, tb0, tb1, p);
+  if (err != cudaSuccess) return err;
+  note_launch();
+  *launched = true;
+  return cudaSuccess;
+}
+
+std::atomic<int> g_ffn_pairs{0};
+
 }  // namespace
+
+void set_ffn_cta_pairs(int on) { g_ffn_pairs.store(on != 0 ? 1 : 0); }
+int ffn_cta_pairs() { return g_ffn_pairs.load(); }
 
 // Before a down launch with the combine fused in: zero the arrival counters and the output
 // rows of tokens none of whose picks was kept (no thread of the launch ever writes those).
@@ -659,6 +987,45 @@ cudaError_t launch_ffn_tc(const Shape& s, const void* a, const int32_t* a_rows,
 
   const int64_t row_blocks_bound = (s.max_rows + BM - 1) / BM + s.E;
   const int sms = sm_count();
+
+  if (a_rows == nullptr && comb == nullptr && g_ffn_pairs.load() != 0) {
+    // the CTA-pair kernel: B maps with 128-row boxes (each CTA loads half of the 256 rows)
+    CUtensorMap td128;
+    if (!make_map_weights(&td128, wd, s.E, s.d, s.f, 128)) {
+      *why = "tensor map encoding failed (pointer alignment or sizes)";
+      return cudaErrorInvalidValue;
+    }
+    const int64_t pair_blocks_bound = (s.max_rows + PBM - 1) / PBM + s.E;
+    TcParams q1 = {};
+    q1.seg_start = offsets;
+    q1.seg_count = kept;
+    q1.E = s.E;
+    q1.K = static_cast<int>(s.d);
+    q1.n_blocks = static_cast<int>((s.f + 127) / 128);
+    q1.N_out = static_cast<int>(s.f);
+    q1.out = static_cast<__nv_bfloat16*>(h);
+    q1.status = status;
+    q1.wait_ns = wait_ns;
+    bool launched = false;
+    err = launch_pair<MODE_SWIGLU>(ta1, tg, tu, q1, pair_blocks_bound * q1.n_blocks, st, &launched);
+    if (err != cudaSuccess) return err;
+    if (launched) {
+      TcParams q2 = q1;
+      q2.K = static_cast<int>(s.f);
+      q2.n_blocks = static_cast<int>((s.d + 255) / 256);
+      q2.N_out = static_cast<int>(s.d);
+      q2.out = static_cast<__nv_bfloat16*>(y);
+      err = launch_pair<MODE_DOWN>(ta2, td128, td128, q2, pair_blocks_bound * q2.n_blocks, st,
+                                   &launched);
+      if (err != cudaSuccess) return err;
+      if (!launched) {
+        *why = "the down launch found no room for a cluster of two";
+        return cudaErrorLaunchOutOfResources;
+      }
+      return cudaSuccess;
+    }
+    // no cluster of two fits: the single-CTA kernel below
+  }
 
   TcParams p1 = {};
   p1.seg_start = offsets;

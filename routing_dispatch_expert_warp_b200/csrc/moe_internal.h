@@ -148,6 +148,11 @@ cudaError_t launch_ep_stats(const Shape& s, const int32_t* mat, const int32_t* e
                             int world, int ranks_per_node, moe_ep_stats_t* out,
                             cudaStream_t st);
 
+// Expert FFN of the plain (permuted-copy) path on CTA pairs (1) or on single CTAs (0, the
+// default); process-wide.
+void set_ffn_cta_pairs(int on);
+int ffn_cta_pairs();
+
 // Process-wide count of this library's kernel launches (every launch site calls it once).
 void note_launch();
 

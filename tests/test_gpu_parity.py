@@ -161,6 +161,54 @@ def test_bucket_tails_of_every_size(counts, d, f):
     check_layer_output(run, run.b.out, r)
 
 
+def _forced_buckets(counts, d, f, seed=5):
+    """A top-1 layer whose bucket sizes are exactly `counts` (a [T, E] bias forces the picks)."""
+    E, T = len(counts), sum(counts)
+    shape = _edge(T, d, f, E, 1)
+    inp = W.make_inputs(shape, device="cuda")
+    owner = torch.cat([torch.full((c,), e, dtype=torch.long) for e, c in enumerate(counts)])
+    owner = owner[torch.randperm(T, generator=torch.Generator().manual_seed(seed))].cuda()
+    bias = torch.full((T, E), -40.0, device="cuda")
+    bias[torch.arange(T, device="cuda"), owner] = 40.0
+    inp.logit_bias = bias.contiguous()
+    return shape, inp
+
+
+@pytest.mark.parametrize("counts,d,f", [
+    # 256-row pair tiles: tails of 1, 127, 128 (the second CTA of the pair has no rows),
+    # 129, 255, whole tiles, 257, and an empty expert
+    ((1, 127, 128, 129, 255, 256, 257, 0, 511, 513), 256, 384),
+    ((300, 0, 5, 700), 512, 256),          # d = 512 (two 256-column down blocks)
+    ((64, 200, 384), 192, 320),            # d and d_ff not multiples of 256 / 128
+])
+def test_ffn_cta_pairs_equal_single_ctas_and_oracle(counts, d, f):
+    """The expert FFN on CTA pairs (256 x 256 tiles, one MMA over two SMs) and on single
+    CTAs (128 x 256 tiles): both match the oracle, and they compute the same sums in the same
+    K order, so h and y_perm agree bitwise."""
+    shape, inp = _forced_buckets(counts, d, f)
+    run = GpuRun(shape, inp)
+    try:
+        M.set_ffn_cta_pairs(True)
+        st = run.all_stages()
+        r = check_routing(run)
+        assert tuple(int(c) for c in r["kept"]) == counts
+        check_ffn_rows(run, r)
+        check_layer_output(run, run.b.out, r)
+        used = int(run.b.expert_offsets[-1])
+        h1, y1 = run.b.h[:used].clone(), run.b.y_perm[:used].clone()
+        M.set_ffn_cta_pairs(False)
+        run.b.h.zero_(), run.b.y_perm.zero_()
+        run.ffn()
+        M.moe_check_device_error(run.ws)
+        torch.cuda.synchronize()
+        check_ffn_rows(run, r)
+        assert torch.equal(run.b.h[:used], h1), "h differs between the two FFN kernels"
+        assert torch.equal(run.b.y_perm[:used], y1), "y_perm differs between the two FFN kernels"
+        check_stats(st, r)
+    finally:
+        M.set_ffn_cta_pairs(False)
+
+
 def test_tied_logits_pick_lower_index():
     shape = _edge(40, 64, 64, 16, 4, gating=W.SIGMOID)
     inp = W.make_inputs(shape, device="cuda")
