@@ -489,8 +489,9 @@ def run_gpu(args) -> None:
                                     else "permuted copy x_perm"),
                        "combine": ("fused into the down GEMM epilogue" if args.fused_combine
                                    else "separate kernel"),
-                       "ffn_kernel": ("CTA pairs, 256 x 256 tiles" if args.ffn_kernel == "pairs"
-                                      else "single CTAs, 128 x 256 tiles"),
+                       "ffn_kernel": {"token_n": "weight rows as M, tokens as N (tails to 16)",
+                                      "token_major": "single CTAs, 128-token x 256-column tiles",
+                                      "pairs": "CTA pairs, 256 x 256 tiles"}[args.ffn_kernel],
                        "parallelism": f"replicas x{world} (EP=1, no exchange)"},
             "roofline": dict(
                 roof,
@@ -613,6 +614,118 @@ def run_ep_emulated(args) -> None:
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)
+
+
+def ep_rank_inputs(shape, rank: int, world: int, device) -> dict:
+    """This rank's part of the expert-parallel layer (weak scaling: every rank brings its own
+    batch of T tokens, as the replicas do): its batch x (seed + 1000 rank); the layer's router
+    weight and per-expert logit bias, the same on every rank; a per-token bias, drawn with
+    the batch; and the weights of the experts it owns -- contiguous blocks of E / world --
+    each from that expert's own seeded stream, so they equal the single-GPU layer's."""
+    if shape.E % world:
+        raise SystemExit(f"E={shape.E} is not a multiple of the {world} ranks")
+    base = W.make_inputs(shape, device=device, weights=False)
+    batch = W.make_inputs(rank_shape(shape, rank), device=device, weights=False) if rank else base
+    per_token = batch.logit_bias is not None and batch.logit_bias.dim() == 2
+    n_local = shape.E // world
+    experts = list(range(rank * n_local, (rank + 1) * n_local))
+    d, f, dt = shape.d_model, shape.d_ff, shape.torch_dtype
+    wg = torch.empty((n_local, f, d), dtype=dt, device=device)
+    wu = torch.empty((n_local, f, d), dtype=dt, device=device)
+    wd = torch.empty((n_local, d, f), dtype=dt, device=device)
+    for i, e in enumerate(experts):
+        wg[i], wu[i], wd[i] = W.expert_weights(shape, e, device)
+    return {"x": batch.x, "w_router": base.w_router,
+            "logit_bias": batch.logit_bias if per_token else base.logit_bias,
+            "w_gate": wg, "w_up": wu, "w_down": wd, "experts": experts}
+
+
+def run_ep_group(args) -> None:
+    """The expert-parallel layer over the job's GPUs, one process per GPU (torchrun; a single
+    process without it): rank r owns experts [r E/N, (r+1) E/N) and its own batch of T tokens;
+    dispatch and combine move rows over peer memory (CUDA IPC mappings, plain 16-byte loads
+    and stores) and the steps are separated by one-element NCCL all-reduces on the stream.
+    Every step of the EP schedule is timed with CUDA events; the job's time is the slowest
+    rank's."""
+    import datetime
+    import torch.distributed as dist
+    from routing_dispatch_expert_warp_b200 import ep as EP
+    if "WORLD_SIZE" not in os.environ:   # one process: a one-rank group on this host
+        import socket
+        with socket.socket() as so:
+            so.bind(("127.0.0.1", 0))
+            port = so.getsockname()[1]
+        os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK="0",
+                          WORLD_SIZE="1", LOCAL_RANK="0")
+    world = int(os.environ["WORLD_SIZE"])
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    shape = workload_shape(args)
+    inp = ep_rank_inputs(shape, rank, world, dev)
+    cfg = M.config_from_shape(shape)
+    grp = EP.EpGroup(cfg, inp["w_router"], inp["w_gate"], inp["w_up"], inp["w_down"],
+                     EP.contiguous_placement(shape.E, world, dev), inp["logit_bias"],
+                     ranks_per_node=world, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    names = [s_ for s_ in EP.SCHEDULE if s_ != "barrier"] + ["end"]
+    mk = lambda: {n: torch.cuda.Event(enable_timing=True) for n in names}
+    for _ in range(args.warmup):
+        flush.zero_()
+        grp.forward(inp["x"])
+    M.moe_check_device_error(grp.me.ws)
+    evs = [mk() for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    clocks.mark_start()
+    for i in range(args.steps):
+        flush.zero_()
+        grp.forward(inp["x"], on_step=lambda n, e=evs[i]: e[n].record(stream))
+    torch.cuda.synchronize(dev)
+    clocks.mark_end()
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    time.sleep(0.2)
+    clk = clocks.stop()
+    M.moe_check_device_error(grp.me.ws)
+    per = {n: sum(e[n].elapsed_time(e[names[i + 1]]) for e in evs) / args.steps
+           for i, n in enumerate(names[:-1])}
+    mine = [sum(e[names[0]].elapsed_time(e["end"]) for e in evs) / args.steps]
+    mine += [per[n] for n in names[:-1]]
+    slowest = max_over_ranks(mine, dist, dev)
+    ms = slowest[0]
+    st = grp.me.stats_dict()
+    if rank == 0:
+        line = {
+            "metric": f"MoE-layer tokens/s, expert parallel over {world} GPU(s)",
+            "value": world * shape.T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak",
+            "dtype": "bf16" if shape.dtype == W.BF16 else "f32",
+            "data": "synthetic (seeded; every rank its own batch of T tokens)",
+            "config": {"workload": shape.name, "T_per_rank": shape.T, "E": shape.E,
+                       "experts_per_rank": shape.E // world, "placement": "contiguous",
+                       "parallelism": f"EP{world}: dispatch/combine over peer memory (CUDA "
+                                      "IPC), NCCL all-reduce barriers",
+                       "l2": "flushed between timed steps (256 MB write)"},
+            "steps_ms_max_over_ranks": dict(zip(names[:-1], slowest[1:])),
+            "ep_stats": {k: st[k] for k in ("local_fraction", "remote_bytes", "pair_bytes_p50",
+                                             "pair_bytes_p99", "rank_load",
+                                             "rank_load_max_to_mean", "cross_node_fraction")},
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    grp.close()
+    dist.destroy_process_group()
 
 
 def run_microbatch(args) -> None:
@@ -890,6 +1003,10 @@ def main():
     ap.add_argument("--ep-emulate", type=int, default=0,
                     help="time the expert-parallel layer with this many ranks emulated on one "
                          "GPU (a separate measurement, not the headline line)")
+    ap.add_argument("--ep", action="store_true",
+                    help="time the expert-parallel layer across the job's GPUs (one process per "
+                         "GPU under torchrun): experts split in contiguous blocks, every rank "
+                         "its own batch (a separate measurement, not the headline line)")
     ap.add_argument("--fused-combine", action="store_true",
                     help="time the expert FFN with the combine fused into its down GEMM")
     ap.add_argument("--gather", action="store_true",
@@ -897,20 +1014,24 @@ def main():
     ap.add_argument("--microbatches", type=int, default=1,
                     help="time the layer as this many microbatches ping-ponging over two "
                          "streams against the one-stream layer (a separate measurement)")
-    ap.add_argument("--ffn-kernel", default="single", choices=["pairs", "single"],
-                    help="the plain expert FFN on CTA pairs (256 x 256 tiles over the two SMs "
-                         "of a TPC) or on single CTAs (128 x 256 tiles)")
+    ap.add_argument("--ffn-kernel", default="token_major",
+                    choices=["token_major", "token_n", "pairs"],
+                    help="the plain expert FFN kernel: 128-token x 256-column tiles, weight rows "
+                         "as the MMA's M and tokens as its N (tails rounded to 16 tokens), or "
+                         "256 x 256 tiles on CTA pairs")
     ap.add_argument("--drop-policy", default="token", choices=sorted(DROP_POLICIES),
                     help="which picks an overflowing expert keeps: token order, pick rank "
                          "first, or highest selection score")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)   # at least three untimed warm-up steps
     if args.impl != "reference":
-        M.set_ffn_cta_pairs(args.ffn_kernel == "pairs")
+        M.set_ffn_kernel(args.ffn_kernel)
     if args.impl == "reference":
         run_reference(args)
     elif args.microbatches > 1:
         run_microbatch(args)
+    elif args.ep:
+        run_ep_group(args)
     elif args.ep_emulate:
         run_ep_emulated(args)
     else:

@@ -532,15 +532,27 @@ const char* moe_status_string(moe_status_t status);
 void moe_set_wait_limit_ns(uint64_t ns);
 
 /* Which kernel runs the bf16 expert FFN of moe_expert_ffn / moe_layer_forward (permuted
- * rows, combine separate), for the whole process; a choice of schedule, not of results
- * (both compute the same sums in the same K order and give bitwise the same h and y_perm).
- * on == 0 (the default): one CTA per 128 x 256 output tile.  on != 0: each 256 x 256 tile
- * is computed by a pair of CTAs on the two SMs of a TPC sharing one tensor-core MMA (a
- * cluster of two), each CTA loading half of each operand -- a third fewer bytes from L2
- * per FLOP, measured slower on the layer's shapes; if no cluster of two fits on the
- * device, the single-CTA kernel runs.  The gathered-A and fused-combine forms and the
- * expert-parallel FFN always use the single-CTA kernel. */
-void moe_set_ffn_cta_pairs(int on);
+ * rows, combine separate), for the whole process.  A choice of schedule, not of results:
+ * all three compute each output as the same fp32 sum in the same K order and give bitwise
+ * the same h and y_perm.
+ *   MOE_FFN_TOKEN_MAJOR (the default): one CTA per 128-token x 256-column tile (a bucket's
+ *     last tile of at most 64 tokens runs at M = 64).
+ *   MOE_FFN_TOKEN_N: the MMA's M = 128 rows are weight rows (output features), its N is up
+ *     to 256 of a bucket's tokens, and a bucket's last tile takes its remaining tokens
+ *     rounded up to 16 -- a ragged bucket wastes at most 15 rows of tensor work.
+ *   MOE_FFN_CTA_PAIRS: each 256-token x 256-column tile on a pair of CTAs on the two SMs of
+ *     a TPC sharing one tensor-core MMA (a cluster of two), each CTA loading half of each
+ *     operand: a third fewer bytes from L2 per FLOP; if no cluster of two fits on the
+ *     device, MOE_FFN_TOKEN_MAJOR runs.
+ * The expert-parallel FFN (moe_ep_expert_ffn) follows the same setting; the gathered-A and
+ * fused-combine forms always run the token-major kernel.  Returns MOE_ERR_INVALID_ARG for
+ * an unknown kind. */
+typedef enum {
+  MOE_FFN_TOKEN_MAJOR = 0,
+  MOE_FFN_CTA_PAIRS = 1,
+  MOE_FFN_TOKEN_N = 2
+} moe_ffn_kernel_t;
+moe_status_t moe_set_ffn_kernel(moe_ffn_kernel_t kind);
 
 /* Self-test of the bounded wait: one block waits on an on-chip barrier that nothing
  * completes, with the current limit, records MOE_ERR_TIMEOUT in the workspace status

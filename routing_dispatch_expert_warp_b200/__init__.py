@@ -28,7 +28,7 @@ __all__ = ["MoEError", "make_config", "workspace_size", "capacity", "max_rows",
            "moe_expert_ffn", "moe_expert_ffn_gather", "moe_expert_ffn_combine", "moe_combine",
            "moe_load_stats", "moe_load_stats_merge", "moe_layer_forward",
            "moe_check_device_error",
-           "moe_selftest_bounded_wait", "set_wait_limit_ns", "set_ffn_cta_pairs", "kernel_launch_count",
+           "moe_selftest_bounded_wait", "set_wait_limit_ns", "set_ffn_kernel", "kernel_launch_count",
            "LayerBuffers", "MoELayer", "HostPipeline"]
 
 
@@ -95,9 +95,14 @@ def set_wait_limit_ns(ns: int) -> None:
     _lib().moe_set_wait_limit_ns(ns)
 
 
-def set_ffn_cta_pairs(on: bool) -> None:
-    """The plain expert FFN on CTA pairs (True) or on single CTAs (False, the default)."""
-    _lib().moe_set_ffn_cta_pairs(1 if on else 0)
+FFN_TOKEN_MAJOR, FFN_CTA_PAIRS, FFN_TOKEN_N = 0, 1, 2
+FFN_KERNELS = {"token_n": FFN_TOKEN_N, "token_major": FFN_TOKEN_MAJOR, "pairs": FFN_CTA_PAIRS}
+
+
+def set_ffn_kernel(kind) -> None:
+    """Which kernel runs the plain expert FFN, process-wide: FFN_TOKEN_MAJOR (the default),
+    FFN_TOKEN_N or FFN_CTA_PAIRS, or their names in FFN_KERNELS."""
+    check(_lib().moe_set_ffn_kernel(FFN_KERNELS.get(kind, kind)))
 
 
 # ------------------------------------------------------------------ stages

@@ -120,7 +120,7 @@ PROTOTYPES = {
     "moe_last_error": (ctypes.c_char_p, []),
     "moe_status_string": (ctypes.c_char_p, [c_i32]),
     "moe_set_wait_limit_ns": (None, [ctypes.c_uint64]),
-    "moe_set_ffn_cta_pairs": (None, [c_i32]),
+    "moe_set_ffn_kernel": (c_i32, [c_i32]),
     "moe_selftest_bounded_wait": (c_i32, [c_vp, c_sz, c_vp]),
     "moe_ep_recv_rows_bound": (c_i64, [P(MoeConfig), P(MoeEpConfig)]),
     "moe_ep_put_counts": (c_i32, [P(MoeConfig), P(MoeEpConfig), c_vp, c_vp, c_vp]),

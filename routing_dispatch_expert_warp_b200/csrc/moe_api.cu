@@ -233,7 +233,12 @@ const char* moe_status_string(moe_status_t st) {
 
 void moe_set_wait_limit_ns(uint64_t ns) { g_wait_ns.store(ns == 0 ? 2000000000ull : ns); }
 
-void moe_set_ffn_cta_pairs(int on) { set_ffn_cta_pairs(on); }
+moe_status_t moe_set_ffn_kernel(moe_ffn_kernel_t kind) {
+  MOE_REQUIRE(kind == MOE_FFN_TOKEN_MAJOR || kind == MOE_FFN_CTA_PAIRS || kind == MOE_FFN_TOKEN_N,
+              "moe_set_ffn_kernel: unknown kernel %d", static_cast<int>(kind));
+  set_ffn_kernel(kind);
+  return MOE_OK;
+}
 
 
 moe_status_t moe_workspace_size(const moe_config_t* cfg, size_t* bytes) {
@@ -283,8 +288,9 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   if (router_uses_tensor_cores(s)) {
     const char* why = "";
-    cudaError_t err = launch_router_tc(s, x, w_router, logit_bias, bias_row_stride, z, topk_idx,
-                                       topk_w, static_cast<uint8_t*>(ws) + lay.router_tc,
+    cudaError_t err = launch_router_tc(s, x, w_router, logit_bias, bias_row_stride, logits, z,
+                                       topk_idx, topk_w,
+                                       static_cast<uint8_t*>(ws) + lay.router_tc,
                                        ws_status(ws, lay), g_wait_ns.load(), strm, &why);
     if (err != cudaSuccess) {
       if (why[0]) return fail(MOE_ERR_CUDA, "moe_route: %s", why);

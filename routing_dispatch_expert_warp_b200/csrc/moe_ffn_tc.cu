@@ -38,6 +38,7 @@
 #include <mutex>
 
 #include "moe_internal.h"
+#include "moe_keys.cuh"
 
 namespace moe {
 namespace {
@@ -85,6 +86,16 @@ struct TcParams {
   __nv_bfloat16* comb_out;    // [T, N_out]
   int k;
   int32_t T;
+  // MODE_ROUTER: the A rows (x) are a_k wide; the K = 2 a_k reduction takes each 64-wide
+  // chunk of x against the hi and then the lo half of the split router weight ([E, 2 a_k]:
+  // hi in columns [0, a_k), lo in [a_k, 2 a_k)); out_f32 may be nullptr when the top-k is
+  // fused and the caller wants no logits.
+  int a_k;
+  int fuse_topk;              // 1: the epilogue selects the top-k and writes the gate weights
+  int gating;                 // MOE_GATE_SOFTMAX / MOE_GATE_SIGMOID
+  const float* sel_bias;      // bias added to the selection score only (or nullptr)
+  int32_t* route_idx;         // [T, k] picks (fused top-k)
+  float* route_w;             // [T, k] gate weights (fused top-k)
 };
 
 // The last of a token's kept picks to finish column block nb has its warp sum the token's
@@ -155,7 +166,7 @@ template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
     const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
     const __grid_constant__ CUtensorMap tm_b1, const TcParams p) {
-  constexpr bool GATED = MODE != MODE_DOWN;  // B tile = two stacked 128-row halves
+  constexpr bool GATED = MODE == MODE_SWIGLU;  // B tile = two stacked 128-row halves
   constexpr int BN_OUT = GATED ? 128 : 256;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[STAGES];
@@ -248,12 +259,16 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
           mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
           armed |= 1u << s;
           armed_parity = (armed_parity & ~(1u << s)) | (ph << s);
-          tma_load_2d(sa, &tm_a, &full_bar[s], kb * BK, row0);
+          // the router takes each 64-wide chunk of its x rows twice in a row, against the hi
+          // and then the lo half of the split weight (the second read hits L2)
+          const int a_col = MODE == MODE_ROUTER ? (kb >> 1) * BK : kb * BK;
+          const int b_col = MODE == MODE_ROUTER ? (kb & 1) * p.a_k + (kb >> 1) * BK : kb * BK;
+          tma_load_2d(sa, &tm_a, &full_bar[s], a_col, row0);
           if (GATED) {
-            tma_load_3d(sb, &tm_b0, &full_bar[s], kb * BK, nb * 128, e);
-            tma_load_3d(sb + B_BYTES / 2, &tm_b1, &full_bar[s], kb * BK, nb * 128, e);
+            tma_load_3d(sb, &tm_b0, &full_bar[s], b_col, nb * 128, e);
+            tma_load_3d(sb + B_BYTES / 2, &tm_b1, &full_bar[s], b_col, nb * 128, e);
           } else {
-            tma_load_3d(sb, &tm_b0, &full_bar[s], kb * BK, nb * 256, e);
+            tma_load_3d(sb, &tm_b0, &full_bar[s], b_col, nb * 256, e);
           }
           if (++s == STAGES) {
             s = 0;
@@ -429,28 +444,99 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
           p.out + static_cast<int64_t>(row0 + rt) * p.N_out + static_cast<int64_t>(nb) * BN_OUT;
       const int cols_left = p.N_out - nb * BN_OUT;
       if (MODE == MODE_ROUTER) {
+        // one token per thread, all experts of the tile (up to 256) in its accumulator row
         const int64_t grow = static_cast<int64_t>(row0 + rt);
-        float* zrow = p.out_f32 + grow * p.N_out + static_cast<int64_t>(nb) * BN_OUT;
-        const float* brow =
-            p.bias != nullptr ? p.bias + grow * p.bias_stride + static_cast<int64_t>(nb) * BN_OUT
-                              : nullptr;
+        float* zrow = p.out_f32 != nullptr ? p.out_f32 + grow * p.N_out : nullptr;
+        const float* brow = p.bias != nullptr ? p.bias + grow * p.bias_stride : nullptr;
+        const float* srow = p.sel_bias != nullptr ? p.sel_bias + grow * p.bias_stride : nullptr;
+        // the k best (key, expert, logit) so far, best first; equal keys keep the expert seen
+        // first, i.e. the lower index
+        uint32_t tk[MOE_MAX_TOPK];
+        int ti[MOE_MAX_TOPK];
+        float tz[MOE_MAX_TOPK];
+#pragma unroll
+        for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+          tk[j] = 0u;
+          ti[j] = 0;
+          tz[j] = 0.f;
+        }
+        uint32_t thr = 0u;  // key of the k-th best so far
 #pragma unroll 1
         for (int c = 0; c < BN_OUT / 32; ++c) {
-          uint32_t hi[32], lo[32];
-          tmem_ld32(taddr + c * 32, hi);
-          tmem_ld32(taddr + 128 + c * 32, lo);
+          uint32_t v[32];
+          tmem_ld32(taddr + c * 32, v);
           tmem_ld_wait();
-          if (row_ok) {
+          if (row_ok && c * 32 < cols_left) {
+            float z[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const int col = c * 32 + i;
-              if (col < cols_left) {
-                float z = __uint_as_float(hi[i]) + __uint_as_float(lo[i]);
-                if (brow != nullptr) z += brow[col];
-                zrow[col] = z;
+              z[i] = __uint_as_float(v[i]);
+              if (brow != nullptr && col < cols_left) z[i] += brow[col];
+            }
+            if (zrow != nullptr) {
+              if (c * 32 + 32 <= cols_left && (p.N_out & 3) == 0) {
+                float4* dst = reinterpret_cast<float4*>(zrow + c * 32);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                  dst[i] = make_float4(z[4 * i], z[4 * i + 1], z[4 * i + 2], z[4 * i + 3]);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                  if (c * 32 + i < cols_left) zrow[c * 32 + i] = z[i];
+              }
+            }
+            if (p.fuse_topk) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int col = c * 32 + i;
+                if (col >= cols_left) continue;
+                const uint32_t key = order_key(srow != nullptr ? z[i] + srow[col] : z[i]);
+                if (key <= thr) continue;
+#pragma unroll
+                for (int j = MOE_MAX_TOPK - 1; j > 0; --j) {
+                  if (key > tk[j - 1]) {
+                    tk[j] = tk[j - 1];
+                    ti[j] = ti[j - 1];
+                    tz[j] = tz[j - 1];
+                  } else if (key > tk[j]) {
+                    tk[j] = key;
+                    ti[j] = col;
+                    tz[j] = z[i];
+                  }
+                }
+                if (key > tk[0]) {
+                  tk[0] = key;
+                  ti[0] = col;
+                  tz[0] = z[i];
+                }
+#pragma unroll
+                for (int j = 0; j < MOE_MAX_TOPK; ++j)
+                  if (j == p.k - 1) thr = tk[j];
               }
             }
           }
+        }
+        if (p.fuse_topk && row_ok) {
+          // gate weights over the k picks, the normaliser summed in pick order
+          float w[MOE_MAX_TOPK];
+          float m = tz[0];
+#pragma unroll
+          for (int j = 1; j < MOE_MAX_TOPK; ++j)
+            if (j < p.k) m = fmaxf(m, tz[j]);
+          float ssum = 0.f;
+#pragma unroll
+          for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+            w[j] = p.gating == MOE_GATE_SOFTMAX ? expf(tz[j] - m) : 1.0f / (1.0f + expf(-tz[j]));
+            if (j < p.k) ssum += w[j];
+          }
+          const float inv = 1.0f / ssum;
+#pragma unroll
+          for (int j = 0; j < MOE_MAX_TOPK; ++j)
+            if (j < p.k) {
+              p.route_idx[grow * p.k + j] = ti[j];
+              p.route_w[grow * p.k + j] = w[j] * inv;
+            }
         }
       } else if (GATED) {
 #pragma unroll 1
@@ -803,13 +889,323 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_pair_kernel(
   }
 }
 
-// W_r [d, E] fp32 -> hi, lo [E, d] bf16 with hi = bf16(W), lo = bf16(W - hi), so that
-// x . W = x . hi + x . lo up to the rounding of lo (a relative 2^-17 of each weight).
-// 32 x 32 tiles transposed through shared memory.  Block (0, 0) also writes the one-bucket
-// table {start 0, count T} the grouped GEMM reads.
+// ------------------------------------------------------------------ token-N variant
+// The same grouped GEMM with the operands' roles swapped: the MMA's M = 128 rows are weight
+// rows (output features) and its N is the bucket's tokens, up to 256 per tile and, in a
+// bucket's last tile, its remaining tokens rounded up to 16 -- so a ragged bucket wastes at
+// most 15 rows of tensor work instead of up to 127 with 128-row token tiles.  Per 64-deep
+// K step a tile loads 16 KB of weights and up to 32 KB of token rows (128-row boxes), the
+// bytes per FLOP of the 128 x 256 token-major tile.
+//   gate/up: a tile is 64 features: A rows 0-63 are those rows of W_g, rows 64-127 the
+//     same rows of W_u, so TMEM lane quarters 0-1 hold gate and 2-3 hold up.  The epilogue
+//     warp of quarter 2 + i hands its up values, 32 tokens at a time, to the warp of
+//     quarter i through a double-buffered shared buffer (mbarrier handshake, bounded
+//     waits); that warp forms silu(gate) * up.
+//   down: a tile is 128 features of y (rows of W_d).
+// The storing warp writes each 32-token chunk (one feature per lane) transposed into a
+// padded per-warp shared buffer and stores each token's 32 features contiguously.  Tiles:
+// (expert, feature block, 256-token block), token blocks innermost.
+constexpr int TN_TOK = 256;                              // tokens per tile (max MMA N)
+constexpr int TN_BOX = 128;                              // token rows per TMA box
+constexpr int TN_STAGES = 4;
+constexpr int TN_A_BYTES = 128 * BK * 2;                 // 16 KB of weight rows
+constexpr int TN_B_BYTES = TN_TOK * BK * 2;              // up to 32 KB of token rows
+constexpr int TN_STAGE_BYTES = TN_A_BYTES + TN_B_BYTES;  // 48 KB
+constexpr int TN_XPOSE_STRIDE = 80;                      // bytes per token row in the buffer
+constexpr int TN_XPOSE_BYTES = 32 * TN_XPOSE_STRIDE;     // per storing warp
+constexpr int TN_XCHG_BYTES = 32 * 32 * 4;               // one chunk of up values (fp32)
+// transposition buffers for the 4 storing warps of down (2 of gate/up), then gate/up's two
+// warp pairs' double-buffered exchange
+constexpr int TN_EPI_BYTES = 4 * TN_XPOSE_BYTES + 2 * 2 * TN_XCHG_BYTES;
+constexpr int TN_DYN_SMEM = TN_STAGES * TN_STAGE_BYTES + TN_EPI_BYTES + 1024;
+
+template <int MODE>
+__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tokn_kernel(
+    const __grid_constant__ CUtensorMap tm_tok, const __grid_constant__ CUtensorMap tm_w0,
+    const __grid_constant__ CUtensorMap tm_w1, const TcParams p) {
+  static_assert(MODE == MODE_DOWN || MODE == MODE_SWIGLU, "expert FFN launches only");
+  constexpr bool GATED = MODE == MODE_SWIGLU;
+  constexpr int FB = GATED ? 64 : 128;  // output features per tile
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[TN_STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[TN_STAGES];
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ __align__(8) uint64_t xfull_bar[2][2];    // [warp pair][buffer]: up values written
+  __shared__ __align__(8) uint64_t xempty_bar[2][2];   // [warp pair][buffer]: up values read
+  __shared__ uint32_t tmem_base_s;
+  __shared__ volatile int abort_s;
+  __shared__ int tile_base[MOE_MAX_EXPERTS + 1];
+  __shared__ int tblocks[MOE_MAX_EXPERTS];
+
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* epi = smem + TN_STAGES * TN_STAGE_BYTES;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (warp == 0) {  // tile table: 256-token blocks per expert and their prefix (x feature blocks)
+    int carry = 0;
+    for (int e0 = 0; e0 < p.E; e0 += 32) {
+      const int e = e0 + lane;
+      const int tb = e < p.E ? (p.seg_count[e] + TN_TOK - 1) / TN_TOK : 0;
+      int v = tb;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += o;
+      }
+      if (e < p.E) {
+        tblocks[e] = tb;
+        tile_base[e] = (carry + v - tb) * p.n_blocks;
+      }
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) {
+      tile_base[p.E] = carry * p.n_blocks;
+      prefetch_tensormap(&tm_tok);
+      prefetch_tensormap(&tm_w0);
+      if (GATED) prefetch_tensormap(&tm_w1);
+    }
+  } else if (warp == 1) {
+    tmem_alloc(&tmem_base_s, TMEM_COLS);
+    tmem_relinquish();
+  } else if (threadIdx.x == 64) {
+    for (int s = 0; s < TN_STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 128);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&xfull_bar[a][b], 1);
+        mbar_init(&xempty_bar[a][b], 1);
+      }
+    }
+    mbar_init(&drain_bar, 1);
+    abort_s = 0;
+    fence_barrier_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem_base = tmem_base_s;
+  const int total_tiles = tile_base[p.E];
+  const int KB = p.K / BK;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    int s = 0;
+    uint32_t ph = 0;
+    uint32_t armed = 0, armed_parity = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      int e, tb, fb;
+      decode_tile(tile, tile_base, tblocks, p.E, p.n_blocks, 0, e, tb, fb);
+      const int tok0 = p.seg_start[e] + tb * TN_TOK;
+      const int n_valid = min(TN_TOK, p.seg_count[e] - tb * TN_TOK);
+      const int nbox = (n_valid + TN_BOX - 1) / TN_BOX;
+      const uint32_t bytes = TN_A_BYTES + static_cast<uint32_t>(nbox) * (TN_BOX * BK * 2);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&empty_bar[s], ph ^ 1u, p.wait_ns, &abort_s)) {
+          if (!abort_s)
+            record_error(p.status, DEV_TIMEOUT, 40, static_cast<unsigned long long>(tile));
+          abort_s = 1;
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + s * TN_STAGE_BYTES;
+        uint8_t* sb = sa + TN_A_BYTES;
+        mbar_arrive_expect_tx(&full_bar[s], bytes);
+        armed |= 1u << s;
+        armed_parity = (armed_parity & ~(1u << s)) | (ph << s);
+        if (GATED) {
+          tma_load_3d(sa, &tm_w0, &full_bar[s], kb * BK, fb * FB, e);
+          tma_load_3d(sa + TN_A_BYTES / 2, &tm_w1, &full_bar[s], kb * BK, fb * FB, e);
+        } else {
+          tma_load_3d(sa, &tm_w0, &full_bar[s], kb * BK, fb * FB, e);
+        }
+        for (int j = 0; j < nbox; ++j)
+          tma_load_2d(sb + j * (TN_BOX * BK * 2), &tm_tok, &full_bar[s], kb * BK,
+                      tok0 + j * TN_BOX);
+        if (++s == TN_STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+    }
+    for (int q = 0; q < TN_STAGES; ++q)
+      if ((armed >> q) & 1u)
+        mbar_wait(&full_bar[q], (armed_parity >> q) & 1u, p.wait_ns, nullptr);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------------- MMA issuer
+    int s = 0;
+    uint32_t ph = 0;
+    int acc = 0;
+    uint32_t aph = 0;
+    bool ok = true;
+    bool issued = false;
+    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      int e, tb, fb;
+      decode_tile(tile, tile_base, tblocks, p.E, p.n_blocks, 0, e, tb, fb);
+      const int n_valid = min(TN_TOK, p.seg_count[e] - tb * TN_TOK);
+      const uint32_t idesc = idesc_bf16_f32(128, (n_valid + 15) & ~15);
+      if (!mbar_wait(&tempty_bar[acc], aph ^ 1u, p.wait_ns, &abort_s)) {
+        if (!abort_s) record_error(p.status, DEV_TIMEOUT, 41, static_cast<unsigned long long>(tile));
+        abort_s = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_COLS);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!mbar_wait(&full_bar[s], ph, p.wait_ns, &abort_s)) {
+          if (!abort_s) record_error(p.status, DEV_TIMEOUT, 42, static_cast<unsigned long long>(tile));
+          abort_s = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = smem_addr(smem + s * TN_STAGE_BYTES);
+        const uint32_t b_addr = a_addr + TN_A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          tc_mma_f16(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
+                     sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+        issued = true;
+        tc_commit(&empty_bar[s]);
+        if (++s == TN_STAGES) {
+          s = 0;
+          ph ^= 1u;
+        }
+      }
+      if (!ok) break;
+      tc_commit(&tfull_bar[acc]);
+      acc ^= 1;
+      if (acc == 0) aph ^= 1u;
+    }
+    if (!ok && issued) {
+      tc_commit(&drain_bar);
+      mbar_wait(&drain_bar, 0, p.wait_ns, nullptr);
+    }
+  } else if (warp >= 2) {
+    // ---------------------------------------------------------------- epilogue
+    const int q = warp & 3;   // TMEM lane quarter this warp may access
+    // gate/up: quarters 2-3 (warps 2-3) hand their up values to quarters 0-1 (warps 4-5)
+    const bool sender = GATED && q >= 2;
+    const int pair = q & 1;
+    uint8_t* xb = epi + (GATED ? pair : warp - 2) * TN_XPOSE_BYTES;
+    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(xb);
+    float* xchg = reinterpret_cast<float*>(epi + 4 * TN_XPOSE_BYTES + pair * 2 * TN_XCHG_BYTES);
+    const int warp_feat0 = GATED ? 32 * pair : 32 * q;   // first feature of this warp's lanes
+    uint32_t nchunk = 0;     // chunks exchanged so far (buffer = nchunk & 1)
+    int acc = 0;
+    uint32_t aph = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      int e, tb, fb;
+      decode_tile(tile, tile_base, tblocks, p.E, p.n_blocks, 0, e, tb, fb);
+      const int tok0 = p.seg_start[e] + tb * TN_TOK;
+      const int n_valid = min(TN_TOK, p.seg_count[e] - tb * TN_TOK);
+      int got = 1;
+      if (lane == 0) got = mbar_wait(&tfull_bar[acc], aph, p.wait_ns, &abort_s) ? 1 : 0;
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) {
+        if (lane == 0 && !abort_s) record_error(p.status, DEV_TIMEOUT, 43, static_cast<unsigned long long>(tile));
+        abort_s = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                             static_cast<uint32_t>(acc * ACC_COLS);
+      const int col0 = fb * FB + warp_feat0;   // first output feature this warp stores
+      const bool feats_ok = col0 < p.N_out;    // N_out is a multiple of 64: all 32 or none
+      const int chunks = (n_valid + 31) >> 5;
+#pragma unroll 1
+      for (int c = 0; c < chunks; ++c, ++nchunk) {
+        uint32_t v[32];
+        tmem_ld32(taddr + c * 32, v);
+        tmem_ld_wait();
+        const uint32_t buf = nchunk & 1u, use = (nchunk >> 1) & 1u;
+        float* xc = xchg + buf * (32 * 32);
+        if (sender) {
+          // wait until the partner has read this buffer's previous chunk, then fill it
+          int w = 1;
+          if (lane == 0) w = mbar_wait(&xempty_bar[pair][buf], use ^ 1u, p.wait_ns, &abort_s) ? 1 : 0;
+          w = __shfl_sync(0xffffffffu, w, 0);
+          if (!w) {
+            if (lane == 0 && !abort_s) record_error(p.status, DEV_TIMEOUT, 44, static_cast<unsigned long long>(tile));
+            abort_s = 1;
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) xc[j * 32 + lane] = __uint_as_float(v[j]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&xfull_bar[pair][buf]);
+          continue;
+        }
+        if (GATED) {
+          int w = 1;
+          if (lane == 0) w = mbar_wait(&xfull_bar[pair][buf], use, p.wait_ns, &abort_s) ? 1 : 0;
+          w = __shfl_sync(0xffffffffu, w, 0);
+          if (!w) {
+            if (lane == 0 && !abort_s) record_error(p.status, DEV_TIMEOUT, 45, static_cast<unsigned long long>(tile));
+            abort_s = 1;
+            ok = false;
+            break;
+          }
+          float u[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) u[j] = xc[j * 32 + lane];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&xempty_bar[pair][buf]);
+          __syncwarp();  // the previous chunk's reads of the transposition buffer are done
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            xs[j * (TN_XPOSE_STRIDE / 2) + lane] =
+                __float2bfloat16_rn(silu_mul(__uint_as_float(v[j]), u[j]));
+        } else {
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            xs[j * (TN_XPOSE_STRIDE / 2) + lane] = __float2bfloat16_rn(__uint_as_float(v[j]));
+        }
+        __syncwarp();
+        const int t = c * 32 + lane;   // this lane stores token t's 32 features
+        if (feats_ok && t < n_valid) {
+          const uint4* src = reinterpret_cast<const uint4*>(xb + lane * TN_XPOSE_STRIDE);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<int64_t>(tok0 + t) * p.N_out +
+                                                col0);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = src[i];
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty_bar[acc]);
+      acc ^= 1;
+      if (acc == 0) aph ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// W_r [d, E] fp32 -> W' [E, 2d] bf16, row e = [hi(W[:, e]), lo(W[:, e])] with
+// hi = bf16(W), lo = bf16(W - hi), so that x . W = [x, x] . W' up to the rounding of lo (a
+// relative 2^-17 of each weight).  32 x 32 tiles transposed through shared memory.  Block
+// (0, 0) also writes the one-bucket table {start 0, count T} the grouped GEMM reads.
 __global__ void __launch_bounds__(256) split_router_weight_kernel(
-    const float* __restrict__ w, int d, int E, __nv_bfloat16* __restrict__ hi,
-    __nv_bfloat16* __restrict__ lo, int32_t* __restrict__ seg, int32_t T) {
+    const float* __restrict__ w, int d, int E, __nv_bfloat16* __restrict__ wsplit,
+    int32_t* __restrict__ seg, int32_t T) {
   __shared__ float tile[32][33];
   const int e0 = blockIdx.x * 32, i0 = blockIdx.y * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -824,8 +1220,8 @@ __global__ void __launch_bounds__(256) split_router_weight_kernel(
       const float v = tile[tx][r];
       const __nv_bfloat16 h = __float2bfloat16_rn(v);
       const __nv_bfloat16 l = __float2bfloat16_rn(v - __bfloat162float(h));
-      hi[static_cast<int64_t>(e) * d + i] = h;
-      lo[static_cast<int64_t>(e) * d + i] = l;
+      wsplit[static_cast<int64_t>(e) * 2 * d + i] = h;
+      wsplit[static_cast<int64_t>(e) * 2 * d + d + i] = l;
     }
   }
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
@@ -859,6 +1255,18 @@ bool make_map_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K * 2)};
   const cuuint32_t box[2] = {BK, BM};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [rows, K] bf16 row-major, box 128 rows x 64 columns, 128-byte swizzle (token-N tiles)
+bool make_map_tokens(CUtensorMap* m, const void* base, int64_t rows, int64_t K) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K * 2)};
+  const cuuint32_t box[2] = {BK, TN_BOX};
   const cuuint32_t estr[2] = {1, 1};
   return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -932,12 +1340,28 @@ cudaError_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb0, const CUt
   return cudaSuccess;
 }
 
-std::atomic<int> g_ffn_pairs{0};
+// One launch of the token-N kernel over at most `tiles` tiles, one CTA per SM.
+template <int MODE>
+cudaError_t launch_tokn(const CUtensorMap& tt, const CUtensorMap& tw0, const CUtensorMap& tw1,
+                        const TcParams& p, int64_t tiles, cudaStream_t st) {
+  cudaError_t err = cudaFuncSetAttribute(grouped_gemm_tokn_kernel<MODE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, TN_DYN_SMEM);
+  if (err != cudaSuccess) return err;
+  int64_t g = tiles;
+  if (g > sm_count()) g = sm_count();
+  if (g < 1) g = 1;
+  grouped_gemm_tokn_kernel<MODE><<<static_cast<unsigned>(g), THREADS, TN_DYN_SMEM, st>>>(tt, tw0,
+                                                                                         tw1, p);
+  note_launch();
+  return cudaGetLastError();
+}
+
+std::atomic<int> g_ffn_kernel{MOE_FFN_TOKEN_MAJOR};
 
 }  // namespace
 
-void set_ffn_cta_pairs(int on) { g_ffn_pairs.store(on != 0 ? 1 : 0); }
-int ffn_cta_pairs() { return g_ffn_pairs.load(); }
+void set_ffn_kernel(int kind) { g_ffn_kernel.store(kind); }
+int ffn_kernel() { return g_ffn_kernel.load(); }
 
 // Before a down launch with the combine fused in: zero the arrival counters and the output
 // rows of tokens none of whose picks was kept (no thread of the launch ever writes those).
@@ -988,7 +1412,39 @@ cudaError_t launch_ffn_tc(const Shape& s, const void* a, const int32_t* a_rows,
   const int64_t row_blocks_bound = (s.max_rows + BM - 1) / BM + s.E;
   const int sms = sm_count();
 
-  if (a_rows == nullptr && comb == nullptr && g_ffn_pairs.load() != 0) {
+  const int kind = g_ffn_kernel.load();
+  if (a_rows == nullptr && comb == nullptr && kind == MOE_FFN_TOKEN_N) {
+    // token-N kernel: weight maps with 64-row (W_g, W_u) and 128-row (W_d) boxes, token
+    // maps with 128-row boxes
+    CUtensorMap tx, tg64, tu64, th, td128;
+    if (!make_map_tokens(&tx, a, s.max_rows, s.d) || !make_map_weights(&tg64, wg, s.E, s.f, s.d, 64) ||
+        !make_map_weights(&tu64, wu, s.E, s.f, s.d, 64) || !make_map_tokens(&th, h, s.max_rows, s.f) ||
+        !make_map_weights(&td128, wd, s.E, s.d, s.f, 128)) {
+      *why = "tensor map encoding failed (pointer alignment or sizes)";
+      return cudaErrorInvalidValue;
+    }
+    const int64_t tok_blocks_bound = (s.max_rows + TN_TOK - 1) / TN_TOK + s.E;
+    TcParams q1 = {};
+    q1.seg_start = offsets;
+    q1.seg_count = kept;
+    q1.E = s.E;
+    q1.K = static_cast<int>(s.d);
+    q1.n_blocks = static_cast<int>((s.f + 63) / 64);
+    q1.N_out = static_cast<int>(s.f);
+    q1.out = static_cast<__nv_bfloat16*>(h);
+    q1.status = status;
+    q1.wait_ns = wait_ns;
+    err = launch_tokn<MODE_SWIGLU>(tx, tg64, tu64, q1, tok_blocks_bound * q1.n_blocks, st);
+    if (err != cudaSuccess) return err;
+    TcParams q2 = q1;
+    q2.K = static_cast<int>(s.f);
+    q2.n_blocks = static_cast<int>((s.d + 127) / 128);
+    q2.N_out = static_cast<int>(s.d);
+    q2.out = static_cast<__nv_bfloat16*>(y);
+    return launch_tokn<MODE_DOWN>(th, td128, td128, q2, tok_blocks_bound * q2.n_blocks, st);
+  }
+
+  if (a_rows == nullptr && comb == nullptr && kind == MOE_FFN_CTA_PAIRS) {
     // the CTA-pair kernel: B maps with 128-row boxes (each CTA loads half of the 256 rows)
     CUtensorMap td128;
     if (!make_map_weights(&td128, wd, s.E, s.d, s.f, 128)) {
@@ -1091,52 +1547,62 @@ size_t router_tc_workspace_bytes(const Shape& s) {
 
 cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_router,
                              const float* bias, int64_t bias_stride, float* logits,
-                             int32_t* topk_idx, float* topk_w, void* split_ws,
-                             DevStatus* status, uint64_t wait_ns, cudaStream_t st,
-                             const char** why) {
+                             float* logits_scratch, int32_t* topk_idx, float* topk_w,
+                             void* split_ws, DevStatus* status, uint64_t wait_ns,
+                             cudaStream_t st, const char** why) {
   if (encode_fn() == nullptr) {
     *why = "cuTensorMapEncodeTiled is not available from the driver";
     return cudaErrorNotSupported;
   }
   int32_t* seg = static_cast<int32_t*>(split_ws);
-  __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(split_ws) + 256);
-  __nv_bfloat16* lo = hi + static_cast<size_t>(s.E) * s.d;
+  __nv_bfloat16* wsplit = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(split_ws) + 256);
   dim3 sgrid((s.E + 31) / 32, static_cast<unsigned>((s.d + 31) / 32));
-  split_router_weight_kernel<<<sgrid, 256, 0, st>>>(w_router, static_cast<int>(s.d), s.E, hi, lo,
+  split_router_weight_kernel<<<sgrid, 256, 0, st>>>(w_router, static_cast<int>(s.d), s.E, wsplit,
                                                     seg, static_cast<int32_t>(s.T));
   note_launch();
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  CUtensorMap ta, th, tl;
-  if (!make_map_rows(&ta, x, s.T, s.d) || !make_map_weights(&th, hi, 1, s.E, s.d, 128) ||
-      !make_map_weights(&tl, lo, 1, s.E, s.d, 128)) {
+  // all E <= 256 experts in one 256-column accumulator: K = 2 d (hi half, then lo half)
+  CUtensorMap ta, tw;
+  if (!make_map_rows(&ta, x, s.T, s.d) || !make_map_weights(&tw, wsplit, 1, s.E, 2 * s.d, 256)) {
     *why = "tensor map encoding failed for the router";
     return cudaErrorInvalidValue;
   }
   err = cudaFuncSetAttribute(grouped_gemm_tc_kernel<MODE_ROUTER>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, DYN_SMEM);
   if (err != cudaSuccess) return err;
+  const bool sel_only = s.bias_mode == MOE_BIAS_SELECTION_ONLY;
+  // the top-k rides in the epilogue unless the picks are limited to groups
+  const bool fuse = s.n_groups <= 1;
   TcParams p = {};
   p.seg_start = seg;
   p.seg_count = seg + 1;
   p.E = 1;
-  p.K = static_cast<int>(s.d);
-  p.n_blocks = (s.E + 127) / 128;
+  p.K = static_cast<int>(2 * s.d);
+  p.a_k = static_cast<int>(s.d);
+  p.n_blocks = 1;
   p.N_out = s.E;
   p.mb_outer = 1;
-  p.out_f32 = logits;
-  // logits carry the bias unless it is for selection only (then the top-k adds it)
-  p.bias = s.bias_mode == MOE_BIAS_SELECTION_ONLY ? nullptr : bias;
+  p.out_f32 = fuse ? logits : (logits != nullptr ? logits : logits_scratch);
+  // logits carry the bias unless it is for selection only (then only the keys add it)
+  p.bias = sel_only ? nullptr : bias;
+  p.sel_bias = sel_only ? bias : nullptr;
   p.bias_stride = bias_stride;
+  p.fuse_topk = fuse ? 1 : 0;
+  p.k = s.k;
+  p.gating = s.gating;
+  p.route_idx = topk_idx;
+  p.route_w = topk_w;
   p.status = status;
   p.wait_ns = wait_ns;
-  int64_t g = ((s.T + BM - 1) / BM) * p.n_blocks;
+  int64_t g = (s.T + BM - 1) / BM;
   if (g > sm_count()) g = sm_count();
   grouped_gemm_tc_kernel<MODE_ROUTER><<<static_cast<unsigned>(g), THREADS, DYN_SMEM, st>>>(
-      ta, th, tl, p);
+      ta, tw, tw, p);
   note_launch();
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  return launch_topk_from_logits(s, logits, bias, bias_stride, topk_idx, topk_w, st);
+  if (fuse) return cudaSuccess;
+  return launch_topk_from_logits(s, p.out_f32, bias, bias_stride, topk_idx, topk_w, st);
 }
 
 }  // namespace moe

@@ -66,11 +66,13 @@ cudaError_t launch_router(const Shape& s, const void* x, const float* w_router,
                           int32_t* topk_idx, float* topk_w, float* partials, cudaStream_t st);
 // Router on tensor cores (bf16 layers, E > 32): W_r split into two bf16 terms.
 bool router_uses_tensor_cores(const Shape& s);
+// logits: the caller's [T, E] buffer or nullptr (then, with the top-k fused into the GEMM,
+// no logits are written; without it they go to logits_scratch).
 cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_router,
                              const float* bias, int64_t bias_stride, float* logits,
-                             int32_t* topk_idx, float* topk_w, void* split_ws,
-                             DevStatus* status, uint64_t wait_ns, cudaStream_t st,
-                             const char** why);
+                             float* logits_scratch, int32_t* topk_idx, float* topk_w,
+                             void* split_ws, DevStatus* status, uint64_t wait_ns,
+                             cudaStream_t st, const char** why);
 size_t router_tc_workspace_bytes(const Shape& s);
 cudaError_t launch_topk_from_logits(const Shape& s, const float* logits, const float* bias,
                                     int64_t bias_stride, int32_t* topk_idx, float* topk_w,
@@ -148,10 +150,10 @@ cudaError_t launch_ep_stats(const Shape& s, const int32_t* mat, const int32_t* e
                             int world, int ranks_per_node, moe_ep_stats_t* out,
                             cudaStream_t st);
 
-// Expert FFN of the plain (permuted-copy) path on CTA pairs (1) or on single CTAs (0, the
-// default); process-wide.
-void set_ffn_cta_pairs(int on);
-int ffn_cta_pairs();
+// Which kernel runs the expert FFN of the plain (permuted-copy) path, process-wide: a
+// moe_ffn_kernel_t value (include/moe.h).
+void set_ffn_kernel(int kind);
+int ffn_kernel();
 
 // Process-wide count of this library's kernel launches (every launch site calls it once).
 void note_launch();

@@ -96,22 +96,37 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
       __syncthreads();
     }
   }
-  // drops per pick rank and per token (thread per token, counters in registers)
+  // drops per pick rank and per token (thread per token, counters in registers); four
+  // tokens' picks are loaded before any is counted, so each thread keeps 4 k loads in flight
   int rank_local[MOE_MAX_TOPK];
 #pragma unroll
   for (int j = 0; j < MOE_MAX_TOPK; ++j) rank_local[j] = 0;
   int td = 0, tf = 0;
-  for (int64_t t = tid; assign_row != nullptr && t < T; t += blockDim.x) {
-    int nd = 0;
+  constexpr int kTokUnroll = 4;
+  const int64_t step = static_cast<int64_t>(blockDim.x);
+  for (int64_t t0 = tid; assign_row != nullptr && t0 < T; t0 += step * kTokUnroll) {
+    int32_t a[kTokUnroll][MOE_MAX_TOPK];
 #pragma unroll
-    for (int j = 0; j < MOE_MAX_TOPK; ++j) {
-      if (j < k && __ldg(assign_row + t * k + j) < 0) {
-        ++rank_local[j];
-        ++nd;
-      }
+    for (int u = 0; u < kTokUnroll; ++u) {
+      const int64_t t = t0 + u * step;
+#pragma unroll
+      for (int j = 0; j < MOE_MAX_TOPK; ++j)
+        a[u][j] = (j < k && t < T) ? __ldg(assign_row + t * k + j) : 0;
     }
-    td += nd > 0;
-    tf += nd == k;
+#pragma unroll
+    for (int u = 0; u < kTokUnroll; ++u) {
+      if (t0 + u * step >= T) break;
+      int nd = 0;
+#pragma unroll
+      for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+        if (j < k && a[u][j] < 0) {
+          ++rank_local[j];
+          ++nd;
+        }
+      }
+      td += nd > 0;
+      tf += nd == k;
+    }
   }
 #pragma unroll
   for (int j = 0; j < MOE_MAX_TOPK; ++j) {

@@ -325,9 +325,10 @@ class EpGroup:
         self._opened = ex["opened"]
         self.tables = {name: _table(ptrs, self.device) for name, ptrs in ex["tables"].items()}
 
-    def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
+    def forward(self, x: torch.Tensor, stream=None,
+                on_step: Optional[Callable[[str], None]] = None) -> torch.Tensor:
         run_schedule([self.me], [x], self.tables,
-                     lambda: self.transport.barrier(self.group, self.device), stream)
+                     lambda: self.transport.barrier(self.group, self.device), stream, on_step)
         return self.me.out
 
     def close(self) -> None:

@@ -119,3 +119,54 @@ def test_peer_tables_and_barrier_order(world):
         last_a = max(t for s in a for t in stamps[s])
         first_b = min(t for s in b for t in stamps[s])
         assert last_a <= first_b, (a, b)
+
+
+def _inputs_worker(rank, world, port, q):
+    import torch
+    import bench
+    from routing_dispatch_expert_warp_b200 import workload as W
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        out = {}
+        for name, shape in (("zipf", W.reduced(W.DSV3_PREFILL_ZIPF, 48, 64, 32, E=16)),
+                            ("chunks", W.reduced(W.MIXTRAL_8X22B_MIXED, 300, 64, 32,
+                                                 n_decode_tokens=4))):
+            inp = bench.ep_rank_inputs(shape, rank, world, "cpu")
+            same = all(torch.equal(inp[k][i], w)
+                       for i, e in enumerate(inp["experts"])
+                       for k, w in zip(("w_gate", "w_up", "w_down"), W.expert_weights(shape, e)))
+            out[name] = (inp["experts"], float(inp["x"].float().sum()),
+                         inp["w_router"].clone(), inp["logit_bias"].clone(), same)
+        dist.barrier()
+        q.put((rank, out))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_bench_ep_rank_inputs_on_two_gloo_ranks():
+    """bench.py --ep's per-rank inputs: the experts split in disjoint contiguous blocks that
+    cover all E, each rank's local weights those of the single-GPU layer, one router weight
+    and one per-expert bias for the layer, and each rank its own batch (and the per-token
+    bias drawn with it)."""
+    import torch
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_inputs_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = dict(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for name, E in (("zipf", 16), ("chunks", 8)):
+        a, b = out[0][name], out[1][name]
+        assert a[0] == list(range(E // 2)) and b[0] == list(range(E // 2, E))
+        assert a[1] != b[1]                                   # distinct batches
+        assert torch.equal(a[2], b[2])                        # one router weight
+        assert a[4] and b[4]                                  # the single-GPU layer's weights
+        if name == "zipf":
+            assert torch.equal(a[3], b[3]) and a[3].dim() == 1   # one per-expert bias
+        else:
+            assert a[3].dim() == 2 and not torch.equal(a[3], b[3])  # per-token, per batch

@@ -177,36 +177,38 @@ def _forced_buckets(counts, d, f, seed=5):
 @pytest.mark.parametrize("counts,d,f", [
     # 256-row pair tiles: tails of 1, 127, 128 (the second CTA of the pair has no rows),
     # 129, 255, whole tiles, 257, and an empty expert
-    ((1, 127, 128, 129, 255, 256, 257, 0, 511, 513), 256, 384),
+    ((1, 127, 128, 129, 255, 256, 257, 0, 511, 513, 15, 16, 17, 33), 256, 384),
     ((300, 0, 5, 700), 512, 256),          # d = 512 (two 256-column down blocks)
     ((64, 200, 384), 192, 320),            # d and d_ff not multiples of 256 / 128
 ])
-def test_ffn_cta_pairs_equal_single_ctas_and_oracle(counts, d, f):
-    """The expert FFN on CTA pairs (256 x 256 tiles, one MMA over two SMs) and on single
-    CTAs (128 x 256 tiles): both match the oracle, and they compute the same sums in the same
-    K order, so h and y_perm agree bitwise."""
+def test_ffn_kernels_equal_each_other_and_oracle(counts, d, f):
+    """The three expert FFN kernels -- token-N (weight rows as M, tails rounded to 16 tokens),
+    token-major (128 x 256 tiles) and CTA pairs (256 x 256 tiles, one MMA over two SMs) --
+    each match the oracle, and they compute the same sums in the same K order, so h and
+    y_perm agree bitwise."""
     shape, inp = _forced_buckets(counts, d, f)
     run = GpuRun(shape, inp)
     try:
-        M.set_ffn_cta_pairs(True)
+        M.set_ffn_kernel("token_n")
         st = run.all_stages()
         r = check_routing(run)
         assert tuple(int(c) for c in r["kept"]) == counts
         check_ffn_rows(run, r)
         check_layer_output(run, run.b.out, r)
+        check_stats(st, r)
         used = int(run.b.expert_offsets[-1])
         h1, y1 = run.b.h[:used].clone(), run.b.y_perm[:used].clone()
-        M.set_ffn_cta_pairs(False)
-        run.b.h.zero_(), run.b.y_perm.zero_()
-        run.ffn()
-        M.moe_check_device_error(run.ws)
-        torch.cuda.synchronize()
-        check_ffn_rows(run, r)
-        assert torch.equal(run.b.h[:used], h1), "h differs between the two FFN kernels"
-        assert torch.equal(run.b.y_perm[:used], y1), "y_perm differs between the two FFN kernels"
-        check_stats(st, r)
+        for kind in ("token_major", "pairs"):
+            M.set_ffn_kernel(kind)
+            run.b.h.zero_(), run.b.y_perm.zero_()
+            run.ffn()
+            M.moe_check_device_error(run.ws)
+            torch.cuda.synchronize()
+            check_ffn_rows(run, r)
+            assert torch.equal(run.b.h[:used], h1), f"h differs: {kind} vs token_n"
+            assert torch.equal(run.b.y_perm[:used], y1), f"y_perm differs: {kind} vs token_n"
     finally:
-        M.set_ffn_cta_pairs(False)
+        M.set_ffn_kernel("token_major")
 
 
 def test_tied_logits_pick_lower_index():
@@ -250,6 +252,11 @@ VARIANTS = [
     # E = 8 with groups (general top-k path), pick-rank drops, chunk bias in score and weight
     W.reduced(W.MIXTRAL_8X22B_MIXED, 900, 256, 384, n_decode_tokens=8, n_groups=4,
               topk_groups=2, drop_policy=1),
+    # tensor-core router with the top-k in its epilogue: selection-only bias, E not a
+    # multiple of 32 (masked expert columns), a per-token bias, T with a 64-row tail tile
+    W.reduced(W.DSV3_PREFILL_ZIPF, 1000, 256, 128, E=200, bias="chunks", bias_mode=1,
+              n_decode_tokens=8),
+    W.reduced(W.DSV3_PREFILL_ZIPF, 1088, 320, 128, E=96, k=6, gating=W.SOFTMAX),
     # E = 8 fused router with selection-only bias; fp32 layer
     W.reduced(W.TINY_FP32, 200, 64, 96, bias="chunks", bias_mode=1, drop_policy=1,
               capacity_factor=0.9),
@@ -273,6 +280,27 @@ def test_routing_variants_match_oracle(shape):
 
 
 # ------------------------------------------------------------------ errors without faults
+@pytest.mark.parametrize("shape", [W.reduced(W.DSV3_PREFILL_ZIPF, 700, 256, 128),
+                                   W.reduced(W.DSV3_PREFILL_ZIPF, 640, 256, 128, bias_mode=1)],
+                         ids=["bias_in_logits", "selection_only_bias"])
+def test_tensor_core_router_without_logits_buffer(shape):
+    """moe_route on the tensor-core router with no logits buffer (the top-k runs in the GEMM's
+    epilogue and no logits are written) picks and weights exactly as with one."""
+    assert (shape.dtype == W.BF16 and shape.E > 32 and shape.T >= 512)
+    run = GpuRun(shape)
+    run.route()
+    idx, w = run.b.topk_idx.clone(), run.b.topk_w.clone()
+    b, i = run.b, run.inp
+    b.topk_idx.fill_(-7), b.topk_w.fill_(-7.0)
+    M.moe_route(run.cfg, i.x, i.w_router, i.logit_bias, None, b.topk_idx, b.topk_w, run.ws)
+    M.moe_check_device_error(run.ws)
+    torch.cuda.synchronize()
+    assert torch.equal(b.topk_idx, idx) and torch.equal(b.topk_w, w)
+    run.dispatch()
+    r = check_routing(run)   # and the picks against the oracle from the returned logits
+    assert r["idx"].shape == (shape.T, shape.k)
+
+
 def test_bad_expert_index_is_reported_not_faulted():
     shape = _edge(50, 64, 64, 8, 2)
     run = GpuRun(shape)
