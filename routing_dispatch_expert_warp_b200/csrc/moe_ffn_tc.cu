@@ -88,8 +88,7 @@ struct TcParams {
   int32_t T;
   // MODE_ROUTER: the A rows (x) are a_k wide; the K = 2 a_k reduction takes each 64-wide
   // chunk of x against the hi and then the lo half of the split router weight ([E, 2 a_k]:
-  // hi in columns [0, a_k), lo in [a_k, 2 a_k)); out_f32 may be nullptr when the top-k is
-  // fused and the caller wants no logits.
+  // hi in columns [0, a_k), lo in [a_k, 2 a_k)).
   int a_k;
   int fuse_topk;              // 1: the epilogue selects the top-k and writes the gate weights
   int gating;                 // MOE_GATE_SOFTMAX / MOE_GATE_SIGMOID
@@ -461,6 +460,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
           tz[j] = 0.f;
         }
         uint32_t thr = 0u;  // key of the k-th best so far
+        const uint32_t kth_mask = 1u << (p.k - 1);
 #pragma unroll 1
         for (int c = 0; c < BN_OUT / 32; ++c) {
           uint32_t v[32];
@@ -487,32 +487,57 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
               }
             }
             if (p.fuse_topk) {
+              // the chunk's selection keys (0 past the last expert), then its keys above the
+              // k-th best so far, largest first -- equal keys lowest expert first -- inserted
+              // behind the equal keys already held (lower experts); every index is static
+              uint32_t key[32];
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
                 const int col = c * 32 + i;
-                if (col >= cols_left) continue;
-                const uint32_t key = order_key(srow != nullptr ? z[i] + srow[col] : z[i]);
-                if (key <= thr) continue;
+                key[i] = col < cols_left ? order_key(srow != nullptr ? z[i] + srow[col] : z[i])
+                                         : 0u;
+              }
+#pragma unroll 1
+              while (true) {
+                uint32_t best = 0u;
+                int bi = 0;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                  if (key[i] > best) {
+                    best = key[i];
+                    bi = i;
+                  }
+                if (best <= thr) break;
+                float bz = 0.f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                  if (i == bi) {
+                    bz = z[i];
+                    key[i] = 0u;
+                  }
+                const int col = c * 32 + bi;
 #pragma unroll
                 for (int j = MOE_MAX_TOPK - 1; j > 0; --j) {
-                  if (key > tk[j - 1]) {
+                  if (best > tk[j - 1]) {
                     tk[j] = tk[j - 1];
                     ti[j] = ti[j - 1];
                     tz[j] = tz[j - 1];
-                  } else if (key > tk[j]) {
-                    tk[j] = key;
+                  } else if (best > tk[j]) {
+                    tk[j] = best;
                     ti[j] = col;
-                    tz[j] = z[i];
+                    tz[j] = bz;
                   }
                 }
-                if (key > tk[0]) {
-                  tk[0] = key;
+                if (best > tk[0]) {
+                  tk[0] = best;
                   ti[0] = col;
-                  tz[0] = z[i];
+                  tz[0] = bz;
                 }
+                // thr = tk[k - 1], as arithmetic on a one-hot mask (no indexed access)
+                thr = 0u;
 #pragma unroll
                 for (int j = 0; j < MOE_MAX_TOPK; ++j)
-                  if (j == p.k - 1) thr = tk[j];
+                  thr |= tk[j] & (0u - ((kth_mask >> j) & 1u));
               }
             }
           }
@@ -1583,7 +1608,9 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_route
   p.n_blocks = 1;
   p.N_out = s.E;
   p.mb_outer = 1;
-  p.out_f32 = fuse ? logits : (logits != nullptr ? logits : logits_scratch);
+  // z always lands somewhere: in the caller's buffer, or in the workspace copy that the
+  // dispatch of score-priority drops and moe_layer_forward read when the caller has none
+  p.out_f32 = logits != nullptr ? logits : logits_scratch;
   // logits carry the bias unless it is for selection only (then only the keys add it)
   p.bias = sel_only ? nullptr : bias;
   p.sel_bias = sel_only ? bias : nullptr;

@@ -66,8 +66,8 @@ cudaError_t launch_router(const Shape& s, const void* x, const float* w_router,
                           int32_t* topk_idx, float* topk_w, float* partials, cudaStream_t st);
 // Router on tensor cores (bf16 layers, E > 32): W_r split into two bf16 terms.
 bool router_uses_tensor_cores(const Shape& s);
-// logits: the caller's [T, E] buffer or nullptr (then, with the top-k fused into the GEMM,
-// no logits are written; without it they go to logits_scratch).
+// logits: the caller's [T, E] buffer, or nullptr (then z goes to logits_scratch, the
+// workspace copy).
 cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_router,
                              const float* bias, int64_t bias_stride, float* logits,
                              float* logits_scratch, int32_t* topk_idx, float* topk_w,

@@ -122,9 +122,10 @@ def test_ep_emulated_twice_is_deterministic():
     torch.cuda.synchronize()
     for a, b in zip(first, second):
         assert torch.equal(a, b)
-    # per rank: router (3 with the tensor-core router at T >= 512, else 2), count + rank,
-    # put_counts, plan (2), dispatch, FFN (2), combine, stats
-    router = 3 if shape.T >= 512 else 2
+    # per rank: router (2: the W_r split + the tensor-core GEMM with the top-k in its
+    # epilogue at T >= 512; the fp32 GEMM + top-k below), count + rank, put_counts, plan (2),
+    # dispatch, FFN (2), combine, stats
+    router = 2
     assert launched == 4 * (router + 2 + 1 + 2 + 1 + 2 + 1 + 1)
 
 

@@ -284,8 +284,8 @@ def test_routing_variants_match_oracle(shape):
                                    W.reduced(W.DSV3_PREFILL_ZIPF, 640, 256, 128, bias_mode=1)],
                          ids=["bias_in_logits", "selection_only_bias"])
 def test_tensor_core_router_without_logits_buffer(shape):
-    """moe_route on the tensor-core router with no logits buffer (the top-k runs in the GEMM's
-    epilogue and no logits are written) picks and weights exactly as with one."""
+    """moe_route on the tensor-core router (top-k in the GEMM's epilogue) with no logits
+    buffer -- z then goes to the workspace -- picks and weights exactly as with one."""
     assert (shape.dtype == W.BF16 and shape.E > 32 and shape.T >= 512)
     run = GpuRun(shape)
     run.route()
@@ -362,7 +362,8 @@ def test_small_e_router_wide_d(shape):
 # ------------------------------------------------------------------ launch accounting
 @pytest.mark.parametrize("shape,router_kernels", [
     (W.reduced(W.MIXTRAL_8X7B, 1000, 512, 768), 2),          # lane-ordered W_r + fused router
-    (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256), 3),     # W_r split + tensor-core GEMM + top-k
+    (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256), 2),     # W_r split + GEMM with the top-k
+    (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256, n_groups=8, topk_groups=4), 3),  # + top-k
     (W.reduced(W.DSV3_DECODE, 128, 512, 256), 2),            # split-K fp32 GEMM + top-k
 ])
 def test_kernel_launch_count_per_layer(shape, router_kernels):

@@ -169,10 +169,13 @@ def test_scored_permute_rows():
                        inp.x[torch.from_numpy(tor[used]).cuda()])
 
 
-def test_layer_forward_with_workspace_logits():
+@pytest.mark.parametrize("T", [400, 700], ids=["fp32_router", "tensor_core_router"])
+def test_layer_forward_with_workspace_logits(T):
     """moe_layer_forward reads the scores from the caller's logits or, when the logits
-    pointer is NULL, from the workspace copy moe_route wrote: same result either way."""
-    shape = W.reduced(W.DSV3_PREFILL_ZIPF, 400, 256, 128, capacity_factor=0.7, bias_mode=1,
+    pointer is NULL, from the workspace copy moe_route wrote: same result either way, with
+    the fp32 router (T < 512) and with the tensor-core router whose GEMM epilogue takes the
+    top-k."""
+    shape = W.reduced(W.DSV3_PREFILL_ZIPF, T, 256, 128, capacity_factor=0.7, bias_mode=1,
                       drop_policy=2)
     inp = W.make_inputs(shape, device="cuda")
     cfg = M.config_from_shape(shape)
@@ -186,7 +189,8 @@ def test_layer_forward_with_workspace_logits():
     torch.cuda.synchronize()
     assert torch.equal(out_a, out_b)
     assert torch.equal(a.bufs.assign_row, b.bufs.assign_row)
-    # router (2: T < 512), 5 ranking kernels, permute, 2 FFN, combine, stats
+    # router (2: fp32 GEMM + top-k, or W_r split + tensor-core GEMM with the top-k), 5
+    # ranking kernels, permute, 2 FFN, combine, stats
     assert launched == 2 + 5 + 1 + 2 + 1 + 1
 
 
