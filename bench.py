@@ -46,6 +46,9 @@ RECORDED_GEMM_TRAFFIC = {
     ("mixtral8x7b_prefill_T4096", False): {
         "bytes": 3671601664, "sources": "d94c516aa4c2f235",
         "profile": "profiles/grouped_gemm_tc_mixtral8x7b_T4096_traffic.md"},
+    ("dsv3_prefill_zipf_T16384", False): {
+        "bytes": 27293616896, "sources": "4185d57893c9f83c",
+        "profile": "profiles/grouped_gemm_tc_dsv3_prefill_T16384_traffic.md"},
 }
 
 
@@ -834,6 +837,57 @@ def run_microbatch(args) -> None:
     print(json.dumps(line), flush=True)
 
 
+def run_dense_calibration(args) -> None:
+    """The expert FFN's GEMMs on one dense expert (E = 1: every token's row in one bucket)
+    through the library's kernels and through cuBLAS (torch.mm) on the same shapes: x [T, d]
+    against W_g, W_u [f, d] and h [T, f] against W_d [d, f], bf16 in, fp32 accumulate.  A
+    calibration of the grouped GEMM against the vendor library, not the layer's timing."""
+    T, d, f = (int(v) for v in args.dense_calibration.split(","))
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1)
+    x = torch.randn(T, d, device=dev, generator=g).to(torch.bfloat16)
+    wg = (torch.randn(1, f, d, device=dev, generator=g) * d ** -0.5).to(torch.bfloat16)
+    wu = (torch.randn(1, f, d, device=dev, generator=g) * d ** -0.5).to(torch.bfloat16)
+    wd = (torch.randn(1, d, f, device=dev, generator=g) * f ** -0.5).to(torch.bfloat16)
+    h = torch.empty(T, f, device=dev, dtype=torch.bfloat16)
+    y = torch.empty(T, d, device=dev, dtype=torch.bfloat16)
+    flops = 6.0 * T * d * f
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            fn()
+        b.record()
+        b.synchronize()
+        return a.elapsed_time(b) / args.steps
+
+    def cublas():
+        torch.mm(x, wg[0].t())
+        torch.mm(x, wu[0].t())
+        torch.mm(h, wd[0].t())
+
+    res = {"cublas_3mm": timed(cublas)}
+    cfg = M.make_config(T, d, f, 1, 1, dtype=M.BF16)
+    ws = M.alloc_workspace(cfg, dev)
+    offs = torch.tensor([0, T], dtype=torch.int32, device=dev)
+    kept = torch.tensor([T], dtype=torch.int32, device=dev)
+    for kind in ("token_major", "pairs", "token_n"):
+        M.set_ffn_kernel(kind)
+        res[kind] = timed(lambda: M.moe_expert_ffn(cfg, x, offs, kept, wg, wu, wd, h, y, ws))
+        M.moe_check_device_error(ws)
+    M.set_ffn_kernel("token_major")
+    line = {"metric": "dense expert FFN GEMMs, TFLOP/s (calibration)", "T": T, "d_model": d,
+            "d_ff": f, "steps": args.steps, "warmup": args.warmup,
+            "ms": res, "tflops": {k: flops / v / 1e9 for k, v in res.items()}}
+    print(json.dumps(line), flush=True)
+
+
 def _cpu_cores() -> dict:
     """Host cores this process may run on (its affinity mask) and the threads numpy's BLAS
     pool uses, which is what the oracle's matrix products run on."""
@@ -1003,6 +1057,9 @@ def main():
     ap.add_argument("--ep-emulate", type=int, default=0,
                     help="time the expert-parallel layer with this many ranks emulated on one "
                          "GPU (a separate measurement, not the headline line)")
+    ap.add_argument("--dense-calibration", default="",
+                    help="T,d,f: time the FFN's three GEMMs on one dense expert through each "
+                         "FFN kernel and through cuBLAS (a calibration, not the headline line)")
     ap.add_argument("--ep", action="store_true",
                     help="time the expert-parallel layer across the job's GPUs (one process per "
                          "GPU under torchrun): experts split in contiguous blocks, every rank "
@@ -1030,6 +1087,8 @@ def main():
         run_reference(args)
     elif args.microbatches > 1:
         run_microbatch(args)
+    elif args.dense_calibration:
+        run_dense_calibration(args)
     elif args.ep:
         run_ep_group(args)
     elif args.ep_emulate:
