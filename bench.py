@@ -44,7 +44,7 @@ GEMM_SOURCES = ("routing_dispatch_expert_warp_b200/csrc/moe_ffn_tc.cu",
                 "routing_dispatch_expert_warp_b200/csrc/moe_internal.h")
 RECORDED_GEMM_TRAFFIC = {
     ("mixtral8x7b_prefill_T4096", False): {
-        "bytes": 3671601664, "sources": "d94c516aa4c2f235",
+        "bytes": 3671003648, "sources": "4185d57893c9f83c",
         "profile": "profiles/grouped_gemm_tc_mixtral8x7b_T4096_traffic.md"},
     ("dsv3_prefill_zipf_T16384", False): {
         "bytes": 27293616896, "sources": "4185d57893c9f83c",
