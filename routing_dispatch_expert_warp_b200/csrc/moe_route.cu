@@ -104,22 +104,6 @@ __device__ __forceinline__ void router_row_fma(const XRaw<TX> (&xr)[CPW][TW], in
   }
 }
 
-template <typename TX>
-__device__ __forceinline__ void load_pair(const TX* p, float& a, float& b);
-template <>
-__device__ __forceinline__ void load_pair<float>(const float* p, float& a, float& b) {
-  const float2 v = __ldg(reinterpret_cast<const float2*>(p));
-  a = v.x;
-  b = v.y;
-}
-template <>
-__device__ __forceinline__ void load_pair<__nv_bfloat16>(const __nv_bfloat16* p, float& a,
-                                                         float& b) {
-  const uint32_t v = __ldg(reinterpret_cast<const unsigned int*>(p));
-  a = bf16_lo(v);
-  b = bf16_hi(v);
-}
-
 // W_r [d, E] re-laid out for the warp access pattern of the small-E router: in chunk c
 // (256 rows of d) lane l owns rows c*256 + 8l .. 8l+7; vector u = rr * (ET/4) + qq holds
 // row 8l + rr, experts 4qq .. 4qq+3, and the 32 lanes' vectors u are consecutive (512 B),

@@ -239,3 +239,13 @@ def test_prototype_arity_matches_the_header():
         params = " ".join(params.split())
         n = 0 if params in ("", "void") else params.count(",") + 1
         assert n == len(_abi.PROTOTYPES[name][1]), (name, n, len(_abi.PROTOTYPES[name][1]))
+
+
+def test_ffn_kernel_choice_is_checked(lib):
+    """moe_set_ffn_kernel takes the three schedules and refuses anything else (no GPU needed:
+    the choice is host state read at the next launch)."""
+    for kind in (1, 2, 0):                   # pairs, token-N, back to token-major (default)
+        assert lib.moe_set_ffn_kernel(kind) == 0
+    assert lib.moe_set_ffn_kernel(3) == 1    # MOE_ERR_INVALID_ARG
+    assert lib.moe_set_ffn_kernel(-1) == 1
+    assert b"moe_set_ffn_kernel" in lib.moe_last_error()
