@@ -309,10 +309,14 @@ def run_gpu(args) -> None:
     mem_point("layer_buffers_and_workspace")
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    # the router weight is the layer's: its split (tensor-core router) is made once, as
+    # MoELayer does, not in every step
+    w_split = M.router_split(cfg, inp.w_router)
 
     def step(ev):
         ev[0].record(stream)
-        M.moe_route(cfg, inp.x, inp.w_router, inp.logit_bias, b.logits, b.topk_idx, b.topk_w, ws)
+        M.moe_route_ex(cfg, inp.x, inp.w_router, w_split, inp.logit_bias, b.logits, b.topk_idx,
+                       b.topk_w, ws)
         ev[1].record(stream)
         M.moe_dispatch_scored(cfg, inp.x, b.topk_idx, b.logits, inp.logit_bias, b.routed_counts,
                               b.kept_counts, b.expert_offsets, b.assign_row, b.token_of_row,

@@ -55,7 +55,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 4
+#define MOE_ABI_VERSION 5
 #define MOE_MAX_EXPERTS 256
 #define MOE_MAX_TOPK 8
 
@@ -180,6 +180,9 @@ typedef struct moe_layer_inputs {
   const void* w_gate;        /* [E, d_ff, d_model] dtype                                  */
   const void* w_up;          /* [E, d_ff, d_model] dtype                                  */
   const void* w_down;        /* [E, d_model, d_ff] dtype                                  */
+  const void* w_router_split;/* NULL, or the split router weight of moe_router_split for
+                                w_router: the tensor-core router then reads it instead of
+                                splitting w_router at every call (see moe_route_ex)          */
 } moe_layer_inputs_t;
 
 /* Outputs and intermediates of a whole layer (device pointers, caller-allocated). */
@@ -295,6 +298,35 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
                        const float* logit_bias, int64_t bias_row_stride, float* logits,
                        int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
                        void* stream);
+
+/*
+ * The split router weight of the tensor-core router, made once instead of at every call.
+ * The router weight is constant across the forwards of a layer, but moe_route splits it
+ * again each time: W' [E, 2 d_model] bf16, row e = [hi(w_router[:, e]), lo(w_router[:, e])],
+ * hi = bf16(w), lo = bf16(w - hi) (round to nearest even), 2 E d_model bf16 values, 16-byte
+ * aligned device memory owned by the caller.
+ * moe_router_split_size: *bytes = that size, or 0 when the layer shape never takes the
+ *   tensor-core router (fp32 layers, E <= 32, d_model not a multiple of 64).
+ * moe_router_split: enqueue the split on `stream`.  MOE_ERR_UNSUPPORTED when the size is 0,
+ *   MOE_ERR_INVALID_ARG when split_bytes is smaller or a pointer is NULL or unaligned.
+ * The pages have no such step: it moves work the router repeats out of the forward.
+ */
+moe_status_t moe_router_split_size(const moe_config_t* cfg, size_t* bytes);
+moe_status_t moe_router_split(const moe_config_t* cfg, const float* w_router, void* w_split,
+                              size_t split_bytes, void* stream);
+
+/*
+ * moe_route with an optional argument: w_router_split NULL is moe_route; otherwise it is the
+ * moe_router_split output for w_router, which the tensor-core router reads instead of
+ * splitting w_router (one kernel launch instead of two; the result is bitwise the same).  The
+ * other router paths (fp32, E <= 32, T < 512) read w_router and ignore it, so w_router is
+ * required either way.  A split that was not made from this w_router gives the logits of the
+ * weight it was made from.
+ */
+moe_status_t moe_route_ex(const moe_config_t* cfg, const void* x, const float* w_router,
+                          const void* w_router_split, const float* logit_bias,
+                          int64_t bias_row_stride, float* logits, int32_t* topk_idx,
+                          float* topk_w, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Dispatch ([EP-serving] "Technical insight"; [EP-checks] "Profile all-to-all ...": pack
@@ -503,9 +535,10 @@ moe_status_t moe_pick_rank_counts(const moe_config_t* cfg, const int32_t* topk_i
                                   void* stream);
 
 /*
- * The whole layer: moe_route, moe_dispatch_scored (given the logits moe_route wrote:
- * bufs->logits, or the workspace's copy when that is NULL; with the drop policies other than
- * MOE_DROP_SCORE this is moe_dispatch), moe_expert_ffn, moe_combine and (when bufs->stats is
+ * The whole layer: moe_route_ex (with in->w_router_split), moe_dispatch_scored (given the
+ * logits the router wrote: bufs->logits, or the workspace's copy when that is NULL; with the
+ * drop policies other than MOE_DROP_SCORE this is moe_dispatch), moe_expert_ffn,
+ * moe_combine and (when bufs->stats is
  * not NULL) moe_load_stats, enqueued back to back on one stream without a host
  * synchronisation.  bufs->x_perm NULL: dispatch writes no permuted copy and the gate/up GEMM
  * gathers rows of x (moe_expert_ffn_gather).  Returns the first failing stage's status.

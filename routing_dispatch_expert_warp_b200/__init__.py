@@ -23,7 +23,8 @@ BIAS_SCORE_AND_WEIGHT, BIAS_SELECTION_ONLY = 0, 1
 DROP_TOKEN_ORDER, DROP_PICK_RANK, DROP_SCORE = 0, 1, 2
 
 __all__ = ["MoEError", "make_config", "workspace_size", "capacity", "max_rows",
-           "alloc_workspace", "moe_route", "moe_dispatch", "moe_dispatch_scored",
+           "alloc_workspace", "moe_route", "moe_route_ex", "router_split_size", "router_split",
+           "moe_dispatch", "moe_dispatch_scored",
            "moe_dispatch_static_scratch", "moe_static_scratch_check", "moe_pick_rank_counts",
            "moe_expert_ffn", "moe_expert_ffn_gather", "moe_expert_ffn_combine", "moe_combine",
            "moe_load_stats", "moe_load_stats_merge", "moe_layer_forward",
@@ -111,6 +112,35 @@ def moe_route(cfg, x, w_router, logit_bias, logits, topk_idx, topk_w, ws, stream
     check(_lib().moe_route(ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(logit_bias), stride,
                            _ptr(logits), _ptr(topk_idx), _ptr(topk_w), _ptr(ws), ws.numel(),
                            _stream(stream)))
+
+
+def moe_route_ex(cfg, x, w_router, w_router_split, logit_bias, logits, topk_idx, topk_w, ws,
+                 stream=None):
+    """moe_route reading a split router weight made by router_split (or None: moe_route)."""
+    stride = 0 if (logit_bias is None or logit_bias.dim() == 1) else logit_bias.shape[1]
+    check(_lib().moe_route_ex(ctypes.byref(cfg), _ptr(x), _ptr(w_router), _ptr(w_router_split),
+                              _ptr(logit_bias), stride, _ptr(logits), _ptr(topk_idx),
+                              _ptr(topk_w), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def router_split_size(cfg) -> int:
+    """Bytes of the split router weight for cfg (0: the layer never uses the tensor-core
+    router)."""
+    n = ctypes.c_size_t(0)
+    check(_lib().moe_router_split_size(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
+def router_split(cfg, w_router, stream=None) -> Optional[torch.Tensor]:
+    """The split router weight of w_router (a uint8 device tensor), or None when the layer
+    never uses the tensor-core router.  It stays valid while w_router is unchanged."""
+    n = router_split_size(cfg)
+    if n == 0:
+        return None
+    out = torch.empty(n, dtype=torch.uint8, device=w_router.device)
+    check(_lib().moe_router_split(ctypes.byref(cfg), _ptr(w_router), _ptr(out), n,
+                                  _stream(stream)))
+    return out
 
 
 def moe_dispatch(cfg, x, topk_idx, routed_counts, kept_counts, expert_offsets, assign_row,
@@ -294,7 +324,10 @@ class MoELayer:
     returns the output tensor (a view of the layer's own buffer, overwritten by the next
     call).  gather=True drops the permuted copy of x: dispatch only ranks the assignments
     and the gate/up GEMM gathers its rows from x (same results and less memory, but slower
-    than the permuted copy on B200)."""
+    than the permuted copy on B200).
+
+    The split router weight of the tensor-core router is made once here (router_split);
+    call resplit_router() after changing w_router in place."""
 
     def __init__(self, cfg: MoeConfig, w_router, w_gate, w_up, w_down, logit_bias=None,
                  device="cuda", gather: bool = False):
@@ -304,13 +337,18 @@ class MoELayer:
         self.ws = alloc_workspace(cfg, device)
         self.bufs = LayerBuffers.allocate(cfg, device, gather=gather)
         self._structs = self.bufs.as_struct(True)
+        self.resplit_router()
+
+    def resplit_router(self, stream=None) -> None:
+        self.w_router_split = router_split(self.cfg, self.w_router, stream)
 
     def inputs(self, x) -> MoeLayerInputs:
         b = self.logit_bias
         return MoeLayerInputs(
             x=_ptr(x), w_router=_ptr(self.w_router), logit_bias=_ptr(b),
             bias_row_stride=0 if (b is None or b.dim() == 1) else b.shape[1],
-            w_gate=_ptr(self.w_gate), w_up=_ptr(self.w_up), w_down=_ptr(self.w_down))
+            w_gate=_ptr(self.w_gate), w_up=_ptr(self.w_up), w_down=_ptr(self.w_down),
+            w_router_split=_ptr(self.w_router_split))
 
     def forward(self, x: torch.Tensor, stream=None) -> torch.Tensor:
         moe_layer_forward(self.cfg, self.inputs(x), self._structs, self.ws, stream)

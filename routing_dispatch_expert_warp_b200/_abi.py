@@ -46,7 +46,8 @@ class MoeLoadStats(ctypes.Structure):
 
 class MoeLayerInputs(ctypes.Structure):
     _fields_ = [("x", c_vp), ("w_router", c_vp), ("logit_bias", c_vp),
-                ("bias_row_stride", c_i64), ("w_gate", c_vp), ("w_up", c_vp), ("w_down", c_vp)]
+                ("bias_row_stride", c_i64), ("w_gate", c_vp), ("w_up", c_vp), ("w_down", c_vp),
+                ("w_router_split", c_vp)]
 
 
 class MoeLayerBuffers(ctypes.Structure):
@@ -95,6 +96,10 @@ PROTOTYPES = {
     "moe_max_rows": (c_i64, [P(MoeConfig)]),
     "moe_route": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_sz,
                           c_vp]),
+    "moe_route_ex": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp,
+                             c_vp, c_sz, c_vp]),
+    "moe_router_split_size": (c_i32, [P(MoeConfig), P(c_sz)]),
+    "moe_router_split": (c_i32, [P(MoeConfig), c_vp, c_vp, c_sz, c_vp]),
     "moe_dispatch": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                              c_vp, c_sz, c_vp]),
     "moe_dispatch_scored": (c_i32, [P(MoeConfig), c_vp, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp,

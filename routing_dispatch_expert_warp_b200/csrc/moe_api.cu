@@ -274,6 +274,41 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
                        const float* logit_bias, int64_t bias_row_stride, float* logits,
                        int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes,
                        void* stream) {
+  return moe_route_ex(cfg, x, w_router, nullptr, logit_bias, bias_row_stride, logits, topk_idx,
+                      topk_w, ws, ws_bytes, stream);
+}
+
+moe_status_t moe_router_split_size(const moe_config_t* cfg, size_t* bytes) {
+  MOE_REQUIRE(bytes != nullptr, "moe_router_split_size: bytes is NULL");
+  Shape s;
+  moe_status_t st = check_config(cfg, &s);
+  if (st != MOE_OK) return st;
+  *bytes = router_split_bytes(s);
+  return MOE_OK;
+}
+
+moe_status_t moe_router_split(const moe_config_t* cfg, const float* w_router, void* w_split,
+                              size_t split_bytes, void* stream) {
+  Shape s;
+  moe_status_t st = check_config(cfg, &s);
+  if (st != MOE_OK) return st;
+  const size_t need = router_split_bytes(s);
+  if (need == 0)
+    return fail(MOE_ERR_UNSUPPORTED,
+                "moe_router_split: this layer shape never uses the tensor-core router");
+  MOE_REQUIRE(w_router && w_split, "moe_router_split: NULL pointer");
+  MOE_REQUIRE(aligned16(w_router) && aligned16(w_split),
+              "moe_router_split: w_router and w_split must be 16-byte aligned");
+  MOE_REQUIRE(split_bytes >= need, "moe_router_split: split_bytes %zu < %zu", split_bytes, need);
+  cudaError_t err = launch_router_split(s, w_router, w_split, static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return cuda_fail(err, "moe_router_split launch");
+  return MOE_OK;
+}
+
+moe_status_t moe_route_ex(const moe_config_t* cfg, const void* x, const float* w_router,
+                          const void* w_router_split, const float* logit_bias,
+                          int64_t bias_row_stride, float* logits, int32_t* topk_idx,
+                          float* topk_w, void* ws, size_t ws_bytes, void* stream) {
   Shape s;
   moe_status_t st = check_config(cfg, &s);
   if (st != MOE_OK) return st;
@@ -281,6 +316,8 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
   if ((st = check_ws(s, ws, ws_bytes, &lay)) != MOE_OK) return st;
   MOE_REQUIRE(x && w_router && topk_idx && topk_w, "moe_route: NULL input/output pointer");
   MOE_REQUIRE(aligned16(x) && aligned16(w_router), "moe_route: x and w_router must be 16-byte aligned");
+  MOE_REQUIRE(w_router_split == nullptr || aligned16(w_router_split),
+              "moe_route_ex: w_router_split must be 16-byte aligned");
   MOE_REQUIRE(bias_row_stride == 0 || bias_row_stride >= s.E,
               "moe_route: bias_row_stride must be 0 or >= E");
   float* z = logits;
@@ -288,8 +325,8 @@ moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_ro
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   if (router_uses_tensor_cores(s)) {
     const char* why = "";
-    cudaError_t err = launch_router_tc(s, x, w_router, logit_bias, bias_row_stride, logits, z,
-                                       topk_idx, topk_w,
+    cudaError_t err = launch_router_tc(s, x, w_router, w_router_split, logit_bias,
+                                       bias_row_stride, logits, z, topk_idx, topk_w,
                                        static_cast<uint8_t*>(ws) + lay.router_tc,
                                        ws_status(ws, lay), g_wait_ns.load(), strm, &why);
     if (err != cudaSuccess) {
@@ -558,10 +595,11 @@ moe_status_t moe_layer_forward(const moe_config_t* cfg, const moe_layer_inputs_t
                                const moe_layer_buffers_t* b, void* ws, size_t ws_bytes,
                                void* stream) {
   MOE_REQUIRE(in != nullptr && b != nullptr, "moe_layer_forward: NULL inputs or buffers");
-  moe_status_t st = moe_route(cfg, in->x, in->w_router, in->logit_bias, in->bias_row_stride,
-                              b->logits, b->topk_idx, b->topk_w, ws, ws_bytes, stream);
+  moe_status_t st = moe_route_ex(cfg, in->x, in->w_router, in->w_router_split, in->logit_bias,
+                                 in->bias_row_stride, b->logits, b->topk_idx, b->topk_w, ws,
+                                 ws_bytes, stream);
   if (st != MOE_OK) return st;
-  // the logits moe_route wrote: the caller's array, else the workspace's
+  // the logits the router wrote: the caller's array, else the workspace's
   const float* z = b->logits;
   if (z == nullptr) {
     Shape s;

@@ -14,9 +14,10 @@
 namespace moe {
 namespace {
 
-// A thread owns NV 16-byte vectors of one output row (NV = 4 when the row allows it): its
-// k x NV source loads are independent and issued together before the pick-ordered sums.
-template <bool BF16, int NV>
+// A thread owns NV 16-byte vectors of one output row.  It first reads the token's k rows and
+// weights, then issues all k x NV source loads at once (KMAX x NV <= 8 uint4 in flight per
+// thread), and only then adds them up in pick order.
+template <bool BF16, int KMAX, int NV>
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y_perm,
                                                       const int32_t* __restrict__ assign_row,
                                                       const float* __restrict__ topk_w,
@@ -29,21 +30,37 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t t = i / groups_per_row;
     const int64_t v0 = (i - t * groups_per_row) * NV;
+    int32_t rows[KMAX];
+    float ws[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      rows[j] = -1;
+      ws[j] = 0.f;
+      if (j < k) {
+        rows[j] = __ldg(assign_row + t * k + j);
+        ws[j] = __ldg(topk_w + t * k + j);
+      }
+    }
+    uint4 src[KMAX][NV];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j)
+#pragma unroll
+      for (int u = 0; u < NV; ++u)
+        src[j][u] = rows[j] >= 0
+                        ? __ldg(y_perm + static_cast<int64_t>(rows[j]) * vec_per_row + v0 + u)
+                        : make_uint4(0u, 0u, 0u, 0u);
     float acc[NV][NE];
 #pragma unroll
     for (int u = 0; u < NV; ++u)
 #pragma unroll
       for (int q = 0; q < NE; ++q) acc[u][q] = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int32_t r = __ldg(assign_row + t * k + j);
-      if (r < 0) continue;
-      const float w = __ldg(topk_w + t * k + j);
-      uint4 src[NV];
 #pragma unroll
-      for (int u = 0; u < NV; ++u) src[u] = __ldg(y_perm + static_cast<int64_t>(r) * vec_per_row + v0 + u);
+    for (int j = 0; j < KMAX; ++j) {
+      if (rows[j] < 0) continue;  // dropped picks (and j >= k) contribute nothing
+      const float w = ws[j];
 #pragma unroll
       for (int u = 0; u < NV; ++u) {
-        const uint32_t uu[4] = {src[u].x, src[u].y, src[u].z, src[u].w};
+        const uint32_t uu[4] = {src[j][u].x, src[j][u].y, src[j][u].z, src[j][u].w};
         if (BF16) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -71,26 +88,40 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
   }
 }
 
-template <bool BF16>
-cudaError_t launch_combine_typed(const Shape& s, const void* y_perm, const int32_t* assign_row,
-                                 const float* topk_w, void* out, cudaStream_t st) {
+template <bool BF16, int KMAX, int NV>
+cudaError_t launch_combine_shaped(const Shape& s, const uint4* y, const int32_t* assign_row,
+                                  const float* topk_w, uint4* o, cudaStream_t st) {
   const int64_t vec_per_row = s.d * s.elem / 16;
-  const bool wide = vec_per_row % 4 == 0;
-  const int64_t total = s.T * (wide ? vec_per_row / 4 : vec_per_row);
+  const int64_t total = s.T * (vec_per_row / NV);
   int64_t blocks = (total + 255) / 256;
   const int64_t cap = static_cast<int64_t>(sm_count()) * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  const uint4* y = static_cast<const uint4*>(y_perm);
-  uint4* o = static_cast<uint4*>(out);
-  if (wide)
-    combine_kernel<BF16, 4><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-        y, assign_row, topk_w, s.T, s.k, vec_per_row, o);
-  else
-    combine_kernel<BF16, 1><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-        y, assign_row, topk_w, s.T, s.k, vec_per_row, o);
+  combine_kernel<BF16, KMAX, NV><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      y, assign_row, topk_w, s.T, s.k, vec_per_row, o);
   note_launch();
   return cudaGetLastError();
+}
+
+// KMAX = k rounded up to 2, 4 or 8; NV = 8 / KMAX vectors per thread when the row allows it
+template <bool BF16, int KMAX>
+cudaError_t launch_combine_k(const Shape& s, const uint4* y, const int32_t* assign_row,
+                             const float* topk_w, uint4* o, cudaStream_t st) {
+  constexpr int NV = 8 / KMAX;
+  const int64_t vec_per_row = s.d * s.elem / 16;
+  if (NV > 1 && vec_per_row % NV == 0)
+    return launch_combine_shaped<BF16, KMAX, NV>(s, y, assign_row, topk_w, o, st);
+  return launch_combine_shaped<BF16, KMAX, 1>(s, y, assign_row, topk_w, o, st);
+}
+
+template <bool BF16>
+cudaError_t launch_combine_typed(const Shape& s, const void* y_perm, const int32_t* assign_row,
+                                 const float* topk_w, void* out, cudaStream_t st) {
+  const uint4* y = static_cast<const uint4*>(y_perm);
+  uint4* o = static_cast<uint4*>(out);
+  if (s.k <= 2) return launch_combine_k<BF16, 2>(s, y, assign_row, topk_w, o, st);
+  if (s.k <= 4) return launch_combine_k<BF16, 4>(s, y, assign_row, topk_w, o, st);
+  return launch_combine_k<BF16, 8>(s, y, assign_row, topk_w, o, st);
 }
 
 }  // namespace

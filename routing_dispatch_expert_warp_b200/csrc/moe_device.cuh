@@ -116,6 +116,21 @@ __device__ __forceinline__ void bulk_wait_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// Shared-memory writes of this thread made visible to the async proxy (a later bulk store
+// of the same bytes by another thread of the CTA, after a barrier)
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Tiled tensor store from this CTA's shared memory, tracked by bulk groups; elements past the
+// tensor's bounds are not written.  `map` is a __grid_constant__ kernel parameter.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src_smem,
+                                             int32_t c0, int32_t c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_addr(src_smem)), "r"(c0), "r"(c1)
+               : "memory");
+}
+
 // Tiled tensor loads into this CTA's shared memory.  `map` is a __grid_constant__ kernel parameter.
 __device__ __forceinline__ void tma_load_2d(void* dst_smem, const CUtensorMap* map,
                                             uint64_t* bar, int32_t c0, int32_t c1) {

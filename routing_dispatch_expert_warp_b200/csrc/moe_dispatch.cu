@@ -27,6 +27,9 @@
 //              Writes assign_row and token_of_row (-1 for rows no assignment uses).
 //   3. permute: token-major row copy with bulk (TMA) copies: each row of x is read from HBM
 //              once into shared memory and written to each of its kept rows of x_perm.
+// With at most kSelfCountMaxPicks picks and no score filter, 1 and 2 are one launch: every
+// rank block counts all picks itself (a few KB of topk_idx from L2) instead of reading the
+// count kernel's per-block histograms.
 #include <mutex>
 
 #include "moe_internal.h"
@@ -115,11 +118,18 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_count_kernel(
 // rows no assignment uses are marked -1 in token_of_row.  With a filter, hist counts the
 // kept picks only, the others get row -1, and routed (the demand, counted by an earlier
 // unfiltered pass) is left as it is.
+//
+// SELF_COUNT (no filter, few picks): there is no count kernel and no hist.  Every block
+// counts all T x k picks itself -- per plane and expert, the total and the part from tokens
+// before its own -- which is what the sums over hist give; it also records invalid experts.
+constexpr int64_t kSelfCountMaxPicks = 32768;
+
+template <bool SELF_COUNT>
 __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
     const int32_t* __restrict__ topk_idx, int64_t T, int k, int E, int64_t C, int layout,
     int planes, int64_t nblk, const int32_t* __restrict__ hist, int32_t* __restrict__ routed,
     int32_t* __restrict__ kept, int32_t* __restrict__ offsets, int32_t* __restrict__ assign_row,
-    int32_t* __restrict__ token_of_row, int64_t max_rows, ScoreFilter flt) {
+    int32_t* __restrict__ token_of_row, int64_t max_rows, ScoreFilter flt, DevStatus* status) {
   static_assert(kDispatchBlockTokens == MOE_MAX_EXPERTS, "one thread per expert");
   __shared__ uint32_t masks[kWarps][MOE_MAX_EXPERTS];
   __shared__ int32_t wbase[kWarps][MOE_MAX_EXPERTS];
@@ -127,12 +137,71 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
   __shared__ int32_t off_s[MOE_MAX_EXPERTS];
   __shared__ int32_t kept_s[MOE_MAX_EXPERTS];
   __shared__ int64_t scan[MOE_MAX_EXPERTS];
+  __shared__ int32_t self_tot[SELF_COUNT ? MOE_MAX_TOPK : 1][MOE_MAX_EXPERTS];
+  __shared__ int32_t self_bef[SELF_COUNT ? MOE_MAX_TOPK : 1][MOE_MAX_EXPERTS];
 
   const int e = threadIdx.x;
+  if (SELF_COUNT) {
+    for (int i = threadIdx.x; i < planes * MOE_MAX_EXPERTS; i += blockDim.x) {
+      (&self_tot[0][0])[i] = 0;
+      (&self_bef[0][0])[i] = 0;
+    }
+    __syncthreads();
+    // warp w takes tokens 32 w + 256 n + lane, one pick slot j at a time, the loads of 8
+    // batches in flight together; a 32-token batch lies wholly before this block's first
+    // token or wholly at or after it
+    constexpr int U = 8;
+    const int lane = threadIdx.x & 31;
+    const int64_t t_lo = static_cast<int64_t>(blockIdx.x) * kDispatchBlockTokens;
+    for (int j = 0; j < k; ++j) {
+      const int p = planes > 1 ? j : 0;
+      int tot = 0, bef = 0;  // E <= 32: lane ee's counts of expert ee
+      for (int64_t tb = (threadIdx.x >> 5) * 32; tb < T; tb += U * kDispatchBlockTokens) {
+        int ev[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int64_t t = tb + u * kDispatchBlockTokens + lane;
+          ev[u] = t < T ? __ldg(topk_idx + t * k + j) : -1;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int ee = (ev[u] < 0 || ev[u] >= E) ? -1 : ev[u];
+          const bool early = tb + u * kDispatchBlockTokens < t_lo;
+          if (E <= 32) {
+            for (int x = 0; x < E; ++x) {
+              const int c = __popc(__ballot_sync(0xffffffffu, ee == x));
+              if (lane == x) {
+                tot += c;
+                if (early) bef += c;
+              }
+            }
+          } else {
+            const uint32_t grp = __match_any_sync(0xffffffffu, ee);
+            if (ee >= 0 && lane == __ffs(grp) - 1) {
+              atomicAdd(&self_tot[p][ee], __popc(grp));
+              if (early) atomicAdd(&self_bef[p][ee], __popc(grp));
+            }
+          }
+        }
+      }
+      if (E <= 32 && lane < E) {
+        atomicAdd(&self_tot[p][lane], tot);
+        atomicAdd(&self_bef[p][lane], bef);
+      }
+    }
+    __syncthreads();
+  }
   int64_t run = 0;  // routed total over all planes
   if (e < E) {
     for (int p = 0; p < planes; ++p) {
       int64_t tot = 0, before = 0;
+      if (SELF_COUNT) {
+        tot = self_tot[p][e];
+        before = self_bef[p][e];
+        pbase[p][e] = static_cast<int32_t>(run + before);
+        run += tot;
+        continue;
+      }
       int64_t b = 0;
       for (; b + 8 <= nblk; b += 8) {  // loads issued 8 at a time, sums in block order
         int32_t c[8];
@@ -183,7 +252,8 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
   const uint32_t below = (1u << (threadIdx.x & 31)) - 1u;
   for (int p = 0; p < planes; ++p) {
     __syncthreads();  // pbase / off_s ready; masks of the previous plane no longer read
-    build_masks(topk_idx, T, k, E, masks, nullptr, p, planes, flt);
+    build_masks(topk_idx, T, k, E, masks, SELF_COUNT && p == 0 ? status : nullptr, p, planes,
+                flt);
     if (e < E) {
       int32_t wb = pbase[p][e];
 #pragma unroll
@@ -349,9 +419,13 @@ __global__ void __launch_bounds__(kCountThreads) pick_rank_counts_kernel(
   if (threadIdx.x == 0) differs[j] = static_cast<int32_t>(d_s);
 }
 
-// Token-major bulk copy.  One thread per block issues everything: a ring of NBUF shared
-// buffers, LOOKAHEAD loads in flight, stores of the rows already loaded in flight
-// behind them.  A work item is one segment (<= 16 KB) of one token's row.
+// Token-major bulk copy.  One lane per block issues every copy: a ring of NBUF shared
+// buffers, LOOKAHEAD loads in flight, stores of the rows already loaded in flight behind
+// them.  A work item is one segment (<= 16 KB) of one token's row.  The whole warp fetches
+// the rows each item goes to, 32 items (a chunk) per lane-parallel load: while lane 0 copies
+// chunk c, the loads for chunk c + 2 are in flight in registers and chunk c + 1 (which the
+// lookahead reaches) already sits in shared memory, so the issuing lane never waits on a
+// global load after the first chunk.
 constexpr uint32_t kPermMaxSeg = 16384;
 constexpr int kPermMaxNBuf = 16;
 
@@ -362,10 +436,16 @@ __global__ void __launch_bounds__(32) permute_rows_kernel(
     DevStatus* status, uint64_t wait_ns) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ __align__(8) uint64_t full[kPermNBuf];
-  static_assert(kPermNBuf <= kPermMaxNBuf && kPermLookahead < kPermNBuf, "ring shape");
-  if (threadIdx.x != 0) return;
-  for (int b = 0; b < kPermNBuf; ++b) mbar_init(&full[b], 1);
-  fence_barrier_init();
+  __shared__ int32_t meta_rows[3][32][MOE_MAX_TOPK];  // rows of the items of three chunks
+  __shared__ uint32_t meta_any[3];                    // bit l: item l has a kept row
+  static_assert(kPermNBuf <= kPermMaxNBuf && kPermLookahead < kPermNBuf &&
+                    kPermLookahead <= 32,
+                "ring shape; the lookahead stays inside the next chunk");
+  const int lane = threadIdx.x;
+  if (lane == 0) {
+    for (int b = 0; b < kPermNBuf; ++b) mbar_init(&full[b], 1);
+    fence_barrier_init();
+  }
 
   const int64_t items = T * segs_per_row;
   const int64_t first = blockIdx.x, step = gridDim.x;
@@ -373,65 +453,101 @@ __global__ void __launch_bounds__(32) permute_rows_kernel(
   uint32_t phase_bits = 0;  // parity of the next completion per buffer
   uint32_t armed = 0;       // buffers with a load in flight
 
-  auto item_rows_any = [&](int64_t it) {
-    const int64_t t = it / segs_per_row;
-    for (int j = 0; j < k; ++j)
-      if (assign_row[t * k + j] >= 0) return true;
-    return false;
+  int32_t mr[MOE_MAX_TOPK];  // this lane's item of the chunk in flight
+  auto fetch = [&](int64_t c) {  // issue the loads of chunk c's rows (item c * 32 + lane)
+    const int64_t i = c * 32 + lane;
+    const int64_t t = i < n ? (first + i * step) / segs_per_row : -1;
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_TOPK; ++j)
+      mr[j] = (t >= 0 && j < k) ? __ldg(assign_row + t * k + j) : -1;
+  };
+  auto publish = [&](int64_t c) {  // the fetched rows into buffer c % 3 (whole warp)
+    bool any = false;
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+      meta_rows[c % 3][lane][j] = mr[j];
+      any = any || mr[j] >= 0;
+    }
+    const uint32_t bits = __ballot_sync(0xffffffffu, any);
+    if (lane == 0) meta_any[c % 3] = bits;
+  };
+  auto has_rows = [&](int64_t i) { return ((meta_any[(i >> 5) % 3] >> (i & 31)) & 1u) != 0u; };
+  auto seg_of = [&](int64_t i, int64_t& t, int64_t& off) {
+    const int64_t it = first + i * step;
+    t = it / segs_per_row;
+    off = (it - t * segs_per_row) * seg_bytes;
+    return static_cast<uint32_t>(row_bytes - off < static_cast<int64_t>(seg_bytes)
+                                     ? row_bytes - off
+                                     : seg_bytes);
   };
   auto issue_load = [&](int64_t i) {
-    const int64_t it = first + i * step;
-    const int64_t t = it / segs_per_row, sg = it % segs_per_row;
+    int64_t t, off;
+    const uint32_t bytes = seg_of(i, t, off);
     const int b = static_cast<int>(i % kPermNBuf);
-    const int64_t off = sg * seg_bytes;
-    const uint32_t bytes = static_cast<uint32_t>(
-        row_bytes - off < static_cast<int64_t>(seg_bytes) ? row_bytes - off : seg_bytes);
     armed |= 1u << b;
     mbar_arrive_expect_tx(&full[b], bytes);
     bulk_load(smem + static_cast<size_t>(b) * seg_bytes, x + t * row_bytes + off, bytes,
               &full[b]);
   };
 
+  fetch(0);
+  publish(0);
+  if (n > 32) fetch(1);
+  __syncwarp();
   // Tokens whose picks were all dropped are skipped: their buffer is never filled and
   // their barrier never armed, so skipping must be decided identically at issue and use.
-  for (int64_t i = 0; i < n && i < kPermLookahead; ++i)
-    if (item_rows_any(first + i * step)) issue_load(i);
+  if (lane == 0)
+    for (int64_t i = 0; i < n && i < kPermLookahead; ++i)
+      if (has_rows(i)) issue_load(i);
 
-  for (int64_t i = 0; i < n; ++i) {
-    const int64_t it = first + i * step;
-    const int b = static_cast<int>(i % kPermNBuf);
-    if (item_rows_any(it)) {
-      const int64_t t = it / segs_per_row, sg = it % segs_per_row;
-      const int64_t off = sg * seg_bytes;
-      const uint32_t bytes = static_cast<uint32_t>(
-          row_bytes - off < static_cast<int64_t>(seg_bytes) ? row_bytes - off : seg_bytes);
-      if (!mbar_wait(&full[b], (phase_bits >> b) & 1u, wait_ns, nullptr)) {
-        record_error(status, DEV_TIMEOUT, 10, static_cast<unsigned long long>(it));
-        // drain: let every load still in flight land before the block exits
-        for (int q = 0; q < kPermNBuf; ++q)
-          if ((armed >> q) & 1u) mbar_wait(&full[q], (phase_bits >> q) & 1u, wait_ns, nullptr);
-        bulk_wait_all();
-        return;
-      }
-      phase_bits ^= (1u << b);
-      armed &= ~(1u << b);
-      for (int j = 0; j < k; ++j) {
-        const int32_t r = assign_row[t * k + j];
-        if (r >= 0)
-          bulk_store(x_perm + static_cast<int64_t>(r) * row_bytes + off,
-                     smem + static_cast<size_t>(b) * seg_bytes, bytes);
+  for (int64_t c = 0; c * 32 < n; ++c) {
+    // chunk c + 1 into the buffer chunk c - 2 used (the lookahead reads it from here on),
+    // then the loads of chunk c + 2 go out and land while lane 0 copies chunk c
+    if ((c + 1) * 32 < n) publish(c + 1);
+    if ((c + 2) * 32 < n) fetch(c + 2);
+    __syncwarp();
+    int failed = 0;
+    if (lane == 0) {
+      const int64_t end = (c + 1) * 32 < n ? (c + 1) * 32 : n;
+      for (int64_t i = c * 32; i < end; ++i) {
+        const int b = static_cast<int>(i % kPermNBuf);
+        if (has_rows(i)) {
+          int64_t t, off;
+          const uint32_t bytes = seg_of(i, t, off);
+          if (!mbar_wait(&full[b], (phase_bits >> b) & 1u, wait_ns, nullptr)) {
+            record_error(status, DEV_TIMEOUT, 10,
+                         static_cast<unsigned long long>(first + i * step));
+            // drain: let every load still in flight land before the block exits
+            for (int q = 0; q < kPermNBuf; ++q)
+              if ((armed >> q) & 1u) mbar_wait(&full[q], (phase_bits >> q) & 1u, wait_ns, nullptr);
+            bulk_wait_all();
+            failed = 1;
+            break;
+          }
+          phase_bits ^= (1u << b);
+          armed &= ~(1u << b);
+          const int32_t* rows = meta_rows[(i >> 5) % 3][i & 31];
+          for (int j = 0; j < k; ++j) {
+            const int32_t r = rows[j];
+            if (r >= 0)
+              bulk_store(x_perm + static_cast<int64_t>(r) * row_bytes + off,
+                         smem + static_cast<size_t>(b) * seg_bytes, bytes);
+          }
+        }
+        bulk_commit();  // one group per item (possibly empty) keeps the group count regular
+        const int64_t nxt = i + kPermLookahead;
+        if (nxt < n) {
+          // buffer nxt % NBUF was last read by the stores of item nxt - NBUF; at most
+          // NBUF - LOOKAHEAD groups committed after it may still be reading
+          bulk_wait_read<kPermNBuf - kPermLookahead>();
+          if (has_rows(nxt)) issue_load(nxt);
+        }
       }
     }
-    bulk_commit();  // one group per item (possibly empty) keeps the group count regular
-    const int64_t nxt = i + kPermLookahead;
-    if (nxt < n) {
-      // buffer nxt % NBUF was last read by the stores of item nxt - NBUF; at most
-      // NBUF - LOOKAHEAD groups committed after it may still be reading
-      bulk_wait_read<kPermNBuf - kPermLookahead>();
-      if (item_rows_any(first + nxt * step)) issue_load(nxt);
-    }
+    failed = __shfl_sync(0xffffffffu, failed, 0);
+    if (failed) return;
   }
-  bulk_wait_all();
+  if (lane == 0) bulk_wait_all();
 }
 
 }  // namespace
@@ -497,9 +613,9 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
         topk_idx, s.T, s.k, s.E, 1, hist, status, all);
     note_launch();
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    dispatch_rank_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
+    dispatch_rank_kernel<false><<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
         topk_idx, s.T, s.k, s.E, -1, MOE_LAYOUT_COMPACT, 1, nblk, hist, routed, sc.kept,
-        sc.offsets, sc.assign_row, sc.token_of_row, s.T * s.k, all);
+        sc.offsets, sc.assign_row, sc.token_of_row, s.T * s.k, all, nullptr);
     note_launch();
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     // 2. per expert, the priority of its C-th best pick
@@ -513,9 +629,16 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
         topk_idx, s.T, s.k, s.E, 1, hist, nullptr, flt);
     note_launch();
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    dispatch_rank_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
+    dispatch_rank_kernel<false><<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
         topk_idx, s.T, s.k, s.E, s.C, s.layout, 1, nblk, hist, routed, kept, offsets,
-        assign_row, token_of_row, s.max_rows, flt);
+        assign_row, token_of_row, s.max_rows, flt, nullptr);
+    note_launch();
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  } else if (s.T * s.k <= kSelfCountMaxPicks) {
+    // few picks: one launch, every block counting all picks itself
+    dispatch_rank_kernel<true><<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
+        topk_idx, s.T, s.k, s.E, s.C, s.layout, planes, nblk, nullptr, routed, kept, offsets,
+        assign_row, token_of_row, s.max_rows, all, status);
     note_launch();
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   } else {
@@ -523,9 +646,9 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
         topk_idx, s.T, s.k, s.E, planes, hist, status, all);
     note_launch();
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    dispatch_rank_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
+    dispatch_rank_kernel<false><<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
         topk_idx, s.T, s.k, s.E, s.C, s.layout, planes, nblk, hist, routed, kept, offsets,
-        assign_row, token_of_row, s.max_rows, all);
+        assign_row, token_of_row, s.max_rows, all, nullptr);
     note_launch();
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }

@@ -53,9 +53,11 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
-// per epilogue warp: 32 rows x 64 bytes (one 32-column chunk of bf16), rows 80 bytes apart
-constexpr int XSTAGE_STRIDE = 80;
-constexpr int XSTAGE_BYTES = 32 * XSTAGE_STRIDE;
+// per epilogue warp: two buffers of 32 rows x 64 bytes (one 32-column chunk of bf16) in the
+// layout of a 64-byte-swizzled tensor tile (16-byte piece c of row r at r * 64 +
+// ((c ^ ((r >> 1) & 3)) * 16)), 2 KB apart from a 1 KB-aligned base
+constexpr int XBUF_BYTES = 32 * 64;
+constexpr int XSTAGE_BYTES = 2 * XBUF_BYTES;
 constexpr int DYN_SMEM = STAGES * STAGE_BYTES + 4 * XSTAGE_BYTES + 1024;  // + alignment slack
 
 enum TcMode { MODE_DOWN = 0, MODE_SWIGLU = 1, MODE_ROUTER = 2 };
@@ -98,6 +100,7 @@ struct TcParams {
   const float* sel_bias;      // bias added to the selection score only (or nullptr)
   int32_t* route_idx;         // [T, k] picks (fused top-k)
   float* route_w;             // [T, k] gate weights (fused top-k)
+  int32_t router_rows;        // MODE_ROUTER: its one bucket is rows [0, router_rows) of x
 };
 
 // The last of a token's kept picks to finish column block nb has its warp sum the token's
@@ -164,37 +167,55 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
   return g / (1.0f + __expf(-g)) * u;
 }
 
-// One 32-column chunk of a 128-row tile, bf16, from the warp that holds TMEM lane quarter q:
-// each lane's row (16 packed words) goes into the warp's staging buffer, then every 4 lanes
-// store one row's 64 bytes, 8 rows per store instruction instead of 32 scattered 16-byte
-// pieces.  Rows at or past `valid` are not stored; with M = 64 tiles TMEM lane i < 16 of
-// quarter q holds tile row 16 q + i.
+// One 32-column chunk of a 128-row tile, bf16, from the warp that holds TMEM lane quarter q.
+// Each lane writes its row (16 packed words) into the warp's staging buffer `buf` in the
+// 64-byte-swizzled layout.  When all 32 rows of the quarter are bucket rows (`tma_rows`),
+// lane 0 stores the 32 x 32 block with one tensor store; otherwise every 4 lanes store one
+// row's 64 bytes, 8 rows per instruction, skipping rows at or past `valid` (with M = 64
+// tiles TMEM lane i < 16 of quarter q holds tile row 16 q + i).  The caller has made sure
+// that no earlier tensor store still reads `buf`; lane 0 commits one bulk group per call.
 __device__ __forceinline__ void store_chunk_staged(uint8_t* buf, const uint32_t (&pk)[16],
+                                                   const CUtensorMap* tm_out,
                                                    __nv_bfloat16* out, int64_t n_out, int row0,
                                                    int64_t col, int q, int valid, bool m64,
-                                                   bool cols_ok, int lane) {
-  __syncwarp();  // the previous chunk's reads of the buffer are done
-  uint4* mine = reinterpret_cast<uint4*>(buf + lane * XSTAGE_STRIDE);
+                                                   bool cols_ok, bool tma_rows, int lane) {
+  const int sw = (lane >> 1) & 3;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) mine[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-  __syncwarp();
-  if (!cols_ok) return;
-  const int seg = lane & 3;
+  for (int i = 0; i < 4; ++i)
+    *reinterpret_cast<uint4*>(buf + lane * 64 + ((i ^ sw) << 4)) =
+        make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+  if (tma_rows) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && cols_ok)
+      tma_store_2d(tm_out, buf, static_cast<int32_t>(col), row0 + 32 * q);
+  } else {
+    __syncwarp();
+    if (cols_ok) {
+      const int seg = lane & 3;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int sr = 8 * i + (lane >> 2);  // staging row = TMEM lane within the quarter
-    const int tr = m64 ? (sr < 16 ? 16 * q + sr : BM) : 32 * q + sr;
-    if (tr < valid) {
-      const uint4 v = *reinterpret_cast<const uint4*>(buf + sr * XSTAGE_STRIDE + seg * 16);
-      *reinterpret_cast<uint4*>(out + static_cast<int64_t>(row0 + tr) * n_out + col + seg * 8) = v;
+      for (int i = 0; i < 4; ++i) {
+        const int sr = 8 * i + (lane >> 2);  // staging row = TMEM lane within the quarter
+        const int tr = m64 ? (sr < 16 ? 16 * q + sr : BM) : 32 * q + sr;
+        if (tr < valid) {
+          const uint4 v =
+              *reinterpret_cast<const uint4*>(buf + sr * 64 + ((seg ^ ((sr >> 1) & 3)) << 4));
+          *reinterpret_cast<uint4*>(out + static_cast<int64_t>(row0 + tr) * n_out + col +
+                                    seg * 8) = v;
+        }
+      }
     }
   }
+  if (lane == 0) bulk_commit();  // one group per chunk, empty or not
 }
 
+// tm_out (MODE_DOWN): the output y_perm [rows, N_out], 32 x 32 boxes, 64-byte swizzle, for
+// the epilogue's tensor stores; the other modes do not read it.
 template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
     const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
-    const __grid_constant__ CUtensorMap tm_b1, const TcParams p) {
+    const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_out,
+    const TcParams p) {
   constexpr bool GATED = MODE == MODE_SWIGLU;  // B tile = two stacked 128-row halves
   constexpr int BN_OUT = GATED ? 128 : 256;
   extern __shared__ uint8_t smem_raw[];
@@ -212,12 +233,16 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // the router's one bucket is rows [0, router_rows) of x; the FFN's buckets are the
+  // dispatch's offsets and kept counts
+  auto seg_start = [&](int e) { return MODE == MODE_ROUTER ? 0 : p.seg_start[e]; };
+  auto seg_count = [&](int e) { return MODE == MODE_ROUTER ? p.router_rows : p.seg_count[e]; };
 
   if (warp == 0) {  // tile table: m-blocks per expert and their prefix (x n_blocks)
     int carry = 0;
     for (int e0 = 0; e0 < p.E; e0 += 32) {
       const int e = e0 + lane;
-      const int mb = e < p.E ? (p.seg_count[e] + BM - 1) / BM : 0;
+      const int mb = e < p.E ? (seg_count(e) + BM - 1) / BM : 0;
       int v = mb;
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -274,7 +299,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
       for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
         int e, mb, nb;
         decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, p.mb_outer, e, mb, nb);
-        const int row0 = p.seg_start[e] + mb * BM;
+        const int row0 = seg_start(e) + mb * BM;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty_bar[s], ph ^ 1u, p.wait_ns, &abort_s)) {
             if (!abort_s)
@@ -329,10 +354,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
     for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
       int e, mb, nb;
       decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, p.mb_outer, e, mb, nb);
-      const int row0 = p.seg_start[e] + mb * BM;
+      const int row0 = seg_start(e) + mb * BM;
       // rows past the bucket read token 0; the epilogue never stores them
       const uint8_t* src[4];
-      const int valid = p.seg_count[e] - mb * BM;
+      const int valid = seg_count(e) - mb * BM;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = lane + 32 * i;
@@ -405,7 +430,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
       int e, mb, nb;
       decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, p.mb_outer, e, mb, nb);
       const uint32_t idesc =
-          p.seg_count[e] - mb * BM <= BM / 2 ? idesc_half : idesc_full;
+          seg_count(e) - mb * BM <= BM / 2 ? idesc_half : idesc_full;
       if (!mbar_wait(&tempty_bar[acc], aph ^ 1u, p.wait_ns, &abort_s)) {
         if (!abort_s) record_error(p.status, DEV_TIMEOUT, 21, static_cast<unsigned long long>(tile));
         abort_s = 1;
@@ -454,8 +479,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       int e, mb, nb;
       decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, p.mb_outer, e, mb, nb);
-      const int row0 = p.seg_start[e] + mb * BM;
-      const int valid = p.seg_count[e] - mb * BM;
+      const int row0 = seg_start(e) + mb * BM;
+      const int valid = seg_count(e) - mb * BM;
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&tfull_bar[acc], aph, p.wait_ns, &abort_s) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -618,9 +643,11 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
         }
       } else {
         // down tiles (K = d_ff) end every few K steps with 64 KB of output: stores go through
-        // the staging buffer, 8 rows of 64 bytes per instruction (4.8% faster on the
-        // DeepSeek-shaped buckets); the fused combine needs each row stored by its owner
+        // the staging buffers, a 32 x 32 tensor store per chunk where the quarter's 32 rows
+        // are all bucket rows, else 8 rows of 64 bytes per instruction; the fused combine
+        // needs each row stored by its owner
         const bool staged = p.comb_out == nullptr;
+        const bool tma_rows = valid > BM / 2 && valid >= 32 * (q + 1);
 #pragma unroll 1
         for (int c = 0; c < BN_OUT / 32; ++c) {
           uint32_t v[32];
@@ -631,9 +658,12 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
           for (int i = 0; i < 16; ++i)
             pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
           if (staged) {
-            store_chunk_staged(xstage, pk, p.out, p.N_out, row0,
+            // buffer c & 1 was last read by the store of two chunks ago (one group may stay)
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+            store_chunk_staged(xstage + (c & 1) * XBUF_BYTES, pk, &tm_out, p.out, p.N_out, row0,
                                static_cast<int64_t>(nb) * BN_OUT + c * 32, q, valid,
-                               valid <= BM / 2, c * 32 < cols_left, lane);
+                               valid <= BM / 2, c * 32 < cols_left, tma_rows, lane);
           } else if (row_ok && c * 32 < cols_left) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
@@ -674,6 +704,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
         }
       }
     }
+    if (lane == 0) bulk_wait_all();  // this warp's tensor stores have written y_perm
   }
 
   tc_fence_before();
@@ -1267,11 +1298,9 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tokn_kernel(
 
 // W_r [d, E] fp32 -> W' [E, 2d] bf16, row e = [hi(W[:, e]), lo(W[:, e])] with
 // hi = bf16(W), lo = bf16(W - hi), so that x . W = [x, x] . W' up to the rounding of lo (a
-// relative 2^-17 of each weight).  32 x 32 tiles transposed through shared memory.  Block
-// (0, 0) also writes the one-bucket table {start 0, count T} the grouped GEMM reads.
+// relative 2^-17 of each weight).  32 x 32 tiles transposed through shared memory.
 __global__ void __launch_bounds__(256) split_router_weight_kernel(
-    const float* __restrict__ w, int d, int E, __nv_bfloat16* __restrict__ wsplit,
-    int32_t* __restrict__ seg, int32_t T) {
+    const float* __restrict__ w, int d, int E, __nv_bfloat16* __restrict__ wsplit) {
   __shared__ float tile[32][33];
   const int e0 = blockIdx.x * 32, i0 = blockIdx.y * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -1289,10 +1318,6 @@ __global__ void __launch_bounds__(256) split_router_weight_kernel(
       wsplit[static_cast<int64_t>(e) * 2 * d + i] = h;
       wsplit[static_cast<int64_t>(e) * 2 * d + d + i] = l;
     }
-  }
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
-    seg[0] = 0;
-    seg[1] = T;
   }
 }
 
@@ -1337,6 +1362,18 @@ bool make_map_tokens(CUtensorMap* m, const void* base, int64_t rows, int64_t K) 
   return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [rows, N] bf16 row-major output, box 32 rows x 32 columns, 64-byte swizzle (epilogue stores)
+bool make_map_out(CUtensorMap* m, const void* base, int64_t rows, int64_t N) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N * 2)};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1456,14 +1493,15 @@ cudaError_t launch_ffn_tc(const Shape& s, const void* a, const int32_t* a_rows,
     *why = "cuTensorMapEncodeTiled is not available from the driver";
     return cudaErrorNotSupported;
   }
-  CUtensorMap ta1, tg, tu, ta2, td;
+  CUtensorMap ta1, tg, tu, ta2, td, ty;
   // gathered A is copied by the producer warp itself; the A map then only stays valid
   const bool a_ok = make_map_rows(&ta1, a, a_rows != nullptr ? s.T : s.max_rows, s.d);
   if (!a_ok ||
       !make_map_weights(&tg, wg, s.E, s.f, s.d, 128) ||
       !make_map_weights(&tu, wu, s.E, s.f, s.d, 128) ||
       !make_map_rows(&ta2, h, s.max_rows, s.f) ||
-      !make_map_weights(&td, wd, s.E, s.d, s.f, 256)) {
+      !make_map_weights(&td, wd, s.E, s.d, s.f, 256) ||
+      !make_map_out(&ty, y, s.max_rows, s.d)) {
     *why = "tensor map encoding failed (pointer alignment or sizes)";
     return cudaErrorInvalidValue;
   }
@@ -1564,8 +1602,8 @@ cudaError_t launch_ffn_tc(const Shape& s, const void* a, const int32_t* a_rows,
   p1.a_src = a;
   int64_t g1 = row_blocks_bound * p1.n_blocks;
   if (g1 > sms) g1 = sms;
-  grouped_gemm_tc_kernel<MODE_SWIGLU><<<static_cast<unsigned>(g1), THREADS, DYN_SMEM, st>>>(ta1, tg, tu,
-                                                                                    p1);
+  grouped_gemm_tc_kernel<MODE_SWIGLU><<<static_cast<unsigned>(g1), THREADS, DYN_SMEM, st>>>(
+      ta1, tg, tu, ty, p1);
   note_launch();
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
 
@@ -1596,41 +1634,55 @@ cudaError_t launch_ffn_tc(const Shape& s, const void* a, const int32_t* a_rows,
   }
   int64_t g2 = row_blocks_bound * p2.n_blocks;
   if (g2 > sms) g2 = sms;
-  grouped_gemm_tc_kernel<MODE_DOWN><<<static_cast<unsigned>(g2), THREADS, DYN_SMEM, st>>>(ta2, td, td,
-                                                                                     p2);
+  grouped_gemm_tc_kernel<MODE_DOWN><<<static_cast<unsigned>(g2), THREADS, DYN_SMEM, st>>>(
+      ta2, td, td, ty, p2);
   note_launch();
   return cudaGetLastError();
 }
 
 bool router_uses_tensor_cores(const Shape& s) {
-  return s.dtype == MOE_BF16 && s.E > 32 && s.d % 64 == 0 && s.T >= 512;
+  return router_split_applies(s) && s.T >= 512;
+}
+
+bool router_split_applies(const Shape& s) {
+  return s.dtype == MOE_BF16 && s.E > 32 && s.d % 64 == 0;
+}
+
+size_t router_split_bytes(const Shape& s) {
+  if (!router_split_applies(s)) return 0;
+  return 2 * static_cast<size_t>(s.E) * s.d * sizeof(__nv_bfloat16);
 }
 
 size_t router_tc_workspace_bytes(const Shape& s) {
-  if (!router_uses_tensor_cores(s)) return 0;
-  return 256 + 2 * static_cast<size_t>(s.E) * s.d * sizeof(__nv_bfloat16);
+  return router_uses_tensor_cores(s) ? router_split_bytes(s) : 0;
+}
+
+cudaError_t launch_router_split(const Shape& s, const float* w_router, void* w_split,
+                                cudaStream_t st) {
+  dim3 sgrid((s.E + 31) / 32, static_cast<unsigned>((s.d + 31) / 32));
+  split_router_weight_kernel<<<sgrid, 256, 0, st>>>(w_router, static_cast<int>(s.d), s.E,
+                                                    static_cast<__nv_bfloat16*>(w_split));
+  note_launch();
+  return cudaGetLastError();
 }
 
 cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_router,
-                             const float* bias, int64_t bias_stride, float* logits,
-                             float* logits_scratch, int32_t* topk_idx, float* topk_w,
-                             void* split_ws, DevStatus* status, uint64_t wait_ns,
+                             const void* w_split, const float* bias, int64_t bias_stride,
+                             float* logits, float* logits_scratch, int32_t* topk_idx,
+                             float* topk_w, void* split_ws, DevStatus* status, uint64_t wait_ns,
                              cudaStream_t st, const char** why) {
   if (encode_fn() == nullptr) {
     *why = "cuTensorMapEncodeTiled is not available from the driver";
     return cudaErrorNotSupported;
   }
-  int32_t* seg = static_cast<int32_t*>(split_ws);
-  __nv_bfloat16* wsplit = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(split_ws) + 256);
-  dim3 sgrid((s.E + 31) / 32, static_cast<unsigned>((s.d + 31) / 32));
-  split_router_weight_kernel<<<sgrid, 256, 0, st>>>(w_router, static_cast<int>(s.d), s.E, wsplit,
-                                                    seg, static_cast<int32_t>(s.T));
-  note_launch();
-  cudaError_t err = cudaGetLastError();
-  if (err != cudaSuccess) return err;
+  cudaError_t err;
+  if (w_split == nullptr) {  // split W_r into the workspace for this call
+    if ((err = launch_router_split(s, w_router, split_ws, st)) != cudaSuccess) return err;
+    w_split = split_ws;
+  }
   // all E <= 256 experts in one 256-column accumulator: K = 2 d (hi half, then lo half)
   CUtensorMap ta, tw;
-  if (!make_map_rows(&ta, x, s.T, s.d) || !make_map_weights(&tw, wsplit, 1, s.E, 2 * s.d, 256)) {
+  if (!make_map_rows(&ta, x, s.T, s.d) || !make_map_weights(&tw, w_split, 1, s.E, 2 * s.d, 256)) {
     *why = "tensor map encoding failed for the router";
     return cudaErrorInvalidValue;
   }
@@ -1641,8 +1693,7 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_route
   // the top-k rides in the epilogue unless the picks are limited to groups
   const bool fuse = s.n_groups <= 1;
   TcParams p = {};
-  p.seg_start = seg;
-  p.seg_count = seg + 1;
+  p.router_rows = static_cast<int32_t>(s.T);
   p.E = 1;
   p.K = static_cast<int>(2 * s.d);
   p.a_k = static_cast<int>(s.d);
@@ -1666,7 +1717,7 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_route
   int64_t g = (s.T + BM - 1) / BM;
   if (g > sm_count()) g = sm_count();
   grouped_gemm_tc_kernel<MODE_ROUTER><<<static_cast<unsigned>(g), THREADS, DYN_SMEM, st>>>(
-      ta, tw, tw, p);
+      ta, tw, tw, tw, p);
   note_launch();
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   if (fuse) return cudaSuccess;

@@ -64,14 +64,20 @@ int router_splits(const Shape& s);
 cudaError_t launch_router(const Shape& s, const void* x, const float* w_router,
                           const float* bias, int64_t bias_stride, float* logits,
                           int32_t* topk_idx, float* topk_w, float* partials, cudaStream_t st);
-// Router on tensor cores (bf16 layers, E > 32): W_r split into two bf16 terms.
+// Router on tensor cores (bf16 layers, E > 32, d % 64 == 0, T >= 512): W_r split into two
+// bf16 terms, W' = [E, 2 d] (hi | lo along K).
 bool router_uses_tensor_cores(const Shape& s);
-// logits: the caller's [T, E] buffer, or nullptr (then z goes to logits_scratch, the
-// workspace copy).
+bool router_split_applies(const Shape& s);   // the layer shape admits the split (any T)
+size_t router_split_bytes(const Shape& s);   // bytes of W' (0 when the split does not apply)
+cudaError_t launch_router_split(const Shape& s, const float* w_router, void* w_split,
+                                cudaStream_t st);
+// w_split: W' made earlier by launch_router_split, or nullptr (then W_r is split into
+// split_ws for this call).  logits: the caller's [T, E] buffer, or nullptr (then z goes to
+// logits_scratch, the workspace copy).
 cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_router,
-                             const float* bias, int64_t bias_stride, float* logits,
-                             float* logits_scratch, int32_t* topk_idx, float* topk_w,
-                             void* split_ws, DevStatus* status, uint64_t wait_ns,
+                             const void* w_split, const float* bias, int64_t bias_stride,
+                             float* logits, float* logits_scratch, int32_t* topk_idx,
+                             float* topk_w, void* split_ws, DevStatus* status, uint64_t wait_ns,
                              cudaStream_t st, const char** why);
 size_t router_tc_workspace_bytes(const Shape& s);
 cudaError_t launch_topk_from_logits(const Shape& s, const float* logits, const float* bias,

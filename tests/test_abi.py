@@ -41,7 +41,7 @@ def test_every_declared_symbol_is_exported(lib):
     assert not missing, missing
     for n in names:
         assert getattr(lib, n) is not None
-    assert lib.moe_abi_version() == 4
+    assert lib.moe_abi_version() == 5
 
 
 def test_struct_layout_matches_header(tmp_path):
@@ -249,3 +249,32 @@ def test_ffn_kernel_choice_is_checked(lib):
     assert lib.moe_set_ffn_kernel(3) == 1    # MOE_ERR_INVALID_ARG
     assert lib.moe_set_ffn_kernel(-1) == 1
     assert b"moe_set_ffn_kernel" in lib.moe_last_error()
+
+
+def test_router_split_sizes_and_checks(lib):
+    """The split router weight: 2 E d bf16 values where the layer can take the tensor-core
+    router (bf16, E > 32, d a multiple of 64; T does not matter), none otherwise; the
+    argument checks run on the host before anything is enqueued."""
+    L = lib
+    big = M.make_config(256, 512, 128, 256, 8, dtype=M.BF16)
+    small_t = M.make_config(16, 512, 128, 256, 8, dtype=M.BF16)
+    assert M.router_split_size(big) == 2 * 256 * 512 * 2
+    assert M.router_split_size(small_t) == M.router_split_size(big)
+    for cfg in (M.make_config(256, 512, 128, 8, 2, dtype=M.BF16),      # E <= 32
+                M.make_config(256, 512, 128, 256, 8, dtype=M.F32),     # fp32 layer
+                M.make_config(256, 96, 128, 256, 8, dtype=M.BF16)):    # d % 64 != 0
+        assert M.router_split_size(cfg) == 0
+        st = L.moe_router_split(ctypes.byref(cfg), 16, 256, 1 << 20, None)
+        assert st == 2 and b"tensor-core router" in L.moe_last_error()  # MOE_ERR_UNSUPPORTED
+    n = M.router_split_size(big)
+    assert L.moe_router_split(ctypes.byref(big), None, 256, n, None) == 1
+    assert L.moe_router_split(ctypes.byref(big), 16, 258, n, None) == 1   # misaligned
+    assert L.moe_router_split(ctypes.byref(big), 16, 256, n - 2, None) == 1
+    assert b"split_bytes" in L.moe_last_error()
+    ws_bytes = M.workspace_size(big)
+    st = L.moe_route_ex(ctypes.byref(big), 16, 16, 258, None, 0, None, 16, 16, 256, ws_bytes,
+                        None)
+    assert st == 1 and b"w_router_split" in L.moe_last_error()
+    st = L.moe_route_ex(ctypes.byref(big), 16, None, 256, None, 0, None, 16, 16, 256, ws_bytes,
+                        None)
+    assert st == 1   # w_router is required even with a split

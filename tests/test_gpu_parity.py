@@ -301,6 +301,43 @@ def test_tensor_core_router_without_logits_buffer(shape):
     assert r["idx"].shape == (shape.T, shape.k)
 
 
+@pytest.mark.parametrize("shape", [
+    W.reduced(W.DSV3_PREFILL_ZIPF, 1000, 256, 128),                        # tensor-core router
+    W.reduced(W.DSV3_PREFILL_ZIPF, 1088, 320, 128, E=200, bias="chunks", bias_mode=1,
+              n_decode_tokens=8),                                          # masked experts
+    W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256, n_groups=8, topk_groups=4),  # + top-k kernel
+    W.reduced(W.DSV3_PREFILL_ZIPF, 300, 256, 128),                         # fp32 router: ignored
+], ids=["tc", "tc_E200_selbias", "tc_groups", "fp32_T300"])
+def test_presplit_router_weight_equals_split_per_call(shape):
+    """moe_route_ex given the split W_r of moe_router_split: logits, picks and weights bitwise
+    those of moe_route (which splits W_r at every call), with one launch fewer where the
+    tensor-core router runs; and the split itself is [hi(W_r^T) | lo(W_r^T)] in bf16."""
+    run = GpuRun(shape)
+    run.route()
+    b, i = run.b, run.inp
+    z, idx, w = b.logits.clone(), b.topk_idx.clone(), b.topk_w.clone()
+    split = M.router_split(run.cfg, i.w_router)
+    assert split is not None and split.numel() == 2 * shape.E * shape.d_model * 2
+    wt = i.w_router.t().contiguous()                          # [E, d] fp32
+    hi = wt.to(torch.bfloat16)
+    lo = (wt - hi.float()).to(torch.bfloat16)
+    torch.cuda.synchronize()
+    assert torch.equal(split.view(torch.bfloat16).view(shape.E, 2 * shape.d_model),
+                       torch.cat([hi, lo], dim=1))
+    b.logits.fill_(-7.0), b.topk_idx.fill_(-7), b.topk_w.fill_(-7.0)
+    c0 = M.kernel_launch_count()
+    M.moe_route_ex(run.cfg, i.x, i.w_router, split, i.logit_bias, b.logits, b.topk_idx,
+                   b.topk_w, run.ws)
+    launched = M.kernel_launch_count() - c0
+    M.moe_check_device_error(run.ws)
+    torch.cuda.synchronize()
+    assert torch.equal(b.logits, z) and torch.equal(b.topk_idx, idx) and torch.equal(b.topk_w, w)
+    tc = shape.T >= 512
+    assert launched == (1 if tc and shape.n_groups <= 1 else 2)
+    run.dispatch()
+    check_routing(run)
+
+
 def test_bad_expert_index_is_reported_not_faulted():
     shape = _edge(50, 64, 64, 8, 2)
     run = GpuRun(shape)
@@ -360,20 +397,22 @@ def test_small_e_router_wide_d(shape):
 
 
 # ------------------------------------------------------------------ launch accounting
-@pytest.mark.parametrize("shape,router_kernels", [
-    (W.reduced(W.MIXTRAL_8X7B, 1000, 512, 768), 2),          # lane-ordered W_r + fused router
-    (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256), 2),     # W_r split + GEMM with the top-k
-    (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256, n_groups=8, topk_groups=4), 3),  # + top-k
-    (W.reduced(W.DSV3_DECODE, 128, 512, 256), 2),            # split-K fp32 GEMM + top-k
+@pytest.mark.parametrize("shape,router_kernels,dispatch_kernels", [
+    (W.reduced(W.MIXTRAL_8X7B, 1000, 512, 768), 2, 2),          # lane-ordered W_r + fused router
+    (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256), 2, 2),     # W_r split + GEMM with the top-k
+    (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256, n_groups=8, topk_groups=4), 3, 2),  # + top-k
+    (W.reduced(W.DSV3_DECODE, 128, 512, 256), 2, 2),            # split-K fp32 GEMM + top-k
+    (W.reduced(W.DSV3_PREFILL_ZIPF, 4200, 256, 128), 2, 3),     # 33600 picks: count kernel too
 ])
-def test_kernel_launch_count_per_layer(shape, router_kernels):
-    """One staged layer forward launches the router's kernels, count + rank + permute, the two
-    grouped GEMMs, combine and stats -- and the library's own counter says so."""
+def test_kernel_launch_count_per_layer(shape, router_kernels, dispatch_kernels):
+    """One staged layer forward launches the router's kernels, the ranking (one self-counting
+    kernel up to 32768 picks, count + rank above) and the permute, the two grouped GEMMs,
+    combine and stats -- and the library's own counter says so."""
     run = GpuRun(shape)
     run.all_stages()
     c0 = M.kernel_launch_count()
     run.all_stages()
-    assert M.kernel_launch_count() - c0 == router_kernels + 3 + 2 + 1 + 1
+    assert M.kernel_launch_count() - c0 == router_kernels + dispatch_kernels + 2 + 1 + 1
 
 
 # ------------------------------------------------------------------ dispatch without x_perm
@@ -431,7 +470,7 @@ def test_layer_forward_without_x_perm(shape):
     M.moe_check_device_error(layer.ws)
     torch.cuda.synchronize()
     assert torch.equal(out, run.b.out)
-    assert launched == 8    # router (2), count + rank, two FFN launches, combine, stats: no permute
+    assert launched == 7    # router (2), ranking (1), two FFN launches, combine, stats: no permute
 
 
 # ------------------------------------------------------------------ combine fused into the FFN
