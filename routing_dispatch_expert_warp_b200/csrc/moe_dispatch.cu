@@ -147,47 +147,53 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
       (&self_bef[0][0])[i] = 0;
     }
     __syncthreads();
-    // warp w takes tokens 32 w + 256 n + lane, one pick slot j at a time, the loads of 8
-    // batches in flight together; a 32-token batch lies wholly before this block's first
-    // token or wholly at or after it
-    constexpr int U = 8;
+    // The picks in memory order, i = t k + j: thread l of the block takes picks
+    // 256 (16 n + u) + l, u < 16, their loads in flight together.  A warp's 32 picks of one
+    // u are consecutive and start at a multiple of 32, and this block's first pick
+    // t_lo k is a multiple of 256, so they lie wholly before it or wholly at or after it.
+    // One count plane: E <= 32 counts by ballots into lane registers; otherwise (or with a
+    // plane per pick rank) the lanes holding the same (expert, plane) add their number once.
+    constexpr int U = 16;
     const int lane = threadIdx.x & 31;
-    const int64_t t_lo = static_cast<int64_t>(blockIdx.x) * kDispatchBlockTokens;
-    for (int j = 0; j < k; ++j) {
-      const int p = planes > 1 ? j : 0;
-      int tot = 0, bef = 0;  // E <= 32: lane ee's counts of expert ee
-      for (int64_t tb = (threadIdx.x >> 5) * 32; tb < T; tb += U * kDispatchBlockTokens) {
-        int ev[U];
+    const int64_t picks = T * k;
+    const int64_t i_lo = static_cast<int64_t>(blockIdx.x) * kDispatchBlockTokens * k;
+    const bool ballots = planes == 1 && E <= 32;
+    int tot = 0, bef = 0;  // ballots: lane x's counts of expert x
+    for (int64_t ib = threadIdx.x & ~31; ib < picks; ib += U * kDispatchBlockTokens) {
+      int ev[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int64_t t = tb + u * kDispatchBlockTokens + lane;
-          ev[u] = t < T ? __ldg(topk_idx + t * k + j) : -1;
-        }
+      for (int u = 0; u < U; ++u) {
+        const int64_t i = ib + u * kDispatchBlockTokens + lane;
+        ev[u] = i < picks ? __ldg(topk_idx + i) : -1;
+      }
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int ee = (ev[u] < 0 || ev[u] >= E) ? -1 : ev[u];
-          const bool early = tb + u * kDispatchBlockTokens < t_lo;
-          if (E <= 32) {
-            for (int x = 0; x < E; ++x) {
-              const int c = __popc(__ballot_sync(0xffffffffu, ee == x));
-              if (lane == x) {
-                tot += c;
-                if (early) bef += c;
-              }
+      for (int u = 0; u < U; ++u) {
+        const int64_t i0 = ib + u * kDispatchBlockTokens;
+        if (i0 >= picks) break;  // the same for the whole warp
+        const int ee = (ev[u] < 0 || ev[u] >= E) ? -1 : ev[u];
+        const bool early = i0 < i_lo;
+        if (ballots) {
+          for (int x = 0; x < E; ++x) {
+            const int c = __popc(__ballot_sync(0xffffffffu, ee == x));
+            if (lane == x) {
+              tot += c;
+              if (early) bef += c;
             }
-          } else {
-            const uint32_t grp = __match_any_sync(0xffffffffu, ee);
-            if (ee >= 0 && lane == __ffs(grp) - 1) {
-              atomicAdd(&self_tot[p][ee], __popc(grp));
-              if (early) atomicAdd(&self_bef[p][ee], __popc(grp));
-            }
+          }
+        } else {
+          const int p = planes > 1 ? static_cast<int>((i0 + lane) % k) : 0;
+          const int key = ee < 0 ? -1 : ee * MOE_MAX_TOPK + p;
+          const uint32_t grp = __match_any_sync(0xffffffffu, key);
+          if (ee >= 0 && lane == __ffs(grp) - 1) {
+            atomicAdd(&self_tot[p][ee], __popc(grp));
+            if (early) atomicAdd(&self_bef[p][ee], __popc(grp));
           }
         }
       }
-      if (E <= 32 && lane < E) {
-        atomicAdd(&self_tot[p][lane], tot);
-        atomicAdd(&self_bef[p][lane], bef);
-      }
+    }
+    if (ballots && lane < E) {
+      atomicAdd(&self_tot[0][lane], tot);
+      atomicAdd(&self_bef[0][lane], bef);
     }
     __syncthreads();
   }
