@@ -51,6 +51,9 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = MMA_N * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int THREADS = 192;
+// the router mode runs 8 epilogue warps: two per TMEM lane quarter, each taking half of the
+// 256 expert columns of its 32 tokens, their two top-k lists merged through shared memory
+constexpr int ROUTER_THREADS = 320;
 constexpr int ACC_COLS = 256;
 constexpr int TMEM_COLS = 512;
 // per epilogue warp: two buffers of 32 rows x 64 bytes (one 32-column chunk of bf16) in the
@@ -212,7 +215,7 @@ __device__ __forceinline__ void store_chunk_staged(uint8_t* buf, const uint32_t 
 // tm_out (MODE_DOWN): the output y_perm [rows, N_out], 32 x 32 boxes, 64-byte swizzle, for
 // the epilogue's tensor stores; the other modes do not read it.
 template <int MODE>
-__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
+__global__ void __launch_bounds__(MODE == 2 ? ROUTER_THREADS : THREADS, 1) grouped_gemm_tc_kernel(
     const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
     const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_out,
     const TcParams p) {
@@ -224,10 +227,13 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
   __shared__ __align__(8) uint64_t tfull_bar[2];
   __shared__ __align__(8) uint64_t tempty_bar[2];
   __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ __align__(8) uint64_t mfull_bar;   // router: the upper-half lists are written
+  __shared__ __align__(8) uint64_t mempty_bar;  // router: ... and read
   __shared__ uint32_t tmem_base_s;
   __shared__ volatile int abort_s;
   __shared__ int tile_base[MOE_MAX_EXPERTS + 1];
   __shared__ int mblocks[MOE_MAX_EXPERTS];
+  constexpr unsigned EPI_THREADS = MODE == MODE_ROUTER ? ROUTER_THREADS - 64 : THREADS - 64;
 
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -274,9 +280,11 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull_bar[a], 1);
-      mbar_init(&tempty_bar[a], 128);
+      mbar_init(&tempty_bar[a], EPI_THREADS);
     }
     mbar_init(&drain_bar, 1);
+    mbar_init(&mfull_bar, 128);
+    mbar_init(&mempty_bar, 128);
     abort_s = 0;
     fence_barrier_init();
   }
@@ -300,6 +308,14 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
         int e, mb, nb;
         decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, p.mb_outer, e, mb, nb);
         const int row0 = seg_start(e) + mb * BM;
+        // The router's tiles all read the same split weight: tile t starts its K loop at
+        // chunk pair t * pairs / tiles and wraps, so the blocks in flight read different parts
+        // of it at any moment instead of all the same lines at once.  (The fp32 sum then runs
+        // in a per-tile order: deterministic, a rounding-level difference per tile.)
+        const int pairs = KB >> 1;
+        const int rot = MODE == MODE_ROUTER
+                            ? static_cast<int>(static_cast<int64_t>(tile) * pairs / total_tiles)
+                            : 0;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty_bar[s], ph ^ 1u, p.wait_ns, &abort_s)) {
             if (!abort_s)
@@ -315,8 +331,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
           armed_parity = (armed_parity & ~(1u << s)) | (ph << s);
           // the router takes each 64-wide chunk of its x rows twice in a row, against the hi
           // and then the lo half of the split weight (the second read hits L2)
-          const int a_col = MODE == MODE_ROUTER ? (kb >> 1) * BK : kb * BK;
-          const int b_col = MODE == MODE_ROUTER ? (kb & 1) * p.a_k + (kb >> 1) * BK : kb * BK;
+          int pr = (kb >> 1) + rot;
+          if (pr >= pairs) pr -= pairs;
+          const int a_col = MODE == MODE_ROUTER ? pr * BK : kb * BK;
+          const int b_col = MODE == MODE_ROUTER ? (kb & 1) * p.a_k + pr * BK : kb * BK;
           tma_load_2d(sa, &tm_a, &full_bar[s], a_col, row0);
           if (GATED) {
             tma_load_3d(sb, &tm_b0, &full_bar[s], b_col, nb * 128, e);
@@ -474,8 +492,11 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
     const int q = warp & 3;             // TMEM lane quarter this warp may access
     const int r = q * 32 + lane;        // accumulator row owned by this thread
     uint8_t* xstage = smem + STAGES * STAGE_BYTES + (warp - 2) * XSTAGE_BYTES;
+    // router: warps 2-5 take expert columns [0, 128), warps 6-9 [128, 256)
+    const int half = MODE == MODE_ROUTER ? (warp - 2) >> 2 : 0;
     int acc = 0;
     uint32_t aph = 0;
+    uint32_t mph = 0;  // router: phase of the list handoff
     for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
       int e, mb, nb;
       decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, p.mb_outer, e, mb, nb);
@@ -517,8 +538,28 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
         }
         uint32_t thr = 0u;  // key of the k-th best so far
         const uint32_t kth_mask = 1u << (p.k - 1);
+        // (key, expert, logit) into the list behind the equal keys it holds; static indices
+        auto insert = [&](uint32_t key, int col, float zv) {
+#pragma unroll
+          for (int j = MOE_MAX_TOPK - 1; j > 0; --j) {
+            if (key > tk[j - 1]) {
+              tk[j] = tk[j - 1];
+              ti[j] = ti[j - 1];
+              tz[j] = tz[j - 1];
+            } else if (key > tk[j]) {
+              tk[j] = key;
+              ti[j] = col;
+              tz[j] = zv;
+            }
+          }
+          if (key > tk[0]) {
+            tk[0] = key;
+            ti[0] = col;
+            tz[0] = zv;
+          }
+        };
 #pragma unroll 1
-        for (int c = 0; c < BN_OUT / 32; ++c) {
+        for (int c = 4 * half; c < 4 * half + 4; ++c) {
           uint32_t v[32];
           tmem_ld32(taddr + c * 32, v);
           tmem_ld_wait();
@@ -571,24 +612,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
                     bz = z[i];
                     key[i] = 0u;
                   }
-                const int col = c * 32 + bi;
-#pragma unroll
-                for (int j = MOE_MAX_TOPK - 1; j > 0; --j) {
-                  if (best > tk[j - 1]) {
-                    tk[j] = tk[j - 1];
-                    ti[j] = ti[j - 1];
-                    tz[j] = tz[j - 1];
-                  } else if (best > tk[j]) {
-                    tk[j] = best;
-                    ti[j] = col;
-                    tz[j] = bz;
-                  }
-                }
-                if (best > tk[0]) {
-                  tk[0] = best;
-                  ti[0] = col;
-                  tz[0] = bz;
-                }
+                insert(best, c * 32 + bi, bz);
                 // thr = tk[k - 1], as arithmetic on a one-hot mask (no indexed access)
                 thr = 0u;
 #pragma unroll
@@ -598,7 +622,50 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_tc_kernel(
             }
           }
         }
-        if (p.fuse_topk && row_ok) {
+        if (p.fuse_topk) {
+          // the upper half hands its list to the lower half's thread of the same token, which
+          // inserts it behind its own (the upper experts lose ties); both waits are bounded
+          uint32_t* mk = reinterpret_cast<uint32_t*>(smem + STAGES * STAGE_BYTES);
+          int32_t* mi = reinterpret_cast<int32_t*>(mk + BM * MOE_MAX_TOPK);
+          float* mz = reinterpret_cast<float*>(mi + BM * MOE_MAX_TOPK);
+          const int slot = r * MOE_MAX_TOPK;
+          int mok = 1;
+          if (lane == 0)
+            mok = mbar_wait(half ? &mempty_bar : &mfull_bar, half ? mph ^ 1u : mph, p.wait_ns,
+                            &abort_s) ? 1 : 0;
+          mok = __shfl_sync(0xffffffffu, mok, 0);
+          if (!mok) {
+            if (lane == 0 && !abort_s)
+              record_error(p.status, DEV_TIMEOUT, 24, static_cast<unsigned long long>(tile));
+            abort_s = 1;
+            break;
+          }
+          if (half) {
+#pragma unroll
+            for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+              mk[slot + j] = tk[j];
+              mi[slot + j] = ti[j];
+              mz[slot + j] = tz[j];
+            }
+            mbar_arrive(&mfull_bar);
+          } else {
+            uint32_t ok2[MOE_MAX_TOPK];
+            int oi[MOE_MAX_TOPK];
+            float oz[MOE_MAX_TOPK];
+#pragma unroll
+            for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+              ok2[j] = mk[slot + j];
+              oi[j] = mi[slot + j];
+              oz[j] = mz[slot + j];
+            }
+            mbar_arrive(&mempty_bar);
+#pragma unroll
+            for (int j = 0; j < MOE_MAX_TOPK; ++j)
+              if (j < p.k) insert(ok2[j], oi[j], oz[j]);
+          }
+          mph ^= 1u;
+        }
+        if (p.fuse_topk && row_ok && half == 0) {
           // gate weights over the k picks, the normaliser summed in pick order
           float w[MOE_MAX_TOPK];
           float m = tz[0];
@@ -1716,7 +1783,7 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_route
   p.wait_ns = wait_ns;
   int64_t g = (s.T + BM - 1) / BM;
   if (g > sm_count()) g = sm_count();
-  grouped_gemm_tc_kernel<MODE_ROUTER><<<static_cast<unsigned>(g), THREADS, DYN_SMEM, st>>>(
+  grouped_gemm_tc_kernel<MODE_ROUTER><<<static_cast<unsigned>(g), ROUTER_THREADS, DYN_SMEM, st>>>(
       ta, tw, tw, tw, p);
   note_launch();
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
