@@ -204,6 +204,25 @@ class ClockSampler:
                 "window": "timed region" if inside else "whole sampling period"}
 
 
+def tensor_core_router(shape) -> bool:
+    """The layer shapes whose router runs on the tensor cores (moe_route's rule)."""
+    return (shape.dtype == W.BF16 and shape.E > 32 and shape.d_model % 64 == 0
+            and shape.T >= 512)
+
+
+def route_tensor_roof(shape, work: dict, route_ms: float, peaks: dict) -> dict:
+    """For the tensor-core router, the route stage against the tensor roof: it executes the
+    contraction twice (x against the bf16 hi and lo terms of W_r), 4 T d E FLOP for the
+    2 T d E of the definition."""
+    if not tensor_core_router(shape) or route_ms <= 0:
+        return {}
+    executed = 2.0 * work["route_flops"]
+    tf = executed / (route_ms * 1e-3) / 1e12
+    return {"bound": "tensor (two bf16 terms of W_r)",
+            "executed_TFLOP/s": tf, "frac_tensor": tf / peaks["bf16_tflops"],
+            "algorithmic_TFLOP/s": work["route_flops"] / (route_ms * 1e-3) / 1e12}
+
+
 def algorithmic_work(shape, kept_total: int) -> dict:
     T, d, f, E, k, s = (shape.T, shape.d_model, shape.d_ff, shape.E, shape.k,
                         2 if shape.dtype == W.BF16 else 4)
@@ -211,6 +230,7 @@ def algorithmic_work(shape, kept_total: int) -> dict:
     return {
         "gemm_flops": 6.0 * d * f * kept_total,
         "route_bytes": T * d * s + d * E * 4 + T * E * 4 + T * k * 8,
+        "route_flops": 2.0 * T * d * E,
         "permute_bytes": T * d * s + kept_total * d * s + A * 4,
         "combine_bytes": kept_total * d * s + A * 8 + T * d * s,
     }
@@ -506,8 +526,11 @@ def run_gpu(args) -> None:
                 traffic_source=(recorded_traffic(shape.name, args.gather) or {}).get("profile")),
             "stages_ms": {n: sum(v) / args.steps for n, v in per_stage.items()},
             "stage_bandwidth": {
-                "route": {"GB/s": gbs(work["route_bytes"], "route"),
-                          "frac_hbm": gbs(work["route_bytes"], "route") / peaks["hbm_gbs"]},
+                "route": dict(
+                    {"GB/s": gbs(work["route_bytes"], "route"),
+                     "frac_hbm": gbs(work["route_bytes"], "route") / peaks["hbm_gbs"]},
+                    **route_tensor_roof(shape, work, sum(per_stage["route"]) / args.steps,
+                                        peaks)),
                 "dispatch": ({"us": sum(per_stage["dispatch"]) / args.steps * 1e3,
                               "note": "bookkeeping only (no copy)"} if args.gather else
                              {"GB/s": gbs(work["permute_bytes"], "dispatch"),
