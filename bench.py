@@ -44,10 +44,10 @@ GEMM_SOURCES = ("routing_dispatch_expert_warp_b200/csrc/moe_ffn_tc.cu",
                 "routing_dispatch_expert_warp_b200/csrc/moe_internal.h")
 RECORDED_GEMM_TRAFFIC = {
     ("mixtral8x7b_prefill_T4096", False): {
-        "bytes": 3668596480, "sources": "04a5ee3b94545cd0",
+        "bytes": 3668160256, "sources": "7efdcc28b3b4f6ee",
         "profile": "profiles/grouped_gemm_tc_mixtral8x7b_T4096_traffic.md"},
     ("dsv3_prefill_zipf_T16384", False): {
-        "bytes": 27450647296, "sources": "04a5ee3b94545cd0",
+        "bytes": 27309186048, "sources": "7efdcc28b3b4f6ee",
         "profile": "profiles/grouped_gemm_tc_dsv3_prefill_T16384_traffic.md"},
 }
 

@@ -27,9 +27,6 @@
 //              Writes assign_row and token_of_row (-1 for rows no assignment uses).
 //   3. permute: token-major row copy with bulk (TMA) copies: each row of x is read from HBM
 //              once into shared memory and written to each of its kept rows of x_perm.
-// With at most kSelfCountMaxPicks picks and no score filter, 1 and 2 are one launch: every
-// rank block counts all picks itself (a few KB of topk_idx from L2) instead of reading the
-// count kernel's per-block histograms.
 #include <mutex>
 
 #include "moe_internal.h"
@@ -118,18 +115,11 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_count_kernel(
 // rows no assignment uses are marked -1 in token_of_row.  With a filter, hist counts the
 // kept picks only, the others get row -1, and routed (the demand, counted by an earlier
 // unfiltered pass) is left as it is.
-//
-// SELF_COUNT (no filter, few picks): there is no count kernel and no hist.  Every block
-// counts all T x k picks itself -- per plane and expert, the total and the part from tokens
-// before its own -- which is what the sums over hist give; it also records invalid experts.
-constexpr int64_t kSelfCountMaxPicks = 32768;
-
-template <bool SELF_COUNT>
 __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
     const int32_t* __restrict__ topk_idx, int64_t T, int k, int E, int64_t C, int layout,
     int planes, int64_t nblk, const int32_t* __restrict__ hist, int32_t* __restrict__ routed,
     int32_t* __restrict__ kept, int32_t* __restrict__ offsets, int32_t* __restrict__ assign_row,
-    int32_t* __restrict__ token_of_row, int64_t max_rows, ScoreFilter flt, DevStatus* status) {
+    int32_t* __restrict__ token_of_row, int64_t max_rows, ScoreFilter flt) {
   static_assert(kDispatchBlockTokens == MOE_MAX_EXPERTS, "one thread per expert");
   __shared__ uint32_t masks[kWarps][MOE_MAX_EXPERTS];
   __shared__ int32_t wbase[kWarps][MOE_MAX_EXPERTS];
@@ -137,77 +127,12 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
   __shared__ int32_t off_s[MOE_MAX_EXPERTS];
   __shared__ int32_t kept_s[MOE_MAX_EXPERTS];
   __shared__ int64_t scan[MOE_MAX_EXPERTS];
-  __shared__ int32_t self_tot[SELF_COUNT ? MOE_MAX_TOPK : 1][MOE_MAX_EXPERTS];
-  __shared__ int32_t self_bef[SELF_COUNT ? MOE_MAX_TOPK : 1][MOE_MAX_EXPERTS];
 
   const int e = threadIdx.x;
-  if (SELF_COUNT) {
-    for (int i = threadIdx.x; i < planes * MOE_MAX_EXPERTS; i += blockDim.x) {
-      (&self_tot[0][0])[i] = 0;
-      (&self_bef[0][0])[i] = 0;
-    }
-    __syncthreads();
-    // The picks in memory order, i = t k + j: thread l of the block takes picks
-    // 256 (16 n + u) + l, u < 16, their loads in flight together.  A warp's 32 picks of one
-    // u are consecutive and start at a multiple of 32, and this block's first pick
-    // t_lo k is a multiple of 256, so they lie wholly before it or wholly at or after it.
-    // One count plane: E <= 32 counts by ballots into lane registers; otherwise (or with a
-    // plane per pick rank) the lanes holding the same (expert, plane) add their number once.
-    constexpr int U = 16;
-    const int lane = threadIdx.x & 31;
-    const int64_t picks = T * k;
-    const int64_t i_lo = static_cast<int64_t>(blockIdx.x) * kDispatchBlockTokens * k;
-    const bool ballots = planes == 1 && E <= 32;
-    int tot = 0, bef = 0;  // ballots: lane x's counts of expert x
-    for (int64_t ib = threadIdx.x & ~31; ib < picks; ib += U * kDispatchBlockTokens) {
-      int ev[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t i = ib + u * kDispatchBlockTokens + lane;
-        ev[u] = i < picks ? __ldg(topk_idx + i) : -1;
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t i0 = ib + u * kDispatchBlockTokens;
-        if (i0 >= picks) break;  // the same for the whole warp
-        const int ee = (ev[u] < 0 || ev[u] >= E) ? -1 : ev[u];
-        const bool early = i0 < i_lo;
-        if (ballots) {
-          for (int x = 0; x < E; ++x) {
-            const int c = __popc(__ballot_sync(0xffffffffu, ee == x));
-            if (lane == x) {
-              tot += c;
-              if (early) bef += c;
-            }
-          }
-        } else {
-          const int p = planes > 1 ? static_cast<int>((i0 + lane) % k) : 0;
-          const int key = ee < 0 ? -1 : ee * MOE_MAX_TOPK + p;
-          const uint32_t grp = __match_any_sync(0xffffffffu, key);
-          if (ee >= 0 && lane == __ffs(grp) - 1) {
-            atomicAdd(&self_tot[p][ee], __popc(grp));
-            if (early) atomicAdd(&self_bef[p][ee], __popc(grp));
-          }
-        }
-      }
-    }
-    if (ballots && lane < E) {
-      atomicAdd(&self_tot[0][lane], tot);
-      atomicAdd(&self_bef[0][lane], bef);
-    }
-    __syncthreads();
-  }
   int64_t run = 0;  // routed total over all planes
   if (e < E) {
     for (int p = 0; p < planes; ++p) {
       int64_t tot = 0, before = 0;
-      if (SELF_COUNT) {
-        tot = self_tot[p][e];
-        before = self_bef[p][e];
-        pbase[p][e] = static_cast<int32_t>(run + before);
-        run += tot;
-        continue;
-      }
       int64_t b = 0;
       for (; b + 8 <= nblk; b += 8) {  // loads issued 8 at a time, sums in block order
         int32_t c[8];
@@ -258,8 +183,7 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
   const uint32_t below = (1u << (threadIdx.x & 31)) - 1u;
   for (int p = 0; p < planes; ++p) {
     __syncthreads();  // pbase / off_s ready; masks of the previous plane no longer read
-    build_masks(topk_idx, T, k, E, masks, SELF_COUNT && p == 0 ? status : nullptr, p, planes,
-                flt);
+    build_masks(topk_idx, T, k, E, masks, nullptr, p, planes, flt);
     if (e < E) {
       int32_t wb = pbase[p][e];
 #pragma unroll
@@ -619,9 +543,9 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
         topk_idx, s.T, s.k, s.E, 1, hist, status, all);
     note_launch();
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    dispatch_rank_kernel<false><<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
+    dispatch_rank_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
         topk_idx, s.T, s.k, s.E, -1, MOE_LAYOUT_COMPACT, 1, nblk, hist, routed, sc.kept,
-        sc.offsets, sc.assign_row, sc.token_of_row, s.T * s.k, all, nullptr);
+        sc.offsets, sc.assign_row, sc.token_of_row, s.T * s.k, all);
     note_launch();
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     // 2. per expert, the priority of its C-th best pick
@@ -635,16 +559,9 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
         topk_idx, s.T, s.k, s.E, 1, hist, nullptr, flt);
     note_launch();
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    dispatch_rank_kernel<false><<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
+    dispatch_rank_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
         topk_idx, s.T, s.k, s.E, s.C, s.layout, 1, nblk, hist, routed, kept, offsets,
-        assign_row, token_of_row, s.max_rows, flt, nullptr);
-    note_launch();
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  } else if (s.T * s.k <= kSelfCountMaxPicks) {
-    // few picks: one launch, every block counting all picks itself
-    dispatch_rank_kernel<true><<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
-        topk_idx, s.T, s.k, s.E, s.C, s.layout, planes, nblk, nullptr, routed, kept, offsets,
-        assign_row, token_of_row, s.max_rows, all, status);
+        assign_row, token_of_row, s.max_rows, flt);
     note_launch();
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   } else {
@@ -652,9 +569,9 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
         topk_idx, s.T, s.k, s.E, planes, hist, status, all);
     note_launch();
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    dispatch_rank_kernel<false><<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
+    dispatch_rank_kernel<<<static_cast<unsigned>(nblk), kDispatchBlockTokens, 0, st>>>(
         topk_idx, s.T, s.k, s.E, s.C, s.layout, planes, nblk, hist, routed, kept, offsets,
-        assign_row, token_of_row, s.max_rows, all, nullptr);
+        assign_row, token_of_row, s.max_rows, all);
     note_launch();
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
@@ -665,15 +582,27 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
   // equal segments, each a multiple of 16 bytes
   int64_t seg = (row_bytes + segs - 1) / segs;
   seg = (seg + 15) / 16 * 16;
-  // about 96 KB of ring per block, two blocks per SM; half the ring is loads in flight
+  // about 96 KB of ring per block, two blocks per SM; half the ring is loads in flight.  A
+  // short run (at most 8 items per block of 4 per SM, e.g. 4096 tokens) takes 6-segment rings
+  // in 4 blocks per SM instead: more copies start at once, fewer wait behind each other
   const int64_t items = s.T * segs;
   int64_t grid = static_cast<int64_t>(sm_count()) * 2;
+  const bool short_run = items <= static_cast<int64_t>(sm_count()) * 4 * 8;
+  if (short_run) grid = static_cast<int64_t>(sm_count()) * 4;
   if (grid > items) grid = items;
   if (grid < 1) grid = 1;
   const uint8_t* xb = static_cast<const uint8_t*>(x);
   uint8_t* xp = static_cast<uint8_t*>(x_perm);
   const uint32_t sg = static_cast<uint32_t>(seg);
-  if (seg <= 6 * 1024) {
+  if (short_run || seg > 8 * 1024) {
+    const size_t smem = 6 * static_cast<size_t>(seg);
+    err = cudaFuncSetAttribute(permute_rows_kernel<6, 3>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    permute_rows_kernel<6, 3><<<static_cast<unsigned>(grid), 32, smem, st>>>(
+        xb, assign_row, s.T, s.k, row_bytes, sg, segs, xp, status, wait_ns);
+    note_launch();
+  } else if (seg <= 6 * 1024) {
     const size_t smem = 16 * static_cast<size_t>(seg);
     err = cudaFuncSetAttribute(permute_rows_kernel<16, 8>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -681,20 +610,12 @@ cudaError_t launch_dispatch(const Shape& s, const void* x, const int32_t* topk_i
     permute_rows_kernel<16, 8><<<static_cast<unsigned>(grid), 32, smem, st>>>(
         xb, assign_row, s.T, s.k, row_bytes, sg, segs, xp, status, wait_ns);
     note_launch();
-  } else if (seg <= 8 * 1024) {
+  } else {
     const size_t smem = 12 * static_cast<size_t>(seg);
     err = cudaFuncSetAttribute(permute_rows_kernel<12, 6>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
     permute_rows_kernel<12, 6><<<static_cast<unsigned>(grid), 32, smem, st>>>(
-        xb, assign_row, s.T, s.k, row_bytes, sg, segs, xp, status, wait_ns);
-    note_launch();
-  } else {
-    const size_t smem = 6 * static_cast<size_t>(seg);
-    err = cudaFuncSetAttribute(permute_rows_kernel<6, 3>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
-    permute_rows_kernel<6, 3><<<static_cast<unsigned>(grid), 32, smem, st>>>(
         xb, assign_row, s.T, s.k, row_bytes, sg, segs, xp, status, wait_ns);
     note_launch();
   }

@@ -123,10 +123,10 @@ def test_ep_emulated_twice_is_deterministic():
     for a, b in zip(first, second):
         assert torch.equal(a, b)
     # per rank: router (2: the W_r split + the tensor-core GEMM with the top-k in its
-    # epilogue at T >= 512; the fp32 GEMM + top-k below), the ranking (one self-counting
-    # kernel at 4096 picks), put_counts, plan (2), dispatch, FFN (2), combine, stats
+    # epilogue at T >= 512; the fp32 GEMM + top-k below), count + rank, put_counts, plan (2),
+    # dispatch, FFN (2), combine, stats
     router = 2
-    assert launched == 4 * (router + 1 + 1 + 2 + 1 + 2 + 1 + 1)
+    assert launched == 4 * (router + 2 + 1 + 2 + 1 + 2 + 1 + 1)
 
 
 def test_ep_receive_overflow_is_reported_not_faulted():
