@@ -28,6 +28,12 @@ def test_binding_roof_per_workload():
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert r["achieved"] == pytest.approx(1286.4, rel=1e-3)
     assert r["frac"] == pytest.approx(r["achieved"] / 1674.7)
+    assert r["frac_of_burst"] == r["frac"]
+    assert r["frac_of_sustained"] == pytest.approx(r["achieved"] / 1364.1)
+    # a power-capped timed region divides by the sustained figure, and says so
+    rc = bench.gemm_roofline(W.MIXTRAL_8X7B, 8192, 8, 2.2437, PEAKS, power_capped=True)
+    assert rc["peak"] == 1364.1 and rc["frac"] == pytest.approx(rc["achieved"] / 1364.1)
+    assert rc["frac_of_burst"] == pytest.approx(r["frac"]) and "sustained" in rc["peak_source"]
     # DeepSeek decode: 128 tokens x 8 picks over ~252 experts -> weight streaming binds
     r = bench.gemm_roofline(W.DSV3_DECODE, 1024, 252, 3.2, PEAKS)
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
