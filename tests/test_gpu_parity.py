@@ -225,6 +225,27 @@ def test_tied_logits_pick_lower_index():
     assert np.allclose(f64(run.b.topk_w), 0.25)
 
 
+@pytest.mark.parametrize("k", [1, 8])
+def test_tensor_core_router_ties_across_expert_halves(k):
+    """The tensor-core router (E = 256, T = 600 >= 512: two 128-expert halves per token, their
+    lists merged) with every logit equal to its bias and twelve experts tied on both sides of
+    the half boundary: the picks are the k lowest tied experts in index order, as the oracle's
+    order (equal scores -> lower index) demands."""
+    shape = _edge(600, 128, 64, 256, k, gating=W.SIGMOID)
+    inp = W.make_inputs(shape, device="cuda")
+    inp.x.zero_()                                      # z = x . W_r = 0 exactly
+    tied = [255, 131, 3, 200, 129, 60, 127, 140, 250, 10, 128, 90]
+    bias = torch.full((256,), -2.0, device="cuda")
+    bias[tied] = 1.0
+    inp.logit_bias = bias
+    run = GpuRun(shape, inp)
+    run.all_stages()
+    r = check_routing(run)
+    want = np.array(sorted(tied)[:k])
+    assert (r["idx"] == want).all()
+    assert np.allclose(f64(run.b.topk_w), 1.0 / k)
+
+
 def test_empty_experts_and_padded_layout():
     shape = _edge(256, 128, 128, 64, 2, cf=2.0, layout=W.LAYOUT_PADDED)
     inp = W.make_inputs(shape, device="cuda")
