@@ -359,6 +359,29 @@ def test_presplit_router_weight_equals_split_per_call(shape):
     check_routing(run)
 
 
+@pytest.mark.parametrize("shape", [
+    W.reduced(W.DSV3_PREFILL_ZIPF, 12000, 256, 64),                   # 94 tiles, 8 K steps
+    W.reduced(W.DSV3_PREFILL_ZIPF, 9472, 128, 64),                    # 74 tiles: halves
+    W.reduced(W.DSV3_PREFILL_ZIPF, 10000, 192, 64, E=200, bias="chunks", bias_mode=1,
+              n_decode_tokens=8),                                     # masked experts
+], ids=["T12000_d256", "T9472_d128", "T10000_E200_selbias"])
+def test_tensor_core_router_at_many_tiles(shape):
+    """The tensor-core router over 74-94 token tiles, each starting its K loop at its own
+    chunk of the split weight: logits, picks and weights against the oracle, and bitwise the
+    same on a second call."""
+    run = GpuRun(shape)
+    run.route()
+    b, i = run.b, run.inp
+    z, idx, w = b.logits.clone(), b.topk_idx.clone(), b.topk_w.clone()
+    b.logits.fill_(-7.0), b.topk_idx.fill_(-7), b.topk_w.fill_(-7.0)
+    run.route()
+    M.moe_check_device_error(run.ws)
+    torch.cuda.synchronize()
+    assert torch.equal(b.logits, z) and torch.equal(b.topk_idx, idx) and torch.equal(b.topk_w, w)
+    run.dispatch()
+    check_routing(run)
+
+
 def test_bad_expert_index_is_reported_not_faulted():
     shape = _edge(50, 64, 64, 8, 2)
     run = GpuRun(shape)
