@@ -13,12 +13,15 @@
 //     W_g[e] stacked on the same 128 rows of W_u[e] (256 rows), so one 128x256x16 MMA per
 //     K step produces the gate tile in TMEM columns [0,128) and the up tile in [128,256);
 //     the epilogue writes h = silu(gate) * up as bf16.
-//   down: a 128 x 256 tile of y_perm = h . W_d[e]^T with a plain bf16 epilogue.
-//   router (E > 32, bf16 x): z = x . W_r with W_r split into two bf16 terms hi + lo; the
-//     B tile stacks 128 experts of hi on the same 128 experts of lo, and the epilogue writes
-//     z = (x . hi) + (x . lo) + bias in fp32.
+//   down: a 128 x 256 tile of y_perm = h . W_d[e]^T; the epilogue stages each 32-column
+//     chunk in shared memory and stores whole 32-row groups with tensor stores.
+//   router (E > 32, bf16 x): z = x . W_r with W_r split into two bf16 terms, W' = [E, 2d] =
+//     [hi | lo] along K: all E <= 256 experts of 128 tokens in one accumulator, each 64-wide
+//     chunk of x taken against hi and then lo, each tile starting its K loop at its own chunk;
+//     the epilogue (8 warps, two halves of the experts) writes z + bias in fp32 and, without
+//     a group limit, the top-k and gate weights.
 //
-// Block = 6 warps, one block per SM, persistent over tiles:
+// Block = 6 warps (10 for the router), one block per SM, persistent over tiles:
 //   warp 0 (one lane)   TMA producer: A = 128 x 64 bf16 slice of x_perm/h rows, B = 256 x 64
 //                       slice of the expert's weights, 128-byte swizzle, 4-stage ring.
 //                       With gathered A (dispatch without x_perm) the whole warp copies the
