@@ -51,7 +51,15 @@ def test_full_size_sampled(shape):
     check_layer_output(run, run.b.out, r, tokens=out_toks, label=f"full:{shape.name}{tag}")
     if shape.capacity_factor > 0:
         assert st["max"] <= st["capacity"]
-    del run
+    # the public entry point (moe_layer_forward; the router weight split once at
+    # construction) gives bitwise the staged calls' output
+    i = run.inp
+    layer = M.MoELayer(run.cfg, i.w_router, i.w_gate, i.w_up, i.w_down, i.logit_bias)
+    out = layer(i.x)
+    M.moe_check_device_error(layer.ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out, run.b.out)
+    del layer, run
     torch.cuda.empty_cache()
 
 
