@@ -6,9 +6,10 @@
 // of experts and dropped tokens.  "Capacity factor changes quality, memory and the latency
 // tail": drop rate per layer and per route (first pick, second pick, ...).
 //
-// One block: the E kept counts are sorted in shared memory (bitonic network over the next
-// power of two of E), the drops are counted per pick rank over assign_row, and one thread evaluates
-// the fp64 formulas.  The job record of data-parallel replicas runs the same kernel on the
+// The drops per pick rank and per token are counted over assign_row -- above 32768 picks by
+// a kernel spread over the GPU (one thread per token) into the output record, else by the
+// record kernel itself -- and one block sorts the E kept counts in shared memory (bitonic
+// network over the next power of two of E) and one thread evaluates the fp64 formulas.  The job record of data-parallel replicas runs the same kernel on the
 // replicas' summed counts, taking the token count, capacity and drop counters from the
 // replicas' own records instead of an assign_row.  Percentiles interpolate linearly between order statistics:
 // h = (E - 1) p, v = s[floor h] + (h - floor h) (s[floor h + 1] - s[floor h]).
@@ -38,10 +39,70 @@ __device__ __forceinline__ int warp_sum(int v) {
 
 // Counters are reduced within each warp first and then added with 32-bit shared atomics
 // (one per warp), so the block never serialises on a contended 64-bit atomic.
+// The drop counters over assign_row, spread over the GPU: a thread per token, its k picks
+// loaded at once; each block adds its counts to out (zeroed before the launch) with one
+// 64-bit atomic per counter.  Integer sums, so the order of the additions does not matter.
+constexpr int kDropThreads = 256;
+// up to this many picks one block counts the drops faster than a memset, a spread kernel
+// and the record kernel: 14 against 17 us at 8192 picks, 43 against 25 us at 131072
+constexpr int64_t kStatsOneBlockPicks = 32768;
+__global__ void __launch_bounds__(kDropThreads) drop_count_kernel(
+    const int32_t* __restrict__ assign_row, int64_t T, int k,
+    moe_load_stats_t* __restrict__ out) {
+  __shared__ int s_rank[MOE_MAX_TOPK];
+  __shared__ int s_td, s_tf;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  if (tid < MOE_MAX_TOPK) s_rank[tid] = 0;
+  if (tid == 0) s_td = s_tf = 0;
+  __syncthreads();
+  int rank_local[MOE_MAX_TOPK];
+#pragma unroll
+  for (int j = 0; j < MOE_MAX_TOPK; ++j) rank_local[j] = 0;
+  int td = 0, tf = 0;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * kDropThreads + tid; t < T;
+       t += static_cast<int64_t>(gridDim.x) * kDropThreads) {
+    int32_t a[MOE_MAX_TOPK];
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_TOPK; ++j) a[j] = j < k ? __ldg(assign_row + t * k + j) : 0;
+    int nd = 0;
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_TOPK; ++j)
+      if (j < k && a[j] < 0) {
+        ++rank_local[j];
+        ++nd;
+      }
+    td += nd > 0;
+    tf += nd == k;
+  }
+#pragma unroll
+  for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+    const int v = warp_sum(rank_local[j]);
+    if (lane == 0 && v) atomicAdd(&s_rank[j], v);
+  }
+  td = warp_sum(td);
+  tf = warp_sum(tf);
+  if (lane == 0) {
+    if (td) atomicAdd(&s_td, td);
+    if (tf) atomicAdd(&s_tf, tf);
+  }
+  __syncthreads();
+  if (tid < MOE_MAX_TOPK && tid < k && s_rank[tid])
+    atomicAdd(reinterpret_cast<unsigned long long*>(&out->dropped_by_rank[tid]),
+              static_cast<unsigned long long>(s_rank[tid]));
+  if (tid == 0 && s_td)
+    atomicAdd(reinterpret_cast<unsigned long long*>(&out->tokens_with_drop),
+              static_cast<unsigned long long>(s_td));
+  if (tid == 0 && s_tf)
+    atomicAdd(reinterpret_cast<unsigned long long*>(&out->tokens_fully_dropped),
+              static_cast<unsigned long long>(s_tf));
+}
+
+// counted: the drop counters are already in out (drop_count_kernel); assign_row unused.
 __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
     const int32_t* __restrict__ routed, const int32_t* __restrict__ kept,
     const int32_t* __restrict__ assign_row, int64_t T, int k, int E, int64_t C,
-    const moe_load_stats_t* __restrict__ parts, int n_parts,
+    const moe_load_stats_t* __restrict__ parts, int n_parts, bool counted,
     moe_load_stats_t* __restrict__ out) {
   __shared__ int32_t sorted[MOE_MAX_EXPERTS];
   __shared__ unsigned long long sum_kept, sum_routed;
@@ -146,6 +207,11 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
     int64_t drops[MOE_MAX_TOPK];
     int64_t with_drop = tok_drop, fully = tok_full;
     for (int j = 0; j < MOE_MAX_TOPK; ++j) drops[j] = j < k ? drop_rank[j] : 0;
+    if (counted) {
+      with_drop = out->tokens_with_drop;
+      fully = out->tokens_fully_dropped;
+      for (int j = 0; j < MOE_MAX_TOPK; ++j) drops[j] = j < k ? out->dropped_by_rank[j] : 0;
+    }
     if (parts != nullptr) {  // job record: tokens, capacity and drop counters of the replicas
       T = 0;
       C = 0;
@@ -192,8 +258,25 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(
 
 cudaError_t launch_stats(const Shape& s, const int32_t* routed, const int32_t* kept,
                          const int32_t* assign_row, moe_load_stats_t* out, cudaStream_t st) {
-  stats_kernel<<<1, kStatsThreads, 0, st>>>(routed, kept, assign_row, s.T, s.k, s.E, s.C,
-                                            nullptr, 0, out);
+  if (s.T * s.k <= kStatsOneBlockPicks) {  // few picks: one block scans them itself
+    stats_kernel<<<1, kStatsThreads, 0, st>>>(routed, kept, assign_row, s.T, s.k, s.E, s.C,
+                                              nullptr, 0, false, out);
+    note_launch();
+    return cudaGetLastError();
+  }
+  // the drop counters of assign_row over many blocks into out, then the one-block rest
+  cudaError_t err = cudaMemsetAsync(out, 0, sizeof(moe_load_stats_t), st);
+  if (err != cudaSuccess) return err;
+  int64_t blocks = (s.T + kDropThreads - 1) / kDropThreads;
+  const int64_t cap = static_cast<int64_t>(sm_count()) * 4;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  drop_count_kernel<<<static_cast<unsigned>(blocks), kDropThreads, 0, st>>>(assign_row, s.T,
+                                                                          s.k, out);
+  note_launch();
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  stats_kernel<<<1, kStatsThreads, 0, st>>>(routed, kept, nullptr, s.T, s.k, s.E, s.C,
+                                            nullptr, 0, true, out);
   note_launch();
   return cudaGetLastError();
 }
@@ -202,7 +285,7 @@ cudaError_t launch_stats_merge(const Shape& s, const int32_t* routed_sum,
                                const int32_t* kept_sum, const moe_load_stats_t* parts,
                                int n_parts, moe_load_stats_t* out, cudaStream_t st) {
   stats_kernel<<<1, kStatsThreads, 0, st>>>(routed_sum, kept_sum, nullptr, 0, s.k, s.E, 0,
-                                            parts, n_parts, out);
+                                            parts, n_parts, false, out);
   note_launch();
   return cudaGetLastError();
 }
