@@ -73,9 +73,14 @@ __device__ __forceinline__ void build_masks(const int32_t* __restrict__ topk_idx
   const int w = threadIdx.x >> 5;
   const uint32_t bit = 1u << (threadIdx.x & 31);
   if (t < T) {
-    for (int j = 0; j < k; ++j) {
+    int ev[MOE_MAX_TOPK];  // the token's picks, all loads in flight before any is used
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_TOPK; ++j) ev[j] = j < k ? __ldg(topk_idx + t * k + j) : 0;
+#pragma unroll
+    for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+      if (j >= k) break;
       if (planes > 1 && j != plane) continue;
-      const int e = topk_idx[t * k + j];
+      const int e = ev[j];
       if (e < 0 || e >= E) {
         record_error(status, DEV_BAD_EXPERT, 1, static_cast<unsigned long long>(t * k + j));
         continue;
@@ -133,20 +138,16 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
   if (e < E) {
     for (int p = 0; p < planes; ++p) {
       int64_t tot = 0, before = 0;
-      int64_t b = 0;
-      for (; b + 8 <= nblk; b += 8) {  // loads issued 8 at a time, sums in block order
-        int32_t c[8];
+      for (int64_t b = 0; b < nblk; b += 32) {  // loads issued 32 at a time, sums in block order
+        int32_t c[32];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) c[u] = __ldg(hist + ((b + u) * planes + p) * E + e);
+        for (int u = 0; u < 32; ++u)
+          c[u] = b + u < nblk ? __ldg(hist + ((b + u) * planes + p) * E + e) : 0;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 32; ++u) {
           if (b + u == blockIdx.x) before = tot;
           tot += c[u];
         }
-      }
-      for (; b < nblk; ++b) {
-        if (b == blockIdx.x) before = tot;
-        tot += __ldg(hist + (b * planes + p) * E + e);
       }
       pbase[p][e] = static_cast<int32_t>(run + before);
       run += tot;
@@ -194,9 +195,14 @@ __global__ void __launch_bounds__(kDispatchBlockTokens) dispatch_rank_kernel(
     }
     __syncthreads();
     if (t < T) {
-      for (int j = 0; j < k; ++j) {
+      int ev[MOE_MAX_TOPK];
+#pragma unroll
+      for (int j = 0; j < MOE_MAX_TOPK; ++j) ev[j] = j < k ? __ldg(topk_idx + t * k + j) : 0;
+#pragma unroll
+      for (int j = 0; j < MOE_MAX_TOPK; ++j) {
+        if (j >= k) break;
         if (planes > 1 && j != p) continue;
-        const int ee = topk_idx[t * k + j];
+        const int ee = ev[j];
         int32_t row = -1;
         if (ee >= 0 && ee < E && filter_keeps(flt, t, E, ee)) {
           const int64_t slot = wbase[w][ee] + __popc(masks[w][ee] & below);
