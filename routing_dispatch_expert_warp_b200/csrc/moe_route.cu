@@ -425,7 +425,7 @@ __global__ void __launch_bounds__(256) topk_from_logits_kernel(
     float zv[8];
     uint32_t key[8];
     // the nsplit partial sums of each of the lane's 8 logits, added strictly in split order;
-    // the loads of 4 splits x 8 logits are issued together
+    // the loads of 8 splits x 8 logits are issued together
     float part[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -435,17 +435,17 @@ __global__ void __launch_bounds__(256) topk_from_logits_kernel(
     if (nsplit > 1) {
       const int64_t stride = T * E;
       int sp = 1;
-      for (; sp + 4 <= nsplit; sp += 4) {
-        float b[4][8];
+      for (; sp + 8 <= nsplit; sp += 8) {
+        float b[8][8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < 8; ++u)
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             const int e = lane + 32 * q;
             b[u][q] = e < E ? z[(sp + u) * stride + t * E + e] : 0.f;
           }
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < 8; ++u)
 #pragma unroll
           for (int q = 0; q < 8; ++q) part[q] += b[u][q];
       }
