@@ -206,8 +206,7 @@ class ClockSampler:
 
 def tensor_core_router(shape) -> bool:
     """The layer shapes whose router runs on the tensor cores (moe_route's rule)."""
-    return (shape.dtype == W.BF16 and shape.E > 32 and shape.d_model % 64 == 0
-            and shape.T >= 512)
+    return shape.dtype == W.BF16 and shape.E > 32 and shape.d_model % 64 == 0
 
 
 def route_tensor_roof(shape, work: dict, route_ms: float, peaks: dict) -> dict:

@@ -289,10 +289,12 @@ int64_t moe_max_rows(const moe_config_t* cfg);
  *   topk_idx[t, :] = the k largest z[t, :], best first; equal z -> lower expert index
  *   topk_w[t, :]   = gate weights renormalised over the k picks (cfg->gating)
  * logits may be NULL (then z lives in the workspace).  Needs the workspace.
- * Precision of z: fp32 FMA on CUDA cores, except for bf16 layers with E > 32, T >= 512 and
- * d_model a multiple of 64, where z = x . hi + x . lo runs on the tensor cores with W_r
- * split into two bf16 terms (|z - exact| <= 1e-4 (1 + |z|)).  The top-k is always taken on
- * the fp32 z that is returned, so picks, weights and everything downstream follow z.
+ * Precision of z: fp32 FMA on CUDA cores, except for bf16 layers with E > 32 and d_model a
+ * multiple of 64, where z = x . hi + x . lo runs on the tensor cores with W_r split into two
+ * bf16 terms (|z - exact| <= 1e-4 (1 + |z|)); with few 128-token tiles (fewer than half the
+ * SMs) each tile's K steps are split over several blocks and their fp32 sums added in a
+ * fixed order.  The top-k is always taken on the fp32 z that is returned, so picks, weights
+ * and everything downstream follow z.
  */
 moe_status_t moe_route(const moe_config_t* cfg, const void* x, const float* w_router,
                        const float* logit_bias, int64_t bias_row_stride, float* logits,
@@ -318,9 +320,9 @@ moe_status_t moe_router_split(const moe_config_t* cfg, const float* w_router, vo
 /*
  * moe_route with an optional argument: w_router_split NULL is moe_route; otherwise it is the
  * moe_router_split output for w_router, which the tensor-core router reads instead of
- * splitting w_router (one kernel launch instead of two; the result is bitwise the same).  The
- * other router paths (fp32, E <= 32, T < 512) read w_router and ignore it, so w_router is
- * required either way.  A split that was not made from this w_router gives the logits of the
+ * splitting w_router (one kernel launch fewer; the result is bitwise the same).  The other
+ * router paths (fp32, E <= 32, d_model not a multiple of 64) read w_router and ignore it, so
+ * w_router is required either way.  A split that was not made from this w_router gives the logits of the
  * weight it was made from.
  */
 moe_status_t moe_route_ex(const moe_config_t* cfg, const void* x, const float* w_router,

@@ -150,8 +150,10 @@ WsLayout workspace_layout(const Shape& s) {
     const size_t et = s.E <= 8 ? 8 : (s.E <= 16 ? 16 : 32);
     l.partials_bytes = round_up(static_cast<size_t>((s.d + 255) / 256) * 256 * et * sizeof(float));
   } else {
+    int kb_per = 0;
+    const int parts = router_uses_tensor_cores(s) ? router_tc_splits(s, &kb_per) : splits;
     l.partials_bytes =
-        splits > 1 ? round_up(static_cast<size_t>(splits) * s.T * s.E * sizeof(float)) : 0;
+        parts > 1 ? round_up(static_cast<size_t>(parts) * s.T * s.E * sizeof(float)) : 0;
   }
   off += l.partials_bytes;
   l.router_tc = off;
@@ -325,10 +327,11 @@ moe_status_t moe_route_ex(const moe_config_t* cfg, const void* x, const float* w
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   if (router_uses_tensor_cores(s)) {
     const char* why = "";
-    cudaError_t err = launch_router_tc(s, x, w_router, w_router_split, logit_bias,
-                                       bias_row_stride, logits, z, topk_idx, topk_w,
-                                       static_cast<uint8_t*>(ws) + lay.router_tc,
-                                       ws_status(ws, lay), g_wait_ns.load(), strm, &why);
+    cudaError_t err = launch_router_tc(
+        s, x, w_router, w_router_split, logit_bias, bias_row_stride, logits, z, topk_idx, topk_w,
+        static_cast<uint8_t*>(ws) + lay.router_tc,
+        reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + lay.partials), ws_status(ws, lay),
+        g_wait_ns.load(), strm, &why);
     if (err != cudaSuccess) {
       if (why[0]) return fail(MOE_ERR_CUDA, "moe_route: %s", why);
       return cuda_fail(err, "moe_route (tensor cores) launch");

@@ -107,6 +107,11 @@ struct TcParams {
   int32_t* route_idx;         // [T, k] picks (fused top-k)
   float* route_w;             // [T, k] gate weights (fused top-k)
   int32_t router_rows;        // MODE_ROUTER: its one bucket is rows [0, router_rows) of x
+  // MODE_ROUTER split along K (few tiles): work item i is K steps
+  // [s kb_per_split, (s + 1) kb_per_split) of tile i / ksplit, s = i % ksplit; the epilogue
+  // writes that piece's fp32 sums to out_f32 + s router_rows N_out (no bias, no top-k)
+  int ksplit;
+  int kb_per_split;
 };
 
 // The last of a token's kept picks to finish column block nb has its warp sum the token's
@@ -298,6 +303,15 @@ __global__ void __launch_bounds__(MODE == 2 ? ROUTER_THREADS : THREADS, 1) group
   const uint32_t tmem_base = tmem_base_s;
   const int total_tiles = tile_base[p.E];
   const int KB = p.K / BK;
+  // work items: tiles, or (router split along K) tile x K piece, strided over the grid
+  const int ksplit = MODE == MODE_ROUTER && p.ksplit > 1 ? p.ksplit : 1;
+  const int total_items = total_tiles * ksplit;
+  auto item_range = [&](int item, int& tile, int& piece, int& kb0, int& kb1) {
+    tile = item / ksplit;
+    piece = item - tile * ksplit;
+    kb0 = ksplit > 1 ? piece * p.kb_per_split : 0;
+    kb1 = ksplit > 1 && kb0 + p.kb_per_split < KB ? kb0 + p.kb_per_split : KB;
+  };
 
   if (warp == 0 && p.a_rows == nullptr) {
     // ---------------------------------------------------------------- TMA producer
@@ -307,7 +321,9 @@ __global__ void __launch_bounds__(MODE == 2 ? ROUTER_THREADS : THREADS, 1) group
       uint32_t ph = 0;
       uint32_t armed = 0, armed_parity = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+      for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+        int tile, piece, kb0, kb1;
+        item_range(item, tile, piece, kb0, kb1);
         int e, mb, nb;
         decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, p.mb_outer, e, mb, nb);
         const int row0 = seg_start(e) + mb * BM;
@@ -316,10 +332,10 @@ __global__ void __launch_bounds__(MODE == 2 ? ROUTER_THREADS : THREADS, 1) group
         // of it at any moment instead of all the same lines at once.  (The fp32 sum then runs
         // in a per-tile order: deterministic, a rounding-level difference per tile.)
         const int pairs = KB >> 1;
-        const int rot = MODE == MODE_ROUTER
+        const int rot = MODE == MODE_ROUTER && ksplit == 1
                             ? static_cast<int>(static_cast<int64_t>(tile) * pairs / total_tiles)
                             : 0;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty_bar[s], ph ^ 1u, p.wait_ns, &abort_s)) {
             if (!abort_s)
               record_error(p.status, DEV_TIMEOUT, 20, static_cast<unsigned long long>(tile));
@@ -447,7 +463,9 @@ __global__ void __launch_bounds__(MODE == 2 ? ROUTER_THREADS : THREADS, 1) group
     uint32_t aph = 0;
     bool ok = true;
     bool issued = false;
-    for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
+    for (int item = blockIdx.x; ok && item < total_items; item += gridDim.x) {
+      int tile, piece, kb0, kb1;
+      item_range(item, tile, piece, kb0, kb1);
       int e, mb, nb;
       decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, p.mb_outer, e, mb, nb);
       const uint32_t idesc =
@@ -459,7 +477,7 @@ __global__ void __launch_bounds__(MODE == 2 ? ROUTER_THREADS : THREADS, 1) group
       }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * ACC_COLS);
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&full_bar[s], ph, p.wait_ns, &abort_s)) {
           if (!abort_s) record_error(p.status, DEV_TIMEOUT, 22, static_cast<unsigned long long>(tile));
           abort_s = 1;
@@ -472,7 +490,8 @@ __global__ void __launch_bounds__(MODE == 2 ? ROUTER_THREADS : THREADS, 1) group
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           tc_mma_f16(d_tmem, sw128_kmajor_desc(a_addr + kk * 32),
-                     sw128_kmajor_desc(b_addr + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+                     sw128_kmajor_desc(b_addr + kk * 32), idesc,
+                     (kb != kb0 || kk != 0) ? 1u : 0u);
         }
         issued = true;
         tc_commit(&empty_bar[s]);
@@ -500,7 +519,9 @@ __global__ void __launch_bounds__(MODE == 2 ? ROUTER_THREADS : THREADS, 1) group
     int acc = 0;
     uint32_t aph = 0;
     uint32_t mph = 0;  // router: phase of the list handoff
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+    for (int item = blockIdx.x; item < total_items; item += gridDim.x) {
+      int tile, piece, kb0, kb1;
+      item_range(item, tile, piece, kb0, kb1);
       int e, mb, nb;
       decode_tile(tile, tile_base, mblocks, p.E, p.n_blocks, p.mb_outer, e, mb, nb);
       const int row0 = seg_start(e) + mb * BM;
@@ -522,7 +543,30 @@ __global__ void __launch_bounds__(MODE == 2 ? ROUTER_THREADS : THREADS, 1) group
       __nv_bfloat16* orow =
           p.out + static_cast<int64_t>(row0 + rt) * p.N_out + static_cast<int64_t>(nb) * BN_OUT;
       const int cols_left = p.N_out - nb * BN_OUT;
-      if (MODE == MODE_ROUTER) {
+      if (MODE == MODE_ROUTER && ksplit > 1) {
+        // one K piece of the tile: this thread's row of its half of the experts, as summed
+        float* prow = p.out_f32 +
+                      (static_cast<int64_t>(piece) * p.router_rows + row0 + rt) * p.N_out;
+#pragma unroll 1
+        for (int c = 4 * half; c < 4 * half + 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c * 32, v);
+          tmem_ld_wait();
+          if (row_ok && c * 32 < cols_left) {
+            if (c * 32 + 32 <= cols_left && (p.N_out & 3) == 0) {
+              float4* dst = reinterpret_cast<float4*>(prow + c * 32);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                     __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (c * 32 + i < cols_left) prow[c * 32 + i] = __uint_as_float(v[i]);
+            }
+          }
+        }
+      } else if (MODE == MODE_ROUTER) {
         // one token per thread, all experts of the tile (up to 256) in its accumulator row
         const int64_t grow = static_cast<int64_t>(row0 + rt);
         float* zrow = p.out_f32 != nullptr ? p.out_f32 + grow * p.N_out : nullptr;
@@ -1710,8 +1754,24 @@ cudaError_t launch_ffn_tc(const Shape& s, const void* a, const int32_t* a_rows,
   return cudaGetLastError();
 }
 
-bool router_uses_tensor_cores(const Shape& s) {
-  return router_split_applies(s) && s.T >= 512;
+bool router_uses_tensor_cores(const Shape& s) { return router_split_applies(s); }
+
+// With fewer 128-token tiles than half the SMs, each tile's K steps are split over several
+// blocks (at least 4 K steps, an even number, per piece; at most 16 pieces), whose fp32 sums
+// the top-k kernel adds in piece order.  1: no split.
+int router_tc_splits(const Shape& s, int* kb_per_split) {
+  const int tiles = static_cast<int>((s.T + BM - 1) / BM);
+  const int KB = static_cast<int>(2 * s.d / BK);
+  *kb_per_split = KB;
+  if (2 * tiles >= sm_count()) return 1;
+  int ks = sm_count() / tiles;
+  if (ks > KB / 4) ks = KB / 4;
+  if (ks > 16) ks = 16;
+  if (ks < 2) return 1;
+  int per = (KB + ks - 1) / ks;
+  per += per & 1;
+  *kb_per_split = per;
+  return (KB + per - 1) / per;
 }
 
 bool router_split_applies(const Shape& s) {
@@ -1739,8 +1799,8 @@ cudaError_t launch_router_split(const Shape& s, const float* w_router, void* w_s
 cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_router,
                              const void* w_split, const float* bias, int64_t bias_stride,
                              float* logits, float* logits_scratch, int32_t* topk_idx,
-                             float* topk_w, void* split_ws, DevStatus* status, uint64_t wait_ns,
-                             cudaStream_t st, const char** why) {
+                             float* topk_w, void* split_ws, float* partials, DevStatus* status,
+                             uint64_t wait_ns, cudaStream_t st, const char** why) {
   if (encode_fn() == nullptr) {
     *why = "cuTensorMapEncodeTiled is not available from the driver";
     return cudaErrorNotSupported;
@@ -1760,8 +1820,10 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_route
                              cudaFuncAttributeMaxDynamicSharedMemorySize, DYN_SMEM);
   if (err != cudaSuccess) return err;
   const bool sel_only = s.bias_mode == MOE_BIAS_SELECTION_ONLY;
-  // the top-k rides in the epilogue unless the picks are limited to groups
-  const bool fuse = s.n_groups <= 1;
+  int kb_per_split = 0;
+  const int ksplit = router_tc_splits(s, &kb_per_split);
+  // the top-k rides in the epilogue unless the picks are limited to groups or K is split
+  const bool fuse = s.n_groups <= 1 && ksplit == 1;
   TcParams p = {};
   p.router_rows = static_cast<int32_t>(s.T);
   p.E = 1;
@@ -1785,12 +1847,24 @@ cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_route
   p.status = status;
   p.wait_ns = wait_ns;
   int64_t g = (s.T + BM - 1) / BM;
+  if (ksplit > 1) {  // the pieces' sums go to the partials; bias and top-k come after
+    p.ksplit = ksplit;
+    p.kb_per_split = kb_per_split;
+    p.out_f32 = partials;
+    p.bias = nullptr;
+    p.sel_bias = nullptr;
+    g *= ksplit;
+  }
   if (g > sm_count()) g = sm_count();
   grouped_gemm_tc_kernel<MODE_ROUTER><<<static_cast<unsigned>(g), ROUTER_THREADS, DYN_SMEM, st>>>(
       ta, tw, tw, tw, p);
   note_launch();
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   if (fuse) return cudaSuccess;
+  if (ksplit > 1)
+    return launch_topk_from_partials(s, partials, ksplit, bias, bias_stride,
+                                     logits != nullptr ? logits : logits_scratch, topk_idx,
+                                     topk_w, st);
   return launch_topk_from_logits(s, p.out_f32, bias, bias_stride, topk_idx, topk_w, st);
 }
 

@@ -64,25 +64,33 @@ int router_splits(const Shape& s);
 cudaError_t launch_router(const Shape& s, const void* x, const float* w_router,
                           const float* bias, int64_t bias_stride, float* logits,
                           int32_t* topk_idx, float* topk_w, float* partials, cudaStream_t st);
-// Router on tensor cores (bf16 layers, E > 32, d % 64 == 0, T >= 512): W_r split into two
-// bf16 terms, W' = [E, 2 d] (hi | lo along K).
+// Router on tensor cores (bf16 layers, E > 32, d % 64 == 0): W_r split into two bf16 terms,
+// W' = [E, 2 d] (hi | lo along K).
 bool router_uses_tensor_cores(const Shape& s);
+// pieces each 128-token tile's K steps are split into (1: none) and K steps per piece
+int router_tc_splits(const Shape& s, int* kb_per_split);
 bool router_split_applies(const Shape& s);   // the layer shape admits the split (any T)
 size_t router_split_bytes(const Shape& s);   // bytes of W' (0 when the split does not apply)
 cudaError_t launch_router_split(const Shape& s, const float* w_router, void* w_split,
                                 cudaStream_t st);
 // w_split: W' made earlier by launch_router_split, or nullptr (then W_r is split into
 // split_ws for this call).  logits: the caller's [T, E] buffer, or nullptr (then z goes to
-// logits_scratch, the workspace copy).
+// logits_scratch, the workspace copy).  partials: router_tc_splits(s) x [T, E] fp32 (used
+// only when K is split).
 cudaError_t launch_router_tc(const Shape& s, const void* x, const float* w_router,
                              const void* w_split, const float* bias, int64_t bias_stride,
                              float* logits, float* logits_scratch, int32_t* topk_idx,
-                             float* topk_w, void* split_ws, DevStatus* status, uint64_t wait_ns,
-                             cudaStream_t st, const char** why);
+                             float* topk_w, void* split_ws, float* partials, DevStatus* status,
+                             uint64_t wait_ns, cudaStream_t st, const char** why);
 size_t router_tc_workspace_bytes(const Shape& s);
 cudaError_t launch_topk_from_logits(const Shape& s, const float* logits, const float* bias,
                                     int64_t bias_stride, int32_t* topk_idx, float* topk_w,
                                     cudaStream_t st);
+// top-k over nsplit [T, E] fp32 partial sums (added in split order, then the bias unless it
+// only steers selection), writing the finished logits to `logits`
+cudaError_t launch_topk_from_partials(const Shape& s, const float* partials, int nsplit,
+                                      const float* bias, int64_t bias_stride, float* logits,
+                                      int32_t* topk_idx, float* topk_w, cudaStream_t st);
 // Selection scores for dispatch with drop_policy == MOE_DROP_SCORE: score of (t, e) =
 // logits[t, e] (+ bias[t * bias_stride + e] when the bias is selection-only), and the
 // scratch (dispatch_score_scratch_bytes, 256-byte aligned) the ranking by score needs.

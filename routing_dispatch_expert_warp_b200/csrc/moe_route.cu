@@ -633,6 +633,19 @@ cudaError_t launch_topk_from_logits(const Shape& s, const float* logits, const f
   return cudaGetLastError();
 }
 
+cudaError_t launch_topk_from_partials(const Shape& s, const float* partials, int nsplit,
+                                      const float* bias, int64_t bias_stride, float* logits,
+                                      int32_t* topk_idx, float* topk_w, cudaStream_t st) {
+  const int64_t blocks_needed = (s.T + 7) / 8;
+  const int blocks = static_cast<int>(blocks_needed < 148 * 16 ? blocks_needed : 148 * 16);
+  const bool sel_only = s.bias_mode == MOE_BIAS_SELECTION_ONLY;
+  topk_from_logits_kernel<<<blocks, 256, 0, st>>>(
+      partials, nsplit, bias, bias_stride, sel_only ? 0 : 1, sel_only ? 1 : 0, logits, s.T, s.E,
+      s.k, s.gating, s.n_groups, s.topk_groups, topk_idx, topk_w);
+  note_launch();
+  return cudaGetLastError();
+}
+
 int router_splits(const Shape& s) {
   if (s.E <= 32) return 1;
   const int64_t tiles = ((s.E + RT_N - 1) / RT_N) * ((s.T + RT_M - 1) / RT_M);

@@ -22,8 +22,31 @@ TOL_LOGIT_SPLIT = 1e-4    # tensor-core router with W_r split into two bf16 term
 
 def router_on_tensor_cores(shape) -> bool:
     """The library's documented rule (include/moe.h, moe_route)."""
-    return (shape.dtype == W.BF16 and shape.E > 32 and shape.d_model % 64 == 0
-            and shape.T >= 512)
+    return shape.dtype == W.BF16 and shape.E > 32 and shape.d_model % 64 == 0
+
+
+def router_tc_splits(shape, sms: int) -> int:
+    """Pieces the tensor-core router cuts each 128-token tile's K steps into (1: none): with
+    fewer tiles than half the SMs, sms // tiles pieces, at most K steps / 4 and 16, each an
+    even number of 64-wide K steps."""
+    tiles = (shape.T + 127) // 128
+    kb = 2 * shape.d_model // 64
+    if 2 * tiles >= sms:
+        return 1
+    ks = min(sms // tiles, kb // 4, 16)
+    if ks < 2:
+        return 1
+    per = -(-kb // ks)
+    per += per & 1
+    return -(-kb // per)
+
+
+def router_launches(shape, presplit: bool, sms: int) -> int:
+    """Kernels one moe_route (or moe_route_ex with a split weight) launches."""
+    if router_on_tensor_cores(shape):
+        topk = shape.n_groups > 1 or router_tc_splits(shape, sms) > 1
+        return (0 if presplit else 1) + 1 + (1 if topk else 0)
+    return 2   # lane-ordered W_r + fused small-E router, or the fp32 GEMM + top-k
 
 
 def rel_fro(a, b) -> float:

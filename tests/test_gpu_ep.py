@@ -15,6 +15,8 @@ import routing_dispatch_expert_warp_b200 as M
 from routing_dispatch_expert_warp_b200 import ep as EP
 from routing_dispatch_expert_warp_b200 import workload as W
 
+from moe_parity import router_launches
+
 pytestmark = pytest.mark.gpu
 
 
@@ -122,10 +124,10 @@ def test_ep_emulated_twice_is_deterministic():
     torch.cuda.synchronize()
     for a, b in zip(first, second):
         assert torch.equal(a, b)
-    # per rank: router (2: the W_r split + the tensor-core GEMM with the top-k in its
-    # epilogue at T >= 512; the fp32 GEMM + top-k below), count + rank, put_counts, plan (2),
-    # dispatch, FFN (2), combine, stats
-    router = 2
+    # per rank: router (the W_r split + the tensor-core GEMM, with the top-k in its epilogue
+    # or a kernel of its own when K is split), count + rank, put_counts, plan (2), dispatch,
+    # FFN (2), combine, stats
+    router = router_launches(shape, False, torch.cuda.get_device_properties(0).multi_processor_count)
     assert launched == 4 * (router + 2 + 1 + 2 + 1 + 2 + 1 + 1)
 
 

@@ -14,7 +14,8 @@ import routing_dispatch_expert_warp_b200 as M
 from routing_dispatch_expert_warp_b200 import workload as W
 
 from moe_parity import (GpuRun, check_combine, check_ffn_rows, check_layer_output,
-                        check_permute, check_routing, check_stats, f64, i64, rel_fro)
+                        check_permute, check_routing, check_stats, f64, i64, rel_fro,
+                        router_launches)
 
 pytestmark = pytest.mark.gpu
 
@@ -268,7 +269,7 @@ VARIANTS = [
     # 1024 tokens: tensor-core router
     W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256, n_groups=8, topk_groups=4, bias_mode=1,
               drop_policy=1),
-    # the same regime through the fp32 router (T < 512) and token-order drops
+    # the same regime at 300 tokens (the router's K split over blocks) and token-order drops
     W.reduced(W.DSV3_PREFILL_ZIPF, 300, 256, 128, n_groups=16, topk_groups=2, bias_mode=1),
     # E = 8 with groups (general top-k path), pick-rank drops, chunk bias in score and weight
     W.reduced(W.MIXTRAL_8X22B_MIXED, 900, 256, 384, n_decode_tokens=8, n_groups=4,
@@ -307,7 +308,7 @@ def test_routing_variants_match_oracle(shape):
 def test_tensor_core_router_without_logits_buffer(shape):
     """moe_route on the tensor-core router (top-k in the GEMM's epilogue) with no logits
     buffer -- z then goes to the workspace -- picks and weights exactly as with one."""
-    assert (shape.dtype == W.BF16 and shape.E > 32 and shape.T >= 512)
+    assert shape.dtype == W.BF16 and shape.E > 32 and shape.T >= 512
     run = GpuRun(shape)
     run.route()
     idx, w = run.b.topk_idx.clone(), run.b.topk_w.clone()
@@ -353,8 +354,8 @@ def test_presplit_router_weight_equals_split_per_call(shape):
     M.moe_check_device_error(run.ws)
     torch.cuda.synchronize()
     assert torch.equal(b.logits, z) and torch.equal(b.topk_idx, idx) and torch.equal(b.topk_w, w)
-    tc = shape.T >= 512
-    assert launched == (1 if tc and shape.n_groups <= 1 else 2)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert launched == router_launches(shape, True, sms)
     run.dispatch()
     check_routing(run)
 
@@ -441,22 +442,27 @@ def test_small_e_router_wide_d(shape):
 
 
 # ------------------------------------------------------------------ launch accounting
-@pytest.mark.parametrize("shape,router_kernels,stats_kernels", [
-    (W.reduced(W.MIXTRAL_8X7B, 1000, 512, 768), 2, 1),          # lane-ordered W_r + fused router
-    (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256), 2, 1),     # W_r split + GEMM with the top-k
-    (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256, n_groups=8, topk_groups=4), 3, 1),  # + top-k
-    (W.reduced(W.DSV3_DECODE, 128, 512, 256), 2, 1),            # split-K fp32 GEMM + top-k
-    (W.reduced(W.DSV3_PREFILL_ZIPF, 4200, 256, 128), 2, 2),     # 33600 picks: spread drop count
+@pytest.mark.parametrize("shape,stats_kernels", [
+    (W.reduced(W.MIXTRAL_8X7B, 1000, 512, 768), 1),          # lane-ordered W_r + fused router
+    (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256), 1),     # W_r split + GEMM split along K + top-k
+    (W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256, n_groups=8, topk_groups=4), 1),  # + top-k
+    (W.reduced(W.DSV3_DECODE, 128, 512, 256), 1),            # one tile, K split over blocks
+    (W.reduced(W.DSV3_PREFILL_ZIPF, 12000, 256, 64), 2),     # 94 tiles: top-k in the epilogue
+    (W.reduced(W.DSV3_PREFILL_ZIPF, 4200, 256, 128), 2),     # 33600 picks: spread drop count
 ])
-def test_kernel_launch_count_per_layer(shape, router_kernels, stats_kernels):
-    """One staged layer forward launches the router's kernels, count + rank + permute, the two
-    grouped GEMMs, combine and the statistics (above 32768 picks the drops are counted by a
-    kernel of their own) -- and the library's own counter says so."""
+def test_kernel_launch_count_per_layer(shape, stats_kernels):
+    """One staged layer forward launches the router's kernels (the W_r split, the tensor-core
+    GEMM and, when K is split or the picks are group-limited, the top-k; or the E <= 32
+    router's two), count + rank + permute, the two grouped GEMMs, combine and the statistics
+    (above 32768 picks the drops are counted by a kernel of their own) -- and the library's
+    own counter says so."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
     run = GpuRun(shape)
     run.all_stages()
     c0 = M.kernel_launch_count()
     run.all_stages()
-    assert M.kernel_launch_count() - c0 == router_kernels + 3 + 2 + 1 + stats_kernels
+    assert (M.kernel_launch_count() - c0 ==
+            router_launches(shape, False, sms) + 3 + 2 + 1 + stats_kernels)
 
 
 # ------------------------------------------------------------------ dispatch without x_perm

@@ -12,7 +12,8 @@ import routing_dispatch_expert_warp_b200 as M
 from routing_dispatch_expert_warp_b200 import workload as W
 
 from moe_parity import (GpuRun, check_combine, check_ffn_rows, check_layer_output,
-                        check_permute, check_routing, check_stats, i64)
+                        check_permute, check_routing, check_stats, i64,
+                        router_launches)
 
 pytestmark = pytest.mark.gpu
 
@@ -25,7 +26,7 @@ def _cuda():
 
 
 SCORE_SHAPES = [
-    # group-limited top-8 of 256 with the selection-only bias; tensor-core router (T >= 512)
+    # group-limited top-8 of 256 with the selection-only bias; tensor-core router
     W.reduced(W.DSV3_PREFILL_ZIPF, 1024, 512, 256, n_groups=8, topk_groups=4, bias_mode=1,
               drop_policy=2),
     # heavy drops through the fp32 router, bias inside the logits
@@ -169,12 +170,12 @@ def test_scored_permute_rows():
                        inp.x[torch.from_numpy(tor[used]).cuda()])
 
 
-@pytest.mark.parametrize("T", [400, 700], ids=["fp32_router", "tensor_core_router"])
+@pytest.mark.parametrize("T", [400, 9600], ids=["k_split_router", "epilogue_topk_router"])
 def test_layer_forward_with_workspace_logits(T):
     """moe_layer_forward reads the scores from the caller's logits or, when the logits
     pointer is NULL, from the workspace copy moe_route wrote: same result either way, with
-    the fp32 router (T < 512) and with the tensor-core router whose GEMM epilogue takes the
-    top-k."""
+    the tensor-core router's K split over blocks (few tiles; the top-k kernel writes z) and
+    with its GEMM epilogue taking the top-k (75 tiles)."""
     shape = W.reduced(W.DSV3_PREFILL_ZIPF, T, 256, 128, capacity_factor=0.7, bias_mode=1,
                       drop_policy=2)
     inp = W.make_inputs(shape, device="cuda")
@@ -189,10 +190,11 @@ def test_layer_forward_with_workspace_logits(T):
     torch.cuda.synchronize()
     assert torch.equal(out_a, out_b)
     assert torch.equal(a.bufs.assign_row, b.bufs.assign_row)
-    # router (fp32 GEMM + top-k; or the tensor-core GEMM with the top-k, on the split W_r
-    # MoELayer made once), 5 ranking kernels, permute, 2 FFN, combine, stats
-    router = 2 if T < 512 else 1
-    assert launched == router + 5 + 1 + 2 + 1 + 1
+    # router (the tensor-core GEMM on the split W_r MoELayer made once, and the top-k unless it
+    # rides in the GEMM's epilogue), 5 ranking kernels, permute, 2 FFN, combine, stats
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    stats = 2 if T * shape.k > 32768 else 1   # above 32768 picks: the drop count of its own
+    assert launched == router_launches(shape, True, sms) + 5 + 1 + 2 + 1 + stats
 
 
 # ------------------------------------------------------------------ second-choice counters
