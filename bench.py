@@ -44,10 +44,10 @@ GEMM_SOURCES = ("routing_dispatch_expert_warp_b200/csrc/moe_ffn_tc.cu",
                 "routing_dispatch_expert_warp_b200/csrc/moe_internal.h")
 RECORDED_GEMM_TRAFFIC = {
     ("mixtral8x7b_prefill_T4096", False): {
-        "bytes": 3668160256, "sources": "7efdcc28b3b4f6ee",
+        "bytes": 3668137216, "sources": "9f1036f2df2eb2be",
         "profile": "profiles/grouped_gemm_tc_mixtral8x7b_T4096_traffic.md"},
     ("dsv3_prefill_zipf_T16384", False): {
-        "bytes": 27309186048, "sources": "7efdcc28b3b4f6ee",
+        "bytes": 27606953472, "sources": "9f1036f2df2eb2be",
         "profile": "profiles/grouped_gemm_tc_dsv3_prefill_T16384_traffic.md"},
 }
 
