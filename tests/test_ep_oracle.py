@@ -29,6 +29,32 @@ def test_hand_case_layout_and_stats():
                 assert got == want, key
 
 
+def test_hand_case_with_empty_pairs():
+    """Pair percentiles over every ordered pair of different ranks, empty ones included
+    (tests/golden/ep_hand_g3_e3_empty_pairs.json, derived by hand)."""
+    g = json.load(open(os.path.join(os.path.dirname(GOLDEN), "ep_hand_g3_e3_empty_pairs.json")))
+    lay = EP.recv_layout(g["kept_by_src"], g["expert_rank"])
+    assert lay["base"].tolist() == g["base"]
+    assert lay["offsets"] == g["offsets"] and lay["rows"] == g["rows"]
+    st = EP.ep_stats(g["kept_by_src"], g["expert_rank"], g["ranks_per_node"], g["row_bytes"])
+    for key, want in g["stats"].items():
+        if isinstance(want, float):
+            assert st[key] == pytest.approx(want, rel=1e-12, abs=1e-12), key
+        else:
+            assert st[key] == want, key
+
+
+def test_contiguous_placement_values():
+    # rank g owns the block [g E/world, (g+1) E/world)
+    assert EP.contiguous_placement(8, 2).tolist() == [0, 0, 0, 0, 1, 1, 1, 1]
+    assert EP.contiguous_placement(6, 3).tolist() == [0, 0, 1, 1, 2, 2]
+    assert EP.contiguous_placement(4, 4).tolist() == [0, 1, 2, 3]
+    assert EP.contiguous_placement(5, 1).tolist() == [0, 0, 0, 0, 0]
+    assert EP.local_experts(EP.contiguous_placement(256, 8), 3).tolist() == list(range(96, 128))
+    with pytest.raises(ValueError):
+        EP.contiguous_placement(6, 4)
+
+
 @pytest.mark.parametrize("G,E,seed", [(2, 8, 0), (4, 16, 1), (8, 256, 2), (3, 9, 3)])
 def test_layout_invariants(G, E, seed):
     rng = np.random.default_rng(seed)
@@ -99,6 +125,22 @@ def test_ep_layer_equals_local_layer_per_rank(G, E, k, cf, permuted):
                     if sr[t, j] >= 0 and er[r["idx"][t, j]] == g:
                         used[sr[t, j]] += 1
         assert (used == 1).all()
+
+
+def test_ep_layer_from_given_logits_uses_each_ranks_own():
+    """Started from each rank's fp32 logits (the parity protocol), the EP layer equals the
+    one that computes them itself."""
+    G, E, k, cf, T, d, f = 3, 6, 2, 1.0, 20, 16, 12
+    xs, w_router, wg, wu, wd = _ranks(G, T, d, f, E, k, seed=31)
+    er = EP.contiguous_placement(E, G)
+    z32s = [O.logits_to_fp32(O.router_logits(x, w_router)) for x in xs]
+    a = EP.ep_layer(xs, w_router, None, wg, wu, wd, k, O.SOFTMAX, cf, er)
+    b = EP.ep_layer(xs, w_router, None, wg, wu, wd, k, O.SOFTMAX, cf, er, z32s=z32s)
+    for s in range(G):
+        np.testing.assert_array_equal(a["routes"][s]["idx"], b["routes"][s]["idx"])
+        np.testing.assert_array_equal(a["out"][s], b["out"][s])
+    assert any(not np.array_equal(a["routes"][0]["idx"], a["routes"][s]["idx"])
+               for s in range(1, G))
 
 
 @pytest.mark.parametrize("variant", [

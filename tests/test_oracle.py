@@ -61,6 +61,34 @@ def test_hand_case_stats(golden_dir):
     assert s["tokens_per_expert"] == g["kept"]
 
 
+def test_softmax_weights_of_far_apart_logits():
+    # exp(-1000) underflows to 0 in float64, so the exact weights round to (1, 0, 0) and a
+    # softmax shifted by anything but the largest pick would overflow to inf / inf
+    z = np.array([[500.0, -500.0, 0.0]], dtype=np.float32)
+    w = O.gate_weights(z, np.array([[0, 2, 1]]), O.SOFTMAX)
+    assert w[0].tolist() == [1.0, math.exp(-500.0), 0.0]
+
+
+def test_top5pct_share_counts_ceil_of_five_percent():
+    """The top-5% share sums the ceil(0.05 E) largest kept counts: 2 experts at E = 32
+    (0.05 * 32 = 1.6), 13 at E = 256 (12.8).  Values worked by hand."""
+    # E = 32: counts 10, 9 and thirty 1s, 49 kept in all; the two largest hold 19
+    kept = [10, 9] + [1] * 30
+    rows = np.zeros((49, 1), dtype=np.int64)
+    s = O.load_stats(kept, kept, rows, None)
+    assert s["top5pct_share"] == pytest.approx(19 / 49, abs=1e-15)
+    assert s["max_to_mean"] == pytest.approx(320 / 49, abs=1e-12)   # 10 / (49 / 32)
+    # sorted: thirty 1s, 9, 10.  p50: h = 15.5 between two 1s; p95: h = 29.45 between the
+    # last 1 and 9 -> 1 + 0.45 * 8; p99: h = 30.69 between 9 and 10 -> 9.69
+    assert s["p50"] == pytest.approx(1.0, abs=1e-12)
+    assert s["p95"] == pytest.approx(4.6, abs=1e-12)
+    assert s["p99"] == pytest.approx(9.69, abs=1e-12)
+    # E = 256: thirteen experts with 2, the other 243 with 1: 269 kept, top 13 hold 26
+    kept = [2] * 13 + [1] * 243
+    s = O.load_stats(kept, kept, np.zeros((269, 1), dtype=np.int64), None)
+    assert s["top5pct_share"] == pytest.approx(26 / 269, abs=1e-15)
+
+
 def test_sigmoid_weights_hand_values():
     # sigma(3) = 0.9525741268224334, sigma(2) = 0.8807970779778823 (tabulated values)
     z = np.array([[3.0, 2.0, -1.0]], dtype=np.float32)
@@ -303,6 +331,35 @@ def test_layer_equals_per_token_sum_of_experts():
                         lambda e: (npx(inp.w_gate[e]), npx(inp.w_up[e]), npx(inp.w_down[e])))
     np.testing.assert_allclose(r["out"], o, rtol=1e-12, atol=1e-12)
     assert r["stats"]["dropped"] > 0        # capacity 1.0 with a skewed router drops
+    # each bucket's hidden rows are silu(x W_g^T) * (x W_u^T) of its tokens (torch's ops)
+    for e in range(shape.E):
+        lo, n = int(r["offsets"][e]), int(r["kept"][e])
+        if n == 0:
+            continue
+        xt = torch.from_numpy(npx(inp.x)[r["token_of_row"][lo:lo + n]].astype(np.float64))
+        g = torch.nn.functional.linear(xt, torch.from_numpy(npx(inp.w_gate[e]).astype(np.float64)))
+        u = torch.nn.functional.linear(xt, torch.from_numpy(npx(inp.w_up[e]).astype(np.float64)))
+        np.testing.assert_allclose(r["h_perm"][lo:lo + n],
+                                   (torch.nn.functional.silu(g) * u).numpy(), rtol=1e-12,
+                                   atol=1e-12)
+
+
+def test_permute_fills_padding_rows_with_zeros():
+    x = np.arange(6.0).reshape(3, 2) + 1.0
+    xp = O.permute(x, np.array([2, -1, 0, -1]))
+    assert xp.tolist() == [[5.0, 6.0], [0.0, 0.0], [1.0, 2.0], [0.0, 0.0]]
+
+
+def test_routing_decision_is_taken_on_fp32_logits():
+    # z64 = (1, 1 + 2^-30): expert 1 is larger in float64, but both round to 1.0f, and the
+    # fp32 tie goes to the lower index
+    x = np.array([[1.0]])
+    wr = np.array([[1.0, 1.0 + 2.0 ** -30]])
+    wg, wu, wd = np.ones((2, 1, 1)), np.ones((2, 1, 1)), np.ones((2, 1, 1))
+    r = O.moe_layer(x, wr, None, wg, wu, wd, k=1, gating=O.SOFTMAX, capacity_factor=0.0)
+    assert r["z32"].tolist() == [[1.0, 1.0]]
+    assert r["idx"].tolist() == [[0]]
+    assert r["z64"][0, 1] > r["z64"][0, 0]
 
 
 def test_page_stats_example(golden_dir):
@@ -446,6 +503,7 @@ def test_score_drop_order_hand_case():
     assert c["kept"].tolist() == [[1, 1], [1, 1]]
     assert c["differs"].tolist() == [0, 3]
     assert c["dropped_share"] == [1 / 3, 1 / 3]
+    assert c["differs_share"] == [0.0, 1.0]
     same = O.pick_rank_counts(idx, a["assign_row"], 2, group_of_expert=[0, 0])
     assert same["differs"].tolist() == [0, 0]
 
