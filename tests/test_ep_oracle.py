@@ -5,6 +5,8 @@ import os
 
 import numpy as np
 import pytest
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 from oracle import ep_oracle as EP
 from oracle import moe_oracle as O
@@ -79,6 +81,52 @@ def test_layout_invariants(G, E, seed):
     assert st["remote_bytes"] == (kept.sum() - st["local_assignments"]) * 100
     assert EP.ep_stats(kept, er, G, 100)["cross_node_bytes"] == 0
     assert EP.ep_stats(kept, er, 1, 100)["cross_node_bytes"] == st["remote_bytes"]
+
+
+@settings(max_examples=200, deadline=None)
+@given(G=st.integers(1, 6), per=st.integers(1, 5), rpn=st.integers(1, 4),
+       seed=st.integers(0, 2**31 - 1), sparse=st.booleans())
+def test_record_invariants_random(G, per, rpn, seed, sparse):
+    """Any placement and any kept counts: the pair matrix accounts for every row once, the
+    rank and node loads partition the assignments, sent equals received, the percentiles
+    lie between the smallest and largest pair message, and ranks on one node exchange no
+    cross-node bytes."""
+    E = G * per
+    rng = np.random.default_rng(seed)
+    kept = rng.integers(0, 5, size=(G, E))
+    if sparse:
+        kept[rng.random((G, E)) < 0.6] = 0
+    er = rng.permutation(EP.contiguous_placement(E, G))
+    st_ = EP.ep_stats(kept, er, rpn, 7)
+    total = int(kept.sum())
+    assert st_["total_assignments"] == total == sum(st_["rank_load"]) == sum(st_["node_load"])
+    assert st_["rank_load"] == [int(kept[:, er == g].sum()) for g in range(G)]
+    local = sum(int(kept[g, er == g].sum()) for g in range(G))
+    assert st_["local_assignments"] == local
+    assert st_["remote_bytes"] == (total - local) * 7
+    assert sum(st_["bytes_sent"]) == sum(st_["bytes_recv"]) == st_["remote_bytes"]
+    for g in range(G):
+        assert st_["bytes_sent"][g] == int(kept[g, er != g].sum()) * 7
+        assert st_["bytes_recv"][g] == int(kept[np.arange(G) != g][:, er == g].sum()) * 7
+    pairs = [int(kept[s_, er == g].sum()) * 7 for s_ in range(G) for g in range(G) if s_ != g]
+    if pairs:
+        assert min(pairs) <= st_["pair_bytes_p50"] <= st_["pair_bytes_p99"] <= max(pairs)
+        assert st_["pair_bytes_max"] == max(pairs)
+    assert 0 <= st_["cross_node_bytes"] <= st_["remote_bytes"]
+    if rpn >= G:
+        assert st_["cross_node_bytes"] == 0 and st_["nodes"] == 1
+    if rpn == 1:
+        assert st_["cross_node_bytes"] == st_["remote_bytes"]
+    lay = EP.recv_layout(kept, er)
+    assert lay["rows"] == [int(kept[:, er == g].sum()) for g in range(G)]
+    # the receive slots of every (source, expert) are disjoint and tile each rank's buffer
+    for g in range(G):
+        used = np.zeros(lay["rows"][g], dtype=int)
+        for e in EP.local_experts(er, g):
+            for s_ in range(G):
+                b = lay["base"][s_, e]
+                used[b:b + kept[s_, e]] += 1
+        assert (used == 1).all()
 
 
 def _ranks(G, T, d, f, E, k, seed):
