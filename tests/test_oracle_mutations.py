@@ -294,6 +294,7 @@ def _mutant(path, old, new):
         TO.O, TP.O, TE.O, TE.EP = saved
 
 
+@pytest.mark.filterwarnings("ignore::RuntimeWarning")   # some mutants overflow on purpose
 @pytest.mark.parametrize("row", ROWS, ids=[r[-1].replace(" ", "_") for r in ROWS])
 def test_pin_catches_planted_mistake(row):
     path, old, new, mod, name, kwargs, _what = row
