@@ -487,7 +487,8 @@ moe_status_t moe_combine(const moe_config_t* cfg, const void* y_perm,
 /*
  * Per-layer load statistics (moe_load_stats_t above) from the dispatch outputs, written to
  * the device struct dev_out.  If host_out is not NULL the struct is also copied to host
- * memory and the stream is synchronised -- the only call that synchronises.
+ * memory and the stream is synchronised (as by every call given a host output, and by the
+ * two error checks); with host_out NULL nothing waits.
  */
 moe_status_t moe_load_stats(const moe_config_t* cfg, const int32_t* routed_counts,
                             const int32_t* kept_counts, const int32_t* assign_row,
