@@ -22,6 +22,20 @@ def test_mixtral_work_matches_the_table():
     assert w["route_bytes"] == pytest.approx(33.7e6, rel=1e-2)
 
 
+def test_work_of_a_small_layer_with_drops_by_hand():
+    """Every term of the byte counts, on a layer small enough to add up by hand: T = 4
+    tokens, d = 8, bf16 (s = 2), E = 4, k = 2, so A = 8 picks, of which 5 are kept."""
+    shape = W.reduced(W.MIXTRAL_8X7B, 4, 8, 16).replace(E=4, k=2)
+    w = bench.algorithmic_work(shape, kept_total=5)
+    # x read 4*8*2 = 64, kept rows written 5*8*2 = 80, the 8 picks' rows read 8*4 = 32
+    assert w["permute_bytes"] == 176
+    # kept rows read 80, 8 picks' weights and rows read 8*8 = 64, out written 64
+    assert w["combine_bytes"] == 208
+    # x 64, W_r 8*4*4 = 128, logits 4*4*4 = 64, picks 8*8 = 64
+    assert w["route_bytes"] == 320
+    assert w["gemm_flops"] == 6 * 8 * 16 * 5 and w["route_flops"] == 2 * 4 * 8 * 4
+
+
 def test_binding_roof_per_workload():
     # Mixtral prefill: tensor-bound; 2.244 ms for the FFN -> 1286 TFLOP/s
     r = bench.gemm_roofline(W.MIXTRAL_8X7B, 8192, 8, 2.2437, PEAKS)
@@ -136,3 +150,9 @@ def test_route_tensor_roof_only_for_the_tensor_core_router():
     assert bench.route_tensor_roof(dec, bench.algorithmic_work(dec, 1), 0.2, peaks) != {}
     for shape in (W.MIXTRAL_8X7B, W.TINY_FP32):                  # E = 8, fp32
         assert bench.route_tensor_roof(shape, bench.algorithmic_work(shape, 1), 0.2, peaks) == {}
+    for shape in (ds.replace(E=32),                              # E = 32: the CUDA-core router
+                  ds.replace(dtype=W.F32),                       # fp32 layer
+                  ds.replace(d_model=7168 + 32)):                # d not a multiple of 64
+        assert not bench.tensor_core_router(shape)
+        assert bench.route_tensor_roof(shape, bench.algorithmic_work(shape, 1), 0.2, peaks) == {}
+    assert bench.tensor_core_router(ds.replace(E=33))
